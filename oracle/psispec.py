@@ -1,0 +1,236 @@
+"""The Psi-Spec linear sampler, AR-only decoding and prefill.
+
+What the pages fix (Walkthrough §Ψ-Spec 采样器：起草、验证、两种模式;
+Summary §方法关键点; Walkthrough §一句话直觉):
+
+* the diffusion path drafts a block of B tokens in parallel from a fully
+  noised block; the block's first token is sampled from the AR weights only
+  and is therefore always accepted;
+* the AR path verifies the whole block in parallel; the longest accepted
+  prefix is kept and the first rejected position is redrawn from the
+  renormalised residual max(0, p_AR - q_diff), which is standard
+  speculative rejection sampling, so the output follows the AR distribution;
+* two forwards per iteration, 1 <= TPF <= (B+1)/2, at least 2 tokens out.
+
+Readings where the pages are silent or garbled (each one is an input to the
+tests; the GPU path follows the same readings):
+
+* State: ``c`` committed tokens have keys/values in the cache (positions
+  0..c-1); the last produced token ``pending`` sits at position c and has no
+  keys/values yet.  Prefill caches all prompt tokens but the last, which
+  becomes the pending token; nothing is sampled at prefill.
+* Draft pass: rows [pending (gate 0), MASK x B (gate 1)] at positions
+  c..c+B; the MASK rows form one noised block starting at c+1.  The noise
+  prior is a reserved MASK token id (absorbing state).  Row 0 gives the AR
+  distribution p_1 of position c+1; MASK row i (position c+i) gives the
+  diffusion distribution q_i of the token at its own position.  Row 1's
+  logits are unused because the first token comes from the AR row.
+* Verify pass: rows x_1..x_B at positions c+1..c+B, gate 0, causal.  Row j
+  gives p_{j+1}, the AR distribution of position c+j+1.
+* Accept test for draft i = 2..B: u < p_i(x_i) / q_i(x_i) with a strict
+  inequality, taken in the log domain.  ``a`` counts the first token plus
+  the accepted prefix, a in [1, B].  If a < B the token at position c+a+1 is
+  redrawn from max(0, p_{a+1} - q_{a+1}) normalised (from p when that mass
+  is zero after rounding); otherwise a bonus token is drawn from p_{B+1}.
+  a+1 tokens are emitted.
+* Commit: the keys/values of positions c..c+a become part of the cache; the
+  emitted last token becomes the new pending token at position c+a+1.
+* Inverse-CDF sampling: weights w_v = exp(l_v - max l) in vocabulary order;
+  the token is the smallest t whose inclusive prefix sum exceeds u * sum(w);
+  if rounding leaves none, the last token with positive weight.
+* Uniforms are Philox draws keyed by (seed; stream, position, kind); see
+  :mod:`oracle.philox`.
+"""
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from .model import KVCache
+from .philox import KIND_ACCEPT, KIND_DRAFT, KIND_FIRST, KIND_RESID, uniform
+
+
+# ---------------------------------------------------------------------------
+# Sampler primitives.  Each is pinned in the tests by measuring, by bisection
+# over u, the set of uniforms that produces each outcome and comparing the
+# measure with the closed-form probability.
+# ---------------------------------------------------------------------------
+
+def _inverse_cdf(weights, u):
+    """Smallest t with inclusive prefix sum > u * total; fallback: last w > 0."""
+    c = np.cumsum(weights)
+    hit = np.nonzero(c > u * c[-1])[0]
+    if hit.size:
+        return int(hit[0])
+    return int(np.nonzero(weights > 0)[0][-1])
+
+
+def log_softmax(logits):
+    """logits - logsumexp(logits), max-shifted."""
+    m = np.max(logits)
+    return logits - (m + math.log(np.sum(np.exp(logits - m))))
+
+
+def sample_token(logits, u):
+    """Draw a token from softmax(logits) by inverse CDF with uniform u."""
+    w = np.exp(logits - np.max(logits))
+    return _inverse_cdf(w, u)
+
+
+def accept_draft(p_logits, q_logits, token, u):
+    """Accept test: log u < log p(token) - log q(token), i.e. u < p/q."""
+    lp = log_softmax(p_logits)[token]
+    lq = log_softmax(q_logits)[token]
+    return math.log(u) < lp - lq
+
+
+def residual_token(p_logits, q_logits, u):
+    """Draw from max(0, p - q) renormalised; from p if that mass is zero."""
+    p = np.exp(log_softmax(p_logits))
+    q = np.exp(log_softmax(q_logits))
+    r = np.maximum(p - q, 0.0)
+    if not np.sum(r) > 0.0:
+        return sample_token(p_logits, u)
+    return _inverse_cdf(r, u)
+
+
+def verify_block(p_rows, q_rows, drafts, u_accept, u_resid, bonus_row):
+    """Rejection step over a drafted block.
+
+    ``p_rows[j]`` / ``q_rows[j]`` are the AR and diffusion logits of tested
+    draft j, ``drafts[j]`` its token, ``u_accept[j]`` its accept uniform,
+    ``u_resid[j]`` the uniform used if j is the first rejection.  When every
+    test passes, the bonus token is drawn from ``bonus_row`` with
+    ``u_resid[len(drafts)]`` (no token when ``bonus_row`` is None).
+
+    Returns (n_accepted, next_token or None, accept_bits); tests after the
+    first rejection are evaluated and reported but do not count.
+    """
+    bits = [accept_draft(p_rows[j], q_rows[j], drafts[j], u_accept[j]) for j in range(len(drafts))]
+    n_acc = 0
+    while n_acc < len(drafts) and bits[n_acc]:
+        n_acc += 1
+    if n_acc < len(drafts):
+        nxt = residual_token(p_rows[n_acc], q_rows[n_acc], u_resid[n_acc])
+    elif bonus_row is not None:
+        nxt = sample_token(bonus_row, u_resid[len(drafts)])
+    else:
+        nxt = None
+    return n_acc, nxt, bits
+
+
+# ---------------------------------------------------------------------------
+# Decode state and the decode iterations.
+# ---------------------------------------------------------------------------
+
+@dataclass
+class DecodeState:
+    """One request: committed tokens, cache of positions 0..c-1, pending token."""
+    tokens: list                 # every token so far; tokens[-1] is pending
+    cache: KVCache
+    stream: int = 0
+
+    @property
+    def c(self):
+        return len(self.cache)
+
+    @property
+    def pending(self):
+        return self.tokens[-1]
+
+    def copy(self):
+        return DecodeState(list(self.tokens), self.cache.copy(), self.stream)
+
+
+def prefill(model, prompt, stream=0):
+    """Cache every prompt token but the last; the last becomes pending."""
+    prompt = [int(t) for t in prompt]
+    if len(prompt) < 1:
+        raise ValueError("prompt must hold at least one token")
+    cache = KVCache(model.shape)
+    n = len(prompt) - 1
+    if n > 0:
+        _, k, v = model.forward(cache, prompt[:n], np.arange(n), np.zeros(n))
+        cache.append(k, v, range(n))
+    return DecodeState(prompt, cache, stream)
+
+
+@dataclass
+class StepResult:
+    """Everything one Psi-Spec iteration decided, for stage-by-stage checks."""
+    c: int                              # cached tokens before the step
+    logits_draft: np.ndarray            # [B+1, V] draft pass rows
+    logits_verify: np.ndarray           # [B, V] verify pass rows
+    drafts: list                        # x_1..x_B
+    accept_bits: list                   # tests of x_2..x_B
+    a: int                              # first token + accepted prefix, in [1, B]
+    next_token: int                     # resampled or bonus token
+    emitted: list = field(default_factory=list)   # x_1..x_a, next_token
+
+
+def draft_pass(model, state, B):
+    """Rows [pending, MASK x B] at positions c..c+B, gates [0, 1 x B]."""
+    c = state.c
+    mask_id = model.shape["mask_id"]
+    tokens = [state.pending] + [mask_id] * B
+    pos = np.arange(c, c + B + 1)
+    gates = np.array([0.0] + [1.0] * B)
+    noised = np.array([False] + [True] * B)
+    block = np.array([0] + [c + 1] * B)
+    return model.forward(state.cache, tokens, pos, gates, noised, block)
+
+
+def verify_pass(model, cache_with_pending, c, drafts):
+    """Rows x_1..x_B at positions c+1..c+B, gate 0, over cache 0..c."""
+    B = len(drafts)
+    return model.forward(cache_with_pending, drafts, np.arange(c + 1, c + B + 1), np.zeros(B))
+
+
+def spec_step(model, state, B, seed, drafts=None, uniform_fn=None):
+    """One Psi-Spec iteration; returns (new_state, StepResult).
+
+    ``drafts`` (optional) replaces the sampled block x_1..x_B, so a test can
+    verify exactly the block another implementation drafted.
+    ``uniform_fn(kind, position)`` (optional) replaces the Philox uniforms.
+    """
+    if uniform_fn is None:
+        def uniform_fn(kind, position):
+            return float(uniform(seed, state.stream, position, kind))
+    c = state.c
+    logits_d, kd, vd = draft_pass(model, state, B)
+    if drafts is None:
+        x = [sample_token(logits_d[0], uniform_fn(KIND_FIRST, c + 1))]
+        for i in range(2, B + 1):
+            x.append(sample_token(logits_d[i], uniform_fn(KIND_DRAFT, c + i)))
+    else:
+        x = [int(t) for t in drafts]
+    cache = state.cache.copy()
+    cache.append(kd, vd, [0])                      # pending token's K/V at position c
+    logits_v, kv_k, kv_v = verify_pass(model, cache, c, x)
+
+    # tested draft j (0-based) is x_{j+2} at position c+j+2
+    p_rows = [logits_v[j] for j in range(B - 1)]   # p_{j+2} from verify row j
+    q_rows = [logits_d[j + 2] for j in range(B - 1)]
+    u_acc = [uniform_fn(KIND_ACCEPT, c + j + 2) for j in range(B - 1)]
+    u_res = [uniform_fn(KIND_RESID, c + j + 2) for j in range(B)]
+    n_acc, y, bits = verify_block(p_rows, q_rows, x[1:], u_acc, u_res, logits_v[B - 1])
+    a = 1 + n_acc
+    cache.append(kv_k, kv_v, range(a))             # positions c+1..c+a
+    emitted = x[:a] + [y]
+    new_state = DecodeState(state.tokens + emitted, cache, state.stream)
+    res = StepResult(c, logits_d, logits_v, x, bits, a, y, emitted)
+    return new_state, res
+
+
+def ar_step(model, state, seed, uniform_fn=None):
+    """AR-only decode: one row (pending, gate 0); emits one token."""
+    if uniform_fn is None:
+        def uniform_fn(kind, position):
+            return float(uniform(seed, state.stream, position, kind))
+    c = state.c
+    logits, k, v = model.forward(state.cache, [state.pending], [c], [0.0])
+    y = sample_token(logits[0], uniform_fn(KIND_FIRST, c + 1))
+    cache = state.cache.copy()
+    cache.append(k, v, [0])
+    return DecodeState(state.tokens + [y], cache, state.stream), logits[0], y
