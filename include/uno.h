@@ -1,0 +1,232 @@
+/*
+ * uno.h -- C ABI of libuno: the Psi-Spec decode iteration of a diffusion-
+ * augmented LLM ("Uno") on one NVIDIA B200 (sm_100a).
+ *
+ * The method ("Unlocking Lossless Speedups in LLMs via Discrete Diffusion"):
+ * one causal Transformer keeps its AR weights W_base frozen and carries
+ * "diffusion weights" W_diff as a gated rank-r LoRA on every layer (summary
+ * page "通过离散扩散实现 LLM 无损加速：扩散增强自回归模型", section 方法关键点).
+ * One decode iteration drafts a block of B tokens in parallel with
+ * W_base + W_diff from a fully noised block, the first token from W_base
+ * alone; the AR path (W_base only) then scores the whole block, the longest
+ * accepted prefix is kept and the first rejected position is redrawn from the
+ * renormalised residual max(0, p_AR - q_diff) (blog page "不砸掉重来，给自回归
+ * LLM 装一对“扩散翅膀”：Uno 的无损加速之路", sections 一句话直觉 and
+ * Ψ-Spec 采样器：起草、验证、两种模式).  Draft and verify share one KV cache
+ * (same page, section 一句话直觉).  Every iteration runs two forwards and
+ * emits between 2 and B+1 tokens per request.
+ *
+ * Conventions of every call:
+ *  - Return value: UNO_OK (0) or one of the UNO_ERR_* codes; no exception
+ *    crosses the ABI.  uno_last_error() gives a message for the last failure
+ *    of a context.
+ *  - "dev" pointers are CUDA device pointers, "host" pointers host memory.
+ *  - All device work is enqueued on the context's stream and is
+ *    asynchronous: outputs are valid once the caller synchronises that
+ *    stream.  No call inside the decode loop synchronises the host.
+ *  - Weights are borrowed: caller-owned device buffers that must outlive the
+ *    context.  The library owns the KV pool, the page tables and all
+ *    workspaces.  Output buffers are caller-owned.
+ *  - Weight matrices are row-major [out_features, in_features]
+ *    (torch.nn.Linear layout), dense, in the model dtype; LoRA A is
+ *    [r, in_features] and LoRA B is [out_features, r].
+ */
+#ifndef UNO_H_
+#define UNO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque context. */
+typedef struct uno_ctx uno_ctx;
+
+/* A cudaStream_t passed as an opaque pointer (NULL: the legacy default stream). */
+typedef void *uno_stream_t;
+
+enum uno_dtype { UNO_F32 = 0, UNO_BF16 = 1 };
+
+enum uno_status_code {
+  UNO_OK = 0,
+  UNO_ERR_ARG = 1,          /* invalid argument (NULL, size out of range, unknown id)   */
+  UNO_ERR_OOM = 2,          /* device allocation failed                                   */
+  UNO_ERR_CAPACITY = 3,     /* no free request slot or KV pages                           */
+  UNO_ERR_CUDA = 4,         /* a CUDA runtime call failed                                 */
+  UNO_ERR_DEVICE_CHECK = 5, /* a device-side bounds check fired (see uno_status)          */
+  UNO_ERR_UNSUPPORTED = 6   /* shape or dtype this build has no kernel for                */
+};
+
+/* Projections carrying a LoRA, in this order. */
+enum uno_proj {
+  UNO_PROJ_Q = 0, UNO_PROJ_K, UNO_PROJ_V, UNO_PROJ_O, UNO_PROJ_GATE, UNO_PROJ_UP, UNO_PROJ_DOWN,
+  UNO_N_PROJ
+};
+
+/*
+ * Model shape.  Pre-RMSNorm decoder: x += o(attn(rope(q), rope(k), v)) with
+ * GQA (q head h reads kv head h / (n_heads / n_kv_heads)); x += down(silu(gate)
+ * * up); untied embedding / LM head; rotate-half RoPE with rope_theta; logits
+ * divided by temperature.  mask_id is the reserved token id of the noised
+ * block (the absorbing-state noise prior).
+ */
+typedef struct uno_shape {
+  int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab, mask_id;
+  float rope_theta, rms_eps, temperature;
+  int32_t dtype; /* enum uno_dtype: UNO_F32 (all kernels in fp32) or UNO_BF16 */
+} uno_shape;
+
+/*
+ * Weights (device pointers in the model dtype).  Per-layer entries are HOST
+ * arrays of n_layers device pointers; the arrays are copied by uno_init.
+ *   embed [vocab, d_model], lm_head [vocab, d_model], final_norm [d_model]
+ *   attn_norm[l], ffn_norm[l]          [d_model]
+ *   w[p][l]                             projection p of layer l, [out, in]
+ *   lora_A[p][l] [r, in], lora_B[p][l]  [out, r]
+ */
+typedef struct uno_weights {
+  const void *embed, *lm_head, *final_norm;
+  const void *const *attn_norm;
+  const void *const *ffn_norm;
+  const void *const *w[UNO_N_PROJ];
+  const void *const *lora_A[UNO_N_PROJ];
+  const void *const *lora_B[UNO_N_PROJ];
+} uno_weights;
+
+/*
+ * Create a context.
+ *   lora_rank, lora_alpha: the LoRA scale is alpha / rank.
+ *   block_B:   drafted block size B (2 <= B <= 64).
+ *   max_batch: request slots; max_ctx: tokens one request may hold (prompt
+ *              plus generated).  The KV pool holds max_batch * ceil((max_ctx
+ *              + B + 1) / 64) pages of 64 tokens.
+ *   seed:      Philox key of every uniform the sampler draws.
+ *   stream:    every later call enqueues on this stream.
+ * On success *out receives the context (free it with uno_destroy).
+ */
+int uno_init(const uno_shape *shape, const uno_weights *weights, int lora_rank, float lora_alpha,
+             int block_B, int max_batch, int max_ctx, uint64_t seed, uno_stream_t stream,
+             uno_ctx **out);
+
+/*
+ * Admit n_req requests and prefill them.
+ *   prompts_dev:  int32 [n_req, prompt_stride] token ids (device).
+ *   prompt_lens_host: int32 [n_req], each in [1, max_ctx].
+ *   streams_host: optional uint32 [n_req] random-stream ids (NULL: the slot id).
+ *   req_ids_host_out: int32 [n_req] receives each request's slot id.
+ * Every prompt token but the last is run through the model with the LoRA
+ * gated off and cached; the last becomes the request's pending token.
+ * Fails with UNO_ERR_CAPACITY before any launch when slots run out.
+ */
+int uno_prefill(uno_ctx *ctx, int n_req, const int32_t *prompts_dev, int prompt_stride,
+                const int32_t *prompt_lens_host, const uint32_t *streams_host,
+                int32_t *req_ids_host_out);
+
+/*
+ * One Psi-Spec iteration for n_req admitted requests (req_ids_dev: int32
+ * [n_req] slot ids, distinct, device).  Outputs (device, caller-owned):
+ *   out_tokens_dev int32 [n_req, B+1]: the emitted tokens (first n_new valid);
+ *   n_new_dev      int32 [n_req]: emitted count, in [2, B+1].
+ * The request's cache advances by n_new tokens and its pending token becomes
+ * the last emitted one.  A request whose cache would exceed its pages is
+ * left unchanged and raises the device check flag (see uno_status).
+ */
+int uno_spec_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *out_tokens_dev,
+                  int32_t *n_new_dev);
+
+/* AR-only decode (baseline): one forward, the LoRA off, one token per request
+ * into out_tokens_dev int32 [n_req]. */
+int uno_ar_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *out_tokens_dev);
+
+/* Free a request's slot and pages (stream-ordered after earlier work). */
+int uno_release(uno_ctx *ctx, int req_id);
+
+/* Synchronise the context's stream, free everything. */
+int uno_destroy(uno_ctx *ctx);
+
+/* Message of the last failed call on ctx ("" if none); valid until the next call. */
+const char *uno_last_error(const uno_ctx *ctx);
+
+/* Synchronise the stream and return UNO_ERR_DEVICE_CHECK if a device-side
+ * bounds check fired since the last call (the flag is then cleared). */
+int uno_status(uno_ctx *ctx);
+
+/* Read a request's state (synchronises): cached token count, pending token. */
+int uno_request_state(uno_ctx *ctx, int req_id, int32_t *cached_out, int32_t *pending_out);
+
+/*
+ * Debug taps (synchronous copies of internal buffers of the LAST step, for
+ * stage-by-stage parity tests; not for production use).
+ *   UNO_DBG_LOGITS_DRAFT  f32   [n_req, B+1, vocab] draft-pass logits
+ *   UNO_DBG_LOGITS_VERIFY f32   [n_req, B, vocab]   verify-pass logits
+ *   UNO_DBG_DRAFTS        int32 [n_req, B]          drafted block x_1..x_B
+ *   UNO_DBG_LOGITS_AR     f32   [n_req, vocab]      AR-step logits
+ * bytes must not exceed the buffer's size for max_batch requests.
+ */
+enum uno_debug_buf {
+  UNO_DBG_LOGITS_DRAFT = 0, UNO_DBG_LOGITS_VERIFY = 1, UNO_DBG_DRAFTS = 2, UNO_DBG_LOGITS_AR = 3
+};
+int uno_debug_read(uno_ctx *ctx, int which, void *dst_host, size_t bytes);
+
+/* Copy keys and values of positions [pos0, pos0+n) of layer `layer` of a
+ * request to host buffers k_host, v_host, each [n, n_kv_heads, head_dim] in
+ * the model dtype (synchronises).  Keys are stored after RoPE. */
+int uno_debug_kv(uno_ctx *ctx, int req_id, int layer, int pos0, int n, void *k_host,
+                 void *v_host);
+
+/*
+ * Profiling tap (no counterpart on the pages: measurement plumbing).
+ * Kernel classes: the gated-LoRA GEMMs (incl. the LM head), attention,
+ * draft_sample / AR sampling, spec_verify, and everything else (row assembly,
+ * norms, RoPE/KV write, SwiGLU).
+ * uno_profile_begin zeroes the counters and, for every class in
+ * class_mask (bit 1 << class), records a CUDA event pair around each launch
+ * on the context stream.  uno_profile_end synchronises and fills, per class
+ * (arrays of UNO_K_N), the launch count (all classes), the summed event time
+ * in ms (profiled classes, else 0) and the algorithmic bytes those launches
+ * move (weights, activations and outputs read/written once; KV bytes are
+ * not known on the host and are not included for attention).
+ */
+enum uno_kernel_class { UNO_K_GEMM = 0, UNO_K_ATTN, UNO_K_SAMPLE, UNO_K_VERIFY, UNO_K_OTHER, UNO_K_N };
+int uno_profile_begin(uno_ctx *ctx, unsigned class_mask);
+int uno_profile_end(uno_ctx *ctx, int64_t *launches, double *ms, double *bytes);
+
+/*
+ * spec_verify as a stand-alone kernel: the rejection step of speculative
+ * sampling over drafted blocks (blog page "…Uno 的无损加速之路", section
+ * Ψ-Spec 采样器：起草、验证、两种模式: verify the block in parallel, keep the
+ * longest accepted prefix, redraw the first rejected token from the
+ * renormalised residual max(0, p - q)).
+ *
+ *   p_dev, q_dev:  f32 [n_req, n_tests, vocab] AR / drafter logits (device);
+ *                  row j of request i scores draft drafts_dev[i, j].
+ *   drafts_dev:    int32 [n_req, n_tests] drafted tokens.
+ *   streams_dev:   uint32 [n_req] random-stream id of each request.
+ *   pos0_dev:      int32 [n_req] position of test 0; test j draws its accept
+ *                  uniform at position pos0 + j, the redraw at pos0 + a.
+ *   seed:          Philox key.
+ *   n_out_dev      int32 [n_req]: a, the length of the accepted prefix, in
+ *                  [0, n_tests].
+ *   out_tokens_dev int32 [n_req, n_tests+1]: the a accepted drafts, then at
+ *                  index a the token redrawn from max(0, p_a - q_a)
+ *                  renormalised; -1 there when a == n_tests (no bonus row is
+ *                  given, so no further token is drawn).
+ *   workspace_dev: scratch of at least uno_spec_verify_workspace_bytes()
+ *                  bytes, 256-byte aligned, zero-filled before its first use
+ *                  (the kernel leaves it zeroed again); calls sharing a
+ *                  workspace must not overlap on the GPU.
+ * Returns UNO_ERR_ARG on bad sizes; never synchronises.
+ */
+size_t uno_spec_verify_workspace_bytes(int n_req, int n_tests, int vocab);
+int uno_spec_verify(const float *p_dev, const float *q_dev, const int32_t *drafts_dev,
+                    int n_req, int n_tests, int vocab, uint64_t seed,
+                    const uint32_t *streams_dev, const int32_t *pos0_dev,
+                    int32_t *out_tokens_dev, int32_t *n_out_dev, void *workspace_dev,
+                    size_t workspace_bytes, uno_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* UNO_H_ */

@@ -1,0 +1,170 @@
+// Per-row layer kernels of the model forward: row assembly + embedding
+// gather, RMSNorm, RoPE + paged KV write, SwiGLU.
+//
+// The forward is the frozen AR transformer plus a per-row gated LoRA
+// (summary page "通过离散扩散实现 LLM 无损加速：扩散增强自回归模型", section
+// 方法关键点; blog page "…Uno 的无损加速之路", section Diffusion Distillation：
+// 一步蒸馏 + 块级扩散: the gate turns the adapter off at clean positions and on
+// at noised ones).  The residual stream is fp32; GEMM inputs are in the
+// model dtype.
+#pragma once
+
+#include "common.cuh"
+
+namespace uno {
+
+// Paged KV pool: [n_layers][n_pages][2 (K, V)][n_kv_heads][PAGE][head_dim].
+constexpr int KV_PAGE = 64;
+
+struct KvLayout {
+  void* pool;
+  int n_pages, n_kv_heads, head_dim, pages_per_req;
+  const int32_t* page_table;   // [max_batch][pages_per_req]
+  __device__ __forceinline__ size_t offset(int layer, int slot, int pos, int kv, int head,
+                                           int& ok) const {
+    const int pi = pos / KV_PAGE;
+    ok = (pos >= 0 && pi < pages_per_req);
+    const int page = ok ? page_table[(size_t)slot * pages_per_req + pi] : 0;
+    return ((((size_t)layer * n_pages + page) * 2 + kv) * n_kv_heads + head) * KV_PAGE * head_dim +
+           (size_t)(pos % KV_PAGE) * head_dim;
+  }
+};
+
+// Pass kinds (a pass is one forward over a set of rows).
+enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3 };
+
+struct RowArgs {
+  int kind;
+  int rows_per_req;
+  const int32_t* req_slot;     // [n_req] slot ids (decode passes)
+  const int32_t* cached;       // [max_batch]
+  const int32_t* pending;      // [max_batch]
+  const int32_t* drafts;       // [n_req, B] (verify pass)
+  int B;
+  const int32_t* prompt;       // prefill: this request's prompt (device)
+  int prefill_slot, prefill_pos0;
+  int mask_id, vocab, max_batch;
+  float lora_scale;
+  int32_t* row_pos; int32_t* row_slot; float* row_gate;   // outputs [M]
+  const void* embed; int d;    // [vocab, d] model dtype
+  float* x;                    // [M, d] fp32 residual
+  int32_t* status;
+};
+
+// a1: build the rows of a pass and gather their embeddings.
+template <typename T>
+__global__ void build_rows_kernel(const RowArgs a) {
+  const int row = blockIdx.x;
+  const int req = row / a.rows_per_req, j = row % a.rows_per_req;
+  int slot, tok, pos;
+  float gate = 0.f;
+  if (a.kind == PASS_PREFILL) {
+    slot = a.prefill_slot;
+    tok = a.prompt[j];
+    pos = a.prefill_pos0 + j;
+  } else {
+    slot = a.req_slot[req];
+    if (slot < 0 || slot >= a.max_batch) { raise_status(a.status, ST_BAD_SLOT); slot = 0; }
+    const int c = a.cached[slot];
+    if (a.kind == PASS_DRAFT) {            // [pending, MASK x B] at c..c+B
+      tok = (j == 0) ? a.pending[slot] : a.mask_id;
+      pos = c + j;
+      gate = (j == 0) ? 0.f : a.lora_scale;
+    } else if (a.kind == PASS_VERIFY) {    // x_1..x_B at c+1..c+B
+      tok = a.drafts[(size_t)req * a.B + j];
+      pos = c + 1 + j;
+    } else {                               // AR: pending at c
+      tok = a.pending[slot];
+      pos = c;
+    }
+  }
+  if (tok < 0 || tok >= a.vocab) { raise_status(a.status, ST_BAD_TOKEN); tok = 0; }
+  if (threadIdx.x == 0) {
+    a.row_pos[row] = pos;
+    a.row_slot[row] = slot;
+    a.row_gate[row] = gate;
+  }
+  const T* e = reinterpret_cast<const T*>(a.embed) + (size_t)tok * a.d;
+  float* x = a.x + (size_t)row * a.d;
+  for (int i = threadIdx.x; i < a.d; i += blockDim.x) x[i] = to_f(e[i]);
+}
+
+// RMSNorm: out = x / sqrt(mean(x^2) + eps) * gain, one CTA per row.
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* gain, T* out, int d,
+                                                     int ld_out, float eps) {
+  __shared__ float red[32];
+  const float* xr = x + (size_t)blockIdx.x * d;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < d; i += NT) s += xr[i] * xr[i];
+  s = block_sum<NT>(s, red);
+  const float inv = 1.0f / sqrtf(s / (float)d + eps);
+  T* o = out + (size_t)blockIdx.x * ld_out;
+  for (int i = threadIdx.x; i < d; i += NT) o[i] = from_f<T>(xr[i] * inv * to_f(gain[i]));
+}
+
+// RoPE (rotate-half) on q and k in place in the fused qkv rows, and write the
+// rotated k and v of every row into the paged pool at (slot, position).
+// cos/sin come from a table [max_pos][head_dim / 2] computed on the host in
+// double precision.
+template <typename T>
+__global__ void rope_kv_kernel(T* qkv, int ld_qkv, const int32_t* row_pos, const int32_t* row_slot,
+                               const float* cos_t, const float* sin_t, int max_pos, int H, int Hkv,
+                               int hd, KvLayout kv, int layer, int32_t* status) {
+  const int row = blockIdx.x;
+  const int pos = row_pos[row], slot = row_slot[row];
+  const int half = hd / 2;
+  T* r = qkv + (size_t)row * ld_qkv;
+  int ok_pos = pos < max_pos;
+  const int pc = ok_pos ? pos : 0;
+  // q heads then k heads: pairs (i, i + half)
+  for (int idx = threadIdx.x; idx < (H + Hkv) * half; idx += blockDim.x) {
+    const int h = idx / half, i = idx % half;
+    const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
+    T* base = r + (size_t)h * hd;
+    const float x1 = to_f(base[i]), x2 = to_f(base[i + half]);
+    const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
+    if (h < H) {
+      base[i] = from_f<T>(y1);
+      base[i + half] = from_f<T>(y2);
+    } else {
+      int ok;
+      const size_t off = kv.offset(layer, slot, pos, 0, h - H, ok);
+      if (ok && ok_pos) {
+        T* dst = reinterpret_cast<T*>(kv.pool) + off;
+        dst[i] = from_f<T>(y1);
+        dst[i + half] = from_f<T>(y2);
+      } else if (i == 0) {
+        raise_status(status, ST_POS_OVERFLOW);
+      }
+    }
+  }
+  const T* v = r + (size_t)(H + Hkv) * hd;
+  for (int idx = threadIdx.x; idx < Hkv * hd; idx += blockDim.x) {
+    const int h = idx / hd, i = idx % hd;
+    int ok;
+    const size_t off = kv.offset(layer, slot, pos, 1, h, ok);
+    if (ok && ok_pos) reinterpret_cast<T*>(kv.pool)[off + i] = v[(size_t)h * hd + i];
+  }
+}
+
+// SwiGLU: out[:, f] = silu(gu[:, f]) * gu[:, F + f].
+template <typename T>
+__global__ void swiglu_kernel(const T* gu, int F, T* out) {
+  const int row = blockIdx.x;
+  const T* g = gu + (size_t)row * 2 * F;
+  T* o = out + (size_t)row * F;
+  for (int f = threadIdx.x; f < F; f += blockDim.x) {
+    const float a = to_f(g[f]), b = to_f(g[F + f]);
+    o[f] = from_f<T>(a / (1.0f + expf(-a)) * b);
+  }
+}
+
+// Prefill bookkeeping: cached = P - 1, pending = prompt[P - 1].
+__global__ void init_slot_kernel(const int32_t* prompt, int P, int slot, int32_t* cached,
+                                 int32_t* pending) {
+  cached[slot] = P - 1;
+  pending[slot] = prompt[P - 1];
+}
+
+}  // namespace uno

@@ -120,6 +120,23 @@ def make_prompts(cfg, n_req=None, prompt_len=None, seed=None):
     return np.stack(rows).astype(np.int32) if rows else np.zeros((0, prompt_len), np.int32)
 
 
+def make_drafts(q_logits, seed=1, chunk=256):
+    """int32 [rows] tokens drawn from softmax(q_logits) by the Gumbel-max rule.
+
+    Input generator of the spec_verify microbenchmark (its drafted tokens
+    come from q); it runs on q_logits' device with a seeded torch generator.
+    """
+    gen = torch.Generator(device=q_logits.device)
+    gen.manual_seed(seed)
+    rows, V = q_logits.shape
+    out = torch.empty(rows, dtype=torch.int32, device=q_logits.device)
+    for s in range(0, rows, chunk):
+        e = min(rows, s + chunk)
+        u = torch.rand((e - s, V), generator=gen, device=q_logits.device).clamp_(min=1e-30)
+        out[s:e] = torch.argmax(q_logits[s:e] - torch.log(-torch.log(u)), dim=1).to(torch.int32)
+    return out
+
+
 def make_verify_logits(rows, vocab, device, p_std=3.0, q_noise_std=0.5, seed=0):
     """fp32 (p, q) logits [rows, vocab]: p ~ N(0, p_std), q = p + N(0, q_noise_std)."""
     gen = torch.Generator(device=device)

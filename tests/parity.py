@@ -1,0 +1,139 @@
+"""Stage-by-stage comparison of the CUDA path with the oracle.
+
+The GPU samples in fp32 and the oracle in fp64, so on the same logits and the
+same uniforms the two can only disagree when the uniform lands within
+rounding distance of a decision boundary.  Every disagreement is therefore
+traced: it is accepted only if the oracle's own margin at that boundary is
+below a tolerance derived from fp32 arithmetic, and it is counted.
+
+* sampling: |C_k - u Z| / Z at the CDF boundary k separating the two tokens;
+* accept test: |log u - (log p(t) - log q(t))|.
+"""
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from oracle import psispec as ops
+from oracle.philox import KIND_ACCEPT, KIND_DRAFT, KIND_FIRST, KIND_RESID, uniform
+
+# fp32 relative error of a vocabulary-long sum done in the kernels' order, and
+# of a log-sum-exp, with a safety factor: see the readings in the design notes.
+SAMPLE_TOL = 2e-5
+ACCEPT_TOL = 2e-5
+
+
+@dataclass
+class Tally:
+    positions: int = 0
+    mismatches: int = 0
+    notes: list = field(default_factory=list)
+
+    def add(self, ok, note=None):
+        self.positions += 1
+        if not ok:
+            self.mismatches += 1
+            self.notes.append(note)
+
+
+def _cdf_margin(weights, u, a, b):
+    c = np.cumsum(weights)
+    z = c[-1]
+    lo, hi = min(a, b), max(a, b)
+    return float(np.min(np.abs(c[lo:hi] - u * z)) / z) if hi > lo else 0.0
+
+
+def softmax_weights(logits):
+    l = np.asarray(logits, np.float64)
+    return np.exp(l - l.max())
+
+
+def residual_weights(lp, lq):
+    p = np.exp(ops.log_softmax(np.asarray(lp, np.float64)))
+    q = np.exp(ops.log_softmax(np.asarray(lq, np.float64)))
+    return np.maximum(p - q, 0.0)
+
+
+def check_sample(logits, u, t_gpu, tally, what=""):
+    """The GPU's inverse-CDF draw against the oracle's on the same logits."""
+    l = np.asarray(logits, np.float64)
+    t_o = ops.sample_token(l, u)
+    if t_o == t_gpu:
+        tally.add(True)
+        return
+    m = _cdf_margin(softmax_weights(l), u, t_o, t_gpu)
+    assert m < SAMPLE_TOL, f"{what}: sampled {t_gpu}, oracle {t_o}, margin {m:.3e}"
+    tally.add(False, (what, t_gpu, t_o, m))
+
+
+def check_residual(lp, lq, u, t_gpu, tally, what=""):
+    lp = np.asarray(lp, np.float64)
+    lq = np.asarray(lq, np.float64)
+    t_o = ops.residual_token(lp, lq, u)
+    if t_o == t_gpu:
+        tally.add(True)
+        return
+    w = residual_weights(lp, lq)
+    if not w.sum() > 0:
+        w = softmax_weights(lp)
+    m = _cdf_margin(w, u, t_o, t_gpu)
+    assert m < SAMPLE_TOL, f"{what}: residual {t_gpu}, oracle {t_o}, margin {m:.3e}"
+    tally.add(False, (what, t_gpu, t_o, m))
+
+
+def accept_margin(lp, lq, t, u):
+    lp = np.asarray(lp, np.float64)
+    lq = np.asarray(lq, np.float64)
+    return abs(math.log(u) - (ops.log_softmax(lp)[t] - ops.log_softmax(lq)[t]))
+
+
+def check_verify(p_rows, q_rows, drafts, u_acc, u_res, bonus_row, n_acc_gpu, y_gpu, tally, what=""):
+    """The GPU's accepted prefix and next token against the oracle's rule.
+
+    Returns True when the GPU's decisions equal the oracle's.
+    """
+    n_o, y_o, bits = ops.verify_block(p_rows, q_rows, drafts, u_acc, u_res, bonus_row)
+    if n_o != n_acc_gpu:
+        j = min(n_o, n_acc_gpu)   # first test the two decided differently
+        m = accept_margin(p_rows[j], q_rows[j], drafts[j], u_acc[j])
+        assert m < ACCEPT_TOL, f"{what}: accepted {n_acc_gpu}, oracle {n_o}, margin {m:.3e}"
+        tally.add(False, (what, "accept", n_acc_gpu, n_o, m))
+        return False
+    tally.add(True)
+    if n_acc_gpu < len(drafts):
+        check_residual(p_rows[n_acc_gpu], q_rows[n_acc_gpu], u_res[n_acc_gpu], y_gpu, tally, what)
+    elif bonus_row is not None:
+        check_sample(bonus_row, u_res[len(drafts)], y_gpu, tally, what + " bonus")
+    return True
+
+
+def uniforms(seed, stream, c, B):
+    """Uniforms of one iteration at cached count c, keyed like the kernels."""
+    u = lambda kind, pos: float(uniform(seed, stream, pos, kind))
+    return {
+        "first": u(KIND_FIRST, c + 1),
+        "draft": [u(KIND_DRAFT, c + i) for i in range(2, B + 1)],
+        "accept": [u(KIND_ACCEPT, c + j + 2) for j in range(B - 1)],
+        "resid": [u(KIND_RESID, c + j + 2) for j in range(B)],
+    }
+
+
+def check_step_sampling(ld, lv, drafts, emitted, c, B, seed, stream, tally, what=""):
+    """draft_sample and spec_verify of one request, on the GPU's own logits.
+
+    ld [B+1, V], lv [B, V] (GPU logits), drafts x_1..x_B and emitted tokens
+    (GPU).  Returns True when every decision matched exactly.
+    """
+    us = uniforms(seed, stream, c, B)
+    n0 = tally.mismatches
+    check_sample(ld[0], us["first"], drafts[0], tally, f"{what} x1")
+    for i in range(2, B + 1):
+        check_sample(ld[i], us["draft"][i - 2], drafts[i - 1], tally, f"{what} x{i}")
+    a = len(emitted) - 1
+    assert emitted[:a] == list(drafts[:a]), f"{what}: emitted prefix {emitted} vs drafts {drafts}"
+    p_rows = [lv[j] for j in range(B - 1)]
+    q_rows = [ld[j + 2] for j in range(B - 1)]
+    check_verify(p_rows, q_rows, list(drafts[1:]), us["accept"], us["resid"], lv[B - 1], a - 1,
+                 emitted[-1], tally, what)
+    return tally.mismatches == n0

@@ -1,0 +1,240 @@
+"""Whole Psi-Spec iterations through the C ABI vs the oracle (GPU).
+
+Per iteration and per stage (teacher-forced, so one near-tie cannot make the
+two sequences drift apart):
+  1. draft-pass and verify-pass logits against the oracle's forward of the
+     same state and the same drafted block (fp32: 1e-4, bf16: 2e-2);
+  2. draft_sample and spec_verify decisions against the oracle's sampler run
+     on the GPU's own logits with the same uniforms (near-ties traced);
+  3. in fp32 mode, the emitted tokens against the oracle's own end-to-end
+     iteration;
+  4. the KV cache after commit against the oracle's cache, position by
+     position through the page table.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from lossless_diffusion_draft_b200 import synth, uno
+from oracle import model as om
+from oracle import psispec as ops
+
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(name, n_req, prompt_len, max_ctx, **over):
+    cfg = dict(synth.CONFIGS[name], **over)
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = cfg["dtype"]
+    params_cpu = synth.make_params(cfg, "cpu")
+    params = {k: v.cuda() for k, v in params_cpu.items()}
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], n_req, max_ctx,
+                       cfg["seed"], torch.cuda.current_stream())
+    prompts = synth.make_prompts(cfg, n_req, prompt_len)
+    ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).cuda(), [prompt_len] * n_req,
+                          streams=list(range(n_req)))
+    model = om.Model(synth.model_shape(cfg), {k: v.double().numpy() for k, v in params_cpu.items()})
+    states = [ops.prefill(model, [int(t) for t in prompts[i]], stream=i) for i in range(n_req)]
+    return cfg, ctx, ids, model, states
+
+
+def _kv_check(ctx, cfg, model, state, req, tol):
+    c = state.c
+    Hkv, hd = cfg["n_kv_heads"], cfg["head_dim"]
+    dt = torch.float32 if cfg["dtype"] == "f32" else torch.bfloat16
+    for l in range(cfg["n_layers"]):
+        k = torch.empty((c, Hkv, hd), dtype=dt)
+        v = torch.empty((c, Hkv, hd), dtype=dt)
+        uno.uno_debug_kv(ctx, req, l, 0, c, k, v)
+        np.testing.assert_allclose(k.double().numpy(), state.cache.k[l], atol=tol, rtol=0)
+        np.testing.assert_allclose(v.double().numpy(), state.cache.v[l], atol=tol, rtol=0)
+
+
+def _run(name, n_req, prompt_len, n_steps, logit_tol, kv_tol, end_to_end, max_ctx=None, **over):
+    cfg, ctx, ids, model, states = _setup(name, n_req, prompt_len,
+                                          max_ctx or prompt_len + (n_steps + 1) * 20, **over)
+    B, V, seed = cfg["B"], cfg["vocab"], cfg["seed"]
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((n_req, B + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(n_req, dtype=torch.int32, device="cuda")
+    tally = parity.Tally()
+    e2e = parity.Tally()
+    worst = 0.0
+    for step in range(n_steps):
+        uno.uno_spec_step(ctx, req, out, n_new)
+        uno.uno_status(ctx)
+        ld = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_DRAFT, torch.empty((n_req, B + 1, V)))
+        lv = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_VERIFY, torch.empty((n_req, B, V)))
+        dr = uno.uno_debug_read(ctx, uno.UNO_DBG_DRAFTS, torch.empty((n_req, B), dtype=torch.int32))
+        o, nn = out.cpu().numpy(), n_new.cpu().numpy()
+        for i in range(n_req):
+            st = states[i]
+            drafts = [int(t) for t in dr[i]]
+            emitted = [int(t) for t in o[i, : nn[i]]]
+            assert 2 <= nn[i] <= B + 1
+            # 1. logits: the oracle forwards the same state and the GPU's block
+            new_st, res = ops.spec_step(model, st, B, seed, drafts=drafts)
+            err_d = float(np.max(np.abs(ld[i].double().numpy() - res.logits_draft)))
+            err_v = float(np.max(np.abs(lv[i].double().numpy() - res.logits_verify)))
+            worst = max(worst, err_d, err_v)
+            assert err_d <= logit_tol and err_v <= logit_tol, (step, i, err_d, err_v)
+            # 2. sampler decisions on the GPU's own logits
+            parity.check_step_sampling(ld[i].double().numpy(), lv[i].double().numpy(), drafts,
+                                       emitted, st.c, B, seed, st.stream, tally, f"step {step} req {i}")
+            # 3. end to end on the oracle's own logits (fp32 mode)
+            if end_to_end:
+                _, own = ops.spec_step(model, st, B, seed)
+                same = own.emitted == emitted
+                e2e.add(same, (step, i, own.emitted, emitted))
+            # advance the oracle to the GPU's tokens (teacher forcing)
+            if res.emitted == emitted:
+                states[i] = new_st
+            else:
+                states[i] = ops.prefill(model, st.tokens + emitted, stream=st.stream)
+            c_gpu, pend_gpu = uno.uno_request_state(ctx, ids[i])
+            assert c_gpu == states[i].c and pend_gpu == states[i].pending
+    for i in range(n_req):
+        _kv_check(ctx, cfg, model, states[i], ids[i], kv_tol)
+    ctx.close()
+    return tally, e2e, worst
+
+
+def test_tiny_fp32_generation():
+    """Tiny fp32 model: 32-token prompt, 64 generated tokens, B=4."""
+    tally, e2e, worst = _run("tiny", 1, 32, 20, 1e-4, 1e-4, True, max_ctx=160)
+    assert tally.mismatches == 0 or all(n is not None for n in tally.notes), tally.notes
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
+    # fp32 mode: tokens bit-exact with the oracle's own iteration, except a
+    # traced near-tie (counted in the stage tally above)
+    assert e2e.mismatches <= tally.mismatches, e2e.notes
+
+
+def test_tiny_fp32_batch_and_ragged():
+    """Several requests with prompts of different lengths in one step."""
+    cfg = dict(synth.CONFIGS["tiny"])
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = "f32"
+    params_cpu = synth.make_params(cfg, "cpu")
+    params = {k: v.cuda() for k, v in params_cpu.items()}
+    B = cfg["B"]
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, 5, 200, cfg["seed"],
+                       torch.cuda.current_stream())
+    lens = [1, 2, 63, 64, 65]
+    prompts = synth.make_prompts(cfg, 5, 70)
+    ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).cuda(), lens, streams=[10, 11, 12, 13, 14])
+    model = om.Model(synth.model_shape(cfg), {k: v.double().numpy() for k, v in params_cpu.items()})
+    states = [ops.prefill(model, [int(t) for t in prompts[i, : lens[i]]], stream=10 + i) for i in range(5)]
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((5, B + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(5, dtype=torch.int32, device="cuda")
+    tally = parity.Tally()
+    for step in range(6):
+        uno.uno_spec_step(ctx, req, out, n_new)
+        uno.uno_status(ctx)
+        ld = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_DRAFT, torch.empty((5, B + 1, cfg["vocab"])))
+        lv = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_VERIFY, torch.empty((5, B, cfg["vocab"])))
+        dr = uno.uno_debug_read(ctx, uno.UNO_DBG_DRAFTS, torch.empty((5, B), dtype=torch.int32))
+        for i in range(5):
+            st = states[i]
+            drafts = [int(t) for t in dr[i]]
+            emitted = [int(t) for t in out[i, : int(n_new[i])].cpu()]
+            new_st, res = ops.spec_step(model, st, B, cfg["seed"], drafts=drafts)
+            assert np.max(np.abs(ld[i].double().numpy() - res.logits_draft)) <= 1e-4
+            assert np.max(np.abs(lv[i].double().numpy() - res.logits_verify)) <= 1e-4
+            parity.check_step_sampling(ld[i].double().numpy(), lv[i].double().numpy(), drafts,
+                                       emitted, st.c, B, cfg["seed"], st.stream, tally)
+            states[i] = new_st if res.emitted == emitted else ops.prefill(model, st.tokens + emitted, stream=st.stream)
+    assert tally.mismatches <= 1, tally.notes
+    for i in range(5):
+        _kv_check(ctx, cfg, model, states[i], ids[i], 1e-4)
+    ctx.close()
+
+
+def test_tiny_fp32_ar_step():
+    cfg = dict(synth.CONFIGS["tiny"])
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = "f32"
+    params_cpu = synth.make_params(cfg, "cpu")
+    params = {k: v.cuda() for k, v in params_cpu.items()}
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], 1, 100,
+                       cfg["seed"], torch.cuda.current_stream())
+    prompt = synth.make_prompts(cfg, 1, 20)
+    ids = uno.uno_prefill(ctx, torch.from_numpy(prompt).cuda(), [20], streams=[3])
+    model = om.Model(synth.model_shape(cfg), {k: v.double().numpy() for k, v in params_cpu.items()})
+    st = ops.prefill(model, [int(t) for t in prompt[0]], stream=3)
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tally = parity.Tally()
+    for _ in range(10):
+        uno.uno_ar_step(ctx, req, out)
+        la = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_AR, torch.empty((1, cfg["vocab"])))
+        new_st, logits, y = ops.ar_step(model, st, cfg["seed"])
+        assert np.max(np.abs(la[0].double().numpy() - logits)) <= 1e-4
+        t = int(out[0])
+        u = float(parity.uniforms(cfg["seed"], 3, st.c, cfg["B"])["first"])
+        parity.check_sample(la[0].double().numpy(), u, t, tally)
+        st = new_st if t == y else ops.prefill(model, st.tokens + [t], stream=3)
+    assert tally.mismatches <= 1
+    _kv_check(ctx, cfg, model, st, ids[0], 1e-4)
+    ctx.close()
+
+
+def test_small_bf16_steps():
+    """Small bf16 model (8 layers, d 1024, GQA 16/4, vocab 32000, B=8) on
+    short prompts: logits within 2e-2 of the fp64 oracle."""
+    tally, _, worst = _run("small", 3, 40, 3, 2e-2, 2e-2, False, max_ctx=120)
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
+
+
+def test_capacity_and_bad_ids():
+    cfg = dict(synth.CONFIGS["tiny"])
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = "f32"
+    params = {k: v.cuda() for k, v in synth.make_params(cfg, "cpu").items()}
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], 2, 64, 0,
+                       torch.cuda.current_stream())
+    prompts = torch.from_numpy(synth.make_prompts(cfg, 3, 8)).cuda()
+    with pytest.raises(uno.UnoError) as e:
+        uno.uno_prefill(ctx, prompts, [8, 8, 8])
+    assert e.value.code == uno.UNO_ERR_CAPACITY
+    ids = uno.uno_prefill(ctx, prompts[:2], [8, 8])
+    with pytest.raises(uno.UnoError) as e:
+        uno.uno_prefill(ctx, prompts[:1], [8])
+    assert e.value.code == uno.UNO_ERR_CAPACITY
+    uno.uno_release(ctx, ids[0])
+    ids2 = uno.uno_prefill(ctx, prompts[:1], [8])
+    assert ids2 == [ids[0]]
+    with pytest.raises(uno.UnoError) as e:
+        uno.uno_release(ctx, 7)
+    assert e.value.code == uno.UNO_ERR_ARG
+    with pytest.raises(uno.UnoError) as e:
+        uno.uno_prefill(ctx, prompts[:1], [65])   # longer than max_ctx
+    ctx.close()
+
+
+def test_context_overflow_raises_device_flag():
+    """A request whose cache would pass its pages is flagged, not overrun."""
+    cfg = dict(synth.CONFIGS["tiny"])
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = "f32"
+    params = {k: v.cuda() for k, v in synth.make_params(cfg, "cpu").items()}
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], 1, 40, 0,
+                       torch.cuda.current_stream())
+    ids = uno.uno_prefill(ctx, torch.from_numpy(synth.make_prompts(cfg, 1, 40)).cuda(), [40])
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((1, cfg["B"] + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flagged = False
+    for _ in range(40):
+        uno.uno_spec_step(ctx, req, out, n_new)
+        try:
+            uno.uno_status(ctx)
+        except uno.UnoError as e:
+            assert e.code == uno.UNO_ERR_DEVICE_CHECK
+            flagged = True
+            break
+    assert flagged
+    ctx.close()
