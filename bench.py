@@ -255,6 +255,21 @@ def run_uno(args, rank, world, device):
     for k in range(K):
         uno.uno_spec_step(ctx, req, out, n_new_all[k])
     kprof = uno.uno_profile_end(ctx)
+    shapes = {}
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    for rec in uno.uno_profile_records(ctx):
+        key = (rec["cls"], rec["m"], rec["n"], rec["k"], rec["r"])
+        cnt, ms_sum = shapes.get(key, (0, 0.0))
+        shapes[key] = (cnt + 1, ms_sum + rec["ms"])
+    detail = []
+    for (cls, m, n, k, r), (cnt, ms_sum) in sorted(shapes.items(), key=lambda kv: -kv[1][1]):
+        row = {"cls": cls, "calls_per_step": cnt / K, "us_per_call": 1e3 * ms_sum / cnt,
+               "ms_per_step": ms_sum / K}
+        if cls == "gemm":
+            row.update(m=m, n=n, k=k, r=r)
+            wbytes = (n * k + n * r + m * k + m * r) * esz
+            row["GBps"] = wbytes / (ms_sum / cnt / 1e3) / 1e9
+        detail.append(row)
 
     # end to end through the C ABI with host buffers
     req_h = torch.tensor(ids, dtype=torch.int32).pin_memory()
@@ -287,7 +302,7 @@ def run_uno(args, rank, world, device):
 
     info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, tokens=tokens_all, K=K, W=W,
                 e2e_ms=e2e_ms_max, e2e_tokens=e2e_tokens_all, clocks=clk.summary(),
-                launches=launches, kprof=kprof, prefill_s=prefill_s,
+                launches=launches, kprof=kprof, prefill_s=prefill_s, detail=detail[:24],
                 ctx_window=[ctx_before, ctx_after], weight_bytes=weight_bytes,
                 h2d=req_h.numel() * 4, d2h=(out_h.numel() + nn_h.numel()) * 4)
     ctx.close()
@@ -420,6 +435,7 @@ def main():
         "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": info["h2d"],
                 "d2h_bytes_per_step": info["d2h"]},
         "gpu_launches": info["launches"], "clocks": info["clocks"],
+        "kernel_detail": info["detail"],
         "prefill_s": info["prefill_s"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

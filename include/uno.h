@@ -140,6 +140,15 @@ int uno_spec_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *
  * into out_tokens_dev int32 [n_req]. */
 int uno_ar_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *out_tokens_dev);
 
+/* CUDA graphs (no counterpart on the pages: launch plumbing).  With graphs on
+ * (the default), the first uno_spec_step / uno_ar_step call with a given
+ * (n_req, req_ids_dev, output pointers) runs eagerly, the second captures the
+ * step into a CUDA graph on an internal stream and launches it on the
+ * context stream, and later calls replay it.  Calls while profiling run
+ * eagerly.  enable = 0 turns capture off (already captured graphs are kept
+ * but not used). */
+int uno_set_graphs(uno_ctx *ctx, int enable);
+
 /* Free a request's slot and pages (stream-ordered after earlier work). */
 int uno_release(uno_ctx *ctx, int req_id);
 
@@ -177,6 +186,37 @@ int uno_debug_kv(uno_ctx *ctx, int req_id, int layer, int pos0, int n, void *k_h
                  void *v_host);
 
 /*
+ * gated_lora_linear as a stand-alone call: the projection the diffusion and
+ * AR paths share, with the adapter switched per row (summary page "通过离散
+ * 扩散实现 LLM 无损加速：扩散增强自回归模型", section 方法关键点: rank-r LoRA
+ * diffusion weights on every layer; blog page "…Uno 的无损加速之路", section
+ * Diffusion Distillation：一步蒸馏 + 块级扩散: the gate switches the adapter off
+ * at clean positions and on at noised ones):
+ *
+ *   U = round(gate[m] * scale * X A^T)           [M, r], model dtype
+ *   Y = X W^T + U Bl^T                            [M, N], fp32
+ *
+ *   dtype: UNO_F32 or UNO_BF16 (X, W, A, Bl in that dtype, row-major dense:
+ *   X [M, K], W [N, K], A [r, K], Bl [N, r]); A == NULL: no adapter (r
+ *   ignored); gate_dev: f32 [M] or NULL (all rows gated on).
+ *   workspace_dev: at least uno_gated_lora_linear_workspace_bytes() bytes,
+ *   256-byte aligned, zero-filled before its first use (left zeroed after);
+ *   calls sharing one workspace must not overlap on the GPU.
+ * bf16 shapes with K and r multiples of 64 run on the tcgen05 kernel; the
+ * others on the SIMT kernel.  Never synchronises.
+ */
+size_t uno_gated_lora_linear_workspace_bytes(int M, int N, int K, int r, int dtype);
+int uno_gated_lora_linear(int dtype, const void *X_dev, const void *W_dev, const void *A_dev,
+                          const void *Bl_dev, const float *gate_dev, int M, int N, int K, int r,
+                          float scale, float *Y_dev, void *workspace_dev, size_t workspace_bytes,
+                          uno_stream_t stream);
+
+/* Diagnostic (no counterpart on the pages): process-wide launch counts of
+ * out[0] tensor-core GEMM, out[1] SIMT GEMM, out[2] tensor-core attention,
+ * out[3] SIMT attention kernels, so a caller can tell which path ran. */
+int uno_debug_launch_counts(int64_t *out);
+
+/*
  * Profiling tap (no counterpart on the pages: measurement plumbing).
  * Kernel classes: the gated-LoRA GEMMs (incl. the LM head), attention,
  * draft_sample / AR sampling, spec_verify, and everything else (row assembly,
@@ -192,6 +232,15 @@ int uno_debug_kv(uno_ctx *ctx, int req_id, int layer, int pos0, int n, void *k_h
 enum uno_kernel_class { UNO_K_GEMM = 0, UNO_K_ATTN, UNO_K_SAMPLE, UNO_K_VERIFY, UNO_K_OTHER, UNO_K_N };
 int uno_profile_begin(uno_ctx *ctx, unsigned class_mask);
 int uno_profile_end(uno_ctx *ctx, int64_t *launches, double *ms, double *bytes);
+/* One profiled launch: its class, for GEMMs the shape (rows m, columns n,
+ * depth k, adapter rank r or 0), and its event time. */
+typedef struct uno_prof_record {
+  int32_t cls, m, n, k, r;
+  float ms;
+} uno_prof_record;
+/* Copies up to max records of the last uno_profile_end into out (may be NULL)
+ * and returns how many there are (negative on a bad context). */
+int uno_profile_records(uno_ctx *ctx, uno_prof_record *out, int max);
 
 /*
  * spec_verify as a stand-alone kernel: the rejection step of speculative

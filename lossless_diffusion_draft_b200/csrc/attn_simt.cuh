@@ -28,6 +28,7 @@ constexpr int ATT_KT = 32;       // keys per tile
 struct AttnParams {
   const void* qkv; int ld_qkv;   // rotated q in columns [0, H*hd)
   void* out; int ld_out;         // [M, H*hd]
+  void* out_lo;                  // rounding residual rows (split GEMM input) or null
   KvLayout kv; int layer;
   int H, Hkv;
   float scale;
@@ -145,7 +146,9 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
         const int d = lane + 32 * e;
-        if (d < HD) out[(size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d] = from_f<T>(o_i[t][e] * inv);
+        if (d < HD)
+          store_split<T>(out, reinterpret_cast<T*>(p.out_lo),
+                         (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d, o_i[t][e] * inv);
       }
     }
     return;
@@ -190,7 +193,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
       O += __ldcg(w + d) * f;
     }
     const int tk = qi / G, g = qi % G;
-    out[(size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d] = from_f<T>(O / L);
+    store_split<T>(out, reinterpret_cast<T*>(p.out_lo),
+                   (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d, O / L);
   }
 }
 

@@ -1,0 +1,391 @@
+// Paged-KV grouped-query attention with the block-causal mask on the
+// 5th-generation tensor cores (bf16 K/V and q, fp32 scores and softmax).
+//
+// Mask (blog page "不砸掉重来，给自回归 LLM 装一对“扩散翅膀”：Uno 的无损加速之路",
+// section Diffusion Distillation：一步蒸馏 + 块级扩散): the clean sequence is
+// causal; a noised block is causal inside itself and sees every clean token
+// before it.  In the decode passes every key of a request (cache, pending
+// token, block) is in the pool and the rule is "key position <= query
+// position" for every row.
+//
+// One CTA takes (key split, query tile, request x kv head).  Its 128 query
+// rows are (token, head of the kv group) pairs, so the GQA group shares each
+// K/V tile: 17 draft rows x 4 heads = 68 rows per KV stream.
+//   warp 4  TMA: one KV page (64 keys) per tile, K and V as 64x64 boxes of the
+//           pool viewed as a 2-D [rows, head_dim] tensor;
+//   warp 5  MMA: S = Q K^T (M=128, N=64) into a double-buffered TMEM score
+//           tile; O_t = P V (M=128, N=head_dim, B operand MN-major) into a
+//           double-buffered TMEM output tile;
+//   warps 0-3 (thread = query row): read the score row, online softmax in the
+//           log2 domain, write P (bf16) to shared memory in the MMA's
+//           swizzled layout, and fold each O_t into a register accumulator
+//           with the running max correction.
+// With several key splits each CTA writes (m, l, O) partials and
+// attn_merge_kernel (one CTA per query row) adds them in split order.  Every
+// wait is bounded.
+#pragma once
+
+#include "layers.cuh"
+#include "tc_common.cuh"
+
+namespace uno {
+
+constexpr int ATC_THREADS = 192;
+constexpr int ATC_QROWS = 128;
+constexpr int ATC_KT = 64;          // keys per tile = one KV page
+constexpr int ATC_STAGES = 4;
+constexpr int ST_ATTN_TIMEOUT = 16;
+
+struct AttnTcParams {
+  const bf16* q; int ld_q;          // rotated q rows [M, H * HD]
+  bf16* out; int ld_out;            // [M, H * HD]
+  bf16* out_lo;                     // rounding residual rows (split GEMM input) or null
+  int layer, H, Hkv, n_pages, pages_per_req;
+  const int32_t* page_table;
+  float scale_log2;                 // log2(e) / sqrt(HD)
+  int rows_per_req;
+  const int32_t* row_pos; const int32_t* row_slot;
+  int n_splits, n_qtiles;
+  float* ws;                        // split partials [group][split][128][HD + 2]
+  int32_t* status;
+};
+
+template <int HD>
+struct AtcCfg {
+  static constexpr int NB = HD / 64;
+  static constexpr int Q_BYTES = ATC_QROWS * HD * 2;
+  static constexpr int KV_BYTES = ATC_KT * HD * 2;      // K or V of one stage
+  static constexpr int P_BYTES = ATC_QROWS * ATC_KT * 2;
+  static constexpr int SMEM = Q_BYTES + ATC_STAGES * 2 * KV_BYTES + 2 * P_BYTES + 1024 + 256;
+  static constexpr int TMEM_COLS = (2 * ATC_KT + 2 * HD) <= 256 ? 256 : 512;
+  static constexpr int S_COL = 0;             // score tiles at columns 0, 64
+  static constexpr int O_COL = 2 * ATC_KT;    // output tiles at 128, 128 + HD
+};
+
+// One query row of the output in bf16, plus its rounding residual if `lo`.
+template <int HD>
+__device__ __forceinline__ void attn_store_row(bf16* dst, bf16* lo, const float* o, float inv) {
+#pragma unroll
+  for (int d = 0; d < HD; d += 2) {
+    const float a = o[d] * inv, b = o[d + 1] * inv;
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    *reinterpret_cast<__nv_bfloat162*>(dst + d) = h;
+    if (lo)
+      *reinterpret_cast<__nv_bfloat162*>(lo + d) =
+          __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(ATC_THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, const AttnTcParams p) {
+  using C = AtcCfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint8_t* sQ = smem;                                   // NB boxes [128 rows x 64]
+  uint8_t* sK = sQ + C::Q_BYTES;                        // [STAGES] NB boxes [64 keys x 64]
+  uint8_t* sV = sK + ATC_STAGES * C::KV_BYTES;          // [STAGES] NB boxes [64 keys x 64]
+  uint8_t* sP = sV + ATC_STAGES * C::KV_BYTES;          // [2] [128 rows x 64 keys]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  uint64_t* kv_full = bars;                             // [STAGES]
+  uint64_t* kv_empty = bars + ATC_STAGES;               // [STAGES]
+  uint64_t* s_full = bars + 2 * ATC_STAGES;             // [2]
+  uint64_t* s_empty = s_full + 2;                       // [2] (4 warps)
+  uint64_t* p_full = s_empty + 2;                       // [2] (4 warps)
+  uint64_t* o_full = p_full + 2;                        // [2]
+  uint64_t* o_empty = o_full + 2;                       // [2] (4 warps)
+  uint64_t* drain = o_empty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  volatile int* s_ok = reinterpret_cast<volatile int*>(s_tmem + 4);   // [4]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
+  const int req = z / p.Hkv, kvh = z % p.Hkv;
+  const int G = p.H / p.Hkv;
+  const int TQ = ATC_QROWS / G;                  // tokens per query tile
+  const int tok0 = qt * TQ;
+  const int ntok = min(TQ, p.rows_per_req - tok0);
+  const int nq = ntok * G;
+  const int row0 = req * p.rows_per_req + tok0;
+  const int slot = p.row_slot[row0];
+  const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
+  int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
+  if (ntiles > p.pages_per_req) {
+    if (threadIdx.x == 0 && split == 0) raise_status(p.status, ST_POS_OVERFLOW);
+    ntiles = p.pages_per_req;
+  }
+  const int t_begin = (int)((long long)ntiles * split / p.n_splits);
+  const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
+  const int n = t_end - t_begin;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ATC_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // query rows -> shared memory, K-major 128-byte swizzle (zero rows past nq)
+  if (warp < 4) {
+    const int r = threadIdx.x;
+    const uint4* src = nullptr;
+    if (r < nq) {
+      const int tk = r / G, g = r % G;
+      src = reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + tk) * p.ld_q + (size_t)(kvh * G + g) * HD);
+    }
+#pragma unroll
+    for (int j = 0; j < HD / 8; ++j) {
+      const uint4 v = src ? src[j] : make_uint4(0, 0, 0, 0);
+      const int box = j >> 3, c = j & 7;
+      *reinterpret_cast<uint4*>(sQ + box * (ATC_QROWS * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
+    fence_async_smem();
+  }
+  if (warp == 4 && lane == 0) prefetch_map(&kvmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n && !*s_abort; ++i) {
+        const int stage = i % ATC_STAGES;
+        const uint32_t phase = (uint32_t)(i / ATC_STAGES) & 1;
+        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
+        mbar_expect_tx(&kv_full[stage], 2 * C::KV_BYTES);
+        const int page = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+        const int rk = (((p.layer * p.n_pages + page) * 2 + 0) * p.Hkv + kvh) * KV_PAGE;
+        const int rv = (((p.layer * p.n_pages + page) * 2 + 1) * p.Hkv + kvh) * KV_PAGE;
+#pragma unroll
+        for (int b = 0; b < C::NB; ++b) {
+          tma_load_2d(sK + stage * C::KV_BYTES + b * (ATC_KT * 128), &kvmap, &kv_full[stage], b * 64, rk);
+          tma_load_2d(sV + stage * C::KV_BYTES + b * (ATC_KT * 128), &kvmap, &kv_full[stage], b * 64, rv);
+        }
+        ++issued;
+      }
+      if (*s_abort) {
+        for (int i = max(0, issued - ATC_STAGES); i < issued; ++i)
+          mbar_wait(&kv_full[i % ATC_STAGES], (uint32_t)(i / ATC_STAGES) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(ATC_QROWS, ATC_KT);
+      constexpr uint32_t idesc_pv = idesc_bf16(ATC_QROWS, HD) | (1u << 16);   // B MN-major
+      bool issued_any = false;
+      auto qk = [&](int i) -> bool {
+        const int stage = i % ATC_STAGES, sb = i & 1;
+        if (!mbar_wait(&kv_full[stage], (uint32_t)(i / ATC_STAGES) & 1)) return false;
+        if (!mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + C::S_COL + sb * ATC_KT;
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const int b = ks >> 2, kk = ks & 3;
+          mma_bf16(d, sdesc_k128(smem_u32(sQ + b * (ATC_QROWS * 128)) + kk * 32),
+                   sdesc_k128(smem_u32(sK + stage * C::KV_BYTES + b * (ATC_KT * 128)) + kk * 32),
+                   idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        issued_any = true;
+        mma_commit(&s_full[sb]);
+        return true;
+      };
+      bool ok = qk(0);
+      for (int i = 0; i < n && ok; ++i) {
+        if (i + 1 < n && !qk(i + 1)) { ok = false; break; }
+        const int stage = i % ATC_STAGES, b2 = i & 1;
+        if (!mbar_wait(&p_full[b2], (uint32_t)(i >> 1) & 1)) { ok = false; break; }
+        if (!mbar_wait(&o_empty[b2], ((uint32_t)(i >> 1) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + C::O_COL + b2 * HD;
+#pragma unroll
+        for (int ks = 0; ks < ATC_KT / 16; ++ks)
+          mma_bf16(d, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
+                   sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
+                   idesc_pv, ks > 0 ? 1u : 0u);
+        mma_commit(&o_full[b2]);
+        mma_commit(&kv_empty[stage]);
+      }
+      if (!ok) {
+        *s_abort = 1;
+        if (issued_any) {
+          mma_commit(drain);
+          mbar_wait(drain, 0);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
+    const int r = threadIdx.x;
+    const int qpos = (r < nq) ? p.row_pos[row0 + r / G] : -1;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float o[HD];
+#pragma unroll
+    for (int d = 0; d < HD; ++d) o[d] = 0.f;
+    float m = -INFINITY, l = 0.f, corr_prev = 1.f;
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+      const int sb = i & 1;
+      bool w = !*s_abort && mbar_wait(&s_full[sb], (uint32_t)(i >> 1) & 1);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+      float s[ATC_KT];
+#pragma unroll
+      for (int c0 = 0; c0 < ATC_KT; c0 += 16) tmem_ld16(lane_base + C::S_COL + sb * ATC_KT + c0, s + c0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      const int kp0 = (t_begin + i) * ATC_KT;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < ATC_KT; ++j) {
+        s[j] = (kp0 + j <= qpos) ? s[j] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[j]);
+      }
+      const float m_new = fmaxf(m, mx);
+      const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
+      float psum = 0.f;
+      uint32_t pk[ATC_KT / 2];
+#pragma unroll
+      for (int j = 0; j < ATC_KT; j += 2) {
+        const float a = (m_new == -INFINITY) ? 0.f : exp2f(s[j] - m_new);
+        const float b = (m_new == -INFINITY) ? 0.f : exp2f(s[j + 1] - m_new);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+        psum += __low2float(h2) + __high2float(h2);    // the P the MMA will use
+        pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      l = l * corr + psum;
+      m = m_new;
+      // fold the previous tile's output (its P used the previous max)
+      if (i > 0) {
+        const int ob = (i - 1) & 1;
+        bool w2 = !*s_abort && mbar_wait(&o_full[ob], (uint32_t)((i - 1) >> 1) & 1);
+        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += 16) {
+          float v[16];
+          tmem_ld16(lane_base + C::O_COL + ob * HD + c0, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * corr_prev + v[e];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[ob]);
+      }
+      corr_prev = corr;
+      // P row -> shared memory (K-major over keys, 128-byte swizzle)
+      uint8_t* prow = sP + sb * C::P_BYTES + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+    }
+    if (ok && n > 0) {
+      const int ob = (n - 1) & 1;
+      bool w2 = !*s_abort && mbar_wait(&o_full[ob], (uint32_t)((n - 1) >> 1) & 1);
+      if (__all_sync(0xffffffffu, w2)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += 16) {
+          float v[16];
+          tmem_ld16(lane_base + C::O_COL + ob * HD + c0, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * corr_prev + v[e];
+        }
+        tc_fence_before();
+      } else {
+        ok = false;
+      }
+    }
+    // epilogue-uniform decision
+    if (lane == 0) s_ok[warp] = ok ? 1 : 0;
+    epi_bar();
+    const bool all_ok = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
+    if (!all_ok) {
+      *s_abort = 1;
+    } else if (p.n_splits == 1) {
+      if (r < nq) {
+        const int tk = r / G, g = r % G;
+        const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD;
+        attn_store_row<HD>(p.out + oo, p.out_lo ? p.out_lo + oo : nullptr, o, 1.f / l);
+      }
+    } else if (r < nq) {
+      // split partial (o unnormalised, m in log2 units, l); merged by
+      // attn_merge_kernel
+      const size_t group = (size_t)z * p.n_qtiles + qt;
+      float* w = p.ws + ((group * p.n_splits + split) * ATC_QROWS + r) * (HD + 2);
+#pragma unroll
+      for (int d = 0; d < HD; d += 4)
+        *reinterpret_cast<float4*>(w + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
+      w[HD] = m;
+      w[HD + 1] = l;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*s_abort && threadIdx.x == 0) raise_status(p.status, ST_ATTN_TIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS));
+  }
+}
+
+// Merge of the split partials: one CTA per (query row, group), one thread
+// per head_dim element; splits are added in split order.
+template <int HD>
+__global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
+  const int r = blockIdx.x, group = blockIdx.y;
+  const int z = group / p.n_qtiles, qt = group % p.n_qtiles;
+  const int req = z / p.Hkv, kvh = z % p.Hkv;
+  const int G = p.H / p.Hkv;
+  const int TQ = ATC_QROWS / G;
+  const int tok0 = qt * TQ;
+  const int ntok = min(TQ, p.rows_per_req - tok0);
+  if (r >= ntok * G) return;
+  const int d = threadIdx.x;
+  const size_t sstride = (size_t)ATC_QROWS * (HD + 2);
+  const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * (HD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, wg[s * sstride + HD]);
+  float L = 0.f, O = 0.f;
+  for (int s = 0; s < p.n_splits; ++s) {
+    const float* ws = wg + s * sstride;
+    const float ms = ws[HD];
+    if (ms == -INFINITY) continue;
+    const float f = exp2f(ms - M);
+    L += ws[HD + 1] * f;
+    O += ws[d] * f;
+  }
+  const int row0 = req * p.rows_per_req + tok0;
+  const int tk = r / G, g = r % G;
+  const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;
+  store_split<bf16>(p.out, p.out_lo, oo, O / L);
+}
+
+}  // namespace uno

@@ -20,7 +20,7 @@ enum Epilogue : int {
   EPI_STORE = 0,      // out (model dtype) = acc * alpha
   EPI_STORE_F32 = 1,  // out (fp32) = acc * alpha
   EPI_ADD_F32 = 2,    // out (fp32) += acc            (residual stream)
-  EPI_GATED = 3       // out (model dtype) = acc * row_gate[m]   (LoRA down-projection)
+  EPI_GATED = 3       // out (model dtype) = acc * alpha * row_gate[m]   (LoRA down-projection)
 };
 
 struct GemmSeg {
@@ -37,6 +37,8 @@ struct GemmParams {
   const void* U; int ldu; int r;   // LoRA-B extension (U null: none)
   int epi; void* out; int ldo; float alpha;
   const float* row_gate;
+  int lo_off;        // > 0: X and U also hold lo rows (x - bf16(x)) this many rows below
+  void* out_lo;      // EPI_GATED: where the lo part of the output goes (or null)
 };
 
 template <typename T, int MT, int NC>
@@ -138,9 +140,13 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmParams p) {
         case EPI_ADD_F32:
           reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + n] += v;
           break;
-        default:
-          reinterpret_cast<T*>(p.out)[(size_t)row * p.ldo + n] = from_f<T>(v * p.row_gate[row]);
+        default: {
+          const float y = v * p.alpha * p.row_gate[row];
+          const T hi = from_f<T>(y);
+          reinterpret_cast<T*>(p.out)[(size_t)row * p.ldo + n] = hi;
+          if (p.out_lo) reinterpret_cast<T*>(p.out_lo)[(size_t)row * p.ldo + n] = from_f<T>(y - to_f(hi));
           break;
+        }
       }
     }
   }

@@ -1,0 +1,347 @@
+// Gated-LoRA linear layer on the 5th-generation tensor cores (tcgen05 + TMEM,
+// operands staged by TMA), for bf16 models.
+//
+//   Y[m, n] = sum_k X[m, k] W[n, k] + sum_j U[m, uoff + j] Bl[n, j]
+//
+// Decode passes have few rows (17 per request in the draft pass) and stream
+// the whole weight set once per pass, so the kernel is built around the
+// weight stream:
+//  * swap-AB: a 128-row tile of W is the MMA's A operand (M = 128) and the
+//    token rows are its N dimension (NT = 16..256), so no MMA row is wasted
+//    on padding tokens;
+//  * the LoRA-B product is folded in as extra K-blocks: after the K/64 blocks
+//    of (W, X) the same accumulator takes r/64 blocks of (Bl, U), so the
+//    base weights and the adapter share one pass over the output tile;
+//  * stream-K: the (tile, k-block) units are split evenly over one persistent
+//    CTA per SM, so every SM streams the same number of weight bytes whatever
+//    the tile count; a tile cut between CTAs is finished by whichever
+//    contributor arrives last (atomic counter, no waiting), which adds the
+//    fp32 partials in a fixed order (deterministic) and runs the epilogue;
+//  * warp roles: warp 4 issues TMA loads into a STAGES-deep ring, warp 5
+//    issues tcgen05.mma into a double-buffered TMEM accumulator, warps 0-3
+//    drain TMEM (tcgen05.ld) and write the epilogue while the next part's
+//    MMAs run.
+// Every mbarrier wait is bounded (about two seconds of global time); on
+// timeout the kernel raises a status bit, stops, waits (bounded) for its own
+// TMA copies, frees its TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "tc_common.cuh"
+
+namespace uno {
+
+constexpr int TC_THREADS = 192;
+constexpr int TC_BM = 128;         // weight rows per tile (MMA M)
+constexpr int TC_BK = 64;          // k elements per block (128 bytes of bf16)
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
+constexpr int ST_GEMM_TIMEOUT = 8;
+
+struct TcMaps {
+  CUtensorMap x;       // activations [rows, K], box {64, NT}
+  CUtensorMap u;       // LoRA intermediate [rows, 3r], box {64, NT}
+  CUtensorMap w[3];    // weights of each segment [n, K], box {64, 128}
+  CUtensorMap b[3];    // LoRA-B of each segment [n, r], box {64, 128}
+};
+
+struct TcSeg { int n0, n, u_off; };
+
+struct TcParams {
+  int M, N, KB, RB;          // rows, columns, k-blocks of K, k-blocks of r (0: no LoRA)
+  int n_tiles, m_tiles;
+  int nseg; TcSeg seg[3];
+  int units, grid;           // stream-K: units = tiles * (KB + RB), split over grid CTAs
+  int max_parts;             // partial slots per tile
+  int epi; void* out; int ldo; float alpha; const float* row_gate;
+  float* ws; unsigned* counters;
+  int32_t* status;
+  int lo_off;                // split mode: row offset of the lo rows of X and U
+  void* out_lo;              // EPI_GATED in split mode: lo part of the output (out + lo_off rows)
+};
+
+// ---------------------------------------------------------------------------
+// Stream-K partition.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int sk_start(int i, int units, int grid) {
+  return (int)(((long long)i * units) / grid);
+}
+__device__ __forceinline__ int sk_owner(int u, int units, int grid) {
+  int i = (int)(((long long)u * grid) / units);
+  while (i + 1 < grid && sk_start(i + 1, units, grid) <= u) ++i;
+  while (i > 0 && sk_start(i, units, grid) > u) --i;
+  return i;
+}
+
+// SPLIT: every activation row x is fed as two bf16 rows hi = bf16(x) and
+// lo = bf16(x - hi) (rows lo_off apart in the buffer); the MMA's N covers
+// both (2 NT columns) and the epilogue adds column m and column NT + m, so
+// the product sees x to ~16 mantissa bits while the weights stream once.
+template <int NT, bool SPLIT>
+struct TcCfg {
+  static constexpr int NMMA = SPLIT ? 2 * NT : NT;           // MMA N
+  static constexpr int B_BYTES = NMMA * TC_BK * 2;
+  static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = NMMA < 32 ? 64 : 2 * NMMA;  // two accumulators, power of two
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+// Partial-tile slot of a contributor: its first part uses slot 0, its last
+// part slot 1 (parts in between cover whole tiles and need none).
+__device__ __forceinline__ float* tc_slot(float* ws, int cta, int slot, int NT) {
+  return ws + ((size_t)cta * 2 + slot) * NT * TC_BM;
+}
+
+__device__ __forceinline__ void tc_store(const TcParams& p, int m, int n, float v) {
+  const size_t o = (size_t)m * p.ldo + n;
+  switch (p.epi) {
+    case EPI_STORE: reinterpret_cast<bf16*>(p.out)[o] = from_f<bf16>(v * p.alpha); break;
+    case EPI_STORE_F32: reinterpret_cast<float*>(p.out)[o] = v * p.alpha; break;
+    case EPI_ADD_F32: reinterpret_cast<float*>(p.out)[o] += v; break;
+    default: {
+      const float y = v * p.alpha * p.row_gate[m];
+      const bf16 hi = from_f<bf16>(y);
+      reinterpret_cast<bf16*>(p.out)[o] = hi;
+      if (p.out_lo) reinterpret_cast<bf16*>(p.out_lo)[o] = from_f<bf16>(y - to_f(hi));
+      break;
+    }
+  }
+}
+
+template <int NT, bool SPLIT>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  using C = TcCfg<NT, SPLIT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * TC_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* full = bars;                      // [STAGES] TMA -> MMA
+  uint64_t* empty = bars + C::STAGES;         // [STAGES] MMA -> TMA
+  uint64_t* tfull = bars + 2 * C::STAGES;     // [2] MMA -> epilogue
+  uint64_t* tempty = tfull + 2;               // [2] epilogue -> MMA
+  uint64_t* drain = tempty + 2;               // MMA drain on abort
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);
+  volatile int* s_ok = reinterpret_cast<volatile int*>(s_tmem + 4);   // [2][4]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KBt = p.KB + p.RB;
+  const int u0 = sk_start(blockIdx.x, p.units, p.grid);
+  const int u1 = sk_start(blockIdx.x + 1, p.units, p.grid);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);   // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_map(&maps.x);
+    for (int s = 0; s < p.nseg; ++s) prefetch_map(&maps.w[s]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      for (int u = u0; u < u1 && !*s_abort;) {
+        const int t = u / KBt, kb0 = u % KBt;
+        const int kb1 = min(KBt, kb0 + (u1 - u));
+        const int nt = t / p.m_tiles, mt = t % p.m_tiles;
+        const int n_row = nt * TC_BM;
+        int sg = 0;
+        for (int s = 1; s < p.nseg; ++s)
+          if (n_row >= p.seg[s].n0) sg = s;
+        const int n_loc = n_row - p.seg[sg].n0;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { *s_abort = 1; break; }
+          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * TC_A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          if (kb < p.KB) {
+            tma_load_2d(a_dst, &maps.w[sg], &full[stage], kb * TC_BK, n_loc);
+            tma_load_2d(b_dst, &maps.x, &full[stage], kb * TC_BK, mt * NT);
+            if (SPLIT)
+              tma_load_2d(b_dst + NT * 128, &maps.x, &full[stage], kb * TC_BK, p.lo_off + mt * NT);
+          } else {
+            const int j = (kb - p.KB) * TC_BK;
+            tma_load_2d(a_dst, &maps.b[sg], &full[stage], j, n_loc);
+            tma_load_2d(b_dst, &maps.u, &full[stage], p.seg[sg].u_off + j, mt * NT);
+            if (SPLIT)
+              tma_load_2d(b_dst + NT * 128, &maps.u, &full[stage], p.seg[sg].u_off + j,
+                          p.lo_off + mt * NT);
+          }
+          ++issued;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        u += kb1 - kb0;
+      }
+      if (*s_abort) {
+        // wait (bounded) for the copies still in flight: the last
+        // min(issued, STAGES) issues, walking the ring backwards
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < min(issued, C::STAGES); ++i) {
+          if (st == 0) { st = C::STAGES; ph ^= 1; }
+          --st;
+          mbar_wait(&full[st], ph);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(TC_BM, C::NMMA);
+      int stage = 0, part = 0, issued = 0;
+      uint32_t phase = 0;
+      for (int u = u0; u < u1 && !*s_abort; ++part) {
+        const int kb0 = u % KBt;
+        const int kb1 = min(KBt, kb0 + (u1 - u));
+        const int buf = part & 1;
+        const uint32_t use = (uint32_t)(part >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1)) { *s_abort = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * C::NMMA);
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(sA + stage * TC_A_BYTES);
+          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k)
+            mma_bf16(d, sdesc_k128(a + k * 32), sdesc_k128(b + k * 32), idesc,
+                     (kb > kb0 || k > 0) ? 1u : 0u);
+          ++issued;
+          mma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) { *s_abort = 1; break; }
+        mma_commit(&tfull[buf]);
+        u += kb1 - kb0;
+      }
+      if (*s_abort && issued) {
+        mma_commit(drain);          // tracks every MMA this thread issued
+        mbar_wait(drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    const int n_local = warp * 32 + lane;
+    int part = 0;
+    for (int u = u0; u < u1; ++part) {
+      const int t = u / KBt, kb0 = u % KBt;
+      const int kb1 = min(KBt, kb0 + (u1 - u));
+      u += kb1 - kb0;
+      const int buf = part & 1;
+      const uint32_t use = (uint32_t)(part >> 1);
+      // warp-uniform, then epilogue-uniform decision to go on
+      bool ok = !*s_abort && mbar_wait(&tfull[buf], use & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) s_ok[(part & 1) * 4 + warp] = ok ? 1 : 0;
+      epi_bar();
+      const int pb = (part & 1) * 4;
+      if (!(s_ok[pb] && s_ok[pb + 1] && s_ok[pb + 2] && s_ok[pb + 3])) { *s_abort = 1; break; }
+      tc_fence_after();
+      const int nt = t / p.m_tiles, mt = t % p.m_tiles;
+      const int n = nt * TC_BM + n_local;
+      const int m0 = mt * NT;
+      const int mrows = min(NT, p.M - m0);
+      const bool whole = (kb0 == 0 && kb1 == KBt);
+      const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * C::NMMA);
+      float* wsl = tc_slot(p.ws, blockIdx.x, part == 0 ? 0 : 1, NT);
+#pragma unroll 1
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        if (SPLIT) {
+          float vl[16];
+          tmem_ld16(tbase + NT + c0, vl);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += vl[i];
+        }
+        if (whole) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < mrows) tc_store(p, m0 + c0 + i, n, v[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < mrows) wsl[(size_t)(c0 + i) * TC_BM + n_local] = v[i];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (!whole) {
+        __threadfence();
+        epi_bar();
+        const int first = sk_owner(t * KBt, p.units, p.grid);
+        const int last = sk_owner(t * KBt + KBt - 1, p.units, p.grid);
+        if (threadIdx.x == 0) {
+          const unsigned done = atomicAdd(&p.counters[t], 1u);
+          const bool is_last = (done == (unsigned)(last - first));
+          *s_last = is_last ? 1 : 0;
+          if (is_last) p.counters[t] = 0u;
+        }
+        epi_bar();
+        if (*s_last) {
+          __threadfence();
+          // contributors in CTA order (deterministic); four rows at a time so
+          // that independent loads are in flight together
+#pragma unroll 1
+          for (int m = 0; m < mrows; m += 4) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+            for (int i = first; i <= last; ++i) {
+              const int slot = (sk_start(i, p.units, p.grid) >= t * KBt) ? 0 : 1;
+              const float* src = tc_slot(p.ws, i, slot, NT) + (size_t)m * TC_BM + n_local;
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (m + j < mrows) acc[j] += __ldcg(src + (size_t)j * TC_BM);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (m + j < mrows) tc_store(p, m0 + m + j, n, acc[j]);
+          }
+        }
+        epi_bar();   // s_last is reused by the next cut part
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*s_abort && threadIdx.x == 0) raise_status(p.status, ST_GEMM_TIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS));
+  }
+}
+
+}  // namespace uno

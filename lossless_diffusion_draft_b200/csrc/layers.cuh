@@ -89,44 +89,57 @@ __global__ void build_rows_kernel(const RowArgs a) {
   for (int i = threadIdx.x; i < a.d; i += blockDim.x) x[i] = to_f(e[i]);
 }
 
+// Store y in the model dtype; with `lo` also the rounding residual
+// y - round(y) (the GEMMs' split-activation rows).
+template <typename T>
+__device__ __forceinline__ void store_split(T* hi, T* lo, size_t i, float y) {
+  const T h = from_f<T>(y);
+  hi[i] = h;
+  if (lo) lo[i] = from_f<T>(y - to_f(h));
+}
+
 // RMSNorm: out = x / sqrt(mean(x^2) + eps) * gain, one CTA per row.
 template <typename T, int NT>
-__global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* gain, T* out, int d,
-                                                     int ld_out, float eps) {
+__global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* gain, T* out, T* lo,
+                                                     int d, int ld_out, float eps) {
   __shared__ float red[32];
   const float* xr = x + (size_t)blockIdx.x * d;
   float s = 0.f;
   for (int i = threadIdx.x; i < d; i += NT) s += xr[i] * xr[i];
   s = block_sum<NT>(s, red);
   const float inv = 1.0f / sqrtf(s / (float)d + eps);
-  T* o = out + (size_t)blockIdx.x * ld_out;
-  for (int i = threadIdx.x; i < d; i += NT) o[i] = from_f<T>(xr[i] * inv * to_f(gain[i]));
+  const size_t o = (size_t)blockIdx.x * ld_out;
+  for (int i = threadIdx.x; i < d; i += NT)
+    store_split<T>(out + o, lo ? lo + o : nullptr, i, xr[i] * inv * to_f(gain[i]));
 }
 
-// RoPE (rotate-half) on q and k in place in the fused qkv rows, and write the
-// rotated k and v of every row into the paged pool at (slot, position).
+// RoPE (rotate-half) on q and k of the fused fp32 qkv rows: the rotated q goes
+// to q_out (model dtype, the attention's input) and the rotated k and the v
+// of every row into the paged pool at (slot, position), each rounded once.
 // cos/sin come from a table [max_pos][head_dim / 2] computed on the host in
 // double precision.
 template <typename T>
-__global__ void rope_kv_kernel(T* qkv, int ld_qkv, const int32_t* row_pos, const int32_t* row_slot,
-                               const float* cos_t, const float* sin_t, int max_pos, int H, int Hkv,
-                               int hd, KvLayout kv, int layer, int32_t* status) {
+__global__ void rope_kv_kernel(const float* qkv, int ld_qkv, T* q_out, int ld_q,
+                               const int32_t* row_pos, const int32_t* row_slot, const float* cos_t,
+                               const float* sin_t, int max_pos, int H, int Hkv, int hd, KvLayout kv,
+                               int layer, int32_t* status) {
   const int row = blockIdx.x;
   const int pos = row_pos[row], slot = row_slot[row];
   const int half = hd / 2;
-  T* r = qkv + (size_t)row * ld_qkv;
+  const float* r = qkv + (size_t)row * ld_qkv;
   int ok_pos = pos < max_pos;
   const int pc = ok_pos ? pos : 0;
   // q heads then k heads: pairs (i, i + half)
   for (int idx = threadIdx.x; idx < (H + Hkv) * half; idx += blockDim.x) {
     const int h = idx / half, i = idx % half;
     const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
-    T* base = r + (size_t)h * hd;
-    const float x1 = to_f(base[i]), x2 = to_f(base[i + half]);
+    const float* base = r + (size_t)h * hd;
+    const float x1 = base[i], x2 = base[i + half];
     const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
     if (h < H) {
-      base[i] = from_f<T>(y1);
-      base[i + half] = from_f<T>(y2);
+      T* q = q_out + (size_t)row * ld_q + (size_t)h * hd;
+      q[i] = from_f<T>(y1);
+      q[i + half] = from_f<T>(y2);
     } else {
       int ok;
       const size_t off = kv.offset(layer, slot, pos, 0, h - H, ok);
@@ -139,24 +152,24 @@ __global__ void rope_kv_kernel(T* qkv, int ld_qkv, const int32_t* row_pos, const
       }
     }
   }
-  const T* v = r + (size_t)(H + Hkv) * hd;
+  const float* v = r + (size_t)(H + Hkv) * hd;
   for (int idx = threadIdx.x; idx < Hkv * hd; idx += blockDim.x) {
     const int h = idx / hd, i = idx % hd;
     int ok;
     const size_t off = kv.offset(layer, slot, pos, 1, h, ok);
-    if (ok && ok_pos) reinterpret_cast<T*>(kv.pool)[off + i] = v[(size_t)h * hd + i];
+    if (ok && ok_pos) reinterpret_cast<T*>(kv.pool)[off + i] = from_f<T>(v[(size_t)h * hd + i]);
   }
 }
 
-// SwiGLU: out[:, f] = silu(gu[:, f]) * gu[:, F + f].
+// SwiGLU: out[:, f] = silu(gu[:, f]) * gu[:, F + f], from the fp32 gate|up rows.
 template <typename T>
-__global__ void swiglu_kernel(const T* gu, int F, T* out) {
+__global__ void swiglu_kernel(const float* gu, int F, T* out, T* lo) {
   const int row = blockIdx.x;
-  const T* g = gu + (size_t)row * 2 * F;
-  T* o = out + (size_t)row * F;
+  const float* g = gu + (size_t)row * 2 * F;
+  const size_t o = (size_t)row * F;
   for (int f = threadIdx.x; f < F; f += blockDim.x) {
-    const float a = to_f(g[f]), b = to_f(g[F + f]);
-    o[f] = from_f<T>(a / (1.0f + expf(-a)) * b);
+    const float a = g[f], b = g[F + f];
+    store_split<T>(out + o, lo ? lo + o : nullptr, f, a / (1.0f + expf(-a)) * b);
   }
 }
 

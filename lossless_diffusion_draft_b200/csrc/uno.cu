@@ -19,14 +19,213 @@
 #include <string>
 #include <vector>
 
+#include <map>
+#include <tuple>
+
 #include "../../include/uno.h"
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 #include "layers.cuh"
 #include "sampling.cuh"
 
 using namespace uno;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// GEMM environment: tensor-core workspace and the TMA descriptor cache.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+struct MapKey {
+  const void* p;
+  uint64_t rows, cols, ld;
+  uint32_t box_rows;
+  bool operator<(const MapKey& o) const {
+    return std::tie(p, rows, cols, ld, box_rows) < std::tie(o.p, o.rows, o.cols, o.ld, o.box_rows);
+  }
+};
+
+constexpr int TC_COUNTERS = 1 << 16;
+constexpr int TC_MIN_UNITS = 8;
+
+// Process-wide launch counts per kernel path (read by uno_debug_launch_counts).
+int64_t g_launches[4] = {0, 0, 0, 0};   // tc gemm, simt gemm, tc attention, simt attention
+
+struct GemmEnv {
+  int sm_count = 148;
+  int x_rows_alloc = 0;           // rows the activation buffers hold (>= any box)
+  float* ws = nullptr;            // [sm_count][2][256][128] fp32 partial tiles
+  unsigned* counters = nullptr;   // [TC_COUNTERS], zero, left zero
+  int32_t* status = nullptr;
+  std::map<MapKey, CUtensorMap> maps;
+  bool tc_disabled = false;
+
+  static size_t ws_bytes(int sm) { return (size_t)sm * 2 * 256 * TC_BM * 4; }
+
+  // bf16 2-D row-major tensor [rows, cols] with row stride ld elements; box
+  // of 64 columns (128 bytes, 128-byte swizzle) by box_rows rows.
+  const CUtensorMap* map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                         uint32_t box_rows) {
+    MapKey k{base, rows, cols, ld, box_rows};
+    auto it = maps.find(k);
+    if (it != maps.end()) return &it->second;
+    EncodeTiledFn f = encode_fn();
+    if (!f) return nullptr;
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)TC_BK, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    if (f(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return nullptr;
+    return &maps.emplace(k, m).first->second;
+  }
+};
+
+template <int NT, bool SPLIT>
+bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  // A box may not be larger than the tensor: the activation tensors are
+  // described with at least NT rows (the buffers hold x_rows_alloc >= 256
+  // rows); rows past M only feed output columns the epilogue never stores.
+  // In split mode they also cover the lo rows lo_off below.
+  const uint64_t xrows = (SPLIT ? (uint64_t)p.lo_off : 0) + std::max<uint64_t>(p.M, NT);
+  if ((uint64_t)env.x_rows_alloc < xrows) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (p.seg[s].n < TC_BM) return false;
+  const CUtensorMap* mx = env.map(p.X, xrows, p.K, p.ldx, NT);
+  if (!mx) return false;
+  maps.x = *mx;
+  maps.u = *mx;
+  if (p.U) {
+    const CUtensorMap* mu = env.map(p.U, xrows, p.ldu, p.ldu, NT);
+    if (!mu) return false;
+    maps.u = *mu;
+  }
+  TcParams tp{};
+  tp.M = p.M;
+  tp.N = p.N;
+  tp.KB = p.K / TC_BK;
+  tp.RB = p.U ? p.r / TC_BK : 0;
+  tp.nseg = p.nseg;
+  for (int s = 0; s < p.nseg; ++s) {
+    const GemmSeg& g = p.seg[s];
+    const CUtensorMap* mw = env.map(g.W, g.n, p.K, p.K, TC_BM);
+    if (!mw) return false;
+    maps.w[s] = *mw;
+    maps.b[s] = *mw;
+    if (p.U) {
+      if (!g.lB) return false;
+      const CUtensorMap* mb = env.map(g.lB, g.n, p.r, p.r, TC_BM);
+      if (!mb) return false;
+      maps.b[s] = *mb;
+    }
+    tp.seg[s] = TcSeg{g.n0, g.n, g.u_off};
+  }
+  tp.n_tiles = (p.N + TC_BM - 1) / TC_BM;
+  tp.m_tiles = (p.M + NT - 1) / NT;
+  if ((long long)tp.n_tiles * tp.m_tiles > TC_COUNTERS) return false;
+  tp.units = tp.n_tiles * tp.m_tiles * (tp.KB + tp.RB);
+  // at least TC_MIN_UNITS k-blocks per CTA: a tile is then cut into few
+  // parts and its last contributor has few partials to add
+  tp.grid = std::max(1, std::min(env.sm_count, tp.units / TC_MIN_UNITS));
+  tp.max_parts = 2;
+  tp.epi = p.epi;
+  tp.out = p.out;
+  tp.ldo = p.ldo;
+  tp.alpha = p.alpha;
+  tp.row_gate = p.row_gate;
+  tp.ws = env.ws;
+  tp.counters = env.counters;
+  tp.status = env.status;
+  tp.lo_off = SPLIT ? p.lo_off : 0;
+  tp.out_lo = p.out_lo;
+  using Cfg = TcCfg<NT, SPLIT>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
+      return false;
+    attr = true;
+  }
+  gemm_tc_kernel<NT, SPLIT><<<tp.grid, TC_THREADS, Cfg::SMEM, st>>>(maps, tp);
+  g_launches[0]++;
+  return true;
+}
+
+// Whether the tensor-core kernel takes this bf16 GEMM: K and r in 64-element
+// blocks, every segment but the last a whole number of 128-row tiles, 16-byte
+// aligned rows.
+bool tc_shape_ok(const GemmParams& p) {
+  if (p.K % TC_BK || (p.U && p.r % TC_BK) || p.ldx % 8 || (p.U && p.ldu % 8)) return false;
+  for (int s = 0; s + 1 < p.nseg; ++s)
+    if (p.seg[s].n % TC_BM) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if ((uintptr_t)p.seg[s].W & 15 || (p.U && ((uintptr_t)p.seg[s].lB & 15))) return false;
+  return ((uintptr_t)p.X & 15) == 0 && (!p.U || ((uintptr_t)p.U & 15) == 0);
+}
+
+template <typename T>
+void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st) {
+  const dim3 block(256);
+  g_launches[1]++;
+  if (p.M <= 8) {
+    gemm_simt_kernel<T, 8, 4><<<dim3((p.N + 31) / 32, (p.M + 7) / 8), block, 0, st>>>(p);
+  } else if (p.M <= 16) {
+    gemm_simt_kernel<T, 16, 4><<<dim3((p.N + 31) / 32, (p.M + 15) / 16), block, 0, st>>>(p);
+  } else {
+    gemm_simt_kernel<T, 32, 2><<<dim3((p.N + 15) / 16, (p.M + 31) / 32), block, 0, st>>>(p);
+  }
+}
+
+// Runs one gated-LoRA GEMM: tcgen05 for bf16 shapes it takes, SIMT otherwise.
+template <typename T>
+void gemm_run(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
+  if (p.M <= 0 || p.N <= 0) return;
+  if (sizeof(T) == 2 && !env.tc_disabled && tc_shape_ok(p)) {
+    bool ok;
+    if (p.lo_off > 0 && p.M <= 128) {
+      if (p.M <= 16) ok = launch_tc<16, true>(env, p, st);
+      else if (p.M <= 32) ok = launch_tc<32, true>(env, p, st);
+      else if (p.M <= 64) ok = launch_tc<64, true>(env, p, st);
+      else ok = launch_tc<128, true>(env, p, st);
+    } else {
+      if (p.M <= 16) ok = launch_tc<16, false>(env, p, st);
+      else if (p.M <= 32) ok = launch_tc<32, false>(env, p, st);
+      else if (p.M <= 64) ok = launch_tc<64, false>(env, p, st);
+      else if (p.M <= 128) ok = launch_tc<128, false>(env, p, st);
+      else ok = launch_tc<256, false>(env, p, st);
+    }
+    if (ok) return;
+  }
+  gemm_simt_dispatch<T>(p, st);
+}
+
+}  // namespace
 
 struct uno_ctx {
   uno_shape s{};
@@ -54,10 +253,11 @@ struct uno_ctx {
   // activations (sized for M_max rows)
   int M_max = 0;
   float* x = nullptr;          // [M, d] fp32 residual
-  void* xn = nullptr;          // [M, max(d, F)]
-  void* qkv = nullptr;         // [M, (H + 2 Hkv) hd]
+  void* xn = nullptr;          // [M, max(d, F)] GEMM input (normed rows, SwiGLU output)
+  float* qkv = nullptr;        // [M, (H + 2 Hkv) hd] fp32 projection output
+  void* qbuf = nullptr;        // [M, H hd] rotated q (attention input)
   void* attn = nullptr;        // [M, H hd]
-  void* gu = nullptr;          // [M, 2F]
+  float* gu = nullptr;         // [M, 2F] fp32 gate|up output
   void* U = nullptr;           // [M, 3r] LoRA intermediate
   int32_t *row_pos = nullptr, *row_slot = nullptr;
   float* row_gate = nullptr;
@@ -83,13 +283,31 @@ struct uno_ctx {
   int32_t* d_status = nullptr;
   int last_n_req = 0;
   std::string err;
+  GemmEnv genv;
+  CUtensorMap kv_map;            // the pool as a 2-D bf16 [rows, head_dim] tensor
+  bool kv_map_ok = false;
+
+  // CUDA graphs of whole steps, keyed by their arguments
+  struct GraphEntry {
+    int kind, n_req;
+    const void *a, *b, *c;
+    int seen = 0;
+    cudaGraphExec_t exec = nullptr;
+    int64_t launches[UNO_K_N] = {};
+    double bytes[UNO_K_N] = {};
+    int64_t glaunch[4] = {};
+  };
+  std::vector<GraphEntry> graphs;
+  bool graphs_enabled = true;
+  cudaStream_t cap_stream = nullptr;
 
   // profiling tap
   unsigned prof_mask = 0;
   int64_t prof_launches[UNO_K_N] = {};
   double prof_bytes[UNO_K_N] = {};
-  struct ProfRec { int cls; cudaEvent_t a, b; };
+  struct ProfRec { int cls, m, n, k, r; cudaEvent_t a, b; };
   std::vector<ProfRec> prof_recs;
+  std::vector<uno_prof_record> prof_done;   // records of the last uno_profile_end
   std::vector<cudaEvent_t> ev_pool;
   size_t ev_next = 0;
 };
@@ -109,8 +327,10 @@ cudaEvent_t next_event(uno_ctx* c) {
 struct Prof {
   uno_ctx* c;
   int cls;
+  int m = 0, n = 0, k = 0, r = 0;
   cudaEvent_t a = nullptr, b = nullptr;
-  Prof(uno_ctx* c_, int cls_, double bytes) : c(c_), cls(cls_) {
+  Prof(uno_ctx* c_, int cls_, double bytes, int m_ = 0, int n_ = 0, int k_ = 0, int r_ = 0)
+      : c(c_), cls(cls_), m(m_), n(n_), k(k_), r(r_) {
     c->prof_launches[cls]++;
     c->prof_bytes[cls] += bytes;
     if (c->prof_mask & (1u << cls)) {
@@ -122,7 +342,7 @@ struct Prof {
   ~Prof() {
     if (b) {
       cudaEventRecord(b, c->stream);
-      c->prof_recs.push_back({cls, a, b});
+      c->prof_recs.push_back({cls, m, n, k, r, a, b});
     }
   }
 };
@@ -192,15 +412,8 @@ template <typename T>
 void launch_gemm(uno_ctx* c, const Gemm& g, cudaStream_t st) {
   const GemmParams& p = g.p;
   if (p.M <= 0 || p.N <= 0) return;
-  Prof prof(c, UNO_K_GEMM, gemm_bytes(p, sizeof(T)));
-  const dim3 block(256);
-  if (p.M <= 8) {
-    gemm_simt_kernel<T, 8, 4><<<dim3(ceil_div(p.N, 32), ceil_div(p.M, 8)), block, 0, st>>>(p);
-  } else if (p.M <= 16) {
-    gemm_simt_kernel<T, 16, 4><<<dim3(ceil_div(p.N, 32), ceil_div(p.M, 16)), block, 0, st>>>(p);
-  } else {
-    gemm_simt_kernel<T, 32, 2><<<dim3(ceil_div(p.N, 16), ceil_div(p.M, 32)), block, 0, st>>>(p);
-  }
+  Prof prof(c, UNO_K_GEMM, gemm_bytes(p, sizeof(T)), p.M, p.N, p.K, p.U ? p.r : 0);
+  gemm_run<T>(c->genv, p, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -218,17 +431,76 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
   const dim3 grid(p.n_splits, p.n_qtiles, n_req * p.Hkv);
   Prof prof(c, UNO_K_ATTN, 0.0);
   attn_simt_kernel<T, HD><<<grid, ATT_THREADS, smem, st>>>(p);
+  g_launches[3]++;
+  return UNO_OK;
+}
+
+template <int HD>
+int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
+                   void* out_lo) {
+  const uno_shape& s = c->s;
+  AttnTcParams p{};
+  p.q = (const bf16*)c->qbuf;
+  p.ld_q = s.n_heads * HD;
+  p.out = (bf16*)c->attn;
+  p.ld_out = s.n_heads * HD;
+  p.out_lo = (bf16*)out_lo;
+  p.layer = layer;
+  p.H = s.n_heads;
+  p.Hkv = s.n_kv_heads;
+  p.n_pages = c->kv.n_pages;
+  p.pages_per_req = c->kv.pages_per_req;
+  p.page_table = c->d_page_table;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  p.rows_per_req = rows_per_req;
+  p.row_pos = c->row_pos;
+  p.row_slot = c->row_slot;
+  const int G = s.n_heads / s.n_kv_heads;
+  p.n_qtiles = ceil_div(rows_per_req, ATC_QROWS / G);
+  const int groups = n_req * s.n_kv_heads * p.n_qtiles;
+  int S = 1;
+  if (decode && groups < c->genv.sm_count) {
+    S = ceil_div(c->genv.sm_count, groups);
+    S = std::max(1, std::min(S, c->kv.pages_per_req / 2));
+    while (S > 1 && (size_t)groups * S * ATC_QROWS * (HD + 2) > c->att_ws_floats) --S;
+    if (groups > c->att_groups_max) S = 1;
+  }
+  p.n_splits = S;
+  p.ws = c->att_ws;
+  p.status = c->d_status;
+  static bool attr = false;
+  if (!attr) {
+    CK(cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            AtcCfg<HD>::SMEM));
+    attr = true;
+  }
+  {
+    Prof prof(c, UNO_K_ATTN, 0.0);
+    attn_tc_kernel<HD><<<dim3(S, p.n_qtiles, n_req * s.n_kv_heads), ATC_THREADS,
+                         AtcCfg<HD>::SMEM, c->stream>>>(c->kv_map, p);
+  }
+  g_launches[2]++;
+  if (S > 1) {
+    Prof prof(c, UNO_K_ATTN, 0.0);
+    attn_merge_kernel<HD><<<dim3(ATC_QROWS, groups), HD, 0, c->stream>>>(p);
+  }
   return UNO_OK;
 }
 
 template <typename T>
-int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode) {
+int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
+                void* out_lo) {
   const uno_shape& s = c->s;
+  if (c->kv_map_ok) {
+    if (s.head_dim == 128) return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo);
+    if (s.head_dim == 64) return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo);
+  }
   AttnParams p{};
-  p.qkv = c->qkv;
-  p.ld_qkv = (s.n_heads + 2 * s.n_kv_heads) * s.head_dim;
+  p.qkv = c->qbuf;
+  p.ld_qkv = s.n_heads * s.head_dim;
   p.out = c->attn;
   p.ld_out = s.n_heads * s.head_dim;
+  p.out_lo = out_lo;
   p.kv = c->kv;
   p.layer = layer;
   p.H = s.n_heads;
@@ -308,15 +580,29 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
 
   const int xn_ld = std::max(d, F);
   const int ldu = 3 * r;
+  const int hhd = H * hd;
+  // Memory-bound passes (few rows) feed every GEMM input as a hi/lo pair of
+  // bf16 rows (x = hi + lo), the lo rows c->M_max rows below the hi rows.
+  const bool split = sizeof(T) == 2 && M <= 128;
+  const int lo = split ? c->M_max : 0;
+  auto lo_rows = [&](void* buf, int ld) -> T* {
+    return split ? reinterpret_cast<T*>(buf) + (size_t)lo * ld : nullptr;
+  };
+  T* xn_lo = lo_rows(c->xn, xn_ld);
+  T* act_lo = lo_rows(c->xn, F);
+  T* attn_lo = lo_rows(c->attn, hhd);
+  T* u_lo = lo_rows(c->U, ldu);
+  auto gated = [&](Gemm& g) { g.epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate); g.p.out_lo = u_lo; };
   for (int l = 0; l < s.n_layers; ++l) {
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->attn_norm[l], (T*)c->xn, d,
-                                               xn_ld, s.rms_eps);
+      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->attn_norm[l], (T*)c->xn, xn_lo,
+                                               d, xn_ld, s.rms_eps);
     });
     if (lora) {
       Gemm g(c->xn, xn_ld, M, d);
       g.seg(c->lA[UNO_PROJ_Q][l], r).seg(c->lA[UNO_PROJ_K][l], r).seg(c->lA[UNO_PROJ_V][l], r);
-      g.epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate);
+      gated(g);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     {
@@ -325,37 +611,43 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
           .seg(c->w[UNO_PROJ_K][l], Hkv * hd, lora ? c->lB[UNO_PROJ_K][l] : nullptr, r)
           .seg(c->w[UNO_PROJ_V][l], Hkv * hd, lora ? c->lB[UNO_PROJ_V][l] : nullptr, 2 * r);
       if (lora) g.lora(c->U, ldu, r);
-      g.epi(EPI_STORE, c->qkv, qkv_ld);
+      g.epi(EPI_STORE_F32, c->qkv, qkv_ld);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     other([&] {
-      rope_kv_kernel<T><<<M, 128, 0, st>>>((T*)c->qkv, qkv_ld, c->row_pos, c->row_slot, c->cos_t,
-                                           c->sin_t, c->max_pos, H, Hkv, hd, c->kv, l, c->d_status);
+      rope_kv_kernel<T><<<M, 128, 0, st>>>(c->qkv, qkv_ld, (T*)c->qbuf, hhd, c->row_pos,
+                                           c->row_slot, c->cos_t, c->sin_t, c->max_pos, H, Hkv, hd,
+                                           c->kv, l, c->d_status);
     });
     {
-      const int rc = launch_attn<T>(c, l, n_req, rows_per_req, kind != PASS_PREFILL);
+      const int rc = launch_attn<T>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo);
       if (rc) return rc;
     }
     if (lora) {
-      Gemm g(c->attn, H * hd, M, H * hd);
-      g.seg(c->lA[UNO_PROJ_O][l], r).epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate);
+      Gemm g(c->attn, hhd, M, hhd);
+      g.seg(c->lA[UNO_PROJ_O][l], r);
+      gated(g);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     {
-      Gemm g(c->attn, H * hd, M, H * hd);
+      Gemm g(c->attn, hhd, M, hhd);
       g.seg(c->w[UNO_PROJ_O][l], d, lora ? c->lB[UNO_PROJ_O][l] : nullptr, 0);
       if (lora) g.lora(c->U, ldu, r);
       g.epi(EPI_ADD_F32, c->x, d);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->ffn_norm[l], (T*)c->xn, d,
-                                               xn_ld, s.rms_eps);
+      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->ffn_norm[l], (T*)c->xn, xn_lo,
+                                               d, xn_ld, s.rms_eps);
     });
     if (lora) {
       Gemm g(c->xn, xn_ld, M, d);
       g.seg(c->lA[UNO_PROJ_GATE][l], r).seg(c->lA[UNO_PROJ_UP][l], r);
-      g.epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate);
+      gated(g);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     {
@@ -363,13 +655,16 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       g.seg(c->w[UNO_PROJ_GATE][l], F, lora ? c->lB[UNO_PROJ_GATE][l] : nullptr, 0)
           .seg(c->w[UNO_PROJ_UP][l], F, lora ? c->lB[UNO_PROJ_UP][l] : nullptr, r);
       if (lora) g.lora(c->U, ldu, r);
-      g.epi(EPI_STORE, c->gu, 2 * F);
+      g.epi(EPI_STORE_F32, c->gu, 2 * F);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
-    other([&] { swiglu_kernel<T><<<M, 256, 0, st>>>((const T*)c->gu, F, (T*)c->xn); });
+    other([&] { swiglu_kernel<T><<<M, 256, 0, st>>>(c->gu, F, (T*)c->xn, act_lo); });
     if (lora) {
       Gemm g(c->xn, F, M, F);
-      g.seg(c->lA[UNO_PROJ_DOWN][l], r).epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate);
+      g.seg(c->lA[UNO_PROJ_DOWN][l], r);
+      gated(g);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
     {
@@ -377,16 +672,18 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       g.seg(c->w[UNO_PROJ_DOWN][l], d, lora ? c->lB[UNO_PROJ_DOWN][l] : nullptr, 0);
       if (lora) g.lora(c->U, ldu, r);
       g.epi(EPI_ADD_F32, c->x, d);
+      g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
   }
   if (logits) {
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->final_norm, (T*)c->xn, d,
-                                               xn_ld, s.rms_eps);
+      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->final_norm, (T*)c->xn, xn_lo,
+                                               d, xn_ld, s.rms_eps);
     });
     Gemm g(c->xn, xn_ld, M, d);
     g.seg(c->lm_head, s.vocab).epi(EPI_STORE_F32, logits, s.vocab, 1.0f / s.temperature);
+    g.p.lo_off = lo;
     launch_gemm<T>(c, g, st);
   }
   CK(cudaGetLastError());
@@ -483,6 +780,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   const int n_pages = max_batch * ppr;
   const size_t kv_bytes = (size_t)L * n_pages * 2 * Hkv * KV_PAGE * hd * c->esz;
   if (dalloc(&c->kv_pool, kv_bytes) != cudaSuccess) return oom("kv pool");
+  // zeroed: keys past a request's length are masked out of the scores, and
+  // the values there must be finite so that P V (with P = 0) stays finite
+  cudaMemset(c->kv_pool, 0, kv_bytes);
   if (dalloc(&c->d_page_table, (size_t)max_batch * ppr * 4) != cudaSuccess) return oom("pages");
   if (dalloc(&c->d_cached, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
   if (dalloc(&c->d_pending, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
@@ -502,11 +802,12 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   c->M_max = M;
   const size_t e = c->esz;
   if (dalloc(&c->x, (size_t)M * d * 4) != cudaSuccess) return oom("x");
-  if (dalloc(&c->xn, (size_t)M * std::max(d, F) * e) != cudaSuccess) return oom("xn");
-  if (dalloc(&c->qkv, (size_t)M * (H + 2 * Hkv) * hd * e) != cudaSuccess) return oom("qkv");
-  if (dalloc(&c->attn, (size_t)M * H * hd * e) != cudaSuccess) return oom("attn");
-  if (dalloc(&c->gu, (size_t)M * 2 * F * e) != cudaSuccess) return oom("gu");
-  if (dalloc(&c->U, (size_t)M * 3 * lora_rank * e) != cudaSuccess) return oom("U");
+  if (dalloc(&c->xn, (size_t)2 * M * std::max(d, F) * e) != cudaSuccess) return oom("xn");
+  if (dalloc(&c->qkv, (size_t)M * (H + 2 * Hkv) * hd * 4) != cudaSuccess) return oom("qkv");
+  if (dalloc(&c->qbuf, (size_t)M * H * hd * e) != cudaSuccess) return oom("q");
+  if (dalloc(&c->attn, (size_t)2 * M * H * hd * e) != cudaSuccess) return oom("attn");
+  if (dalloc(&c->gu, (size_t)M * 2 * F * 4) != cudaSuccess) return oom("gu");
+  if (dalloc(&c->U, (size_t)2 * M * 3 * lora_rank * e) != cudaSuccess) return oom("U");
   if (dalloc(&c->row_pos, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_slot, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_gate, (size_t)M * 4) != cudaSuccess) return oom("rows");
@@ -544,14 +845,36 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   cudaMemset(c->req_counter, 0, (size_t)max_batch * 4);
   cudaMemset(c->drafts, 0, (size_t)max_batch * B * 4);
 
-  // attention split workspace: up to 2 waves of 148 CTAs
+  // attention split workspace: groups x splits <= about two waves of CTAs
   c->att_groups_max = max_batch * Hkv * ceil_div(B + 1, ATT_MAXQ / (H / Hkv));
-  c->att_ws_floats = (size_t)std::max(c->att_groups_max, 2 * 148 + c->att_groups_max) * ATT_MAXQ * (hd + 2);
+  c->att_ws_floats = (size_t)(2 * 148 + c->att_groups_max) * ATC_QROWS * (hd + 2);
   if (dalloc(&c->att_ws, c->att_ws_floats * 4) != cudaSuccess) return oom("attention ws");
   if (dalloc(&c->att_counters, (size_t)c->att_groups_max * 4) != cudaSuccess) return oom("attention ws");
   cudaMemset(c->att_counters, 0, (size_t)c->att_groups_max * 4);
   if (dalloc(&c->d_status, 4) != cudaSuccess) return oom("status");
   cudaMemset(c->d_status, 0, 4);
+
+  // tensor-core GEMM: one persistent CTA per SM, partial tiles, counters
+  {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    c->genv.sm_count = sms;
+    c->genv.x_rows_alloc = 2 * M;   // activation buffers: hi rows then lo rows
+    if (dalloc(&c->genv.ws, GemmEnv::ws_bytes(sms)) != cudaSuccess) return oom("gemm ws");
+    if (dalloc(&c->genv.counters, (size_t)TC_COUNTERS * 4) != cudaSuccess) return oom("gemm ws");
+    cudaMemset(c->genv.counters, 0, (size_t)TC_COUNTERS * 4);
+    c->genv.status = c->d_status;
+  }
+  // tensor-core attention: the pool as a [rows, head_dim] tensor, 64x64 boxes
+  if (s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && ATC_QROWS % G == 0) {
+    const uint64_t rows = (uint64_t)L * n_pages * 2 * Hkv * KV_PAGE;
+    const CUtensorMap* m = c->genv.map(c->kv_pool, rows, hd, hd, KV_PAGE);
+    if (m) {
+      c->kv_map = *m;
+      c->kv_map_ok = true;
+    }
+  }
   if (cudaDeviceSynchronize() != cudaSuccess) {
     uno_destroy(c);
     return UNO_ERR_CUDA;
@@ -565,13 +888,16 @@ int uno_destroy(uno_ctx* c) {
   if (c->stream) cudaStreamSynchronize(c->stream);
   cudaDeviceSynchronize();
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
-                  c->xn, c->qkv, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
+                  c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
                   c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
                   c->lse_ws, c->row_counter, c->req_counter, c->att_ws, c->att_counters,
-                  c->d_status};
+                  c->d_status, c->genv.ws, c->genv.counters};
   for (void* b : bufs)
     if (b) cudaFree(b);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
+  for (auto& g : c->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   delete c;
   return UNO_OK;
 }
@@ -618,14 +944,74 @@ int uno_prefill(uno_ctx* c, int n_req, const int32_t* prompts_dev, int prompt_st
   return UNO_OK;
 }
 
-int uno_spec_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev,
-                  int32_t* n_new_dev) {
-  if (!c) return UNO_ERR_ARG;
-  c->err.clear();
-  if (n_req < 1 || n_req > c->max_batch || !req_ids_dev || !out_tokens_dev || !n_new_dev)
-    return fail(c, UNO_ERR_ARG, "bad spec_step arguments");
+}  // extern "C"
+
+namespace {
+
+// Runs body() eagerly on the first call with a given argument set (which
+// also creates descriptors and kernel attributes), captures it into a CUDA
+// graph on the second call and replays the graph from then on.  Profiling
+// runs eagerly (its event pairs are host-side bookkeeping).
+template <typename F>
+int run_graphed(uno_ctx* c, int kind, int n_req, const void* a, const void* b, const void* d,
+                F&& body) {
+  if (!c->graphs_enabled || c->prof_mask) return body();
+  uno_ctx::GraphEntry* e = nullptr;
+  for (auto& g : c->graphs)
+    if (g.kind == kind && g.n_req == n_req && g.a == a && g.b == b && g.c == d) e = &g;
+  if (!e) {
+    c->graphs.emplace_back();
+    e = &c->graphs.back();
+    e->kind = kind; e->n_req = n_req; e->a = a; e->b = b; e->c = d;
+  }
+  if (e->exec) {
+    CK(cudaGraphLaunch(e->exec, c->stream));
+    for (int k = 0; k < UNO_K_N; ++k) {
+      c->prof_launches[k] += e->launches[k];
+      c->prof_bytes[k] += e->bytes[k];
+    }
+    for (int i = 0; i < 4; ++i) g_launches[i] += e->glaunch[i];
+    return UNO_OK;
+  }
+  if (e->seen++ == 0) return body();
+  if (!c->cap_stream) CK(cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking));
+  int64_t l0[UNO_K_N], g0[4];
+  double b0[UNO_K_N];
+  for (int k = 0; k < UNO_K_N; ++k) { l0[k] = c->prof_launches[k]; b0[k] = c->prof_bytes[k]; }
+  for (int i = 0; i < 4; ++i) g0[i] = g_launches[i];
+  cudaStream_t user = c->stream;
+  c->stream = c->cap_stream;
+  cudaError_t ce = cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal);
+  if (ce != cudaSuccess) {
+    c->stream = user;
+    return fail(c, UNO_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(ce));
+  }
+  const int rc = body();
+  cudaGraph_t graph = nullptr;
+  ce = cudaStreamEndCapture(c->cap_stream, &graph);
+  c->stream = user;
+  if (rc != UNO_OK || ce != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return rc != UNO_OK ? rc : fail(c, UNO_ERR_CUDA, std::string("end capture: ") + cudaGetErrorString(ce));
+  }
+  ce = cudaGraphInstantiate(&e->exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ce != cudaSuccess) {
+    e->exec = nullptr;
+    return fail(c, UNO_ERR_CUDA, std::string("instantiate: ") + cudaGetErrorString(ce));
+  }
+  for (int k = 0; k < UNO_K_N; ++k) {
+    e->launches[k] = c->prof_launches[k] - l0[k];
+    e->bytes[k] = c->prof_bytes[k] - b0[k];
+  }
+  for (int i = 0; i < 4; ++i) e->glaunch[i] = g_launches[i] - g0[i];
+  CK(cudaGraphLaunch(e->exec, c->stream));   // counted once, by the capture above
+  return UNO_OK;
+}
+
+int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev,
+                   int32_t* n_new_dev) {
   const int B = c->B, V = c->s.vocab;
-  c->last_n_req = n_req;
   int rc = forward_any(c, PASS_DRAFT, n_req, B + 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
   {
@@ -687,12 +1073,7 @@ int uno_spec_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* ou
   return UNO_OK;
 }
 
-int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
-  if (!c) return UNO_ERR_ARG;
-  c->err.clear();
-  if (n_req < 1 || n_req > c->max_batch || !req_ids_dev || !out_tokens_dev)
-    return fail(c, UNO_ERR_ARG, "bad ar_step arguments");
-  c->last_n_req = n_req;
+int ar_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
   int rc = forward_any(c, PASS_AR, n_req, 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
   SampleArgs a{};
@@ -719,6 +1100,46 @@ int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_
   return UNO_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int uno_spec_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev,
+                  int32_t* n_new_dev) {
+  if (!c) return UNO_ERR_ARG;
+  c->err.clear();
+  if (n_req < 1 || n_req > c->max_batch || !req_ids_dev || !out_tokens_dev || !n_new_dev)
+    return fail(c, UNO_ERR_ARG, "bad spec_step arguments");
+  c->last_n_req = n_req;
+  return run_graphed(c, 0, n_req, req_ids_dev, out_tokens_dev, n_new_dev, [&] {
+    return spec_step_body(c, n_req, req_ids_dev, out_tokens_dev, n_new_dev);
+  });
+}
+
+int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
+  if (!c) return UNO_ERR_ARG;
+  c->err.clear();
+  if (n_req < 1 || n_req > c->max_batch || !req_ids_dev || !out_tokens_dev)
+    return fail(c, UNO_ERR_ARG, "bad ar_step arguments");
+  c->last_n_req = n_req;
+  return run_graphed(c, 1, n_req, req_ids_dev, out_tokens_dev, nullptr,
+                     [&] { return ar_step_body(c, n_req, req_ids_dev, out_tokens_dev); });
+}
+
+int uno_set_graphs(uno_ctx* c, int enable) {
+  if (!c) return UNO_ERR_ARG;
+  c->graphs_enabled = enable != 0;
+  return UNO_OK;
+}
+
+int uno_profile_records(uno_ctx* c, uno_prof_record* out, int max) {
+  if (!c) return -UNO_ERR_ARG;
+  const int n = (int)c->prof_done.size();
+  if (out)
+    for (int i = 0; i < n && i < max; ++i) out[i] = c->prof_done[i];
+  return n;
+}
+
 int uno_profile_begin(uno_ctx* c, unsigned mask) {
   if (!c) return UNO_ERR_ARG;
   CK(cudaStreamSynchronize(c->stream));
@@ -736,10 +1157,12 @@ int uno_profile_end(uno_ctx* c, int64_t* launches, double* ms, double* bytes) {
   if (!c) return UNO_ERR_ARG;
   CK(cudaStreamSynchronize(c->stream));
   double t[UNO_K_N] = {};
+  c->prof_done.clear();
   for (const auto& r : c->prof_recs) {
     float e = 0.f;
     CK(cudaEventElapsedTime(&e, r.a, r.b));
     t[r.cls] += e;
+    c->prof_done.push_back(uno_prof_record{r.cls, r.m, r.n, r.k, r.r, e});
   }
   for (int k = 0; k < UNO_K_N; ++k) {
     if (launches) launches[k] = c->prof_launches[k];
@@ -823,10 +1246,83 @@ int uno_debug_kv(uno_ctx* c, int req, int layer, int pos0, int n, void* k_host, 
   return UNO_OK;
 }
 
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// ---------------------------------------------------------------------------
+// Stand-alone gated_lora_linear.
+// ---------------------------------------------------------------------------
+static int device_sms() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// Workspace: counters | partial tiles | U [max(M,256), r] | X staging [256, K]
+// (X is staged so that a tensor map never describes fewer rows than a box).
+static constexpr int LIN_MIN_ROWS = 256;
+size_t uno_gated_lora_linear_workspace_bytes(int M, int N, int K, int r, int dtype) {
+  if (M < 1 || N < 1 || K < 1 || r < 0 || (dtype != UNO_F32 && dtype != UNO_BF16)) return 0;
+  const size_t esz = dtype == UNO_BF16 ? 2 : 4;
+  return align256((size_t)TC_COUNTERS * 4) + align256(GemmEnv::ws_bytes(device_sms())) +
+         align256((size_t)std::max(M, LIN_MIN_ROWS) * std::max(r, 1) * esz) +
+         align256((size_t)LIN_MIN_ROWS * K * esz);
+}
+
+int uno_debug_launch_counts(int64_t* out) {
+  if (!out) return UNO_ERR_ARG;
+  for (int i = 0; i < 4; ++i) out[i] = g_launches[i];
+  return UNO_OK;
+}
+
+int uno_gated_lora_linear(int dtype, const void* X, const void* W, const void* A, const void* Bl,
+                          const float* gate, int M, int N, int K, int r, float scale, float* Y,
+                          void* ws, size_t ws_bytes, uno_stream_t stream) {
+  if (!X || !W || !Y || !ws || M < 1 || N < 1 || K < 1 || (A && (!Bl || r < 1)) ||
+      (dtype != UNO_F32 && dtype != UNO_BF16))
+    return UNO_ERR_ARG;
+  const int vec = dtype == UNO_BF16 ? 8 : 4;
+  if (K % vec || (A && r % vec) || ((uintptr_t)ws & 255)) return UNO_ERR_ARG;
+  if (ws_bytes < uno_gated_lora_linear_workspace_bytes(M, N, K, A ? r : 0, dtype)) return UNO_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  GemmEnv env;
+  env.sm_count = device_sms();
+  const size_t esz = dtype == UNO_BF16 ? 2 : 4;
+  char* base = (char*)ws;
+  env.counters = (unsigned*)base;
+  env.ws = (float*)(base + align256((size_t)TC_COUNTERS * 4));
+  void* U = base + align256((size_t)TC_COUNTERS * 4) + align256(GemmEnv::ws_bytes(env.sm_count));
+  void* Xs = (char*)U + align256((size_t)std::max(M, LIN_MIN_ROWS) * std::max(A ? r : 0, 1) * esz);
+  env.x_rows_alloc = std::max(M, LIN_MIN_ROWS);
+  if (M < LIN_MIN_ROWS) {
+    if (cudaMemcpyAsync(Xs, X, (size_t)M * K * esz, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return UNO_ERR_CUDA;
+    X = Xs;
+  }
+  if (A) {
+    GemmParams pa{};
+    pa.X = X; pa.ldx = K; pa.M = M; pa.K = K; pa.N = r;
+    pa.seg[0] = GemmSeg{A, nullptr, 0, r, 0};
+    pa.nseg = 1;
+    pa.epi = gate ? EPI_GATED : EPI_STORE;
+    pa.out = U; pa.ldo = r; pa.alpha = scale; pa.row_gate = gate;
+    if (dtype == UNO_BF16) gemm_run<bf16>(env, pa, st);
+    else gemm_run<float>(env, pa, st);
+  }
+  GemmParams p{};
+  p.X = X; p.ldx = K; p.M = M; p.K = K; p.N = N;
+  p.seg[0] = GemmSeg{W, A ? Bl : nullptr, 0, N, 0};
+  p.nseg = 1;
+  if (A) { p.U = U; p.ldu = r; p.r = r; }
+  p.epi = EPI_STORE_F32; p.out = Y; p.ldo = N; p.alpha = 1.f;
+  if (dtype == UNO_BF16) gemm_run<bf16>(env, p, st);
+  else gemm_run<float>(env, p, st);
+  return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Stand-alone spec_verify.
 // ---------------------------------------------------------------------------
-static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct VerifyWs {
   size_t counters, req_counters, lse, partial, total;

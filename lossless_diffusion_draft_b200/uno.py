@@ -77,6 +77,12 @@ def load_library(path=LIB_PATH):
         "uno_request_state": (i32, [vp, i32, vp, vp]),
         "uno_debug_read": (i32, [vp, i32, vp, sz]),
         "uno_debug_kv": (i32, [vp, i32, i32, i32, i32, vp, vp]),
+        "uno_gated_lora_linear_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
+        "uno_gated_lora_linear": (i32, [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp,
+                                        sz, vp]),
+        "uno_debug_launch_counts": (i32, [vp]),
+        "uno_set_graphs": (i32, [vp, i32]),
+        "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
         "uno_spec_verify_workspace_bytes": (sz, [i32, i32, i32]),
@@ -204,6 +210,10 @@ def uno_ar_step(ctx, req_ids_dev, out_tokens_dev):
     _check(code, ctx.handle)
 
 
+def uno_set_graphs(ctx, enable):
+    _check(load_library().uno_set_graphs(ctx.handle, int(bool(enable))), ctx.handle)
+
+
 def uno_release(ctx, req_id):
     _check(load_library().uno_release(ctx.handle, int(req_id)), ctx.handle)
 
@@ -240,6 +250,30 @@ def uno_debug_kv(ctx, req_id, layer, pos0, n, k_host, v_host):
                                        v_host.data_ptr()), ctx.handle)
 
 
+def uno_gated_lora_linear_workspace_bytes(M, N, K, r, dtype):
+    return int(load_library().uno_gated_lora_linear_workspace_bytes(M, N, K, r, dtype))
+
+
+def uno_gated_lora_linear(X, W, A, Bl, gate, scale, Y, workspace, stream=None):
+    """Y (f32 CUDA [M, N]) = X W^T + round(gate * scale * X A^T) Bl^T; see include/uno.h."""
+    import torch
+    dtype = UNO_BF16 if X.dtype == torch.bfloat16 else UNO_F32
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[0] if A is not None else 0
+    code = load_library().uno_gated_lora_linear(
+        dtype, _ptr(X), _ptr(W), _ptr(A), _ptr(Bl), _ptr(gate), M, N, K, r, scale, _ptr(Y),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(code)
+
+
+def uno_debug_launch_counts():
+    """{'tc_gemm', 'simt_gemm', 'tc_attn', 'simt_attn'}: process-wide launch counts."""
+    out = (ctypes.c_int64 * 4)()
+    _check(load_library().uno_debug_launch_counts(out))
+    return dict(zip(("tc_gemm", "simt_gemm", "tc_attn", "simt_attn"), list(out)))
+
+
 UNO_K_GEMM, UNO_K_ATTN, UNO_K_SAMPLE, UNO_K_VERIFY, UNO_K_OTHER = range(5)
 KERNEL_CLASSES = ("gemm", "attn", "sample", "verify", "other")
 
@@ -254,6 +288,23 @@ def uno_profile_end(ctx):
     launches, ms, nbytes = (ctypes.c_int64 * n)(), (ctypes.c_double * n)(), (ctypes.c_double * n)()
     _check(load_library().uno_profile_end(ctx.handle, launches, ms, nbytes), ctx.handle)
     return {k: (launches[i], ms[i], nbytes[i]) for i, k in enumerate(KERNEL_CLASSES)}
+
+
+class UnoProfRecord(ctypes.Structure):
+    _fields_ = [("cls", ctypes.c_int32), ("m", ctypes.c_int32), ("n", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("r", ctypes.c_int32), ("ms", ctypes.c_float)]
+
+
+def uno_profile_records(ctx):
+    """Per-launch records of the last uno_profile_end: list of dicts."""
+    lib = load_library()
+    n = lib.uno_profile_records(ctx.handle, None, 0)
+    if n < 0:
+        _check(-n, ctx.handle)
+    arr = (UnoProfRecord * max(n, 1))()
+    lib.uno_profile_records(ctx.handle, arr, n)
+    return [{"cls": KERNEL_CLASSES[a.cls], "m": a.m, "n": a.n, "k": a.k, "r": a.r, "ms": a.ms}
+            for a in arr[:n]]
 
 
 def uno_spec_verify_workspace_bytes(n_req, n_tests, vocab):
