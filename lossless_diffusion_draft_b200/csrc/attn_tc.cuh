@@ -35,6 +35,9 @@ constexpr int ATC_QROWS = 128;
 constexpr int ATC_KT = 64;          // keys per tile = one KV page
 constexpr int ATC_STAGES = 4;
 constexpr int ST_ATTN_TIMEOUT = 16;
+// Floats per query row of a split partial: O[HD], m, l, padded so that every
+// row starts on a 16-byte boundary (rows are written with float4 stores).
+__host__ __device__ constexpr int atc_ws_row(int hd) { return hd + 4; }
 
 struct AttnTcParams {
   const bf16* q; int ld_q;          // rotated q rows [M, H * HD]
@@ -46,7 +49,7 @@ struct AttnTcParams {
   int rows_per_req;
   const int32_t* row_pos; const int32_t* row_slot;
   int n_splits, n_qtiles;
-  float* ws;                        // split partials [group][split][128][HD + 2]
+  float* ws;                        // split partials [group][split][128][HD + 4]
   int32_t* status;
 };
 
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       // split partial (o unnormalised, m in log2 units, l); merged by
       // attn_merge_kernel
       const size_t group = (size_t)z * p.n_qtiles + qt;
-      float* w = p.ws + ((group * p.n_splits + split) * ATC_QROWS + r) * (HD + 2);
+      float* w = p.ws + ((group * p.n_splits + split) * ATC_QROWS + r) * atc_ws_row(HD);
 #pragma unroll
       for (int d = 0; d < HD; d += 4)
         *reinterpret_cast<float4*>(w + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
@@ -369,8 +372,8 @@ __global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
   const int ntok = min(TQ, p.rows_per_req - tok0);
   if (r >= ntok * G) return;
   const int d = threadIdx.x;
-  const size_t sstride = (size_t)ATC_QROWS * (HD + 2);
-  const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * (HD + 2);
+  const size_t sstride = (size_t)ATC_QROWS * atc_ws_row(HD);
+  const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * atc_ws_row(HD);
   float M = -INFINITY;
   for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, wg[s * sstride + HD]);
   float L = 0.f, O = 0.f;

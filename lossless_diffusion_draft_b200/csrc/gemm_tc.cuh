@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (whole) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (c0 + i < mrows) tc_store(p, m0 + c0 + i, n, v[i]);
+            if (c0 + i < mrows && n < p.N) tc_store(p, m0 + c0 + i, n, v[i]);
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              if (m + j < mrows) tc_store(p, m0 + m + j, n, acc[j]);
+              if (m + j < mrows && n < p.N) tc_store(p, m0 + m + j, n, acc[j]);
           }
         }
         epi_bar();   // s_last is reused by the next cut part

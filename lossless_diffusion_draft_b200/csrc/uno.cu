@@ -462,7 +462,7 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   if (decode && groups < c->genv.sm_count) {
     S = ceil_div(c->genv.sm_count, groups);
     S = std::max(1, std::min(S, c->kv.pages_per_req / 2));
-    while (S > 1 && (size_t)groups * S * ATC_QROWS * (HD + 2) > c->att_ws_floats) --S;
+    while (S > 1 && (size_t)groups * S * ATC_QROWS * atc_ws_row(HD) > c->att_ws_floats) --S;
     if (groups > c->att_groups_max) S = 1;
   }
   p.n_splits = S;
@@ -847,7 +847,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
 
   // attention split workspace: groups x splits <= about two waves of CTAs
   c->att_groups_max = max_batch * Hkv * ceil_div(B + 1, ATT_MAXQ / (H / Hkv));
-  c->att_ws_floats = (size_t)(2 * 148 + c->att_groups_max) * ATC_QROWS * (hd + 2);
+  c->att_ws_floats = (size_t)(2 * 148 + c->att_groups_max) * ATC_QROWS * atc_ws_row(hd);
   if (dalloc(&c->att_ws, c->att_ws_floats * 4) != cudaSuccess) return oom("attention ws");
   if (dalloc(&c->att_counters, (size_t)c->att_groups_max * 4) != cudaSuccess) return oom("attention ws");
   cudaMemset(c->att_counters, 0, (size_t)c->att_groups_max * 4);

@@ -320,3 +320,4 @@ def uno_spec_verify(p_dev, q_dev, drafts_dev, seed, streams_dev, pos0_dev, out_t
         _ptr(pos0_dev), _ptr(out_tokens_dev), _ptr(n_out_dev), _ptr(workspace_dev),
         workspace_dev.numel() * workspace_dev.element_size(), _stream_ptr(stream))
     _check(code)
+
