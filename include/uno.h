@@ -275,6 +275,36 @@ int uno_spec_verify(const float *p_dev, const float *q_dev, const int32_t *draft
                     int32_t *out_tokens_dev, int32_t *n_out_dev, void *workspace_dev,
                     size_t workspace_bytes, uno_stream_t stream);
 
+/*
+ * uno_spec_verify_noalloc: uno_spec_verify for callers that cannot allocate
+ * device memory at the point of the call (the pages have no counterpart: this
+ * is deployment plumbing).  Examples: a serving process whose device memory
+ * is handed out up front by its own pool, where an extra cudaMalloc would fail
+ * or exceed the budget; or a caller that cannot afford the device-wide
+ * synchronisation that cudaMalloc / cudaFree may imply.  Instead of a
+ * workspace, the call uses a fixed scratch array of
+ * uno_spec_verify_noalloc_max_bytes() bytes (4 MiB) that lives in the
+ * library's device image: every GPU that loads the library holds it until
+ * the process exits.  It allocates nothing (no cudaMalloc, cudaFree or other
+ * allocating routine).
+ *   Arguments, outputs and results are those of uno_spec_verify.
+ *   Sizes whose workspace (uno_spec_verify_workspace_bytes) exceeds the array
+ *   are rejected with UNO_ERR_CAPACITY before anything is enqueued.
+ *   The first call on a device looks up the array's device address on that
+ *   device (it must be the current device) and caches it; make that first
+ *   call before any stream capture.
+ *   All calls share the one array, which keeps the previous call's contents;
+ *   each call clears the part that must start at zero (its completion
+ *   counters) on the given stream before the kernel.  Calls that overlap on
+ *   the GPU (different streams, no ordering between them) race on the array
+ *   and give wrong results: serialise them.
+ */
+size_t uno_spec_verify_noalloc_max_bytes(void);
+int uno_spec_verify_noalloc(const float *p_dev, const float *q_dev, const int32_t *drafts_dev,
+                            int n_req, int n_tests, int vocab, uint64_t seed,
+                            const uint32_t *streams_dev, const int32_t *pos0_dev,
+                            int32_t *out_tokens_dev, int32_t *n_out_dev, uno_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

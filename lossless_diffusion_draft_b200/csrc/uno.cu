@@ -20,6 +20,7 @@
 #include <vector>
 
 #include <map>
+#include <mutex>
 #include <tuple>
 
 #include "../../include/uno.h"
@@ -1381,6 +1382,57 @@ int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n
   const int rows = n_req * 2 * n_tests;
   spec_verify_kernel<<<dim3(nch, rows), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// spec_verify without allocation.
+//
+// Some callers cannot allocate device memory when they need this kernel: a
+// serving process whose device memory is reserved up front by its own pool
+// (where a stray cudaMalloc fails or breaks the budget), or code that must
+// not trigger the implicit device synchronisation cudaMalloc/cudaFree can
+// cause.  For them the scratch lives in a fixed array in this library's
+// device image instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+static constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)4 << 20;   // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is asked
+// for once per device (with that device current) and cached.
+static int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return UNO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return UNO_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return UNO_OK;
+}
+
+size_t uno_spec_verify_noalloc_max_bytes(void) { return NOALLOC_SCRATCH_BYTES; }
+
+int uno_spec_verify_noalloc(const float* p, const float* q, const int32_t* drafts, int n_req,
+                            int n_tests, int vocab, uint64_t seed, const uint32_t* streams,
+                            const int32_t* pos0, int32_t* out_tokens, int32_t* n_out,
+                            uno_stream_t stream) {
+  const size_t need = uno_spec_verify_workspace_bytes(n_req, n_tests, vocab);
+  if (need == 0) return UNO_ERR_ARG;
+  if (need > NOALLOC_SCRATCH_BYTES) return UNO_ERR_CAPACITY;
+  void* ws = nullptr;
+  const int rc = noalloc_scratch(&ws);
+  if (rc != UNO_OK) return rc;
+  // the array keeps the previous call's contents: the completion counters
+  // (the first part of the layout) must start at zero
+  const VerifyWs w = verify_ws_layout(n_req, n_tests, vocab);
+  if (cudaMemsetAsync(ws, 0, w.lse, (cudaStream_t)stream) != cudaSuccess) return UNO_ERR_CUDA;
+  return uno_spec_verify(p, q, drafts, n_req, n_tests, vocab, seed, streams, pos0, out_tokens,
+                         n_out, ws, need, stream);
 }
 
 }  // extern "C"

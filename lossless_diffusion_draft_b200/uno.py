@@ -87,6 +87,8 @@ def load_library(path=LIB_PATH):
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
         "uno_spec_verify_workspace_bytes": (sz, [i32, i32, i32]),
         "uno_spec_verify": (i32, [vp, vp, vp, i32, i32, i32, u64, vp, vp, vp, vp, vp, sz, vp]),
+        "uno_spec_verify_noalloc_max_bytes": (sz, []),
+        "uno_spec_verify_noalloc": (i32, [vp, vp, vp, i32, i32, i32, u64, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -321,3 +323,17 @@ def uno_spec_verify(p_dev, q_dev, drafts_dev, seed, streams_dev, pos0_dev, out_t
         workspace_dev.numel() * workspace_dev.element_size(), _stream_ptr(stream))
     _check(code)
 
+
+def uno_spec_verify_noalloc_max_bytes():
+    return int(load_library().uno_spec_verify_noalloc_max_bytes())
+
+
+def uno_spec_verify_noalloc(p_dev, q_dev, drafts_dev, seed, streams_dev, pos0_dev, out_tokens_dev,
+                            n_out_dev, stream=None):
+    """uno_spec_verify with the library's fixed scratch array instead of a
+    workspace (for callers that cannot allocate device memory)."""
+    n_req, n_tests, vocab = p_dev.shape
+    code = load_library().uno_spec_verify_noalloc(
+        _ptr(p_dev), _ptr(q_dev), _ptr(drafts_dev), n_req, n_tests, vocab, seed, _ptr(streams_dev),
+        _ptr(pos0_dev), _ptr(out_tokens_dev), _ptr(n_out_dev), _stream_ptr(stream))
+    _check(code)
