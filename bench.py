@@ -198,6 +198,8 @@ def run_uno(args, rank, world, device):
     from lossless_diffusion_draft_b200 import synth, uno
 
     cfg = dict(synth.CONFIGS[args.workload])
+    if args.layers:
+        cfg["n_layers"] = args.layers
     shape = synth.model_shape(cfg)
     shape["dtype"] = cfg["dtype"]
     B = cfg["B"]
@@ -209,6 +211,10 @@ def run_uno(args, rank, world, device):
     stream = torch.cuda.current_stream()
     ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, batch, max_ctx,
                        cfg["seed"], stream)
+    if args.no_pdl:
+        uno.uno_set_pdl(ctx, False)
+    if args.no_graphs:
+        uno.uno_set_graphs(ctx, False)
 
     # centre the timed window on the run's mean context
     mean_ctx = prompt_len + gen // 2
@@ -309,6 +315,75 @@ def run_uno(args, rank, world, device):
     return info
 
 
+def run_micro(args, device):
+    """Kernel microbenchmarks (not the headline line): one kernel, K timed calls.
+
+    gemm:        uno_gated_lora_linear at a decode shape (--shape M,N,K,r), bf16;
+                 algorithmic bytes = weights + adapter + activations + fp32 output.
+    spec_verify: the spec_verify workload, p/q fp32 [4096 = 256 x 16, 151936];
+                 algorithmic bytes = both logit tensors read once.
+    """
+    from lossless_diffusion_draft_b200 import synth, uno
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pk = peaks()
+    if args.workload == "gemm":
+        M, N, K, r = (int(x) for x in args.shape.split(","))
+        g = torch.Generator(device=device).manual_seed(0)
+        X = torch.randn((M, K), generator=g, device=device).to(torch.bfloat16)
+        W = (torch.randn((N, K), generator=g, device=device) * 0.02).to(torch.bfloat16)
+        A = (torch.randn((r, K), generator=g, device=device) * 0.02).to(torch.bfloat16) if r else None
+        Bl = (torch.randn((N, r), generator=g, device=device) * 0.002).to(torch.bfloat16) if r else None
+        gate = torch.ones(M, device=device) if r else None
+        Y = torch.empty((M, N), device=device)
+        ws = torch.zeros(uno.uno_gated_lora_linear_workspace_bytes(M, N, K, r, uno.UNO_BF16),
+                         dtype=torch.uint8, device=device)
+        # the weights (>= tens of MB) are rotated through copies so that each
+        # call streams from HBM, not from L2
+        copies = max(1, int(512e6 // max(1, W.numel() * 2)))
+        Ws = [W.clone() for _ in range(min(copies, 8))]
+        call = lambda i: uno.uno_gated_lora_linear(X, Ws[i % len(Ws)], A, Bl, gate, 2.0, Y, ws)
+        nbytes = (N * K + N * r + M * K + M * r + r * K) * 2 + M * N * 4
+        unit, metric = "calls/s", f"gated_lora_linear M={M} N={N} K={K} r={r}"
+    else:
+        cfg = synth.SPEC_VERIFY_BENCH
+        n_req, R, V = cfg["requests"], cfg["rows_per_request"], cfg["vocab"]
+        p, q = synth.make_verify_logits(n_req * R, V, device, cfg["p_std"], cfg["q_noise_std"],
+                                        cfg["logits_seed"])
+        drafts = synth.make_drafts(q, seed=cfg["logits_seed"] + 1).view(n_req, R)
+        p, q = p.view(n_req, R, V), q.view(n_req, R, V)
+        streams = torch.arange(n_req, dtype=torch.int32, device=device)
+        pos0 = torch.zeros(n_req, dtype=torch.int32, device=device)
+        ws = torch.zeros(uno.uno_spec_verify_workspace_bytes(n_req, R, V), dtype=torch.uint8,
+                         device=device)
+        out = torch.empty((n_req, R + 1), dtype=torch.int32, device=device)
+        n_out = torch.empty(n_req, dtype=torch.int32, device=device)
+        call = lambda i: uno.uno_spec_verify(p, q, drafts, cfg["seed"], streams, pos0, out, n_out, ws)
+        nbytes = 2 * n_req * R * V * 4
+        unit, metric = "rows/s", "spec_verify [4096 x 151936] fp32 p and q"
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            call(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    gbs = nbytes / (ms / 1e3) / 1e9
+    value = (4096 if args.workload == "spec_verify" else 1) / (ms / 1e3)
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16" if args.workload == "gemm" else "f32", "data": "synthetic",
+            "config": {"workload": args.workload},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_call": nbytes, "peak_source": pk["source"]},
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -356,7 +431,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="uno", choices=["uno", "reference"])
     ap.add_argument("--workload", default="qwen8b",
-                    choices=["qwen8b", "qwen8b_maxbatch", "small", "tiny"])
+                    choices=["qwen8b", "qwen8b_maxbatch", "small", "tiny", "gemm", "spec_verify"])
+    ap.add_argument("--shape", default="17,4096,4096,128",
+                    help="gemm microbenchmark shape M,N,K,r")
+    ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
+    ap.add_argument("--no-graphs", action="store_true", help="no CUDA-graph capture of steps")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (small cases for profiler captures; the "
+                         "line's config records it)")
     ap.add_argument("--est-tokens-per-step", type=float, default=2.6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -366,6 +448,11 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     from lossless_diffusion_draft_b200 import synth
+    if args.workload in ("gemm", "spec_verify"):
+        from lossless_diffusion_draft_b200 import build
+        build.build()
+        run_micro(args, torch.device("cuda", local))
+        return
     cfg = synth.CONFIGS[args.workload]
     metric = "generated tokens/s (Psi-Spec, 1K in / 8K out)"
 
@@ -425,7 +512,9 @@ def main():
         "steps": info["K"], "warmup": info["W"], "ms_per_step": per_step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg["dtype"],
         "data": "synthetic (random-init weights, uniform-random prompt tokens)",
-        "config": {"workload": args.workload, "batch": info["batch"], "B": info["B"],
+        "config": {"workload": args.workload, "n_layers": info["cfg"]["n_layers"],
+                   "batch": info["batch"], "B": info["B"], "pdl": not args.no_pdl,
+                   "graphs": not args.no_graphs,
                    "prompt_len": cfg["prompt_len"], "gen_tokens": cfg["gen_tokens"],
                    "context_window": info["ctx_window"], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (15+ GB of weights streamed per pass)"},

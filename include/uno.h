@@ -149,6 +149,12 @@ int uno_ar_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *ou
  * but not used). */
 int uno_set_graphs(uno_ctx *ctx, int enable);
 
+/* Programmatic dependent launch (launch plumbing, on by default): each kernel
+ * may start while the previous one finishes and waits inside for its data
+ * (the tensor-core GEMM starts streaming weights first).  enable = 0 launches
+ * kernels in plain stream order.  Changing it drops captured graphs. */
+int uno_set_pdl(uno_ctx *ctx, int enable);
+
 /* Free a request's slot and pages (stream-ordered after earlier work). */
 int uno_release(uno_ctx *ctx, int req_id);
 

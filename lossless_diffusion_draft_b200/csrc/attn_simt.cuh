@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
   float* k_s = q_s + ATT_MAXQ * HD;                  // [KT][HD + 1]
   float* v_s = k_s + ATT_KT * (HD + 1);              // [KT][HD]
   __shared__ bool s_last;
+  pdl_trigger();
+  pdl_wait();
 
   const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
   const int req = z / p.Hkv, kvh = z % p.Hkv;

@@ -14,12 +14,12 @@
 //   warp 4  TMA: one KV page (64 keys) per tile, K and V as 64x64 boxes of the
 //           pool viewed as a 2-D [rows, head_dim] tensor;
 //   warp 5  MMA: S = Q K^T (M=128, N=64) into a double-buffered TMEM score
-//           tile; O_t = P V (M=128, N=head_dim, B operand MN-major) into a
-//           double-buffered TMEM output tile;
-//   warps 0-3 (thread = query row): read the score row, online softmax in the
-//           log2 domain, write P (bf16) to shared memory in the MMA's
-//           swizzled layout, and fold each O_t into a register accumulator
-//           with the running max correction.
+//           tile; O += P V (M=128, N=head_dim, B operand MN-major) into one
+//           TMEM accumulator for the whole key range;
+//   warps 0-3 (thread = query row): read the score row, softmax in the log2
+//           domain against a reference max that moves (rescaling O in TMEM)
+//           only when a tile's max exceeds it by more than 2^8, and write P
+//           (bf16) to shared memory in the MMA's swizzled layout.
 // With several key splits each CTA writes (m, l, O) partials and
 // attn_merge_kernel (one CTA per query row) adds them in split order.  Every
 // wait is bounded.
@@ -60,9 +60,9 @@ struct AtcCfg {
   static constexpr int KV_BYTES = ATC_KT * HD * 2;      // K or V of one stage
   static constexpr int P_BYTES = ATC_QROWS * ATC_KT * 2;
   static constexpr int SMEM = Q_BYTES + ATC_STAGES * 2 * KV_BYTES + 2 * P_BYTES + 1024 + 256;
-  static constexpr int TMEM_COLS = (2 * ATC_KT + 2 * HD) <= 256 ? 256 : 512;
+  static constexpr int TMEM_COLS = 256;       // 2 score tiles + the output accumulator
   static constexpr int S_COL = 0;             // score tiles at columns 0, 64
-  static constexpr int O_COL = 2 * ATC_KT;    // output tiles at 128, 128 + HD
+  static constexpr int O_COL = 2 * ATC_KT;    // output accumulator at 128 .. 128 + HD
 };
 
 // One query row of the output in bf16, plus its rounding residual if `lo`.
@@ -96,13 +96,14 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   uint64_t* s_full = bars + 2 * ATC_STAGES;             // [2]
   uint64_t* s_empty = s_full + 2;                       // [2] (4 warps)
   uint64_t* p_full = s_empty + 2;                       // [2] (4 warps)
-  uint64_t* o_full = p_full + 2;                        // [2]
-  uint64_t* o_empty = o_full + 2;                       // [2] (4 warps)
-  uint64_t* drain = o_empty + 2;
+  uint64_t* o_full = p_full + 2;                        // one phase per PV(i)
+  uint64_t* drain = o_full + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_ok = reinterpret_cast<volatile int*>(s_tmem + 4);   // [4]
 
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
   const int req = z / p.Hkv, kvh = z % p.Hkv;
@@ -132,9 +133,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       mbar_init(&s_full[b], 1);
       mbar_init(&s_empty[b], 4);
       mbar_init(&p_full[b], 4);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_empty[b], 4);
     }
+    mbar_init(o_full, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -218,16 +218,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       for (int i = 0; i < n && ok; ++i) {
         if (i + 1 < n && !qk(i + 1)) { ok = false; break; }
         const int stage = i % ATC_STAGES, b2 = i & 1;
+        // P(i) written (and O rescaled, if the softmax warps moved the max)
         if (!mbar_wait(&p_full[b2], (uint32_t)(i >> 1) & 1)) { ok = false; break; }
-        if (!mbar_wait(&o_empty[b2], ((uint32_t)(i >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem + C::O_COL + b2 * HD;
+        // O accumulates in TMEM across tiles
 #pragma unroll
         for (int ks = 0; ks < ATC_KT / 16; ++ks)
-          mma_bf16(d, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
+          mma_bf16(tmem + C::O_COL, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
                    sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
-                   idesc_pv, ks > 0 ? 1u : 0u);
-        mma_commit(&o_full[b2]);
+                   idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(o_full);            // phase i completes when PV(i) has
         mma_commit(&kv_empty[stage]);
       }
       if (!ok) {
@@ -243,10 +243,14 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     const int r = threadIdx.x;
     const int qpos = (r < nq) ? p.row_pos[row0 + r / G] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    float o[HD];
-#pragma unroll
-    for (int d = 0; d < HD; ++d) o[d] = 0.f;
-    float m = -INFINITY, l = 0.f, corr_prev = 1.f;
+    // Lazy rescaling: P is formed against a reference max m that moves only
+    // when a tile's max exceeds it by more than RESCALE_LOG2 (so P <= 2^8);
+    // O then stays in TMEM and is rewritten only on those (rare) moves.
+    // PV(i) can start only after the softmax signals P(i), so when tile i is
+    // in hand at most PV(0..i-1) have completed: waiting for the o_full phase
+    // of PV(i-1) by parity is unambiguous.
+    constexpr float RESCALE_LOG2 = 8.f;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int sb = i & 1;
@@ -254,8 +258,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       float s[ATC_KT];
-#pragma unroll
-      for (int c0 = 0; c0 < ATC_KT; c0 += 16) tmem_ld16(lane_base + C::S_COL + sb * ATC_KT + c0, s + c0);
+      tmem_ld32(lane_base + C::S_COL + sb * ATC_KT, s);
+      tmem_ld32(lane_base + C::S_COL + sb * ATC_KT + 32, s + 32);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
@@ -266,38 +270,44 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         s[j] = (kp0 + j <= qpos) ? s[j] * p.scale_log2 : -INFINITY;
         mx = fmaxf(mx, s[j]);
       }
-      const float m_new = fmaxf(m, mx);
-      const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
+      bool pv_done = false;           // PV(i-1) known complete
+      const bool need = mx > m + RESCALE_LOG2;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? mx : m;
+        if (i > 0) {
+          bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(i - 1) & 1);
+          if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+          pv_done = true;
+          tc_fence_after();
+          const float corr = (m_new == m) ? 1.f : exp2f(m - m_new);   // m = -inf: O row is 0
+#pragma unroll 1
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            float v[32];
+            tmem_ld32(lane_base + C::O_COL + c0, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= corr;
+            tmem_st32(lane_base + C::O_COL + c0, v);
+          }
+          l *= corr;
+        }
+        m = m_new;
+      }
       float psum = 0.f;
       uint32_t pk[ATC_KT / 2];
 #pragma unroll
       for (int j = 0; j < ATC_KT; j += 2) {
-        const float a = (m_new == -INFINITY) ? 0.f : exp2f(s[j] - m_new);
-        const float b = (m_new == -INFINITY) ? 0.f : exp2f(s[j + 1] - m_new);
+        const float a = (s[j] == -INFINITY) ? 0.f : exp2f(s[j] - m);
+        const float b = (s[j + 1] == -INFINITY) ? 0.f : exp2f(s[j + 1] - m);
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
         psum += __low2float(h2) + __high2float(h2);    // the P the MMA will use
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      l = l * corr + psum;
-      m = m_new;
-      // fold the previous tile's output (its P used the previous max)
-      if (i > 0) {
-        const int ob = (i - 1) & 1;
-        bool w2 = !*s_abort && mbar_wait(&o_full[ob], (uint32_t)((i - 1) >> 1) & 1);
+      l += psum;
+      // the P buffer of this tile was read by PV(i-2): PV(i-1) done implies it
+      if (i > 0 && !pv_done) {
+        bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(i - 1) & 1);
         if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 16) {
-          float v[16];
-          tmem_ld16(lane_base + C::O_COL + ob * HD + c0, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * corr_prev + v[e];
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_empty[ob]);
       }
-      corr_prev = corr;
       // P row -> shared memory (K-major over keys, 128-byte swizzle)
       uint8_t* prow = sP + sb * C::P_BYTES + r * 128;
 #pragma unroll
@@ -305,21 +315,19 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_async_smem();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
+    float o[HD];
+#pragma unroll
+    for (int d = 0; d < HD; ++d) o[d] = 0.f;
     if (ok && n > 0) {
-      const int ob = (n - 1) & 1;
-      bool w2 = !*s_abort && mbar_wait(&o_full[ob], (uint32_t)((n - 1) >> 1) & 1);
+      bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(n - 1) & 1);
       if (__all_sync(0xffffffffu, w2)) {
         tc_fence_after();
 #pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 16) {
-          float v[16];
-          tmem_ld16(lane_base + C::O_COL + ob * HD + c0, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[c0 + e] = o[c0 + e] * corr_prev + v[e];
-        }
+        for (int c0 = 0; c0 < HD; c0 += 32) tmem_ld32(lane_base + C::O_COL + c0, o + c0);
         tc_fence_before();
       } else {
         ok = false;
@@ -363,6 +371,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 // per head_dim element; splits are added in split order.
 template <int HD>
 __global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x, group = blockIdx.y;
   const int z = group / p.n_qtiles, qt = group % p.n_qtiles;
   const int req = z / p.Hkv, kvh = z % p.Hkv;
@@ -371,20 +381,25 @@ __global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
   const int tok0 = qt * TQ;
   const int ntok = min(TQ, p.rows_per_req - tok0);
   if (r >= ntok * G) return;
+  // n_splits <= HD: thread s first takes split s's (m, l)
+  __shared__ float s_w[HD];
+  __shared__ float red[32];
   const int d = threadIdx.x;
   const size_t sstride = (size_t)ATC_QROWS * atc_ws_row(HD);
   const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * atc_ws_row(HD);
-  float M = -INFINITY;
-  for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, wg[s * sstride + HD]);
-  float L = 0.f, O = 0.f;
-  for (int s = 0; s < p.n_splits; ++s) {
-    const float* ws = wg + s * sstride;
-    const float ms = ws[HD];
-    if (ms == -INFINITY) continue;
-    const float f = exp2f(ms - M);
-    L += ws[HD + 1] * f;
-    O += ws[d] * f;
+  float ms = -INFINITY, ls = 0.f;
+  if (d < p.n_splits) {
+    ms = wg[d * sstride + HD];
+    ls = wg[d * sstride + HD + 1];
   }
+  const float M = block_max<HD>(ms, red);
+  const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+  s_w[d] = wt;
+  const float L = block_sum<HD>(ls * wt, red);
+  __syncthreads();
+  float O = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < p.n_splits; ++s) O += wg[s * sstride + d] * s_w[s];
   const int row0 = req * p.rows_per_req + tok0;
   const int tk = r / G, g = r % G;
   const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;

@@ -111,6 +111,17 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return t;
 }
 
+// Programmatic dependent launch.  Kernels are launched so that the next
+// kernel in the stream may start while this one runs: pdl_trigger() lets it
+// launch, and pdl_wait() blocks until the previous kernel has completed and
+// its writes are visible.  Everything before pdl_wait() may touch only data
+// no earlier kernel writes (weights, descriptors, shared memory, TMEM).
+// Without a programmatic launch both return at once.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Device-side error flag bits (read by uno_status).
 enum StatusBits : int32_t {
   ST_POS_OVERFLOW = 1,   // a position beyond the request's KV pages

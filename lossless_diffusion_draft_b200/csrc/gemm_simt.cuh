@@ -44,6 +44,8 @@ struct GemmParams {
 template <typename T, int MT, int NC>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmParams p) {
   constexpr int VEC = Vec16<T>::N;
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_base = (blockIdx.x * 8 + warp) * NC;
   const int m0 = blockIdx.y * MT;

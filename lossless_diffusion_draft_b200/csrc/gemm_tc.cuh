@@ -163,54 +163,68 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  pdl_trigger();
+  // every thread but the TMA issuer waits for the previous kernel here; the
+  // issuer first starts the weight stream (see below)
+  if (!(warp == 4 && lane == 0)) pdl_wait();
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0, issued = 0;
-      uint32_t phase = 0;
-      for (int u = u0; u < u1 && !*s_abort;) {
-        const int t = u / KBt, kb0 = u % KBt;
-        const int kb1 = min(KBt, kb0 + (u1 - u));
-        const int nt = t / p.m_tiles, mt = t % p.m_tiles;
-        const int n_row = nt * TC_BM;
+      // unit u is k-block u % KBt of tile u / KBt; issue i = u - u0 uses
+      // ring stage i % STAGES
+      auto seg_of = [&](int n_row) {
         int sg = 0;
         for (int s = 1; s < p.nseg; ++s)
           if (n_row >= p.seg[s].n0) sg = s;
-        const int n_loc = n_row - p.seg[sg].n0;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { *s_abort = 1; break; }
-          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-          uint8_t* a_dst = sA + stage * TC_A_BYTES;
-          uint8_t* b_dst = sB + stage * C::B_BYTES;
-          if (kb < p.KB) {
-            tma_load_2d(a_dst, &maps.w[sg], &full[stage], kb * TC_BK, n_loc);
-            tma_load_2d(b_dst, &maps.x, &full[stage], kb * TC_BK, mt * NT);
-            if (SPLIT)
-              tma_load_2d(b_dst + NT * 128, &maps.x, &full[stage], kb * TC_BK, p.lo_off + mt * NT);
-          } else {
-            const int j = (kb - p.KB) * TC_BK;
-            tma_load_2d(a_dst, &maps.b[sg], &full[stage], j, n_loc);
-            tma_load_2d(b_dst, &maps.u, &full[stage], p.seg[sg].u_off + j, mt * NT);
-            if (SPLIT)
-              tma_load_2d(b_dst + NT * 128, &maps.u, &full[stage], p.seg[sg].u_off + j,
-                          p.lo_off + mt * NT);
-          }
-          ++issued;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        return sg;
+      };
+      auto load_a = [&](int u, int stage) {     // weights: W, then LoRA-B
+        const int t = u / KBt, kb = u % KBt;
+        const int n_row = (t / p.m_tiles) * TC_BM;
+        const int sg = seg_of(n_row);
+        uint8_t* dst = sA + stage * TC_A_BYTES;
+        if (kb < p.KB) tma_load_2d(dst, &maps.w[sg], &full[stage], kb * TC_BK, n_row - p.seg[sg].n0);
+        else tma_load_2d(dst, &maps.b[sg], &full[stage], (kb - p.KB) * TC_BK, n_row - p.seg[sg].n0);
+      };
+      auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
+        const int t = u / KBt, kb = u % KBt;
+        const int mt = t % p.m_tiles;
+        uint8_t* dst = sB + stage * C::B_BYTES;
+        if (kb < p.KB) {
+          tma_load_2d(dst, &maps.x, &full[stage], kb * TC_BK, mt * NT);
+          if (SPLIT) tma_load_2d(dst + NT * 128, &maps.x, &full[stage], kb * TC_BK, p.lo_off + mt * NT);
+        } else {
+          const int sg = seg_of((t / p.m_tiles) * TC_BM);
+          const int x = p.seg[sg].u_off + (kb - p.KB) * TC_BK;
+          tma_load_2d(dst, &maps.u, &full[stage], x, mt * NT);
+          if (SPLIT) tma_load_2d(dst + NT * 128, &maps.u, &full[stage], x, p.lo_off + mt * NT);
         }
-        u += kb1 - kb0;
+      };
+      const int total = u1 - u0;
+      const int npre = min(total, C::STAGES);
+      // the weights depend on no earlier kernel: their first stages stream
+      // while the previous kernel finishes
+      for (int i = 0; i < npre; ++i) {
+        mbar_expect_tx(&full[i], C::STAGE_BYTES);
+        load_a(u0 + i, i);
+      }
+      pdl_wait();
+      for (int i = 0; i < npre; ++i) load_b(u0 + i, i);
+      int issued = npre;
+      for (int i = npre; i < total && !*s_abort; ++i) {
+        const int stage = i % C::STAGES;
+        if (!mbar_wait(&empty[stage], ((uint32_t)(i / C::STAGES) & 1) ^ 1)) { *s_abort = 1; break; }
+        mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+        load_a(u0 + i, stage);
+        load_b(u0 + i, stage);
+        ++issued;
       }
       if (*s_abort) {
         // wait (bounded) for the copies still in flight: the last
-        // min(issued, STAGES) issues, walking the ring backwards
-        int st = stage;
-        uint32_t ph = phase;
-        for (int i = 0; i < min(issued, C::STAGES); ++i) {
-          if (st == 0) { st = C::STAGES; ph ^= 1; }
-          --st;
-          mbar_wait(&full[st], ph);
-        }
+        // min(issued, STAGES) issues
+        for (int i = max(0, issued - C::STAGES); i < issued; ++i)
+          mbar_wait(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1);
       }
     }
   } else if (warp == 5) {
@@ -312,21 +326,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         epi_bar();
         if (*s_last) {
           __threadfence();
-          // contributors in CTA order (deterministic); four rows at a time so
-          // that independent loads are in flight together
+          // 8 rows x 8 contributors of loads are issued before any add; the
+          // adds run in CTA order (deterministic)
 #pragma unroll 1
-          for (int m = 0; m < mrows; m += 4) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-            for (int i = first; i <= last; ++i) {
-              const int slot = (sk_start(i, p.units, p.grid) >= t * KBt) ? 0 : 1;
-              const float* src = tc_slot(p.ws, i, slot, NT) + (size_t)m * TC_BM + n_local;
+          for (int m = 0; m < mrows; m += 8) {
+            float acc[8];
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (m + j < mrows) acc[j] += __ldcg(src + (size_t)j * TC_BM);
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll 1
+            for (int i0 = first; i0 <= last; i0 += 8) {
+              float v[8][8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int i = i0 + c;
+                const float* src = nullptr;
+                if (i <= last) {
+                  const int slot = (sk_start(i, p.units, p.grid) >= t * KBt) ? 0 : 1;
+                  src = tc_slot(p.ws, i, slot, NT) + (size_t)m * TC_BM + n_local;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  v[c][j] = (src && m + j < mrows) ? __ldcg(src + (size_t)j * TC_BM) : 0.f;
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] += v[c][j];
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 8; ++j)
               if (m + j < mrows && n < p.N) tc_store(p, m0 + m + j, n, acc[j]);
           }
         }

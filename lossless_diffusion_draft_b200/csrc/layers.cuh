@@ -54,6 +54,8 @@ struct RowArgs {
 // a1: build the rows of a pass and gather their embeddings.
 template <typename T>
 __global__ void build_rows_kernel(const RowArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;
   const int req = row / a.rows_per_req, j = row % a.rows_per_req;
   int slot, tok, pos;
@@ -84,9 +86,26 @@ __global__ void build_rows_kernel(const RowArgs a) {
     a.row_slot[row] = slot;
     a.row_gate[row] = gate;
   }
+  // embedding row -> fp32 residual, 16-byte loads, all issued up front
+  constexpr int VEC = Vec16<T>::N;
   const T* e = reinterpret_cast<const T*>(a.embed) + (size_t)tok * a.d;
   float* x = a.x + (size_t)row * a.d;
-  for (int i = threadIdx.x; i < a.d; i += blockDim.x) x[i] = to_f(e[i]);
+  constexpr int NV = 4;
+  float v[NV][VEC];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = (threadIdx.x + k * blockDim.x) * VEC;
+    if (i < a.d) Vec16<T>::load(e + i, v[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = (threadIdx.x + k * blockDim.x) * VEC;
+    if (i < a.d)
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) x[i + j] = v[k][j];
+  }
+  for (int i = (threadIdx.x + NV * blockDim.x) * VEC; i < a.d; i += blockDim.x * VEC)
+    for (int j = 0; j < VEC; ++j) x[i + j] = to_f(e[i + j]);
 }
 
 // Store y in the model dtype; with `lo` also the rounding residual
@@ -98,19 +117,43 @@ __device__ __forceinline__ void store_split(T* hi, T* lo, size_t i, float y) {
   if (lo) lo[i] = from_f<T>(y - to_f(h));
 }
 
-// RMSNorm: out = x / sqrt(mean(x^2) + eps) * gain, one CTA per row.
+// RMSNorm: out = x / sqrt(mean(x^2) + eps) * gain, one CTA per row.  Each
+// thread holds up to RMS_V float4 of the row in registers (all loads issued
+// before the reduction), so d <= 4 * NT * RMS_V.
+constexpr int RMS_V = 8;
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* gain, T* out, T* lo,
                                                      int d, int ld_out, float eps) {
   __shared__ float red[32];
-  const float* xr = x + (size_t)blockIdx.x * d;
+  pdl_trigger();
+  pdl_wait();
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)blockIdx.x * d);
+  const int n4 = d >> 2;
+  float4 v[RMS_V];
   float s = 0.f;
-  for (int i = threadIdx.x; i < d; i += NT) s += xr[i] * xr[i];
+#pragma unroll
+  for (int k = 0; k < RMS_V; ++k) {
+    const int i = threadIdx.x + k * NT;
+    if (i < n4) {
+      v[k] = xr[i];
+      s += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+    }
+  }
   s = block_sum<NT>(s, red);
   const float inv = 1.0f / sqrtf(s / (float)d + eps);
   const size_t o = (size_t)blockIdx.x * ld_out;
-  for (int i = threadIdx.x; i < d; i += NT)
-    store_split<T>(out + o, lo ? lo + o : nullptr, i, xr[i] * inv * to_f(gain[i]));
+  T* lrow = lo ? lo + o : nullptr;
+#pragma unroll
+  for (int k = 0; k < RMS_V; ++k) {
+    const int i = threadIdx.x + k * NT;
+    if (i < n4) {
+      const int e = 4 * i;
+      store_split<T>(out + o, lrow, e + 0, v[k].x * inv * to_f(gain[e + 0]));
+      store_split<T>(out + o, lrow, e + 1, v[k].y * inv * to_f(gain[e + 1]));
+      store_split<T>(out + o, lrow, e + 2, v[k].z * inv * to_f(gain[e + 2]));
+      store_split<T>(out + o, lrow, e + 3, v[k].w * inv * to_f(gain[e + 3]));
+    }
+  }
 }
 
 // RoPE (rotate-half) on q and k of the fused fp32 qkv rows: the rotated q goes
@@ -123,18 +166,19 @@ __global__ void rope_kv_kernel(const float* qkv, int ld_qkv, T* q_out, int ld_q,
                                const int32_t* row_pos, const int32_t* row_slot, const float* cos_t,
                                const float* sin_t, int max_pos, int H, int Hkv, int hd, KvLayout kv,
                                int layer, int32_t* status) {
-  const int row = blockIdx.x;
-  const int pos = row_pos[row], slot = row_slot[row];
+  // grid (rows, H + 2 Hkv heads of the fused q|k|v row), hd / 2 threads: one
+  // rotate-half pair (i, i + hd/2) per thread
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x, h = blockIdx.y, i = threadIdx.x;
   const int half = hd / 2;
-  const float* r = qkv + (size_t)row * ld_qkv;
-  int ok_pos = pos < max_pos;
+  const int pos = row_pos[row], slot = row_slot[row];
+  const int ok_pos = pos < max_pos;
   const int pc = ok_pos ? pos : 0;
-  // q heads then k heads: pairs (i, i + half)
-  for (int idx = threadIdx.x; idx < (H + Hkv) * half; idx += blockDim.x) {
-    const int h = idx / half, i = idx % half;
+  const float* src = qkv + (size_t)row * ld_qkv + (size_t)h * hd;
+  const float x1 = src[i], x2 = src[i + half];
+  if (h < H + Hkv) {
     const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
-    const float* base = r + (size_t)h * hd;
-    const float x1 = base[i], x2 = base[i + half];
     const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
     if (h < H) {
       T* q = q_out + (size_t)row * ld_q + (size_t)h * hd;
@@ -151,31 +195,43 @@ __global__ void rope_kv_kernel(const float* qkv, int ld_qkv, T* q_out, int ld_q,
         raise_status(status, ST_POS_OVERFLOW);
       }
     }
-  }
-  const float* v = r + (size_t)(H + Hkv) * hd;
-  for (int idx = threadIdx.x; idx < Hkv * hd; idx += blockDim.x) {
-    const int h = idx / hd, i = idx % hd;
+  } else {
     int ok;
-    const size_t off = kv.offset(layer, slot, pos, 1, h, ok);
-    if (ok && ok_pos) reinterpret_cast<T*>(kv.pool)[off + i] = from_f<T>(v[(size_t)h * hd + i]);
+    const size_t off = kv.offset(layer, slot, pos, 1, h - H - Hkv, ok);
+    if (ok && ok_pos) {
+      T* dst = reinterpret_cast<T*>(kv.pool) + off;
+      dst[i] = from_f<T>(x1);
+      dst[i + half] = from_f<T>(x2);
+    }
   }
 }
 
 // SwiGLU: out[:, f] = silu(gu[:, f]) * gu[:, F + f], from the fp32 gate|up rows.
+// Grid (rows, ceil(F / (4 * blockDim))): each thread does 4 consecutive
+// features with one float4 load of gate and one of up.
 template <typename T>
 __global__ void swiglu_kernel(const float* gu, int F, T* out, T* lo) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x;
+  const int f = 4 * (blockIdx.y * blockDim.x + threadIdx.x);
+  if (f >= F) return;
   const float* g = gu + (size_t)row * 2 * F;
-  const size_t o = (size_t)row * F;
-  for (int f = threadIdx.x; f < F; f += blockDim.x) {
-    const float a = g[f], b = g[F + f];
-    store_split<T>(out + o, lo ? lo + o : nullptr, f, a / (1.0f + expf(-a)) * b);
-  }
+  const float4 a = *reinterpret_cast<const float4*>(g + f);
+  const float4 b = *reinterpret_cast<const float4*>(g + F + f);
+  const size_t o = (size_t)row * F + f;
+  T* lrow = lo ? lo + o : nullptr;
+  store_split<T>(out + o, lrow, 0, a.x / (1.0f + expf(-a.x)) * b.x);
+  store_split<T>(out + o, lrow, 1, a.y / (1.0f + expf(-a.y)) * b.y);
+  store_split<T>(out + o, lrow, 2, a.z / (1.0f + expf(-a.z)) * b.z);
+  store_split<T>(out + o, lrow, 3, a.w / (1.0f + expf(-a.w)) * b.w);
 }
 
 // Prefill bookkeeping: cached = P - 1, pending = prompt[P - 1].
 __global__ void init_slot_kernel(const int32_t* prompt, int P, int slot, int32_t* cached,
                                  int32_t* pending) {
+  pdl_trigger();
+  pdl_wait();
   cached[slot] = P - 1;
   pending[slot] = prompt[P - 1];
 }

@@ -198,6 +198,8 @@ struct SampleArgs {
 __global__ void __launch_bounds__(SAMPLE_THREADS) sample_rows_kernel(const SampleArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last;
+  pdl_trigger();
+  pdl_wait();
   const int k = blockIdx.x;
   const int rid = blockIdx.y;
   const int req = rid / a.rows_per_req, s = rid % a.rows_per_req;
@@ -270,6 +272,8 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const Verif
   __shared__ float red[32];
   __shared__ bool s_last;
   __shared__ int s_a;
+  pdl_trigger();
+  pdl_wait();
   const int k = blockIdx.x;
   const int rid = blockIdx.y;
   const int req = rid / a.rows_red, r = rid % a.rows_red;

@@ -73,6 +73,25 @@ constexpr int TC_MIN_UNITS = 8;
 // Process-wide launch counts per kernel path (read by uno_debug_launch_counts).
 int64_t g_launches[4] = {0, 0, 0, 0};   // tc gemm, simt gemm, tc attention, simt attention
 
+// Launch with programmatic stream serialisation when `pdl`: the kernel may
+// start while the previous kernel of the stream is still running; inside,
+// pdl_wait() orders every access to data an earlier kernel wrote.
+template <typename... KArgs, typename... Args>
+void klaunch(bool pdl, cudaStream_t st, dim3 grid, dim3 block, size_t smem,
+             void (*kernel)(KArgs...), Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 struct GemmEnv {
   int sm_count = 148;
   int x_rows_alloc = 0;           // rows the activation buffers hold (>= any box)
@@ -81,6 +100,7 @@ struct GemmEnv {
   int32_t* status = nullptr;
   std::map<MapKey, CUtensorMap> maps;
   bool tc_disabled = false;
+  bool pdl = false;               // launch with programmatic stream serialisation
 
   static size_t ws_bytes(int sm) { return (size_t)sm * 2 * 256 * TC_BM * 4; }
 
@@ -173,7 +193,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
       return false;
     attr = true;
   }
-  gemm_tc_kernel<NT, SPLIT><<<tp.grid, TC_THREADS, Cfg::SMEM, st>>>(maps, tp);
+  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM, gemm_tc_kernel<NT, SPLIT>, maps, tp);
   g_launches[0]++;
   return true;
 }
@@ -191,15 +211,15 @@ bool tc_shape_ok(const GemmParams& p) {
 }
 
 template <typename T>
-void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st) {
+void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st, bool pdl) {
   const dim3 block(256);
   g_launches[1]++;
   if (p.M <= 8) {
-    gemm_simt_kernel<T, 8, 4><<<dim3((p.N + 31) / 32, (p.M + 7) / 8), block, 0, st>>>(p);
+    klaunch(pdl, st, dim3((p.N + 31) / 32, (p.M + 7) / 8), block, 0, gemm_simt_kernel<T, 8, 4>, p);
   } else if (p.M <= 16) {
-    gemm_simt_kernel<T, 16, 4><<<dim3((p.N + 31) / 32, (p.M + 15) / 16), block, 0, st>>>(p);
+    klaunch(pdl, st, dim3((p.N + 31) / 32, (p.M + 15) / 16), block, 0, gemm_simt_kernel<T, 16, 4>, p);
   } else {
-    gemm_simt_kernel<T, 32, 2><<<dim3((p.N + 15) / 16, (p.M + 31) / 32), block, 0, st>>>(p);
+    klaunch(pdl, st, dim3((p.N + 15) / 16, (p.M + 31) / 32), block, 0, gemm_simt_kernel<T, 32, 2>, p);
   }
 }
 
@@ -223,7 +243,7 @@ void gemm_run(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
     }
     if (ok) return;
   }
-  gemm_simt_dispatch<T>(p, st);
+  gemm_simt_dispatch<T>(p, st, env.pdl);
 }
 
 }  // namespace
@@ -431,7 +451,7 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
   }
   const dim3 grid(p.n_splits, p.n_qtiles, n_req * p.Hkv);
   Prof prof(c, UNO_K_ATTN, 0.0);
-  attn_simt_kernel<T, HD><<<grid, ATT_THREADS, smem, st>>>(p);
+  klaunch(c->genv.pdl, st, grid, dim3(ATT_THREADS), smem, attn_simt_kernel<T, HD>, p);
   g_launches[3]++;
   return UNO_OK;
 }
@@ -462,7 +482,7 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   int S = 1;
   if (decode && groups < c->genv.sm_count) {
     S = ceil_div(c->genv.sm_count, groups);
-    S = std::max(1, std::min(S, c->kv.pages_per_req / 2));
+    S = std::max(1, std::min(std::min(S, c->kv.pages_per_req / 2), HD));   // merge: S <= HD
     while (S > 1 && (size_t)groups * S * ATC_QROWS * atc_ws_row(HD) > c->att_ws_floats) --S;
     if (groups > c->att_groups_max) S = 1;
   }
@@ -477,13 +497,13 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   }
   {
     Prof prof(c, UNO_K_ATTN, 0.0);
-    attn_tc_kernel<HD><<<dim3(S, p.n_qtiles, n_req * s.n_kv_heads), ATC_THREADS,
-                         AtcCfg<HD>::SMEM, c->stream>>>(c->kv_map, p);
+    klaunch(c->genv.pdl, c->stream, dim3(S, p.n_qtiles, n_req * s.n_kv_heads), dim3(ATC_THREADS),
+            AtcCfg<HD>::SMEM, attn_tc_kernel<HD>, c->kv_map, p);
   }
   g_launches[2]++;
   if (S > 1) {
     Prof prof(c, UNO_K_ATTN, 0.0);
-    attn_merge_kernel<HD><<<dim3(ATC_QROWS, groups), HD, 0, c->stream>>>(p);
+    klaunch(c->genv.pdl, c->stream, dim3(ATC_QROWS, groups), dim3(HD), 0, attn_merge_kernel<HD>, p);
   }
   return UNO_OK;
 }
@@ -572,7 +592,7 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   ra.prefill_pos0 = prefill_pos0;
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
-    build_rows_kernel<T><<<M, 256, 0, st>>>(ra);
+    klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<T>, ra);
   }
   auto other = [&](auto launch) {
     Prof prof(c, UNO_K_OTHER, 0.0);
@@ -596,8 +616,8 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   auto gated = [&](Gemm& g) { g.epi(EPI_GATED, c->U, ldu, 1.f, c->row_gate); g.p.out_lo = u_lo; };
   for (int l = 0; l < s.n_layers; ++l) {
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->attn_norm[l], (T*)c->xn, xn_lo,
-                                               d, xn_ld, s.rms_eps);
+      klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, rmsnorm_kernel<T, 256>, (const float*)c->x,
+              (const T*)c->attn_norm[l], (T*)c->xn, xn_lo, d, xn_ld, s.rms_eps);
     });
     if (lora) {
       Gemm g(c->xn, xn_ld, M, d);
@@ -617,9 +637,11 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       launch_gemm<T>(c, g, st);
     }
     other([&] {
-      rope_kv_kernel<T><<<M, 128, 0, st>>>(c->qkv, qkv_ld, (T*)c->qbuf, hhd, c->row_pos,
-                                           c->row_slot, c->cos_t, c->sin_t, c->max_pos, H, Hkv, hd,
-                                           c->kv, l, c->d_status);
+      klaunch(c->genv.pdl, st, dim3(M, H + 2 * Hkv), dim3(hd / 2), 0, rope_kv_kernel<T>,
+              (const float*)c->qkv,
+              qkv_ld, (T*)c->qbuf, hhd, (const int32_t*)c->row_pos, (const int32_t*)c->row_slot,
+              (const float*)c->cos_t, (const float*)c->sin_t, c->max_pos, H, Hkv, hd, c->kv, l,
+              c->d_status);
     });
     {
       const int rc = launch_attn<T>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo);
@@ -641,8 +663,8 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       launch_gemm<T>(c, g, st);
     }
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->ffn_norm[l], (T*)c->xn, xn_lo,
-                                               d, xn_ld, s.rms_eps);
+      klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, rmsnorm_kernel<T, 256>, (const float*)c->x,
+              (const T*)c->ffn_norm[l], (T*)c->xn, xn_lo, d, xn_ld, s.rms_eps);
     });
     if (lora) {
       Gemm g(c->xn, xn_ld, M, d);
@@ -660,7 +682,11 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       g.p.lo_off = lo;
       launch_gemm<T>(c, g, st);
     }
-    other([&] { swiglu_kernel<T><<<M, 256, 0, st>>>(c->gu, F, (T*)c->xn, act_lo); });
+    other([&] {
+      klaunch(c->genv.pdl, st, dim3(M, ceil_div(F, 4 * 128)), dim3(128), 0, swiglu_kernel<T>,
+              (const float*)c->gu, F,
+              (T*)c->xn, act_lo);
+    });
     if (lora) {
       Gemm g(c->xn, F, M, F);
       g.seg(c->lA[UNO_PROJ_DOWN][l], r);
@@ -679,8 +705,8 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   }
   if (logits) {
     other([&] {
-      rmsnorm_kernel<T, 256><<<M, 256, 0, st>>>(c->x, (const T*)c->final_norm, (T*)c->xn, xn_lo,
-                                               d, xn_ld, s.rms_eps);
+      klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, rmsnorm_kernel<T, 256>, (const float*)c->x,
+              (const T*)c->final_norm, (T*)c->xn, xn_lo, d, xn_ld, s.rms_eps);
     });
     Gemm g(c->xn, xn_ld, M, d);
     g.seg(c->lm_head, s.vocab).epi(EPI_STORE_F32, logits, s.vocab, 1.0f / s.temperature);
@@ -730,6 +756,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   const int G = s.n_heads / s.n_kv_heads;
   const int vec = s.dtype == UNO_BF16 ? 8 : 4;
   if (G > ATT_MAXQ || s.vocab % 4 || s.vocab > MAX_VOCAB || s.d_model % vec || s.ffn_dim % vec ||
+      s.d_model > 4 * 256 * RMS_V ||
       lora_rank % vec ||
       (s.n_heads * s.head_dim) % vec ||
       (s.head_dim != 16 && s.head_dim != 32 && s.head_dim != 64 && s.head_dim != 128))
@@ -861,6 +888,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     c->genv.sm_count = sms;
+    c->genv.pdl = true;
     c->genv.x_rows_alloc = 2 * M;   // activation buffers: hi rows then lo rows
     if (dalloc(&c->genv.ws, GemmEnv::ws_bytes(sms)) != cudaSuccess) return oom("gemm ws");
     if (dalloc(&c->genv.counters, (size_t)TC_COUNTERS * 4) != cudaSuccess) return oom("gemm ws");
@@ -1034,7 +1062,8 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.row_counter = c->row_counter;
     a.status = c->d_status;
     Prof prof(c, UNO_K_SAMPLE, (double)n_req * B * V * 4);
-    sample_rows_kernel<<<dim3(c->nch, n_req * B), SAMPLE_THREADS, 0, c->stream>>>(a);
+    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
+            sample_rows_kernel, a);
   }
   rc = forward_any(c, PASS_VERIFY, n_req, B, req_ids_dev, nullptr, 0, 0, c->logits_v);
   if (rc) return rc;
@@ -1068,7 +1097,8 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.n_p = B;
     a.status = c->d_status;
     Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
-    spec_verify_kernel<<<dim3(c->nch, n_req * B), SAMPLE_THREADS, 0, c->stream>>>(a);
+    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
+            spec_verify_kernel, a);
   }
   CK(cudaGetLastError());
   return UNO_OK;
@@ -1095,7 +1125,8 @@ int ar_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out
   a.status = c->d_status;
   {
     Prof prof(c, UNO_K_SAMPLE, (double)n_req * a.V * 4);
-    sample_rows_kernel<<<dim3(c->nch, n_req), SAMPLE_THREADS, 0, c->stream>>>(a);
+    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req), dim3(SAMPLE_THREADS), 0,
+            sample_rows_kernel, a);
   }
   CK(cudaGetLastError());
   return UNO_OK;
@@ -1130,6 +1161,17 @@ int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_
 int uno_set_graphs(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->graphs_enabled = enable != 0;
+  return UNO_OK;
+}
+
+int uno_set_pdl(uno_ctx* c, int enable) {
+  if (!c) return UNO_ERR_ARG;
+  c->genv.pdl = enable != 0;
+  for (auto& g : c->graphs) {   // graphs captured with the other launch mode
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.seen = 0;
+  }
   return UNO_OK;
 }
 

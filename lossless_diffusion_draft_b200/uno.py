@@ -82,6 +82,7 @@ def load_library(path=LIB_PATH):
                                         sz, vp]),
         "uno_debug_launch_counts": (i32, [vp]),
         "uno_set_graphs": (i32, [vp, i32]),
+        "uno_set_pdl": (i32, [vp, i32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
@@ -214,6 +215,10 @@ def uno_ar_step(ctx, req_ids_dev, out_tokens_dev):
 
 def uno_set_graphs(ctx, enable):
     _check(load_library().uno_set_graphs(ctx.handle, int(bool(enable))), ctx.handle)
+
+
+def uno_set_pdl(ctx, enable):
+    _check(load_library().uno_set_pdl(ctx.handle, int(bool(enable))), ctx.handle)
 
 
 def uno_release(ctx, req_id):
