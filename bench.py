@@ -213,6 +213,7 @@ def run_uno(args, rank, world, device):
                        cfg["seed"], stream)
     if args.no_pdl:
         uno.uno_set_pdl(ctx, False)
+    fused = uno.uno_set_fused(ctx, not args.no_fused) and not args.no_fused
     if args.no_graphs:
         uno.uno_set_graphs(ctx, False)
 
@@ -242,11 +243,15 @@ def run_uno(args, rank, world, device):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
+        # a profiler started with --profile-from-start off sees the timed
+        # steps only
+        torch.cuda.profiler.start()
         ev0.record(stream)
         for k in range(K):
             uno.uno_spec_step(ctx, req, out, n_new_all[k])
         ev1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.profiler.stop()
     prof = uno.uno_profile_end(ctx)
     barrier(world)
     ms = ev0.elapsed_time(ev1)
@@ -306,7 +311,7 @@ def run_uno(args, rank, world, device):
     tokens_all = reduce_sum(tokens, world, device)
     e2e_tokens_all = reduce_sum(e2e_tokens, world, device)
 
-    info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, tokens=tokens_all, K=K, W=W,
+    info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, fused=fused, tokens=tokens_all, K=K, W=W,
                 e2e_ms=e2e_ms_max, e2e_tokens=e2e_tokens_all, clocks=clk.summary(),
                 launches=launches, kprof=kprof, prefill_s=prefill_s, detail=detail[:24],
                 ctx_window=[ctx_before, ctx_after], weight_bytes=weight_bytes,
@@ -435,6 +440,8 @@ def main():
     ap.add_argument("--shape", default="17,4096,4096,128",
                     help="gemm microbenchmark shape M,N,K,r")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="unfused layer pipeline (separate LoRA-A GEMMs, norm, RoPE, SwiGLU)")
     ap.add_argument("--no-graphs", action="store_true", help="no CUDA-graph capture of steps")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for profiler captures; the "
@@ -514,6 +521,7 @@ def main():
         "data": "synthetic (random-init weights, uniform-random prompt tokens)",
         "config": {"workload": args.workload, "n_layers": info["cfg"]["n_layers"],
                    "batch": info["batch"], "B": info["B"], "pdl": not args.no_pdl,
+                   "fused": info["fused"],
                    "graphs": not args.no_graphs,
                    "prompt_len": cfg["prompt_len"], "gen_tokens": cfg["gen_tokens"],
                    "context_window": info["ctx_window"], "parallelism": f"replicas x{world}",

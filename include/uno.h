@@ -155,6 +155,17 @@ int uno_set_graphs(uno_ctx *ctx, int enable);
  * kernels in plain stream order.  Changing it drops captured graphs. */
 int uno_set_pdl(uno_ctx *ctx, int enable);
 
+/* Fused layer pipeline (implementation choice, on by default where it
+ * applies: bf16 models with head_dim 64 or 128, d_model, ffn_dim and the
+ * q / kv widths multiples of 128, d_model <= 8192, LoRA rank 0 or 128).  Each projection
+ * GEMM then leaves fp32 parts that one epilogue kernel reduces and carries
+ * through LoRA-B, the RMSNorm scale, RoPE and the KV write, SwiGLU or the
+ * residual add; the LoRA A matrices stream with the base weights.  enable =
+ * 0 runs the unfused kernels (separate rank-r GEMMs, norm, RoPE, SwiGLU).
+ * Changing it drops captured graphs.  Returns UNO_ERR_UNSUPPORTED (after
+ * recording the setting) when the model does not take the fused pipeline. */
+int uno_set_fused(uno_ctx *ctx, int enable);
+
 /* Free a request's slot and pages (stream-ordered after earlier work). */
 int uno_release(uno_ctx *ctx, int req_id);
 
@@ -270,8 +281,10 @@ int uno_profile_records(uno_ctx *ctx, uno_prof_record *out, int max);
  *                  given, so no further token is drawn).
  *   workspace_dev: scratch of at least uno_spec_verify_workspace_bytes()
  *                  bytes, 256-byte aligned, zero-filled before its first use
- *                  (the kernel leaves it zeroed again); calls sharing a
- *                  workspace must not overlap on the GPU.
+ *                  (the kernels leave its counters zeroed again); calls
+ *                  sharing a workspace must not overlap on the GPU.
+ * Enqueues two kernels on `stream`: the vocabulary reductions and accept
+ * tests, then the residual redraw of each request with a rejection.
  * Returns UNO_ERR_ARG on bad sizes; never synchronises.
  */
 size_t uno_spec_verify_workspace_bytes(int n_req, int n_tests, int vocab);
@@ -301,7 +314,7 @@ int uno_spec_verify(const float *p_dev, const float *q_dev, const int32_t *draft
  *   call before any stream capture.
  *   All calls share the one array, which keeps the previous call's contents;
  *   each call clears the part that must start at zero (its completion
- *   counters) on the given stream before the kernel.  Calls that overlap on
+ *   counters) on the given stream before the kernels.  Calls that overlap on
  *   the GPU (different streams, no ordering between them) race on the array
  *   and give wrong results: serialise them.
  */

@@ -30,10 +30,12 @@ struct GemmSeg {
   int u_off;          // column of U feeding this segment's LoRA-B
 };
 
+constexpr int GEMM_MAX_SEG = 6;
+
 struct GemmParams {
   const void* X; int ldx;    // [M, K] model dtype
   int M, K, N;
-  GemmSeg seg[3]; int nseg;
+  GemmSeg seg[GEMM_MAX_SEG]; int nseg;
   const void* U; int ldu; int r;   // LoRA-B extension (U null: none)
   int epi; void* out; int ldo; float alpha;
   const float* row_gate;
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmParams p) {
     valid[c] = n < p.N;
     int s = 0;
 #pragma unroll
-    for (int t = 1; t < 3; ++t)
+    for (int t = 1; t < GEMM_MAX_SEG; ++t)
       if (t < p.nseg && n >= p.seg[t].n0) s = t;
     const GemmSeg& g = p.seg[s];
     const int nn = valid[c] ? n - g.n0 : 0;

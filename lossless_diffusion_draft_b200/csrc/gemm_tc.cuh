@@ -14,9 +14,16 @@
 //    base weights and the adapter share one pass over the output tile;
 //  * stream-K: the (tile, k-block) units are split evenly over one persistent
 //    CTA per SM, so every SM streams the same number of weight bytes whatever
-//    the tile count; a tile cut between CTAs is finished by whichever
-//    contributor arrives last (atomic counter, no waiting), which adds the
-//    fp32 partials in a fixed order (deterministic) and runs the epilogue;
+//    the tile count.  Two ways to finish a tile:
+//      - in-kernel: a tile cut between CTAs is finished by whichever
+//        contributor arrives last (atomic counter, no waiting), which adds
+//        the fp32 partials in a fixed order (deterministic) and runs the
+//        epilogue;
+//      - DUMP: every part goes to its own fp32 slot, tile + cta (unique: both
+//        grow together along the unit order), and the CTA moves on; a
+//        following epilogue kernel adds a tile's parts in CTA order and fuses
+//        whatever comes next.  The reducing CTA's chain of dependent L2
+//        round trips then leaves the GEMM's critical path;
 //  * warp roles: warp 4 issues TMA loads into a STAGES-deep ring, warp 5
 //    issues tcgen05.mma into a double-buffered TMEM accumulator, warps 0-3
 //    drain TMEM (tcgen05.ld) and write the epilogue while the next part's
@@ -40,11 +47,12 @@ constexpr int TC_BK = 64;          // k elements per block (128 bytes of bf16)
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
 constexpr int ST_GEMM_TIMEOUT = 8;
 
+constexpr int TC_MAX_SEG = GEMM_MAX_SEG;
 struct TcMaps {
-  CUtensorMap x;       // activations [rows, K], box {64, NT}
-  CUtensorMap u;       // LoRA intermediate [rows, 3r], box {64, NT}
-  CUtensorMap w[3];    // weights of each segment [n, K], box {64, 128}
-  CUtensorMap b[3];    // LoRA-B of each segment [n, r], box {64, 128}
+  CUtensorMap x;               // activations [rows, K], box {64, NT}
+  CUtensorMap u;               // LoRA intermediate [rows, 3r], box {64, NT}
+  CUtensorMap w[TC_MAX_SEG];   // weights of each segment [n, K], box {64, 128}
+  CUtensorMap b[3];            // LoRA-B of each segment [n, r], box {64, 128}
 };
 
 struct TcSeg { int n0, n, u_off; };
@@ -52,11 +60,11 @@ struct TcSeg { int n0, n, u_off; };
 struct TcParams {
   int M, N, KB, RB;          // rows, columns, k-blocks of K, k-blocks of r (0: no LoRA)
   int n_tiles, m_tiles;
-  int nseg; TcSeg seg[3];
+  int nseg; TcSeg seg[TC_MAX_SEG];
   int units, grid;           // stream-K: units = tiles * (KB + RB), split over grid CTAs
   int max_parts;             // partial slots per tile
   int epi; void* out; int ldo; float alpha; const float* row_gate;
-  float* ws; unsigned* counters;
+  float* ws; unsigned* counters;   // DUMP: ws holds the part slots [tiles + grid][NT][128]
   int32_t* status;
   int lo_off;                // split mode: row offset of the lo rows of X and U
   void* out_lo;              // EPI_GATED in split mode: lo part of the output (out + lo_off rows)
@@ -111,7 +119,7 @@ __device__ __forceinline__ void tc_store(const TcParams& p, int m, int n, float 
   }
 }
 
-template <int NT, bool SPLIT>
+template <int NT, bool SPLIT, bool DUMP>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
   using C = TcCfg<NT, SPLIT>;
@@ -286,9 +294,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int n = nt * TC_BM + n_local;
       const int m0 = mt * NT;
       const int mrows = min(NT, p.M - m0);
-      const bool whole = (kb0 == 0 && kb1 == KBt);
+      const bool whole = !DUMP && (kb0 == 0 && kb1 == KBt);
       const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * C::NMMA);
-      float* wsl = tc_slot(p.ws, blockIdx.x, part == 0 ? 0 : 1, NT);
+      float* wsl = DUMP ? p.ws + (size_t)(t + blockIdx.x) * NT * TC_BM
+                        : tc_slot(p.ws, blockIdx.x, part == 0 ? 0 : 1, NT);
 #pragma unroll 1
       for (int c0 = 0; c0 < NT; c0 += 16) {
         float v[16];
@@ -312,7 +321,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      if (!whole) {
+      if (!DUMP && !whole) {
         __threadfence();
         epi_bar();
         const int first = sk_owner(t * KBt, p.units, p.grid);

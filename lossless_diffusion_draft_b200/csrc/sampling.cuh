@@ -12,8 +12,10 @@
 // Work split.  A vocabulary row is cut into chunks of `ch` logits; one CTA
 // reduces one (row, chunk) to its (max, sum exp(l - max)) pair.  The last CTA
 // to finish a row (atomic counter, no waiting) combines the row's pairs in
-// chunk order; the last row of a request runs the request's decision.  No CTA
-// ever waits on another, so nothing can hang.
+// chunk order; the last row of a request runs the request's decision.  A
+// rejected request's residual is summed by a second grid, one CTA per
+// (request, chunk), whose last CTA draws the token.  No CTA ever waits on
+// another, so nothing can hang.
 //
 // Inverse-CDF sampling on the device: w_v = expf(l_v - M) with M the row max;
 // Z = sum over chunks (in chunk order) of s_k * expf(m_k - M); the token is in
@@ -85,10 +87,11 @@ struct SoftmaxW {
 };
 struct ResidW {
   const float* p; const float* q; float lse_p, lse_q;
-  __device__ __forceinline__ float operator()(int v) const {
-    const float d = expf(p[v] - lse_p) - expf(q[v] - lse_q);
+  __device__ __forceinline__ float pair(float pv, float qv) const {
+    const float d = expf(pv - lse_p) - expf(qv - lse_q);
     return d > 0.f ? d : 0.f;
   }
+  __device__ __forceinline__ float operator()(int v) const { return pair(p[v], q[v]); }
 };
 
 // First v in [c0, c1) whose running prefix base + sum_{c0..v} w exceeds
@@ -263,10 +266,58 @@ struct VerifyArgs {
   float* lse;                  // [n_req * rows_red]
   unsigned* row_counter;       // [n_req * rows_red]
   unsigned* req_counter;       // [n_req]
+  int32_t* at_ws;              // [n_req] first rejected test, -1: finished by the first stage
+  float* resid_part;           // [n_req, nch] residual chunk sums
+  unsigned* resid_counter;     // [n_req]
   int rows_red;                // rows reduced per request
   int n_p;                     // of which p rows (tests + bonus)
   int32_t* status;
 };
+
+// Slot, position of test 0 and Philox stream of a request.
+__device__ __forceinline__ void verify_request_ctx(const VerifyArgs& a, int req, int* slot,
+                                                   int* pos0, uint32_t* stream) {
+  if (a.req_slot) {
+    *slot = a.req_slot[req];
+    *pos0 = a.cached[*slot] + 2;     // test 0 is x_2 at position c + 2
+    *stream = a.slot_stream[*slot];
+  } else {
+    *slot = -1;
+    *pos0 = a.pos0[req];
+    *stream = a.streams[req];
+  }
+}
+
+// log-normaliser of the draft row of test j.
+__device__ __forceinline__ float verify_lse_q(const VerifyArgs& a, int req, int j) {
+  return a.lse_q_in ? a.lse_q_in[(size_t)req * a.lse_q_stride + a.lse_q_off + j]
+                    : __ldcg(&a.lse[(size_t)req * a.rows_red + a.n_p + j]);
+}
+
+// Outputs and commit of a request with `at` accepted tests and final token y
+// (whole CTA).
+__device__ void verify_finish(const VerifyArgs& a, int req, int slot, int pos0, int at, int y) {
+  const bool decode = a.req_slot != nullptr;
+  const int lead = decode ? 1 : 0;    // decode mode emits x_1 first
+  int32_t* out = a.out_tok + (size_t)req * a.out_stride;
+  for (int j = threadIdx.x; j < at; j += SAMPLE_THREADS)
+    out[lead + j] = a.drafts[(size_t)req * a.drafts_stride + a.drafts_off + j];
+  if (threadIdx.x == 0) {
+    if (decode) {
+      // emitted: x_1, the accepted x_2..x_{1+at}, then y; the cache grows by
+      // n tokens (positions c..c+n-1 hold keys/values) and y becomes pending
+      out[0] = a.first_tok[(size_t)req * a.drafts_stride];
+      const int n = lead + at + 1;
+      out[n - 1] = y;
+      a.n_out[req] = n;
+      a.cached[slot] = pos0 - 2 + n;
+      a.pending[slot] = y;
+    } else {
+      out[at] = y;          // -1 when every test passed and no bonus row exists
+      a.n_out[req] = at;
+    }
+  }
+}
 
 __global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const VerifyArgs a) {
   __shared__ float red[32];
@@ -308,16 +359,9 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const Verif
 
   // ---- request decision (one CTA per request) ----
   const size_t rbase = (size_t)req * a.rows_red;
-  int slot = -1, pos0;
+  int slot, pos0;
   uint32_t stream;
-  if (a.req_slot) {
-    slot = a.req_slot[req];
-    pos0 = a.cached[slot] + 2;     // test 0 is x_2 at position c + 2
-    stream = a.slot_stream[slot];
-  } else {
-    pos0 = a.pos0[req];
-    stream = a.streams[req];
-  }
+  verify_request_ctx(a, req, &slot, &pos0, &stream);
   if (threadIdx.x == 0) s_a = a.n_tests;
   __syncthreads();
   for (int j = threadIdx.x; j < a.n_tests; j += SAMPLE_THREADS) {
@@ -326,70 +370,20 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const Verif
     const float* prow = a.p + ((size_t)req * a.p_req_rows + a.p_row0 + j) * a.V;
     const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + j) * a.V;
     const float lse_p = __ldcg(&a.lse[rbase + j]);
-    const float lse_q = a.lse_q_in ? a.lse_q_in[(size_t)req * a.lse_q_stride + a.lse_q_off + j]
-                                   : __ldcg(&a.lse[rbase + a.n_p + j]);
+    const float lse_q = verify_lse_q(a, req, j);
     const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + j), KIND_ACCEPT);
     const bool acc = logf(u) < (prow[t] - lse_p) - (qrow[t] - lse_q);
     if (!acc) atomicMin(&s_a, j);
   }
   __syncthreads();
   const int at = s_a;   // accepted prefix length among the tests
-  int y = -1;
   if (at < a.n_tests) {
-    const float* prow = a.p + ((size_t)req * a.p_req_rows + a.p_row0 + at) * a.V;
-    const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + at) * a.V;
-    const float lse_p = __ldcg(&a.lse[rbase + at]);
-    const float lse_q = a.lse_q_in ? a.lse_q_in[(size_t)req * a.lse_q_stride + a.lse_q_off + at]
-                                   : __ldcg(&a.lse[rbase + a.n_p + at]);
-    const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + at), KIND_RESID);
-    ResidW w{prow, qrow, lse_p, lse_q};
-    // chunk sums of the residual, chunk order, coalesced
-    __shared__ float s_cs[64];
-    __shared__ float s_Z;
-    float Z = 0.f;
-    for (int kk = 0; kk < a.nch; ++kk) {
-      const int b0 = kk * a.ch, b1 = min(a.V, b0 + a.ch);
-      float sacc = 0.f;
-      for (int v = b0 + threadIdx.x; v < b1; v += SAMPLE_THREADS) sacc += w(v);
-      const float sk = block_sum<SAMPLE_THREADS>(sacc, red);
-      if (threadIdx.x == 0 && kk < 64) s_cs[kk] = sk;
-      Z += sk;
-    }
-    if (threadIdx.x == 0) s_Z = Z;
-    __syncthreads();
-    Z = s_Z;
-    if (Z > 0.f) {
-      const float target = u * Z;
-      __shared__ int s_k;
-      __shared__ float s_base;
-      if (threadIdx.x == 0) {
-        float run = 0.f;
-        int kk = -1, lastk = -1;
-        for (int c = 0; c < a.nch; ++c) {
-          const float sk = s_cs[c];
-          if (sk > 0.f) lastk = c;
-          if (kk < 0 && run + sk > target) { kk = c; s_base = run; }
-          run += sk;
-        }
-        if (kk < 0) { kk = lastk; s_base = 0.f; }
-        s_k = kk;
-      }
-      __syncthreads();
-      const int kk = s_k;
-      const float base = s_base;
-      __syncthreads();
-      int lastpos;
-      const int b0 = kk * a.ch, b1 = min(a.V, b0 + a.ch);
-      y = chunk_crossing(w, b0, b1, base, target, &lastpos, red);
-      if (y < 0) y = lastpos >= 0 ? lastpos : b0;
-    } else {
-      // no residual mass after rounding: draw from p
-      __shared__ RowStat s_rs;
-      if (threadIdx.x == 0) s_rs = combine_row(a.partial + (rbase + at) * a.nch, a.nch);
-      __syncthreads();
-      y = sample_from_partials(prow, a.partial + (rbase + at) * a.nch, a.nch, a.ch, a.V, s_rs, u, red);
-    }
-  } else if (a.bonus_row >= 0) {
+    // a rejection: spec_resid_kernel draws from the residual and finishes
+    if (threadIdx.x == 0) a.at_ws[req] = at;
+    return;
+  }
+  int y = -1;
+  if (a.bonus_row >= 0) {
     const float* prow = a.p + ((size_t)req * a.p_req_rows + a.bonus_row) * a.V;
     const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + a.n_tests), KIND_RESID);
     __shared__ RowStat s_rs2;
@@ -398,28 +392,111 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const Verif
     y = sample_from_partials(prow, a.partial + (rbase + a.n_tests) * a.nch, a.nch, a.ch, a.V,
                              s_rs2, u, red);
   }
+  if (threadIdx.x == 0) a.at_ws[req] = -1;
+  verify_finish(a, req, slot, pos0, at, y);
+}
 
-  // ---- outputs and commit ----
-  const bool decode = a.req_slot != nullptr;
-  const int lead = decode ? 1 : 0;    // decode mode emits x_1 first
-  int32_t* out = a.out_tok + (size_t)req * a.out_stride;
-  for (int j = threadIdx.x; j < at; j += SAMPLE_THREADS)
-    out[lead + j] = a.drafts[(size_t)req * a.drafts_stride + a.drafts_off + j];
-  if (threadIdx.x == 0) {
-    if (decode) {
-      // emitted: x_1, the accepted x_2..x_{1+at}, then y; the cache grows by
-      // n tokens (positions c..c+n-1 hold keys/values) and y becomes pending
-      out[0] = a.first_tok[(size_t)req * a.drafts_stride];
-      const int n = lead + at + 1;
-      out[n - 1] = y;
-      a.n_out[req] = n;
-      a.cached[slot] = pos0 - 2 + n;
-      a.pending[slot] = y;
-    } else {
-      out[at] = y;          // -1 when every test passed and no bonus row exists
-      a.n_out[req] = at;
+// ---------------------------------------------------------------------------
+// spec_verify, second stage: the residual redraw at the first rejected test.
+// Grid (nch, n_req); launched after spec_verify_kernel.  CTA k adds up the
+// residual weights max(0, p_v - q_v) (normalised p and q of the rejected
+// test's rows) over chunk k; the last CTA of a request picks the chunk whose
+// running sum (chunk order) crosses u * Z, finds the token inside it, and
+// writes the outputs and the commit.  Requests without a rejection (at_ws =
+// -1) were finished by the first stage.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const VerifyArgs a) {
+  __shared__ float red[32];
+  __shared__ bool s_last;
+  pdl_trigger();
+  pdl_wait();
+  const int k = blockIdx.x, req = blockIdx.y;
+  const int at = a.at_ws[req];
+  if (at < 0) return;
+  const size_t rbase = (size_t)req * a.rows_red;
+  const float* prow = a.p + ((size_t)req * a.p_req_rows + a.p_row0 + at) * a.V;
+  const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + at) * a.V;
+  const float lse_p = __ldcg(&a.lse[rbase + at]);
+  const float lse_q = verify_lse_q(a, req, at);
+  const ResidW w{prow, qrow, lse_p, lse_q};
+  {
+    // chunk sum: 16-byte loads, all of a thread's loads issued first
+    const int b0 = k * a.ch, b1 = min(a.V, b0 + a.ch);
+    const int n4 = (b1 - b0) >> 2;
+    const float4* p4 = reinterpret_cast<const float4*>(prow + b0);
+    const float4* q4 = reinterpret_cast<const float4*>(qrow + b0);
+    constexpr int MAXIT = 8;
+    float sacc = 0.f;
+    for (int i0 = 0; i0 < n4; i0 += MAXIT * SAMPLE_THREADS) {
+      float4 x[MAXIT], z[MAXIT];
+#pragma unroll
+      for (int i = 0; i < MAXIT; ++i) {
+        const int j = i0 + threadIdx.x + i * SAMPLE_THREADS;
+        if (j < n4) { x[i] = p4[j]; z[i] = q4[j]; }
+      }
+#pragma unroll
+      for (int i = 0; i < MAXIT; ++i) {
+        const int j = i0 + threadIdx.x + i * SAMPLE_THREADS;
+        if (j < n4) sacc += w.pair(x[i].x, z[i].x) + w.pair(x[i].y, z[i].y) +
+                            w.pair(x[i].z, z[i].z) + w.pair(x[i].w, z[i].w);
+      }
+    }
+    for (int v = b0 + (n4 << 2) + threadIdx.x; v < b1; v += SAMPLE_THREADS) sacc += w(v);
+    const float sk = block_sum<SAMPLE_THREADS>(sacc, red);
+    if (threadIdx.x == 0) {
+      a.resid_part[(size_t)req * a.nch + k] = sk;
+      __threadfence();
+      const unsigned done = atomicAdd(&a.resid_counter[req], 1u);
+      const bool last = (done == (unsigned)a.nch - 1);
+      if (last) a.resid_counter[req] = 0u;
+      s_last = last;
     }
   }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  int slot, pos0;
+  uint32_t stream;
+  verify_request_ctx(a, req, &slot, &pos0, &stream);
+  const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + at), KIND_RESID);
+  const float* cs = a.resid_part + (size_t)req * a.nch;
+  __shared__ float s_Z, s_base;
+  __shared__ int s_k;
+  if (threadIdx.x == 0) {
+    float Z = 0.f;
+    for (int c = 0; c < a.nch; ++c) Z += __ldcg(&cs[c]);
+    const float target = u * Z;
+    float run = 0.f;
+    int kk = -1, lastk = -1;
+    float base = 0.f;
+    for (int c = 0; c < a.nch; ++c) {
+      const float sk = __ldcg(&cs[c]);
+      if (sk > 0.f) lastk = c;
+      if (kk < 0 && run + sk > target) { kk = c; base = run; }
+      run += sk;
+    }
+    if (kk < 0) { kk = lastk; base = 0.f; }
+    s_Z = Z;
+    s_k = kk;
+    s_base = base;
+  }
+  __syncthreads();
+  const float Z = s_Z;
+  int y;
+  if (Z > 0.f && s_k >= 0) {
+    int lastpos;
+    const int b0 = s_k * a.ch, b1 = min(a.V, b0 + a.ch);
+    y = chunk_crossing(w, b0, b1, s_base, u * Z, &lastpos, red);
+    if (y < 0) y = lastpos >= 0 ? lastpos : b0;
+  } else {
+    // no residual mass after rounding: draw from p
+    __shared__ RowStat s_rs;
+    if (threadIdx.x == 0) s_rs = combine_row(a.partial + (rbase + at) * a.nch, a.nch);
+    __syncthreads();
+    y = sample_from_partials(prow, a.partial + (rbase + at) * a.nch, a.nch, a.ch, a.V, s_rs, u, red);
+  }
+  verify_finish(a, req, slot, pos0, at, y);
 }
 
 }  // namespace uno

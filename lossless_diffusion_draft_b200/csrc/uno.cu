@@ -27,6 +27,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "layers.cuh"
@@ -96,6 +97,8 @@ struct GemmEnv {
   int sm_count = 148;
   int x_rows_alloc = 0;           // rows the activation buffers hold (>= any box)
   float* ws = nullptr;            // [sm_count][2][256][128] fp32 partial tiles
+  float* part = nullptr;          // DUMP-mode part slots
+  size_t part_bytes = 0;
   unsigned* counters = nullptr;   // [TC_COUNTERS], zero, left zero
   int32_t* status = nullptr;
   std::map<MapKey, CUtensorMap> maps;
@@ -126,8 +129,20 @@ struct GemmEnv {
   }
 };
 
-template <int NT, bool SPLIT>
-bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
+// Stream-K shape of a DUMP-mode launch (what its epilogue kernel needs).
+struct DumpShape {
+  int NT = 0, units = 0, grid = 0, KBt = 0, m_tiles = 0, n_tiles = 0;
+};
+
+// Part slots a DUMP-mode GEMM of M rows and N columns writes, in bytes.
+size_t dump_bytes(int M, int N, int sm_count) {
+  const int NT = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  const size_t slots = (size_t)((N + TC_BM - 1) / TC_BM) * ((M + NT - 1) / NT) + sm_count;
+  return slots * NT * TC_BM * 4;
+}
+
+template <int NT, bool SPLIT, bool DUMP>
+bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape = nullptr) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
   // A box may not be larger than the tensor: the activation tensors are
@@ -138,6 +153,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
   if ((uint64_t)env.x_rows_alloc < xrows) return false;
   for (int s = 0; s < p.nseg; ++s)
     if (p.seg[s].n < TC_BM) return false;
+  if (p.U && p.nseg > 3) return false;   // LoRA-B maps: three segments
   const CUtensorMap* mx = env.map(p.X, xrows, p.K, p.ldx, NT);
   if (!mx) return false;
   maps.x = *mx;
@@ -158,7 +174,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
     const CUtensorMap* mw = env.map(g.W, g.n, p.K, p.K, TC_BM);
     if (!mw) return false;
     maps.w[s] = *mw;
-    maps.b[s] = *mw;
+    if (s < 3) maps.b[s] = *mw;
     if (p.U) {
       if (!g.lB) return false;
       const CUtensorMap* mb = env.map(g.lB, g.n, p.r, p.r, TC_BM);
@@ -182,18 +198,24 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
   tp.row_gate = p.row_gate;
   tp.ws = env.ws;
   tp.counters = env.counters;
+  if (DUMP) {
+    if (!env.part || dump_bytes(p.M, p.N, env.sm_count) > env.part_bytes) return false;
+    tp.ws = env.part;
+    if (shape) *shape = DumpShape{NT, tp.units, tp.grid, tp.KB + tp.RB, tp.m_tiles, tp.n_tiles};
+  }
   tp.status = env.status;
   tp.lo_off = SPLIT ? p.lo_off : 0;
   tp.out_lo = p.out_lo;
   using Cfg = TcCfg<NT, SPLIT>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT, DUMP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
       return false;
     attr = true;
   }
-  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM, gemm_tc_kernel<NT, SPLIT>, maps, tp);
+  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM, gemm_tc_kernel<NT, SPLIT, DUMP>,
+          maps, tp);
   g_launches[0]++;
   return true;
 }
@@ -223,27 +245,37 @@ void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st, bool pdl) {
   }
 }
 
+// Tile width NT by row count; hi/lo split activations up to 128 rows.
+template <bool DUMP>
+bool launch_tc_any(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape) {
+  if (p.lo_off > 0 && p.M <= 128) {
+    if (p.M <= 16) return launch_tc<16, true, DUMP>(env, p, st, shape);
+    if (p.M <= 32) return launch_tc<32, true, DUMP>(env, p, st, shape);
+    if (p.M <= 64) return launch_tc<64, true, DUMP>(env, p, st, shape);
+    return launch_tc<128, true, DUMP>(env, p, st, shape);
+  }
+  if (p.M <= 16) return launch_tc<16, false, DUMP>(env, p, st, shape);
+  if (p.M <= 32) return launch_tc<32, false, DUMP>(env, p, st, shape);
+  if (p.M <= 64) return launch_tc<64, false, DUMP>(env, p, st, shape);
+  if (p.M <= 128) return launch_tc<128, false, DUMP>(env, p, st, shape);
+  return launch_tc<256, false, DUMP>(env, p, st, shape);
+}
+
 // Runs one gated-LoRA GEMM: tcgen05 for bf16 shapes it takes, SIMT otherwise.
 template <typename T>
 void gemm_run(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
   if (p.M <= 0 || p.N <= 0) return;
-  if (sizeof(T) == 2 && !env.tc_disabled && tc_shape_ok(p)) {
-    bool ok;
-    if (p.lo_off > 0 && p.M <= 128) {
-      if (p.M <= 16) ok = launch_tc<16, true>(env, p, st);
-      else if (p.M <= 32) ok = launch_tc<32, true>(env, p, st);
-      else if (p.M <= 64) ok = launch_tc<64, true>(env, p, st);
-      else ok = launch_tc<128, true>(env, p, st);
-    } else {
-      if (p.M <= 16) ok = launch_tc<16, false>(env, p, st);
-      else if (p.M <= 32) ok = launch_tc<32, false>(env, p, st);
-      else if (p.M <= 64) ok = launch_tc<64, false>(env, p, st);
-      else if (p.M <= 128) ok = launch_tc<128, false>(env, p, st);
-      else ok = launch_tc<256, false>(env, p, st);
-    }
-    if (ok) return;
-  }
+  if (sizeof(T) == 2 && !env.tc_disabled && tc_shape_ok(p) &&
+      launch_tc_any<false>(env, p, st, nullptr))
+    return;
   gemm_simt_dispatch<T>(p, st, env.pdl);
+}
+
+// DUMP-mode launch of a bf16 GEMM (false: the tensor-core kernel cannot take
+// it, nothing was launched).
+bool gemm_run_dump(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape) {
+  if (p.M <= 0 || p.N <= 0 || env.tc_disabled || !tc_shape_ok(p)) return false;
+  return launch_tc_any<true>(env, p, st, shape);
 }
 
 }  // namespace
@@ -280,6 +312,9 @@ struct uno_ctx {
   void* attn = nullptr;        // [M, H hd]
   float* gu = nullptr;         // [M, 2F] fp32 gate|up output
   void* U = nullptr;           // [M, 3r] LoRA intermediate
+  float* ss = nullptr;         // [M, d / 128] sums of squares of x per 128-column tile
+  bool fused = false;          // the fused bf16 layer pipeline applies to this model
+  bool fused_enabled = true;
   int32_t *row_pos = nullptr, *row_slot = nullptr;
   float* row_gate = nullptr;
   float *cos_t = nullptr, *sin_t = nullptr;
@@ -294,6 +329,9 @@ struct uno_ctx {
   float* lse_ws = nullptr;                          // [max_batch * 2B]
   unsigned* row_counter = nullptr;                  // [max_batch * 2B]
   unsigned* req_counter = nullptr;                  // [max_batch]
+  int32_t* at_ws = nullptr;                         // [max_batch]
+  float* resid_part = nullptr;                      // [max_batch, nch]
+  unsigned* resid_counter = nullptr;                // [max_batch]
 
   // attention split workspace
   float* att_ws = nullptr;
@@ -372,8 +410,8 @@ struct Prof {
 namespace {
 
 constexpr int PREFILL_CHUNK = 512;
-// The residual pass of spec_verify keeps one sum per vocabulary chunk of
-// 8192 logits in shared memory (64 slots).
+// Largest vocabulary: 64 chunks of 8192 logits (one thread combines a row's
+// chunk pairs serially).
 constexpr int MAX_VOCAB = 64 * 8192;
 
 int fail(uno_ctx* c, int code, const std::string& msg) {
@@ -717,8 +755,190 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   return UNO_OK;
 }
 
+// ---------------------------------------------------------------------------
+// One forward pass, bf16 models on the tensor cores: per layer four DUMP-mode
+// weight streams, each followed by its fused epilogue (epilogue.cuh):
+//
+//   qkv GEMM [Wq|Wk|Wv (|Aq|Ak|Av)] -> epi_qkv   (LoRA-B, norm, RoPE, KV write)
+//   attention (+ split merge)
+//   o GEMM   [Wo (|Ao)]             -> epi_resid (LoRA-B, x +=, ffn-norm input)
+//   gate|up  [Wg|Wu (|Ag|Au)]       -> epi_swiglu
+//   down     [Wd (|Ad)]             -> epi_resid (LoRA-B, x +=, next attn-norm input)
+//
+// then the final RMSNorm and the LM head.  The LoRA A matrices ride in the
+// same weight stream as W (draft pass only), so no pass ever launches a
+// separate rank-r GEMM.
+// ---------------------------------------------------------------------------
+int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* req_ids,
+                  const int32_t* prompt, int prefill_slot, int prefill_pos0, float* logits) {
+  const uno_shape& s = c->s;
+  const int M = n_req * rows_per_req;
+  const int d = s.d_model, H = s.n_heads, Hkv = s.n_kv_heads, hd = s.head_dim, F = s.ffn_dim;
+  const int r = c->r;
+  const int qkv_n = (H + 2 * Hkv) * hd;
+  const bool lora = (kind == PASS_DRAFT) && r > 0;
+  cudaStream_t st = c->stream;
+  const bool pdl = c->genv.pdl;
+
+  RowArgs ra{};
+  ra.kind = kind;
+  ra.rows_per_req = rows_per_req;
+  ra.req_slot = req_ids;
+  ra.cached = c->d_cached;
+  ra.pending = c->d_pending;
+  ra.drafts = c->drafts;
+  ra.B = c->B;
+  ra.prompt = prompt;
+  ra.prefill_slot = prefill_slot;
+  ra.mask_id = s.mask_id;
+  ra.vocab = s.vocab;
+  ra.max_batch = c->max_batch;
+  ra.lora_scale = c->lscale;
+  ra.row_pos = c->row_pos;
+  ra.row_slot = c->row_slot;
+  ra.row_gate = c->row_gate;
+  ra.embed = c->embed;
+  ra.d = d;
+  ra.x = c->x;
+  ra.status = c->d_status;
+  ra.prefill_pos0 = prefill_pos0;
+  {
+    Prof prof(c, UNO_K_OTHER, 0.0);
+    klaunch(pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<bf16>, ra);
+  }
+
+  const int xn_ld = std::max(d, F);
+  const int hhd = H * hd;
+  const bool split = M <= 128;
+  const int lo = split ? c->M_max : 0;
+  bf16* attn_lo = split ? (bf16*)c->attn + (size_t)lo * hhd : nullptr;
+  const int row_groups = ceil_div(M, EPI_RG);
+
+  EpiArgs ea{};
+  ea.M = M;
+  ea.lo_off = lo;
+  ea.n_ss = d / TC_BM;
+  ea.d_model = (float)d;
+  ea.eps = s.rms_eps;
+  ea.q_out = (bf16*)c->qbuf;
+  ea.ld_q = hhd;
+  ea.H = H; ea.Hkv = Hkv; ea.hd = hd;
+  ea.row_pos = c->row_pos;
+  ea.row_slot = c->row_slot;
+  ea.cos_t = c->cos_t;
+  ea.sin_t = c->sin_t;
+  ea.max_pos = c->max_pos;
+  ea.kv = c->kv;
+  ea.x = c->x;
+  ea.d = d;
+  ea.xn = (bf16*)c->xn;
+  ea.ld_xn = xn_ld;
+  ea.ss_out = c->ss;
+  ea.F = F;
+  ea.h = (bf16*)c->xn;
+  ea.status = c->d_status;
+  ea.lr.row_gate = c->row_gate;
+
+  // DUMP-mode GEMM over X [M, K]: the base segments, then (draft pass) the
+  // LoRA A matrices of the same projections as extra output tiles
+  auto gemm = [&](const void* X, int ldx, int K, std::initializer_list<std::pair<const void*, int>> w,
+                  std::initializer_list<const void*> A, PartView* pv) -> int {
+    Gemm g(X, ldx, M, K);
+    for (const auto& e : w) g.seg(e.first, e.second);
+    const int n_base = g.p.N;
+    if (lora)
+      for (const void* a : A) g.seg(a, r);
+    g.p.lo_off = lo;
+    DumpShape sh;
+    {
+      Prof prof(c, UNO_K_GEMM, gemm_bytes(g.p, 2) - (double)M * g.p.N * 2, M, g.p.N, K, 0);
+      if (!gemm_run_dump(c->genv, g.p, st, &sh))
+        return fail(c, UNO_ERR_UNSUPPORTED, "tensor-core GEMM rejected a layer projection");
+    }
+    *pv = PartView{c->genv.part, sh.NT, sh.units, sh.grid, sh.KBt, sh.m_tiles};
+    ea.lr.u_tile0 = n_base / TC_BM;
+    return UNO_OK;
+  };
+  auto set_lora = [&](std::initializer_list<std::pair<const void*, int>> b) {
+    ea.lora = lora ? 1 : 0;
+    ea.lr.nseg = 0;
+    int n0 = 0;
+    for (const auto& e : b) {
+      ea.lr.Bl[ea.lr.nseg] = (const bf16*)e.first;
+      ea.lr.seg_n0[ea.lr.nseg] = n0;
+      n0 += e.second;
+      ea.lr.nseg++;
+    }
+  };
+  auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int threads = TC_BM) {
+    Prof prof(c, UNO_K_OTHER, 0.0);
+    klaunch(pdl, st, dim3(tiles, row_groups), dim3(threads), 0, kernel, ea);
+  };
+
+  // layer-0 input: g * x and the sums of squares of the embedding rows
+  ea.prep = 1;
+  ea.lora = 0;
+  ea.g_next = (const bf16*)c->attn_norm[0];
+  epi(epi_resid_kernel, d / TC_BM);
+  ea.prep = 0;
+
+  for (int l = 0; l < s.n_layers; ++l) {
+    ea.layer = l;
+    int rc = gemm(c->xn, xn_ld, d,
+                  {{c->w[UNO_PROJ_Q][l], H * hd}, {c->w[UNO_PROJ_K][l], Hkv * hd},
+                   {c->w[UNO_PROJ_V][l], Hkv * hd}},
+                  {c->lA[UNO_PROJ_Q][l], c->lA[UNO_PROJ_K][l], c->lA[UNO_PROJ_V][l]}, &ea.pv);
+    if (rc) return rc;
+    set_lora({{c->lB[UNO_PROJ_Q][l], H * hd}, {c->lB[UNO_PROJ_K][l], Hkv * hd},
+              {c->lB[UNO_PROJ_V][l], Hkv * hd}});
+    ea.ss = c->ss;
+    epi(epi_qkv_kernel, qkv_n / TC_BM);
+
+    rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo);
+    if (rc) return rc;
+
+    rc = gemm(c->attn, hhd, hhd, {{c->w[UNO_PROJ_O][l], d}}, {c->lA[UNO_PROJ_O][l]}, &ea.pv);
+    if (rc) return rc;
+    set_lora({{c->lB[UNO_PROJ_O][l], d}});
+    ea.ss = nullptr;
+    ea.g_next = (const bf16*)c->ffn_norm[l];
+    epi(epi_resid_kernel, d / TC_BM);
+
+    rc = gemm(c->xn, xn_ld, d, {{c->w[UNO_PROJ_GATE][l], F}, {c->w[UNO_PROJ_UP][l], F}},
+              {c->lA[UNO_PROJ_GATE][l], c->lA[UNO_PROJ_UP][l]}, &ea.pv);
+    if (rc) return rc;
+    set_lora({{c->lB[UNO_PROJ_GATE][l], F}, {c->lB[UNO_PROJ_UP][l], F}});
+    ea.ss = c->ss;
+    epi(epi_swiglu_kernel, F / TC_BM, 2 * TC_BM);
+
+    rc = gemm(c->xn, F, F, {{c->w[UNO_PROJ_DOWN][l], d}}, {c->lA[UNO_PROJ_DOWN][l]}, &ea.pv);
+    if (rc) return rc;
+    set_lora({{c->lB[UNO_PROJ_DOWN][l], d}});
+    ea.ss = nullptr;
+    ea.g_next = l + 1 < s.n_layers ? (const bf16*)c->attn_norm[l + 1] : nullptr;
+    epi(epi_resid_kernel, d / TC_BM);
+  }
+  if (logits) {
+    bf16* xn_lo = split ? (bf16*)c->xn + (size_t)lo * xn_ld : nullptr;
+    {
+      Prof prof(c, UNO_K_OTHER, 0.0);
+      klaunch(pdl, st, dim3(M), dim3(256), 0, rmsnorm_kernel<bf16, 256>, (const float*)c->x,
+              (const bf16*)c->final_norm, (bf16*)c->xn, xn_lo, d, xn_ld, s.rms_eps);
+    }
+    Gemm g(c->xn, xn_ld, M, d);
+    g.seg(c->lm_head, s.vocab).epi(EPI_STORE_F32, logits, s.vocab, 1.0f / s.temperature);
+    g.p.lo_off = lo;
+    launch_gemm<bf16>(c, g, st);
+  }
+  CK(cudaGetLastError());
+  return UNO_OK;
+}
+
 int forward_any(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* req_ids,
                 const int32_t* prompt, int prefill_slot, int prefill_pos0, float* logits) {
+  if (c->fused && c->fused_enabled)
+    return forward_fused(c, kind, n_req, rows_per_req, req_ids, prompt, prefill_slot, prefill_pos0,
+                         logits);
   if (c->s.dtype == UNO_BF16)
     return forward<bf16>(c, kind, n_req, rows_per_req, req_ids, prompt, prefill_slot, prefill_pos0,
                          logits);
@@ -869,8 +1089,12 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->lse_ws, rows_ws * 4) != cudaSuccess) return oom("lse");
   if (dalloc(&c->row_counter, rows_ws * 4) != cudaSuccess) return oom("counters");
   if (dalloc(&c->req_counter, (size_t)max_batch * 4) != cudaSuccess) return oom("counters");
+  if (dalloc(&c->at_ws, (size_t)max_batch * 4) != cudaSuccess) return oom("verify ws");
+  if (dalloc(&c->resid_part, (size_t)max_batch * c->nch * 4) != cudaSuccess) return oom("verify ws");
+  if (dalloc(&c->resid_counter, (size_t)max_batch * 4) != cudaSuccess) return oom("counters");
   cudaMemset(c->row_counter, 0, rows_ws * 4);
   cudaMemset(c->req_counter, 0, (size_t)max_batch * 4);
+  cudaMemset(c->resid_counter, 0, (size_t)max_batch * 4);
   cudaMemset(c->drafts, 0, (size_t)max_batch * B * 4);
 
   // attention split workspace: groups x splits <= about two waves of CTAs
@@ -894,6 +1118,30 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
     if (dalloc(&c->genv.counters, (size_t)TC_COUNTERS * 4) != cudaSuccess) return oom("gemm ws");
     cudaMemset(c->genv.counters, 0, (size_t)TC_COUNTERS * 4);
     c->genv.status = c->d_status;
+  }
+  // fused bf16 layer pipeline: 128-column tiles must not straddle q/k/v or
+  // heads, the adapter rank must fill whole tiles, weights 16-byte aligned
+  {
+    bool ok = s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && d % TC_BM == 0 &&
+              F % TC_BM == 0 && (H * hd) % TC_BM == 0 && (Hkv * hd) % TC_BM == 0 &&
+              (lora_rank == 0 || lora_rank == EPI_R) && d <= EPI_MAX_SS * TC_BM;
+    for (int pj = 0; pj < UNO_N_PROJ && ok; ++pj)
+      for (int l = 0; l < L && ok; ++l) {
+        ok = ((uintptr_t)c->w[pj][l] & 15) == 0;
+        if (lora_rank) ok = ok && ((uintptr_t)c->lA[pj][l] & 15) == 0 && ((uintptr_t)c->lB[pj][l] & 15) == 0;
+      }
+    if (ok) {
+      size_t part = 0;
+      const int rr = lora_rank;
+      for (int m = 1; m <= M; ++m) {
+        const int ns[4] = {(H + 2 * Hkv) * hd + 3 * rr, d + rr, 2 * F + 2 * rr, d + rr};
+        for (int k = 0; k < 4; ++k) part = std::max(part, dump_bytes(m, ns[k], c->genv.sm_count));
+      }
+      if (dalloc(&c->genv.part, part) != cudaSuccess) return oom("gemm parts");
+      c->genv.part_bytes = part;
+      if (dalloc(&c->ss, (size_t)M * (d / TC_BM) * 4) != cudaSuccess) return oom("norm sums");
+      c->fused = true;
+    }
   }
   // tensor-core attention: the pool as a [rows, head_dim] tensor, 64x64 boxes
   if (s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && ATC_QROWS % G == 0) {
@@ -919,8 +1167,9 @@ int uno_destroy(uno_ctx* c) {
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
                   c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
                   c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
-                  c->lse_ws, c->row_counter, c->req_counter, c->att_ws, c->att_counters,
-                  c->d_status, c->genv.ws, c->genv.counters};
+                  c->lse_ws, c->row_counter, c->req_counter, c->at_ws, c->resid_part,
+                  c->resid_counter, c->att_ws, c->att_counters,
+                  c->d_status, c->genv.ws, c->genv.counters, c->genv.part, c->ss};
   for (void* b : bufs)
     if (b) cudaFree(b);
   for (cudaEvent_t e : c->ev_pool) cudaEventDestroy(e);
@@ -1093,12 +1342,22 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.lse = c->lse_ws;
     a.row_counter = c->row_counter;
     a.req_counter = c->req_counter;
+    a.at_ws = c->at_ws;
+    a.resid_part = c->resid_part;
+    a.resid_counter = c->resid_counter;
     a.rows_red = B;      // B - 1 test rows + the bonus row; lse of q comes from draft_sample
     a.n_p = B;
     a.status = c->d_status;
-    Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
-    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
-            spec_verify_kernel, a);
+    {
+      Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
+      klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
+              spec_verify_kernel, a);
+    }
+    {
+      Prof prof(c, UNO_K_VERIFY, (double)n_req * 2 * V * 4);
+      klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req), dim3(SAMPLE_THREADS), 0,
+              spec_resid_kernel, a);
+    }
   }
   CK(cudaGetLastError());
   return UNO_OK;
@@ -1173,6 +1432,17 @@ int uno_set_pdl(uno_ctx* c, int enable) {
     g.seen = 0;
   }
   return UNO_OK;
+}
+
+int uno_set_fused(uno_ctx* c, int enable) {
+  if (!c) return UNO_ERR_ARG;
+  c->fused_enabled = enable != 0;
+  for (auto& g : c->graphs) {   // graphs captured with the other pipeline
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.seen = 0;
+  }
+  return c->fused ? UNO_OK : UNO_ERR_UNSUPPORTED;
 }
 
 int uno_profile_records(uno_ctx* c, uno_prof_record* out, int max) {
@@ -1368,7 +1638,7 @@ int uno_gated_lora_linear(int dtype, const void* X, const void* W, const void* A
 // ---------------------------------------------------------------------------
 
 struct VerifyWs {
-  size_t counters, req_counters, lse, partial, total;
+  size_t counters, req_counters, resid_counters, lse, partial, at, resid, total;
 };
 static VerifyWs verify_ws_layout(int n_req, int n_tests, int vocab) {
   int ch, nch;
@@ -1377,9 +1647,12 @@ static VerifyWs verify_ws_layout(int n_req, int n_tests, int vocab) {
   VerifyWs w{};
   w.counters = 0;
   w.req_counters = align256(rows * 4);
-  w.lse = w.req_counters + align256((size_t)n_req * 4);
+  w.resid_counters = w.req_counters + align256((size_t)n_req * 4);
+  w.lse = w.resid_counters + align256((size_t)n_req * 4);   // counters end here
   w.partial = w.lse + align256(rows * 4);
-  w.total = w.partial + align256(rows * nch * sizeof(float2));
+  w.at = w.partial + align256(rows * nch * sizeof(float2));
+  w.resid = w.at + align256((size_t)n_req * 4);
+  w.total = w.resid + align256((size_t)n_req * nch * 4);
   return w;
 }
 
@@ -1418,11 +1691,15 @@ int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n
   a.req_counter = (unsigned*)(base + w.req_counters);
   a.lse = (float*)(base + w.lse);
   a.partial = (float2*)(base + w.partial);
+  a.at_ws = (int32_t*)(base + w.at);
+  a.resid_part = (float*)(base + w.resid);
+  a.resid_counter = (unsigned*)(base + w.resid_counters);
   a.rows_red = 2 * n_tests;
   a.n_p = n_tests;
   a.status = nullptr;
   const int rows = n_req * 2 * n_tests;
   spec_verify_kernel<<<dim3(nch, rows), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
+  spec_resid_kernel<<<dim3(nch, n_req), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 

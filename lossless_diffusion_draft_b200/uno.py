@@ -83,6 +83,7 @@ def load_library(path=LIB_PATH):
         "uno_debug_launch_counts": (i32, [vp]),
         "uno_set_graphs": (i32, [vp, i32]),
         "uno_set_pdl": (i32, [vp, i32]),
+        "uno_set_fused": (i32, [vp, i32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
@@ -219,6 +220,15 @@ def uno_set_graphs(ctx, enable):
 
 def uno_set_pdl(ctx, enable):
     _check(load_library().uno_set_pdl(ctx.handle, int(bool(enable))), ctx.handle)
+
+
+def uno_set_fused(ctx, enable):
+    """Returns False when the model does not take the fused pipeline."""
+    code = load_library().uno_set_fused(ctx.handle, int(bool(enable)))
+    if code == UNO_ERR_UNSUPPORTED:
+        return False
+    _check(code, ctx.handle)
+    return True
 
 
 def uno_release(ctx, req_id):

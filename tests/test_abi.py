@@ -49,13 +49,16 @@ def test_null_context_calls(lib):
 
 
 def test_spec_verify_workspace_and_argument_checks(lib):
-    # counters (rows) | request counters | lse (rows) | partial pairs (rows x chunks)
+    # counters (rows) | request counters | residual counters (requests) |
+    # lse (rows) | partial pairs (rows x chunks) | first rejection (requests) |
+    # residual chunk sums (requests x chunks)
     n_req, n_tests, V = 256, 16, 151936
     rows = n_req * 2 * n_tests
     nch = -(-V // 8192)
     def a256(x):
         return (x + 255) // 256 * 256
-    want = a256(rows * 4) + a256(n_req * 4) + a256(rows * 4) + a256(rows * nch * 8)
+    want = (a256(rows * 4) + a256(n_req * 4) + a256(n_req * 4) + a256(rows * 4) +
+            a256(rows * nch * 8) + a256(n_req * 4) + a256(n_req * nch * 4))
     assert uno.uno_spec_verify_workspace_bytes(n_req, n_tests, V) == want
     assert uno.uno_spec_verify_workspace_bytes(0, 16, V) == 0
     null = None

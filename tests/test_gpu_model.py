@@ -25,7 +25,7 @@ import parity
 pytestmark = pytest.mark.gpu
 
 
-def _setup(name, n_req, prompt_len, max_ctx, **over):
+def _setup(name, n_req, prompt_len, max_ctx, fused=True, **over):
     cfg = dict(synth.CONFIGS[name], **over)
     shape = synth.model_shape(cfg)
     shape["dtype"] = cfg["dtype"]
@@ -33,6 +33,8 @@ def _setup(name, n_req, prompt_len, max_ctx, **over):
     params = {k: v.cuda() for k, v in params_cpu.items()}
     ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], n_req, max_ctx,
                        cfg["seed"], torch.cuda.current_stream())
+    if not fused:
+        uno.uno_set_fused(ctx, False)
     prompts = synth.make_prompts(cfg, n_req, prompt_len)
     ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).cuda(), [prompt_len] * n_req,
                           streams=list(range(n_req)))
@@ -53,9 +55,10 @@ def _kv_check(ctx, cfg, model, state, req, tol):
         np.testing.assert_allclose(v.double().numpy(), state.cache.v[l], atol=tol, rtol=0)
 
 
-def _run(name, n_req, prompt_len, n_steps, logit_tol, kv_tol, end_to_end, max_ctx=None, **over):
+def _run(name, n_req, prompt_len, n_steps, logit_tol, kv_tol, end_to_end, max_ctx=None,
+         fused=True, **over):
     cfg, ctx, ids, model, states = _setup(name, n_req, prompt_len,
-                                          max_ctx or prompt_len + (n_steps + 1) * 20, **over)
+                                          max_ctx or prompt_len + (n_steps + 1) * 20, fused, **over)
     B, V, seed = cfg["B"], cfg["vocab"], cfg["seed"]
     req = torch.tensor(ids, dtype=torch.int32, device="cuda")
     out = torch.zeros((n_req, B + 1), dtype=torch.int32, device="cuda")
@@ -182,16 +185,31 @@ def test_tiny_fp32_ar_step():
     ctx.close()
 
 
-def test_small_bf16_steps():
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "unfused"])
+def test_small_bf16_steps(fused):
     """Small bf16 model (8 layers, d 1024, GQA 16/4, vocab 32000, B=8) on
-    short prompts: logits within 2e-2 of the fp64 oracle."""
+    short prompts: logits within 2e-2 of the fp64 oracle, with the fused
+    layer pipeline (GEMM parts reduced by the epilogue kernels) and without."""
     before = uno.uno_debug_launch_counts()
-    tally, _, worst = _run("small", 3, 40, 3, 2e-2, 2e-2, False, max_ctx=120)
+    tally, _, worst = _run("small", 3, 40, 3, 2e-2, 2e-2, False, max_ctx=120, fused=fused)
     after = uno.uno_debug_launch_counts()
     assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
     # the bf16 decode path runs on the tensor-core kernels only
     assert after["tc_gemm"] > before["tc_gemm"] and after["tc_attn"] > before["tc_attn"]
     assert after["simt_gemm"] == before["simt_gemm"]
+
+
+def test_fused_pipeline_applies():
+    """The fused pipeline takes the bf16 workloads' shapes and refuses fp32."""
+    for name, want in (("small", True), ("tiny", False)):
+        cfg = dict(synth.CONFIGS[name])
+        shape = synth.model_shape(cfg)
+        shape["dtype"] = cfg["dtype"]
+        params = {k: v.cuda() for k, v in synth.make_params(cfg, "cpu").items()}
+        ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], cfg["B"], 1, 64, 0,
+                           torch.cuda.current_stream())
+        assert uno.uno_set_fused(ctx, True) is want
+        ctx.close()
 
 
 def test_capacity_and_bad_ids():
