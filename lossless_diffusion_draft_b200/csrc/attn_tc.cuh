@@ -34,6 +34,7 @@ constexpr int ATC_THREADS = 192;
 constexpr int ATC_QROWS = 128;
 constexpr int ATC_KT = 64;          // keys per tile = one KV page
 constexpr int ATC_STAGES = 4;
+constexpr int ATC_PAGE_PF = 64;     // page numbers a CTA fetches up front
 constexpr int ST_ATTN_TIMEOUT = 16;
 // Floats per query row of a split partial: O[HD], m, l, padded so that every
 // row starts on a 16-byte boundary (rows are written with float4 stores).
@@ -113,6 +114,24 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   const int ntok = min(TQ, p.rows_per_req - tok0);
   const int nq = ntok * G;
   const int row0 = req * p.rows_per_req + tok0;
+  // the q rows (warps 0-3, one row per thread) and the row's position are
+  // fetched first; nothing below waits for them before the shared-memory store
+  uint4 qv[HD / 8];
+  int qpos = -1;
+  if (warp < 4) {
+    const int r = threadIdx.x;
+    if (r < nq) {
+      const int tk = r / G, g = r % G;
+      const uint4* src =
+          reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + tk) * p.ld_q + (size_t)(kvh * G + g) * HD);
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) qv[j] = src[j];
+      qpos = p.row_pos[row0 + tk];
+    } else {
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) qv[j] = make_uint4(0, 0, 0, 0);
+    }
+  }
   const int slot = p.row_slot[row0];
   const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
   int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
@@ -148,20 +167,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   // query rows -> shared memory, K-major 128-byte swizzle (zero rows past nq)
   if (warp < 4) {
     const int r = threadIdx.x;
-    const uint4* src = nullptr;
-    if (r < nq) {
-      const int tk = r / G, g = r % G;
-      src = reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + tk) * p.ld_q + (size_t)(kvh * G + g) * HD);
-    }
 #pragma unroll
     for (int j = 0; j < HD / 8; ++j) {
-      const uint4 v = src ? src[j] : make_uint4(0, 0, 0, 0);
       const int box = j >> 3, c = j & 7;
-      *reinterpret_cast<uint4*>(sQ + box * (ATC_QROWS * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(sQ + box * (ATC_QROWS * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = qv[j];
     }
     fence_async_smem();
   }
-  if (warp == 4 && lane == 0) prefetch_map(&kvmap);
+  // the split's page numbers, fetched in one round while the q rows load
+  __shared__ int s_pages[ATC_PAGE_PF];
+  if (warp == 4) {
+    if (lane == 0) prefetch_map(&kvmap);
+    for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32)
+      s_pages[i] = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -176,7 +195,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         const uint32_t phase = (uint32_t)(i / ATC_STAGES) & 1;
         if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
         mbar_expect_tx(&kv_full[stage], 2 * C::KV_BYTES);
-        const int page = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+        const int page = i < ATC_PAGE_PF ? s_pages[i]
+                                         : p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
         const int rk = (((p.layer * p.n_pages + page) * 2 + 0) * p.Hkv + kvh) * KV_PAGE;
         const int rv = (((p.layer * p.n_pages + page) * 2 + 1) * p.Hkv + kvh) * KV_PAGE;
 #pragma unroll
@@ -241,7 +261,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   } else {
     // ------------------------------------------------------------ softmax (warps 0-3)
     const int r = threadIdx.x;
-    const int qpos = (r < nq) ? p.row_pos[row0 + r / G] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     // Lazy rescaling: P is formed against a reference max m that moves only
     // when a tile's max exceeds it by more than RESCALE_LOG2 (so P <= 2^8);
@@ -263,13 +282,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
+      // raw scores; keys past the row's position (only in its last tile) -> -inf
       const int kp0 = (t_begin + i) * ATC_KT;
       float mx = -INFINITY;
+      if (kp0 + ATC_KT - 1 <= qpos) {
 #pragma unroll
-      for (int j = 0; j < ATC_KT; ++j) {
-        s[j] = (kp0 + j <= qpos) ? s[j] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < ATC_KT; ++j) mx = fmaxf(mx, s[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < ATC_KT; ++j) {
+          if (kp0 + j > qpos) s[j] = -INFINITY;
+          mx = fmaxf(mx, s[j]);
+        }
       }
+      mx *= p.scale_log2;             // log2 units (the scale is positive)
       bool pv_done = false;           // PV(i-1) known complete
       const bool need = mx > m + RESCALE_LOG2;
       if (__any_sync(0xffffffffu, need)) {
@@ -292,12 +318,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         }
         m = m_new;
       }
+      // P = 2^(s * scale - m) <= 2^RESCALE_LOG2 by the hardware ex2 (P is
+      // rounded to bf16 next, far coarser than its error); a row with no key
+      // yet (m = -inf) has s = -inf everywhere and gets P = 0
+      const float nm = (m == -INFINITY) ? 0.f : -m;
       float psum = 0.f;
       uint32_t pk[ATC_KT / 2];
 #pragma unroll
       for (int j = 0; j < ATC_KT; j += 2) {
-        const float a = (s[j] == -INFINITY) ? 0.f : exp2f(s[j] - m);
-        const float b = (s[j + 1] == -INFINITY) ? 0.f : exp2f(s[j + 1] - m);
+        const float a = fast_exp2(fmaf(s[j], p.scale_log2, nm));
+        const float b = fast_exp2(fmaf(s[j + 1], p.scale_log2, nm));
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
         psum += __low2float(h2) + __high2float(h2);    // the P the MMA will use
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -368,7 +398,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 }
 
 // Merge of the split partials: one CTA per (query row, group), one thread
-// per head_dim element; splits are added in split order.
+// per head_dim element.  Every thread loads all splits' (m, l) (the same
+// addresses across the CTA) together with its own O column, so the merge is
+// one round of loads; the splits are added in split order.
+constexpr int ATC_MAX_SPLITS = 32;
 template <int HD>
 __global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
   pdl_trigger();
@@ -381,25 +414,33 @@ __global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
   const int tok0 = qt * TQ;
   const int ntok = min(TQ, p.rows_per_req - tok0);
   if (r >= ntok * G) return;
-  // n_splits <= HD: thread s first takes split s's (m, l)
-  __shared__ float s_w[HD];
-  __shared__ float red[32];
   const int d = threadIdx.x;
   const size_t sstride = (size_t)ATC_QROWS * atc_ws_row(HD);
   const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * atc_ws_row(HD);
-  float ms = -INFINITY, ls = 0.f;
-  if (d < p.n_splits) {
-    ms = wg[d * sstride + HD];
-    ls = wg[d * sstride + HD + 1];
+  float ms[ATC_MAX_SPLITS], ls[ATC_MAX_SPLITS], os[ATC_MAX_SPLITS];
+#pragma unroll
+  for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
+    if (s < p.n_splits) {
+      const float2 ml = *reinterpret_cast<const float2*>(wg + s * sstride + HD);
+      ms[s] = ml.x;
+      ls[s] = ml.y;
+      os[s] = wg[s * sstride + d];
+    } else {
+      ms[s] = -INFINITY;
+      ls[s] = 0.f;
+      os[s] = 0.f;
+    }
   }
-  const float M = block_max<HD>(ms, red);
-  const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-  s_w[d] = wt;
-  const float L = block_sum<HD>(ls * wt, red);
-  __syncthreads();
-  float O = 0.f;
-#pragma unroll 8
-  for (int s = 0; s < p.n_splits; ++s) O += wg[s * sstride + d] * s_w[s];
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < ATC_MAX_SPLITS; ++s) M = fmaxf(M, ms[s]);
+  float L = 0.f, O = 0.f;
+#pragma unroll
+  for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
+    const float w = (ms[s] == -INFINITY) ? 0.f : exp2f(ms[s] - M);
+    L += ls[s] * w;
+    O += os[s] * w;
+  }
   const int row0 = req * p.rows_per_req + tok0;
   const int tk = r / G, g = r % G;
   const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;

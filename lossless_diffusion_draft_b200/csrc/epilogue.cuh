@@ -35,7 +35,7 @@
 
 namespace uno {
 
-constexpr int EPI_RG = 8;            // token rows per CTA
+constexpr int EPI_RG = 9;            // token rows per CTA (a 17-row draft pass: two groups)
 constexpr int EPI_R = TC_BM;         // LoRA rank the fused epilogue takes (one U tile)
 
 // Where a DUMP-mode GEMM left its parts.
@@ -54,7 +54,7 @@ struct LoraEpi {
 };
 
 struct EpiArgs {
-  PartView pv;
+  PartView pv;                       // (prep: NT = M, m_tiles = 1, no parts read)
   int M;
   int lo_off;                        // split rows: lo rows this many rows below (0: none)
   // RMSNorm scale of the GEMM input (null: input not normalised)
@@ -82,6 +82,21 @@ struct EpiArgs {
 // part_issue loads the first C contributors (issued before any use);
 // part_add adds them in CTA order, the first contributor's part first, then
 // reads any further contributors C at a time.
+// Row groups never straddle an m-tile of the GEMM (the part slots are per
+// m-tile): blockIdx.y = m-tile * groups_per_tile + group.  Returns false for
+// a group past the rows (whole CTA).
+__host__ __device__ __forceinline__ int epi_groups_per_tile(int NT, int M) {
+  return ((NT < M ? NT : M) + EPI_RG - 1) / EPI_RG;
+}
+__device__ __forceinline__ bool row_group(const EpiArgs& a, int* m0, int* nrows) {
+  const int gpt = epi_groups_per_tile(a.pv.NT, a.M);
+  const int mt = blockIdx.y / gpt, g = blockIdx.y % gpt;
+  *m0 = mt * a.pv.NT + g * EPI_RG;
+  const int end = min(a.M, (mt + 1) * a.pv.NT);
+  *nrows = min(EPI_RG, end - *m0);
+  return *nrows > 0;
+}
+
 template <int C>
 struct PartLoad {
   float x[C][EPI_RG];
@@ -239,8 +254,9 @@ __global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
   __shared__ float sY[EPI_RG][TC_BM];
   pdl_trigger();
   pdl_wait();
-  const int nt = blockIdx.x, m0 = blockIdx.y * EPI_RG;
-  const int nrows = min(EPI_RG, a.M - m0);
+  const int nt = blockIdx.x;
+  int m0, nrows;
+  if (!row_group(a, &m0, &nrows)) return;
   const int i = threadIdx.x;
   const int n = nt * TC_BM + i;
   const int qcols = a.H * a.hd, kcols = a.Hkv * a.hd;
@@ -250,11 +266,12 @@ __global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
   const int ci = hi < half ? hi : hi - half;
 
   // ---- every global load first
+  const bool kv_tile = n >= qcols;
   int pos[EPI_RG], slot[EPI_RG];
 #pragma unroll
   for (int j = 0; j < EPI_RG; ++j) {
     pos[j] = j < nrows ? a.row_pos[m0 + j] : 0;
-    slot[j] = (j < nrows && n >= qcols) ? a.row_slot[m0 + j] : 0;   // k and v tiles
+    slot[j] = (j < nrows && kv_tile) ? a.row_slot[m0 + j] : 0;
   }
   float ssv[4];
   ss_issue(a, m0, nrows, ssv);
@@ -268,12 +285,18 @@ __global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
     gate_issue(a, m0, nrows, gate);
   }
   part_issue(a.pv, nt, m0, nrows, i, LP);
+  // second round, addressed by the rows' positions and slots: RoPE table
+  // entries and the KV pages
   float cs[EPI_RG], sn[EPI_RG];
+  int page[EPI_RG], pok[EPI_RG];
 #pragma unroll
   for (int j = 0; j < EPI_RG; ++j) {
     const int pc = (pos[j] >= 0 && pos[j] < a.max_pos) ? pos[j] : 0;
     cs[j] = rot ? a.cos_t[(size_t)pc * half + ci] : 0.f;
     sn[j] = rot ? a.sin_t[(size_t)pc * half + ci] : 0.f;
+    int ok = 0;
+    page[j] = (j < nrows && kv_tile) ? a.kv.page_of(slot[j], pos[j], ok) : 0;
+    pok[j] = ok;
   }
 
   // ---- then the arithmetic
@@ -286,7 +309,9 @@ __global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
   for (int j = 0; j < EPI_RG; ++j) sY[j][i] = acc[j] * s_inv[j];
   __syncthreads();
 
-  for (int j = 0; j < nrows; ++j) {
+#pragma unroll
+  for (int j = 0; j < EPI_RG; ++j) {
+    if (j >= nrows) continue;
     const int m = m0 + j;
     const bool ok_pos = pos[j] >= 0 && pos[j] < a.max_pos;
     float y = sY[j][i];
@@ -298,9 +323,8 @@ __global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
     } else {
       const bool is_k = n < qcols + kcols;
       const int head = (n - (is_k ? qcols : qcols + kcols)) / a.hd;
-      int ok;
-      const size_t off = a.kv.offset(a.layer, slot[j], pos[j], is_k ? 0 : 1, head, ok);
-      if (ok && ok_pos) reinterpret_cast<bf16*>(a.kv.pool)[off + hi] = from_f<bf16>(y);
+      const size_t off = a.kv.offset_in_page(a.layer, page[j], pos[j], is_k ? 0 : 1, head);
+      if (pok[j] && ok_pos) reinterpret_cast<bf16*>(a.kv.pool)[off + hi] = from_f<bf16>(y);
       else if (hi == 0 && is_k) raise_status(a.status, ST_POS_OVERFLOW);
     }
   }
@@ -341,8 +365,9 @@ __global__ void __launch_bounds__(TC_BM) epi_resid_kernel(const EpiArgs a) {
   __shared__ __align__(16) float sU[EPI_RG * EPI_R];
   pdl_trigger();
   pdl_wait();
-  const int nt = blockIdx.x, m0 = blockIdx.y * EPI_RG;
-  const int nrows = min(EPI_RG, a.M - m0);
+  const int nt = blockIdx.x;
+  int m0, nrows;
+  if (!row_group(a, &m0, &nrows)) return;
   const int i = threadIdx.x;
   const int n = nt * TC_BM + i;
 
@@ -391,8 +416,9 @@ __global__ void __launch_bounds__(2 * TC_BM) epi_swiglu_kernel(const EpiArgs a) 
   __shared__ float sUp[EPI_RG][TC_BM];
   pdl_trigger();
   pdl_wait();
-  const int ft = blockIdx.x, m0 = blockIdx.y * EPI_RG;
-  const int nrows = min(EPI_RG, a.M - m0);
+  const int ft = blockIdx.x;
+  int m0, nrows;
+  if (!row_group(a, &m0, &nrows)) return;
   const int half = threadIdx.x / TC_BM;      // 0: gate, 1: up
   const int i = threadIdx.x % TC_BM;
   const int f = ft * TC_BM + i;

@@ -73,11 +73,13 @@ struct TcParams {
 // ---------------------------------------------------------------------------
 // Stream-K partition.
 // ---------------------------------------------------------------------------
+// 32-bit arithmetic: units * grid stays below 2^32 for every launch (the
+// host checks), and a 64-bit division is a long software sequence.
 __device__ __forceinline__ int sk_start(int i, int units, int grid) {
-  return (int)(((long long)i * units) / grid);
+  return (int)(((unsigned)i * (unsigned)units) / (unsigned)grid);
 }
 __device__ __forceinline__ int sk_owner(int u, int units, int grid) {
-  int i = (int)(((long long)u * grid) / units);
+  int i = (int)(((unsigned)u * (unsigned)grid) / (unsigned)units);
   while (i + 1 < grid && sk_start(i + 1, units, grid) <= u) ++i;
   while (i > 0 && sk_start(i, units, grid) > u) --i;
   return i;
@@ -187,14 +189,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (n_row >= p.seg[s].n0) sg = s;
         return sg;
       };
-      auto load_a = [&](int u, int stage) {     // weights: W, then LoRA-B
+      // weight tile of unit u: W, then LoRA-B
+      auto coords_a = [&](int u, const CUtensorMap*& map, int& x, int& y) {
         const int t = u / KBt, kb = u % KBt;
         const int n_row = (t / p.m_tiles) * TC_BM;
         const int sg = seg_of(n_row);
-        uint8_t* dst = sA + stage * TC_A_BYTES;
-        if (kb < p.KB) tma_load_2d(dst, &maps.w[sg], &full[stage], kb * TC_BK, n_row - p.seg[sg].n0);
-        else tma_load_2d(dst, &maps.b[sg], &full[stage], (kb - p.KB) * TC_BK, n_row - p.seg[sg].n0);
+        map = kb < p.KB ? &maps.w[sg] : &maps.b[sg];
+        x = (kb < p.KB ? kb : kb - p.KB) * TC_BK;
+        y = n_row - p.seg[sg].n0;
       };
+      auto load_a = [&](int u, int stage) {
+        const CUtensorMap* map;
+        int x, y;
+        coords_a(u, map, x, y);
+        tma_load_2d(sA + stage * TC_A_BYTES, map, &full[stage], x, y);
+      };
+
       auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
         const int t = u / KBt, kb = u % KBt;
         const int mt = t % p.m_tiles;

@@ -22,9 +22,16 @@ struct KvLayout {
   const int32_t* page_table;   // [max_batch][pages_per_req]
   __device__ __forceinline__ size_t offset(int layer, int slot, int pos, int kv, int head,
                                            int& ok) const {
+    return offset_in_page(layer, page_of(slot, pos, ok), pos, kv, head);
+  }
+  // page of (slot, pos); ok = 0 (page 0 returned) when pos is outside the slot's pages
+  __device__ __forceinline__ int page_of(int slot, int pos, int& ok) const {
     const int pi = pos / KV_PAGE;
     ok = (pos >= 0 && pi < pages_per_req);
-    const int page = ok ? page_table[(size_t)slot * pages_per_req + pi] : 0;
+    return ok ? page_table[(size_t)slot * pages_per_req + pi] : 0;
+  }
+  __device__ __forceinline__ size_t offset_in_page(int layer, int page, int pos, int kv,
+                                                   int head) const {
     return ((((size_t)layer * n_pages + page) * 2 + kv) * n_kv_heads + head) * KV_PAGE * head_dim +
            (size_t)(pos % KV_PAGE) * head_dim;
   }

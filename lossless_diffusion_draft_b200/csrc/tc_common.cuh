@@ -114,6 +114,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 2^x by the special-function unit (ex2.approx: about 2 ulp; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void epi_bar() {   // named barrier of the 4 epilogue warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }

@@ -186,6 +186,8 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.n_tiles = (p.N + TC_BM - 1) / TC_BM;
   tp.m_tiles = (p.M + NT - 1) / NT;
   if ((long long)tp.n_tiles * tp.m_tiles > TC_COUNTERS) return false;
+  // the device's stream-K arithmetic is 32-bit: units * grid < 2^32
+  if ((long long)tp.n_tiles * tp.m_tiles * (tp.KB + tp.RB) * env.sm_count >= (1LL << 32)) return false;
   tp.units = tp.n_tiles * tp.m_tiles * (tp.KB + tp.RB);
   // at least TC_MIN_UNITS k-blocks per CTA: a tile is then cut into few
   // parts and its last contributor has few partials to add
@@ -519,8 +521,9 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   const int groups = n_req * s.n_kv_heads * p.n_qtiles;
   int S = 1;
   if (decode && groups < c->genv.sm_count) {
-    S = ceil_div(c->genv.sm_count, groups);
-    S = std::max(1, std::min(std::min(S, c->kv.pages_per_req / 2), HD));   // merge: S <= HD
+    // one CTA per SM (shared memory): at most sm_count CTAs, else a second wave
+    S = c->genv.sm_count / groups;
+    S = std::max(1, std::min(std::min(S, c->kv.pages_per_req / 2), ATC_MAX_SPLITS));
     while (S > 1 && (size_t)groups * S * ATC_QROWS * atc_ws_row(HD) > c->att_ws_floats) --S;
     if (groups > c->att_groups_max) S = 1;
   }
@@ -812,7 +815,6 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   const bool split = M <= 128;
   const int lo = split ? c->M_max : 0;
   bf16* attn_lo = split ? (bf16*)c->attn + (size_t)lo * hhd : nullptr;
-  const int row_groups = ceil_div(M, EPI_RG);
 
   EpiArgs ea{};
   ea.M = M;
@@ -872,12 +874,14 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   };
   auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int threads = TC_BM) {
     Prof prof(c, UNO_K_OTHER, 0.0);
-    klaunch(pdl, st, dim3(tiles, row_groups), dim3(threads), 0, kernel, ea);
+    const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M);
+    klaunch(pdl, st, dim3(tiles, groups), dim3(threads), 0, kernel, ea);
   };
 
   // layer-0 input: g * x and the sums of squares of the embedding rows
   ea.prep = 1;
   ea.lora = 0;
+  ea.pv = PartView{nullptr, M, 0, 1, 1, 1};
   ea.g_next = (const bf16*)c->attn_norm[0];
   epi(epi_resid_kernel, d / TC_BM);
   ea.prep = 0;

@@ -199,6 +199,14 @@ def test_small_bf16_steps(fused):
     assert after["simt_gemm"] == before["simt_gemm"]
 
 
+def test_small_bf16_long_prefill():
+    """A 300-token prompt: the prefill pass has more rows than one GEMM token
+    tile (two m-tiles of 256 rows), so the epilogue's row groups follow the
+    m-tiles; the cache it writes must give oracle logits in the next step."""
+    tally, _, worst = _run("small", 1, 300, 1, 2e-2, 2e-2, False, max_ctx=340)
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
+
+
 def test_fused_pipeline_applies():
     """The fused pipeline takes the bf16 workloads' shapes and refuses fp32."""
     for name, want in (("small", True), ("tiny", False)):
