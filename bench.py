@@ -166,6 +166,41 @@ def oracle_step_sample(cfg, context, tokens_per_step, budget_s=20.0):
     return step_s, desc
 
 
+# ---------------------------------------------------------------------------
+# DRAM traffic of the dominant kernel, from the committed ncu summary.  The
+# summary records a hash of the kernel's source files; the figure is used
+# only while the sources still hash the same (else the traffic is unknown).
+# ---------------------------------------------------------------------------
+GEMM_SOURCES = ("lossless_diffusion_draft_b200/csrc/gemm_tc.cuh",
+                "lossless_diffusion_draft_b200/csrc/tc_common.cuh")
+GEMM_PROFILE = "profiles/gemm_tc_gate_up_qwen8b.md"
+
+
+def source_hash(paths):
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(top):
+    import re
+    path = os.path.join(ROOT, GEMM_PROFILE)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    shape = re.search(r"shape:\s*M=(\d+) N=(\d+) K=(\d+)", text)
+    b = re.search(r"dram_bytes_per_launch:\s*(\d+)", text)
+    if not (h and shape and b) or h.group(1) != source_hash(GEMM_SOURCES):
+        return None
+    if tuple(int(x) for x in shape.groups()) != (top["m"], top["n"], top["k"]):
+        return None
+    return int(b.group(1))
+
+
 def synth_shape(cfg):
     from lossless_diffusion_draft_b200 import synth
     return synth.model_shape(cfg)
@@ -182,8 +217,9 @@ def cpu_cores():
 # Workload set-up.
 # ---------------------------------------------------------------------------
 def kv_bytes_per_token(cfg):
-    esz = 2 if cfg["dtype"] == "bf16" else 4
-    return cfg["n_layers"] * 2 * cfg["n_kv_heads"] * cfg["head_dim"] * esz
+    # bf16 models: K as an fp16 hi/lo pair and V in fp16 (three planes)
+    esz, planes = (2, 3) if cfg["dtype"] == "bf16" else (4, 2)
+    return cfg["n_layers"] * planes * cfg["n_kv_heads"] * cfg["head_dim"] * esz
 
 
 def max_batch_that_fits(cfg, weight_bytes, max_ctx):
@@ -241,6 +277,7 @@ def run_uno(args, rank, world, device):
     barrier(world)
     uno.uno_profile_begin(ctx, 0)          # launch counting only
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_step = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
         # a profiler started with --profile-from-start off sees the timed
@@ -249,12 +286,15 @@ def run_uno(args, rank, world, device):
         ev0.record(stream)
         for k in range(K):
             uno.uno_spec_step(ctx, req, out, n_new_all[k])
+            ev_step[k].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize()
         torch.cuda.profiler.stop()
     prof = uno.uno_profile_end(ctx)
     barrier(world)
     ms = ev0.elapsed_time(ev1)
+    step_ms = [ev0.elapsed_time(ev_step[0])] + [ev_step[k - 1].elapsed_time(ev_step[k])
+                                                 for k in range(1, K)]
     tokens = int(n_new_all.sum().item())
     ctx_after = uno.uno_request_state(ctx, ids[0])[0]
     launches = sum(v[0] for v in prof.values())
@@ -305,13 +345,29 @@ def run_uno(args, rank, world, device):
     e2e_ms = e0.elapsed_time(e1)
     uno.uno_status(ctx)
 
+    # the AR-only decode of the same model from the same kernels (one token per
+    # request per step, LoRA never read): the baseline Psi-Spec is measured
+    # against
+    ar_out = torch.zeros(batch, dtype=torch.int32, device=device)
+    for _ in range(W):
+        uno.uno_ar_step(ctx, req, ar_out)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(K):
+        uno.uno_ar_step(ctx, req, ar_out)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    ar_ms = a0.elapsed_time(a1) / K
+    uno.uno_status(ctx)
+
     # aggregate over ranks: tokens summed, time = max
     ms_max = reduce_max(ms, world, device)
     e2e_ms_max = reduce_max(e2e_ms, world, device)
     tokens_all = reduce_sum(tokens, world, device)
     e2e_tokens_all = reduce_sum(e2e_tokens, world, device)
 
-    info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, fused=fused, tokens=tokens_all, K=K, W=W,
+    info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, fused=fused, step_ms=step_ms, ar_ms=ar_ms, tokens=tokens_all, K=K, W=W,
                 e2e_ms=e2e_ms_max, e2e_tokens=e2e_tokens_all, clocks=clk.summary(),
                 launches=launches, kprof=kprof, prefill_s=prefill_s, detail=detail[:24],
                 ctx_window=[ctx_before, ctx_after], weight_bytes=weight_bytes,
@@ -352,7 +408,7 @@ def run_micro(args, device):
         unit, metric = "calls/s", f"gated_lora_linear M={M} N={N} K={K} r={r}"
     else:
         cfg = synth.SPEC_VERIFY_BENCH
-        n_req, R, V = cfg["requests"], cfg["rows_per_request"], cfg["vocab"]
+        n_req, R, V = args.sv_requests or cfg["requests"], cfg["rows_per_request"], cfg["vocab"]
         p, q = synth.make_verify_logits(n_req * R, V, device, cfg["p_std"], cfg["q_noise_std"],
                                         cfg["logits_seed"])
         drafts = synth.make_drafts(q, seed=cfg["logits_seed"] + 1).view(n_req, R)
@@ -377,11 +433,14 @@ def run_micro(args, device):
         torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1) / args.steps
     gbs = nbytes / (ms / 1e3) / 1e9
-    value = (4096 if args.workload == "spec_verify" else 1) / (ms / 1e3)
+    value = (nbytes // (2 * V * 4) if args.workload == "spec_verify" else 1) / (ms / 1e3)
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "dtype": "bf16" if args.workload == "gemm" else "f32", "data": "synthetic",
-            "config": {"workload": args.workload},
+            "config": ({"workload": args.workload, "requests": nbytes // (2 * V * 4) // 16,
+                        "rows": nbytes // (2 * V * 4), "vocab": V}
+                       if args.workload == "spec_verify" else
+                       {"workload": args.workload, "shape": args.shape}),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_call": nbytes, "peak_source": pk["source"]},
@@ -439,6 +498,9 @@ def main():
                     choices=["qwen8b", "qwen8b_maxbatch", "small", "tiny", "gemm", "spec_verify"])
     ap.add_argument("--shape", default="17,4096,4096,128",
                     help="gemm microbenchmark shape M,N,K,r")
+    ap.add_argument("--sv-requests", type=int, default=0,
+                    help="spec_verify microbenchmark: requests (default: the workload's 256); "
+                         "fewer only for small profiler captures")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
     ap.add_argument("--no-fused", action="store_true",
                     help="unfused layer pipeline (separate LoRA-A GEMMs, norm, RoPE, SwiGLU)")
@@ -503,11 +565,29 @@ def main():
     kp = info["kprof"]
     g_launch, g_ms, g_bytes = kp["gemm"]
     g_gbs = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else None
-    roofline = {"bound": "hbm", "kernel": "gated_lora_linear (all GEMM launches of the step)",
-                "achieved": g_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": (g_gbs / pk["hbm_gbs"]) if g_gbs else None, "traffic": None,
-                "peak_source": pk["source"], "launches": g_launch,
-                "avg_launch_us": g_ms * 1e3 / max(1, g_launch)}
+    # the dominant kernel: the GEMM shape with the largest share of the step
+    gemms = [d for d in info["detail"] if d["cls"] == "gemm"]
+    top = max(gemms, key=lambda d: d["ms_per_step"]) if gemms else None
+    if top:
+        esz = 2 if cfg["dtype"] == "bf16" else 4
+        top_bytes = (top["n"] * top["k"] + top["n"] * top["r"] + top["m"] * top["k"] +
+                     top["m"] * top["r"]) * esz
+        achieved = top_bytes / (top["us_per_call"] * 1e-6) / 1e9
+        traffic = profiled_traffic(top)
+        roofline = {"bound": "hbm",
+                    "kernel": f"gated_lora_linear M={top['m']} N={top['n']} K={top['k']} "
+                              "(gemm_tc_kernel, the step's largest GEMM)",
+                    "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                    "algorithmic_bytes": top_bytes, "avg_launch_us": top["us_per_call"],
+                    "launches_per_step": top["calls_per_step"], "peak_source": pk["source"],
+                    "all_gemm_launches": {"achieved_GBps": g_gbs, "launches": g_launch,
+                                          "avg_launch_us": g_ms * 1e3 / max(1, g_launch)}}
+    else:
+        roofline = {"bound": "hbm", "kernel": "gated_lora_linear (SIMT)", "achieved": g_gbs,
+                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": (g_gbs / pk["hbm_gbs"]) if g_gbs else None, "traffic": None,
+                    "peak_source": pk["source"]}
     per_step_ms = info["ms"] / info["K"]
     sb = step_bytes(info)
     step_roof = {"algorithmic_bytes_per_step": sb, "achieved_GBps": sb / (per_step_ms / 1e3) / 1e9,
@@ -527,6 +607,12 @@ def main():
                    "context_window": info["ctx_window"], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (15+ GB of weights streamed per pass)"},
         "tokens_per_step": info["tokens"] / info["K"],
+        "step_latency_ms": {"median": statistics.median(info["step_ms"]),
+                            "min": min(info["step_ms"]), "max": max(info["step_ms"])},
+        "mean_accepted_a": info["tokens"] / info["K"] / info["batch"] / max(1, world) - 1,
+        "ar_only": {"value": info["batch"] / (info["ar_ms"] / 1e3), "unit": "tokens/s",
+                    "ms_per_step": info["ar_ms"],
+                    "note": "uno_ar_step on the same requests and kernels, one token per request"},
         "tpf": info["tokens"] / info["K"] / info["batch"] / 2 / max(1, world),
         "roofline": roofline, "step_roofline": step_roof, "kernel_breakdown": breakdown,
         "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": info["h2d"],

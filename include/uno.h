@@ -100,8 +100,9 @@ typedef struct uno_weights {
  *   lora_rank, lora_alpha: the LoRA scale is alpha / rank.
  *   block_B:   drafted block size B (2 <= B <= 64).
  *   max_batch: request slots; max_ctx: tokens one request may hold (prompt
- *              plus generated).  The KV pool holds max_batch * ceil((max_ctx
- *              + B + 1) / 64) pages of 64 tokens.
+ *              plus generated).  The KV pool (element type: see
+ *              uno_debug_kv) holds max_batch * ceil((max_ctx + B + 1) / 64)
+ *              pages of 64 tokens.
  *   seed:      Philox key of every uniform the sampler draws.
  *   stream:    every later call enqueues on this stream.
  * On success *out receives the context (free it with uno_destroy).
@@ -198,7 +199,11 @@ int uno_debug_read(uno_ctx *ctx, int which, void *dst_host, size_t bytes);
 
 /* Copy keys and values of positions [pos0, pos0+n) of layer `layer` of a
  * request to host buffers k_host, v_host, each [n, n_kv_heads, head_dim] in
- * the model dtype (synchronises).  Keys are stored after RoPE. */
+ * the cache's element type: fp32 for fp32 models, fp16 for bf16 models (the
+ * attention operands q, K, V and P of a bf16 model are fp16: two bytes like
+ * bf16, with three more mantissa bits; q and K are kept as fp16 hi/lo pairs,
+ * and the keys returned here are the high parts).  Synchronises.  Keys are
+ * stored after RoPE. */
 int uno_debug_kv(uno_ctx *ctx, int req_id, int layer, int pos0, int n, void *k_host,
                  void *v_host);
 

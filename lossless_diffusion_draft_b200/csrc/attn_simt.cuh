@@ -27,6 +27,7 @@ constexpr int ATT_KT = 32;       // keys per tile
 
 struct AttnParams {
   const void* qkv; int ld_qkv;   // rotated q in columns [0, H*hd)
+  const void* q_lo;              // its rounding residual rows (same layout), or null
   void* out; int ld_out;         // [M, H*hd]
   void* out_lo;                  // rounding residual rows (split GEMM input) or null
   KvLayout kv; int layer;
@@ -66,11 +67,14 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
   const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const T* qkv = reinterpret_cast<const T*>(p.qkv);
+  typedef typename KvOf<T>::type KV;   // q and the KV cache
+  const KV* qkv = reinterpret_cast<const KV*>(p.qkv);
   for (int idx = threadIdx.x; idx < nq * HD; idx += ATT_THREADS) {
     const int qi = idx / HD, d = idx % HD;
     const int tk = qi / G, g = qi % G;
-    q_s[idx] = to_f(qkv[(size_t)(row0 + tk) * p.ld_qkv + (size_t)(kvh * G + g) * HD + d]) * p.scale;
+    const size_t e = (size_t)(row0 + tk) * p.ld_qkv + (size_t)(kvh * G + g) * HD + d;
+    const float qlo = p.q_lo ? to_f(reinterpret_cast<const KV*>(p.q_lo)[e]) : 0.f;
+    q_s[idx] = (to_f(qkv[e]) + qlo) * p.scale;
   }
   float m_i[QPW], l_i[QPW], o_i[QPW][EPL];
   int qpos[QPW];
@@ -83,7 +87,7 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
     qpos[t] = (qi < nq) ? p.row_pos[row0 + qi / G] : -1;
   }
 
-  const T* pool = reinterpret_cast<const T*>(p.kv.pool);
+  const KV* pool = reinterpret_cast<const KV*>(p.kv.pool);
   for (int tile = t_begin; tile < t_end; ++tile) {
     __syncthreads();
     for (int idx = threadIdx.x; idx < ATT_KT * HD; idx += ATT_THREADS) {
@@ -95,7 +99,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
         const size_t off = p.kv.offset(p.layer, slot, kp, 0, kvh, ok);
         if (ok) {
           kval = to_f(pool[off + d]);
-          vval = to_f(pool[off + (size_t)p.kv.n_kv_heads * KV_PAGE * HD + d]);
+          if (p.kv.n_planes == 3) kval += to_f(pool[off + p.kv.plane_stride() + d]);   // K lo
+          vval = to_f(pool[off + p.kv.v_plane() * p.kv.plane_stride() + d]);
         }
       }
       k_s[j * (HD + 1) + d] = kval;

@@ -1,5 +1,6 @@
 // Paged-KV grouped-query attention with the block-causal mask on the
-// 5th-generation tensor cores (bf16 K/V and q, fp32 scores and softmax).
+// 5th-generation tensor cores (fp16 q, K, V and P; fp32 scores, softmax and
+// accumulators).
 //
 // Mask (blog page "不砸掉重来，给自回归 LLM 装一对“扩散翅膀”：Uno 的无损加速之路",
 // section Diffusion Distillation：一步蒸馏 + 块级扩散): the clean sequence is
@@ -19,7 +20,7 @@
 //   warps 0-3 (thread = query row): read the score row, softmax in the log2
 //           domain against a reference max that moves (rescaling O in TMEM)
 //           only when a tile's max exceeds it by more than 2^8, and write P
-//           (bf16) to shared memory in the MMA's swizzled layout.
+//           (fp16) to shared memory in the MMA's swizzled layout.
 // With several key splits each CTA writes (m, l, O) partials and
 // attn_merge_kernel (one CTA per query row) adds them in split order.  Every
 // wait is bounded.
@@ -33,7 +34,6 @@ namespace uno {
 constexpr int ATC_THREADS = 192;
 constexpr int ATC_QROWS = 128;
 constexpr int ATC_KT = 64;          // keys per tile = one KV page
-constexpr int ATC_STAGES = 4;
 constexpr int ATC_PAGE_PF = 64;     // page numbers a CTA fetches up front
 constexpr int ST_ATTN_TIMEOUT = 16;
 // Floats per query row of a split partial: O[HD], m, l, padded so that every
@@ -41,7 +41,8 @@ constexpr int ST_ATTN_TIMEOUT = 16;
 __host__ __device__ constexpr int atc_ws_row(int hd) { return hd + 4; }
 
 struct AttnTcParams {
-  const bf16* q; int ld_q;          // rotated q rows [M, H * HD]
+  const f16* q; int ld_q;           // rotated q rows [M, H * HD] (fp16 hi; lo rows q_lo_row below)
+  int q_lo_row;
   bf16* out; int ld_out;            // [M, H * HD]
   bf16* out_lo;                     // rounding residual rows (split GEMM input) or null
   int layer, H, Hkv, n_pages, pages_per_req;
@@ -60,7 +61,10 @@ struct AtcCfg {
   static constexpr int Q_BYTES = ATC_QROWS * HD * 2;
   static constexpr int KV_BYTES = ATC_KT * HD * 2;      // K or V of one stage
   static constexpr int P_BYTES = ATC_QROWS * ATC_KT * 2;
-  static constexpr int SMEM = Q_BYTES + ATC_STAGES * 2 * KV_BYTES + 2 * P_BYTES + 1024 + 256;
+  // stages of K hi, K lo and V: four fit beside q hi/lo and P for head_dim
+  // 64, two for 128
+  static constexpr int STAGES = HD <= 64 ? 4 : 2;
+  static constexpr int SMEM = 2 * Q_BYTES + STAGES * 3 * KV_BYTES + 2 * P_BYTES + 1024 + 256;
   static constexpr int TMEM_COLS = 256;       // 2 score tiles + the output accumulator
   static constexpr int S_COL = 0;             // score tiles at columns 0, 64
   static constexpr int O_COL = 2 * ATC_KT;    // output accumulator at 128 .. 128 + HD
@@ -82,24 +86,28 @@ __device__ __forceinline__ void attn_store_row(bf16* dst, bf16* lo, const float*
 
 template <int HD>
 __global__ void __launch_bounds__(ATC_THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, const AttnTcParams p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
+                   const AttnTcParams p) {
   using C = AtcCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                                   // NB boxes [128 rows x 64]
-  uint8_t* sK = sQ + C::Q_BYTES;                        // [STAGES] NB boxes [64 keys x 64]
-  uint8_t* sV = sK + ATC_STAGES * C::KV_BYTES;          // [STAGES] NB boxes [64 keys x 64]
-  uint8_t* sP = sV + ATC_STAGES * C::KV_BYTES;          // [2] [128 rows x 64 keys]
+  uint8_t* sQ = smem;                                   // q hi: NB boxes [128 rows x 64]
+  uint8_t* sQl = sQ + C::Q_BYTES;                       // q lo
+  uint8_t* sK = sQl + C::Q_BYTES;                       // [STAGES] K hi: NB boxes [64 keys x 64]
+  uint8_t* sKl = sK + C::STAGES * C::KV_BYTES;          // [STAGES] K lo
+  uint8_t* sV = sKl + C::STAGES * C::KV_BYTES;          // [STAGES] V
+  uint8_t* sP = sV + C::STAGES * C::KV_BYTES;           // [2] [128 rows x 64 keys]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
   uint64_t* kv_full = bars;                             // [STAGES]
-  uint64_t* kv_empty = bars + ATC_STAGES;               // [STAGES]
-  uint64_t* s_full = bars + 2 * ATC_STAGES;             // [2]
+  uint64_t* kv_empty = bars + C::STAGES;                // [STAGES]
+  uint64_t* s_full = bars + 2 * C::STAGES;              // [2]
   uint64_t* s_empty = s_full + 2;                       // [2] (4 warps)
   uint64_t* p_full = s_empty + 2;                       // [2] (4 warps)
   uint64_t* o_full = p_full + 2;                        // one phase per PV(i)
   uint64_t* drain = o_full + 1;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_full = drain + 1;                         // q hi and lo landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_ok = reinterpret_cast<volatile int*>(s_tmem + 4);   // [4]
 
@@ -114,24 +122,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   const int ntok = min(TQ, p.rows_per_req - tok0);
   const int nq = ntok * G;
   const int row0 = req * p.rows_per_req + tok0;
-  // the q rows (warps 0-3, one row per thread) and the row's position are
-  // fetched first; nothing below waits for them before the shared-memory store
-  uint4 qv[HD / 8];
+  // the position of each query row (warps 0-3, one row per thread)
   int qpos = -1;
-  if (warp < 4) {
-    const int r = threadIdx.x;
-    if (r < nq) {
-      const int tk = r / G, g = r % G;
-      const uint4* src =
-          reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + tk) * p.ld_q + (size_t)(kvh * G + g) * HD);
-#pragma unroll
-      for (int j = 0; j < HD / 8; ++j) qv[j] = src[j];
-      qpos = p.row_pos[row0 + tk];
-    } else {
-#pragma unroll
-      for (int j = 0; j < HD / 8; ++j) qv[j] = make_uint4(0, 0, 0, 0);
-    }
-  }
+  if (warp < 4 && threadIdx.x < nq) qpos = p.row_pos[row0 + threadIdx.x / G];
   const int slot = p.row_slot[row0];
   const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
   int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
@@ -144,7 +137,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   const int n = t_end - t_begin;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ATC_STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
@@ -155,6 +148,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     }
     mbar_init(o_full, 1);
     mbar_init(drain, 1);
+    mbar_init(q_full, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -164,20 +158,13 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                  "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // query rows -> shared memory, K-major 128-byte swizzle (zero rows past nq)
-  if (warp < 4) {
-    const int r = threadIdx.x;
-#pragma unroll
-    for (int j = 0; j < HD / 8; ++j) {
-      const int box = j >> 3, c = j & 7;
-      *reinterpret_cast<uint4*>(sQ + box * (ATC_QROWS * 128) + r * 128 + ((c ^ (r & 7)) << 4)) = qv[j];
-    }
-    fence_async_smem();
-  }
   // the split's page numbers, fetched in one round while the q rows load
   __shared__ int s_pages[ATC_PAGE_PF];
   if (warp == 4) {
-    if (lane == 0) prefetch_map(&kvmap);
+    if (lane == 0) {
+      prefetch_map(&kvmap);
+      prefetch_map(&qmap);
+    }
     for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32)
       s_pages[i] = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
   }
@@ -189,62 +176,85 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < n && !*s_abort; ++i) {
-        const int stage = i % ATC_STAGES;
-        const uint32_t phase = (uint32_t)(i / ATC_STAGES) & 1;
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
-        mbar_expect_tx(&kv_full[stage], 2 * C::KV_BYTES);
-        const int page = i < ATC_PAGE_PF ? s_pages[i]
-                                         : p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
-        const int rk = (((p.layer * p.n_pages + page) * 2 + 0) * p.Hkv + kvh) * KV_PAGE;
-        const int rv = (((p.layer * p.n_pages + page) * 2 + 1) * p.Hkv + kvh) * KV_PAGE;
+      // q hi and lo tiles: rows (token, head of the group) as a 3-D box of the
+      // [rows, H, HD] q buffer; rows past the request are masked, not stored
+      if (n > 0) {
+        mbar_expect_tx(q_full, 2 * C::Q_BYTES);
 #pragma unroll
         for (int b = 0; b < C::NB; ++b) {
-          tma_load_2d(sK + stage * C::KV_BYTES + b * (ATC_KT * 128), &kvmap, &kv_full[stage], b * 64, rk);
-          tma_load_2d(sV + stage * C::KV_BYTES + b * (ATC_KT * 128), &kvmap, &kv_full[stage], b * 64, rv);
+          tma_load_3d(sQ + b * (ATC_QROWS * 128), &qmap, q_full, b * 64, kvh * G, row0);
+          tma_load_3d(sQl + b * (ATC_QROWS * 128), &qmap, q_full, b * 64, kvh * G, p.q_lo_row + row0);
+        }
+      }
+      int issued = 0;
+      for (int i = 0; i < n && !*s_abort; ++i) {
+        const int stage = i % C::STAGES;
+        const uint32_t phase = (uint32_t)(i / C::STAGES) & 1;
+        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
+        mbar_expect_tx(&kv_full[stage], 3 * C::KV_BYTES);
+        const int page = i < ATC_PAGE_PF ? s_pages[i]
+                                         : p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+        // pool rows of the page's K hi, K lo and V planes for this kv head
+        const int rk = (((p.layer * p.n_pages + page) * 3 + 0) * p.Hkv + kvh) * KV_PAGE;
+        const int rkl = rk + p.Hkv * KV_PAGE;
+        const int rv = rkl + p.Hkv * KV_PAGE;
+#pragma unroll
+        for (int b = 0; b < C::NB; ++b) {
+          const int o = stage * C::KV_BYTES + b * (ATC_KT * 128);
+          tma_load_2d(sK + o, &kvmap, &kv_full[stage], b * 64, rk);
+          tma_load_2d(sKl + o, &kvmap, &kv_full[stage], b * 64, rkl);
+          tma_load_2d(sV + o, &kvmap, &kv_full[stage], b * 64, rv);
         }
         ++issued;
       }
       if (*s_abort) {
-        for (int i = max(0, issued - ATC_STAGES); i < issued; ++i)
-          mbar_wait(&kv_full[i % ATC_STAGES], (uint32_t)(i / ATC_STAGES) & 1);
+        for (int i = max(0, issued - C::STAGES); i < issued; ++i)
+          mbar_wait(&kv_full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1);
       }
+      if (n > 0) mbar_wait(q_full, 0);   // no copy in flight past this point
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(ATC_QROWS, ATC_KT);
-      constexpr uint32_t idesc_pv = idesc_bf16(ATC_QROWS, HD) | (1u << 16);   // B MN-major
+      constexpr uint32_t idesc_qk = idesc_f16(ATC_QROWS, ATC_KT);
+      constexpr uint32_t idesc_pv = idesc_f16(ATC_QROWS, HD) | (1u << 16);   // B MN-major
       bool issued_any = false;
+      bool ok = mbar_wait(q_full, 0);
       auto qk = [&](int i) -> bool {
-        const int stage = i % ATC_STAGES, sb = i & 1;
-        if (!mbar_wait(&kv_full[stage], (uint32_t)(i / ATC_STAGES) & 1)) return false;
+        const int stage = i % C::STAGES, sb = i & 1;
+        if (!mbar_wait(&kv_full[stage], (uint32_t)(i / C::STAGES) & 1)) return false;
         if (!mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t d = tmem + C::S_COL + sb * ATC_KT;
+        // S = q_hi K_hi^T + q_lo K_hi^T + q_hi K_lo^T (the lo x lo term is below
+        // fp32 rounding of S)
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
           const int b = ks >> 2, kk = ks & 3;
-          mma_bf16(d, sdesc_k128(smem_u32(sQ + b * (ATC_QROWS * 128)) + kk * 32),
-                   sdesc_k128(smem_u32(sK + stage * C::KV_BYTES + b * (ATC_KT * 128)) + kk * 32),
-                   idesc_qk, ks > 0 ? 1u : 0u);
+          const int o = stage * C::KV_BYTES + b * (ATC_KT * 128);
+          const uint64_t kh = sdesc_k128(smem_u32(sK + o) + kk * 32);
+          const uint64_t kl = sdesc_k128(smem_u32(sKl + o) + kk * 32);
+          const uint64_t qh = sdesc_k128(smem_u32(sQ + b * (ATC_QROWS * 128)) + kk * 32);
+          const uint64_t ql = sdesc_k128(smem_u32(sQl + b * (ATC_QROWS * 128)) + kk * 32);
+          mma_f16(d, qh, kh, idesc_qk, ks > 0 ? 1u : 0u);
+          mma_f16(d, ql, kh, idesc_qk, 1u);
+          mma_f16(d, qh, kl, idesc_qk, 1u);
         }
         issued_any = true;
         mma_commit(&s_full[sb]);
         return true;
       };
-      bool ok = qk(0);
+      ok = ok && qk(0);
       for (int i = 0; i < n && ok; ++i) {
         if (i + 1 < n && !qk(i + 1)) { ok = false; break; }
-        const int stage = i % ATC_STAGES, b2 = i & 1;
+        const int stage = i % C::STAGES, b2 = i & 1;
         // P(i) written (and O rescaled, if the softmax warps moved the max)
         if (!mbar_wait(&p_full[b2], (uint32_t)(i >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         // O accumulates in TMEM across tiles
 #pragma unroll
         for (int ks = 0; ks < ATC_KT / 16; ++ks)
-          mma_bf16(tmem + C::O_COL, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
+          mma_f16(tmem + C::O_COL, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
                    sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
                    idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         mma_commit(o_full);            // phase i completes when PV(i) has
@@ -319,7 +329,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         m = m_new;
       }
       // P = 2^(s * scale - m) <= 2^RESCALE_LOG2 by the hardware ex2 (P is
-      // rounded to bf16 next, far coarser than its error); a row with no key
+      // rounded to fp16 next, far coarser than its error); a row with no key
       // yet (m = -inf) has s = -inf everywhere and gets P = 0
       const float nm = (m == -INFINITY) ? 0.f : -m;
       float psum = 0.f;
@@ -328,7 +338,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       for (int j = 0; j < ATC_KT; j += 2) {
         const float a = fast_exp2(fmaf(s[j], p.scale_log2, nm));
         const float b = fast_exp2(fmaf(s[j + 1], p.scale_log2, nm));
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+        const __half2 h2 = __floats2half2_rn(a, b);
         psum += __low2float(h2) + __high2float(h2);    // the P the MMA will use
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,12 +14,22 @@ namespace uno {
 // is fp32.
 // ---------------------------------------------------------------------------
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(f16 x) { return __half2float(x); }
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ f16 from_f<f16>(float x) { return __float2half_rn(x); }
+
+// Element type of the attention operands - the rotated q rows, the paged KV
+// cache and the probabilities P - for a model of element type T: fp16 for
+// bf16 models (the same two bytes with three more mantissa bits; q, K, V and
+// P are rounded once each), T otherwise.
+template <typename T> struct KvOf { typedef T type; };
+template <> struct KvOf<bf16> { typedef f16 type; };
 
 // 16-byte vector load of VEC elements converted to fp32.
 template <typename T> struct Vec16;

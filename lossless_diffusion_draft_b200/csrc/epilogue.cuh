@@ -26,7 +26,7 @@
 // gates it per row.
 //
 // One CTA takes one 128-column tile of the output (two for SwiGLU) and
-// EPI_RG rows; a thread owns one column.  Every load a thread needs is issued before the first use,
+// EPI_RG rows; EPI_NQ threads share a column, each with a few of the rows.  Every load a thread needs is issued before the first use,
 // so a CTA costs about one memory round trip.
 #pragma once
 
@@ -62,7 +62,7 @@ struct EpiArgs {
   int n_ss; float d_model, eps;
   int lora; LoraEpi lr;
   // epi_qkv
-  bf16* q_out; int ld_q;
+  f16* q_out; int ld_q;              // rotated q rows, fp16 hi (lo rows lo_off below)
   int H, Hkv, hd;
   const int32_t* row_pos; const int32_t* row_slot;
   const float* cos_t; const float* sin_t; int max_pos;
@@ -78,10 +78,16 @@ struct EpiArgs {
   int32_t* status;
 };
 
-// Parts of tile column col of output tile nt, rows m0 .. m0 + nrows.
-// part_issue loads the first C contributors (issued before any use);
-// part_add adds them in CTA order, the first contributor's part first, then
-// reads any further contributors C at a time.
+// Thread layout of every epilogue CTA: EPI_NQ row slots x 128 columns.
+// Thread t owns column t % 128 and, in slot q = t / 128, the rows
+// j = q + EPI_NQ * s (s < EPI_RPT) of the CTA's EPI_RG rows.  With several
+// warps per scheduler and a few rows per thread, the loads of a CTA stay in
+// flight together and the arithmetic hides its latency.
+constexpr int EPI_NQ = 2;
+constexpr int EPI_RPT = (EPI_RG + EPI_NQ - 1) / EPI_NQ;
+constexpr int EPI_THREADS = EPI_NQ * TC_BM;
+constexpr int EPI_KQ = EPI_R / EPI_NQ;    // rank columns of a thread's share of the LoRA-B dot
+
 // Row groups never straddle an m-tile of the GEMM (the part slots are per
 // m-tile): blockIdx.y = m-tile * groups_per_tile + group.  Returns false for
 // a group past the rows (whole CTA).
@@ -97,73 +103,76 @@ __device__ __forceinline__ bool row_group(const EpiArgs& a, int* m0, int* nrows)
   return *nrows > 0;
 }
 
+// Parts of column col of output tile nt for the thread's rows (m0 + q + NQ s).
+// part_issue loads the first C contributors (issued before any use);
+// part_add adds them in CTA order, the first contributor's part first, then
+// reads any further contributors C at a time.
 template <int C>
 struct PartLoad {
-  float x[C][EPI_RG];
+  float x[C][EPI_RPT];
   int first, last;
   const float* base; size_t slot;
 };
 template <int C>
 __device__ __forceinline__ void part_issue(const PartView& v, int nt, int m0, int nrows, int col,
-                                           PartLoad<C>& L) {
+                                           int q, PartLoad<C>& L) {
   const int mt = m0 / v.NT;
   const int t = nt * v.m_tiles + mt;
   L.first = sk_owner(t * v.KBt, v.units, v.grid);
   L.last = sk_owner(t * v.KBt + v.KBt - 1, v.units, v.grid);
   L.slot = (size_t)v.NT * TC_BM;
-  L.base = v.ws + ((size_t)t * v.NT + (m0 - mt * v.NT)) * TC_BM + col;
+  L.base = v.ws + ((size_t)t * v.NT + (m0 - mt * v.NT) + q) * TC_BM + col;
 #pragma unroll
   for (int c = 0; c < C; ++c) {
     const int i = L.first + c;
 #pragma unroll
-    for (int j = 0; j < EPI_RG; ++j)
-      L.x[c][j] = (i <= L.last && j < nrows) ? __ldcg(L.base + (size_t)i * L.slot + (size_t)j * TC_BM)
-                                              : 0.f;
+    for (int s = 0; s < EPI_RPT; ++s)
+      L.x[c][s] = (i <= L.last && q + EPI_NQ * s < nrows)
+                      ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(EPI_NQ * s) * TC_BM) : 0.f;
   }
 }
 template <int C>
-__device__ __forceinline__ void part_add(PartLoad<C>& L, int nrows, float (&acc)[EPI_RG]) {
+__device__ __forceinline__ void part_add(PartLoad<C>& L, int nrows, int q, float (&acc)[EPI_RPT]) {
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) acc[j] = 0.f;
+  for (int s = 0; s < EPI_RPT; ++s) acc[s] = 0.f;
   for (int i0 = L.first;; i0 += C) {
 #pragma unroll
     for (int c = 0; c < C; ++c)
 #pragma unroll
-      for (int j = 0; j < EPI_RG; ++j) acc[j] += L.x[c][j];
+      for (int s = 0; s < EPI_RPT; ++s) acc[s] += L.x[c][s];
     if (i0 + C > L.last) break;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       const int i = i0 + C + c;
 #pragma unroll
-      for (int j = 0; j < EPI_RG; ++j)
-        L.x[c][j] = (i <= L.last && j < nrows)
-                        ? __ldcg(L.base + (size_t)i * L.slot + (size_t)j * TC_BM) : 0.f;
+      for (int s = 0; s < EPI_RPT; ++s)
+        L.x[c][s] = (i <= L.last && q + EPI_NQ * s < nrows)
+                        ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(EPI_NQ * s) * TC_BM) : 0.f;
     }
   }
 }
 
-// Sums of squares of rows m0 .. m0 + nrows (all tiles): one load per
-// (row, tile) by threads 0..127, all issued together.
+// Sums of squares of rows m0 .. m0 + nrows (all n_ss tiles of each): the
+// (row, tile) values are spread over the CTA's threads, all loads issued
+// together.
 constexpr int EPI_MAX_SS = 64;        // d_model <= 64 * 128
-__device__ __forceinline__ void ss_issue(const EpiArgs& a, int m0, int nrows, float (&v)[4]) {
-  const int n = nrows * a.n_ss;
+constexpr int EPI_SS_PT = (EPI_RG * EPI_MAX_SS + EPI_THREADS - 1) / EPI_THREADS;
+struct SsLoad { float v[EPI_SS_PT]; };
+__device__ __forceinline__ void ss_issue(const EpiArgs& a, int m0, int nrows, SsLoad& L) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int e = threadIdx.x + k * TC_BM;
-    v[k] = (a.ss && threadIdx.x < TC_BM && e < n) ? __ldcg(a.ss + (size_t)m0 * a.n_ss + e) : 0.f;
+  for (int k = 0; k < EPI_SS_PT; ++k) {
+    const int e = threadIdx.x + k * EPI_THREADS;
+    L.v[k] = (a.ss && e < nrows * a.n_ss) ? __ldcg(a.ss + (size_t)m0 * a.n_ss + e) : 0.f;
   }
 }
 // 1 / sqrt(mean(x^2) + eps) per row into s_inv (tiles added in tile order);
-// 1 without a norm.  Call with the values of ss_issue; syncs the CTA.
-__device__ __forceinline__ void ss_finish(const EpiArgs& a, int nrows, const float (&v)[4],
-                                          float* s_ss, float* s_inv) {
-  const int n = nrows * a.n_ss;
-  if (threadIdx.x < TC_BM) {
+// 1 without a norm.  Syncs the CTA (twice).
+__device__ __forceinline__ void ss_finish(const EpiArgs& a, int nrows, const SsLoad& L, float* s_ss,
+                                          float* s_inv) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int e = threadIdx.x + k * TC_BM;
-      if (e < n) s_ss[e] = v[k];
-    }
+  for (int k = 0; k < EPI_SS_PT; ++k) {
+    const int e = threadIdx.x + k * EPI_THREADS;
+    if (e < nrows * a.n_ss) s_ss[e] = L.v[k];
   }
   __syncthreads();
   const int j = threadIdx.x;
@@ -187,274 +196,324 @@ __device__ __forceinline__ int lora_seg(const LoraEpi& lr, int n) {
   return s;
 }
 
-// One B row of the adapter (EPI_R bf16), loaded whole.
-struct BRow { uint4 b[EPI_R / 8]; };
-__device__ __forceinline__ void brow_issue(const EpiArgs& a, int s, int nb, BRow& B) {
-  const uint4* src = reinterpret_cast<const uint4*>(a.lr.Bl[s] + (size_t)nb * EPI_R);
+// The thread's quarter of one adapter row: B[nb][q*EPI_KQ .. +EPI_KQ].
+struct BPart { uint4 b[EPI_KQ / 8]; };
+__device__ __forceinline__ void bpart_issue(const EpiArgs& a, int s, int nb, int q, BPart& B) {
+  const uint4* src = reinterpret_cast<const uint4*>(a.lr.Bl[s] + (size_t)nb * EPI_R + q * EPI_KQ);
 #pragma unroll
-  for (int e = 0; e < EPI_R / 8; ++e) B.b[e] = __ldg(src + e);
+  for (int e = 0; e < EPI_KQ / 8; ++e) B.b[e] = __ldg(src + e);
 }
 
-// acc[j] += gate[j] * sum_k sU[j][k] B[k].
-__device__ __forceinline__ void lora_dot(const BRow& B, const float* sU, const float (&gate)[EPI_RG],
-                                         float (&acc)[EPI_RG]) {
-  float dot[EPI_RG];
+// LoRA-B for column col: every thread forms the partial dot of its rank
+// quarter for all rows (sU[j][k] B[k]), the partials go through shared
+// memory and each thread adds the NQ quarters of its own rows in quarter
+// order: acc[s] += gate[s] * dot.  Syncs the CTA.
+__device__ __forceinline__ void lora_apply(const BPart& B, const float* sU, float* sDot, int col,
+                                           int q, int nrows, const float (&gate)[EPI_RPT],
+                                           float (&acc)[EPI_RPT]) {
+  float bf[EPI_KQ];
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) dot[j] = 0.f;
-#pragma unroll
-  for (int e = 0; e < EPI_R / 8; ++e) {
+  for (int e = 0; e < EPI_KQ / 8; ++e) {
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&B.b[e]);
-    float bf[8];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      bf[2 * h] = __low2float(b2[h]);
-      bf[2 * h + 1] = __high2float(b2[h]);
-    }
-#pragma unroll
-    for (int j = 0; j < EPI_RG; ++j) {
-      const float4* u4 = reinterpret_cast<const float4*>(sU + j * EPI_R + e * 8);
-      const float4 x0 = u4[0], x1 = u4[1];
-      dot[j] += x0.x * bf[0] + x0.y * bf[1] + x0.z * bf[2] + x0.w * bf[3] + x1.x * bf[4] +
-                x1.y * bf[5] + x1.z * bf[6] + x1.w * bf[7];
+      bf[8 * e + 2 * h] = __low2float(b2[h]);
+      bf[8 * e + 2 * h + 1] = __high2float(b2[h]);
     }
   }
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) acc[j] += gate[j] * dot[j];
+  for (int j = 0; j < EPI_RG; ++j) {
+    if (j >= nrows) break;
+    const float4* u4 = reinterpret_cast<const float4*>(sU + j * EPI_R + q * EPI_KQ);
+    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < EPI_KQ / 4; k += 2) {
+      const float4 x0 = u4[k], x1 = u4[k + 1];
+      d0 += x0.x * bf[4 * k] + x0.y * bf[4 * k + 1] + x0.z * bf[4 * k + 2] + x0.w * bf[4 * k + 3];
+      d1 += x1.x * bf[4 * k + 4] + x1.y * bf[4 * k + 5] + x1.z * bf[4 * k + 6] + x1.w * bf[4 * k + 7];
+    }
+    sDot[(q * EPI_RG + j) * TC_BM + col] = d0 + d1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    if (j < nrows) {
+      float t = 0.f;
+#pragma unroll
+      for (int qq = 0; qq < EPI_NQ; ++qq) t += sDot[(qq * EPI_RG + j) * TC_BM + col];
+      acc[s] += gate[s] * t;
+    }
+  }
 }
 
-// The U tile of segment s (column col of its EPI_R rank columns): loads, then
-// its sums into sU[EPI_RG][EPI_R].  The caller syncs before sU is read.
+// The U tile of segment s, column col, the thread's rows: loads, then the
+// sums into sU[EPI_RG][EPI_R].  The caller syncs before sU is read.
 template <int C>
-__device__ __forceinline__ void u_issue(const EpiArgs& a, int s, int m0, int nrows, int col,
+__device__ __forceinline__ void u_issue(const EpiArgs& a, int seg, int m0, int nrows, int col, int q,
                                         PartLoad<C>& L) {
-  part_issue(a.pv, a.lr.u_tile0 + s, m0, nrows, col, L);
+  part_issue(a.pv, a.lr.u_tile0 + seg, m0, nrows, col, q, L);
 }
 template <int C>
-__device__ __forceinline__ void u_store(PartLoad<C>& L, int nrows, int col, float* sU) {
-  float u[EPI_RG];
-  part_add(L, nrows, u);
+__device__ __forceinline__ void u_store(PartLoad<C>& L, int nrows, int col, int q, float* sU) {
+  float u[EPI_RPT];
+  part_add(L, nrows, q, u);
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) sU[j * EPI_R + col] = u[j];
+  for (int s = 0; s < EPI_RPT; ++s)
+    if (q + EPI_NQ * s < nrows) sU[(q + EPI_NQ * s) * EPI_R + col] = u[s];
 }
 
-// Row gates of the CTA's rows (0 past M).
-__device__ __forceinline__ void gate_issue(const EpiArgs& a, int m0, int nrows, float (&g)[EPI_RG]) {
+// Row gates of the thread's rows (0 past M).
+__device__ __forceinline__ void gate_issue(const EpiArgs& a, int m0, int nrows, int q,
+                                           float (&g)[EPI_RPT]) {
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) g[j] = j < nrows ? __ldg(a.lr.row_gate + m0 + j) : 0.f;
+  for (int s = 0; s < EPI_RPT; ++s)
+    g[s] = q + EPI_NQ * s < nrows ? __ldg(a.lr.row_gate + m0 + q + EPI_NQ * s) : 0.f;
 }
 
 // ---------------------------------------------------------------------------
-// q|k|v: grid ((H + 2 Hkv) hd / 128, ceil(M / EPI_RG)), 128 threads.
+// q|k|v: grid ((H + 2 Hkv) hd / 128, row groups), EPI_THREADS threads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(TC_BM) epi_qkv_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(EPI_THREADS) epi_qkv_kernel(const EpiArgs a) {
   constexpr int C = 4;
   __shared__ float s_inv[EPI_RG];
   __shared__ float s_ss[EPI_RG * EPI_MAX_SS];
   __shared__ __align__(16) float sU[EPI_RG * EPI_R];
+  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
   __shared__ float sY[EPI_RG][TC_BM];
   pdl_trigger();
   pdl_wait();
   const int nt = blockIdx.x;
   int m0, nrows;
   if (!row_group(a, &m0, &nrows)) return;
-  const int i = threadIdx.x;
-  const int n = nt * TC_BM + i;
+  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  const int n = nt * TC_BM + col;
   const int qcols = a.H * a.hd, kcols = a.Hkv * a.hd;
   const int half = a.hd / 2;
   const int hi = n % a.hd;                 // index inside the head
   const bool rot = n < qcols + kcols;      // q and k are rotated, v is not
+  const bool kv_tile = n >= qcols;
   const int ci = hi < half ? hi : hi - half;
 
   // ---- every global load first
-  const bool kv_tile = n >= qcols;
-  int pos[EPI_RG], slot[EPI_RG];
+  int pos[EPI_RPT], slot[EPI_RPT];
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) {
-    pos[j] = j < nrows ? a.row_pos[m0 + j] : 0;
-    slot[j] = (j < nrows && kv_tile) ? a.row_slot[m0 + j] : 0;
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    pos[s] = j < nrows ? a.row_pos[m0 + j] : 0;
+    slot[s] = (j < nrows && kv_tile) ? a.row_slot[m0 + j] : 0;
   }
-  float ssv[4];
+  SsLoad ssv;
   ss_issue(a, m0, nrows, ssv);
-  const int s = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
+  const int seg = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
   PartLoad<C> LU, LP;
-  BRow B;
-  float gate[EPI_RG];
+  BPart B;
+  float gate[EPI_RPT];
   if (a.lora) {
-    u_issue(a, s, m0, nrows, i, LU);
-    brow_issue(a, s, n - a.lr.seg_n0[s], B);
-    gate_issue(a, m0, nrows, gate);
+    u_issue(a, seg, m0, nrows, col, q, LU);
+    bpart_issue(a, seg, n - a.lr.seg_n0[seg], q, B);
+    gate_issue(a, m0, nrows, q, gate);
   }
-  part_issue(a.pv, nt, m0, nrows, i, LP);
+  part_issue(a.pv, nt, m0, nrows, col, q, LP);
   // second round, addressed by the rows' positions and slots: RoPE table
   // entries and the KV pages
-  float cs[EPI_RG], sn[EPI_RG];
-  int page[EPI_RG], pok[EPI_RG];
+  float cs[EPI_RPT], sn[EPI_RPT];
+  int page[EPI_RPT], pok[EPI_RPT];
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) {
-    const int pc = (pos[j] >= 0 && pos[j] < a.max_pos) ? pos[j] : 0;
-    cs[j] = rot ? a.cos_t[(size_t)pc * half + ci] : 0.f;
-    sn[j] = rot ? a.sin_t[(size_t)pc * half + ci] : 0.f;
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    const int pc = (pos[s] >= 0 && pos[s] < a.max_pos) ? pos[s] : 0;
+    cs[s] = rot ? a.cos_t[(size_t)pc * half + ci] : 0.f;
+    sn[s] = rot ? a.sin_t[(size_t)pc * half + ci] : 0.f;
     int ok = 0;
-    page[j] = (j < nrows && kv_tile) ? a.kv.page_of(slot[j], pos[j], ok) : 0;
-    pok[j] = ok;
+    page[s] = (j < nrows && kv_tile) ? a.kv.page_of(slot[s], pos[s], ok) : 0;
+    pok[s] = ok;
   }
 
   // ---- then the arithmetic
-  if (a.lora) u_store(LU, nrows, i, sU);
+  if (a.lora) u_store(LU, nrows, col, q, sU);
   ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
-  float acc[EPI_RG];
-  part_add(LP, nrows, acc);
-  if (a.lora) lora_dot(B, sU, gate, acc);
+  float acc[EPI_RPT];
+  part_add(LP, nrows, q, acc);
+  if (a.lora) lora_apply(B, sU, sDot, col, q, nrows, gate, acc);
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) sY[j][i] = acc[j] * s_inv[j];
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    if (j < nrows) sY[j][col] = acc[s] * s_inv[j];
+  }
   __syncthreads();
 
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) {
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
     if (j >= nrows) continue;
     const int m = m0 + j;
-    const bool ok_pos = pos[j] >= 0 && pos[j] < a.max_pos;
-    float y = sY[j][i];
+    const bool ok_pos = pos[s] >= 0 && pos[s] < a.max_pos;
+    float y = sY[j][col];
     // rotate-half: (x1, x2) -> (x1 c - x2 s, x2 c + x1 s)
-    if (rot) y = hi < half ? sY[j][i] * cs[j] - sY[j][i + half] * sn[j]
-                           : sY[j][i] * cs[j] + sY[j][i - half] * sn[j];
+    if (rot) y = hi < half ? sY[j][col] * cs[s] - sY[j][col + half] * sn[s]
+                           : sY[j][col] * cs[s] + sY[j][col - half] * sn[s];
     if (n < qcols) {
-      a.q_out[(size_t)m * a.ld_q + n] = from_f<bf16>(y);
+      // q as an fp16 hi/lo pair (lo rows lo_off below): the attention adds
+      // q_hi K + q_lo K
+      const f16 qh = from_f<f16>(y);
+      a.q_out[(size_t)m * a.ld_q + n] = qh;
+      a.q_out[(size_t)(a.lo_off + m) * a.ld_q + n] = from_f<f16>(y - to_f(qh));
     } else {
       const bool is_k = n < qcols + kcols;
       const int head = (n - (is_k ? qcols : qcols + kcols)) / a.hd;
-      const size_t off = a.kv.offset_in_page(a.layer, page[j], pos[j], is_k ? 0 : 1, head);
-      if (pok[j] && ok_pos) reinterpret_cast<bf16*>(a.kv.pool)[off + hi] = from_f<bf16>(y);
-      else if (hi == 0 && is_k) raise_status(a.status, ST_POS_OVERFLOW);
+      const size_t off =
+          a.kv.offset_in_page(a.layer, page[s], pos[s], is_k ? 0 : a.kv.v_plane(), head) + hi;
+      if (pok[s] && ok_pos) {
+        f16* pool = reinterpret_cast<f16*>(a.kv.pool);
+        const f16 yh = from_f<f16>(y);
+        pool[off] = yh;
+        if (is_k) pool[off + a.kv.plane_stride()] = from_f<f16>(y - to_f(yh));   // K lo plane
+      } else if (hi == 0 && is_k) {
+        raise_status(a.status, ST_POS_OVERFLOW);
+      }
     }
   }
 }
 
 // g * x rows for the next GEMM (hi/lo) and the tile's sums of squares of x.
-__device__ __forceinline__ void next_input(const EpiArgs& a, int nt, int m0, int nrows, float g,
-                                           const float (&xv)[EPI_RG]) {
-  __shared__ float red[TC_BM / 32][EPI_RG];
-  const int i = threadIdx.x, n = nt * TC_BM + i;
+__device__ __forceinline__ void next_input(const EpiArgs& a, int nt, int m0, int nrows, int col,
+                                           int q, float g, const float (&xv)[EPI_RPT]) {
+  __shared__ float red[EPI_THREADS / 32][EPI_RPT];
+  const int n = nt * TC_BM + col;
   bf16* lo = a.lo_off ? a.xn + (size_t)a.lo_off * a.ld_xn : nullptr;
-  float sq[EPI_RG];
+  float sq[EPI_RPT];
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) {
-    sq[j] = xv[j] * xv[j];
-    if (j < nrows) store_split<bf16>(a.xn, lo, (size_t)(m0 + j) * a.ld_xn + n, g * xv[j]);
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    sq[s] = xv[s] * xv[s];
+    if (j < nrows) store_split<bf16>(a.xn, lo, (size_t)(m0 + j) * a.ld_xn + n, g * xv[s]);
   }
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) sq[j] = warp_sum(sq[j]);
-  if ((i & 31) == 0)
+  for (int s = 0; s < EPI_RPT; ++s) sq[s] = warp_sum(sq[s]);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0)
 #pragma unroll
-    for (int j = 0; j < EPI_RG; ++j) red[i >> 5][j] = sq[j];
+    for (int s = 0; s < EPI_RPT; ++s) red[w][s] = sq[s];
   __syncthreads();
-  if (i < nrows) {
+  // row j = qq + NQ s lives in the 4 warps of slot qq
+  const int j = threadIdx.x;
+  if (j < nrows) {
+    const int qq = j % EPI_NQ, s = j / EPI_NQ;
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < TC_BM / 32; ++w) t += red[w][i];
-    a.ss_out[(size_t)(m0 + i) * (a.d / TC_BM) + nt] = t;
+    for (int k = 0; k < TC_BM / 32; ++k) t += red[qq * (TC_BM / 32) + k][s];
+    a.ss_out[(size_t)(m0 + j) * (a.d / TC_BM) + nt] = t;
   }
 }
 
 // ---------------------------------------------------------------------------
-// o / down (and, with prep = 1, the layer-0 input): grid (d / 128,
-// ceil(M / EPI_RG)), 128 threads.  x += y; then the next GEMM's input.
+// o / down (and, with prep = 1, the layer-0 input): grid (d / 128, row
+// groups), EPI_THREADS threads.  x += y; then the next GEMM's input.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(TC_BM) epi_resid_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(EPI_THREADS) epi_resid_kernel(const EpiArgs a) {
   constexpr int C = 6;
   __shared__ __align__(16) float sU[EPI_RG * EPI_R];
+  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
   pdl_trigger();
   pdl_wait();
   const int nt = blockIdx.x;
   int m0, nrows;
   if (!row_group(a, &m0, &nrows)) return;
-  const int i = threadIdx.x;
-  const int n = nt * TC_BM + i;
+  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  const int n = nt * TC_BM + col;
 
   // ---- every global load first
-  float xv[EPI_RG];
+  float xv[EPI_RPT];
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) xv[j] = j < nrows ? a.x[(size_t)(m0 + j) * a.d + n] : 0.f;
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    xv[s] = j < nrows ? a.x[(size_t)(m0 + j) * a.d + n] : 0.f;
+  }
   const float g = a.g_next ? to_f(a.g_next[n]) : 0.f;
   if (!a.prep) {
     PartLoad<C> LU, LP;
-    BRow B;
-    float gate[EPI_RG];
+    BPart B;
+    float gate[EPI_RPT];
     if (a.lora) {
-      u_issue(a, 0, m0, nrows, i, LU);
-      brow_issue(a, 0, n, B);
-      gate_issue(a, m0, nrows, gate);
+      u_issue(a, 0, m0, nrows, col, q, LU);
+      bpart_issue(a, 0, n, q, B);
+      gate_issue(a, m0, nrows, q, gate);
     }
-    part_issue(a.pv, nt, m0, nrows, i, LP);
+    part_issue(a.pv, nt, m0, nrows, col, q, LP);
     // ---- then the arithmetic
-    float acc[EPI_RG];
+    float acc[EPI_RPT];
     if (a.lora) {
-      u_store(LU, nrows, i, sU);
+      u_store(LU, nrows, col, q, sU);
       __syncthreads();
     }
-    part_add(LP, nrows, acc);
-    if (a.lora) lora_dot(B, sU, gate, acc);
+    part_add(LP, nrows, q, acc);
+    if (a.lora) lora_apply(B, sU, sDot, col, q, nrows, gate, acc);
 #pragma unroll
-    for (int j = 0; j < EPI_RG; ++j) {
-      xv[j] += acc[j];
-      if (j < nrows) a.x[(size_t)(m0 + j) * a.d + n] = xv[j];
+    for (int s = 0; s < EPI_RPT; ++s) {
+      const int j = q + EPI_NQ * s;
+      xv[s] += acc[s];
+      if (j < nrows) a.x[(size_t)(m0 + j) * a.d + n] = xv[s];
     }
   }
-  if (a.g_next) next_input(a, nt, m0, nrows, g, xv);
+  if (a.g_next) next_input(a, nt, m0, nrows, col, q, g, xv);
 }
 
 // ---------------------------------------------------------------------------
-// gate|up -> silu(gate) * up: grid (F / 128, ceil(M / EPI_RG)), 256 threads:
-// threads 0..127 take the gate tile, 128..255 the up tile of the same
-// features, so each thread holds one tile's loads.
+// gate|up -> silu(gate) * up: grid (F / 128, row groups), EPI_THREADS
+// threads; each thread takes the gate and the up column of one feature.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(2 * TC_BM) epi_swiglu_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(EPI_THREADS) epi_swiglu_kernel(const EpiArgs a) {
   constexpr int C = 4;
   __shared__ float s_inv[EPI_RG];
   __shared__ float s_ss[EPI_RG * EPI_MAX_SS];
   __shared__ __align__(16) float sU[2][EPI_RG * EPI_R];
-  __shared__ float sUp[EPI_RG][TC_BM];
+  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
   pdl_trigger();
   pdl_wait();
   const int ft = blockIdx.x;
   int m0, nrows;
   if (!row_group(a, &m0, &nrows)) return;
-  const int half = threadIdx.x / TC_BM;      // 0: gate, 1: up
-  const int i = threadIdx.x % TC_BM;
-  const int f = ft * TC_BM + i;
-  const int tile = half ? a.F / TC_BM + ft : ft;
+  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  const int f = ft * TC_BM + col;
+  const int ut = a.F / TC_BM + ft;         // the up tile of the same features
 
   // ---- every global load first
-  float ssv[4];
+  SsLoad ssv;
   ss_issue(a, m0, nrows, ssv);
-  PartLoad<C> LP, LU;
-  BRow B;
-  float gate[EPI_RG];
-  part_issue(a.pv, tile, m0, nrows, i, LP);
+  PartLoad<C> LG, LUp, L0, L1;
+  BPart B0, B1;
+  float gate[EPI_RPT];
+  part_issue(a.pv, ft, m0, nrows, col, q, LG);
+  part_issue(a.pv, ut, m0, nrows, col, q, LUp);
   if (a.lora) {
-    u_issue(a, half, m0, nrows, i, LU);
-    brow_issue(a, half, f, B);
-    gate_issue(a, m0, nrows, gate);
+    u_issue(a, 0, m0, nrows, col, q, L0);
+    u_issue(a, 1, m0, nrows, col, q, L1);
+    bpart_issue(a, 0, f, q, B0);
+    bpart_issue(a, 1, f, q, B1);
+    gate_issue(a, m0, nrows, q, gate);
   }
   // ---- then the arithmetic
-  if (a.lora) u_store(LU, nrows, i, sU[half]);
-  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
-  float v[EPI_RG];
-  part_add(LP, nrows, v);
-  if (a.lora) lora_dot(B, sU[half], gate, v);
-  if (half) {
-#pragma unroll
-    for (int j = 0; j < EPI_RG; ++j) sUp[j][i] = v[j];
+  if (a.lora) {
+    u_store(L0, nrows, col, q, sU[0]);
+    u_store(L1, nrows, col, q, sU[1]);
   }
-  __syncthreads();
-  if (!half) {
-    bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
+  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
+  float g[EPI_RPT], u[EPI_RPT];
+  part_add(LG, nrows, q, g);
+  part_add(LUp, nrows, q, u);
+  if (a.lora) {
+    lora_apply(B0, sU[0], sDot, col, q, nrows, gate, g);
+    __syncthreads();                         // sDot is reused
+    lora_apply(B1, sU[1], sDot, col, q, nrows, gate, u);
+  }
+  bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
 #pragma unroll
-    for (int j = 0; j < EPI_RG; ++j) {
-      if (j < nrows) {
-        const float gv = v[j] * s_inv[j], uv = sUp[j][i] * s_inv[j];
-        store_split<bf16>(a.h, lo, (size_t)(m0 + j) * a.F + f, gv / (1.0f + expf(-gv)) * uv);
-      }
+  for (int s = 0; s < EPI_RPT; ++s) {
+    const int j = q + EPI_NQ * s;
+    if (j < nrows) {
+      const float gv = g[s] * s_inv[j], uv = u[s] * s_inv[j];
+      store_split<bf16>(a.h, lo, (size_t)(m0 + j) * a.F + f, gv / (1.0f + expf(-gv)) * uv);
     }
   }
 }

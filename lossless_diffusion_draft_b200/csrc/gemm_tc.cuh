@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < TC_BK / 16; ++k)
-            mma_bf16(d, sdesc_k128(a + k * 32), sdesc_k128(b + k * 32), idesc,
+            mma_f16(d, sdesc_k128(a + k * 32), sdesc_k128(b + k * 32), idesc,
                      (kb > kb0 || k > 0) ? 1u : 0u);
           ++issued;
           mma_commit(&empty[stage]);

@@ -13,16 +13,21 @@
 
 namespace uno {
 
-// Paged KV pool: [n_layers][n_pages][2 (K, V)][n_kv_heads][PAGE][head_dim].
+// Paged KV pool: [n_layers][n_pages][n_planes][n_kv_heads][PAGE][head_dim].
+// Planes: fp32 models K, V; bf16 models K_hi, K_lo, V in fp16 (the keys as a
+// hi/lo pair: their rounding is the largest term of the logit error left
+// once q is a pair too).
 constexpr int KV_PAGE = 64;
 
 struct KvLayout {
   void* pool;
   int n_pages, n_kv_heads, head_dim, pages_per_req;
   const int32_t* page_table;   // [max_batch][pages_per_req]
-  __device__ __forceinline__ size_t offset(int layer, int slot, int pos, int kv, int head,
+  int n_planes;                // 2 (K, V) or 3 (K_hi, K_lo, V)
+  __device__ __forceinline__ int v_plane() const { return n_planes - 1; }
+  __device__ __forceinline__ size_t offset(int layer, int slot, int pos, int plane, int head,
                                            int& ok) const {
-    return offset_in_page(layer, page_of(slot, pos, ok), pos, kv, head);
+    return offset_in_page(layer, page_of(slot, pos, ok), pos, plane, head);
   }
   // page of (slot, pos); ok = 0 (page 0 returned) when pos is outside the slot's pages
   __device__ __forceinline__ int page_of(int slot, int pos, int& ok) const {
@@ -30,10 +35,15 @@ struct KvLayout {
     ok = (pos >= 0 && pi < pages_per_req);
     return ok ? page_table[(size_t)slot * pages_per_req + pi] : 0;
   }
-  __device__ __forceinline__ size_t offset_in_page(int layer, int page, int pos, int kv,
+  __device__ __forceinline__ size_t offset_in_page(int layer, int page, int pos, int plane,
                                                    int head) const {
-    return ((((size_t)layer * n_pages + page) * 2 + kv) * n_kv_heads + head) * KV_PAGE * head_dim +
+    return ((((size_t)layer * n_pages + page) * n_planes + plane) * n_kv_heads + head) * KV_PAGE *
+               head_dim +
            (size_t)(pos % KV_PAGE) * head_dim;
+  }
+  // distance between planes of the same (page, head, position), in elements
+  __device__ __forceinline__ size_t plane_stride() const {
+    return (size_t)n_kv_heads * KV_PAGE * head_dim;
   }
 };
 
@@ -164,17 +174,20 @@ __global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* ga
 }
 
 // RoPE (rotate-half) on q and k of the fused fp32 qkv rows: the rotated q goes
-// to q_out (model dtype, the attention's input) and the rotated k and the v
-// of every row into the paged pool at (slot, position), each rounded once.
+// to q_out (the attention's input) and the rotated k and the v of every row
+// into the paged pool at (slot, position), each rounded once to the
+// attention operand type (KvOf).
 // cos/sin come from a table [max_pos][head_dim / 2] computed on the host in
 // double precision.
 template <typename T>
-__global__ void rope_kv_kernel(const float* qkv, int ld_qkv, T* q_out, int ld_q,
+__global__ void rope_kv_kernel(const float* qkv, int ld_qkv, typename KvOf<T>::type* q_out,
+                               typename KvOf<T>::type* q_lo, int ld_q,
                                const int32_t* row_pos, const int32_t* row_slot, const float* cos_t,
                                const float* sin_t, int max_pos, int H, int Hkv, int hd, KvLayout kv,
                                int layer, int32_t* status) {
   // grid (rows, H + 2 Hkv heads of the fused q|k|v row), hd / 2 threads: one
   // rotate-half pair (i, i + hd/2) per thread
+  typedef typename KvOf<T>::type KV;
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x, h = blockIdx.y, i = threadIdx.x;
@@ -188,27 +201,37 @@ __global__ void rope_kv_kernel(const float* qkv, int ld_qkv, T* q_out, int ld_q,
     const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
     const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
     if (h < H) {
-      T* q = q_out + (size_t)row * ld_q + (size_t)h * hd;
-      q[i] = from_f<T>(y1);
-      q[i + half] = from_f<T>(y2);
+      const size_t qi = (size_t)row * ld_q + (size_t)h * hd;
+      const KV a1 = from_f<KV>(y1), a2 = from_f<KV>(y2);
+      q_out[qi + i] = a1;
+      q_out[qi + i + half] = a2;
+      if (q_lo) {   // rounding residual (the attention adds q_hi K + q_lo K)
+        q_lo[qi + i] = from_f<KV>(y1 - to_f(a1));
+        q_lo[qi + i + half] = from_f<KV>(y2 - to_f(a2));
+      }
     } else {
       int ok;
       const size_t off = kv.offset(layer, slot, pos, 0, h - H, ok);
       if (ok && ok_pos) {
-        T* dst = reinterpret_cast<T*>(kv.pool) + off;
-        dst[i] = from_f<T>(y1);
-        dst[i + half] = from_f<T>(y2);
+        KV* dst = reinterpret_cast<KV*>(kv.pool) + off;
+        const KV b1 = from_f<KV>(y1), b2 = from_f<KV>(y2);
+        dst[i] = b1;
+        dst[i + half] = b2;
+        if (kv.n_planes == 3) {   // K lo plane
+          dst[kv.plane_stride() + i] = from_f<KV>(y1 - to_f(b1));
+          dst[kv.plane_stride() + i + half] = from_f<KV>(y2 - to_f(b2));
+        }
       } else if (i == 0) {
         raise_status(status, ST_POS_OVERFLOW);
       }
     }
   } else {
     int ok;
-    const size_t off = kv.offset(layer, slot, pos, 1, h - H - Hkv, ok);
+    const size_t off = kv.offset(layer, slot, pos, kv.v_plane(), h - H - Hkv, ok);
     if (ok && ok_pos) {
-      T* dst = reinterpret_cast<T*>(kv.pool) + off;
-      dst[i] = from_f<T>(x1);
-      dst[i + half] = from_f<T>(x2);
+      KV* dst = reinterpret_cast<KV*>(kv.pool) + off;
+      dst[i] = from_f<KV>(x1);
+      dst[i + half] = from_f<KV>(x2);
     }
   }
 }

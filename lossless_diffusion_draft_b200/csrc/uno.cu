@@ -107,11 +107,11 @@ struct GemmEnv {
 
   static size_t ws_bytes(int sm) { return (size_t)sm * 2 * 256 * TC_BM * 4; }
 
-  // bf16 2-D row-major tensor [rows, cols] with row stride ld elements; box
-  // of 64 columns (128 bytes, 128-byte swizzle) by box_rows rows.
+  // bf16 (or fp16) 2-D row-major tensor [rows, cols] with row stride ld
+  // elements; box of 64 columns (128 bytes, 128-byte swizzle) by box_rows rows.
   const CUtensorMap* map(const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
-                         uint32_t box_rows) {
-    MapKey k{base, rows, cols, ld, box_rows};
+                         uint32_t box_rows, bool fp16 = false) {
+    MapKey k{base, rows, cols, ld, box_rows | (fp16 ? 0x80000000u : 0u)};
     auto it = maps.find(k);
     if (it != maps.end()) return &it->second;
     EncodeTiledFn f = encode_fn();
@@ -121,7 +121,8 @@ struct GemmEnv {
     const cuuint64_t strides[1] = {ld * 2};
     const cuuint32_t box[2] = {(cuuint32_t)TC_BK, box_rows};
     const cuuint32_t es[2] = {1, 1};
-    if (f(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+    if (f(&m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+          const_cast<void*>(base), dims, strides, box, es,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return nullptr;
@@ -134,9 +135,15 @@ struct DumpShape {
   int NT = 0, units = 0, grid = 0, KBt = 0, m_tiles = 0, n_tiles = 0;
 };
 
+// Token tile width by row count: with split (hi/lo) activations the MMA's N
+// holds 2 NT columns, so NT <= 128 and larger passes take several m-tiles.
+int tc_nt(int M, bool split) {
+  return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : (M <= 128 || split) ? 128 : 256;
+}
+
 // Part slots a DUMP-mode GEMM of M rows and N columns writes, in bytes.
-size_t dump_bytes(int M, int N, int sm_count) {
-  const int NT = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+size_t dump_bytes(int M, int N, int sm_count, bool split) {
+  const int NT = tc_nt(M, split);
   const size_t slots = (size_t)((N + TC_BM - 1) / TC_BM) * ((M + NT - 1) / NT) + sm_count;
   return slots * NT * TC_BM * 4;
 }
@@ -201,7 +208,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.ws = env.ws;
   tp.counters = env.counters;
   if (DUMP) {
-    if (!env.part || dump_bytes(p.M, p.N, env.sm_count) > env.part_bytes) return false;
+    if (!env.part || dump_bytes(p.M, p.N, env.sm_count, SPLIT) > env.part_bytes) return false;
     tp.ws = env.part;
     if (shape) *shape = DumpShape{NT, tp.units, tp.grid, tp.KB + tp.RB, tp.m_tiles, tp.n_tiles};
   }
@@ -250,7 +257,7 @@ void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st, bool pdl) {
 // Tile width NT by row count; hi/lo split activations up to 128 rows.
 template <bool DUMP>
 bool launch_tc_any(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape) {
-  if (p.lo_off > 0 && p.M <= 128) {
+  if (p.lo_off > 0) {
     if (p.M <= 16) return launch_tc<16, true, DUMP>(env, p, st, shape);
     if (p.M <= 32) return launch_tc<32, true, DUMP>(env, p, st, shape);
     if (p.M <= 64) return launch_tc<64, true, DUMP>(env, p, st, shape);
@@ -345,7 +352,8 @@ struct uno_ctx {
   int last_n_req = 0;
   std::string err;
   GemmEnv genv;
-  CUtensorMap kv_map;            // the pool as a 2-D bf16 [rows, head_dim] tensor
+  CUtensorMap kv_map;            // the pool as a 2-D fp16 [rows, head_dim] tensor
+  CUtensorMap q_map;             // q rows as a 3-D fp16 [2 M_max rows, H, head_dim] tensor
   bool kv_map_ok = false;
 
   // CUDA graphs of whole steps, keyed by their arguments
@@ -501,7 +509,8 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
                    void* out_lo) {
   const uno_shape& s = c->s;
   AttnTcParams p{};
-  p.q = (const bf16*)c->qbuf;
+  p.q = (const f16*)c->qbuf;
+  p.q_lo_row = c->M_max;
   p.ld_q = s.n_heads * HD;
   p.out = (bf16*)c->attn;
   p.ld_out = s.n_heads * HD;
@@ -539,7 +548,7 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   {
     Prof prof(c, UNO_K_ATTN, 0.0);
     klaunch(c->genv.pdl, c->stream, dim3(S, p.n_qtiles, n_req * s.n_kv_heads), dim3(ATC_THREADS),
-            AtcCfg<HD>::SMEM, attn_tc_kernel<HD>, c->kv_map, p);
+            AtcCfg<HD>::SMEM, attn_tc_kernel<HD>, c->kv_map, c->q_map, p);
   }
   g_launches[2]++;
   if (S > 1) {
@@ -559,6 +568,8 @@ int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
   }
   AttnParams p{};
   p.qkv = c->qbuf;
+  p.q_lo = sizeof(T) == 2 ? (const char*)c->qbuf + (size_t)c->M_max * s.n_heads * s.head_dim * 2
+                          : nullptr;
   p.ld_qkv = s.n_heads * s.head_dim;
   p.out = c->attn;
   p.ld_out = s.n_heads * s.head_dim;
@@ -643,9 +654,9 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   const int xn_ld = std::max(d, F);
   const int ldu = 3 * r;
   const int hhd = H * hd;
-  // Memory-bound passes (few rows) feed every GEMM input as a hi/lo pair of
-  // bf16 rows (x = hi + lo), the lo rows c->M_max rows below the hi rows.
-  const bool split = sizeof(T) == 2 && M <= 128;
+  // bf16 models feed every GEMM input as a hi/lo pair of bf16 rows
+  // (x = hi + lo), the lo rows c->M_max rows below the hi rows.
+  const bool split = sizeof(T) == 2;
   const int lo = split ? c->M_max : 0;
   auto lo_rows = [&](void* buf, int ld) -> T* {
     return split ? reinterpret_cast<T*>(buf) + (size_t)lo * ld : nullptr;
@@ -680,7 +691,9 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
     other([&] {
       klaunch(c->genv.pdl, st, dim3(M, H + 2 * Hkv), dim3(hd / 2), 0, rope_kv_kernel<T>,
               (const float*)c->qkv,
-              qkv_ld, (T*)c->qbuf, hhd, (const int32_t*)c->row_pos, (const int32_t*)c->row_slot,
+              qkv_ld, (typename KvOf<T>::type*)c->qbuf,
+              split ? (typename KvOf<T>::type*)c->qbuf + (size_t)c->M_max * hhd : nullptr, hhd,
+              (const int32_t*)c->row_pos, (const int32_t*)c->row_slot,
               (const float*)c->cos_t, (const float*)c->sin_t, c->max_pos, H, Hkv, hd, c->kv, l,
               c->d_status);
     });
@@ -812,9 +825,11 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
 
   const int xn_ld = std::max(d, F);
   const int hhd = H * hd;
-  const bool split = M <= 128;
-  const int lo = split ? c->M_max : 0;
-  bf16* attn_lo = split ? (bf16*)c->attn + (size_t)lo * hhd : nullptr;
+  // every GEMM input is a hi/lo pair of bf16 rows (x = hi + lo), the lo rows
+  // M_max rows below the hi rows
+  const bool split = true;
+  const int lo = c->M_max;
+  bf16* attn_lo = (bf16*)c->attn + (size_t)lo * hhd;
 
   EpiArgs ea{};
   ea.M = M;
@@ -822,7 +837,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ea.n_ss = d / TC_BM;
   ea.d_model = (float)d;
   ea.eps = s.rms_eps;
-  ea.q_out = (bf16*)c->qbuf;
+  ea.q_out = (f16*)c->qbuf;
   ea.ld_q = hhd;
   ea.H = H; ea.Hkv = Hkv; ea.hd = hd;
   ea.row_pos = c->row_pos;
@@ -872,10 +887,10 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
       ea.lr.nseg++;
     }
   };
-  auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int threads = TC_BM) {
+  auto epi = [&](void (*kernel)(const EpiArgs), int tiles) {
     Prof prof(c, UNO_K_OTHER, 0.0);
     const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M);
-    klaunch(pdl, st, dim3(tiles, groups), dim3(threads), 0, kernel, ea);
+    klaunch(pdl, st, dim3(tiles, groups), dim3(EPI_THREADS), 0, kernel, ea);
   };
 
   // layer-0 input: g * x and the sums of squares of the embedding rows
@@ -913,7 +928,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_GATE][l], F}, {c->lB[UNO_PROJ_UP][l], F}});
     ea.ss = c->ss;
-    epi(epi_swiglu_kernel, F / TC_BM, 2 * TC_BM);
+    epi(epi_swiglu_kernel, F / TC_BM);
 
     rc = gemm(c->xn, F, F, {{c->w[UNO_PROJ_DOWN][l], d}}, {c->lA[UNO_PROJ_DOWN][l]}, &ea.pv);
     if (rc) return rc;
@@ -1030,7 +1045,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   // KV pool
   const int ppr = ceil_div(max_ctx + B + 2, KV_PAGE);
   const int n_pages = max_batch * ppr;
-  const size_t kv_bytes = (size_t)L * n_pages * 2 * Hkv * KV_PAGE * hd * c->esz;
+  // planes per page: K, V (fp32 models) or K hi, K lo, V in fp16 (bf16 models)
+  const int planes = s.dtype == UNO_BF16 ? 3 : 2;
+  const size_t kv_bytes = (size_t)L * n_pages * planes * Hkv * KV_PAGE * hd * c->esz;
   if (dalloc(&c->kv_pool, kv_bytes) != cudaSuccess) return oom("kv pool");
   // zeroed: keys past a request's length are masked out of the scores, and
   // the values there must be finite so that P V (with P = 0) stays finite
@@ -1039,7 +1056,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->d_cached, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
   if (dalloc(&c->d_pending, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
   if (dalloc(&c->d_stream, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
-  c->kv = KvLayout{c->kv_pool, n_pages, Hkv, hd, ppr, c->d_page_table};
+  c->kv = KvLayout{c->kv_pool, n_pages, Hkv, hd, ppr, c->d_page_table, planes};
   c->free_pages.resize(n_pages);
   for (int i = 0; i < n_pages; ++i) c->free_pages[i] = n_pages - 1 - i;
   c->slot_used.assign(max_batch, 0);
@@ -1056,7 +1073,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->x, (size_t)M * d * 4) != cudaSuccess) return oom("x");
   if (dalloc(&c->xn, (size_t)2 * M * std::max(d, F) * e) != cudaSuccess) return oom("xn");
   if (dalloc(&c->qkv, (size_t)M * (H + 2 * Hkv) * hd * 4) != cudaSuccess) return oom("qkv");
-  if (dalloc(&c->qbuf, (size_t)M * H * hd * e) != cudaSuccess) return oom("q");
+  // q rows: hi rows [0, M), lo rows (bf16 models) from M_max on
+  if (dalloc(&c->qbuf, (size_t)2 * M * H * hd * e) != cudaSuccess) return oom("q");
+  cudaMemset(c->qbuf, 0, (size_t)2 * M * H * hd * e);
   if (dalloc(&c->attn, (size_t)2 * M * H * hd * e) != cudaSuccess) return oom("attn");
   if (dalloc(&c->gu, (size_t)M * 2 * F * 4) != cudaSuccess) return oom("gu");
   if (dalloc(&c->U, (size_t)2 * M * 3 * lora_rank * e) != cudaSuccess) return oom("U");
@@ -1139,7 +1158,8 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
       const int rr = lora_rank;
       for (int m = 1; m <= M; ++m) {
         const int ns[4] = {(H + 2 * Hkv) * hd + 3 * rr, d + rr, 2 * F + 2 * rr, d + rr};
-        for (int k = 0; k < 4; ++k) part = std::max(part, dump_bytes(m, ns[k], c->genv.sm_count));
+        for (int k = 0; k < 4; ++k)
+          part = std::max(part, dump_bytes(m, ns[k], c->genv.sm_count, /*split=*/true));
       }
       if (dalloc(&c->genv.part, part) != cudaSuccess) return oom("gemm parts");
       c->genv.part_bytes = part;
@@ -1147,11 +1167,22 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
       c->fused = true;
     }
   }
-  // tensor-core attention: the pool as a [rows, head_dim] tensor, 64x64 boxes
+  // tensor-core attention: the pool (fp16 for bf16 models) as a [rows, head_dim]
+  // tensor, 64x64 boxes
   if (s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && ATC_QROWS % G == 0) {
-    const uint64_t rows = (uint64_t)L * n_pages * 2 * Hkv * KV_PAGE;
-    const CUtensorMap* m = c->genv.map(c->kv_pool, rows, hd, hd, KV_PAGE);
-    if (m) {
+    const uint64_t rows = (uint64_t)L * n_pages * planes * Hkv * KV_PAGE;
+    const CUtensorMap* m = c->genv.map(c->kv_pool, rows, hd, hd, KV_PAGE, /*fp16=*/true);
+    // q: box (64 of head_dim, the G heads of a kv head, the query tile's tokens)
+    EncodeTiledFn f = encode_fn();
+    const cuuint64_t qdims[3] = {(cuuint64_t)hd, (cuuint64_t)H, (cuuint64_t)2 * M};
+    const cuuint64_t qstrides[2] = {(cuuint64_t)hd * 2, (cuuint64_t)H * hd * 2};
+    const cuuint32_t qbox[3] = {64, (cuuint32_t)G, (cuuint32_t)(ATC_QROWS / G)};
+    const cuuint32_t qes[3] = {1, 1, 1};
+    const bool qok = f && f(&c->q_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, c->qbuf, qdims, qstrides,
+                            qbox, qes, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (m && qok) {
       c->kv_map = *m;
       c->kv_map_ok = true;
     }
@@ -1554,7 +1585,9 @@ int uno_debug_kv(uno_ctx* c, int req, int layer, int pos0, int n, void* k_host, 
     const int page = c->h_page_table[(size_t)req * ppr + pos / KV_PAGE];
     for (int h = 0; h < Hkv; ++h)
       for (int kv = 0; kv < 2; ++kv) {
-        const size_t off = ((((size_t)layer * c->kv.n_pages + page) * 2 + kv) * Hkv + h) * KV_PAGE * hd +
+        const int plane = kv ? c->kv.n_planes - 1 : 0;   // K (hi), V
+        const size_t off = ((((size_t)layer * c->kv.n_pages + page) * c->kv.n_planes + plane) * Hkv + h) *
+                               KV_PAGE * hd +
                            (size_t)(pos % KV_PAGE) * hd;
         char* dst = (char*)(kv ? v_host : k_host) + ((size_t)i * Hkv + h) * row;
         CK(cudaMemcpy(dst, (char*)c->kv_pool + off * c->esz, row, cudaMemcpyDeviceToHost));

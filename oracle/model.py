@@ -203,6 +203,16 @@ class KVCache:
             self.v[l] = np.concatenate([self.v[l], v_rows[l][take]], axis=0)
 
 
+class _Float64View:
+    """Read-only float64 view of a parameter mapping, converted per access."""
+
+    def __init__(self, params):
+        self._params = params
+
+    def __getitem__(self, name):
+        return np.asarray(self._params[name], dtype=np.float64)
+
+
 class Model:
     """A model of a given shape with float64 parameters.
 
@@ -213,7 +223,12 @@ class Model:
 
     def __init__(self, shape, params):
         self.shape = dict(shape)
-        self.p = {k: np.asarray(v, dtype=np.float64) for k, v in params.items()}
+        if isinstance(params, dict):
+            self.p = {k: np.asarray(v, dtype=np.float64) for k, v in params.items()}
+        else:
+            # any other mapping is read on demand, one parameter at a time (a
+            # model too large to hold in float64 at once); same values
+            self.p = _Float64View(params)
         self.scale = shape["lora_alpha"] / shape["lora_rank"]
 
     def _lin(self, l, proj, x, gate):

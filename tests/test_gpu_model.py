@@ -46,7 +46,7 @@ def _setup(name, n_req, prompt_len, max_ctx, fused=True, **over):
 def _kv_check(ctx, cfg, model, state, req, tol):
     c = state.c
     Hkv, hd = cfg["n_kv_heads"], cfg["head_dim"]
-    dt = torch.float32 if cfg["dtype"] == "f32" else torch.bfloat16
+    dt = torch.float32 if cfg["dtype"] == "f32" else torch.float16   # the cache is fp16 for bf16 models
     for l in range(cfg["n_layers"]):
         k = torch.empty((c, Hkv, hd), dtype=dt)
         v = torch.empty((c, Hkv, hd), dtype=dt)
