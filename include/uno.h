@@ -157,8 +157,9 @@ int uno_set_graphs(uno_ctx *ctx, int enable);
 int uno_set_pdl(uno_ctx *ctx, int enable);
 
 /* Fused layer pipeline (implementation choice, on by default where it
- * applies: bf16 models with head_dim 64 or 128, d_model, ffn_dim and the
- * q / kv widths multiples of 128, d_model <= 8192, LoRA rank 0 or 128).  Each projection
+ * applies: passes of at most 128 rows of bf16 models with head_dim 64 or
+ * 128, d_model, ffn_dim and the q / kv widths multiples of 128, d_model <=
+ * 8192, LoRA rank 0 or 128).  Each projection
  * GEMM then leaves fp32 parts that one epilogue kernel reduces and carries
  * through LoRA-B, the RMSNorm scale, RoPE and the KV write, SwiGLU or the
  * residual add; the LoRA A matrices stream with the base weights.  enable =

@@ -407,16 +407,18 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   }
 }
 
-// Merge of the split partials: one CTA per (query row, group), one thread
-// per head_dim element.  Every thread loads all splits' (m, l) (the same
-// addresses across the CTA) together with its own O column, so the merge is
-// one round of loads; the splits are added in split order.
+// Merge of the split partials: one CTA per (ATC_MERGE_ROWS query rows,
+// group), one thread per (row, head_dim element).  Every thread loads all
+// splits' (m, l) (the same addresses across a row) together with its own O
+// column, so the merge is one round of loads; the splits are added in split
+// order.
 constexpr int ATC_MAX_SPLITS = 32;
+constexpr int ATC_MERGE_ROWS = 4;
 template <int HD>
-__global__ void __launch_bounds__(HD) attn_merge_kernel(const AttnTcParams p) {
+__global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const AttnTcParams p) {
   pdl_trigger();
   pdl_wait();
-  const int r = blockIdx.x, group = blockIdx.y;
+  const int r = blockIdx.x * ATC_MERGE_ROWS + threadIdx.y, group = blockIdx.y;
   const int z = group / p.n_qtiles, qt = group % p.n_qtiles;
   const int req = z / p.Hkv, kvh = z % p.Hkv;
   const int G = p.H / p.Hkv;

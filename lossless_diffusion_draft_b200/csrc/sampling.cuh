@@ -34,17 +34,25 @@ namespace uno {
 constexpr int SAMPLE_THREADS = 256;
 
 // ---------------------------------------------------------------------------
-// Phase A: reduce one chunk of one row to (max, sum exp(l - max)).
+// Phase A: reduce one chunk of one row to (max, sum exp(l - max)).  Each
+// thread reduces its own logits to a (max, sum) pair; the pairs are combined
+// across the CTA in a fixed tree (warp butterfly, then the warps in order),
+// so one reduction serves both statistics.
 // ---------------------------------------------------------------------------
+constexpr int CHUNK_IT = 8;   // float4 per thread: a chunk holds <= 8 * 4 * 256 = 8192 logits
+__device__ __forceinline__ float2 ms_combine(float2 a, float2 b) {
+  const float M = fmaxf(a.x, b.x);
+  if (M == -INFINITY) return make_float2(M, 0.f);
+  return make_float2(M, a.y * expf(a.x - M) + b.y * expf(b.x - M));
+}
 __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red) {
   // float4 path: rows start on 16-byte boundaries (vocab % 4 == 0 is required)
   const int n4 = (c1 - c0) >> 2;
   const float4* r4 = reinterpret_cast<const float4*>(row + c0);
-  constexpr int MAXIT = 16;  // chunk <= 16 * 4 * 256 = 16384 logits
-  float4 v[MAXIT];
+  float4 v[CHUNK_IT];
   float m = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < MAXIT; ++i) {
+  for (int i = 0; i < CHUNK_IT; ++i) {
     const int j = threadIdx.x + i * SAMPLE_THREADS;
     if (j < n4) {
       v[i] = __ldcs(r4 + j);
@@ -53,18 +61,29 @@ __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1,
   }
   // scalar tail (chunk length not a multiple of 4: only the row's last chunk)
   for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) m = fmaxf(m, row[j]);
-  const float M = block_max<SAMPLE_THREADS>(m, red);
   float s = 0.f;
-  if (M != -INFINITY) {
+  if (m != -INFINITY) {
 #pragma unroll
-    for (int i = 0; i < MAXIT; ++i) {
+    for (int i = 0; i < CHUNK_IT; ++i) {
       const int j = threadIdx.x + i * SAMPLE_THREADS;
-      if (j < n4) s += expf(v[i].x - M) + expf(v[i].y - M) + expf(v[i].z - M) + expf(v[i].w - M);
+      if (j < n4) s += expf(v[i].x - m) + expf(v[i].y - m) + expf(v[i].z - m) + expf(v[i].w - m);
     }
-    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += expf(row[j] - M);
+    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += expf(row[j] - m);
   }
-  const float S = block_sum<SAMPLE_THREADS>(s, red);
-  return make_float2(M, S);
+  float2 ms = make_float2(m, s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    ms = ms_combine(ms, make_float2(__shfl_xor_sync(0xffffffffu, ms.x, o),
+                                    __shfl_xor_sync(0xffffffffu, ms.y, o)));
+  float2* red2 = reinterpret_cast<float2*>(red);     // SAMPLE_THREADS / 32 pairs
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  __syncthreads();                                    // red may hold a previous reduction
+  if (lane == 0) red2[wid] = ms;
+  __syncthreads();
+  float2 t = red2[0];
+#pragma unroll
+  for (int w = 1; w < SAMPLE_THREADS / 32; ++w) t = ms_combine(t, red2[w]);
+  return t;
 }
 
 // Row-level combine of chunk pairs (run by one thread, chunk order).
@@ -80,10 +99,15 @@ __device__ __forceinline__ RowStat combine_row(const float2* part, int nch) {
   return {M, Z};
 }
 
-// Weight functors used by the crossing scan.
+// Weight functors used by the crossing scan (get4: four weights from v, a
+// multiple of 4).
 struct SoftmaxW {
   const float* row; float M;
   __device__ __forceinline__ float operator()(int v) const { return expf(row[v] - M); }
+  __device__ __forceinline__ void get4(int v, float* w) const {
+    const float4 x = *reinterpret_cast<const float4*>(row + v);
+    w[0] = expf(x.x - M); w[1] = expf(x.y - M); w[2] = expf(x.z - M); w[3] = expf(x.w - M);
+  }
 };
 struct ResidW {
   const float* p; const float* q; float lse_p, lse_q;
@@ -92,26 +116,41 @@ struct ResidW {
     return d > 0.f ? d : 0.f;
   }
   __device__ __forceinline__ float operator()(int v) const { return pair(p[v], q[v]); }
+  __device__ __forceinline__ void get4(int v, float* w) const {
+    const float4 x = *reinterpret_cast<const float4*>(p + v);
+    const float4 y = *reinterpret_cast<const float4*>(q + v);
+    w[0] = pair(x.x, y.x); w[1] = pair(x.y, y.y); w[2] = pair(x.z, y.z); w[3] = pair(x.w, y.w);
+  }
 };
 
 // First v in [c0, c1) whose running prefix base + sum_{c0..v} w exceeds
-// target (thread-contiguous segments, fixed order); -1 if none.  `last_pos`
-// receives the last v with w > 0 (-1 if none).  All threads participate.
+// target (thread-contiguous segments of a multiple of 4 elements, fixed
+// order); -1 if none.  `last_pos` receives the last v with w > 0 (-1 if
+// none).  c0 and c1 are multiples of 4 and c1 - c0 <= 4 * CHUNK_IT *
+// SAMPLE_THREADS.  Each thread reads its segment once (16-byte loads) and
+// keeps the weights in registers for the scan.  All threads participate.
 template <typename W>
 __device__ int chunk_crossing(const W& w, int c0, int c1, float base, float target, int* last_pos,
                               float* red) {
+  constexpr int SEG = 4 * CHUNK_IT;   // elements per thread at most
   __shared__ float s_tot[SAMPLE_THREADS / 32];
   __shared__ int s_i[2];
   const int len = c1 - c0;
-  const int per = (len + SAMPLE_THREADS - 1) / SAMPLE_THREADS;
+  const int per = ((len + 4 * SAMPLE_THREADS - 1) / (4 * SAMPLE_THREADS)) * 4;
   const int b = c0 + threadIdx.x * per;
   const int e = min(c1, b + per);
+  float wv[SEG];
+#pragma unroll
+  for (int k = 0; k < SEG; k += 4) {
+    if (b + k < e) w.get4(b + k, wv + k);
+    else wv[k] = wv[k + 1] = wv[k + 2] = wv[k + 3] = 0.f;
+  }
   float tsum = 0.f;
   int lastpos = -1;
-  for (int v = b; v < e; ++v) {
-    const float x = w(v);
-    tsum += x;
-    if (x > 0.f) lastpos = v;
+#pragma unroll
+  for (int k = 0; k < SEG; ++k) {
+    tsum += wv[k];
+    if (wv[k] > 0.f) lastpos = b + k;
   }
   // block exclusive scan of tsum
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -128,9 +167,10 @@ __device__ int chunk_crossing(const W& w, int c0, int c1, float base, float targ
   for (int k = 0; k < wid; ++k) wbase += s_tot[k];
   float run = base + wbase + (incl - tsum);
   int hit = INT_MAX;
-  for (int v = b; v < e; ++v) {
-    run += w(v);
-    if (run > target) { hit = v; break; }
+#pragma unroll
+  for (int k = 0; k < SEG; ++k) {
+    run += wv[k];
+    if (hit == INT_MAX && b + k < e && run > target) hit = b + k;
   }
   if (hit != INT_MAX) atomicMin(&s_i[0], hit);
   if (lastpos >= 0) atomicMax(&s_i[1], lastpos);
@@ -198,7 +238,7 @@ struct SampleArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(SAMPLE_THREADS) sample_rows_kernel(const SampleArgs a) {
+__global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const SampleArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last;
   pdl_trigger();
@@ -319,7 +359,7 @@ __device__ void verify_finish(const VerifyArgs& a, int req, int slot, int pos0, 
   }
 }
 
-__global__ void __launch_bounds__(SAMPLE_THREADS) spec_verify_kernel(const VerifyArgs a) {
+__global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last;
   __shared__ int s_a;

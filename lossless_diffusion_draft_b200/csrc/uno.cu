@@ -420,6 +420,7 @@ struct Prof {
 namespace {
 
 constexpr int PREFILL_CHUNK = 512;
+constexpr int FUSED_MAX_ROWS = 128;   // rows of a pass the fused pipeline takes
 // Largest vocabulary: 64 chunks of 8192 logits (one thread combines a row's
 // chunk pairs serially).
 constexpr int MAX_VOCAB = 64 * 8192;
@@ -553,7 +554,10 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   g_launches[2]++;
   if (S > 1) {
     Prof prof(c, UNO_K_ATTN, 0.0);
-    klaunch(c->genv.pdl, c->stream, dim3(ATC_QROWS, groups), dim3(HD), 0, attn_merge_kernel<HD>, p);
+    // only the rows a query tile can hold: tokens per request x heads per kv head
+    const int rows = std::min(ATC_QROWS, rows_per_req * G);
+    klaunch(c->genv.pdl, c->stream, dim3(ceil_div(rows, ATC_MERGE_ROWS), groups),
+            dim3(HD, ATC_MERGE_ROWS), 0, attn_merge_kernel<HD>, p);
   }
   return UNO_OK;
 }
@@ -955,7 +959,11 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
 
 int forward_any(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* req_ids,
                 const int32_t* prompt, int prefill_slot, int prefill_pos0, float* logits) {
-  if (c->fused && c->fused_enabled)
+  // The fused pipeline is built for memory-bound passes (its epilogues do
+  // LoRA-B on the CUDA cores and are sized for a few dozen rows); a pass
+  // larger than one GEMM token tile runs the unfused kernels, where LoRA-B is
+  // a tensor-core K extension and the row kernels are bandwidth-bound.
+  if (c->fused && c->fused_enabled && n_req * rows_per_req <= FUSED_MAX_ROWS)
     return forward_fused(c, kind, n_req, rows_per_req, req_ids, prompt, prefill_slot, prefill_pos0,
                          logits);
   if (c->s.dtype == UNO_BF16)
