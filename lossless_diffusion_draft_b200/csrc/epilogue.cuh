@@ -463,8 +463,11 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_resid_kernel(const EpiArgs a)
 // gate|up -> silu(gate) * up: grid (F / 128, row groups), EPI_THREADS
 // threads; each thread takes the gate and the up column of one feature.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(EPI_THREADS) epi_swiglu_kernel(const EpiArgs a) {
-  constexpr int C = 4;
+__global__ void __launch_bounds__(EPI_THREADS, 2) epi_swiglu_kernel(const EpiArgs a) {
+  // two CTAs per SM (one wave for the decode passes' 2 x F / 128 CTAs): up's
+  // adapter half is read after gate's dot, and gate|up tiles have at most two
+  // contributors at these sizes (more take further rounds)
+  constexpr int C = 2;
   __shared__ float s_inv[EPI_RG];
   __shared__ float s_ss[EPI_RG * EPI_MAX_SS];
   __shared__ __align__(16) float sU[2][EPI_RG * EPI_R];
@@ -478,19 +481,18 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_swiglu_kernel(const EpiArgs a
   const int f = ft * TC_BM + col;
   const int ut = a.F / TC_BM + ft;         // the up tile of the same features
 
-  // ---- every global load first
+  // ---- the global loads (up's adapter half comes after gate's dot)
   SsLoad ssv;
   ss_issue(a, m0, nrows, ssv);
   PartLoad<C> LG, LUp, L0, L1;
-  BPart B0, B1;
+  BPart B;
   float gate[EPI_RPT];
   part_issue(a.pv, ft, m0, nrows, col, q, LG);
   part_issue(a.pv, ut, m0, nrows, col, q, LUp);
   if (a.lora) {
     u_issue(a, 0, m0, nrows, col, q, L0);
     u_issue(a, 1, m0, nrows, col, q, L1);
-    bpart_issue(a, 0, f, q, B0);
-    bpart_issue(a, 1, f, q, B1);
+    bpart_issue(a, 0, f, q, B);
     gate_issue(a, m0, nrows, q, gate);
   }
   // ---- then the arithmetic
@@ -503,9 +505,10 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_swiglu_kernel(const EpiArgs a
   part_add(LG, nrows, q, g);
   part_add(LUp, nrows, q, u);
   if (a.lora) {
-    lora_apply(B0, sU[0], sDot, col, q, nrows, gate, g);
+    lora_apply(B, sU[0], sDot, col, q, nrows, gate, g);
+    bpart_issue(a, 1, f, q, B);
     __syncthreads();                         // sDot is reused
-    lora_apply(B1, sU[1], sDot, col, q, nrows, gate, u);
+    lora_apply(B, sU[1], sDot, col, q, nrows, gate, u);
   }
   bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
 #pragma unroll

@@ -58,7 +58,7 @@ struct TcMaps {
 struct TcSeg { int n0, n, u_off; };
 
 struct TcParams {
-  int M, N, KB, RB;          // rows, columns, k-blocks of K, k-blocks of r (0: no LoRA)
+  int M, N, KB, RB;          // rows, columns, units (KPS k-blocks) of K and of r (0: no LoRA)
   int n_tiles, m_tiles;
   int nseg; TcSeg seg[TC_MAX_SEG];
   int units, grid;           // stream-K: units = tiles * (KB + RB), split over grid CTAs
@@ -89,12 +89,18 @@ __device__ __forceinline__ int sk_owner(int u, int units, int grid) {
 // lo = bf16(x - hi) (rows lo_off apart in the buffer); the MMA's N covers
 // both (2 NT columns) and the epilogue adds column m and column NT + m, so
 // the product sees x to ~16 mantissa bits while the weights stream once.
-template <int NT, bool SPLIT>
+// KPS: 64-element k-blocks per pipeline stage (a unit of stream-K work).  Two
+// put 256 contiguous bytes of every weight row in flight together.
+template <int NT, bool SPLIT, int KPS>
 struct TcCfg {
   static constexpr int NMMA = SPLIT ? 2 * NT : NT;           // MMA N
-  static constexpr int B_BYTES = NMMA * TC_BK * 2;
-  static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int B_SUB = NMMA * TC_BK * 2;             // one k-block of activations
+  static constexpr int A_BYTES = KPS * TC_A_BYTES;
+  static constexpr int B_BYTES = KPS * B_SUB;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int MAX_STAGES = 8 / KPS;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > MAX_STAGES ? MAX_STAGES
+                                                                         : (200 * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = NMMA < 32 ? 64 : 2 * NMMA;  // two accumulators, power of two
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
@@ -121,15 +127,15 @@ __device__ __forceinline__ void tc_store(const TcParams& p, int m, int n, float 
   }
 }
 
-template <int NT, bool SPLIT, bool DUMP>
+template <int NT, bool SPLIT, bool DUMP, int KPS>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
-  using C = TcCfg<NT, SPLIT>;
+  using C = TcCfg<NT, SPLIT, KPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + C::STAGES * TC_A_BYTES;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
   uint64_t* full = bars;                      // [STAGES] TMA -> MMA
   uint64_t* empty = bars + C::STAGES;         // [STAGES] MMA -> TMA
@@ -195,28 +201,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int n_row = (t / p.m_tiles) * TC_BM;
         const int sg = seg_of(n_row);
         map = kb < p.KB ? &maps.w[sg] : &maps.b[sg];
-        x = (kb < p.KB ? kb : kb - p.KB) * TC_BK;
+        x = (kb < p.KB ? kb : kb - p.KB) * TC_BK * KPS;
         y = n_row - p.seg[sg].n0;
       };
       auto load_a = [&](int u, int stage) {
         const CUtensorMap* map;
         int x, y;
         coords_a(u, map, x, y);
-        tma_load_2d(sA + stage * TC_A_BYTES, map, &full[stage], x, y);
+#pragma unroll
+        for (int j = 0; j < KPS; ++j)
+          tma_load_2d(sA + stage * C::A_BYTES + j * TC_A_BYTES, map, &full[stage], x + j * TC_BK, y);
       };
 
       auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
         const int t = u / KBt, kb = u % KBt;
         const int mt = t % p.m_tiles;
-        uint8_t* dst = sB + stage * C::B_BYTES;
-        if (kb < p.KB) {
-          tma_load_2d(dst, &maps.x, &full[stage], kb * TC_BK, mt * NT);
-          if (SPLIT) tma_load_2d(dst + NT * 128, &maps.x, &full[stage], kb * TC_BK, p.lo_off + mt * NT);
-        } else {
-          const int sg = seg_of((t / p.m_tiles) * TC_BM);
-          const int x = p.seg[sg].u_off + (kb - p.KB) * TC_BK;
-          tma_load_2d(dst, &maps.u, &full[stage], x, mt * NT);
-          if (SPLIT) tma_load_2d(dst + NT * 128, &maps.u, &full[stage], x, p.lo_off + mt * NT);
+#pragma unroll
+        for (int j = 0; j < KPS; ++j) {
+          uint8_t* dst = sB + stage * C::B_BYTES + j * C::B_SUB;
+          if (kb < p.KB) {
+            const int x = (kb * KPS + j) * TC_BK;
+            tma_load_2d(dst, &maps.x, &full[stage], x, mt * NT);
+            if (SPLIT) tma_load_2d(dst + NT * 128, &maps.x, &full[stage], x, p.lo_off + mt * NT);
+          } else {
+            const int sg = seg_of((t / p.m_tiles) * TC_BM);
+            const int x = p.seg[sg].u_off + ((kb - p.KB) * KPS + j) * TC_BK;
+            tma_load_2d(dst, &maps.u, &full[stage], x, mt * NT);
+            if (SPLIT) tma_load_2d(dst + NT * 128, &maps.u, &full[stage], x, p.lo_off + mt * NT);
+          }
         }
       };
       const int total = u1 - u0;
@@ -263,12 +275,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a = smem_u32(sA + stage * TC_A_BYTES);
-          const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < TC_BK / 16; ++k)
-            mma_f16(d, sdesc_k128(a + k * 32), sdesc_k128(b + k * 32), idesc,
-                     (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < KPS; ++j) {
+            const uint32_t a = smem_u32(sA + stage * C::A_BYTES + j * TC_A_BYTES);
+            const uint32_t b = smem_u32(sB + stage * C::B_BYTES + j * C::B_SUB);
+#pragma unroll
+            for (int k = 0; k < TC_BK / 16; ++k)
+              mma_f16(d, sdesc_k128(a + k * 32), sdesc_k128(b + k * 32), idesc,
+                      (kb > kb0 || j > 0 || k > 0) ? 1u : 0u);
+          }
           ++issued;
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }

@@ -148,7 +148,7 @@ size_t dump_bytes(int M, int N, int sm_count, bool split) {
   return slots * NT * TC_BM * 4;
 }
 
-template <int NT, bool SPLIT, bool DUMP>
+template <int NT, bool SPLIT, bool DUMP, int KPS>
 bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape = nullptr) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -173,8 +173,8 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   TcParams tp{};
   tp.M = p.M;
   tp.N = p.N;
-  tp.KB = p.K / TC_BK;
-  tp.RB = p.U ? p.r / TC_BK : 0;
+  tp.KB = p.K / (TC_BK * KPS);
+  tp.RB = p.U ? p.r / (TC_BK * KPS) : 0;
   tp.nseg = p.nseg;
   for (int s = 0; s < p.nseg; ++s) {
     const GemmSeg& g = p.seg[s];
@@ -215,16 +215,16 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.status = env.status;
   tp.lo_off = SPLIT ? p.lo_off : 0;
   tp.out_lo = p.out_lo;
-  using Cfg = TcCfg<NT, SPLIT>;
+  using Cfg = TcCfg<NT, SPLIT, KPS>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT, DUMP>,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT, DUMP, KPS>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
       return false;
     attr = true;
   }
-  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM, gemm_tc_kernel<NT, SPLIT, DUMP>,
-          maps, tp);
+  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM,
+          gemm_tc_kernel<NT, SPLIT, DUMP, KPS>, maps, tp);
   g_launches[0]++;
   return true;
 }
@@ -255,19 +255,26 @@ void gemm_simt_dispatch(const GemmParams& p, cudaStream_t st, bool pdl) {
 }
 
 // Tile width NT by row count; hi/lo split activations up to 128 rows.
+template <bool DUMP, int KPS>
+bool launch_tc_kps(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape) {
+  if (p.lo_off > 0) {
+    if (p.M <= 16) return launch_tc<16, true, DUMP, KPS>(env, p, st, shape);
+    if (p.M <= 32) return launch_tc<32, true, DUMP, KPS>(env, p, st, shape);
+    if (p.M <= 64) return launch_tc<64, true, DUMP, KPS>(env, p, st, shape);
+    return launch_tc<128, true, DUMP, KPS>(env, p, st, shape);
+  }
+  if (p.M <= 16) return launch_tc<16, false, DUMP, KPS>(env, p, st, shape);
+  if (p.M <= 32) return launch_tc<32, false, DUMP, KPS>(env, p, st, shape);
+  if (p.M <= 64) return launch_tc<64, false, DUMP, KPS>(env, p, st, shape);
+  if (p.M <= 128) return launch_tc<128, false, DUMP, KPS>(env, p, st, shape);
+  return launch_tc<256, false, DUMP, KPS>(env, p, st, shape);
+}
+// Two k-blocks per stage where K and the adapter rank allow it.
 template <bool DUMP>
 bool launch_tc_any(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* shape) {
-  if (p.lo_off > 0) {
-    if (p.M <= 16) return launch_tc<16, true, DUMP>(env, p, st, shape);
-    if (p.M <= 32) return launch_tc<32, true, DUMP>(env, p, st, shape);
-    if (p.M <= 64) return launch_tc<64, true, DUMP>(env, p, st, shape);
-    return launch_tc<128, true, DUMP>(env, p, st, shape);
-  }
-  if (p.M <= 16) return launch_tc<16, false, DUMP>(env, p, st, shape);
-  if (p.M <= 32) return launch_tc<32, false, DUMP>(env, p, st, shape);
-  if (p.M <= 64) return launch_tc<64, false, DUMP>(env, p, st, shape);
-  if (p.M <= 128) return launch_tc<128, false, DUMP>(env, p, st, shape);
-  return launch_tc<256, false, DUMP>(env, p, st, shape);
+  if (p.K % (2 * TC_BK) == 0 && (!p.U || p.r % (2 * TC_BK) == 0))
+    return launch_tc_kps<DUMP, 2>(env, p, st, shape);
+  return launch_tc_kps<DUMP, 1>(env, p, st, shape);
 }
 
 // Runs one gated-LoRA GEMM: tcgen05 for bf16 shapes it takes, SIMT otherwise.
