@@ -61,10 +61,10 @@ struct AtcCfg {
   static constexpr int Q_BYTES = ATC_QROWS * HD * 2;
   static constexpr int KV_BYTES = ATC_KT * HD * 2;      // K or V of one stage
   static constexpr int P_BYTES = ATC_QROWS * ATC_KT * 2;
-  // stages of K hi, K lo and V: four fit beside q hi/lo and P for head_dim
-  // 64, two for 128
-  static constexpr int STAGES = HD <= 64 ? 4 : 2;
-  static constexpr int SMEM = 2 * Q_BYTES + STAGES * 3 * KV_BYTES + 2 * P_BYTES + 1024 + 256;
+  // stages of K hi, K lo and V beside q hi/lo and one P tile: three for
+  // head_dim 128 (224 KB), six for 64
+  static constexpr int STAGES = HD <= 64 ? 6 : 3;
+  static constexpr int SMEM = 2 * Q_BYTES + STAGES * 3 * KV_BYTES + P_BYTES + 1024 + 256;
   static constexpr int TMEM_COLS = 256;       // 2 score tiles + the output accumulator
   static constexpr int S_COL = 0;             // score tiles at columns 0, 64
   static constexpr int O_COL = 2 * ATC_KT;    // output accumulator at 128 .. 128 + HD
@@ -97,8 +97,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   uint8_t* sK = sQl + C::Q_BYTES;                       // [STAGES] K hi: NB boxes [64 keys x 64]
   uint8_t* sKl = sK + C::STAGES * C::KV_BYTES;          // [STAGES] K lo
   uint8_t* sV = sKl + C::STAGES * C::KV_BYTES;          // [STAGES] V
-  uint8_t* sP = sV + C::STAGES * C::KV_BYTES;           // [2] [128 rows x 64 keys]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * C::P_BYTES);
+  // one P tile [128 rows x 64 keys]: P(i) is written only after PV(i-1), its
+  // previous reader, has completed (the softmax waits for that anyway)
+  uint8_t* sP = sV + C::STAGES * C::KV_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
   uint64_t* kv_full = bars;                             // [STAGES]
   uint64_t* kv_empty = bars + C::STAGES;                // [STAGES]
   uint64_t* s_full = bars + 2 * C::STAGES;              // [2]
@@ -254,7 +256,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         // O accumulates in TMEM across tiles
 #pragma unroll
         for (int ks = 0; ks < ATC_KT / 16; ++ks)
-          mma_f16(tmem + C::O_COL, sdesc_k128(smem_u32(sP + b2 * C::P_BYTES) + ks * 32),
+          mma_f16(tmem + C::O_COL, sdesc_k128(smem_u32(sP) + ks * 32),
                    sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
                    idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         mma_commit(o_full);            // phase i completes when PV(i) has
@@ -343,13 +345,13 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       l += psum;
-      // the P buffer of this tile was read by PV(i-2): PV(i-1) done implies it
+      // the P tile was last read by PV(i-1): wait for it before overwriting
       if (i > 0 && !pv_done) {
         bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(i - 1) & 1);
         if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
       }
       // P row -> shared memory (K-major over keys, 128-byte swizzle)
-      uint8_t* prow = sP + sb * C::P_BYTES + r * 128;
+      uint8_t* prow = sP + r * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
