@@ -414,8 +414,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 // splits' (m, l) (the same addresses across a row) together with its own O
 // column, so the merge is one round of loads; the splits are added in split
 // order.
-constexpr int ATC_MAX_SPLITS = 32;
-constexpr int ATC_MERGE_ROWS = 4;
+// Registers stay small enough (rows x head_dim threads) that a GEMM CTA of
+// the next projection fits on the same SM and starts its weight stream.
+constexpr int ATC_MAX_SPLITS = 24;
+constexpr int ATC_MERGE_ROWS = 2;
 template <int HD>
 __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const AttnTcParams p) {
   pdl_trigger();

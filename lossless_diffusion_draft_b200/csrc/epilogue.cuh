@@ -25,9 +25,10 @@
 // multiplies U by the rows of B on the CUDA cores (r MACs per output) and
 // gates it per row.
 //
-// One CTA takes one 128-column tile of the output (two for SwiGLU) and
-// EPI_RG rows; EPI_NQ threads share a column, each with a few of the rows.  Every load a thread needs is issued before the first use,
-// so a CTA costs about one memory round trip.
+// One CTA takes one 128-column tile of the output (two for SwiGLU) and a
+// group of rows (Geo below); a few slot threads share a column, each with a
+// few of the rows.  Every load a thread needs is issued before the first
+// use, so a CTA costs about one memory round trip.
 #pragma once
 
 #include "gemm_tc.cuh"
@@ -35,7 +36,6 @@
 
 namespace uno {
 
-constexpr int EPI_RG = 9;            // token rows per CTA (a 17-row draft pass: two groups)
 constexpr int EPI_R = TC_BM;         // LoRA rank the fused epilogue takes (one U tile)
 
 // Where a DUMP-mode GEMM left its parts.
@@ -78,28 +78,37 @@ struct EpiArgs {
   int32_t* status;
 };
 
-// Thread layout of every epilogue CTA: EPI_NQ row slots x 128 columns.
-// Thread t owns column t % 128 and, in slot q = t / 128, the rows
-// j = q + EPI_NQ * s (s < EPI_RPT) of the CTA's EPI_RG rows.  With several
-// warps per scheduler and a few rows per thread, the loads of a CTA stay in
-// flight together and the arithmetic hides its latency.
-constexpr int EPI_NQ = 2;
-constexpr int EPI_RPT = (EPI_RG + EPI_NQ - 1) / EPI_NQ;
-constexpr int EPI_THREADS = EPI_NQ * TC_BM;
-constexpr int EPI_KQ = EPI_R / EPI_NQ;    // rank columns of a thread's share of the LoRA-B dot
+// Thread layout of an epilogue CTA: NQ row slots x 128 columns, the NQ
+// slot threads of a column in adjacent lanes (thread t: slot q = t % NQ,
+// column t / NQ).  A thread owns rows j = q + NQ s (s < RPT) of the CTA's RG
+// rows.  The LoRA-B dot of a column is split by rank over its slot threads,
+// whose partials meet in a fixed shuffle butterfly.
+constexpr int EPI_MAX_SS = 64;        // d_model <= 64 * 128
+template <int RG_, int NQ_>
+struct Geo {
+  static constexpr int RG = RG_, NQ = NQ_;
+  static constexpr int RPT = (RG + NQ - 1) / NQ;
+  static constexpr int THREADS = NQ * TC_BM;
+  static constexpr int KQ = EPI_R / NQ;                     // rank columns per slot thread
+  static constexpr int SS_PT = (RG * EPI_MAX_SS + THREADS - 1) / THREADS;
+};
+typedef Geo<9, 2> GeoQkv;     // 17-row draft pass: two row groups
+typedef Geo<9, 2> GeoResid;
+typedef Geo<9, 2> GeoSwiglu;
 
 // Row groups never straddle an m-tile of the GEMM (the part slots are per
 // m-tile): blockIdx.y = m-tile * groups_per_tile + group.  Returns false for
 // a group past the rows (whole CTA).
-__host__ __device__ __forceinline__ int epi_groups_per_tile(int NT, int M) {
-  return ((NT < M ? NT : M) + EPI_RG - 1) / EPI_RG;
+__host__ __device__ __forceinline__ int epi_groups_per_tile(int NT, int M, int RG) {
+  return ((NT < M ? NT : M) + RG - 1) / RG;
 }
+template <class G>
 __device__ __forceinline__ bool row_group(const EpiArgs& a, int* m0, int* nrows) {
-  const int gpt = epi_groups_per_tile(a.pv.NT, a.M);
+  const int gpt = epi_groups_per_tile(a.pv.NT, a.M, G::RG);
   const int mt = blockIdx.y / gpt, g = blockIdx.y % gpt;
-  *m0 = mt * a.pv.NT + g * EPI_RG;
+  *m0 = mt * a.pv.NT + g * G::RG;
   const int end = min(a.M, (mt + 1) * a.pv.NT);
-  *nrows = min(EPI_RG, end - *m0);
+  *nrows = min(G::RG, end - *m0);
   return *nrows > 0;
 }
 
@@ -107,47 +116,47 @@ __device__ __forceinline__ bool row_group(const EpiArgs& a, int* m0, int* nrows)
 // part_issue loads the first C contributors (issued before any use);
 // part_add adds them in CTA order, the first contributor's part first, then
 // reads any further contributors C at a time.
-template <int C>
+template <class G, int C>
 struct PartLoad {
-  float x[C][EPI_RPT];
-  int first, last;
-  const float* base; size_t slot;
+  float x[C][G::RPT];
+  int first, last, slot;             // slot: floats between contributors' parts
+  const float* base;
 };
-template <int C>
+template <class G, int C>
 __device__ __forceinline__ void part_issue(const PartView& v, int nt, int m0, int nrows, int col,
-                                           int q, PartLoad<C>& L) {
+                                           int q, PartLoad<G, C>& L) {
   const int mt = m0 / v.NT;
   const int t = nt * v.m_tiles + mt;
   L.first = sk_owner(t * v.KBt, v.units, v.grid);
   L.last = sk_owner(t * v.KBt + v.KBt - 1, v.units, v.grid);
-  L.slot = (size_t)v.NT * TC_BM;
+  L.slot = v.NT * TC_BM;
   L.base = v.ws + ((size_t)t * v.NT + (m0 - mt * v.NT) + q) * TC_BM + col;
 #pragma unroll
   for (int c = 0; c < C; ++c) {
     const int i = L.first + c;
 #pragma unroll
-    for (int s = 0; s < EPI_RPT; ++s)
-      L.x[c][s] = (i <= L.last && q + EPI_NQ * s < nrows)
-                      ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(EPI_NQ * s) * TC_BM) : 0.f;
+    for (int s = 0; s < G::RPT; ++s)
+      L.x[c][s] = (i <= L.last && q + G::NQ * s < nrows)
+                      ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(G::NQ * s) * TC_BM) : 0.f;
   }
 }
-template <int C>
-__device__ __forceinline__ void part_add(PartLoad<C>& L, int nrows, int q, float (&acc)[EPI_RPT]) {
+template <class G, int C>
+__device__ __forceinline__ void part_add(PartLoad<G, C>& L, int nrows, int q, float (&acc)[G::RPT]) {
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) acc[s] = 0.f;
+  for (int s = 0; s < G::RPT; ++s) acc[s] = 0.f;
   for (int i0 = L.first;; i0 += C) {
 #pragma unroll
     for (int c = 0; c < C; ++c)
 #pragma unroll
-      for (int s = 0; s < EPI_RPT; ++s) acc[s] += L.x[c][s];
+      for (int s = 0; s < G::RPT; ++s) acc[s] += L.x[c][s];
     if (i0 + C > L.last) break;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
       const int i = i0 + C + c;
 #pragma unroll
-      for (int s = 0; s < EPI_RPT; ++s)
-        L.x[c][s] = (i <= L.last && q + EPI_NQ * s < nrows)
-                        ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(EPI_NQ * s) * TC_BM) : 0.f;
+      for (int s = 0; s < G::RPT; ++s)
+        L.x[c][s] = (i <= L.last && q + G::NQ * s < nrows)
+                        ? __ldcg(L.base + (size_t)i * L.slot + (size_t)(G::NQ * s) * TC_BM) : 0.f;
     }
   }
 }
@@ -155,28 +164,29 @@ __device__ __forceinline__ void part_add(PartLoad<C>& L, int nrows, int q, float
 // Sums of squares of rows m0 .. m0 + nrows (all n_ss tiles of each): the
 // (row, tile) values are spread over the CTA's threads, all loads issued
 // together.
-constexpr int EPI_MAX_SS = 64;        // d_model <= 64 * 128
-constexpr int EPI_SS_PT = (EPI_RG * EPI_MAX_SS + EPI_THREADS - 1) / EPI_THREADS;
-struct SsLoad { float v[EPI_SS_PT]; };
-__device__ __forceinline__ void ss_issue(const EpiArgs& a, int m0, int nrows, SsLoad& L) {
+template <class G>
+struct SsLoad { float v[G::SS_PT]; };
+template <class G>
+__device__ __forceinline__ void ss_issue(const EpiArgs& a, int m0, int nrows, SsLoad<G>& L) {
 #pragma unroll
-  for (int k = 0; k < EPI_SS_PT; ++k) {
-    const int e = threadIdx.x + k * EPI_THREADS;
+  for (int k = 0; k < G::SS_PT; ++k) {
+    const int e = threadIdx.x + k * G::THREADS;
     L.v[k] = (a.ss && e < nrows * a.n_ss) ? __ldcg(a.ss + (size_t)m0 * a.n_ss + e) : 0.f;
   }
 }
 // 1 / sqrt(mean(x^2) + eps) per row into s_inv (tiles added in tile order);
 // 1 without a norm.  Syncs the CTA (twice).
-__device__ __forceinline__ void ss_finish(const EpiArgs& a, int nrows, const SsLoad& L, float* s_ss,
-                                          float* s_inv) {
+template <class G>
+__device__ __forceinline__ void ss_finish(const EpiArgs& a, int nrows, const SsLoad<G>& L,
+                                          float* s_ss, float* s_inv) {
 #pragma unroll
-  for (int k = 0; k < EPI_SS_PT; ++k) {
-    const int e = threadIdx.x + k * EPI_THREADS;
+  for (int k = 0; k < G::SS_PT; ++k) {
+    const int e = threadIdx.x + k * G::THREADS;
     if (e < nrows * a.n_ss) s_ss[e] = L.v[k];
   }
   __syncthreads();
   const int j = threadIdx.x;
-  if (j < EPI_RG) {
+  if (j < G::RG) {
     float inv = 1.f;
     if (a.ss && j < nrows) {
       float t = 0.f;
@@ -196,97 +206,126 @@ __device__ __forceinline__ int lora_seg(const LoraEpi& lr, int n) {
   return s;
 }
 
-// The thread's quarter of one adapter row: B[nb][q*EPI_KQ .. +EPI_KQ].
-struct BPart { uint4 b[EPI_KQ / 8]; };
-__device__ __forceinline__ void bpart_issue(const EpiArgs& a, int s, int nb, int q, BPart& B) {
-  const uint4* src = reinterpret_cast<const uint4*>(a.lr.Bl[s] + (size_t)nb * EPI_R + q * EPI_KQ);
+// The slot thread's share of one adapter row: B[nb][q KQ .. q KQ + KQ].
+template <class G>
+struct BPart { uint4 b[G::KQ / 8]; };
+template <class G>
+__device__ __forceinline__ void bpart_issue(const EpiArgs& a, int seg, int nb, int q, BPart<G>& B) {
+  const uint4* src = reinterpret_cast<const uint4*>(a.lr.Bl[seg] + (size_t)nb * EPI_R + q * G::KQ);
 #pragma unroll
-  for (int e = 0; e < EPI_KQ / 8; ++e) B.b[e] = __ldg(src + e);
+  for (int e = 0; e < G::KQ / 8; ++e) B.b[e] = __ldg(src + e);
 }
 
-// LoRA-B for column col: every thread forms the partial dot of its rank
-// quarter for all rows (sU[j][k] B[k]), the partials go through shared
-// memory and each thread adds the NQ quarters of its own rows in quarter
-// order: acc[s] += gate[s] * dot.  Syncs the CTA.
-__device__ __forceinline__ void lora_apply(const BPart& B, const float* sU, float* sDot, int col,
-                                           int q, int nrows, const float (&gate)[EPI_RPT],
-                                           float (&acc)[EPI_RPT]) {
-  float bf[EPI_KQ];
+// The same share into L2 only (one prefetch per 128-byte line).
+template <class G>
+__device__ __forceinline__ void bpart_prefetch(const EpiArgs& a, int seg, int nb, int q, const BPart<G>&) {
+  const char* src = reinterpret_cast<const char*>(a.lr.Bl[seg] + (size_t)nb * EPI_R + q * G::KQ);
 #pragma unroll
-  for (int e = 0; e < EPI_KQ / 8; ++e) {
+  for (int e = 0; e < G::KQ * 2; e += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + e));
+}
+
+// LoRA-B for column col: the slot thread forms the partial dot of its rank
+// share for every row (sU[j][k] B[k]); the NQ partials of the column are then
+// reduce-scattered over the slot lanes (shuffles, compile-time register
+// indices), so each row's sum is formed once, in a fixed order, by the thread
+// owning the row, which adds gate * dot.  sU must be complete (caller syncs).
+template <class G>
+__device__ __forceinline__ void lora_apply(const BPart<G>& B, const float* sU, int q, int nrows,
+                                           const float (&gate)[G::RPT], float (&acc)[G::RPT]) {
+  static_assert(G::NQ == 2 || G::NQ == 4, "two or four slot threads per column");
+  constexpr int RGP = G::RPT * G::NQ;       // rows padded to whole slot groups
+  float p[RGP];
+#pragma unroll
+  for (int j = 0; j < RGP; ++j) p[j] = 0.f;
+  // rank outer (eight adapter values unpacked at a time), rows inner
+#pragma unroll
+  for (int e = 0; e < G::KQ / 8; ++e) {
+    float bf[8];
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&B.b[e]);
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      bf[8 * e + 2 * h] = __low2float(b2[h]);
-      bf[8 * e + 2 * h + 1] = __high2float(b2[h]);
+      bf[2 * h] = __low2float(b2[h]);
+      bf[2 * h + 1] = __high2float(b2[h]);
+    }
+#pragma unroll
+    for (int j = 0; j < RGP; ++j) {
+      if (j < nrows) {
+        const float4* u4 = reinterpret_cast<const float4*>(sU + j * EPI_R + q * G::KQ + 8 * e);
+        const float4 x0 = u4[0], x1 = u4[1];
+        p[j] += x0.x * bf[0] + x0.y * bf[1] + x0.z * bf[2] + x0.w * bf[3] +
+                x1.x * bf[4] + x1.y * bf[5] + x1.z * bf[6] + x1.w * bf[7];
+      }
+    }
+  }
+  float tot[G::RPT];
+  if (G::NQ == 2) {
+    // rows 2s + r: slot r keeps row r, sends the other
+#pragma unroll
+    for (int s = 0; s < G::RPT; ++s) {
+      const float keep = q ? p[2 * s + 1] : p[2 * s], send = q ? p[2 * s] : p[2 * s + 1];
+      tot[s] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+  } else {
+    // rows 4s + r: first between slots q and q ^ 2 (keep r with the same bit 1
+    // as q), then between q and q ^ 1
+#pragma unroll
+    for (int s = 0; s < G::RPT; ++s) {
+      float h[2];
+#pragma unroll
+      for (int r1 = 0; r1 < 2; ++r1) {
+        const float keep = (q & 2) ? p[4 * s + 2 + r1] : p[4 * s + r1];
+        const float send = (q & 2) ? p[4 * s + r1] : p[4 * s + 2 + r1];
+        h[r1] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      const float keep = (q & 1) ? h[1] : h[0], send = (q & 1) ? h[0] : h[1];
+      tot[s] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
     }
   }
 #pragma unroll
-  for (int j = 0; j < EPI_RG; ++j) {
-    if (j >= nrows) break;
-    const float4* u4 = reinterpret_cast<const float4*>(sU + j * EPI_R + q * EPI_KQ);
-    float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < EPI_KQ / 4; k += 2) {
-      const float4 x0 = u4[k], x1 = u4[k + 1];
-      d0 += x0.x * bf[4 * k] + x0.y * bf[4 * k + 1] + x0.z * bf[4 * k + 2] + x0.w * bf[4 * k + 3];
-      d1 += x1.x * bf[4 * k + 4] + x1.y * bf[4 * k + 5] + x1.z * bf[4 * k + 6] + x1.w * bf[4 * k + 7];
-    }
-    sDot[(q * EPI_RG + j) * TC_BM + col] = d0 + d1;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
-    if (j < nrows) {
-      float t = 0.f;
-#pragma unroll
-      for (int qq = 0; qq < EPI_NQ; ++qq) t += sDot[(qq * EPI_RG + j) * TC_BM + col];
-      acc[s] += gate[s] * t;
-    }
-  }
+  for (int s = 0; s < G::RPT; ++s)
+    if (q + G::NQ * s < nrows) acc[s] += gate[s] * tot[s];
 }
 
-// The U tile of segment s, column col, the thread's rows: loads, then the
-// sums into sU[EPI_RG][EPI_R].  The caller syncs before sU is read.
-template <int C>
+// The U tile of segment seg, column col, the thread's rows: loads, then the
+// sums into sU[RG][EPI_R].  The caller syncs before sU is read.
+template <class G, int C>
 __device__ __forceinline__ void u_issue(const EpiArgs& a, int seg, int m0, int nrows, int col, int q,
-                                        PartLoad<C>& L) {
+                                        PartLoad<G, C>& L) {
   part_issue(a.pv, a.lr.u_tile0 + seg, m0, nrows, col, q, L);
 }
-template <int C>
-__device__ __forceinline__ void u_store(PartLoad<C>& L, int nrows, int col, int q, float* sU) {
-  float u[EPI_RPT];
+template <class G, int C>
+__device__ __forceinline__ void u_store(PartLoad<G, C>& L, int nrows, int col, int q, float* sU) {
+  float u[G::RPT];
   part_add(L, nrows, q, u);
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s)
-    if (q + EPI_NQ * s < nrows) sU[(q + EPI_NQ * s) * EPI_R + col] = u[s];
+  for (int s = 0; s < G::RPT; ++s)
+    if (q + G::NQ * s < nrows) sU[(q + G::NQ * s) * EPI_R + col] = u[s];
 }
 
 // Row gates of the thread's rows (0 past M).
+template <class G>
 __device__ __forceinline__ void gate_issue(const EpiArgs& a, int m0, int nrows, int q,
-                                           float (&g)[EPI_RPT]) {
+                                           float (&g)[G::RPT]) {
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s)
-    g[s] = q + EPI_NQ * s < nrows ? __ldg(a.lr.row_gate + m0 + q + EPI_NQ * s) : 0.f;
+  for (int s = 0; s < G::RPT; ++s)
+    g[s] = q + G::NQ * s < nrows ? __ldg(a.lr.row_gate + m0 + q + G::NQ * s) : 0.f;
 }
 
 // ---------------------------------------------------------------------------
-// q|k|v: grid ((H + 2 Hkv) hd / 128, row groups), EPI_THREADS threads.
+// q|k|v: grid ((H + 2 Hkv) hd / 128, row groups), GeoQkv::THREADS threads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(EPI_THREADS) epi_qkv_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs a) {
+  typedef GeoQkv G;
   constexpr int C = 4;
-  __shared__ float s_inv[EPI_RG];
-  __shared__ float s_ss[EPI_RG * EPI_MAX_SS];
-  __shared__ __align__(16) float sU[EPI_RG * EPI_R];
-  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
-  __shared__ float sY[EPI_RG][TC_BM];
+  __shared__ float s_inv[G::RG];
+  __shared__ float s_ss[G::RG * EPI_MAX_SS];
+  __shared__ __align__(16) float sU[G::RG * EPI_R];
+  __shared__ float sY[G::RG][TC_BM];
   pdl_trigger();
-  pdl_wait();
   const int nt = blockIdx.x;
   int m0, nrows;
-  if (!row_group(a, &m0, &nrows)) return;
-  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  if (!row_group<G>(a, &m0, &nrows)) return;
+  const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int n = nt * TC_BM + col;
   const int qcols = a.H * a.hd, kcols = a.Hkv * a.hd;
   const int half = a.hd / 2;
@@ -294,34 +333,36 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_qkv_kernel(const EpiArgs a) {
   const bool rot = n < qcols + kcols;      // q and k are rotated, v is not
   const bool kv_tile = n >= qcols;
   const int ci = hi < half ? hi : hi - half;
+  // the adapter row is a weight: read while the GEMM before is still running
+  const int seg = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
+  BPart<G> B;
+  if (a.lora) bpart_issue(a, seg, n - a.lr.seg_n0[seg], q, B);
+  pdl_wait();
 
   // ---- every global load first
-  int pos[EPI_RPT], slot[EPI_RPT];
+  int pos[G::RPT], slot[G::RPT];
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     pos[s] = j < nrows ? a.row_pos[m0 + j] : 0;
     slot[s] = (j < nrows && kv_tile) ? a.row_slot[m0 + j] : 0;
   }
-  SsLoad ssv;
+  SsLoad<G> ssv;
   ss_issue(a, m0, nrows, ssv);
-  const int seg = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
-  PartLoad<C> LU, LP;
-  BPart B;
-  float gate[EPI_RPT];
+  PartLoad<G, C> LU, LP;
+  float gate[G::RPT];
   if (a.lora) {
     u_issue(a, seg, m0, nrows, col, q, LU);
-    bpart_issue(a, seg, n - a.lr.seg_n0[seg], q, B);
-    gate_issue(a, m0, nrows, q, gate);
+    gate_issue<G>(a, m0, nrows, q, gate);
   }
   part_issue(a.pv, nt, m0, nrows, col, q, LP);
   // second round, addressed by the rows' positions and slots: RoPE table
   // entries and the KV pages
-  float cs[EPI_RPT], sn[EPI_RPT];
-  int page[EPI_RPT], pok[EPI_RPT];
+  float cs[G::RPT], sn[G::RPT];
+  int page[G::RPT], pok[G::RPT];
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     const int pc = (pos[s] >= 0 && pos[s] < a.max_pos) ? pos[s] : 0;
     cs[s] = rot ? a.cos_t[(size_t)pc * half + ci] : 0.f;
     sn[s] = rot ? a.sin_t[(size_t)pc * half + ci] : 0.f;
@@ -333,19 +374,19 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_qkv_kernel(const EpiArgs a) {
   // ---- then the arithmetic
   if (a.lora) u_store(LU, nrows, col, q, sU);
   ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
-  float acc[EPI_RPT];
+  float acc[G::RPT];
   part_add(LP, nrows, q, acc);
-  if (a.lora) lora_apply(B, sU, sDot, col, q, nrows, gate, acc);
+  if (a.lora) lora_apply<G>(B, sU, q, nrows, gate, acc);
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     if (j < nrows) sY[j][col] = acc[s] * s_inv[j];
   }
   __syncthreads();
 
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     if (j >= nrows) continue;
     const int m = m0 + j;
     const bool ok_pos = pos[s] >= 0 && pos[s] < a.max_pos;
@@ -376,124 +417,133 @@ __global__ void __launch_bounds__(EPI_THREADS) epi_qkv_kernel(const EpiArgs a) {
   }
 }
 
-// g * x rows for the next GEMM (hi/lo) and the tile's sums of squares of x.
+// g * x rows for the next GEMM (hi/lo) and the tile's sums of squares of x:
+// lanes of one slot add over the warp's columns, then the warps in order.
+template <class G>
 __device__ __forceinline__ void next_input(const EpiArgs& a, int nt, int m0, int nrows, int col,
-                                           int q, float g, const float (&xv)[EPI_RPT]) {
-  __shared__ float red[EPI_THREADS / 32][EPI_RPT];
+                                           int q, float g, const float (&xv)[G::RPT]) {
+  __shared__ float red[G::THREADS / 32][G::NQ][G::RPT];
   const int n = nt * TC_BM + col;
   bf16* lo = a.lo_off ? a.xn + (size_t)a.lo_off * a.ld_xn : nullptr;
-  float sq[EPI_RPT];
+  float sq[G::RPT];
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     sq[s] = xv[s] * xv[s];
     if (j < nrows) store_split<bf16>(a.xn, lo, (size_t)(m0 + j) * a.ld_xn + n, g * xv[s]);
   }
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) sq[s] = warp_sum(sq[s]);
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0)
+  for (int o = G::NQ; o < 32; o <<= 1)
 #pragma unroll
-    for (int s = 0; s < EPI_RPT; ++s) red[w][s] = sq[s];
+    for (int s = 0; s < G::RPT; ++s) sq[s] += __shfl_xor_sync(0xffffffffu, sq[s], o);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) < G::NQ)
+#pragma unroll
+    for (int s = 0; s < G::RPT; ++s) red[w][q][s] = sq[s];
   __syncthreads();
-  // row j = qq + NQ s lives in the 4 warps of slot qq
   const int j = threadIdx.x;
   if (j < nrows) {
-    const int qq = j % EPI_NQ, s = j / EPI_NQ;
+    const int qq = j % G::NQ, s = j / G::NQ;
     float t = 0.f;
 #pragma unroll
-    for (int k = 0; k < TC_BM / 32; ++k) t += red[qq * (TC_BM / 32) + k][s];
+    for (int k = 0; k < G::THREADS / 32; ++k) t += red[k][qq][s];
     a.ss_out[(size_t)(m0 + j) * (a.d / TC_BM) + nt] = t;
   }
 }
 
 // ---------------------------------------------------------------------------
 // o / down (and, with prep = 1, the layer-0 input): grid (d / 128, row
-// groups), EPI_THREADS threads.  x += y; then the next GEMM's input.
+// groups), GeoResid::THREADS threads.  x += y; then the next GEMM's input.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(EPI_THREADS) epi_resid_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiArgs a) {
+  typedef GeoResid G;
   constexpr int C = 6;
-  __shared__ __align__(16) float sU[EPI_RG * EPI_R];
-  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
+  __shared__ __align__(16) float sU[G::RG * EPI_R];
   pdl_trigger();
-  pdl_wait();
   const int nt = blockIdx.x;
   int m0, nrows;
-  if (!row_group(a, &m0, &nrows)) return;
-  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  if (!row_group<G>(a, &m0, &nrows)) return;
+  const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int n = nt * TC_BM + col;
+  // weights (the next norm's gain, the adapter row) before the dependency wait
+  const float g = a.g_next ? to_f(a.g_next[n]) : 0.f;
+  BPart<G> B;
+  if (!a.prep && a.lora) bpart_issue(a, 0, n, q, B);
+  pdl_wait();
 
   // ---- every global load first
-  float xv[EPI_RPT];
+  float xv[G::RPT];
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     xv[s] = j < nrows ? a.x[(size_t)(m0 + j) * a.d + n] : 0.f;
   }
-  const float g = a.g_next ? to_f(a.g_next[n]) : 0.f;
   if (!a.prep) {
-    PartLoad<C> LU, LP;
-    BPart B;
-    float gate[EPI_RPT];
+    PartLoad<G, C> LU, LP;
+    float gate[G::RPT];
     if (a.lora) {
       u_issue(a, 0, m0, nrows, col, q, LU);
-      bpart_issue(a, 0, n, q, B);
-      gate_issue(a, m0, nrows, q, gate);
+      gate_issue<G>(a, m0, nrows, q, gate);
     }
     part_issue(a.pv, nt, m0, nrows, col, q, LP);
     // ---- then the arithmetic
-    float acc[EPI_RPT];
+    float acc[G::RPT];
     if (a.lora) {
       u_store(LU, nrows, col, q, sU);
       __syncthreads();
     }
     part_add(LP, nrows, q, acc);
-    if (a.lora) lora_apply(B, sU, sDot, col, q, nrows, gate, acc);
+    if (a.lora) lora_apply<G>(B, sU, q, nrows, gate, acc);
 #pragma unroll
-    for (int s = 0; s < EPI_RPT; ++s) {
-      const int j = q + EPI_NQ * s;
+    for (int s = 0; s < G::RPT; ++s) {
+      const int j = q + G::NQ * s;
       xv[s] += acc[s];
       if (j < nrows) a.x[(size_t)(m0 + j) * a.d + n] = xv[s];
     }
   }
-  if (a.g_next) next_input(a, nt, m0, nrows, col, q, g, xv);
+  if (a.g_next) next_input<G>(a, nt, m0, nrows, col, q, g, xv);
 }
 
 // ---------------------------------------------------------------------------
-// gate|up -> silu(gate) * up: grid (F / 128, row groups), EPI_THREADS
+// gate|up -> silu(gate) * up: grid (F / 128, row groups), GeoSwiglu::THREADS
 // threads; each thread takes the gate and the up column of one feature.
+// Two CTAs per SM (one wave for the decode passes' 2 x F / 128 CTAs): up's
+// adapter half is read after gate's dot.  Gate|up tiles have at most two
+// contributors at these sizes (more take further rounds).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(EPI_THREADS, 2) epi_swiglu_kernel(const EpiArgs a) {
-  // two CTAs per SM (one wave for the decode passes' 2 x F / 128 CTAs): up's
-  // adapter half is read after gate's dot, and gate|up tiles have at most two
-  // contributors at these sizes (more take further rounds)
+__global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const EpiArgs a) {
+  typedef GeoSwiglu G;
   constexpr int C = 2;
-  __shared__ float s_inv[EPI_RG];
-  __shared__ float s_ss[EPI_RG * EPI_MAX_SS];
-  __shared__ __align__(16) float sU[2][EPI_RG * EPI_R];
-  __shared__ float sDot[EPI_NQ * EPI_RG * TC_BM];
+  __shared__ float s_inv[G::RG];
+  __shared__ float s_ss[G::RG * EPI_MAX_SS];
+  __shared__ __align__(16) float sU[2][G::RG * EPI_R];
   pdl_trigger();
-  pdl_wait();
   const int ft = blockIdx.x;
   int m0, nrows;
-  if (!row_group(a, &m0, &nrows)) return;
-  const int col = threadIdx.x % TC_BM, q = threadIdx.x / TC_BM;
+  if (!row_group<G>(a, &m0, &nrows)) return;
+  const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int f = ft * TC_BM + col;
   const int ut = a.F / TC_BM + ft;         // the up tile of the same features
+  // adapter rows are weights: gate's into registers and up's into L2 while
+  // the GEMM before is still running
+  BPart<G> B;
+  if (a.lora) {
+    bpart_issue(a, 0, f, q, B);
+    bpart_prefetch(a, 1, f, q, B);
+  }
+  pdl_wait();
 
-  // ---- the global loads (up's adapter half comes after gate's dot)
-  SsLoad ssv;
+  // ---- every global load first
+  SsLoad<G> ssv;
   ss_issue(a, m0, nrows, ssv);
-  PartLoad<C> LG, LUp, L0, L1;
-  BPart B;
-  float gate[EPI_RPT];
+  PartLoad<G, C> LG, LUp, L0, L1;
+  float gate[G::RPT];
   part_issue(a.pv, ft, m0, nrows, col, q, LG);
   part_issue(a.pv, ut, m0, nrows, col, q, LUp);
   if (a.lora) {
     u_issue(a, 0, m0, nrows, col, q, L0);
     u_issue(a, 1, m0, nrows, col, q, L1);
-    bpart_issue(a, 0, f, q, B);
-    gate_issue(a, m0, nrows, q, gate);
+    gate_issue<G>(a, m0, nrows, q, gate);
   }
   // ---- then the arithmetic
   if (a.lora) {
@@ -501,19 +551,18 @@ __global__ void __launch_bounds__(EPI_THREADS, 2) epi_swiglu_kernel(const EpiArg
     u_store(L1, nrows, col, q, sU[1]);
   }
   ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
-  float g[EPI_RPT], u[EPI_RPT];
+  float g[G::RPT], u[G::RPT];
   part_add(LG, nrows, q, g);
   part_add(LUp, nrows, q, u);
   if (a.lora) {
-    lora_apply(B, sU[0], sDot, col, q, nrows, gate, g);
-    bpart_issue(a, 1, f, q, B);
-    __syncthreads();                         // sDot is reused
-    lora_apply(B, sU[1], sDot, col, q, nrows, gate, u);
+    lora_apply<G>(B, sU[0], q, nrows, gate, g);
+    bpart_issue(a, 1, f, q, B);              // up's adapter half after gate's dot
+    lora_apply<G>(B, sU[1], q, nrows, gate, u);
   }
   bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
 #pragma unroll
-  for (int s = 0; s < EPI_RPT; ++s) {
-    const int j = q + EPI_NQ * s;
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
     if (j < nrows) {
       const float gv = g[s] * s_inv[j], uv = u[s] * s_inv[j];
       store_split<bf16>(a.h, lo, (size_t)(m0 + j) * a.F + f, gv / (1.0f + expf(-gv)) * uv);

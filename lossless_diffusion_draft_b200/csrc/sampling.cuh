@@ -17,8 +17,9 @@
 // (request, chunk), whose last CTA draws the token.  No CTA ever waits on
 // another, so nothing can hang.
 //
-// Inverse-CDF sampling on the device: w_v = expf(l_v - M) with M the row max;
-// Z = sum over chunks (in chunk order) of s_k * expf(m_k - M); the token is in
+// Inverse-CDF sampling on the device: w_v = exp(l_v - M) with M the row max
+// (exp_rel below); Z = sum over chunks (a chunk-order scan) of
+// s_k * expf(m_k - M), s_k the chunk's sum relative to its own max m_k; the token is in
 // the first chunk whose running prefix exceeds u * Z, at the first element
 // whose within-chunk inclusive prefix (thread-contiguous order, fixed) pushes
 // the running sum above u * Z.  When rounding leaves no crossing, the last
@@ -33,19 +34,29 @@ namespace uno {
 
 constexpr int SAMPLE_THREADS = 256;
 
+// exp(x - m) as 2^(x log2 e - m log2 e): one FMA (mL = m log2 e, computed
+// once per row or chunk) and the special-function unit's ex2.approx (about
+// 2 ulp).  The rounding of mL scales every weight of the row or chunk by the
+// same factor (relative 1e-6 at |m| ~ 20), which the normaliser divides out.
+// Every per-logit exponential of this file goes through here, so the chunk
+// sums and the element weights of the crossing scan use the same values.
+constexpr float SAMPLE_LOG2E = 1.4426950408889634f;
+__device__ __forceinline__ float exp_rel(float x, float mL) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(fmaf(x, SAMPLE_LOG2E, -mL)));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
-// Phase A: reduce one chunk of one row to (max, sum exp(l - max)).  Each
-// thread reduces its own logits to a (max, sum) pair; the pairs are combined
-// across the CTA in a fixed tree (warp butterfly, then the warps in order),
-// so one reduction serves both statistics.
+// Phase A: reduce one chunk of one row to (max, sum exp(l - max)).  The
+// CTA's max comes first (warp butterfly, then the warps' maxima in order),
+// then every logit takes one exponential against it and the sums are added
+// by a butterfly and the warps in order: a fixed tree, and no rescaling.
 // ---------------------------------------------------------------------------
 constexpr int CHUNK_IT = 8;   // float4 per thread: a chunk holds <= 8 * 4 * 256 = 8192 logits
-__device__ __forceinline__ float2 ms_combine(float2 a, float2 b) {
-  const float M = fmaxf(a.x, b.x);
-  if (M == -INFINITY) return make_float2(M, 0.f);
-  return make_float2(M, a.y * expf(a.x - M) + b.y * expf(b.x - M));
-}
+// red: at least 2 * SAMPLE_THREADS / 32 floats of shared memory.
 __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red) {
+  constexpr int NW = SAMPLE_THREADS / 32;
   // float4 path: rows start on 16-byte boundaries (vocab % 4 == 0 is required)
   const int n4 = (c1 - c0) >> 2;
   const float4* r4 = reinterpret_cast<const float4*>(row + c0);
@@ -61,58 +72,117 @@ __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1,
   }
   // scalar tail (chunk length not a multiple of 4: only the row's last chunk)
   for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) m = fmaxf(m, row[j]);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();                                    // red may hold a previous reduction
+  if (lane == 0) red[wid] = m;
+  __syncthreads();
+  float M = red[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
   float s = 0.f;
-  if (m != -INFINITY) {
+  if (M != -INFINITY) {
+    const float mL = M * SAMPLE_LOG2E;
 #pragma unroll
     for (int i = 0; i < CHUNK_IT; ++i) {
       const int j = threadIdx.x + i * SAMPLE_THREADS;
-      if (j < n4) s += expf(v[i].x - m) + expf(v[i].y - m) + expf(v[i].z - m) + expf(v[i].w - m);
+      if (j < n4)
+        s += (exp_rel(v[i].x, mL) + exp_rel(v[i].y, mL)) + (exp_rel(v[i].z, mL) + exp_rel(v[i].w, mL));
     }
-    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += expf(row[j] - m);
+    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += exp_rel(row[j], mL);
   }
-  float2 ms = make_float2(m, s);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-    ms = ms_combine(ms, make_float2(__shfl_xor_sync(0xffffffffu, ms.x, o),
-                                    __shfl_xor_sync(0xffffffffu, ms.y, o)));
-  float2* red2 = reinterpret_cast<float2*>(red);     // SAMPLE_THREADS / 32 pairs
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  __syncthreads();                                    // red may hold a previous reduction
-  if (lane == 0) red2[wid] = ms;
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[NW + wid] = s;                   // other slots than the maxima
   __syncthreads();
-  float2 t = red2[0];
+  float S = 0.f;
 #pragma unroll
-  for (int w = 1; w < SAMPLE_THREADS / 32; ++w) t = ms_combine(t, red2[w]);
-  return t;
+  for (int w = 0; w < NW; ++w) S += red[NW + w];
+  return make_float2(M, S);
 }
 
-// Row-level combine of chunk pairs (run by one thread, chunk order).
-struct RowStat { float M, Z; };
-__device__ __forceinline__ RowStat combine_row(const float2* part, int nch) {
-  float M = -INFINITY;
-  for (int k = 0; k < nch; ++k) M = fmaxf(M, __ldcg(&part[k].x));
-  float Z = 0.f;
-  for (int k = 0; k < nch; ++k) {
-    const float2 pk = __ldcg(&part[k]);
-    if (pk.x != -INFINITY) Z += pk.y * expf(pk.x - M);
+// Chunk-level prefix in chunk order, run by one whole warp: lane l holds
+// chunks l, l + 32, ...; each group of 32 is scanned with shuffles (fixed
+// tree) and carried into the next.  Returns on every lane: the first chunk
+// whose inclusive prefix exceeds `target` (-1 if none) with its exclusive
+// prefix, the last chunk of positive weight (-1 if none) and the total.
+// Every caller that needs the row's Z and its running prefix goes through
+// this one routine, so the two agree bit for bit.
+struct ChunkPick { int k; float base; int lastk; float total; };
+template <typename F>
+__device__ __forceinline__ ChunkPick warp_chunk_pick(const F& wk, int nch, float target) {
+  const int lane = threadIdx.x & 31;
+  ChunkPick r{-1, 0.f, -1, 0.f};
+  float carry = 0.f;
+  for (int g = 0; g < nch; g += 32) {
+    const int c = g + lane;
+    const float w = c < nch ? wk(c) : 0.f;
+    float incl = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.f;
+    incl += carry;
+    excl += carry;
+    const unsigned hit = __ballot_sync(0xffffffffu, c < nch && incl > target);
+    if (r.k < 0 && hit) {
+      const int l = __ffs(hit) - 1;
+      r.k = g + l;
+      r.base = __shfl_sync(0xffffffffu, excl, l);
+    }
+    const unsigned pos = __ballot_sync(0xffffffffu, c < nch && w > 0.f);
+    if (pos) r.lastk = g + 31 - __clz(pos);
+    carry = __shfl_sync(0xffffffffu, incl, 31);
   }
-  return {M, Z};
+  r.total = carry;
+  return r;
+}
+
+// Weight of chunk k relative to the row max M: s_k * exp(m_k - M).
+struct ChunkW {
+  const float2* part; float M;
+  __device__ __forceinline__ float operator()(int k) const {
+    const float2 pk = __ldcg(&part[k]);
+    return pk.x != -INFINITY ? pk.y * expf(pk.x - M) : 0.f;
+  }
+};
+
+// Row-level combine of chunk pairs (one whole warp; the result on every lane).
+struct RowStat { float M, Z; };
+// Plain per-chunk sums (the residual's).
+struct PartW {
+  const float* s;
+  __device__ __forceinline__ float operator()(int k) const { return __ldcg(&s[k]); }
+};
+__device__ __forceinline__ RowStat combine_row(const float2* part, int nch) {
+  const int lane = threadIdx.x & 31;
+  float M = -INFINITY;
+  for (int k = lane; k < nch; k += 32) M = fmaxf(M, __ldcg(&part[k].x));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (M == -INFINITY) return {M, 0.f};
+  const ChunkPick cp = warp_chunk_pick(ChunkW{part, M}, nch, INFINITY);
+  return {M, cp.total};
 }
 
 // Weight functors used by the crossing scan (get4: four weights from v, a
 // multiple of 4).
 struct SoftmaxW {
-  const float* row; float M;
-  __device__ __forceinline__ float operator()(int v) const { return expf(row[v] - M); }
+  const float* row; float ML;          // row max x log2 e
+  __device__ __forceinline__ float operator()(int v) const { return exp_rel(row[v], ML); }
   __device__ __forceinline__ void get4(int v, float* w) const {
     const float4 x = *reinterpret_cast<const float4*>(row + v);
-    w[0] = expf(x.x - M); w[1] = expf(x.y - M); w[2] = expf(x.z - M); w[3] = expf(x.w - M);
+    w[0] = exp_rel(x.x, ML); w[1] = exp_rel(x.y, ML); w[2] = exp_rel(x.z, ML); w[3] = exp_rel(x.w, ML);
   }
 };
 struct ResidW {
-  const float* p; const float* q; float lse_p, lse_q;
+  const float* p; const float* q; float lpL, lqL;   // lse_p, lse_q x log2 e
   __device__ __forceinline__ float pair(float pv, float qv) const {
-    const float d = expf(pv - lse_p) - expf(qv - lse_q);
+    const float d = exp_rel(pv, lpL) - exp_rel(qv, lqL);
     return d > 0.f ? d : 0.f;
   }
   __device__ __forceinline__ float operator()(int v) const { return pair(p[v], q[v]); }
@@ -187,28 +257,19 @@ __device__ int sample_from_partials(const float* row, const float2* part, int nc
                                     const RowStat& rs, float u, float* red) {
   __shared__ int s_k;
   __shared__ float s_base;
-  __shared__ int s_lastk;
   const float target = u * rs.Z;
-  if (threadIdx.x == 0) {
-    float run = 0.f;
-    int kk = -1, lastk = -1;
-    for (int k = 0; k < nch; ++k) {
-      const float2 pk = __ldcg(&part[k]);
-      const float sk = (pk.x != -INFINITY) ? pk.y * expf(pk.x - rs.M) : 0.f;
-      if (sk > 0.f) lastk = k;
-      if (kk < 0 && run + sk > target) { kk = k; s_base = run; }
-      run += sk;
-    }
-    if (kk < 0) { kk = lastk; s_base = 0.f; }
-    s_k = kk;
-    s_lastk = lastk;
+  if (threadIdx.x < 32) {
+    ChunkPick cp{-1, 0.f, -1, 0.f};
+    if (rs.M != -INFINITY) cp = warp_chunk_pick(ChunkW{part, rs.M}, nch, target);
+    if (cp.k < 0) { cp.k = cp.lastk; cp.base = 0.f; }
+    if (threadIdx.x == 0) { s_k = cp.k; s_base = cp.base; }
   }
   __syncthreads();
   const int k = s_k;
   const float base = s_base;
   __syncthreads();
   if (k < 0) return 0;  // empty row (all -inf): only reachable with invalid logits
-  SoftmaxW w{row, rs.M};
+  SoftmaxW w{row, rs.M * SAMPLE_LOG2E};
   int lastpos;
   const int c0 = k * ch, c1 = min(V, c0 + ch);
   int t = chunk_crossing(w, c0, c1, base, target, &lastpos, red);
@@ -262,7 +323,10 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   __threadfence();
   const float2* part = a.partial + (size_t)rid * a.nch;
   __shared__ RowStat s_rs;
-  if (threadIdx.x == 0) s_rs = combine_row(part, a.nch);
+  if (threadIdx.x < 32) {
+    const RowStat rs = combine_row(part, a.nch);
+    if (threadIdx.x == 0) s_rs = rs;
+  }
   __syncthreads();
   const RowStat rs = s_rs;
   const int slot = a.req_slot[req];
@@ -359,45 +423,11 @@ __device__ void verify_finish(const VerifyArgs& a, int req, int slot, int pos0, 
   }
 }
 
-__global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const VerifyArgs a) {
-  __shared__ float red[32];
-  __shared__ bool s_last;
+// The decision of request req once every reduced row's lse is in a.lse
+// (whole CTA): the accept tests, the first rejection, and either the bonus
+// draw and the commit here or the hand-over to spec_resid_kernel.
+__device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
   __shared__ int s_a;
-  pdl_trigger();
-  pdl_wait();
-  const int k = blockIdx.x;
-  const int rid = blockIdx.y;
-  const int req = rid / a.rows_red, r = rid % a.rows_red;
-  const float* row;
-  if (r < a.n_p) {
-    const int br = (r < a.n_tests) ? a.p_row0 + r : a.bonus_row;
-    row = a.p + ((size_t)req * a.p_req_rows + br) * a.V;
-  } else {
-    row = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + (r - a.n_p)) * a.V;
-  }
-  const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
-  const float2 pr = reduce_chunk(row, c0, c1, red);
-  if (threadIdx.x == 0) {
-    a.partial[(size_t)rid * a.nch + k] = pr;
-    __threadfence();
-    const unsigned done = atomicAdd(&a.row_counter[rid], 1u);
-    bool last = (done == (unsigned)a.nch - 1);
-    if (last) {
-      a.row_counter[rid] = 0u;
-      const RowStat rs = combine_row(a.partial + (size_t)rid * a.nch, a.nch);
-      a.lse[rid] = rs.M + logf(rs.Z);
-      __threadfence();
-      const unsigned rdone = atomicAdd(&a.req_counter[req], 1u);
-      last = (rdone == (unsigned)a.rows_red - 1);
-      if (last) a.req_counter[req] = 0u;
-    }
-    s_last = last;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // ---- request decision (one CTA per request) ----
   const size_t rbase = (size_t)req * a.rows_red;
   int slot, pos0;
   uint32_t stream;
@@ -427,13 +457,98 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const Ve
     const float* prow = a.p + ((size_t)req * a.p_req_rows + a.bonus_row) * a.V;
     const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + a.n_tests), KIND_RESID);
     __shared__ RowStat s_rs2;
-    if (threadIdx.x == 0) s_rs2 = combine_row(a.partial + (rbase + a.n_tests) * a.nch, a.nch);
+    if (threadIdx.x < 32) {
+      const RowStat rs = combine_row(a.partial + (rbase + a.n_tests) * a.nch, a.nch);
+      if (threadIdx.x == 0) s_rs2 = rs;
+    }
     __syncthreads();
     y = sample_from_partials(prow, a.partial + (rbase + a.n_tests) * a.nch, a.nch, a.ch, a.V,
                              s_rs2, u, red);
   }
   if (threadIdx.x == 0) a.at_ws[req] = -1;
   verify_finish(a, req, slot, pos0, at, y);
+}
+
+// The row a (request, reduced row) CTA reads.
+__device__ __forceinline__ const float* verify_row(const VerifyArgs& a, int req, int r) {
+  if (r < a.n_p) {
+    const int br = (r < a.n_tests) ? a.p_row0 + r : a.bonus_row;
+    return a.p + ((size_t)req * a.p_req_rows + br) * a.V;
+  }
+  return a.q + ((size_t)req * a.q_req_rows + a.q_row0 + (r - a.n_p)) * a.V;
+}
+
+// Fused form (few rows): grid (nch, n_req * rows_red).  The last chunk CTA
+// of a row forms its lse, the last row of a request decides.
+__global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const VerifyArgs a) {
+  __shared__ float red[32];
+  __shared__ bool s_last, s_req_last;
+  pdl_trigger();
+  pdl_wait();
+  const int k = blockIdx.x;
+  const int rid = blockIdx.y;
+  const int req = rid / a.rows_red, r = rid % a.rows_red;
+  const float* row = verify_row(a, req, r);
+  const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
+  const float2 pr = reduce_chunk(row, c0, c1, red);
+  if (threadIdx.x == 0) {
+    a.partial[(size_t)rid * a.nch + k] = pr;
+    __threadfence();
+    const unsigned done = atomicAdd(&a.row_counter[rid], 1u);
+    s_last = (done == (unsigned)a.nch - 1);
+    if (s_last) a.row_counter[rid] = 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // last chunk of the row: its lse; the last row of the request decides
+  if (threadIdx.x < 32) {
+    const RowStat rs = combine_row(a.partial + (size_t)rid * a.nch, a.nch);
+    if (threadIdx.x == 0) {
+      a.lse[rid] = rs.M + logf(rs.Z);
+      __threadfence();
+      const unsigned rdone = atomicAdd(&a.req_counter[req], 1u);
+      s_req_last = (rdone == (unsigned)a.rows_red - 1);
+      if (s_req_last) a.req_counter[req] = 0u;
+    }
+  }
+  __syncthreads();
+  if (!s_req_last) return;
+  __threadfence();
+  verify_decide(a, req, red);
+}
+
+// Split form (many rows), first kernel: grid (nch, n_req * rows_red), every
+// CTA reduces its chunk, writes the pair and exits (no counters, no waiting
+// on a round trip), so the loads of the next CTAs keep HBM busy.
+__global__ void __launch_bounds__(SAMPLE_THREADS, 4) spec_reduce_kernel(const VerifyArgs a) {
+  __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
+  const int k = blockIdx.x;
+  const int rid = blockIdx.y;
+  const float* row = verify_row(a, rid / a.rows_red, rid % a.rows_red);
+  const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
+  const float2 pr = reduce_chunk(row, c0, c1, red);
+  if (threadIdx.x == 0) a.partial[(size_t)rid * a.nch + k] = pr;
+}
+
+// Split form, second kernel: one CTA per request; warp w forms the lse of
+// rows w, w + 8, ... (the same chunk-order combine as the fused form), then
+// the CTA decides.
+__global__ void __launch_bounds__(SAMPLE_THREADS) spec_decide_kernel(const VerifyArgs a) {
+  __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
+  const int req = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  for (int r = warp; r < a.rows_red; r += SAMPLE_THREADS / 32) {
+    const size_t rid = (size_t)req * a.rows_red + r;
+    const RowStat rs = combine_row(a.partial + rid * a.nch, a.nch);
+    if ((threadIdx.x & 31) == 0) a.lse[rid] = rs.M + logf(rs.Z);
+  }
+  __syncthreads();
+  verify_decide(a, req, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -458,7 +573,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
   const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + at) * a.V;
   const float lse_p = __ldcg(&a.lse[rbase + at]);
   const float lse_q = verify_lse_q(a, req, at);
-  const ResidW w{prow, qrow, lse_p, lse_q};
+  const ResidW w{prow, qrow, lse_p * SAMPLE_LOG2E, lse_q * SAMPLE_LOG2E};
   {
     // chunk sum: 16-byte loads, all of a thread's loads issued first
     const int b0 = k * a.ch, b1 = min(a.V, b0 + a.ch);
@@ -503,23 +618,14 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
   const float* cs = a.resid_part + (size_t)req * a.nch;
   __shared__ float s_Z, s_base;
   __shared__ int s_k;
-  if (threadIdx.x == 0) {
-    float Z = 0.f;
-    for (int c = 0; c < a.nch; ++c) Z += __ldcg(&cs[c]);
-    const float target = u * Z;
-    float run = 0.f;
-    int kk = -1, lastk = -1;
-    float base = 0.f;
-    for (int c = 0; c < a.nch; ++c) {
-      const float sk = __ldcg(&cs[c]);
-      if (sk > 0.f) lastk = c;
-      if (kk < 0 && run + sk > target) { kk = c; base = run; }
-      run += sk;
-    }
-    if (kk < 0) { kk = lastk; base = 0.f; }
-    s_Z = Z;
-    s_k = kk;
-    s_base = base;
+  if (threadIdx.x < 32) {
+    // Z and the crossing chunk come from one chunk-order scan; the target
+    // u * Z needs Z first, so the scan runs twice (the second only reads)
+    const PartW pw{cs};
+    const float Z = warp_chunk_pick(pw, a.nch, INFINITY).total;
+    ChunkPick cp = warp_chunk_pick(pw, a.nch, u * Z);
+    if (cp.k < 0) { cp.k = cp.lastk; cp.base = 0.f; }
+    if (threadIdx.x == 0) { s_Z = Z; s_k = cp.k; s_base = cp.base; }
   }
   __syncthreads();
   const float Z = s_Z;
@@ -532,7 +638,10 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
   } else {
     // no residual mass after rounding: draw from p
     __shared__ RowStat s_rs;
-    if (threadIdx.x == 0) s_rs = combine_row(a.partial + (rbase + at) * a.nch, a.nch);
+    if (threadIdx.x < 32) {
+      const RowStat rs = combine_row(a.partial + (rbase + at) * a.nch, a.nch);
+      if (threadIdx.x == 0) s_rs = rs;
+    }
     __syncthreads();
     y = sample_from_partials(prow, a.partial + (rbase + at) * a.nch, a.nch, a.ch, a.V, s_rs, u, red);
   }

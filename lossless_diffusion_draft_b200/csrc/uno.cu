@@ -93,6 +93,24 @@ void klaunch(bool pdl, cudaStream_t st, dim3 grid, dim3 block, size_t smem,
   cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// spec_verify's first stage.  Few (row, chunk) CTAs: the fused kernel (the
+// last CTA of a row forms its lse, the last row decides; one launch).  Many:
+// the reduction CTAs carry no counters and exit at once, and one CTA per
+// request combines and decides (one launch more, HBM kept busy).
+constexpr long long VERIFY_SPLIT_CTAS = 4096;
+// Returns the number of kernels launched.
+int launch_verify(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req,
+                  long long split_ctas = VERIFY_SPLIT_CTAS) {
+  const dim3 grid(a.nch, n_req * a.rows_red);
+  if ((long long)a.nch * n_req * a.rows_red <= split_ctas) {
+    klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_verify_kernel, a);
+    return 1;
+  }
+  klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_reduce_kernel, a);
+  klaunch(pdl, st, dim3(n_req), dim3(SAMPLE_THREADS), 0, spec_decide_kernel, a);
+  return 2;
+}
+
 struct GemmEnv {
   int sm_count = 148;
   int x_rows_alloc = 0;           // rows the activation buffers hold (>= any box)
@@ -331,6 +349,7 @@ struct uno_ctx {
   float* ss = nullptr;         // [M, d / 128] sums of squares of x per 128-column tile
   bool fused = false;          // the fused bf16 layer pipeline applies to this model
   bool fused_enabled = true;
+  int verify_split_ctas = 4096;   // spec_verify: split form above this many CTAs
   int32_t *row_pos = nullptr, *row_slot = nullptr;
   float* row_gate = nullptr;
   float *cos_t = nullptr, *sin_t = nullptr;
@@ -898,10 +917,12 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
       ea.lr.nseg++;
     }
   };
-  auto epi = [&](void (*kernel)(const EpiArgs), int tiles) {
+  // one epilogue launch: rg rows per CTA (row groups inside the GEMM's
+  // m-tiles), `threads` threads
+  auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int rg, int threads) {
     Prof prof(c, UNO_K_OTHER, 0.0);
-    const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M);
-    klaunch(pdl, st, dim3(tiles, groups), dim3(EPI_THREADS), 0, kernel, ea);
+    const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M, rg);
+    klaunch(pdl, st, dim3(tiles, groups), dim3(threads), 0, kernel, ea);
   };
 
   // layer-0 input: g * x and the sums of squares of the embedding rows
@@ -909,7 +930,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ea.lora = 0;
   ea.pv = PartView{nullptr, M, 0, 1, 1, 1};
   ea.g_next = (const bf16*)c->attn_norm[0];
-  epi(epi_resid_kernel, d / TC_BM);
+  epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
   ea.prep = 0;
 
   for (int l = 0; l < s.n_layers; ++l) {
@@ -922,7 +943,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_Q][l], H * hd}, {c->lB[UNO_PROJ_K][l], Hkv * hd},
               {c->lB[UNO_PROJ_V][l], Hkv * hd}});
     ea.ss = c->ss;
-    epi(epi_qkv_kernel, qkv_n / TC_BM);
+    epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS);
 
     rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo);
     if (rc) return rc;
@@ -932,21 +953,21 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_O][l], d}});
     ea.ss = nullptr;
     ea.g_next = (const bf16*)c->ffn_norm[l];
-    epi(epi_resid_kernel, d / TC_BM);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
 
     rc = gemm(c->xn, xn_ld, d, {{c->w[UNO_PROJ_GATE][l], F}, {c->w[UNO_PROJ_UP][l], F}},
               {c->lA[UNO_PROJ_GATE][l], c->lA[UNO_PROJ_UP][l]}, &ea.pv);
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_GATE][l], F}, {c->lB[UNO_PROJ_UP][l], F}});
     ea.ss = c->ss;
-    epi(epi_swiglu_kernel, F / TC_BM);
+    epi(epi_swiglu_kernel, F / TC_BM, GeoSwiglu::RG, GeoSwiglu::THREADS);
 
     rc = gemm(c->xn, F, F, {{c->w[UNO_PROJ_DOWN][l], d}}, {c->lA[UNO_PROJ_DOWN][l]}, &ea.pv);
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_DOWN][l], d}});
     ea.ss = nullptr;
     ea.g_next = l + 1 < s.n_layers ? (const bf16*)c->attn_norm[l + 1] : nullptr;
-    epi(epi_resid_kernel, d / TC_BM);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
   }
   if (logits) {
     bf16* xn_lo = split ? (bf16*)c->xn + (size_t)lo * xn_ld : nullptr;
@@ -1400,8 +1421,7 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.status = c->d_status;
     {
       Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
-      klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
-              spec_verify_kernel, a);
+      c->prof_launches[UNO_K_VERIFY] += launch_verify(c->genv.pdl, c->stream, a, n_req, c->verify_split_ctas) - 1;
     }
     {
       Prof prof(c, UNO_K_VERIFY, (double)n_req * 2 * V * 4);
@@ -1493,6 +1513,17 @@ int uno_set_fused(uno_ctx* c, int enable) {
     g.seen = 0;
   }
   return c->fused ? UNO_OK : UNO_ERR_UNSUPPORTED;
+}
+
+int uno_set_verify_split(uno_ctx* c, int max_ctas) {
+  if (!c || max_ctas < 0) return UNO_ERR_ARG;
+  c->verify_split_ctas = max_ctas;
+  for (auto& g : c->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.seen = 0;
+  }
+  return UNO_OK;
 }
 
 int uno_profile_records(uno_ctx* c, uno_prof_record* out, int max) {
@@ -1749,8 +1780,7 @@ int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n
   a.rows_red = 2 * n_tests;
   a.n_p = n_tests;
   a.status = nullptr;
-  const int rows = n_req * 2 * n_tests;
-  spec_verify_kernel<<<dim3(nch, rows), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
+  launch_verify(false, (cudaStream_t)stream, a, n_req);
   spec_resid_kernel<<<dim3(nch, n_req), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }

@@ -25,7 +25,7 @@ import parity
 pytestmark = pytest.mark.gpu
 
 
-def _setup(name, n_req, prompt_len, max_ctx, fused=True, **over):
+def _setup(name, n_req, prompt_len, max_ctx, fused=True, verify_split=None, **over):
     cfg = dict(synth.CONFIGS[name], **over)
     shape = synth.model_shape(cfg)
     shape["dtype"] = cfg["dtype"]
@@ -35,6 +35,8 @@ def _setup(name, n_req, prompt_len, max_ctx, fused=True, **over):
                        cfg["seed"], torch.cuda.current_stream())
     if not fused:
         uno.uno_set_fused(ctx, False)
+    if verify_split is not None:
+        uno.uno_set_verify_split(ctx, verify_split)
     prompts = synth.make_prompts(cfg, n_req, prompt_len)
     ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).cuda(), [prompt_len] * n_req,
                           streams=list(range(n_req)))
@@ -56,9 +58,10 @@ def _kv_check(ctx, cfg, model, state, req, tol):
 
 
 def _run(name, n_req, prompt_len, n_steps, logit_tol, kv_tol, end_to_end, max_ctx=None,
-         fused=True, **over):
+         fused=True, verify_split=None, **over):
     cfg, ctx, ids, model, states = _setup(name, n_req, prompt_len,
-                                          max_ctx or prompt_len + (n_steps + 1) * 20, fused, **over)
+                                          max_ctx or prompt_len + (n_steps + 1) * 20, fused,
+                                          verify_split, **over)
     B, V, seed = cfg["B"], cfg["vocab"], cfg["seed"]
     req = torch.tensor(ids, dtype=torch.int32, device="cuda")
     out = torch.zeros((n_req, B + 1), dtype=torch.int32, device="cuda")
@@ -112,6 +115,15 @@ def test_tiny_fp32_generation():
     assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
     # fp32 mode: tokens bit-exact with the oracle's own iteration, except a
     # traced near-tie (counted in the stage tally above)
+    assert e2e.mismatches <= tally.mismatches, e2e.notes
+
+
+def test_tiny_fp32_split_verify():
+    """spec_verify in its split form (reduction kernel, then one deciding CTA
+    per request), forced at a size the fused form would take: the same
+    bit-exact fp32 decisions, for several requests."""
+    tally, e2e, _ = _run("tiny", 3, 32, 12, 1e-4, 1e-4, True, max_ctx=160, verify_split=0)
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
     assert e2e.mismatches <= tally.mismatches, e2e.notes
 
 

@@ -59,8 +59,10 @@ def _make(n_req, n_tests, V, seed=0):
     return p, q, drafts, streams, pos0
 
 
+# the last case has more (row, chunk) CTAs than the fused form takes: the
+# split reduce / decide kernels run
 @pytest.mark.parametrize("n_req,n_tests,V", [(1, 1, 16), (7, 16, 1000), (33, 5, 8196),
-                                             (16, 16, 20004), (3, 16, 151936)])
+                                             (16, 16, 20004), (3, 16, 151936), (40, 16, 65536)])
 def test_spec_verify_matches_oracle(n_req, n_tests, V):
     p, q, drafts, streams, pos0 = _make(n_req, n_tests, V)
     out, n_out, ws = _run_gpu(p.cuda(), q.cuda(), torch.from_numpy(drafts).cuda(),
