@@ -249,6 +249,8 @@ def run_uno(args, rank, world, device):
                        cfg["seed"], stream)
     if args.no_pdl:
         uno.uno_set_pdl(ctx, False)
+    if args.no_counter_sync:
+        uno.uno_set_counter_sync(ctx, False)
     fused = uno.uno_set_fused(ctx, not args.no_fused) and not args.no_fused
     if args.no_graphs:
         uno.uno_set_graphs(ctx, False)
@@ -505,6 +507,8 @@ def main():
     ap.add_argument("--no-fused", action="store_true",
                     help="unfused layer pipeline (separate LoRA-A GEMMs, norm, RoPE, SwiGLU)")
     ap.add_argument("--no-graphs", action="store_true", help="no CUDA-graph capture of steps")
+    ap.add_argument("--no-counter-sync", action="store_true",
+                    help="fused pipeline: GEMMs wait on grid dependencies, not completion counters")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for profiler captures; the "
                          "line's config records it)")

@@ -156,6 +156,17 @@ int uno_set_graphs(uno_ctx *ctx, int enable);
  * kernels in plain stream order.  Changing it drops captured graphs. */
 int uno_set_pdl(uno_ctx *ctx, int enable);
 
+/* Completion counters in the fused layer pipeline (implementation choice,
+ * on by default).  Each projection GEMM then waits for the kernel right
+ * before it (the epilogue or attention merge that wrote its input rows)
+ * through a counter that kernel's CTAs increment as they finish, instead of
+ * waiting for that whole grid to be retired; its weight stream has started
+ * before either wait.  The counters are zeroed by each pass's first kernel.
+ * A wait that outlasts about a second gives up and raises the device flag
+ * (uno_status returns UNO_ERR_DEVICE_CHECK).  enable = 0 uses grid
+ * dependencies only.  Changing it drops captured graphs. */
+int uno_set_counter_sync(uno_ctx *ctx, int enable);
+
 /* Fused layer pipeline (implementation choice, on by default where it
  * applies: passes of at most 128 rows of bf16 models with head_dim 64 or
  * 128, d_model, ffn_dim and the q / kv widths multiples of 128, d_model <=

@@ -53,6 +53,7 @@ struct AttnTcParams {
   int n_splits, n_qtiles;
   float* ws;                        // split partials [group][split][128][HD + 4]
   int32_t* status;
+  unsigned* done;                   // merge: completion counter for the next GEMM (or null)
 };
 
 template <int HD>
@@ -429,38 +430,40 @@ __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const A
   const int TQ = ATC_QROWS / G;
   const int tok0 = qt * TQ;
   const int ntok = min(TQ, p.rows_per_req - tok0);
-  if (r >= ntok * G) return;
-  const int d = threadIdx.x;
-  const size_t sstride = (size_t)ATC_QROWS * atc_ws_row(HD);
-  const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * atc_ws_row(HD);
-  float ms[ATC_MAX_SPLITS], ls[ATC_MAX_SPLITS], os[ATC_MAX_SPLITS];
+  if (r < ntok * G) {
+    const int d = threadIdx.x;
+    const size_t sstride = (size_t)ATC_QROWS * atc_ws_row(HD);
+    const float* wg = p.ws + ((size_t)group * p.n_splits * ATC_QROWS + r) * atc_ws_row(HD);
+    float ms[ATC_MAX_SPLITS], ls[ATC_MAX_SPLITS], os[ATC_MAX_SPLITS];
 #pragma unroll
-  for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
-    if (s < p.n_splits) {
-      const float2 ml = *reinterpret_cast<const float2*>(wg + s * sstride + HD);
-      ms[s] = ml.x;
-      ls[s] = ml.y;
-      os[s] = wg[s * sstride + d];
-    } else {
-      ms[s] = -INFINITY;
-      ls[s] = 0.f;
-      os[s] = 0.f;
+    for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
+      if (s < p.n_splits) {
+        const float2 ml = *reinterpret_cast<const float2*>(wg + s * sstride + HD);
+        ms[s] = ml.x;
+        ls[s] = ml.y;
+        os[s] = wg[s * sstride + d];
+      } else {
+        ms[s] = -INFINITY;
+        ls[s] = 0.f;
+        os[s] = 0.f;
+      }
     }
-  }
-  float M = -INFINITY;
+    float M = -INFINITY;
 #pragma unroll
-  for (int s = 0; s < ATC_MAX_SPLITS; ++s) M = fmaxf(M, ms[s]);
-  float L = 0.f, O = 0.f;
+    for (int s = 0; s < ATC_MAX_SPLITS; ++s) M = fmaxf(M, ms[s]);
+    float L = 0.f, O = 0.f;
 #pragma unroll
-  for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
-    const float w = (ms[s] == -INFINITY) ? 0.f : exp2f(ms[s] - M);
-    L += ls[s] * w;
-    O += os[s] * w;
+    for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
+      const float w = (ms[s] == -INFINITY) ? 0.f : exp2f(ms[s] - M);
+      L += ls[s] * w;
+      O += os[s] * w;
+    }
+    const int row0 = req * p.rows_per_req + tok0;
+    const int tk = r / G, g = r % G;
+    const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;
+    store_split<bf16>(p.out, p.out_lo, oo, O / L);
   }
-  const int row0 = req * p.rows_per_req + tok0;
-  const int tk = r / G, g = r % G;
-  const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;
-  store_split<bf16>(p.out, p.out_lo, oo, O / L);
+  dep_signal(p.done);
 }
 
 }  // namespace uno

@@ -133,11 +133,38 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Completion counters: a finer dependency than pdl_wait() for a kernel that
+// needs only the outputs of the kernel right before it.  Every CTA of the
+// producer ends with dep_signal (a CTA barrier, then one release add at GPU
+// scope: the CTA's writes are visible to whoever acquires the count); the
+// consumer polls with acquire loads until all producer CTAs have counted.
+// A consumer launched programmatically starts only after every producer CTA
+// has started, so the producers it waits for are all resident and the wait
+// ends; it is bounded anyway (false after about a second).  The counters of
+// a pass are zeroed by its first kernel after that kernel's pdl_wait() and
+// before its pdl_trigger(), so no kernel of the pass can see a stale count.
+__device__ __forceinline__ void dep_signal(unsigned* ctr) {   // whole CTA, at its end
+  if (!ctr) return;
+  __syncthreads();
+  if (threadIdx.x == 0 && threadIdx.y == 0)
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+__device__ __forceinline__ bool dep_wait(const unsigned* ctr, unsigned target) {   // one thread
+  for (int i = 0; i < (1 << 21); ++i) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    __nanosleep(20);
+  }
+  return false;
+}
+
 // Device-side error flag bits (read by uno_status).
 enum StatusBits : int32_t {
   ST_POS_OVERFLOW = 1,   // a position beyond the request's KV pages
   ST_BAD_TOKEN = 2,      // a token id outside [0, vocab)
   ST_BAD_SLOT = 4,       // a request id outside [0, max_batch) or not admitted
+  ST_DEP_TIMEOUT = 32,   // a completion-counter wait gave up
 };
 __device__ __forceinline__ void raise_status(int32_t* st, int32_t bit) {
   if (st) atomicOr(st, bit);

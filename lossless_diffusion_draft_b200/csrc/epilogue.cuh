@@ -76,6 +76,7 @@ struct EpiArgs {
   // epi_swiglu
   int F; bf16* h;                    // [M][F] (lo rows lo_off below)
   int32_t* status;
+  unsigned* done;                    // completion counter the next GEMM waits on (or null)
 };
 
 // Thread layout of an epilogue CTA: NQ row slots x 128 columns, the NQ
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiA
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
-  if (!row_group<G>(a, &m0, &nrows)) return;
+  if (!row_group<G>(a, &m0, &nrows)) { dep_signal(a.done); return; }
   const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int n = nt * TC_BM + col;
   // weights (the next norm's gain, the adapter row) before the dependency wait
@@ -502,6 +503,7 @@ __global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiA
     }
   }
   if (a.g_next) next_input<G>(a, nt, m0, nrows, col, q, g, xv);
+  dep_signal(a.done);
 }
 
 // ---------------------------------------------------------------------------
@@ -520,7 +522,7 @@ __global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const
   pdl_trigger();
   const int ft = blockIdx.x;
   int m0, nrows;
-  if (!row_group<G>(a, &m0, &nrows)) return;
+  if (!row_group<G>(a, &m0, &nrows)) { dep_signal(a.done); return; }
   const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int f = ft * TC_BM + col;
   const int ut = a.F / TC_BM + ft;         // the up tile of the same features
@@ -568,6 +570,7 @@ __global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const
       store_split<bf16>(a.h, lo, (size_t)(m0 + j) * a.F + f, gv / (1.0f + expf(-gv)) * uv);
     }
   }
+  dep_signal(a.done);
 }
 
 }  // namespace uno

@@ -41,6 +41,9 @@ struct GemmParams {
   const float* row_gate;
   int lo_off;        // > 0: X and U also hold lo rows (x - bf16(x)) this many rows below
   void* out_lo;      // EPI_GATED: where the lo part of the output goes (or null)
+  // tensor-core DUMP launches: completion counter of the kernel that wrote X
+  // and its CTA count (null: the launch waits with pdl_wait)
+  const unsigned* dep; unsigned dep_count;
 };
 
 template <typename T, int MT, int NC>

@@ -68,6 +68,9 @@ struct TcParams {
   int32_t* status;
   int lo_off;                // split mode: row offset of the lo rows of X and U
   void* out_lo;              // EPI_GATED in split mode: lo part of the output (out + lo_off rows)
+  // completion counter of the kernel that wrote X (null: pdl_wait instead);
+  // DUMP mode only, where X is the one input an earlier kernel wrote
+  const unsigned* dep; unsigned dep_count;
 };
 
 // ---------------------------------------------------------------------------
@@ -181,8 +184,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = *s_tmem;
   pdl_trigger();
   // every thread but the TMA issuer waits for the previous kernel here; the
-  // issuer first starts the weight stream (see below)
-  if (!(warp == 4 && lane == 0)) pdl_wait();
+  // issuer first starts the weight stream (see below).  With a completion
+  // counter only the issuer waits, for the X rows: the other threads read
+  // nothing an earlier kernel wrote (in DUMP mode they only store parts, and
+  // those stores follow MMAs on X tiles loaded after the wait).
+  if (!p.dep && !(warp == 4 && lane == 0)) pdl_wait();
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
@@ -239,7 +245,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mbar_expect_tx(&full[i], C::STAGE_BYTES);
         load_a(u0 + i, i);
       }
-      pdl_wait();
+      if (p.dep) {
+        if (!dep_wait(p.dep, p.dep_count)) raise_status(p.status, ST_DEP_TIMEOUT);
+        // the X rows were written by generic stores; the loads below are TMA
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      } else {
+        pdl_wait();
+      }
       for (int i = 0; i < npre; ++i) load_b(u0 + i, i);
       int issued = npre;
       for (int i = npre; i < total && !*s_abort; ++i) {

@@ -66,13 +66,24 @@ struct RowArgs {
   const void* embed; int d;    // [vocab, d] model dtype
   float* x;                    // [M, d] fp32 residual
   int32_t* status;
+  unsigned* zero_ctr; int n_zero;   // the pass's completion counters (zeroed here), or null
 };
 
 // a1: build the rows of a pass and gather their embeddings.
 template <typename T>
 __global__ void build_rows_kernel(const RowArgs a) {
-  pdl_trigger();
-  pdl_wait();
+  if (a.zero_ctr) {
+    // after every earlier kernel has completed, before any later one starts
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.n_zero; i += gridDim.x * blockDim.x)
+      a.zero_ctr[i] = 0u;
+    __threadfence();
+    __syncthreads();
+    pdl_trigger();
+  } else {
+    pdl_trigger();
+    pdl_wait();
+  }
   const int row = blockIdx.x;
   const int req = row / a.rows_per_req, j = row % a.rows_per_req;
   int slot, tok, pos;

@@ -233,6 +233,8 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.status = env.status;
   tp.lo_off = SPLIT ? p.lo_off : 0;
   tp.out_lo = p.out_lo;
+  tp.dep = DUMP ? p.dep : nullptr;
+  tp.dep_count = p.dep_count;
   using Cfg = TcCfg<NT, SPLIT, KPS>;
   static bool attr = false;
   if (!attr) {
@@ -352,6 +354,11 @@ struct uno_ctx {
   int verify_split_ctas = 4096;   // spec_verify: split form above this many CTAs
   int32_t *row_pos = nullptr, *row_slot = nullptr;
   float* row_gate = nullptr;
+  // completion counters of the fused pass (GEMMs wait on the kernel before
+  // them through these instead of pdl_wait), zeroed by each pass's first kernel
+  unsigned* dep_ctr = nullptr;
+  int n_dep_ctr = 0;
+  bool counter_sync = true;
   float *cos_t = nullptr, *sin_t = nullptr;
   int max_pos = 0;
 
@@ -533,7 +540,7 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
 
 template <int HD>
 int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                   void* out_lo) {
+                   void* out_lo, unsigned* done, unsigned* done_ctas) {
   const uno_shape& s = c->s;
   AttnTcParams p{};
   p.q = (const f16*)c->qbuf;
@@ -582,19 +589,29 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
     Prof prof(c, UNO_K_ATTN, 0.0);
     // only the rows a query tile can hold: tokens per request x heads per kv head
     const int rows = std::min(ATC_QROWS, rows_per_req * G);
+    p.done = done;
+    if (done) *done_ctas = (unsigned)(ceil_div(rows, ATC_MERGE_ROWS) * groups);
     klaunch(c->genv.pdl, c->stream, dim3(ceil_div(rows, ATC_MERGE_ROWS), groups),
             dim3(HD, ATC_MERGE_ROWS), 0, attn_merge_kernel<HD>, p);
   }
   return UNO_OK;
 }
 
+// done (optional): completion counter for the kernel that writes the output
+// last (the merge); *done_ctas receives its CTA count, 0 when no counter
+// was signalled (then the next kernel waits with pdl_wait).
 template <typename T>
 int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                void* out_lo) {
+                void* out_lo, unsigned* done = nullptr, unsigned* done_ctas = nullptr) {
   const uno_shape& s = c->s;
+  unsigned dummy = 0;
+  if (!done_ctas) done_ctas = &dummy;
+  *done_ctas = 0;
   if (c->kv_map_ok) {
-    if (s.head_dim == 128) return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo);
-    if (s.head_dim == 64) return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo);
+    if (s.head_dim == 128)
+      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas);
+    if (s.head_dim == 64)
+      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas);
   }
   AttnParams p{};
   p.qkv = c->qbuf;
@@ -848,6 +865,18 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ra.x = c->x;
   ra.status = c->d_status;
   ra.prefill_pos0 = prefill_pos0;
+  // completion counters: each GEMM waits for the kernel right before it
+  // (its X rows) through a counter that kernel's CTAs add to; the counters
+  // are zeroed by build_rows
+  const bool csync = c->counter_sync && c->dep_ctr;
+  int n_ctr = 0;
+  const unsigned* dep = nullptr;   // counter of the last signalling kernel
+  unsigned dep_n = 0;              // and its CTA count
+  auto next_ctr = [&]() -> unsigned* {
+    return (csync && n_ctr < c->n_dep_ctr) ? c->dep_ctr + n_ctr++ : nullptr;
+  };
+  ra.zero_ctr = csync ? c->dep_ctr : nullptr;
+  ra.n_zero = c->n_dep_ctr;
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
     klaunch(pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<bf16>, ra);
@@ -896,6 +925,9 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     if (lora)
       for (const void* a : A) g.seg(a, r);
     g.p.lo_off = lo;
+    g.p.dep = dep;
+    g.p.dep_count = dep_n;
+    dep = nullptr;
     DumpShape sh;
     {
       Prof prof(c, UNO_K_GEMM, gemm_bytes(g.p, 2) - (double)M * g.p.N * 2, M, g.p.N, K, 0);
@@ -919,9 +951,13 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   };
   // one epilogue launch: rg rows per CTA (row groups inside the GEMM's
   // m-tiles), `threads` threads
-  auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int rg, int threads) {
+  // `signal`: the next kernel is a GEMM that waits on this one's counter
+  auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int rg, int threads, bool signal) {
     Prof prof(c, UNO_K_OTHER, 0.0);
     const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M, rg);
+    ea.done = signal ? next_ctr() : nullptr;
+    dep = ea.done;
+    dep_n = (unsigned)(tiles * groups);
     klaunch(pdl, st, dim3(tiles, groups), dim3(threads), 0, kernel, ea);
   };
 
@@ -930,7 +966,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ea.lora = 0;
   ea.pv = PartView{nullptr, M, 0, 1, 1, 1};
   ea.g_next = (const bf16*)c->attn_norm[0];
-  epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
+  epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, true);
   ea.prep = 0;
 
   for (int l = 0; l < s.n_layers; ++l) {
@@ -943,31 +979,35 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_Q][l], H * hd}, {c->lB[UNO_PROJ_K][l], Hkv * hd},
               {c->lB[UNO_PROJ_V][l], Hkv * hd}});
     ea.ss = c->ss;
-    epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS);
+    epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS, false);
 
-    rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo);
-    if (rc) return rc;
+    {
+      unsigned* done = next_ctr();
+      rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo, done, &dep_n);
+      if (rc) return rc;
+      dep = dep_n ? done : nullptr;   // no merge launched: the o GEMM waits with pdl_wait
+    }
 
     rc = gemm(c->attn, hhd, hhd, {{c->w[UNO_PROJ_O][l], d}}, {c->lA[UNO_PROJ_O][l]}, &ea.pv);
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_O][l], d}});
     ea.ss = nullptr;
     ea.g_next = (const bf16*)c->ffn_norm[l];
-    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, true);
 
     rc = gemm(c->xn, xn_ld, d, {{c->w[UNO_PROJ_GATE][l], F}, {c->w[UNO_PROJ_UP][l], F}},
               {c->lA[UNO_PROJ_GATE][l], c->lA[UNO_PROJ_UP][l]}, &ea.pv);
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_GATE][l], F}, {c->lB[UNO_PROJ_UP][l], F}});
     ea.ss = c->ss;
-    epi(epi_swiglu_kernel, F / TC_BM, GeoSwiglu::RG, GeoSwiglu::THREADS);
+    epi(epi_swiglu_kernel, F / TC_BM, GeoSwiglu::RG, GeoSwiglu::THREADS, true);
 
     rc = gemm(c->xn, F, F, {{c->w[UNO_PROJ_DOWN][l], d}}, {c->lA[UNO_PROJ_DOWN][l]}, &ea.pv);
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_DOWN][l], d}});
     ea.ss = nullptr;
     ea.g_next = l + 1 < s.n_layers ? (const bf16*)c->attn_norm[l + 1] : nullptr;
-    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, l + 1 < s.n_layers);
   }
   if (logits) {
     bf16* xn_lo = split ? (bf16*)c->xn + (size_t)lo * xn_ld : nullptr;
@@ -1118,6 +1158,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->row_pos, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_slot, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_gate, (size_t)M * 4) != cudaSuccess) return oom("rows");
+  c->n_dep_ctr = 4 * s.n_layers + 8;
+  if (dalloc(&c->dep_ctr, (size_t)c->n_dep_ctr * 4) != cudaSuccess) return oom("counters");
+  cudaMemset(c->dep_ctr, 0, (size_t)c->n_dep_ctr * 4);
 
   // RoPE table, double precision on the host
   c->max_pos = ppr * KV_PAGE;
@@ -1237,7 +1280,7 @@ int uno_destroy(uno_ctx* c) {
   cudaDeviceSynchronize();
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
                   c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
-                  c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
+                  c->dep_ctr, c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
                   c->lse_ws, c->row_counter, c->req_counter, c->at_ws, c->resid_part,
                   c->resid_counter, c->att_ws, c->att_counters,
                   c->d_status, c->genv.ws, c->genv.counters, c->genv.part, c->ss};
@@ -1490,6 +1533,17 @@ int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_
 int uno_set_graphs(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->graphs_enabled = enable != 0;
+  return UNO_OK;
+}
+
+int uno_set_counter_sync(uno_ctx* c, int enable) {
+  if (!c) return UNO_ERR_ARG;
+  c->counter_sync = enable != 0;
+  for (auto& g : c->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.seen = 0;
+  }
   return UNO_OK;
 }
 

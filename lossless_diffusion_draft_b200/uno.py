@@ -85,6 +85,7 @@ def load_library(path=LIB_PATH):
         "uno_set_pdl": (i32, [vp, i32]),
         "uno_set_fused": (i32, [vp, i32]),
         "uno_set_verify_split": (i32, [vp, i32]),
+        "uno_set_counter_sync": (i32, [vp, i32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
@@ -235,6 +236,11 @@ def uno_set_fused(ctx, enable):
 def uno_set_verify_split(ctx, max_ctas):
     """spec_verify in its split form above max_ctas (row, chunk) CTAs (0: always)."""
     _check(load_library().uno_set_verify_split(ctx.handle, int(max_ctas)), ctx.handle)
+
+
+def uno_set_counter_sync(ctx, enable):
+    """Fused pipeline: GEMMs wait on completion counters (True) or grid dependencies."""
+    _check(load_library().uno_set_counter_sync(ctx.handle, int(bool(enable))), ctx.handle)
 
 
 def uno_release(ctx, req_id):
