@@ -115,30 +115,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   volatile int* s_ok = reinterpret_cast<volatile int*>(s_tmem + 4);   // [4]
 
   pdl_trigger();
-  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
-  const int req = z / p.Hkv, kvh = z % p.Hkv;
-  const int G = p.H / p.Hkv;
-  const int TQ = ATC_QROWS / G;                  // tokens per query tile
-  const int tok0 = qt * TQ;
-  const int ntok = min(TQ, p.rows_per_req - tok0);
-  const int nq = ntok * G;
-  const int row0 = req * p.rows_per_req + tok0;
-  // the position of each query row (warps 0-3, one row per thread)
-  int qpos = -1;
-  if (warp < 4 && threadIdx.x < nq) qpos = p.row_pos[row0 + threadIdx.x / G];
-  const int slot = p.row_slot[row0];
-  const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
-  int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
-  if (ntiles > p.pages_per_req) {
-    if (threadIdx.x == 0 && split == 0) raise_status(p.status, ST_POS_OVERFLOW);
-    ntiles = p.pages_per_req;
-  }
-  const int t_begin = (int)((long long)ntiles * split / p.n_splits);
-  const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
-  const int n = t_end - t_begin;
-
+  // barriers, TMEM and descriptors depend on no earlier kernel: set up
+  // before the wait
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -161,13 +140,36 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                  "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  if (warp == 4 && lane == 0) {
+    prefetch_map(&kvmap);
+    prefetch_map(&qmap);
+  }
+  pdl_wait();
+  const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
+  const int req = z / p.Hkv, kvh = z % p.Hkv;
+  const int G = p.H / p.Hkv;
+  const int TQ = ATC_QROWS / G;                  // tokens per query tile
+  const int tok0 = qt * TQ;
+  const int ntok = min(TQ, p.rows_per_req - tok0);
+  const int nq = ntok * G;
+  const int row0 = req * p.rows_per_req + tok0;
+  // the position of each query row (warps 0-3, one row per thread)
+  int qpos = -1;
+  if (warp < 4 && threadIdx.x < nq) qpos = p.row_pos[row0 + threadIdx.x / G];
+  const int slot = p.row_slot[row0];
+  const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
+  int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
+  if (ntiles > p.pages_per_req) {
+    if (threadIdx.x == 0 && split == 0) raise_status(p.status, ST_POS_OVERFLOW);
+    ntiles = p.pages_per_req;
+  }
+  const int t_begin = (int)((long long)ntiles * split / p.n_splits);
+  const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
+  const int n = t_end - t_begin;
+
   // the split's page numbers, fetched in one round while the q rows load
   __shared__ int s_pages[ATC_PAGE_PF];
   if (warp == 4) {
-    if (lane == 0) {
-      prefetch_map(&kvmap);
-      prefetch_map(&qmap);
-    }
     for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32)
       s_pages[i] = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
   }

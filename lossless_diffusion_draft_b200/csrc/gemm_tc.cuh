@@ -155,7 +155,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int u0 = sk_start(blockIdx.x, p.units, p.grid);
   const int u1 = sk_start(blockIdx.x + 1, p.units, p.grid);
 
-  if (threadIdx.x == 0) {
+  // unit u is k-block u % KBt of tile u / KBt; issue i = u - u0 uses
+  // ring stage i % STAGES
+  auto seg_of = [&](int n_row) {
+    int sg = 0;
+    for (int s = 1; s < p.nseg; ++s)
+      if (n_row >= p.seg[s].n0) sg = s;
+    return sg;
+  };
+  // weight tile of unit u: W, then LoRA-B
+  auto coords_a = [&](int u, const CUtensorMap*& map, int& x, int& y) {
+    const int t = u / KBt, kb = u % KBt;
+    const int n_row = (t / p.m_tiles) * TC_BM;
+    const int sg = seg_of(n_row);
+    map = kb < p.KB ? &maps.w[sg] : &maps.b[sg];
+    x = (kb < p.KB ? kb : kb - p.KB) * TC_BK * KPS;
+    y = n_row - p.seg[sg].n0;
+  };
+  auto load_a = [&](int u, int stage) {
+    const CUtensorMap* map;
+    int x, y;
+    coords_a(u, map, x, y);
+#pragma unroll
+    for (int j = 0; j < KPS; ++j)
+      tma_load_2d(sA + stage * C::A_BYTES + j * TC_A_BYTES, map, &full[stage], x + j * TC_BK, y);
+  };
+
+  auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
+    const int t = u / KBt, kb = u % KBt;
+    const int mt = t % p.m_tiles;
+#pragma unroll
+    for (int j = 0; j < KPS; ++j) {
+      uint8_t* dst = sB + stage * C::B_BYTES + j * C::B_SUB;
+      if (kb < p.KB) {
+        const int x = (kb * KPS + j) * TC_BK;
+        tma_load_2d(dst, &maps.x, &full[stage], x, mt * NT);
+        if (SPLIT) tma_load_2d(dst + NT * 128, &maps.x, &full[stage], x, p.lo_off + mt * NT);
+      } else {
+        const int sg = seg_of((t / p.m_tiles) * TC_BM);
+        const int x = p.seg[sg].u_off + ((kb - p.KB) * KPS + j) * TC_BK;
+        tma_load_2d(dst, &maps.u, &full[stage], x, mt * NT);
+        if (SPLIT) tma_load_2d(dst + NT * 128, &maps.u, &full[stage], x, p.lo_off + mt * NT);
+      }
+    }
+  };
+  const int total = u1 - u0;
+  const int npre = min(total, C::STAGES);
+
+  // The TMA issuer sets up the barriers and starts the weight stream (the
+  // weights depend on no earlier kernel) while warp 0 allocates TMEM: the
+  // first stages' copies are under way before the CTA's first barrier.
+  if (warp == 4 && lane == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -167,6 +217,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     mbar_init(drain, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_map(&maps.x);
+    for (int s = 0; s < p.nseg; ++s) prefetch_map(&maps.w[s]);
+    if (p.dep) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.dep));
+    for (int i = 0; i < npre; ++i) {
+      mbar_expect_tx(&full[i], C::STAGE_BYTES);
+      load_a(u0 + i, i);
+    }
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -174,17 +231,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                  "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_map(&maps.x);
-    for (int s = 0; s < p.nseg; ++s) prefetch_map(&maps.w[s]);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   pdl_trigger();
-  // every thread but the TMA issuer waits for the previous kernel here; the
-  // issuer first starts the weight stream (see below).  With a completion
+  // every thread but the TMA issuer waits for the previous kernel here (the
+  // issuer has started the weight stream above).  With a completion
   // counter only the issuer waits, for the X rows: the other threads read
   // nothing an earlier kernel wrote (in DUMP mode they only store parts, and
   // those stores follow MMAs on X tiles loaded after the wait).
@@ -193,58 +246,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      // unit u is k-block u % KBt of tile u / KBt; issue i = u - u0 uses
-      // ring stage i % STAGES
-      auto seg_of = [&](int n_row) {
-        int sg = 0;
-        for (int s = 1; s < p.nseg; ++s)
-          if (n_row >= p.seg[s].n0) sg = s;
-        return sg;
-      };
-      // weight tile of unit u: W, then LoRA-B
-      auto coords_a = [&](int u, const CUtensorMap*& map, int& x, int& y) {
-        const int t = u / KBt, kb = u % KBt;
-        const int n_row = (t / p.m_tiles) * TC_BM;
-        const int sg = seg_of(n_row);
-        map = kb < p.KB ? &maps.w[sg] : &maps.b[sg];
-        x = (kb < p.KB ? kb : kb - p.KB) * TC_BK * KPS;
-        y = n_row - p.seg[sg].n0;
-      };
-      auto load_a = [&](int u, int stage) {
-        const CUtensorMap* map;
-        int x, y;
-        coords_a(u, map, x, y);
-#pragma unroll
-        for (int j = 0; j < KPS; ++j)
-          tma_load_2d(sA + stage * C::A_BYTES + j * TC_A_BYTES, map, &full[stage], x + j * TC_BK, y);
-      };
-
-      auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
-        const int t = u / KBt, kb = u % KBt;
-        const int mt = t % p.m_tiles;
-#pragma unroll
-        for (int j = 0; j < KPS; ++j) {
-          uint8_t* dst = sB + stage * C::B_BYTES + j * C::B_SUB;
-          if (kb < p.KB) {
-            const int x = (kb * KPS + j) * TC_BK;
-            tma_load_2d(dst, &maps.x, &full[stage], x, mt * NT);
-            if (SPLIT) tma_load_2d(dst + NT * 128, &maps.x, &full[stage], x, p.lo_off + mt * NT);
-          } else {
-            const int sg = seg_of((t / p.m_tiles) * TC_BM);
-            const int x = p.seg[sg].u_off + ((kb - p.KB) * KPS + j) * TC_BK;
-            tma_load_2d(dst, &maps.u, &full[stage], x, mt * NT);
-            if (SPLIT) tma_load_2d(dst + NT * 128, &maps.u, &full[stage], x, p.lo_off + mt * NT);
-          }
-        }
-      };
-      const int total = u1 - u0;
-      const int npre = min(total, C::STAGES);
-      // the weights depend on no earlier kernel: their first stages stream
-      // while the previous kernel finishes
-      for (int i = 0; i < npre; ++i) {
-        mbar_expect_tx(&full[i], C::STAGE_BYTES);
-        load_a(u0 + i, i);
-      }
       if (p.dep) {
         if (!dep_wait(p.dep, p.dep_count)) raise_status(p.status, ST_DEP_TIMEOUT);
         // the X rows were written by generic stores; the loads below are TMA
