@@ -36,6 +36,7 @@ constexpr int ATC_QROWS = 128;
 constexpr int ATC_KT = 64;          // keys per tile = one KV page
 constexpr int ATC_PAGE_PF = 64;     // page numbers a CTA fetches up front
 constexpr int ST_ATTN_TIMEOUT = 16;
+constexpr int ATC_PF_LANES = 8;     // producer-warp lanes issuing the L2 prefetch
 // Floats per query row of a split partial: O[HD], m, l, padded so that every
 // row starts on a 16-byte boundary (rows are written with float4 stores).
 __host__ __device__ constexpr int atc_ws_row(int hd) { return hd + 4; }
@@ -54,6 +55,10 @@ struct AttnTcParams {
   float* ws;                        // split partials [group][split][128][HD + 4]
   int32_t* status;
   unsigned* done;                   // merge: completion counter for the next GEMM (or null)
+  // weights of the projection after the attention, prefetched into L2 by the
+  // producer warp's idle lanes while the KV stream leaves HBM bandwidth
+  // unused (null: none); 16-byte aligned, a multiple of 16 bytes
+  const char* l2_pf; unsigned long long l2_pf_bytes;
 };
 
 template <int HD>
@@ -143,6 +148,18 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   if (warp == 4 && lane == 0) {
     prefetch_map(&kvmap);
     prefetch_map(&qmap);
+  }
+  if (p.l2_pf && warp == 4 && lane >= 1 && lane <= ATC_PF_LANES) {
+    // this CTA's share of the next projection's weights, in 16-byte units
+    const unsigned long long units = p.l2_pf_bytes >> 4;
+    const unsigned long long ctas = (unsigned long long)gridDim.x * gridDim.y * gridDim.z;
+    const unsigned long long cta = blockIdx.x + gridDim.x * (blockIdx.y + (unsigned long long)gridDim.y * blockIdx.z);
+    const unsigned long long parts = ctas * ATC_PF_LANES, part = cta * ATC_PF_LANES + (lane - 1);
+    const unsigned long long u0 = units * part / parts, u1 = units * (part + 1) / parts;
+    if (u1 > u0)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.l2_pf + (u0 << 4)),
+                   "r"((unsigned)((u1 - u0) << 4))
+                   : "memory");
   }
   pdl_wait();
   const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;

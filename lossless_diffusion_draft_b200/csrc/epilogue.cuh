@@ -22,8 +22,8 @@
 // Distillation：一步蒸馏 + 块级扩散): y = W x + gate * (alpha / r) * B (A x).
 // The GEMM streams the A matrices as extra output tiles next to W, so the
 // rank-r product U = A (g * x) comes out of the same pass; the epilogue
-// multiplies U by the rows of B on the CUDA cores (r MACs per output) and
-// gates it per row.
+// multiplies U by the rows of B (a small tensor-core product per CTA, below)
+// and gates it per row.
 //
 // One CTA takes one 128-column tile of the output (two for SwiGLU) and a
 // group of rows (Geo below); a few slot threads share a column, each with a
@@ -90,6 +90,8 @@ struct Geo {
   static constexpr int RG = RG_, NQ = NQ_;
   static constexpr int RPT = (RG + NQ - 1) / NQ;
   static constexpr int THREADS = NQ * TC_BM;
+  // LoRA-B tiles: 16 MMA rows, eight warps of 16 columns
+  static_assert(RG <= 16 && THREADS == 256, "row group fits one MMA tile; 8 warps x 16 columns");
   static constexpr int KQ = EPI_R / NQ;                     // rank columns per slot thread
   static constexpr int SS_PT = (RG * EPI_MAX_SS + THREADS - 1) / THREADS;
 };
@@ -207,100 +209,131 @@ __device__ __forceinline__ int lora_seg(const LoraEpi& lr, int n) {
   return s;
 }
 
-// The slot thread's share of one adapter row: B[nb][q KQ .. q KQ + KQ].
-template <class G>
-struct BPart { uint4 b[G::KQ / 8]; };
-template <class G>
-__device__ __forceinline__ void bpart_issue(const EpiArgs& a, int seg, int nb, int q, BPart<G>& B) {
-  const uint4* src = reinterpret_cast<const uint4*>(a.lr.Bl[seg] + (size_t)nb * EPI_R + q * G::KQ);
+// ---------------------------------------------------------------------------
+// LoRA-B on the tensor cores: dot[j][c] = sum_k U[j][k] B[c][k] for the
+// CTA's rows j (at most 16) and 128 columns c, as mma.sync m16n8k16 (bf16
+// in, fp32 accumulate) with U fed as a bf16 hi/lo pair (~16 mantissa bits,
+// like the GEMM inputs) and B, a bf16 weight, exact.  Warp w takes the
+// columns 16 w .. 16 w + 15 (two n-tiles of 8).  The rank order inside a
+// k-step is free as long as U and B agree: in k-step s, thread t of a quad
+// puts ranks 32 t + 4 s + {0, 1} in the k-slots {2t, 2t+1} and
+// 32 t + 4 s + {2, 3} in {2t+8, 2t+9}.  Its B values for its column are then
+// the 32 contiguous ranks 32 t .. 32 t + 31 (four 16-byte loads per n-tile,
+// issued before the dependency wait), and its U values of a row are 8
+// contiguous bf16 per pair of k-steps (one 16-byte shared-memory load).
+// ---------------------------------------------------------------------------
+constexpr int EPI_UP = EPI_R + 8;   // row pitch of the bf16 U tiles: 272 B, conflict-free loads
+static_assert(EPI_R == 128, "the k-step rank order covers 128 ranks");
+
+struct BFrag { uint4 b[2][4]; };    // [n-tile][16-byte piece of the thread's 32 ranks]
+// col0: the adapter row (segment column) of the warp's first column
+__device__ __forceinline__ void bfrag_issue(const EpiArgs& a, int seg, int col0, BFrag& B) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int e = 0; e < G::KQ / 8; ++e) B.b[e] = __ldg(src + e);
+  for (int nt = 0; nt < 2; ++nt) {
+    const uint4* src =
+        reinterpret_cast<const uint4*>(a.lr.Bl[seg] + (size_t)(col0 + 8 * nt + g) * EPI_R + 32 * t);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) B.b[nt][e] = __ldg(src + e);
+  }
+}
+// The same bytes into L2 only (one prefetch per thread and n-tile: 64 bytes).
+__device__ __forceinline__ void bfrag_prefetch(const EpiArgs& a, int seg, int col0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lr.Bl[seg] + (size_t)(col0 + 8 * nt + g) * EPI_R + 32 * t));
 }
 
-// The same share into L2 only (one prefetch per 128-byte line).
-template <class G>
-__device__ __forceinline__ void bpart_prefetch(const EpiArgs& a, int seg, int nb, int q, const BPart<G>&) {
-  const char* src = reinterpret_cast<const char*>(a.lr.Bl[seg] + (size_t)nb * EPI_R + q * G::KQ);
-#pragma unroll
-  for (int e = 0; e < G::KQ * 2; e += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + e));
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// LoRA-B for column col: the slot thread forms the partial dot of its rank
-// share for every row (sU[j][k] B[k]); the NQ partials of the column are then
-// reduce-scattered over the slot lanes (shuffles, compile-time register
-// indices), so each row's sum is formed once, in a fixed order, by the thread
-// owning the row, which adds gate * dot.  sU must be complete (caller syncs).
-template <class G>
-__device__ __forceinline__ void lora_apply(const BPart<G>& B, const float* sU, int q, int nrows,
-                                           const float (&gate)[G::RPT], float (&acc)[G::RPT]) {
-  static_assert(G::NQ == 2 || G::NQ == 4, "two or four slot threads per column");
-  constexpr int RGP = G::RPT * G::NQ;       // rows padded to whole slot groups
-  float p[RGP];
+// The dots of the CTA's first `rows` rows into sDot[row][128].  sUh / sUl
+// ([16][EPI_UP] bf16) must be complete (caller syncs); rows past `rows`
+// may hold anything (an MMA row depends only on its own U row).
+__device__ __forceinline__ void lora_mma(const BFrag& B, const bf16* sUh, const bf16* sUl,
+                                         float* sDot, int rows) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-  for (int j = 0; j < RGP; ++j) p[j] = 0.f;
-  // rank outer (eight adapter values unpacked at a time), rows inner
+  for (int s2 = 0; s2 < 4; ++s2) {
+    const int o = 32 * t + 8 * s2;   // ranks 32 t + 8 s2 .. + 7: k-steps 2 s2 and 2 s2 + 1
+    const uint4 h0 = *reinterpret_cast<const uint4*>(sUh + g * EPI_UP + o);
+    const uint4 h1 = *reinterpret_cast<const uint4*>(sUh + (g + 8) * EPI_UP + o);
+    const uint4 l0 = *reinterpret_cast<const uint4*>(sUl + g * EPI_UP + o);
+    const uint4 l1 = *reinterpret_cast<const uint4*>(sUl + (g + 8) * EPI_UP + o);
 #pragma unroll
-  for (int e = 0; e < G::KQ / 8; ++e) {
-    float bf[8];
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&B.b[e]);
+    for (int half = 0; half < 2; ++half) {
+      const int ks = 2 * s2 + half;
+      // A registers: (row g, slots 2t..), (row g+8, 2t..), (row g, 2t+8..), (row g+8, 2t+8..)
+      const uint32_t ah[4] = {half ? h0.z : h0.x, half ? h1.z : h1.x, half ? h0.w : h0.y,
+                              half ? h1.w : h1.y};
+      const uint32_t al[4] = {half ? l0.z : l0.x, half ? l1.z : l1.x, half ? l0.w : l0.y,
+                              half ? l1.w : l1.y};
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      bf[2 * h] = __low2float(b2[h]);
-      bf[2 * h + 1] = __high2float(b2[h]);
-    }
-#pragma unroll
-    for (int j = 0; j < RGP; ++j) {
-      if (j < nrows) {
-        const float4* u4 = reinterpret_cast<const float4*>(sU + j * EPI_R + q * G::KQ + 8 * e);
-        const float4 x0 = u4[0], x1 = u4[1];
-        p[j] += x0.x * bf[0] + x0.y * bf[1] + x0.z * bf[2] + x0.w * bf[3] +
-                x1.x * bf[4] + x1.y * bf[5] + x1.z * bf[6] + x1.w * bf[7];
+      for (int nt = 0; nt < 2; ++nt) {
+        const uint4 bb = B.b[nt][ks >> 1];
+        const uint32_t b0 = (ks & 1) ? bb.z : bb.x, b1 = (ks & 1) ? bb.w : bb.y;
+        mma_bf16_16816(d[nt], ah, b0, b1);
+        mma_bf16_16816(d[nt], al, b0, b1);
       }
     }
   }
-  float tot[G::RPT];
-  if (G::NQ == 2) {
-    // rows 2s + r: slot r keeps row r, sends the other
+  // accumulator: (row g, columns 2t, 2t+1) and (row g+8, the same columns)
 #pragma unroll
-    for (int s = 0; s < G::RPT; ++s) {
-      const float keep = q ? p[2 * s + 1] : p[2 * s], send = q ? p[2 * s] : p[2 * s + 1];
-      tot[s] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  for (int nt = 0; nt < 2; ++nt) {
+    const int c = 16 * warp + 8 * nt + 2 * t;
+    if (g < rows) {
+      sDot[g * TC_BM + c] = d[nt][0];
+      sDot[g * TC_BM + c + 1] = d[nt][1];
     }
-  } else {
-    // rows 4s + r: first between slots q and q ^ 2 (keep r with the same bit 1
-    // as q), then between q and q ^ 1
-#pragma unroll
-    for (int s = 0; s < G::RPT; ++s) {
-      float h[2];
-#pragma unroll
-      for (int r1 = 0; r1 < 2; ++r1) {
-        const float keep = (q & 2) ? p[4 * s + 2 + r1] : p[4 * s + r1];
-        const float send = (q & 2) ? p[4 * s + r1] : p[4 * s + 2 + r1];
-        h[r1] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-      }
-      const float keep = (q & 1) ? h[1] : h[0], send = (q & 1) ? h[0] : h[1];
-      tot[s] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    if (g + 8 < rows) {
+      sDot[(g + 8) * TC_BM + c] = d[nt][2];
+      sDot[(g + 8) * TC_BM + c + 1] = d[nt][3];
     }
   }
-#pragma unroll
-  for (int s = 0; s < G::RPT; ++s)
-    if (q + G::NQ * s < nrows) acc[s] += gate[s] * tot[s];
 }
 
-// The U tile of segment seg, column col, the thread's rows: loads, then the
-// sums into sU[RG][EPI_R].  The caller syncs before sU is read.
+// acc += gate * dot for the thread's rows of column col (sDot complete:
+// caller syncs).
+template <class G>
+__device__ __forceinline__ void lora_add(const float* sDot, int col, int q, int nrows,
+                                         const float (&gate)[G::RPT], float (&acc)[G::RPT]) {
+#pragma unroll
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
+    if (j < nrows) acc[s] += gate[s] * sDot[j * TC_BM + col];
+  }
+}
+
+// The U tile of segment seg, column (rank) col, the thread's rows: loads,
+// then the sums as a bf16 hi/lo pair into sUh / sUl [16][EPI_UP].  The
+// caller syncs before they are read.
 template <class G, int C>
 __device__ __forceinline__ void u_issue(const EpiArgs& a, int seg, int m0, int nrows, int col, int q,
                                         PartLoad<G, C>& L) {
   part_issue(a.pv, a.lr.u_tile0 + seg, m0, nrows, col, q, L);
 }
 template <class G, int C>
-__device__ __forceinline__ void u_store(PartLoad<G, C>& L, int nrows, int col, int q, float* sU) {
+__device__ __forceinline__ void u_store(PartLoad<G, C>& L, int nrows, int col, int q, bf16* sUh,
+                                        bf16* sUl) {
   float u[G::RPT];
   part_add(L, nrows, q, u);
 #pragma unroll
-  for (int s = 0; s < G::RPT; ++s)
-    if (q + G::NQ * s < nrows) sU[(q + G::NQ * s) * EPI_R + col] = u[s];
+  for (int s = 0; s < G::RPT; ++s) {
+    const int j = q + G::NQ * s;
+    if (j < nrows) {
+      const bf16 h = from_f<bf16>(u[s]);
+      sUh[j * EPI_UP + col] = h;
+      sUl[j * EPI_UP + col] = from_f<bf16>(u[s] - to_f(h));
+    }
+  }
 }
 
 // Row gates of the thread's rows (0 past M).
@@ -320,8 +353,9 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   constexpr int C = 4;
   __shared__ float s_inv[G::RG];
   __shared__ float s_ss[G::RG * EPI_MAX_SS];
-  __shared__ __align__(16) float sU[G::RG * EPI_R];
-  __shared__ float sY[G::RG][TC_BM];
+  __shared__ __align__(16) bf16 sUh[16 * EPI_UP];
+  __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
+  __shared__ float sY[G::RG][TC_BM];          // LoRA dots first, then the rows for RoPE
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
@@ -334,10 +368,10 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   const bool rot = n < qcols + kcols;      // q and k are rotated, v is not
   const bool kv_tile = n >= qcols;
   const int ci = hi < half ? hi : hi - half;
-  // the adapter row is a weight: read while the GEMM before is still running
+  // the adapter rows are weights: read while the GEMM before is still running
   const int seg = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
-  BPart<G> B;
-  if (a.lora) bpart_issue(a, seg, n - a.lr.seg_n0[seg], q, B);
+  BFrag B;
+  if (a.lora) bfrag_issue(a, seg, nt * TC_BM + 16 * (threadIdx.x >> 5) - a.lr.seg_n0[seg], B);
   pdl_wait();
 
   // ---- every global load first
@@ -373,11 +407,17 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   }
 
   // ---- then the arithmetic
-  if (a.lora) u_store(LU, nrows, col, q, sU);
-  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
+  if (a.lora) u_store(LU, nrows, col, q, sUh, sUl);
+  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sUh / sUl complete too
   float acc[G::RPT];
   part_add(LP, nrows, q, acc);
-  if (a.lora) lora_apply<G>(B, sU, q, nrows, gate, acc);
+  if (a.lora) {
+    lora_mma(B, sUh, sUl, &sY[0][0], nrows);
+    __syncthreads();
+    // each thread reads the dots of its own (row, column) entries, which
+    // only it rewrites below
+    lora_add<G>(&sY[0][0], col, q, nrows, gate, acc);
+  }
 #pragma unroll
   for (int s = 0; s < G::RPT; ++s) {
     const int j = q + G::NQ * s;
@@ -459,7 +499,9 @@ __device__ __forceinline__ void next_input(const EpiArgs& a, int nt, int m0, int
 __global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiArgs a) {
   typedef GeoResid G;
   constexpr int C = 6;
-  __shared__ __align__(16) float sU[G::RG * EPI_R];
+  __shared__ __align__(16) bf16 sUh[16 * EPI_UP];
+  __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
+  __shared__ float sDot[G::RG * TC_BM];
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
@@ -468,8 +510,8 @@ __global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiA
   const int n = nt * TC_BM + col;
   // weights (the next norm's gain, the adapter row) before the dependency wait
   const float g = a.g_next ? to_f(a.g_next[n]) : 0.f;
-  BPart<G> B;
-  if (!a.prep && a.lora) bpart_issue(a, 0, n, q, B);
+  BFrag B;
+  if (!a.prep && a.lora) bfrag_issue(a, 0, nt * TC_BM + 16 * (threadIdx.x >> 5), B);
   pdl_wait();
 
   // ---- every global load first
@@ -490,11 +532,15 @@ __global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiA
     // ---- then the arithmetic
     float acc[G::RPT];
     if (a.lora) {
-      u_store(LU, nrows, col, q, sU);
+      u_store(LU, nrows, col, q, sUh, sUl);
       __syncthreads();
+      lora_mma(B, sUh, sUl, sDot, nrows);
     }
     part_add(LP, nrows, q, acc);
-    if (a.lora) lora_apply<G>(B, sU, q, nrows, gate, acc);
+    if (a.lora) {
+      __syncthreads();
+      lora_add<G>(sDot, col, q, nrows, gate, acc);
+    }
 #pragma unroll
     for (int s = 0; s < G::RPT; ++s) {
       const int j = q + G::NQ * s;
@@ -518,7 +564,9 @@ __global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const
   constexpr int C = 2;
   __shared__ float s_inv[G::RG];
   __shared__ float s_ss[G::RG * EPI_MAX_SS];
-  __shared__ __align__(16) float sU[2][G::RG * EPI_R];
+  __shared__ __align__(16) bf16 sUh[16 * EPI_UP];     // one adapter at a time
+  __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
+  __shared__ float sDot[G::RG * TC_BM];
   pdl_trigger();
   const int ft = blockIdx.x;
   int m0, nrows;
@@ -528,10 +576,11 @@ __global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const
   const int ut = a.F / TC_BM + ft;         // the up tile of the same features
   // adapter rows are weights: gate's into registers and up's into L2 while
   // the GEMM before is still running
-  BPart<G> B;
+  BFrag B;
+  const int fw = ft * TC_BM + 16 * (threadIdx.x >> 5);   // the warp's first feature
   if (a.lora) {
-    bpart_issue(a, 0, f, q, B);
-    bpart_prefetch(a, 1, f, q, B);
+    bfrag_issue(a, 0, fw, B);
+    bfrag_prefetch(a, 1, fw);
   }
   pdl_wait();
 
@@ -548,18 +597,23 @@ __global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const
     gate_issue<G>(a, m0, nrows, q, gate);
   }
   // ---- then the arithmetic
-  if (a.lora) {
-    u_store(L0, nrows, col, q, sU[0]);
-    u_store(L1, nrows, col, q, sU[1]);
-  }
-  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sU complete too
+  if (a.lora) u_store(L0, nrows, col, q, sUh, sUl);
+  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sUh / sUl complete too
   float g[G::RPT], u[G::RPT];
   part_add(LG, nrows, q, g);
   part_add(LUp, nrows, q, u);
   if (a.lora) {
-    lora_apply<G>(B, sU[0], q, nrows, gate, g);
-    bpart_issue(a, 1, f, q, B);              // up's adapter half after gate's dot
-    lora_apply<G>(B, sU[1], q, nrows, gate, u);
+    // gate's dots, then up's through the same tiles (up's adapter rows were
+    // prefetched into L2 before the wait)
+    lora_mma(B, sUh, sUl, sDot, nrows);
+    bfrag_issue(a, 1, fw, B);
+    __syncthreads();
+    lora_add<G>(sDot, col, q, nrows, gate, g);
+    u_store(L1, nrows, col, q, sUh, sUl);
+    __syncthreads();
+    lora_mma(B, sUh, sUl, sDot, nrows);
+    __syncthreads();
+    lora_add<G>(sDot, col, q, nrows, gate, u);
   }
   bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
 #pragma unroll

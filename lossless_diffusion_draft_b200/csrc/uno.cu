@@ -540,7 +540,8 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
 
 template <int HD>
 int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                   void* out_lo, unsigned* done, unsigned* done_ctas) {
+                   void* out_lo, unsigned* done, unsigned* done_ctas, const void* l2_pf,
+                   size_t l2_pf_bytes) {
   const uno_shape& s = c->s;
   AttnTcParams p{};
   p.q = (const f16*)c->qbuf;
@@ -573,6 +574,9 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   p.n_splits = S;
   p.ws = c->att_ws;
   p.status = c->d_status;
+  const bool pf_ok = l2_pf && l2_pf_bytes >= 16 && ((uintptr_t)l2_pf & 15) == 0;
+  p.l2_pf = pf_ok ? (const char*)l2_pf : nullptr;
+  p.l2_pf_bytes = pf_ok ? (unsigned long long)(l2_pf_bytes & ~(size_t)15) : 0ull;
   static bool attr = false;
   if (!attr) {
     CK(cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -600,18 +604,23 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
 // done (optional): completion counter for the kernel that writes the output
 // last (the merge); *done_ctas receives its CTA count, 0 when no counter
 // was signalled (then the next kernel waits with pdl_wait).
+// l2_pf (optional): weights of the next projection, prefetched into L2 by the
+// tensor-core attention while it runs.
 template <typename T>
 int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                void* out_lo, unsigned* done = nullptr, unsigned* done_ctas = nullptr) {
+                void* out_lo, unsigned* done = nullptr, unsigned* done_ctas = nullptr,
+                const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
   const uno_shape& s = c->s;
   unsigned dummy = 0;
   if (!done_ctas) done_ctas = &dummy;
   *done_ctas = 0;
   if (c->kv_map_ok) {
     if (s.head_dim == 128)
-      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas);
+      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas,
+                                 l2_pf, l2_pf_bytes);
     if (s.head_dim == 64)
-      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas);
+      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas,
+                                l2_pf, l2_pf_bytes);
   }
   AttnParams p{};
   p.qkv = c->qbuf;
@@ -981,12 +990,15 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     ea.ss = c->ss;
     epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS, false);
 
-    {
-      unsigned* done = next_ctr();
-      rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo, done, &dep_n);
-      if (rc) return rc;
-      dep = dep_n ? done : nullptr;   // no merge launched: the o GEMM waits with pdl_wait
-    }
+    // the o GEMM waits for the attention merge with the grid wait: its CTAs
+    // start only as the attention CTAs leave the SMs, and measured, its
+    // counter poll then completed later than the grid wait
+    // while the attention streams K/V, its idle lanes pull W_o into L2: the o
+    // GEMM's CTAs can only start as the attention CTAs leave the SMs
+    rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo, nullptr,
+                           nullptr, c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2);
+    if (rc) return rc;
+    dep = nullptr;
 
     rc = gemm(c->attn, hhd, hhd, {{c->w[UNO_PROJ_O][l], d}}, {c->lA[UNO_PROJ_O][l]}, &ea.pv);
     if (rc) return rc;
