@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           tma_load_3d(sQl + b * (ATC_QROWS * 128), &qmap, q_full, b * 64, kvh * G, p.q_lo_row + row0);
         }
       }
+      const uint64_t pol = l2_evict_first_policy();   // K/V are read once per pass
       int issued = 0;
       for (int i = 0; i < n && !*s_abort; ++i) {
         const int stage = i % C::STAGES;
@@ -223,9 +224,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 #pragma unroll
         for (int b = 0; b < C::NB; ++b) {
           const int o = stage * C::KV_BYTES + b * (ATC_KT * 128);
-          tma_load_2d(sK + o, &kvmap, &kv_full[stage], b * 64, rk);
-          tma_load_2d(sKl + o, &kvmap, &kv_full[stage], b * 64, rkl);
-          tma_load_2d(sV + o, &kvmap, &kv_full[stage], b * 64, rv);
+          tma_load_2d_stream(sK + o, &kvmap, &kv_full[stage], b * 64, rk, pol);
+          tma_load_2d_stream(sKl + o, &kvmap, &kv_full[stage], b * 64, rkl, pol);
+          tma_load_2d_stream(sV + o, &kvmap, &kv_full[stage], b * 64, rv, pol);
         }
         ++issued;
       }

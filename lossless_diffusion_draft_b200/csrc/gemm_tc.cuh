@@ -172,14 +172,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     x = (kb < p.KB ? kb : kb - p.KB) * TC_BK * KPS;
     y = n_row - p.seg[sg].n0;
   };
+  uint64_t pol_stream = 0;   // set by the TMA issuer
   auto load_a = [&](int u, int stage) {
     const CUtensorMap* map;
     int x, y;
     coords_a(u, map, x, y);
 #pragma unroll
     for (int j = 0; j < KPS; ++j)
-      tma_load_2d(sA + stage * C::A_BYTES + j * TC_A_BYTES, map, &full[stage], x + j * TC_BK, y);
+      tma_load_2d_stream(sA + stage * C::A_BYTES + j * TC_A_BYTES, map, &full[stage], x + j * TC_BK,
+                         y, pol_stream);
   };
+
 
   auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
     const int t = u / KBt, kb = u % KBt;
@@ -220,6 +223,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     prefetch_map(&maps.x);
     for (int s = 0; s < p.nseg; ++s) prefetch_map(&maps.w[s]);
     if (p.dep) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.dep));
+    pol_stream = l2_evict_first_policy();
     for (int i = 0; i < npre; ++i) {
       mbar_expect_tx(&full[i], C::STAGE_BYTES);
       load_a(u0 + i, i);

@@ -235,6 +235,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.out_lo = p.out_lo;
   tp.dep = DUMP ? p.dep : nullptr;
   tp.dep_count = p.dep_count;
+
   using Cfg = TcCfg<NT, SPLIT, KPS>;
   static bool attr = false;
   if (!attr) {

@@ -118,6 +118,34 @@ def test_tiny_fp32_generation():
     assert e2e.mismatches <= tally.mismatches, e2e.notes
 
 
+def test_tiny_fp32_temperature():
+    """Temperature 0.7 (the LM head scales the logits by 1 / T; draft, accept
+    test, residual and bonus all see the tempered distributions): bit-exact
+    fp32 decisions against the oracle, which divides its logits by T."""
+    tally, e2e, _ = _run("tiny", 2, 32, 12, 1e-4, 1e-4, True, max_ctx=160, temperature=0.7)
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
+    assert e2e.mismatches <= tally.mismatches, e2e.notes
+
+
+def test_small_bf16_temperature_scales_logits():
+    """bf16 model at T = 1.25: the draft-pass logits are the T = 1 logits
+    times 1 / T (same kernels, same order: equal up to one fp32 rounding)."""
+    outs = []
+    for t in (1.0, 1.25):
+        cfg, ctx, ids, model, states = _setup("small", 2, 24, 100, temperature=t)
+        req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+        out = torch.zeros((2, cfg["B"] + 1), dtype=torch.int32, device="cuda")
+        n_new = torch.zeros(2, dtype=torch.int32, device="cuda")
+        uno.uno_spec_step(ctx, req, out, n_new)
+        uno.uno_status(ctx)
+        # the draft pass's inputs (prompt, pending token, MASK rows) do not
+        # depend on T: only the LM head's scale differs
+        ld = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_DRAFT, torch.empty((2, cfg["B"] + 1, cfg["vocab"])))
+        outs.append(ld.clone())
+        ctx.close()
+    torch.testing.assert_close(outs[1], outs[0] / 1.25, rtol=2e-6, atol=1e-6)
+
+
 def test_tiny_fp32_split_verify():
     """spec_verify in its split form (reduction kernel, then one deciding CTA
     per request), forced at a size the fused form would take: the same

@@ -222,3 +222,23 @@ def test_synth_param_list_matches_oracle(name):
     a = [(n, tuple(s)) for n, s, _ in synth.param_list(cfg)]
     b = [(n, tuple(s)) for n, s in om.param_names(synth.model_shape(cfg))]
     assert a == b
+
+
+def test_temperature_divides_the_logits():
+    """Logits at temperature T are the T = 1 logits divided by T (the model
+    forward does not depend on T), and softmax(l / T) sharpens as T falls:
+    at T -> 0 the distribution concentrates on the argmax."""
+    shape = _tiny_shape()
+    p = _random_params(shape, 4)
+    toks, pos = [3, 1, 4, 1, 5], np.arange(5)
+    l1, _, _ = om.Model(shape, p).forward(om.KVCache(shape), toks, pos, np.zeros(5))
+    for t in (0.7, 1.3):
+        lt, _, _ = om.Model(_tiny_shape(temperature=t), p).forward(om.KVCache(shape), toks, pos,
+                                                                     np.zeros(5))
+        np.testing.assert_allclose(lt, l1 / t, rtol=1e-12, atol=1e-14)
+    lc, _, _ = om.Model(_tiny_shape(temperature=1e-3), p).forward(om.KVCache(shape), toks, pos,
+                                                                  np.zeros(5))
+    probs = np.exp(lc - lc.max(axis=-1, keepdims=True))
+    probs /= probs.sum(axis=-1, keepdims=True)
+    assert np.all(probs.argmax(axis=-1) == l1.argmax(axis=-1))
+    assert np.all(probs.max(axis=-1) > 0.99)
