@@ -54,7 +54,6 @@ struct AttnTcParams {
   int n_splits, n_qtiles;
   float* ws;                        // split partials [group][split][128][HD + 4]
   int32_t* status;
-  unsigned* done;                   // merge: completion counter for the next GEMM (or null)
   // weights of the projection after the attention, prefetched into L2 by the
   // producer warp's idle lanes while the KV stream leaves HBM bandwidth
   // unused (null: none); 16-byte aligned, a multiple of 16 bytes
@@ -483,7 +482,6 @@ __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const A
     const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD + d;
     store_split<bf16>(p.out, p.out_lo, oo, O / L);
   }
-  dep_signal(p.done);
 }
 
 }  // namespace uno

@@ -541,8 +541,7 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
 
 template <int HD>
 int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                   void* out_lo, unsigned* done, unsigned* done_ctas, const void* l2_pf,
-                   size_t l2_pf_bytes) {
+                   void* out_lo, const void* l2_pf, size_t l2_pf_bytes) {
   const uno_shape& s = c->s;
   AttnTcParams p{};
   p.q = (const f16*)c->qbuf;
@@ -594,34 +593,23 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
     Prof prof(c, UNO_K_ATTN, 0.0);
     // only the rows a query tile can hold: tokens per request x heads per kv head
     const int rows = std::min(ATC_QROWS, rows_per_req * G);
-    p.done = done;
-    if (done) *done_ctas = (unsigned)(ceil_div(rows, ATC_MERGE_ROWS) * groups);
     klaunch(c->genv.pdl, c->stream, dim3(ceil_div(rows, ATC_MERGE_ROWS), groups),
             dim3(HD, ATC_MERGE_ROWS), 0, attn_merge_kernel<HD>, p);
   }
   return UNO_OK;
 }
 
-// done (optional): completion counter for the kernel that writes the output
-// last (the merge); *done_ctas receives its CTA count, 0 when no counter
-// was signalled (then the next kernel waits with pdl_wait).
 // l2_pf (optional): weights of the next projection, prefetched into L2 by the
 // tensor-core attention while it runs.
 template <typename T>
 int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                void* out_lo, unsigned* done = nullptr, unsigned* done_ctas = nullptr,
-                const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
+                void* out_lo, const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
   const uno_shape& s = c->s;
-  unsigned dummy = 0;
-  if (!done_ctas) done_ctas = &dummy;
-  *done_ctas = 0;
   if (c->kv_map_ok) {
     if (s.head_dim == 128)
-      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas,
-                                 l2_pf, l2_pf_bytes);
+      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes);
     if (s.head_dim == 64)
-      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, done, done_ctas,
-                                l2_pf, l2_pf_bytes);
+      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes);
   }
   AttnParams p{};
   p.qkv = c->qbuf;
@@ -991,13 +979,12 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     ea.ss = c->ss;
     epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS, false);
 
-    // the o GEMM waits for the attention merge with the grid wait: its CTAs
-    // start only as the attention CTAs leave the SMs, and measured, its
-    // counter poll then completed later than the grid wait
-    // while the attention streams K/V, its idle lanes pull W_o into L2: the o
-    // GEMM's CTAs can only start as the attention CTAs leave the SMs
-    rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo, nullptr,
-                           nullptr, c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2);
+    // the o GEMM waits for the attention merge with the grid wait (its CTAs
+    // start only as the attention CTAs leave the SMs; measured, a counter
+    // poll completed later); while the attention streams K/V, its idle lanes
+    // pull W_o into L2
+    rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo,
+                           c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2);
     if (rc) return rc;
     dep = nullptr;
 
