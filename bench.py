@@ -267,7 +267,7 @@ def run_uno(args, rank, world, device):
     start_ctx = max(prompt_len, int(mean_ctx - (args.warmup + args.steps) * est_tok / 2))
     P = start_ctx + 1
     prompts = synth.make_prompts(cfg, batch, P, seed=cfg["seed"] + 1000 * rank)
-    streams = [rank * batch + i for i in range(batch)]
+    streams = replica_streams(rank, batch)
     t0 = time.time()
     ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).to(device), [P] * batch, streams=streams)
     torch.cuda.synchronize()
@@ -454,6 +454,12 @@ def run_micro(args, device):
                          "algorithmic_bytes_per_call": nbytes, "peak_source": pk["source"]},
             "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
+
+
+def replica_streams(rank, batch):
+    """Philox streams of a rank's requests: each replica draws from its own,
+    disjoint from every other rank's."""
+    return [rank * batch + i for i in range(batch)]
 
 
 def barrier(world):

@@ -1,0 +1,80 @@
+"""Host side of bench.py (CPU): the reference arm's JSON line, rank-0-only
+printing, and the multi-rank aggregation over gloo (world size 2)."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _run_bench(args, env_extra):
+    env = dict(os.environ, **env_extra)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                   {"WORLD_SIZE": "1", "RANK": "0"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_silently():
+    r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                   {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_replica_streams_are_disjoint():
+    seen = set()
+    for rank in range(8):
+        s = bench.replica_streams(rank, 80)
+        assert len(s) == 80 and not seen.intersection(s)
+        seen.update(s)
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dev = torch.device("cpu")
+        # per-rank step times and token counts: time is the max, tokens the sum
+        ms = bench.reduce_max(10.0 + 5.0 * rank, world, dev)
+        tok = bench.reduce_sum(100 + rank, world, dev)
+        bench.barrier(world)
+        out[rank] = (ms, tok)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregation_over_two_gloo_ranks():
+    port = 29500 + os.getpid() % 1000
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        assert out[0] == out[1] == (15.0, 201)
+
+
+def test_single_rank_aggregation_is_identity():
+    assert bench.reduce_max(3.5, 1, None) == 3.5
+    assert bench.reduce_sum(7, 1, None) == 7

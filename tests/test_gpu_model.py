@@ -343,7 +343,8 @@ def test_counter_sync_matches_grid_dependencies():
     """The fused pipeline with its GEMMs waiting on completion counters gives
     bit-identical logits and tokens to the same pipeline with grid
     dependencies only (the arithmetic and its order are the same), also
-    when the steps replay from captured graphs, and raises no device flag."""
+    when the steps replay from captured graphs and with plain stream-ordered
+    launches, and raises no device flag."""
     cfg = dict(synth.CONFIGS["small"])
     shape = synth.model_shape(cfg)
     shape["dtype"] = cfg["dtype"]
@@ -351,12 +352,15 @@ def test_counter_sync_matches_grid_dependencies():
     prompts = torch.from_numpy(synth.make_prompts(cfg, 3, 40)).cuda()
     B, V = cfg["B"], cfg["vocab"]
     runs = []
-    for counters, graphs in ((False, False), (True, False), (True, True)):
+    # (counters, graphs, programmatic launch)
+    for counters, graphs, pdl in ((False, False, True), (True, False, True), (True, True, True),
+                                  (True, False, False)):
         ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, 3, 200,
                            cfg["seed"], torch.cuda.current_stream())
         assert uno.uno_set_fused(ctx, True)
         uno.uno_set_counter_sync(ctx, counters)
         uno.uno_set_graphs(ctx, graphs)
+        uno.uno_set_pdl(ctx, pdl)
         ids = uno.uno_prefill(ctx, prompts, [40] * 3, streams=[0, 1, 2])
         req = torch.tensor(ids, dtype=torch.int32, device="cuda")
         out = torch.zeros((3, B + 1), dtype=torch.int32, device="cuda")
