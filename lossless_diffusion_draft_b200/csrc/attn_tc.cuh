@@ -22,8 +22,9 @@
 //           only when a tile's max exceeds it by more than 2^8, and write P
 //           (fp16) to shared memory in the MMA's swizzled layout.
 // With several key splits each CTA writes (m, l, O) partials and
-// attn_merge_kernel (one CTA per query row) adds them in split order.  Every
-// wait is bounded.
+// attn_merge_kernel (ATC_MERGE_ROWS query rows per CTA) adds them in split
+// order.  Every wait is bounded.  While it runs, idle lanes of the producer
+// warp prefetch the next projection's weights into L2.
 #pragma once
 
 #include "layers.cuh"

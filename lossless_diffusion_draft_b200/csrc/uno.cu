@@ -1027,10 +1027,11 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
 
 int forward_any(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* req_ids,
                 const int32_t* prompt, int prefill_slot, int prefill_pos0, float* logits) {
-  // The fused pipeline is built for memory-bound passes (its epilogues do
-  // LoRA-B on the CUDA cores and are sized for a few dozen rows); a pass
-  // larger than one GEMM token tile runs the unfused kernels, where LoRA-B is
-  // a tensor-core K extension and the row kernels are bandwidth-bound.
+  // The fused pipeline is built for memory-bound passes (its epilogues are
+  // sized for a few dozen rows, one 16-row MMA tile of LoRA-B per CTA); a
+  // pass larger than one GEMM token tile runs the unfused kernels, where
+  // LoRA-B is a K extension of the tensor-core GEMM and the row kernels are
+  // bandwidth-bound.
   if (c->fused && c->fused_enabled && n_req * rows_per_req <= FUSED_MAX_ROWS)
     return forward_fused(c, kind, n_req, rows_per_req, req_ids, prompt, prefill_slot, prefill_pos0,
                          logits);
