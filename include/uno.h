@@ -309,9 +309,11 @@ int uno_profile_records(uno_ctx *ctx, uno_prof_record *out, int max);
  *                  bytes, 256-byte aligned, zero-filled before its first use
  *                  (the kernels leave its counters zeroed again); calls
  *                  sharing a workspace must not overlap on the GPU.
- * Enqueues two kernels on `stream`: the vocabulary reductions and accept
- * tests, then the residual redraw of each request with a rejection.
- * Returns UNO_ERR_ARG on bad sizes; never synchronises.
+ * Enqueues on `stream` the vocabulary reductions with the accept tests (one
+ * kernel for up to 4096 (row, 8192-logit chunk) CTAs; above that a
+ * reduction kernel and one deciding CTA per request), then the residual
+ * redraw of each request with a rejection.  Returns UNO_ERR_ARG on bad
+ * sizes; never synchronises.
  */
 size_t uno_spec_verify_workspace_bytes(int n_req, int n_tests, int vocab);
 int uno_spec_verify(const float *p_dev, const float *q_dev, const int32_t *drafts_dev,
