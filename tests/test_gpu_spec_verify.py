@@ -116,6 +116,36 @@ def test_special_cases():
     assert out[1, 0] != 7
 
 
+def test_special_cases_split_form():
+    """The closed forms of test_special_cases at a size that takes the split
+    form (8 requests x 32 rows x 19 chunks > 4096 CTAs): q == p accepts every
+    draft; q one-hot on a token p gives no mass rejects test 0 and redraws
+    from the residual, which is p itself."""
+    n_req, n_tests, V = 8, 16, 151936
+    g = torch.Generator().manual_seed(9)
+    p = torch.randn((n_req, n_tests, V), generator=g) * 3
+    q = p.clone()
+    for i in range(1, n_req, 2):
+        q[i] = -float("inf")
+        q[i, :, 11 + i] = 0.0
+        p[i, :, 11 + i] = -float("inf")
+    drafts = np.array([[(5 * i + j) % V for j in range(n_tests)] if i % 2 == 0 else [11 + i] * n_tests
+                       for i in range(n_req)], np.int32)
+    streams = np.arange(n_req, dtype=np.uint32) + 40
+    pos0 = (np.arange(n_req, dtype=np.int32) * 13) % 1000
+    out, n_out, _ = _run_gpu(p.cuda(), q.cuda(), torch.from_numpy(drafts).cuda(),
+                             torch.from_numpy(streams.view(np.int32)).cuda(), torch.from_numpy(pos0).cuda())
+    tally = parity.Tally()
+    for i in range(n_req):
+        if i % 2 == 0:
+            assert n_out[i] == n_tests and list(out[i, :n_tests]) == list(drafts[i]) and out[i, -1] == -1
+        else:
+            assert n_out[i] == 0 and out[i, 0] != 11 + i
+            u = float(uniform(SEED, int(streams[i]), int(pos0[i]), KIND_RESID))
+            parity.check_sample(p[i, 0].double().numpy(), u, int(out[i, 0]), tally, f"residual=p {i}")
+    assert tally.mismatches <= 1, tally.notes
+
+
 def test_microbenchmark_size_sampled():
     """The spec_verify microbenchmark workload at full size: every request's
     output is valid, and sampled requests match the oracle."""
