@@ -458,97 +458,142 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   }
 }
 
-// g * x rows for the next GEMM (hi/lo) and the tile's sums of squares of x:
-// lanes of one slot add over the warp's columns, then the warps in order.
-template <class G>
-__device__ __forceinline__ void next_input(const EpiArgs& a, int nt, int m0, int nrows, int col,
-                                           int q, float g, const float (&xv)[G::RPT]) {
-  __shared__ float red[G::THREADS / 32][G::NQ][G::RPT];
-  const int n = nt * TC_BM + col;
-  bf16* lo = a.lo_off ? a.xn + (size_t)a.lo_off * a.ld_xn : nullptr;
-  float sq[G::RPT];
+// ---------------------------------------------------------------------------
+// o / down (and, with prep = 1, the layer-0 input): grid (d / 128, row groups
+// of GeoResid::RG), RESID_THREADS threads.  Thread t owns one unit: row
+// t / 32 of the group and the four columns 4 (t % 32) .. + 3 of the tile, so
+// warp w holds row w and every global access is a 16-byte one (a
+// contributor's part of the CTA's rows is one contiguous block).  x += y;
+// then the next GEMM's input g * x (hi/lo) and the row's sum of squares over
+// the tile (a warp reduction).
+// ---------------------------------------------------------------------------
+constexpr int RESID_THREADS = GeoResid::RG * 32;
+
+// The parts of output tile nt for one unit: contributors issued C at a
+// time; part4_add adds them in CTA order.
+template <int C>
+struct Part4 {
+  float4 x[C];
+  int first, last, slot;
+  const float* base;
+};
+template <int C>
+__device__ __forceinline__ void part4_issue(const PartView& v, int nt, int m0, int j, int c0, bool live,
+                                            Part4<C>& L) {
+  const int mt = m0 / v.NT;
+  const int t = nt * v.m_tiles + mt;
+  L.first = sk_owner(t * v.KBt, v.units, v.grid);
+  L.last = sk_owner(t * v.KBt + v.KBt - 1, v.units, v.grid);
+  L.slot = v.NT * TC_BM;
+  L.base = v.ws + ((size_t)t * v.NT + (m0 - mt * v.NT) + j) * TC_BM + c0;
 #pragma unroll
-  for (int s = 0; s < G::RPT; ++s) {
-    const int j = q + G::NQ * s;
-    sq[s] = xv[s] * xv[s];
-    if (j < nrows) store_split<bf16>(a.xn, lo, (size_t)(m0 + j) * a.ld_xn + n, g * xv[s]);
+  for (int c = 0; c < C; ++c) {
+    const int i = L.first + c;
+    L.x[c] = (live && i <= L.last) ? __ldcg(reinterpret_cast<const float4*>(L.base + (size_t)i * L.slot))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+template <int C>
+__device__ __forceinline__ float4 part4_add(Part4<C>& L, bool live) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = L.first;; i0 += C) {
 #pragma unroll
-  for (int o = G::NQ; o < 32; o <<= 1)
+    for (int c = 0; c < C; ++c) {
+      acc.x += L.x[c].x; acc.y += L.x[c].y; acc.z += L.x[c].z; acc.w += L.x[c].w;
+    }
+    if (i0 + C > L.last) break;
 #pragma unroll
-    for (int s = 0; s < G::RPT; ++s) sq[s] += __shfl_xor_sync(0xffffffffu, sq[s], o);
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) < G::NQ)
-#pragma unroll
-    for (int s = 0; s < G::RPT; ++s) red[w][q][s] = sq[s];
-  __syncthreads();
-  const int j = threadIdx.x;
-  if (j < nrows) {
-    const int qq = j % G::NQ, s = j / G::NQ;
-    float t = 0.f;
-#pragma unroll
-    for (int k = 0; k < G::THREADS / 32; ++k) t += red[k][qq][s];
-    a.ss_out[(size_t)(m0 + j) * (a.d / TC_BM) + nt] = t;
+    for (int c = 0; c < C; ++c) {
+      const int i = i0 + C + c;
+      L.x[c] = (live && i <= L.last)
+                   ? __ldcg(reinterpret_cast<const float4*>(L.base + (size_t)i * L.slot))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  return acc;
+}
+__device__ __forceinline__ void store4_split(bf16* hi, bf16* lo, size_t i, float4 y) {
+  const __nv_bfloat162 h01 = __floats2bfloat162_rn(y.x, y.y), h23 = __floats2bfloat162_rn(y.z, y.w);
+  uint2 hv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+  hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+  *reinterpret_cast<uint2*>(hi + i) = hv;
+  if (lo) {
+    const __nv_bfloat162 l01 = __floats2bfloat162_rn(y.x - __low2float(h01), y.y - __high2float(h01));
+    const __nv_bfloat162 l23 = __floats2bfloat162_rn(y.z - __low2float(h23), y.w - __high2float(h23));
+    uint2 lv;
+    lv.x = *reinterpret_cast<const uint32_t*>(&l01);
+    lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+    *reinterpret_cast<uint2*>(lo + i) = lv;
   }
 }
 
-// ---------------------------------------------------------------------------
-// o / down (and, with prep = 1, the layer-0 input): grid (d / 128, row
-// groups), GeoResid::THREADS threads.  x += y; then the next GEMM's input.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(GeoResid::THREADS) epi_resid_kernel(const EpiArgs a) {
+__global__ void __launch_bounds__(RESID_THREADS) epi_resid_kernel(const EpiArgs a) {
   typedef GeoResid G;
   constexpr int C = 6;
   __shared__ __align__(16) bf16 sUh[16 * EPI_UP];
   __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
-  __shared__ float sDot[G::RG * TC_BM];
+  __shared__ __align__(16) float sDot[G::RG * TC_BM];
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
   if (!row_group<G>(a, &m0, &nrows)) { dep_signal(a.done); return; }
-  const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
-  const int n = nt * TC_BM + col;
-  // weights (the next norm's gain, the adapter row) before the dependency wait
-  const float g = a.g_next ? to_f(a.g_next[n]) : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = warp;                        // the unit's row in the group
+  const int c0 = 4 * lane;                   // its first column in the tile
+  const int n = nt * TC_BM + c0;
+  const bool live = j < nrows;
+  const bool lora = !a.prep && a.lora;
+  // weights (the next norm's gains, the adapter rows) before the dependency wait
+  float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (a.g_next) {
+    const uint2 gg = __ldg(reinterpret_cast<const uint2*>(a.g_next + n));
+    const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&gg.x);
+    const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&gg.y);
+    g4 = make_float4(__low2float(g01), __high2float(g01), __low2float(g23), __high2float(g23));
+  }
   BFrag B;
-  if (!a.prep && a.lora) bfrag_issue(a, 0, nt * TC_BM + 16 * (threadIdx.x >> 5), B);
+  if (lora && warp < 8) bfrag_issue(a, 0, nt * TC_BM + 16 * warp, B);
   pdl_wait();
 
   // ---- every global load first
-  float xv[G::RPT];
-#pragma unroll
-  for (int s = 0; s < G::RPT; ++s) {
-    const int j = q + G::NQ * s;
-    xv[s] = j < nrows ? a.x[(size_t)(m0 + j) * a.d + n] : 0.f;
-  }
+  const size_t xi = (size_t)(m0 + j) * a.d + n;
+  float4 xv = live ? *reinterpret_cast<const float4*>(a.x + xi) : make_float4(0.f, 0.f, 0.f, 0.f);
   if (!a.prep) {
-    PartLoad<G, C> LU, LP;
-    float gate[G::RPT];
-    if (a.lora) {
-      u_issue(a, 0, m0, nrows, col, q, LU);
-      gate_issue<G>(a, m0, nrows, q, gate);
+    Part4<C> LU, LP;
+    float gt = 0.f;
+    if (lora) {
+      part4_issue(a.pv, a.lr.u_tile0, m0, j, c0, live, LU);
+      gt = live ? __ldg(a.lr.row_gate + m0 + j) : 0.f;
     }
-    part_issue(a.pv, nt, m0, nrows, col, q, LP);
+    part4_issue(a.pv, nt, m0, j, c0, live, LP);
     // ---- then the arithmetic
-    float acc[G::RPT];
-    if (a.lora) {
-      u_store(LU, nrows, col, q, sUh, sUl);
+    if (lora) {
+      // U's rows as bf16 hi/lo for the tensor-core LoRA-B
+      const float4 u = part4_add(LU, live);
+      if (live) store4_split(sUh, sUl, (size_t)j * EPI_UP + c0, u);
       __syncthreads();
-      lora_mma(B, sUh, sUl, sDot, nrows);
+      if (warp < 8) lora_mma(B, sUh, sUl, sDot, nrows);
     }
-    part_add(LP, nrows, q, acc);
-    if (a.lora) {
+    float4 y = part4_add(LP, live);
+    if (lora) {
       __syncthreads();
-      lora_add<G>(sDot, col, q, nrows, gate, acc);
+      const float4 dt = *reinterpret_cast<const float4*>(sDot + j * TC_BM + c0);
+      y.x += gt * dt.x; y.y += gt * dt.y; y.z += gt * dt.z; y.w += gt * dt.w;
     }
-#pragma unroll
-    for (int s = 0; s < G::RPT; ++s) {
-      const int j = q + G::NQ * s;
-      xv[s] += acc[s];
-      if (j < nrows) a.x[(size_t)(m0 + j) * a.d + n] = xv[s];
-    }
+    xv.x += y.x; xv.y += y.y; xv.z += y.z; xv.w += y.w;
+    if (live) *reinterpret_cast<float4*>(a.x + xi) = xv;
   }
-  if (a.g_next) next_input<G>(a, nt, m0, nrows, col, q, g, xv);
+  if (a.g_next) {
+    bf16* lo = a.lo_off ? a.xn + (size_t)a.lo_off * a.ld_xn : nullptr;
+    if (live)
+      store4_split(a.xn, lo, (size_t)(m0 + j) * a.ld_xn + n,
+                   make_float4(g4.x * xv.x, g4.y * xv.y, g4.z * xv.z, g4.w * xv.w));
+    float sq = xv.x * xv.x + xv.y * xv.y + xv.z * xv.z + xv.w * xv.w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (live && lane == 0) a.ss_out[(size_t)(m0 + j) * (a.d / TC_BM) + nt] = sq;
+  }
   dep_signal(a.done);
 }
 

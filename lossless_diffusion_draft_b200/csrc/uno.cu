@@ -964,7 +964,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ea.lora = 0;
   ea.pv = PartView{nullptr, M, 0, 1, 1, 1};
   ea.g_next = (const bf16*)c->attn_norm[0];
-  epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, true);
+  epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, RESID_THREADS, true);
   ea.prep = 0;
 
   for (int l = 0; l < s.n_layers; ++l) {
@@ -993,7 +993,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_O][l], d}});
     ea.ss = nullptr;
     ea.g_next = (const bf16*)c->ffn_norm[l];
-    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, true);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, RESID_THREADS, true);
 
     rc = gemm(c->xn, xn_ld, d, {{c->w[UNO_PROJ_GATE][l], F}, {c->w[UNO_PROJ_UP][l], F}},
               {c->lA[UNO_PROJ_GATE][l], c->lA[UNO_PROJ_UP][l]}, &ea.pv);
@@ -1007,7 +1007,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_DOWN][l], d}});
     ea.ss = nullptr;
     ea.g_next = l + 1 < s.n_layers ? (const bf16*)c->attn_norm[l + 1] : nullptr;
-    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, GeoResid::THREADS, l + 1 < s.n_layers);
+    epi(epi_resid_kernel, d / TC_BM, GeoResid::RG, RESID_THREADS, l + 1 < s.n_layers);
   }
   if (logits) {
     bf16* xn_lo = split ? (bf16*)c->xn + (size_t)lo * xn_ld : nullptr;
