@@ -78,6 +78,31 @@ def sample_token(logits, u):
     return _inverse_cdf(w, u)
 
 
+def top_p_logits(logits, top_p):
+    """Nucleus filter of one row (Walkthrough §我的判断: the lossless claim is
+    stated for the sampling distribution with temperature 1 and top-p 0.95).
+
+    Reading: the nucleus is the smallest set of most probable tokens whose
+    probability reaches ``top_p`` -- tokens ordered by probability, ties by
+    token id, and the token that crosses ``top_p`` is kept; every other
+    logit becomes -inf, so softmax of the result is the renormalised
+    filtered distribution.  Speculative sampling applies the same filter to
+    the AR rows p and to the drafter's rows q, and is then lossless with
+    respect to the filtered p.  ``top_p >= 1`` keeps every token.
+    """
+    logits = np.asarray(logits, dtype=np.float64)
+    if top_p >= 1.0:
+        return logits.copy()
+    p = np.exp(log_softmax(logits))
+    order = np.lexsort((np.arange(p.size), -p))      # most probable first, ties by id
+    cum = np.cumsum(p[order])
+    k = min(int(np.searchsorted(cum, top_p, side="left")), p.size - 1)
+    out = np.full_like(logits, -np.inf)
+    keep = order[: k + 1]
+    out[keep] = logits[keep]
+    return out
+
+
 def accept_draft(p_logits, q_logits, token, u):
     """Accept test: log u < log p(token) - log q(token), i.e. u < p/q."""
     lp = log_softmax(p_logits)[token]
@@ -187,22 +212,25 @@ def verify_pass(model, cache_with_pending, c, drafts):
     return model.forward(cache_with_pending, drafts, np.arange(c + 1, c + B + 1), np.zeros(B))
 
 
-def spec_step(model, state, B, seed, drafts=None, uniform_fn=None):
+def spec_step(model, state, B, seed, drafts=None, uniform_fn=None, top_p=None):
     """One Psi-Spec iteration; returns (new_state, StepResult).
 
     ``drafts`` (optional) replaces the sampled block x_1..x_B, so a test can
     verify exactly the block another implementation drafted.
     ``uniform_fn(kind, position)`` (optional) replaces the Philox uniforms.
+    ``top_p`` (optional) filters every sampled or verified row, p and q
+    alike, with :func:`top_p_logits`; the StepResult keeps the raw logits.
     """
     if uniform_fn is None:
         def uniform_fn(kind, position):
             return float(uniform(seed, state.stream, position, kind))
+    filt = (lambda l: l) if top_p is None else (lambda l: top_p_logits(l, top_p))
     c = state.c
     logits_d, kd, vd = draft_pass(model, state, B)
     if drafts is None:
-        x = [sample_token(logits_d[0], uniform_fn(KIND_FIRST, c + 1))]
+        x = [sample_token(filt(logits_d[0]), uniform_fn(KIND_FIRST, c + 1))]
         for i in range(2, B + 1):
-            x.append(sample_token(logits_d[i], uniform_fn(KIND_DRAFT, c + i)))
+            x.append(sample_token(filt(logits_d[i]), uniform_fn(KIND_DRAFT, c + i)))
     else:
         x = [int(t) for t in drafts]
     cache = state.cache.copy()
@@ -210,11 +238,11 @@ def spec_step(model, state, B, seed, drafts=None, uniform_fn=None):
     logits_v, kv_k, kv_v = verify_pass(model, cache, c, x)
 
     # tested draft j (0-based) is x_{j+2} at position c+j+2
-    p_rows = [logits_v[j] for j in range(B - 1)]   # p_{j+2} from verify row j
-    q_rows = [logits_d[j + 2] for j in range(B - 1)]
+    p_rows = [filt(logits_v[j]) for j in range(B - 1)]   # p_{j+2} from verify row j
+    q_rows = [filt(logits_d[j + 2]) for j in range(B - 1)]
     u_acc = [uniform_fn(KIND_ACCEPT, c + j + 2) for j in range(B - 1)]
     u_res = [uniform_fn(KIND_RESID, c + j + 2) for j in range(B)]
-    n_acc, y, bits = verify_block(p_rows, q_rows, x[1:], u_acc, u_res, logits_v[B - 1])
+    n_acc, y, bits = verify_block(p_rows, q_rows, x[1:], u_acc, u_res, filt(logits_v[B - 1]))
     a = 1 + n_acc
     cache.append(kv_k, kv_v, range(a))             # positions c+1..c+a
     emitted = x[:a] + [y]
@@ -223,14 +251,16 @@ def spec_step(model, state, B, seed, drafts=None, uniform_fn=None):
     return new_state, res
 
 
-def ar_step(model, state, seed, uniform_fn=None):
-    """AR-only decode: one row (pending, gate 0); emits one token."""
+def ar_step(model, state, seed, uniform_fn=None, top_p=None):
+    """AR-only decode: one row (pending, gate 0); emits one token (from the
+    ``top_p`` nucleus when given)."""
     if uniform_fn is None:
         def uniform_fn(kind, position):
             return float(uniform(seed, state.stream, position, kind))
     c = state.c
     logits, k, v = model.forward(state.cache, [state.pending], [c], [0.0])
-    y = sample_token(logits[0], uniform_fn(KIND_FIRST, c + 1))
+    row = logits[0] if top_p is None else top_p_logits(logits[0], top_p)
+    y = sample_token(row, uniform_fn(KIND_FIRST, c + 1))
     cache = state.cache.copy()
     cache.append(k, v, [0])
     return DecodeState(state.tokens + [y], cache, state.stream), logits[0], y

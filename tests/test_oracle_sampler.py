@@ -336,3 +336,113 @@ def test_step_invariants_over_a_generation():
         assert all(res.accept_bits[: res.a - 1])
         if res.a < B:
             assert not res.accept_bits[res.a - 1]
+
+
+# ---------------------------------------------------------------------------
+# top-p (nucleus) filtering.
+# ---------------------------------------------------------------------------
+
+def _filtered_probs(logits, top_p):
+    f = ops.top_p_logits(np.asarray(logits, dtype=np.float64), top_p)
+    e = np.exp(f - np.max(f))
+    return e / e.sum()
+
+
+def test_top_p_fixtures():
+    """Hand-computed nuclei on exact binary fractions (cumulative sums away
+    from the thresholds): the token that crosses top_p is kept, ties go by
+    token id, top_p >= 1 keeps everything, a tiny top_p is greedy."""
+    l = np.log([0.5, 0.25, 0.125, 0.125])
+    np.testing.assert_allclose(_filtered_probs(l, 0.4), [1, 0, 0, 0], atol=1e-15)
+    np.testing.assert_allclose(_filtered_probs(l, 0.7), [2 / 3, 1 / 3, 0, 0], rtol=1e-13)
+    np.testing.assert_allclose(_filtered_probs(l, 0.8), [4 / 7, 2 / 7, 1 / 7, 0], rtol=1e-13)
+    np.testing.assert_array_equal(ops.top_p_logits(l, 1.0), l)
+    # ties: the most probable tokens 1, 2, 3 share 0.3; two of them (by id) reach 0.5
+    lt = np.log([0.1, 0.3, 0.3, 0.3])
+    np.testing.assert_allclose(_filtered_probs(lt, 0.5), [0, 0.5, 0.5, 0], atol=1e-15)
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        z = rng.standard_normal(50) * 3
+        g = _filtered_probs(z, 1e-9)
+        assert g[np.argmax(z)] == 1.0 and np.count_nonzero(g) == 1
+
+
+def test_top_p_nucleus_is_minimal():
+    """On random rows: the kept mass reaches top_p, dropping the least
+    probable kept token falls below it, and no dropped token is more
+    probable than a kept one."""
+    rng = np.random.default_rng(4)
+    for trial in range(50):
+        z = rng.standard_normal(200) * (0.5 + trial / 10)
+        top_p = float(rng.uniform(0.05, 0.99))
+        p = _softmax(z)
+        kept = np.isfinite(ops.top_p_logits(z, top_p))
+        assert p[kept].sum() >= top_p
+        assert p[kept].sum() - p[kept].min() < top_p
+        if (~kept).any():
+            assert p[~kept].max() <= p[kept].min()
+
+
+def test_top_p_one_leaves_the_iteration_unchanged():
+    shape, prm = _tiny_v16(2)
+    m = MemoModel(shape, prm)
+    st = ops.prefill(m, [2, 7, 11])
+    for _ in range(4):
+        n1, r1 = ops.spec_step(m, st, 3, seed=5)
+        n2, r2 = ops.spec_step(m, st, 3, seed=5, top_p=1.0)
+        assert r1.emitted == r2.emitted and r1.accept_bits == r2.accept_bits
+        st = n1
+
+
+def test_top_p_enumeration_is_lossless():
+    """With p and q filtered alike (top-p 0.9), one iteration's first two
+    emitted tokens follow the filtered AR chain p'(t1) p'(t2 | t1) exactly."""
+    shape, prm = _tiny_v16(0)
+    m = MemoModel(shape, prm)
+    state = ops.prefill(m, [3, 9, 1, 4])
+    B, V, top_p = 2, shape["vocab"], 0.9
+    leaves = defaultdict(float)
+
+    def run(assign, probe_key=None, probe_u=None):
+        requested = []
+
+        def ufn(kind, pos):
+            key = (kind, pos)
+            requested.append(key)
+            if key == probe_key:
+                return probe_u
+            return assign.get(key, 0.5)
+
+        _, res = ops.spec_step(m, state, B, seed=0, uniform_fn=ufn, top_p=top_p)
+        return requested, (tuple(res.drafts), tuple(res.accept_bits), res.a, res.next_token), res
+
+    def dfs(assign, weight):
+        requested, _, res = run(assign)
+        free = [k for k in requested if k not in assign]
+        if not free:
+            leaves[tuple(res.emitted)] += weight
+            return
+        key = free[0]
+        meas, points = outcome_measures(lambda u: run(assign, key, u)[1], with_points=True)
+        for trace, w in meas.items():
+            if w >= 1e-14:
+                dfs({**assign, key: points[trace]}, weight * w)
+
+    dfs({}, 1.0)
+    law = np.zeros((V, V))
+    for emitted, w in leaves.items():
+        law[emitted[0], emitted[1]] += w
+    assert abs(law.sum() - 1.0) < 1e-12
+    c = state.c
+    l1, k1, v1 = m.forward(state.cache, [state.pending], [c], [0.0])
+    p1 = _filtered_probs(l1[0], top_p)
+    cache = state.cache.copy()
+    cache.append(k1, v1, [0])
+    want = np.zeros((V, V))
+    for t1 in range(V):
+        if p1[t1] > 0:
+            l2, _, _ = m.forward(cache, [t1], [c + 1], [0.0])
+            want[t1] = p1[t1] * _filtered_probs(l2[0], top_p)
+    assert np.max(np.abs(law - want)) < 1e-12
+    # the filter removes tokens: some outcomes have zero probability
+    assert np.count_nonzero(want) < V * V
