@@ -96,7 +96,7 @@ struct Geo {
   static constexpr int SS_PT = (RG * EPI_MAX_SS + THREADS - 1) / THREADS;
 };
 typedef Geo<9, 2> GeoQkv;     // 17-row draft pass: two row groups
-typedef Geo<9, 2> GeoResid;
+typedef Geo<9, 2> GeoResid;   // its row groups only: the residual kernel has a 16-byte unit layout
 typedef Geo<9, 2> GeoSwiglu;
 
 // Row groups never straddle an m-tile of the GEMM (the part slots are per
