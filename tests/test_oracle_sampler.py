@@ -446,3 +446,14 @@ def test_top_p_enumeration_is_lossless():
     assert np.max(np.abs(law - want)) < 1e-12
     # the filter removes tokens: some outcomes have zero probability
     assert np.count_nonzero(want) < V * V
+
+
+def test_top_p_with_masked_logits():
+    """Rows that already hold -inf (tokens with no mass): they are never
+    kept, and a row with one finite logit keeps exactly that token."""
+    z = np.array([0.3, -np.inf, 1.2, -np.inf, -0.5])
+    kept = np.isfinite(ops.top_p_logits(z, 0.99))
+    assert not kept[1] and not kept[3] and kept[2]
+    one = np.array([-np.inf, -np.inf, 0.7, -np.inf])
+    np.testing.assert_array_equal(np.isfinite(ops.top_p_logits(one, 0.5)), [False, False, True, False])
+    np.testing.assert_allclose(_filtered_probs(one, 0.95), [0, 0, 1, 0])
