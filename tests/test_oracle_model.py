@@ -242,3 +242,125 @@ def test_temperature_divides_the_logits():
     probs /= probs.sum(axis=-1, keepdims=True)
     assert np.all(probs.argmax(axis=-1) == l1.argmax(axis=-1))
     assert np.all(probs.max(axis=-1) > 0.99)
+
+
+# ---------------------------------------------------------------------------
+# Layer composition.  The elementary ops above are pinned one by one; these
+# closed forms pin how Model.forward puts them together: which RMSNorm feeds
+# which block, that the attention and FFN outputs enter only through o and
+# down as residual adds, that SiLU acts on the gate projection and multiplies
+# the up projection, and the final norm / untied head / temperature.
+# (Walkthrough §一句话直觉: one causal Transformer whose frozen AR weights
+# carry the diffusion path as a gated LoRA; the decoder layout is the
+# Qwen3-style pre-norm block the workloads name.)
+# ---------------------------------------------------------------------------
+
+def _one_layer_shape(**kw):
+    s = dict(n_layers=1, d_model=4, n_heads=1, n_kv_heads=1, head_dim=4, ffn_dim=2, vocab=4,
+             mask_id=3, rope_theta=1e4, rms_eps=0.0, lora_rank=1, lora_alpha=1.0, temperature=1.0)
+    s.update(kw)
+    return s
+
+
+def _zero_params(shape):
+    return {name: np.zeros(shp) for name, shp in om.param_names(shape)}
+
+
+def test_composition_skeleton_with_o_and_down_zeroed():
+    """w_o = w_down = 0 in every layer: the residual stream keeps the raw
+    embedding row, so logits = lm_head . rmsnorm(embed[t], final_norm) / T
+    whatever the attention, gate, up weights, gains and LoRA gates are."""
+    shape = _tiny_shape(temperature=0.8)
+    p = _random_params(shape, 11)
+    for l in range(shape["n_layers"]):
+        for proj in ("o", "down"):
+            p[f"l{l}.w_{proj}"] = np.zeros_like(p[f"l{l}.w_{proj}"])
+            p[f"l{l}.lora_{proj}.B"] = np.zeros_like(p[f"l{l}.lora_{proj}.B"])
+    m = om.Model(shape, p)
+    toks = [5, 9, 2, 11, 30]
+    logits, _, _ = m.forward(om.KVCache(shape), toks, np.arange(5), [0, 1, 0, 1, 1])
+    e = p["embed"][toks]
+    g = p["final_norm"]
+    for i in range(5):
+        rms = math.sqrt(sum(v * v for v in e[i]) / shape["d_model"] + shape["rms_eps"])
+        want = [sum(p["lm_head"][t][j] * e[i][j] / rms * g[j] for j in range(shape["d_model"])) / 0.8
+                for t in range(shape["vocab"])]
+        np.testing.assert_allclose(logits[i], want, rtol=1e-12, atol=1e-12)
+
+
+def test_composition_attention_branch_uses_attn_norm():
+    """One token, one layer, w_down = 0, W_v = W_o = I, lm_head = I, final
+    gain 1, eps 0.  A single key gets softmax weight 1, so the attention
+    output is that token's value row and x1 = x + g_attn * x / rms(x).
+    x = (3, 0, 4, 0): rms = 2.5, x / rms = (1.2, 0, 1.6, 0); attn_norm gains
+    (1, 2, 3, 4) give x1 = (4.2, 0, 8.8, 0).  The ffn_norm gains (5, ...)
+    would give (9, 0, 12, 0) if the two norms were swapped."""
+    shape = _one_layer_shape()
+    p = _zero_params(shape)
+    p["embed"][1] = [3.0, 0.0, 4.0, 0.0]
+    p["l0.attn_norm"] = np.array([1.0, 2.0, 3.0, 4.0])
+    p["l0.ffn_norm"] = np.array([5.0, 5.0, 5.0, 5.0])
+    p["l0.w_v"] = np.eye(4)
+    p["l0.w_o"] = np.eye(4)
+    p["l0.w_q"] = np.eye(4)
+    p["l0.w_k"] = np.eye(4)
+    p["lm_head"] = np.eye(4)
+    p["final_norm"] = np.ones(4)
+    logits, k_rows, v_rows = om.Model(shape, p).forward(om.KVCache(shape), [1], [0], [0.0])
+    x1 = np.array([4.2, 0.0, 8.8, 0.0])
+    rms1 = math.sqrt((4.2 ** 2 + 8.8 ** 2) / 4)
+    np.testing.assert_allclose(logits[0], x1 / rms1, rtol=1e-13, atol=1e-15)
+    # the cached value row is W_v applied to the attn-normed input
+    np.testing.assert_allclose(v_rows[0][0, 0], [1.2, 0.0, 4.8, 0.0], rtol=1e-13, atol=1e-15)
+
+
+def test_composition_ffn_is_silu_gate_times_up_on_ffn_norm():
+    """One token, one layer, w_o = 0 (x1 = x).  x = (2, 2, 2, 2), eps 0:
+    x / rms = 1 everywhere; ffn_norm gains 0.5 give n = (0.5, ...).  W_gate
+    row 0 = (4, 0, 0, 0) -> gate 2; W_up row 0 = (0, -6, 0, 0) -> up -3;
+    W_down column 0 = e_0.  x2 = x + silu(2) * (-3) e_0 with
+    silu(2) = 2 / (1 + e^-2).  Swapping the roles would give
+    silu(-3) * 2 = -6 / (1 + e^3); the attn_norm gains (7, ...) would give
+    gate 28, up -42 if the two norms were swapped."""
+    shape = _one_layer_shape()
+    p = _zero_params(shape)
+    p["embed"][2] = [2.0, 2.0, 2.0, 2.0]
+    p["l0.attn_norm"] = np.full(4, 7.0)
+    p["l0.ffn_norm"] = np.full(4, 0.5)
+    p["l0.w_gate"][0] = [4.0, 0.0, 0.0, 0.0]
+    p["l0.w_up"][0] = [0.0, -6.0, 0.0, 0.0]
+    p["l0.w_down"][:, 0] = [1.0, 0.0, 0.0, 0.0]
+    p["lm_head"] = np.eye(4)
+    p["final_norm"] = np.ones(4)
+    logits, _, _ = om.Model(shape, p).forward(om.KVCache(shape), [2], [0], [0.0])
+    act = -3.0 * 2.0 / (1.0 + math.exp(-2.0))
+    x2 = np.array([2.0 + act, 2.0, 2.0, 2.0])
+    np.testing.assert_allclose(logits[0], x2 / math.sqrt(np.mean(x2 * x2)), rtol=1e-13, atol=1e-15)
+    swapped = np.array([2.0 + 2.0 * (-3.0) / (1.0 + math.exp(3.0)), 2.0, 2.0, 2.0])
+    assert np.max(np.abs(logits[0] - swapped / math.sqrt(np.mean(swapped * swapped)))) > 0.1
+
+
+def test_composition_gated_lora_on_every_projection():
+    """With the gate on, each projection is W + (alpha / r) B A: a model with
+    adapters and gate 1 equals the adapter-free model whose base weights are
+    W + (alpha / r) B A, on every one of the seven projections at once (and
+    gate 0 equals the plain base model)."""
+    shape = _tiny_shape()
+    p = _random_params(shape, 12, lora_b_std=0.3)
+    merged = dict(p)
+    plain = dict(p)
+    scale = shape["lora_alpha"] / shape["lora_rank"]
+    for l in range(shape["n_layers"]):
+        for proj in om.PROJ:
+            A, B = p[f"l{l}.lora_{proj}.A"], p[f"l{l}.lora_{proj}.B"]
+            merged[f"l{l}.w_{proj}"] = p[f"l{l}.w_{proj}"] + scale * (B @ A)
+            merged[f"l{l}.lora_{proj}.B"] = np.zeros_like(B)
+            plain[f"l{l}.lora_{proj}.B"] = np.zeros_like(B)
+    toks, pos = [4, 8, 15, 16, 23], np.arange(5)
+    on, _, _ = om.Model(shape, p).forward(om.KVCache(shape), toks, pos, np.ones(5))
+    want, _, _ = om.Model(shape, merged).forward(om.KVCache(shape), toks, pos, np.zeros(5))
+    np.testing.assert_allclose(on, want, rtol=1e-10, atol=1e-10)
+    off, _, _ = om.Model(shape, p).forward(om.KVCache(shape), toks, pos, np.zeros(5))
+    base, _, _ = om.Model(shape, plain).forward(om.KVCache(shape), toks, pos, np.zeros(5))
+    np.testing.assert_array_equal(off, base)
+    assert np.max(np.abs(on - off)) > 1e-2
