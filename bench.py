@@ -18,7 +18,7 @@ rank runs an independent replica on its own requests (the path has no
 exchange step): replicas only, weak scaling.
 
 --impl reference times the CPU oracle instead, on a bounded sample of the
-same workload (see `oracle_step_sample`).
+same workload (see `OracleSample`).
 """
 
 import argparse
@@ -59,12 +59,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, enabled=True):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.enabled = enabled
 
     def __enter__(self):
+        if not self.enabled:
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
@@ -118,58 +121,83 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample).
 # ---------------------------------------------------------------------------
-def oracle_step_sample(cfg, context, tokens_per_step, budget_s=20.0):
-    """Seconds per Psi-Spec iteration of the oracle, from a bounded sample.
+class OracleSample:
+    """The CPU oracle on a bounded sample of a workload's Psi-Spec iteration.
 
-    The sample runs the oracle's draft and verify forwards through ONE layer
-    of the workload's shape (random float64 weights, a KV cache of `context`
-    positions) plus the final norm, the LM head and the sampler over the
-    block; the per-iteration time is layers x (one-layer time) + head time.
+    The oracle's own iteration (draft forward, draft_sample, verify forward,
+    spec_verify with its residual or bonus draw, commit) runs on a ONE-layer
+    model of the workload's shape - full vocabulary, random float64 weights
+    (base N(0, 0.02), LoRA B N(0, b_std)), a KV cache of `context` random
+    positions - which gives the cost of the LM head and the sampler and the
+    tokens the iteration emits.  The draft and verify forwards of one layer
+    alone (a 16-token vocabulary, so no head cost) are timed beside it.  The
+    iteration time of the L-layer model is then
+        T(iteration, 1 layer) + (L - 1) * T(one layer's two forwards),
+    and the tokens per iteration are those the sampled iterations emitted.
     """
-    from oracle import model as om
-    from oracle import psispec as ops
 
-    one = dict(synth_shape(cfg), n_layers=1)
-    rng = np.random.default_rng(0)
-    params = {}
-    for name, shp in om.param_names(one):
-        params[name] = np.ones(shp) if name.endswith("norm") else rng.standard_normal(shp) * 0.02
-    m = om.Model(one, params)
-    Hkv, hd, B = one["n_kv_heads"], one["head_dim"], cfg["B"]
-    cache = om.KVCache(one)
-    cache.k[0] = rng.standard_normal((context, Hkv, hd))
-    cache.v[0] = rng.standard_normal((context, Hkv, hd))
-    st = ops.DecodeState(list(rng.integers(0, one["vocab"] - 1, context + 1)), cache, 0)
-    head = params["lm_head"]
-    t0 = time.perf_counter()
-    reps = 0
-    layer_t = head_t = 0.0
-    while True:
-        a = time.perf_counter()
-        # one layer of the draft pass (B+1 rows) and of the verify pass (B rows)
-        ops.draft_pass(m, st, B)
+    def __init__(self, cfg, context, seed=0):
+        from oracle import model as om
+        from oracle import psispec as ops
+        self.om, self.ops, self.cfg = om, ops, cfg
+        self.L = cfg["n_layers"]
+        rng = np.random.default_rng(seed)
+        self.full = self._model(dict(synth_shape(cfg), n_layers=1), rng)
+        small = dict(synth_shape(cfg), n_layers=1, vocab=16, mask_id=15)
+        self.layer = self._model(small, rng)
+        Hkv, hd = cfg["n_kv_heads"], cfg["head_dim"]
+        cache = om.KVCache(self.full.shape)
+        cache.k[0] = rng.standard_normal((context, Hkv, hd))
+        cache.v[0] = rng.standard_normal((context, Hkv, hd))
+        toks = [int(t) for t in rng.integers(0, cfg["vocab"] - 1, context + 1)]
+        self.state = ops.DecodeState(toks, cache, 0)
+        self.context = context
+
+    def _model(self, shape, rng):
+        params = {}
+        for name, shp in self.om.param_names(shape):
+            if name.endswith("norm"):
+                params[name] = np.ones(shp)
+            else:
+                std = self.cfg["lora_b_std"] if name.endswith(".B") else 0.02
+                params[name] = rng.standard_normal(shp, dtype=np.float32).astype(np.float64) * std
+        return self.om.Model(shape, params)
+
+    def step(self, it):
+        """One sampled iteration: (seconds for the L-layer model, tokens emitted)."""
+        ops, B = self.ops, self.cfg["B"]
+        st = self.state
+        t0 = time.perf_counter()
+        _, res = ops.spec_step(self.full, st, B, self.cfg["seed"] + it)
+        t1 = time.perf_counter()
+        small = ops.DecodeState([1] * (st.c + 1), st.cache, 0)
+        ops.draft_pass(self.layer, small, B)
         cache2 = st.cache.copy()
-        ops.verify_pass(m, cache2, st.c, [int(t) for t in rng.integers(0, one["vocab"], B)])
-        b = time.perf_counter()
-        # LM head over the 2B+1 rows, and the sampler over the block
-        h = rng.standard_normal((2 * B + 1, one["d_model"]))
-        logits = h @ head.T
-        for i in range(B):
-            ops.sample_token(logits[i], 0.5)
-        ops.verify_block(list(logits[B:2 * B - 1]), list(logits[1:B]), [1] * (B - 1),
-                         [0.5] * (B - 1), [0.5] * B, logits[2 * B])
-        c = time.perf_counter()
-        layer_t += b - a
-        head_t += c - b
-        reps += 1
-        if c - t0 > budget_s or reps >= 3:
+        ops.verify_pass(self.layer, cache2, st.c, [1] * B)
+        t2 = time.perf_counter()
+        return (t1 - t0) + (self.L - 1) * (t2 - t1), len(res.emitted)
+
+    def describe(self, n):
+        return (f"oracle (numpy float64) Psi-Spec iterations on a 1-layer model of the workload's "
+                f"shape (full vocabulary) at context {self.context}, plus {self.L - 1} x the draft and "
+                f"verify forwards of one layer; {n} sampled iterations; tokens per iteration "
+                f"measured from those iterations")
+
+
+def oracle_baseline(cfg, context, budget_s=20.0, max_iters=3):
+    """(tokens/s, seconds per iteration, tokens per iteration, description)."""
+    s = OracleSample(cfg, context)
+    t0 = time.perf_counter()
+    times, toks = [], []
+    while True:
+        t, n = s.step(len(times))
+        times.append(t)
+        toks.append(n)
+        if time.perf_counter() - t0 > budget_s or len(times) >= max_iters:
             break
-    # the one-layer passes include the embedding/head of the 1-layer model;
-    # subtract nothing (a small overestimate of the per-layer time)
-    step_s = cfg["n_layers"] * layer_t / reps + head_t / reps
-    desc = (f"oracle (numpy float64) draft+verify forwards of 1 of {cfg['n_layers']} layers at "
-            f"context {context} plus LM head and sampler, x{reps}, scaled to {cfg['n_layers']} layers")
-    return step_s, desc
+    step_s = sum(times) / len(times)
+    tpi = sum(toks) / len(toks)
+    return tpi / step_s, step_s, tpi, s.describe(len(times))
 
 
 # ---------------------------------------------------------------------------
@@ -236,83 +264,14 @@ def max_batch_that_fits(cfg, weight_bytes, max_ctx):
     return max(1, int((free - reserve) // per_req))
 
 
-def run_uno(args, rank, world, device):
-    from lossless_diffusion_draft_b200 import synth, uno
-
-    cfg = dict(synth.CONFIGS[args.workload])
-    if args.layers:
-        cfg["n_layers"] = args.layers
-    shape = synth.model_shape(cfg)
-    shape["dtype"] = cfg["dtype"]
-    B = cfg["B"]
-    prompt_len, gen = cfg["prompt_len"], cfg["gen_tokens"]
-    max_ctx = prompt_len + gen + B + 1
-    params = synth.make_params(cfg, device)
-    weight_bytes = sum(t.numel() * t.element_size() for t in params.values())
-    batch = cfg["batch"] or max_batch_that_fits(cfg, weight_bytes, max_ctx)
-    stream = torch.cuda.current_stream()
-    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, batch, max_ctx,
-                       cfg["seed"], stream)
-    if args.no_pdl:
-        uno.uno_set_pdl(ctx, False)
-    if args.no_counter_sync:
-        uno.uno_set_counter_sync(ctx, False)
-    fused = uno.uno_set_fused(ctx, not args.no_fused) and not args.no_fused
-    if args.no_graphs:
-        uno.uno_set_graphs(ctx, False)
-
-    # centre the timed window on the run's mean context
-    mean_ctx = prompt_len + gen // 2
-    est_tok = args.est_tokens_per_step
-    start_ctx = max(prompt_len, int(mean_ctx - (args.warmup + args.steps) * est_tok / 2))
-    P = start_ctx + 1
-    prompts = synth.make_prompts(cfg, batch, P, seed=cfg["seed"] + 1000 * rank)
-    streams = replica_streams(rank, batch)
-    t0 = time.time()
-    ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).to(device), [P] * batch, streams=streams)
-    torch.cuda.synchronize()
-    prefill_s = time.time() - t0
-    req = torch.tensor(ids, dtype=torch.int32, device=device)
-    out = torch.zeros((batch, B + 1), dtype=torch.int32, device=device)
-    K, W = args.steps, args.warmup
-    n_new_all = torch.zeros((K, batch), dtype=torch.int32, device=device)
-    for _ in range(W):
-        uno.uno_spec_step(ctx, req, out, n_new_all[0])
-    torch.cuda.synchronize()
-    uno.uno_status(ctx)
-    ctx_before = [uno.uno_request_state(ctx, i)[0] for i in ids[:1]][0]
-
-    barrier(world)
-    uno.uno_profile_begin(ctx, 0)          # launch counting only
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev_step = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        # a profiler started with --profile-from-start off sees the timed
-        # steps only
-        torch.cuda.profiler.start()
-        ev0.record(stream)
-        for k in range(K):
-            uno.uno_spec_step(ctx, req, out, n_new_all[k])
-            ev_step[k].record(stream)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        torch.cuda.profiler.stop()
-    prof = uno.uno_profile_end(ctx)
-    barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    step_ms = [ev0.elapsed_time(ev_step[0])] + [ev_step[k - 1].elapsed_time(ev_step[k])
-                                                 for k in range(1, K)]
-    tokens = int(n_new_all.sum().item())
-    ctx_after = uno.uno_request_state(ctx, ids[0])[0]
-    launches = sum(v[0] for v in prof.values())
-
-    # per-kernel-class device time: the same number of steps again with event
-    # pairs around every launch of the profiled classes
+def step_profile(ctx, req, out, n_new, K, cfg):
+    """Per-launch event times of K more steps, grouped by kernel class and GEMM
+    shape: (per-class {launches, ms}, detail rows sorted by time per step)."""
+    from lossless_diffusion_draft_b200 import uno
     uno.uno_profile_begin(ctx, (1 << uno.UNO_K_GEMM) | (1 << uno.UNO_K_ATTN) |
                           (1 << uno.UNO_K_SAMPLE) | (1 << uno.UNO_K_VERIFY) | (1 << uno.UNO_K_OTHER))
-    for k in range(K):
-        uno.uno_spec_step(ctx, req, out, n_new_all[k])
+    for _ in range(K):
+        uno.uno_spec_step(ctx, req, out, n_new)
     kprof = uno.uno_profile_end(ctx)
     shapes = {}
     esz = 2 if cfg["dtype"] == "bf16" else 4
@@ -329,59 +288,285 @@ def run_uno(args, rank, world, device):
             wbytes = (n * k + n * r + m * k + m * r) * esz
             row["GBps"] = wbytes / (ms_sum / cnt / 1e3) / 1e9
         detail.append(row)
+    return kprof, detail
 
-    # end to end through the C ABI with host buffers
-    req_h = torch.tensor(ids, dtype=torch.int32).pin_memory()
-    out_h = torch.zeros((batch, B + 1), dtype=torch.int32).pin_memory()
-    nn_h = torch.zeros(batch, dtype=torch.int32).pin_memory()
-    req_d = torch.empty_like(req)
-    nn_d = torch.zeros(batch, dtype=torch.int32, device=device)
-    e2e_tokens = 0
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for k in range(K):
-        req_d.copy_(req_h, non_blocking=True)
-        uno.uno_spec_step(ctx, req_d, out, nn_d)
-        out_h.copy_(out, non_blocking=True)
-        nn_h.copy_(nn_d, non_blocking=True)
-        stream.synchronize()
-        e2e_tokens += int(nn_h.sum())
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    uno.uno_status(ctx)
 
-    # the AR-only decode of the same model from the same kernels (one token per
-    # request per step, LoRA never read): the baseline Psi-Spec is measured
-    # against
-    ar_out = torch.zeros(batch, dtype=torch.int32, device=device)
-    for _ in range(W):
-        uno.uno_ar_step(ctx, req, ar_out)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(K):
-        uno.uno_ar_step(ctx, req, ar_out)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    ar_ms = a0.elapsed_time(a1) / K
-    uno.uno_status(ctx)
+class Workload:
+    """A context with `batch` requests prefilled to `context` tokens each."""
 
-    # aggregate over ranks: tokens summed, time = max
-    ms_max = reduce_max(ms, world, device)
-    e2e_ms_max = reduce_max(e2e_ms, world, device)
-    tokens_all = reduce_sum(tokens, world, device)
-    e2e_tokens_all = reduce_sum(e2e_tokens, world, device)
+    def __init__(self, cfg, params, batch, context, rank, device, args):
+        from lossless_diffusion_draft_b200 import synth, uno
+        self.uno, self.cfg, self.batch, self.device = uno, cfg, batch, device
+        shape = synth.model_shape(cfg)
+        shape["dtype"] = cfg["dtype"]
+        B = cfg["B"]
+        self.B = B
+        self.max_ctx = cfg["prompt_len"] + cfg["gen_tokens"] + B + 1
+        self.ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, batch,
+                                self.max_ctx, cfg["seed"], torch.cuda.current_stream())
+        if args.no_pdl:
+            uno.uno_set_pdl(self.ctx, False)
+        if args.no_counter_sync:
+            uno.uno_set_counter_sync(self.ctx, False)
+        self.fused = uno.uno_set_fused(self.ctx, not args.no_fused) and not args.no_fused
+        if args.no_graphs:
+            uno.uno_set_graphs(self.ctx, False)
+        self.rank = rank
+        self.ids = None
+        self.out = torch.zeros((batch, B + 1), dtype=torch.int32, device=device)
+        self.prefill(context)
 
-    info = dict(cfg=cfg, batch=batch, B=B, ms=ms_max, fused=fused, step_ms=step_ms, ar_ms=ar_ms, tokens=tokens_all, K=K, W=W,
-                e2e_ms=e2e_ms_max, e2e_tokens=e2e_tokens_all, clocks=clk.summary(),
-                launches=launches, kprof=kprof, prefill_s=prefill_s, detail=detail[:24],
-                ctx_window=[ctx_before, ctx_after], weight_bytes=weight_bytes,
-                h2d=req_h.numel() * 4, d2h=(out_h.numel() + nn_h.numel()) * 4)
-    ctx.close()
-    return info
+    def prefill(self, context):
+        """(Re-)admit every request with a synthetic prompt of `context` + 1
+        tokens (cached: `context`, pending: the last)."""
+        from lossless_diffusion_draft_b200 import synth
+        uno = self.uno
+        if self.ids is not None:
+            for i in self.ids:
+                uno.uno_release(self.ctx, i)
+        P = context + 1
+        prompts = synth.make_prompts(self.cfg, self.batch, P, seed=self.cfg["seed"] + 1000 * self.rank)
+        t0 = time.time()
+        self.ids = uno.uno_prefill(self.ctx, torch.from_numpy(prompts).to(self.device),
+                                   [P] * self.batch, streams=replica_streams(self.rank, self.batch))
+        torch.cuda.synchronize()
+        self.prefill_s = time.time() - t0
+        self.req = torch.tensor(self.ids, dtype=torch.int32, device=self.device)
+
+    def cached(self):
+        return self.uno.uno_request_state(self.ctx, self.ids[0])[0]
+
+    def time_steps(self, K, W, world, ar=False, clocks=True):
+        """K timed steps after W untimed ones (device time by CUDA events,
+        barrier and synchronize on both sides): dict(ms, tokens, step_ms,
+        clocks, ctx_window, launches)."""
+        uno, stream = self.uno, torch.cuda.current_stream()
+        B = self.B
+        n_new = torch.zeros((max(K, 1), self.batch), dtype=torch.int32, device=self.device)
+        ar_out = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+        step = (lambda k: uno.uno_ar_step(self.ctx, self.req, ar_out)) if ar else \
+               (lambda k: uno.uno_spec_step(self.ctx, self.req, self.out, n_new[k]))
+        for _ in range(W):
+            step(0)
+        torch.cuda.synchronize()
+        uno.uno_status(self.ctx)
+        c0 = self.cached()
+        barrier(world)
+        uno.uno_profile_begin(self.ctx, 0)          # launch counting only
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        with ClockSampler(torch.cuda.current_device(), enabled=clocks) as clk:
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for k in range(K):
+                step(k)
+                ev[k].record(stream)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        prof = uno.uno_profile_end(self.ctx)
+        barrier(world)
+        uno.uno_status(self.ctx)
+        step_ms = [ev0.elapsed_time(ev[0])] + [ev[k - 1].elapsed_time(ev[k]) for k in range(1, K)]
+        tokens = K * self.batch if ar else int(n_new.sum().item())
+        return dict(ms=ev0.elapsed_time(ev1), tokens=tokens, step_ms=step_ms,
+                    clocks=clk.summary() if clocks else None, ctx_window=[c0, self.cached()],
+                    launches=sum(v[0] for v in prof.values()), K=K)
+
+    def e2e(self, K, world):
+        """The same steps end to end through the C ABI: request ids copied from
+        pinned host memory, emitted tokens and counts copied back, every step."""
+        uno, stream = self.uno, torch.cuda.current_stream()
+        req_h = torch.tensor(self.ids, dtype=torch.int32).pin_memory()
+        out_h = torch.zeros((self.batch, self.B + 1), dtype=torch.int32).pin_memory()
+        nn_h = torch.zeros(self.batch, dtype=torch.int32).pin_memory()
+        req_d = torch.empty_like(self.req)
+        nn_d = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+        tokens = 0
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            req_d.copy_(req_h, non_blocking=True)
+            uno.uno_spec_step(self.ctx, req_d, self.out, nn_d)
+            out_h.copy_(self.out, non_blocking=True)
+            nn_h.copy_(nn_d, non_blocking=True)
+            stream.synchronize()
+            tokens += int(nn_h.sum())
+        e1.record(stream)
+        torch.cuda.synchronize()
+        uno.uno_status(self.ctx)
+        return dict(ms=e0.elapsed_time(e1), tokens=tokens, h2d=req_h.numel() * 4,
+                    d2h=(out_h.numel() + nn_h.numel()) * 4)
+
+    def close(self):
+        self.ctx.close()
+
+
+def gemm_roofline(detail, cfg, pk, steps_in_long_run=True):
+    """Roofline of the step's dominant GEMM (largest share of the step):
+    HBM-bound (algorithmic bytes over the measured copy rate) or tensor-bound
+    (algorithmic flops over the measured bf16 rate, sustained: the kernel
+    runs inside a long step), whichever binds."""
+    gemms = [d for d in detail if d["cls"] == "gemm"]
+    if not gemms:
+        return None
+    top = max(gemms, key=lambda d: d["ms_per_step"])
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    top_bytes = (top["n"] * top["k"] + top["n"] * top["r"] + top["m"] * top["k"] +
+                 top["m"] * top["r"]) * esz
+    top_flops = 2.0 * top["m"] * top["n"] * (top["k"] + top["r"])
+    sec = top["us_per_call"] * 1e-6
+    t_hbm = top_bytes / (pk["hbm_gbs"] * 1e9)
+    tc_peak = (pk["bf16_tflops_sustained"] or pk["bf16_tflops"]) if steps_in_long_run else pk["bf16_tflops"]
+    t_tc = top_flops / (tc_peak * 1e12)
+    common = {"kernel": f"gated_lora_linear M={top['m']} N={top['n']} K={top['k']} r={top['r']} "
+                        "(gemm_tc_kernel, the step's largest GEMM)",
+              "algorithmic_bytes": top_bytes, "algorithmic_flops": top_flops,
+              "avg_launch_us": top["us_per_call"], "launches_per_step": top["calls_per_step"],
+              "peak_source": pk["source"]}
+    if t_tc > t_hbm:
+        tflops = top_flops / sec / 1e12
+        # bf16 models feed every activation row as a hi/lo pair of bf16 rows:
+        # the tensor cores execute twice the algorithmic flops
+        executed = 2 * tflops if cfg["dtype"] == "bf16" else tflops
+        return dict({"bound": "tensor", "achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": tflops / tc_peak, "traffic": None, "peak_kind": "bf16 sustained",
+                     "executed_TFLOPs": executed, "executed_frac": executed / tc_peak}, **common)
+    achieved = top_bytes / sec / 1e9
+    return dict({"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                 "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(top)}, **common)
+
+
+def run_uno(args, rank, world, device):
+    """The headline workload (and, on one GPU, the other measurements the
+    line carries); returns the JSON line's fields."""
+    from lossless_diffusion_draft_b200 import synth, uno
+
+    cfg = dict(synth.CONFIGS[args.workload])
+    if args.layers:
+        cfg["n_layers"] = args.layers
+    B, prompt_len, gen = cfg["B"], cfg["prompt_len"], cfg["gen_tokens"]
+    pk = peaks()
+    params = synth.make_params(cfg, device)
+    weight_bytes = sum(t.numel() * t.element_size() for t in params.values())
+    max_ctx = prompt_len + gen + B + 1
+    batch = cfg["batch"] or max_batch_that_fits(cfg, weight_bytes, max_ctx)
+    K, W = args.steps, args.warmup
+    # the timed window is centred on the run's mean context
+    mean_ctx = prompt_len + gen // 2
+    start = max(prompt_len, int(mean_ctx - (W + K) * args.est_tokens_per_step / 2))
+    wl = Workload(cfg, params, batch, start, rank, device, args)
+    head = wl.time_steps(K, W, world)
+    kprof, detail = step_profile(wl.ctx, wl.req, wl.out, torch.zeros(batch, dtype=torch.int32,
+                                                                     device=device), K, cfg)
+    e2e = wl.e2e(K, world)
+    ar = wl.time_steps(K, W, world, ar=True, clocks=False)
+    res = dict(cfg=cfg, batch=batch, head=head, kprof=kprof, detail=detail, e2e=e2e, ar=ar,
+               fused=wl.fused, prefill_s=wl.prefill_s, weight_bytes=weight_bytes, pk=pk)
+
+    extras = world == 1 and not args.headline_only and args.workload == "qwen8b"
+    if extras:
+        # contexts across the 1K -> 9K run (the step's cost grows with the
+        # context: KV bytes); a whole-run estimate from them by Simpson's rule
+        pts = {}
+        # the last point ends inside the request's pages even if every step
+        # emitted B + 1 tokens
+        for c0 in (prompt_len, prompt_len + gen - (W + K) * (B + 1)):
+            wl.prefill(c0)
+            pts[c0] = wl.time_steps(K, W, world, clocks=False)
+        pts[head["ctx_window"][0]] = head
+        res["contexts"] = pts
+        # the benchmark tap: a trained drafter's acceptance (a = 4: five
+        # tokens per iteration, TPF 2.5) at the mean context
+        wl.prefill(start)
+        uno.uno_debug_set_fixed_accept(wl.ctx, 4)
+        res["fixed_accept"] = dict(wl.time_steps(K, W, world, clocks=False), a=4)
+        uno.uno_debug_set_fixed_accept(wl.ctx, 0)
+    wl.close()
+    if extras:
+        del wl
+        torch.cuda.empty_cache()
+        res["max_batch"] = run_max_batch(args, cfg, params, rank, world, device, pk)
+        res["spec_verify_micro"] = spec_verify_micro(args, device, pk)
+    return res
+
+
+def run_max_batch(args, cfg, params, rank, world, device, pk):
+    """The same model at the largest batch whose KV cache (1024 + 8192 tokens
+    per request) fits beside the weights, at the run's mean context."""
+    cfg = dict(cfg, batch=0)
+    B, prompt_len, gen = cfg["B"], cfg["prompt_len"], cfg["gen_tokens"]
+    weight_bytes = sum(t.numel() * t.element_size() for t in params.values())
+    max_ctx = prompt_len + gen + B + 1
+    batch = max_batch_that_fits(cfg, weight_bytes, max_ctx)
+    K, W = max(3, args.steps // 2), 3
+    start = max(prompt_len, int(prompt_len + gen // 2 - (W + K) * args.est_tokens_per_step / 2))
+    wl = Workload(cfg, params, batch, start, rank, device, args)
+    head = wl.time_steps(K, W, world)
+    _, detail = step_profile(wl.ctx, wl.req, wl.out, torch.zeros(batch, dtype=torch.int32,
+                                                                 device=device), 2, cfg)
+    e2e = wl.e2e(K, world)
+    ar = wl.time_steps(K, W, world, ar=True, clocks=False)
+    wl.close()
+    ms = head["ms"] / head["K"]
+    value = head["tokens"] / (head["ms"] / 1e3)
+    ar_value = ar["tokens"] / (ar["ms"] / 1e3)
+    return {"value": value, "unit": "tokens/s", "batch": batch, "steps": K, "warmup": W,
+            "ms_per_step": ms, "tokens_per_step": head["tokens"] / K,
+            "tpf": head["tokens"] / K / batch / 2, "context_window": head["ctx_window"],
+            "prefill_s": wl.prefill_s,
+            "e2e": {"value": e2e["tokens"] / (e2e["ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "ar_only": {"value": ar_value, "unit": "tokens/s", "ms_per_step": ar["ms"] / ar["K"]},
+            "psi_spec_over_ar": value / ar_value,
+            "roofline": gemm_roofline(detail, cfg, pk), "clocks": head["clocks"],
+            "kernel_detail": detail[:8]}
+
+
+def spec_verify_micro(args, device, pk, n_req=None):
+    """spec_verify on the microbenchmark workload: fp32 p, q [4096 = 256 x 16,
+    151936] (p ~ N(0, 3), q = p + N(0, 0.5)), drafts drawn from q, Philox
+    seed 7.  Algorithmic bytes: both logit tensors read once."""
+    from lossless_diffusion_draft_b200 import synth, uno
+    cfg = synth.SPEC_VERIFY_BENCH
+    n_req, R, V = n_req or cfg["requests"], cfg["rows_per_request"], cfg["vocab"]
+    p, q = synth.make_verify_logits(n_req * R, V, device, cfg["p_std"], cfg["q_noise_std"],
+                                    cfg["logits_seed"])
+    drafts = synth.make_drafts(q, seed=cfg["logits_seed"] + 1).view(n_req, R)
+    p, q = p.view(n_req, R, V), q.view(n_req, R, V)
+    streams = torch.arange(n_req, dtype=torch.int32, device=device)
+    pos0 = torch.zeros(n_req, dtype=torch.int32, device=device)
+    ws = torch.zeros(uno.uno_spec_verify_workspace_bytes(n_req, R, V), dtype=torch.uint8,
+                     device=device)
+    out = torch.empty((n_req, R + 1), dtype=torch.int32, device=device)
+    n_out = torch.empty(n_req, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    call = lambda: uno.uno_spec_verify(p, q, drafts, cfg["seed"], streams, pos0, out, n_out, ws)
+    K = max(args.steps, 10)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for _ in range(K):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / K
+    nbytes = 2 * n_req * R * V * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    a = n_out.float().mean().item()
+    del p, q
+    torch.cuda.empty_cache()
+    return {"metric": f"spec_verify [{n_req * R} x {V}] fp32 p and q", "value": n_req * R / (ms / 1e3),
+            "unit": "rows/s", "ms_per_call": ms, "calls": K, "mean_accepted": a,
+            "l2": "inputs (4.98 GB) larger than L2",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_call": nbytes, "peak_source": pk["source"]},
+            "clocks": clk.summary()}
 
 
 def run_micro(args, device):
@@ -483,10 +668,11 @@ def reduce_sum(x, world, device):
     return int(t.item())
 
 
-def step_bytes(info):
-    """Algorithmic HBM bytes of one iteration (per request KV at the window's
-    mean context; weights once per pass for the whole batch)."""
-    cfg = info["cfg"]
+def step_bytes(cfg, batch, ctx_window):
+    """Algorithmic HBM bytes of one iteration: base weights once per pass (the
+    embedding table is only gathered), the adapters once (draft pass), each
+    request's KV at the window's mean context once per pass, and the fp32
+    logits written and read once."""
     esz = 2 if cfg["dtype"] == "bf16" else 4
     from lossless_diffusion_draft_b200 import synth
     base = lora = 0
@@ -496,16 +682,52 @@ def step_bytes(info):
             lora += n
         elif name != "embed":
             base += n
-    ctx = sum(info["ctx_window"]) / 2
-    kv = ctx * kv_bytes_per_token(cfg) * 2 * info["batch"]
-    logits = (2 * cfg["B"] + 1) * cfg["vocab"] * 4 * 2 * info["batch"]
+    ctx = sum(ctx_window) / 2
+    kv = ctx * kv_bytes_per_token(cfg) * 2 * batch
+    logits = (2 * cfg["B"] + 1) * cfg["vocab"] * 4 * 2 * batch
     return 2 * base + lora + kv + logits
+
+
+def reference_arm(args, rank, cfg, metric):
+    """The CPU oracle, timed as it stands on the host cores: each step is one
+    bounded sample of the workload's iteration (see OracleSample)."""
+    if rank != 0:
+        return
+    ctx_len = cfg["prompt_len"] + cfg["gen_tokens"] // 2
+    sample = OracleSample(cfg, ctx_len)
+    times, toks = [], []
+    for i in range(args.warmup + args.steps):
+        t, n = sample.step(i)
+        if i >= args.warmup:
+            times.append(t)
+            toks.append(n)
+    step_s = sum(times) / len(times)
+    tpi = sum(toks) / len(toks)
+    batch = cfg["batch"] or 1
+    value = tpi * batch / step_s
+    desc = sample.describe(len(times))
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": cfg["batch"], "B": cfg["B"],
+                       "context": ctx_len},
+            "tokens_per_step": tpi * batch,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def rate(t):
+    return t["tokens"] / (t["ms"] / 1e3)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="uno", choices=["uno", "reference"])
     ap.add_argument("--workload", default="qwen8b",
@@ -525,6 +747,9 @@ def main():
                     help="override the layer count (small cases for profiler captures; the "
                          "line's config records it)")
     ap.add_argument("--est-tokens-per-step", type=float, default=2.6)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="the batch-1 headline alone (no context sweep, fixed-accept run, "
+                         "max-batch line or spec_verify microbenchmark)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
@@ -542,28 +767,7 @@ def main():
     metric = "generated tokens/s (Psi-Spec, 1K in / 8K out)"
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        ctx_len = cfg["prompt_len"] + cfg["gen_tokens"] // 2
-        tps = args.est_tokens_per_step
-        times = []
-        desc = ""
-        for i in range(args.warmup + args.steps):
-            s, desc = oracle_step_sample(cfg, ctx_len, tps, budget_s=0.0)
-            if i >= args.warmup:
-                times.append(s)
-        step_s = sum(times) / len(times)
-        value = tps * cfg["batch"] / step_s if cfg["batch"] else tps / step_s
-        line = {"impl": "reference", "metric": metric, "value": value, "unit": "tokens/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": args.workload, "batch": cfg["batch"], "B": cfg["B"]},
-                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
-                                 "kind": "oracle", "sample": desc + f"; {tps} tokens per iteration assumed"},
-                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        reference_arm(args, rank, cfg, metric)
         return
 
     if world > 1:
@@ -574,90 +778,96 @@ def main():
     from lossless_diffusion_draft_b200 import build
     build.build()
 
-    info = run_uno(args, rank, world, device)
-    pk = peaks()
-    value = info["tokens"] / (info["ms"] / 1e3)
-    e2e = info["e2e_tokens"] / (info["e2e_ms"] / 1e3)
-    kp = info["kprof"]
-    g_launch, g_ms, g_bytes = kp["gemm"]
-    g_gbs = g_bytes / (g_ms / 1e3) / 1e9 if g_ms > 0 else None
-    # the dominant kernel: the GEMM shape with the largest share of the step
-    gemms = [d for d in info["detail"] if d["cls"] == "gemm"]
-    top = max(gemms, key=lambda d: d["ms_per_step"]) if gemms else None
-    if top:
-        esz = 2 if cfg["dtype"] == "bf16" else 4
-        top_bytes = (top["n"] * top["k"] + top["n"] * top["r"] + top["m"] * top["k"] +
-                     top["m"] * top["r"]) * esz
-        achieved = top_bytes / (top["us_per_call"] * 1e-6) / 1e9
-        traffic = profiled_traffic(top)
-        top_flops = 2.0 * top["m"] * top["n"] * (top["k"] + top["r"])
-        # which roof binds: bytes at the measured copy rate against flops at
-        # the measured bf16 rate (sustained: the kernel runs inside a long step)
-        t_hbm = top_bytes / (pk["hbm_gbs"] * 1e9)
-        tc_peak = pk["bf16_tflops_sustained"] or pk["bf16_tflops"]
-        t_tc = top_flops / (tc_peak * 1e12)
-        kernel_desc = (f"gated_lora_linear M={top['m']} N={top['n']} K={top['k']} "
-                       "(gemm_tc_kernel, the step's largest GEMM)")
-        common = {"kernel": kernel_desc, "algorithmic_bytes": top_bytes,
-                  "algorithmic_flops": top_flops, "avg_launch_us": top["us_per_call"],
-                  "launches_per_step": top["calls_per_step"], "peak_source": pk["source"],
-                  "all_gemm_launches": {"achieved_GBps": g_gbs, "launches": g_launch,
-                                        "avg_launch_us": g_ms * 1e3 / max(1, g_launch)}}
-        if t_tc > t_hbm:
-            tflops = top_flops / (top["us_per_call"] * 1e-6) / 1e12
-            roofline = dict({"bound": "tensor", "achieved": tflops, "peak": tc_peak,
-                             "unit": "TFLOP/s", "frac": tflops / tc_peak, "traffic": None,
-                             "peak_kind": "bf16 sustained",
-                             "note": "every activation row is fed as a bf16 hi/lo pair, so the "
-                                     "tensor cores execute twice the algorithmic flops"}, **common)
-        else:
-            roofline = dict({"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                             "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                             "traffic": traffic}, **common)
-    else:
-        roofline = {"bound": "hbm", "kernel": "gated_lora_linear (SIMT)", "achieved": g_gbs,
-                    "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": (g_gbs / pk["hbm_gbs"]) if g_gbs else None, "traffic": None,
-                    "peak_source": pk["source"]}
-    per_step_ms = info["ms"] / info["K"]
-    sb = step_bytes(info)
+    res = run_uno(args, rank, world, device)
+    cfg, pk, head = res["cfg"], res["pk"], res["head"]
+    K = head["K"]
+    ms_max = reduce_max(head["ms"], world, device)
+    tokens_all = reduce_sum(head["tokens"], world, device)
+    e2e_ms = reduce_max(res["e2e"]["ms"], world, device)
+    e2e_tokens = reduce_sum(res["e2e"]["tokens"], world, device)
+    value = tokens_all / (ms_max / 1e3)
+    per_step_ms = ms_max / K
+    batch = res["batch"]
+    sb = step_bytes(cfg, batch, head["ctx_window"])
     step_roof = {"algorithmic_bytes_per_step": sb, "achieved_GBps": sb / (per_step_ms / 1e3) / 1e9,
-                 "frac_of_hbm_peak": sb / (per_step_ms / 1e3) / 1e9 / pk["hbm_gbs"]}
-    breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / info["K"]} for k, v in kp.items()}
-
+                 "frac_of_hbm_peak": sb / (per_step_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                 "peak_source": pk["source"]}
+    kp = res["kprof"]
+    g_launch, g_ms, g_bytes = kp["gemm"]
+    roofline = gemm_roofline(res["detail"], cfg, pk) or {}
+    if g_ms > 0:
+        roofline["all_gemm_launches"] = {"achieved_GBps": g_bytes / (g_ms / 1e3) / 1e9,
+                                         "launches": g_launch,
+                                         "avg_launch_us": g_ms * 1e3 / max(1, g_launch)}
+    tps = head["tokens"] / K / batch
     line = {
         "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": info["K"], "warmup": info["W"], "ms_per_step": per_step_ms,
+        "steps": K, "warmup": args.warmup, "ms_per_step": per_step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg["dtype"],
         "data": "synthetic (random-init weights, uniform-random prompt tokens)",
-        "config": {"workload": args.workload, "n_layers": info["cfg"]["n_layers"],
-                   "batch": info["batch"], "B": info["B"], "pdl": not args.no_pdl,
-                   "fused": info["fused"],
-                   "graphs": not args.no_graphs,
+        "config": {"workload": args.workload, "n_layers": cfg["n_layers"],
+                   "batch": batch, "B": cfg["B"], "pdl": not args.no_pdl,
+                   "fused": res["fused"], "graphs": not args.no_graphs,
                    "prompt_len": cfg["prompt_len"], "gen_tokens": cfg["gen_tokens"],
-                   "context_window": info["ctx_window"], "parallelism": f"replicas x{world}",
+                   "context_window": head["ctx_window"], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (15+ GB of weights streamed per pass)"},
-        "tokens_per_step": info["tokens"] / info["K"],
-        "step_latency_ms": {"median": statistics.median(info["step_ms"]),
-                            "min": min(info["step_ms"]), "max": max(info["step_ms"])},
-        "mean_accepted_a": info["tokens"] / info["K"] / info["batch"] / max(1, world) - 1,
-        "ar_only": {"value": info["batch"] / (info["ar_ms"] / 1e3), "unit": "tokens/s",
-                    "ms_per_step": info["ar_ms"],
+        "tokens_per_step": tokens_all / K,
+        "step_latency_ms": {"median": statistics.median(head["step_ms"]),
+                            "min": min(head["step_ms"]), "max": max(head["step_ms"])},
+        "mean_accepted_a": tps - 1,
+        "tpf": tps / 2,
+        "ar_only": {"value": rate(res["ar"]), "unit": "tokens/s",
+                    "ms_per_step": res["ar"]["ms"] / res["ar"]["K"],
                     "note": "uno_ar_step on the same requests and kernels, one token per request"},
-        "tpf": info["tokens"] / info["K"] / info["batch"] / 2 / max(1, world),
-        "roofline": roofline, "step_roofline": step_roof, "kernel_breakdown": breakdown,
-        "e2e": {"value": e2e, "unit": "tokens/s", "h2d_bytes_per_step": info["h2d"],
-                "d2h_bytes_per_step": info["d2h"]},
-        "gpu_launches": info["launches"], "clocks": info["clocks"],
-        "kernel_detail": info["detail"],
-        "prefill_s": info["prefill_s"],
+        "roofline": roofline, "step_roofline": step_roof,
+        "kernel_breakdown": {k: {"launches": v[0], "ms_per_step": v[1] / K} for k, v in kp.items()},
+        "e2e": {"value": e2e_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"]},
+        "gpu_launches": head["launches"], "clocks": head["clocks"],
+        "kernel_detail": res["detail"][:24],
+        "prefill_s": res["prefill_s"],
     }
+    if "contexts" in res:
+        pts = sorted(res["contexts"].items())
+        by_ctx = {}
+        for c0, t in pts:
+            by_ctx[str(c0)] = {"ms_per_step": t["ms"] / t["K"], "tokens_per_step": t["tokens"] / t["K"],
+                               "tokens_per_s": rate(t), "context_window": t["ctx_window"],
+                               "frac_of_hbm_peak": step_bytes(cfg, batch, t["ctx_window"]) /
+                               (t["ms"] / t["K"] / 1e3) / 1e9 / pk["hbm_gbs"]}
+        lat = [t["ms"] / t["K"] for _, t in pts]
+        tok = sum(t["tokens"] for _, t in pts) / sum(t["K"] for _, t in pts)
+        mean_lat = (lat[0] + 4 * lat[1] + lat[2]) / 6          # Simpson over 1K .. 9K
+        line["contexts"] = {
+            "steps_per_point": K, "points": by_ctx,
+            "whole_run_estimate": {
+                "tokens_per_s": tok / (mean_lat / 1e3), "mean_ms_per_step": mean_lat,
+                "tokens_per_step": tok,
+                "note": "the 1K-in / 8K-out run: step latency averaged over the context range by "
+                        "Simpson's rule on the three measured points, at the tokens per step "
+                        "measured there"}}
+        head_lat = per_step_ms
+        line["tpf_projection"] = {
+            "tokens_per_s": 2 * 2.25 / (head_lat / 1e3), "tpf": 2.25,
+            "note": "projection, not a measurement: the measured iteration latency at the mean "
+                    "context times the pages' tokens per forward for the Qwen3-8B adapter (2.25), "
+                    "as the pages convert decode steps to tokens by TPF"}
+        fa = res["fixed_accept"]
+        line["fixed_accept"] = {
+            "a": fa["a"], "tokens_per_s": rate(fa), "ms_per_step": fa["ms"] / fa["K"],
+            "tokens_per_step": fa["tokens"] / fa["K"], "tpf": fa["tokens"] / fa["K"] / batch / 2,
+            "note": "measured with the uno_debug_set_fixed_accept tap forcing a = 4 accepted "
+                    "tokens (TPF 2.5, the pages' trained-adapter range); not a parity run"}
+    if "max_batch" in res:
+        line["max_batch"] = res["max_batch"]
+    if "spec_verify_micro" in res:
+        line["spec_verify_micro"] = res["spec_verify_micro"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps = info["tokens"] / info["K"] / info["batch"]
-        ctx_len = sum(info["ctx_window"]) // 2
-        s, desc = oracle_step_sample(cfg, ctx_len, tps)
-        line["cpu_baseline"] = {"value": tps * info["batch"] / s, "unit": "tokens/s",
-                                "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+        ctx_len = sum(head["ctx_window"]) // 2
+        v, step_s, tpi, desc = oracle_baseline(cfg, ctx_len)
+        line["cpu_baseline"] = {"value": v * batch, "unit": "tokens/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": desc, "s_per_iteration": step_s,
+                                "tokens_per_iteration": tpi}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

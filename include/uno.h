@@ -188,6 +188,30 @@ int uno_set_fused(uno_ctx *ctx, int enable);
  * UNO_ERR_ARG. */
 int uno_set_verify_split(uno_ctx *ctx, int max_ctas);
 
+/*
+ * Benchmark tap (no counterpart on the pages; never used by the parity
+ * tests): force the accepted length of every later uno_spec_step to
+ * a (1 <= a <= B: the first token plus a - 1 accepted drafts), whatever the
+ * accept tests say; the token after the prefix is still drawn from the
+ * residual (a < B) or the bonus row (a = B).  Random-init weights accept
+ * few drafts, so this gives a step at the acceptance of a trained drafter
+ * (the pages convert decode steps to tokens by the average tokens per
+ * forward).  a <= 0 turns it off; a > B: UNO_ERR_ARG.  Drops captured graphs.
+ */
+int uno_debug_set_fixed_accept(uno_ctx *ctx, int a);
+
+/*
+ * Test tap of the bounded waits (no counterpart on the pages): every later
+ * completion-counter wait of the fused pipeline (see uno_set_counter_sync)
+ * gives up after limit_ns nanoseconds (default 1e9), and `extra` is added to
+ * every counter's target, so extra > 0 makes each such wait run out: the
+ * waiting GEMM then raises the device flag (uno_status returns
+ * UNO_ERR_DEVICE_CHECK) and goes on, so the step ends with meaningless
+ * results instead of hanging.  extra = 0 restores normal waits.
+ * limit_ns = 0: UNO_ERR_ARG.  Drops captured graphs.
+ */
+int uno_debug_set_dep_wait(uno_ctx *ctx, uint64_t limit_ns, uint32_t extra);
+
 /* Free a request's slot and pages (stream-ordered after earlier work). */
 int uno_release(uno_ctx *ctx, int req_id);
 
@@ -335,11 +359,15 @@ int uno_spec_verify(const float *p_dev, const float *q_dev, const int32_t *draft
  * the process exits.  It allocates nothing (no cudaMalloc, cudaFree or other
  * allocating routine).
  *   Arguments, outputs and results are those of uno_spec_verify.
- *   Sizes whose workspace (uno_spec_verify_workspace_bytes) exceeds the array
- *   are rejected with UNO_ERR_CAPACITY before anything is enqueued.
+ *   Every argument is checked before anything is enqueued: invalid ones give
+ *   UNO_ERR_ARG, and sizes whose workspace (uno_spec_verify_workspace_bytes)
+ *   exceeds the array give UNO_ERR_CAPACITY; a rejected call touches neither
+ *   the array nor the stream.
  *   The first call on a device looks up the array's device address on that
- *   device (it must be the current device) and caches it; make that first
- *   call before any stream capture.
+ *   device (it must be the current device) and caches it with the id of the
+ *   device's CUDA context; a call in a new context (after cudaDeviceReset)
+ *   looks it up again.  Make the first call on a device, and the first one
+ *   after a reset, before any stream capture.
  *   All calls share the one array, which keeps the previous call's contents;
  *   each call clears the part that must start at zero (its completion
  *   counters) on the given stream before the kernels.  Calls that overlap on

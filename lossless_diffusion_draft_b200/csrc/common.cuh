@@ -149,14 +149,20 @@ __device__ __forceinline__ void dep_signal(unsigned* ctr) {   // whole CTA, at i
   if (threadIdx.x == 0 && threadIdx.y == 0)
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
-__device__ __forceinline__ bool dep_wait(const unsigned* ctr, unsigned target) {   // one thread
-  for (int i = 0; i < (1 << 21); ++i) {
+// limit_ns: how long to poll (global timer) before giving up.
+__device__ __forceinline__ bool dep_wait(const unsigned* ctr, unsigned target,
+                                         unsigned long long limit_ns) {   // one thread
+  unsigned long long t0 = 0;
+  for (int i = 0;; ++i) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (i == 0) t0 = t;
+    else if (t - t0 > limit_ns) return false;
     __nanosleep(20);
   }
-  return false;
 }
 
 // Device-side error flag bits (read by uno_status).

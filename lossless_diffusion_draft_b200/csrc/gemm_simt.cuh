@@ -44,6 +44,7 @@ struct GemmParams {
   // tensor-core DUMP launches: completion counter of the kernel that wrote X
   // and its CTA count (null: the launch waits with pdl_wait)
   const unsigned* dep; unsigned dep_count;
+  unsigned long long dep_limit_ns;   // the counter wait gives up after this long
 };
 
 template <typename T, int MT, int NC>

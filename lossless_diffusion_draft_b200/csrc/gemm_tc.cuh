@@ -71,6 +71,7 @@ struct TcParams {
   // completion counter of the kernel that wrote X (null: pdl_wait instead);
   // DUMP mode only, where X is the one input an earlier kernel wrote
   const unsigned* dep; unsigned dep_count;
+  unsigned long long dep_limit_ns;   // give up the counter wait after this long
 };
 
 // ---------------------------------------------------------------------------
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       if (p.dep) {
-        if (!dep_wait(p.dep, p.dep_count)) raise_status(p.status, ST_DEP_TIMEOUT);
+        if (!dep_wait(p.dep, p.dep_count, p.dep_limit_ns)) raise_status(p.status, ST_DEP_TIMEOUT);
         // the X rows were written by generic stores; the loads below are TMA
         asm volatile("fence.proxy.async.global;" ::: "memory");
       } else {

@@ -376,6 +376,10 @@ struct VerifyArgs {
   int rows_red;                // rows reduced per request
   int n_p;                     // of which p rows (tests + bonus)
   int32_t* status;
+  // benchmark tap (-1: off): the accepted prefix is forced to min(fixed_at,
+  // n_tests) tests instead of the accept tests' outcome; the residual
+  // redraw or the bonus draw then runs as usual
+  int fixed_at;
 };
 
 // Slot, position of test 0 and Philox stream of a request.
@@ -446,7 +450,7 @@ __device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
     if (!acc) atomicMin(&s_a, j);
   }
   __syncthreads();
-  const int at = s_a;   // accepted prefix length among the tests
+  const int at = a.fixed_at >= 0 ? min(a.fixed_at, a.n_tests) : s_a;   // accepted tests
   if (at < a.n_tests) {
     // a rejection: spec_resid_kernel draws from the residual and finishes
     if (threadIdx.x == 0) a.at_ws[req] = at;

@@ -69,10 +69,27 @@ struct MapKey {
 };
 
 constexpr int TC_COUNTERS = 1 << 16;
+// A completion-counter wait gives up (and raises the device flag) after this long.
+constexpr unsigned long long DEP_WAIT_NS = 1000000000ull;
 constexpr int TC_MIN_UNITS = 8;
 
 // Process-wide launch counts per kernel path (read by uno_debug_launch_counts).
 int64_t g_launches[4] = {0, 0, 0, 0};   // tc gemm, simt gemm, tc attention, simt attention
+
+// cudaFuncSetAttribute acts on the current device only, so a kernel's
+// dynamic shared-memory limit is raised once per device (`done` is the
+// kernel's own per-device record; devices past its size are set every time).
+constexpr int ATTR_DEVS = 64;
+template <typename K>
+cudaError_t smem_attr_once(K kernel, int bytes, bool* done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  if (dev >= 0 && dev < ATTR_DEVS && done[dev]) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < ATTR_DEVS) done[dev] = true;
+  return e;
+}
 
 // Launch with programmatic stream serialisation when `pdl`: the kernel may
 // start while the previous kernel of the stream is still running; inside,
@@ -235,15 +252,12 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.out_lo = p.out_lo;
   tp.dep = DUMP ? p.dep : nullptr;
   tp.dep_count = p.dep_count;
+  tp.dep_limit_ns = p.dep_limit_ns ? p.dep_limit_ns : DEP_WAIT_NS;
 
   using Cfg = TcCfg<NT, SPLIT, KPS>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<NT, SPLIT, DUMP, KPS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
-      return false;
-    attr = true;
-  }
+  static bool attr[ATTR_DEVS] = {};
+  if (smem_attr_once(gemm_tc_kernel<NT, SPLIT, DUMP, KPS>, Cfg::SMEM, attr) != cudaSuccess)
+    return false;
   klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), Cfg::SMEM,
           gemm_tc_kernel<NT, SPLIT, DUMP, KPS>, maps, tp);
   g_launches[0]++;
@@ -360,6 +374,9 @@ struct uno_ctx {
   unsigned* dep_ctr = nullptr;
   int n_dep_ctr = 0;
   bool counter_sync = true;
+  unsigned long long dep_limit_ns = DEP_WAIT_NS;   // test tap: counter-wait limit
+  unsigned dep_extra = 0;                          // test tap: added to every counter target
+  int fixed_accept = -1;                           // bench tap: forced a (first token + accepted)
   float *cos_t = nullptr, *sin_t = nullptr;
   int max_pos = 0;
 
@@ -526,12 +543,8 @@ void launch_gemm(uno_ctx* c, const Gemm& g, cudaStream_t st) {
 template <typename T, int HD>
 int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
   const size_t smem = (size_t)(ATT_MAXQ * HD + ATT_KT * (HD + 1) + ATT_KT * HD) * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    CK(cudaFuncSetAttribute(attn_simt_kernel<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            (int)smem));
-    attr_set = true;
-  }
+  static bool attr[ATTR_DEVS] = {};
+  CK(smem_attr_once(attn_simt_kernel<T, HD>, (int)smem, attr));
   const dim3 grid(p.n_splits, p.n_qtiles, n_req * p.Hkv);
   Prof prof(c, UNO_K_ATTN, 0.0);
   klaunch(c->genv.pdl, st, grid, dim3(ATT_THREADS), smem, attn_simt_kernel<T, HD>, p);
@@ -577,12 +590,8 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   const bool pf_ok = l2_pf && l2_pf_bytes >= 16 && ((uintptr_t)l2_pf & 15) == 0;
   p.l2_pf = pf_ok ? (const char*)l2_pf : nullptr;
   p.l2_pf_bytes = pf_ok ? (unsigned long long)(l2_pf_bytes & ~(size_t)15) : 0ull;
-  static bool attr = false;
-  if (!attr) {
-    CK(cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            AtcCfg<HD>::SMEM));
-    attr = true;
-  }
+  static bool attr[ATTR_DEVS] = {};
+  CK(smem_attr_once(attn_tc_kernel<HD>, AtcCfg<HD>::SMEM, attr));
   {
     Prof prof(c, UNO_K_ATTN, 0.0);
     klaunch(c->genv.pdl, c->stream, dim3(S, p.n_qtiles, n_req * s.n_kv_heads), dim3(ATC_THREADS),
@@ -924,7 +933,8 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
       for (const void* a : A) g.seg(a, r);
     g.p.lo_off = lo;
     g.p.dep = dep;
-    g.p.dep_count = dep_n;
+    g.p.dep_count = dep ? dep_n + c->dep_extra : dep_n;
+    g.p.dep_limit_ns = c->dep_limit_ns;
     dep = nullptr;
     DumpShape sh;
     {
@@ -1463,6 +1473,7 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.rows_red = B;      // B - 1 test rows + the bonus row; lse of q comes from draft_sample
     a.n_p = B;
     a.status = c->d_status;
+    a.fixed_at = c->fixed_accept > 0 ? c->fixed_accept - 1 : -1;
     {
       Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
       c->prof_launches[UNO_K_VERIFY] += launch_verify(c->genv.pdl, c->stream, a, n_req, c->verify_split_ctas) - 1;
@@ -1531,6 +1542,38 @@ int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_
                      [&] { return ar_step_body(c, n_req, req_ids_dev, out_tokens_dev); });
 }
 
+}  // extern "C"
+
+namespace {
+// Drops every captured graph: a setting baked into the kernels' arguments
+// changed, so the next calls capture again.
+void drop_graphs(uno_ctx* c) {
+  for (auto& g : c->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.seen = 0;
+  }
+}
+}  // namespace
+
+extern "C" {
+
+int uno_debug_set_fixed_accept(uno_ctx* c, int a) {
+  if (!c) return UNO_ERR_ARG;
+  if (a > c->B) return fail(c, UNO_ERR_ARG, "fixed accept beyond the block size");
+  c->fixed_accept = a > 0 ? a : -1;
+  drop_graphs(c);
+  return UNO_OK;
+}
+
+int uno_debug_set_dep_wait(uno_ctx* c, uint64_t limit_ns, uint32_t extra) {
+  if (!c || limit_ns == 0) return UNO_ERR_ARG;
+  c->dep_limit_ns = limit_ns;
+  c->dep_extra = extra;
+  drop_graphs(c);
+  return UNO_OK;
+}
+
 int uno_set_graphs(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->graphs_enabled = enable != 0;
@@ -1540,44 +1583,28 @@ int uno_set_graphs(uno_ctx* c, int enable) {
 int uno_set_counter_sync(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->counter_sync = enable != 0;
-  for (auto& g : c->graphs) {
-    if (g.exec) cudaGraphExecDestroy(g.exec);
-    g.exec = nullptr;
-    g.seen = 0;
-  }
+  drop_graphs(c);
   return UNO_OK;
 }
 
 int uno_set_pdl(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->genv.pdl = enable != 0;
-  for (auto& g : c->graphs) {   // graphs captured with the other launch mode
-    if (g.exec) cudaGraphExecDestroy(g.exec);
-    g.exec = nullptr;
-    g.seen = 0;
-  }
+  drop_graphs(c);   // graphs captured with the other launch mode
   return UNO_OK;
 }
 
 int uno_set_fused(uno_ctx* c, int enable) {
   if (!c) return UNO_ERR_ARG;
   c->fused_enabled = enable != 0;
-  for (auto& g : c->graphs) {   // graphs captured with the other pipeline
-    if (g.exec) cudaGraphExecDestroy(g.exec);
-    g.exec = nullptr;
-    g.seen = 0;
-  }
+  drop_graphs(c);   // graphs captured with the other pipeline
   return c->fused ? UNO_OK : UNO_ERR_UNSUPPORTED;
 }
 
 int uno_set_verify_split(uno_ctx* c, int max_ctas) {
   if (!c || max_ctas < 0) return UNO_ERR_ARG;
   c->verify_split_ctas = max_ctas;
-  for (auto& g : c->graphs) {
-    if (g.exec) cudaGraphExecDestroy(g.exec);
-    g.exec = nullptr;
-    g.seen = 0;
-  }
+  drop_graphs(c);
   return UNO_OK;
 }
 
@@ -1799,18 +1826,31 @@ size_t uno_spec_verify_workspace_bytes(int n_req, int n_tests, int vocab) {
   return verify_ws_layout(n_req, n_tests, vocab).total;
 }
 
+// Host-side checks of a stand-alone spec_verify call (everything but the
+// workspace): UNO_OK or UNO_ERR_ARG, decided before anything is enqueued.
+static int verify_args_check(const float* p, const float* q, const int32_t* drafts, int n_req,
+                             int n_tests, int vocab, const uint32_t* streams, const int32_t* pos0,
+                             const int32_t* out_tokens, const int32_t* n_out) {
+  if (!p || !q || !drafts || !streams || !pos0 || !out_tokens || !n_out) return UNO_ERR_ARG;
+  if (n_req < 1 || n_tests < 1 || vocab < 4 || vocab % 4 || vocab > MAX_VOCAB || n_tests > 1024)
+    return UNO_ERR_ARG;
+  // grid rows of the reduction (row, chunk) CTAs
+  if ((long long)n_req * 2 * n_tests > 65535LL) return UNO_ERR_ARG;
+  return UNO_OK;
+}
+
 int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n_req, int n_tests,
                     int vocab, uint64_t seed, const uint32_t* streams, const int32_t* pos0,
                     int32_t* out_tokens, int32_t* n_out, void* ws, size_t ws_bytes,
                     uno_stream_t stream) {
-  if (!p || !q || !drafts || !streams || !pos0 || !out_tokens || !n_out || !ws) return UNO_ERR_ARG;
-  if (n_req < 1 || n_tests < 1 || vocab < 4 || vocab % 4 || vocab > MAX_VOCAB || n_tests > 1024)
-    return UNO_ERR_ARG;
+  const int rc = verify_args_check(p, q, drafts, n_req, n_tests, vocab, streams, pos0, out_tokens,
+                                   n_out);
+  if (rc != UNO_OK) return rc;
+  if (!ws) return UNO_ERR_ARG;
   const VerifyWs w = verify_ws_layout(n_req, n_tests, vocab);
   if (ws_bytes < w.total || ((uintptr_t)ws & 255)) return UNO_ERR_ARG;
   int ch, nch;
   chunking(vocab, &ch, &nch);
-  if ((long long)n_req * 2 * n_tests > 65535LL) return UNO_ERR_ARG;
   VerifyArgs a{};
   a.p = p; a.q = q;
   a.V = vocab; a.nch = nch; a.ch = ch;
@@ -1835,6 +1875,7 @@ int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n
   a.rows_red = 2 * n_tests;
   a.n_p = n_tests;
   a.status = nullptr;
+  a.fixed_at = -1;
   launch_verify(false, (cudaStream_t)stream, a, n_req);
   spec_resid_kernel<<<dim3(nch, n_req), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
@@ -1855,17 +1896,39 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is asked
-// for once per device (with that device current) and cached.
+// for once per device (with that device current) and cached, together with
+// the unique id of the device's current context: after a cudaDeviceReset
+// the library's image is loaded again into a new context, the id changes
+// and the address is looked up again.
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+static bool current_ctx_id(unsigned long long* id) {
+  static CtxGetIdFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetIdFn)f;
+  }
+  return fn && fn(nullptr, id) == CUDA_SUCCESS;   // null: the calling thread's current context
+}
+
 static int noalloc_scratch(void** out) {
   static std::mutex mu;
   static void* addr[256] = {};
+  static unsigned long long ctx_id[256] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return UNO_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  if (!addr[dev] || !have_id || id != ctx_id[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return UNO_ERR_CUDA;
     addr[dev] = p;
+    ctx_id[dev] = have_id ? id : 0;
   }
   *out = addr[dev];
   return UNO_OK;
@@ -1877,6 +1940,10 @@ int uno_spec_verify_noalloc(const float* p, const float* q, const int32_t* draft
                             int n_tests, int vocab, uint64_t seed, const uint32_t* streams,
                             const int32_t* pos0, int32_t* out_tokens, int32_t* n_out,
                             uno_stream_t stream) {
+  // every argument check before anything is enqueued on the shared array
+  const int arc = verify_args_check(p, q, drafts, n_req, n_tests, vocab, streams, pos0, out_tokens,
+                                    n_out);
+  if (arc != UNO_OK) return arc;
   const size_t need = uno_spec_verify_workspace_bytes(n_req, n_tests, vocab);
   if (need == 0) return UNO_ERR_ARG;
   if (need > NOALLOC_SCRATCH_BYTES) return UNO_ERR_CAPACITY;

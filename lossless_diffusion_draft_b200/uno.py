@@ -86,6 +86,8 @@ def load_library(path=LIB_PATH):
         "uno_set_fused": (i32, [vp, i32]),
         "uno_set_verify_split": (i32, [vp, i32]),
         "uno_set_counter_sync": (i32, [vp, i32]),
+        "uno_debug_set_fixed_accept": (i32, [vp, i32]),
+        "uno_debug_set_dep_wait": (i32, [vp, u64, ctypes.c_uint32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
         "uno_profile_end": (i32, [vp, vp, vp, vp]),
@@ -241,6 +243,18 @@ def uno_set_verify_split(ctx, max_ctas):
 def uno_set_counter_sync(ctx, enable):
     """Fused pipeline: GEMMs wait on completion counters (True) or grid dependencies."""
     _check(load_library().uno_set_counter_sync(ctx.handle, int(bool(enable))), ctx.handle)
+
+
+def uno_debug_set_fixed_accept(ctx, a):
+    """Benchmark tap: force the accepted length a (first token + accepted
+    drafts) of later steps; a <= 0 turns it off."""
+    _check(load_library().uno_debug_set_fixed_accept(ctx.handle, int(a)), ctx.handle)
+
+
+def uno_debug_set_dep_wait(ctx, limit_ns, extra=0):
+    """Test tap: counter waits give up after limit_ns; extra > 0 makes them
+    unreachable (the step then raises the device flag instead of hanging)."""
+    _check(load_library().uno_debug_set_dep_wait(ctx.handle, int(limit_ns), int(extra)), ctx.handle)
 
 
 def uno_release(ctx, req_id):

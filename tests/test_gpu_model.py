@@ -377,3 +377,65 @@ def test_counter_sync_matches_grid_dependencies():
         assert seq == runs[0][0]
         for a, b in zip(logits, runs[0][1]):
             assert torch.equal(a, b)
+
+
+def test_small_bf16_many_rows_unfused_and_unsplit_attention():
+    """A decode batch past the fused pipeline's 128 rows and past one
+    attention CTA per SM: 40 requests x 9 draft rows = 360 rows take the
+    unfused kernels with several GEMM token tiles, and 40 x 4 kv heads = 160
+    (query tile, request x kv head) groups leave no room for key splits, so
+    attention runs unsplit.  Logits, decisions and every layer's KV cache
+    against the oracle, two iterations."""
+    before = uno.uno_debug_launch_counts()
+    tally, _, worst = _run("small", 40, 24, 2, 2e-2, 2e-2, False, max_ctx=80)
+    after = uno.uno_debug_launch_counts()
+    assert tally.mismatches <= max(1, tally.positions // 1000), tally.notes
+    assert after["tc_gemm"] > before["tc_gemm"] and after["tc_attn"] > before["tc_attn"]
+
+
+def test_counter_wait_runs_out_and_raises_the_flag():
+    """Bounded waits: with every completion-counter target made unreachable
+    and a 2 ms limit, each waiting GEMM gives up, raises the device flag and
+    goes on, so the step ends (no hang) and uno_status reports
+    UNO_ERR_DEVICE_CHECK; with the targets restored the next step is clean."""
+    cfg, ctx, ids, model, states = _setup("small", 2, 24, 100, n_layers=2)
+    B = cfg["B"]
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((2, B + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(2, dtype=torch.int32, device="cuda")
+    assert uno.uno_set_fused(ctx, True)
+    uno.uno_set_counter_sync(ctx, True)
+    uno.uno_debug_set_dep_wait(ctx, 2_000_000, extra=1)
+    uno.uno_spec_step(ctx, req, out, n_new)
+    with pytest.raises(uno.UnoError) as e:
+        uno.uno_status(ctx)
+    assert e.value.code == uno.UNO_ERR_DEVICE_CHECK
+    uno.uno_debug_set_dep_wait(ctx, 1_000_000_000, extra=0)
+    uno.uno_spec_step(ctx, req, out, n_new)
+    uno.uno_status(ctx)
+    nn = n_new.cpu()
+    assert all(2 <= int(x) <= B + 1 for x in nn)
+    ctx.close()
+
+
+def test_fixed_accept_tap():
+    """The benchmark tap forces a = 3 accepted tokens: every request emits
+    x_1..x_3 and one more token, and the cache advances by 4."""
+    cfg, ctx, ids, model, states = _setup("small", 3, 24, 100, n_layers=2)
+    B = cfg["B"]
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((3, B + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(3, dtype=torch.int32, device="cuda")
+    uno.uno_debug_set_fixed_accept(ctx, 3)
+    for _ in range(2):
+        c0 = [uno.uno_request_state(ctx, i)[0] for i in ids]
+        uno.uno_spec_step(ctx, req, out, n_new)
+        uno.uno_status(ctx)
+        dr = uno.uno_debug_read(ctx, uno.UNO_DBG_DRAFTS, torch.empty((3, B), dtype=torch.int32))
+        assert n_new.cpu().tolist() == [4, 4, 4]
+        for i in range(3):
+            assert out[i, :3].cpu().tolist() == dr[i, :3].tolist()
+            assert uno.uno_request_state(ctx, ids[i])[0] == c0[i] + 4
+    with pytest.raises(uno.UnoError):
+        uno.uno_debug_set_fixed_accept(ctx, B + 1)
+    ctx.close()

@@ -50,11 +50,24 @@ def _no_alloc(p, q, drafts, streams, pos0, seed):
 def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
     build.build()
     uno.load_library()
-    # two different workloads back to back: the shared scratch array keeps the
-    # first call's contents, the second call must not be disturbed by them
-    for call, (n_req, n_tests, V) in enumerate([(64, 16, 32000), (37, 9, 151936)]):
+    # different workloads back to back: the shared scratch array keeps each
+    # call's contents, the next call must not be disturbed by them.  The first
+    # two need more than 4096 (row, chunk) CTAs and take the split form; the
+    # third (4 x 16 rows x 4 chunks = 256 CTAs) takes the fused form, whose
+    # row and request completion counters live in the array and start at
+    # zero only because the call clears them.  Before it, a rejected call
+    # (vocab not a multiple of 4) must leave the array and the stream alone.
+    for call, (n_req, n_tests, V) in enumerate([(64, 16, 32000), (37, 9, 151936), (4, 8, 32000)]):
         seed = 11 + call
         args = _inputs(n_req, n_tests, V, seed)
+        if call == 2:
+            p, q, drafts, streams, pos0 = args
+            out = torch.empty((n_req, n_tests + 1), dtype=torch.int32, device="cuda")
+            n_out = torch.empty((n_req,), dtype=torch.int32, device="cuda")
+            code = uno.load_library().uno_spec_verify_noalloc(
+                p.data_ptr(), q.data_ptr(), drafts.data_ptr(), n_req, n_tests, 6, 0,
+                streams.data_ptr(), pos0.data_ptr(), out.data_ptr(), n_out.data_ptr(), None)
+            assert code == uno.UNO_ERR_ARG
         need = uno.uno_spec_verify_workspace_bytes(n_req, n_tests, V)
         assert need <= uno.uno_spec_verify_noalloc_max_bytes()
         want_out, want_n = _with_workspace(*args, seed)
@@ -67,7 +80,7 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
 
 def test_noalloc_rejects_sizes_beyond_its_array():
     cap = uno.uno_spec_verify_noalloc_max_bytes()
-    n_req, n_tests, V = 4096, 16, 151936          # the microbenchmark batch: > 4 MiB of scratch
+    n_req, n_tests, V = 1024, 16, 151936          # 16384 rows: > 4 MiB of scratch
     assert uno.uno_spec_verify_workspace_bytes(n_req, n_tests, V) > cap
     dummy = torch.zeros(1, dtype=torch.float32, device="cuda")
     code = uno.load_library().uno_spec_verify_noalloc(
