@@ -543,7 +543,8 @@ def spec_verify_micro(args, device, pk, n_req=None):
     n_out = torch.empty(n_req, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
     call = lambda: uno.uno_spec_verify(p, q, drafts, cfg["seed"], streams, pos0, out, n_out, ws)
-    K = max(args.steps, 10)
+    # about half a second of calls, so the clock sampler sees several samples
+    K = max(args.steps, 500)
     for _ in range(max(args.warmup, 3)):
         call()
     torch.cuda.synchronize()

@@ -126,6 +126,27 @@ int uno_prefill(uno_ctx *ctx, int n_req, const int32_t *prompts_dev, int prompt_
                 int32_t *req_ids_host_out);
 
 /*
+ * The training-form forward (blog page "…Uno 的无损加速之路", section Diffusion
+ * Distillation：一步蒸馏 + 块级扩散): one pass over the concatenation [x, z] of
+ * a clean sequence x and its noised copy z (2L rows, context 2L) with the
+ * block-causal mask - a clean token sees the clean tokens up to its own
+ * position; a noised token sees the clean tokens before its block (blocks of
+ * B positions from position 0) and the noised tokens of its own block up to
+ * its own position - and the adapter gated off on x and on on z, so one
+ * forward gives the AR (teacher) logits of x and the diffusion (student)
+ * logits of z.  Forward only: no loss (the pages' loss formulas are missing).
+ *   tokens_dev: int32 [n_seq, 2L] (device): x_0..x_{L-1}, then z_0..z_{L-1}
+ *               (z_i at position i; the noise prior's tokens, e.g. MASK).
+ *   logits_dev: f32 [n_seq, 2L, vocab] (device, caller-owned), row order as
+ *               the tokens.
+ * Needs n_seq * 2L <= max(512, max_batch * (B + 1)) rows (else
+ * UNO_ERR_CAPACITY), L <= max_ctx, and 2 n_seq free request slots (their
+ * pages hold the clean and the noised keys during the call and are free
+ * again after it).  Stream-ordered, no host synchronisation after the setup.
+ */
+int uno_train_forward(uno_ctx *ctx, int n_seq, const int32_t *tokens_dev, int L, float *logits_dev);
+
+/*
  * One Psi-Spec iteration for n_req admitted requests (req_ids_dev: int32
  * [n_req] slot ids, distinct, device).  Outputs (device, caller-owned):
  *   out_tokens_dev int32 [n_req, B+1]: the emitted tokens (first n_new valid);
@@ -212,6 +233,39 @@ int uno_debug_set_fixed_accept(uno_ctx *ctx, int a);
  */
 int uno_debug_set_dep_wait(uno_ctx *ctx, uint64_t limit_ns, uint32_t extra);
 
+/*
+ * Nucleus (top-p) sampling (blog page "…Uno 的无损加速之路", section 我的判断:
+ * the evaluation setting is temperature 1 with top-p 0.95, and losslessness
+ * holds with respect to that sampling distribution).  With top_p < 1 every
+ * row a later step samples or verifies - the AR rows p and the drafter's
+ * rows q alike - is restricted to its nucleus: the smallest set of most
+ * probable tokens whose probability reaches top_p (tokens ordered by
+ * probability, ties by token id; the token that crosses top_p is kept), and
+ * renormalised.  Drafting, the accept tests, the residual max(0, p - q), the
+ * bonus token and uno_ar_step all see the filtered distributions, so the
+ * output follows the AR model's filtered distribution.  top_p = 1 (the
+ * default) turns the filter off; top_p outside (0, 1]: UNO_ERR_ARG.  Drops
+ * captured graphs.
+ */
+int uno_set_top_p(uno_ctx *ctx, float top_p);
+
+/*
+ * The nucleus of rows of logits as a stand-alone kernel (the filter
+ * uno_set_top_p applies, one CTA per row):
+ *   logits_dev: f32 [rows, vocab] (device, 16-byte aligned, vocab % 4 == 0);
+ *   top_p in (0, 1);
+ *   out_dev:    int32 [rows, 2] (device): per row the order-preserving key
+ *               of the crossing logit l* (the float's bits b, as unsigned:
+ *               ~b if the sign is set, else b | 0x80000000; -0 counts as +0)
+ *               and id_cut.  Token v is in the nucleus iff key(l_v) > key
+ *               or (key(l_v) == key and v <= id_cut).
+ * The probability masses are summed as exact fixed-point integers (weights
+ * exp(l - max) in units of 2^-40), so the result is deterministic.  Never
+ * synchronises; UNO_ERR_ARG on bad sizes or pointers.
+ */
+int uno_top_p_filter(const float *logits_dev, int rows, int vocab, float top_p, int32_t *out_dev,
+                     uno_stream_t stream);
+
 /* Free a request's slot and pages (stream-ordered after earlier work). */
 int uno_release(uno_ctx *ctx, int req_id);
 
@@ -235,10 +289,16 @@ int uno_request_state(uno_ctx *ctx, int req_id, int32_t *cached_out, int32_t *pe
  *   UNO_DBG_LOGITS_VERIFY f32   [n_req, B, vocab]   verify-pass logits
  *   UNO_DBG_DRAFTS        int32 [n_req, B]          drafted block x_1..x_B
  *   UNO_DBG_LOGITS_AR     f32   [n_req, vocab]      AR-step logits
+ *   UNO_DBG_TOPP_DRAFT    int32 [n_req, B+1, 2]     nucleus of each draft row (top_p < 1;
+ *                                                   row 1 unused; AR step: [n_req, 1, 2])
+ *   UNO_DBG_TOPP_VERIFY   int32 [n_req, B, 2]       nucleus of each verify row
+ * A nucleus entry is (key, id_cut) as uno_top_p_filter writes it.  The
+ * logits are those of the model (before any nucleus filter).
  * bytes must not exceed the buffer's size for max_batch requests.
  */
 enum uno_debug_buf {
-  UNO_DBG_LOGITS_DRAFT = 0, UNO_DBG_LOGITS_VERIFY = 1, UNO_DBG_DRAFTS = 2, UNO_DBG_LOGITS_AR = 3
+  UNO_DBG_LOGITS_DRAFT = 0, UNO_DBG_LOGITS_VERIFY = 1, UNO_DBG_DRAFTS = 2, UNO_DBG_LOGITS_AR = 3,
+  UNO_DBG_TOPP_DRAFT = 4, UNO_DBG_TOPP_VERIFY = 5
 };
 int uno_debug_read(uno_ctx *ctx, int which, void *dst_host, size_t bytes);
 

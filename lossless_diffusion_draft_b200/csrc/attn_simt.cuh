@@ -3,10 +3,11 @@
 //
 // Mask (blog page "…Uno 的无损加速之路", section Diffusion Distillation：一步蒸馏 +
 // 块级扩散): the clean sequence is causal; a noised block is causal inside
-// itself and sees every clean token before it.  In a decode pass the keys are
-// [cache 0..c-1, pending c, block c+1..c+B], all written to the pool by the
-// RoPE/KV kernel before this one runs, and the rule reduces to "key position
-// <= query position" for every row of both passes.
+// itself and sees every clean token before it.  A row's keys are the two
+// ranges of RowKeys (layers.cuh).  In a decode pass the keys are [cache
+// 0..c-1, pending c, block c+1..c+B] of one slot, all written to the pool by
+// the RoPE/KV kernel before this one runs, and the rule reduces to "key
+// position <= query position" for every row of both passes.
 //
 // One CTA takes (split s, query tile, request x kv head): up to 72 query rows
 // (tokens x the kv head's query heads), streams its share of the key range in
@@ -35,6 +36,7 @@ struct AttnParams {
   float scale;
   int rows_per_req;
   const int32_t* row_pos; const int32_t* row_slot;
+  RowKeys keys;                   // per-row key ranges (block-causal rule)
   int n_splits, n_qtiles;
   float* ws; unsigned* counters;  // split partials, per-group counters (zero, left zero)
 };
@@ -60,9 +62,10 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
   if (ntok <= 0) return;
   const int nq = ntok * G;
   const int row0 = req * p.rows_per_req + tok0;
-  const int slot = p.row_slot[row0];
-  const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
-  const int ntiles = (nkeys + ATT_KT - 1) / ATT_KT;
+  // the tile list: key tiles of the clean range, then of the noised range
+  const KeyTiles kt = p.keys.tiles(p.row_pos, p.row_slot, row0, ntok, ATT_KT,
+                                   p.kv.pages_per_req * (KV_PAGE / ATT_KT));
+  const int ntiles = kt.n1 + kt.n2;
   const int t_begin = (int)((long long)ntiles * split / p.n_splits);
   const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -77,26 +80,30 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
     q_s[idx] = (to_f(qkv[e]) + qlo) * p.scale;
   }
   float m_i[QPW], l_i[QPW], o_i[QPW][EPL];
-  int qpos[QPW];
+  int qlim[QPW], qlo2[QPW], qhi2[QPW];   // each row's clean range [0, lim), noised [lo2, hi2)
 #pragma unroll
   for (int t = 0; t < QPW; ++t) {
     m_i[t] = -INFINITY; l_i[t] = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) o_i[t][e] = 0.f;
     const int qi = warp + 4 * t;
-    qpos[t] = (qi < nq) ? p.row_pos[row0 + qi / G] : -1;
+    qlim[t] = qlo2[t] = qhi2[t] = 0;
+    if (qi < nq) p.keys.ranges(p.row_pos, row0 + qi / G, qlim[t], qlo2[t], qhi2[t]);
   }
 
   const KV* pool = reinterpret_cast<const KV*>(p.kv.pool);
   for (int tile = t_begin; tile < t_end; ++tile) {
+    const bool seg2 = tile >= kt.n1;
+    const int kp0 = (seg2 ? kt.p2 + (tile - kt.n1) : tile) * ATT_KT;
+    const int tslot = seg2 ? kt.slot2 : kt.slot1;
     __syncthreads();
     for (int idx = threadIdx.x; idx < ATT_KT * HD; idx += ATT_THREADS) {
       const int j = idx / HD, d = idx % HD;
-      const int kp = tile * ATT_KT + j;
+      const int kp = kp0 + j;
       float kval = 0.f, vval = 0.f;
-      if (kp < nkeys) {
+      {
         int ok;
-        const size_t off = p.kv.offset(p.layer, slot, kp, 0, kvh, ok);
+        const size_t off = p.kv.offset(p.layer, tslot, kp, 0, kvh, ok);
         if (ok) {
           kval = to_f(pool[off + d]);
           if (p.kv.n_planes == 3) kval += to_f(pool[off + p.kv.plane_stride() + d]);   // K lo
@@ -107,13 +114,13 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_simt_kernel(const AttnParams
       v_s[j * HD + d] = vval;
     }
     __syncthreads();
-    const int kp = tile * ATT_KT + lane;
+    const int kp = kp0 + lane;
 #pragma unroll
     for (int t = 0; t < QPW; ++t) {
       const int qi = warp + 4 * t;
       if (qi >= nq) continue;
       float sc = -INFINITY;
-      if (kp < nkeys && kp <= qpos[t]) {
+      if (seg2 ? (kp >= qlo2[t] && kp < qhi2[t]) : kp < qlim[t]) {
         float dot = 0.f;
         const float* qr = q_s + qi * HD;
         const float* kr = k_s + lane * (HD + 1);

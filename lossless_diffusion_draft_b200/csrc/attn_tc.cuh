@@ -5,9 +5,11 @@
 // Mask (blog page "不砸掉重来，给自回归 LLM 装一对“扩散翅膀”：Uno 的无损加速之路",
 // section Diffusion Distillation：一步蒸馏 + 块级扩散): the clean sequence is
 // causal; a noised block is causal inside itself and sees every clean token
-// before it.  In the decode passes every key of a request (cache, pending
-// token, block) is in the pool and the rule is "key position <= query
-// position" for every row.
+// before it.  A row's keys are two ranges (RowKeys in layers.cuh): clean keys
+// of its clean slot at positions [0, lim), and, for a noised row of the
+// training form [x, z], noised keys of its own slot at [block start, pos].
+// In the decode passes every key of a request (cache, pending token, block)
+// is in its one slot and the rule is "key position <= query position".
 //
 // One CTA takes (key split, query tile, request x kv head).  Its 128 query
 // rows are (token, head of the kv group) pairs, so the GQA group shares each
@@ -52,6 +54,7 @@ struct AttnTcParams {
   float scale_log2;                 // log2(e) / sqrt(HD)
   int rows_per_req;
   const int32_t* row_pos; const int32_t* row_slot;
+  RowKeys keys;                     // per-row key ranges (block-causal rule)
   int n_splits, n_qtiles;
   float* ws;                        // split partials [group][split][128][HD + 4]
   int32_t* status;
@@ -170,25 +173,26 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   const int ntok = min(TQ, p.rows_per_req - tok0);
   const int nq = ntok * G;
   const int row0 = req * p.rows_per_req + tok0;
-  // the position of each query row (warps 0-3, one row per thread)
-  int qpos = -1;
-  if (warp < 4 && threadIdx.x < nq) qpos = p.row_pos[row0 + threadIdx.x / G];
-  const int slot = p.row_slot[row0];
-  const int nkeys = p.row_pos[row0 + ntok - 1] + 1;
-  int ntiles = (nkeys + ATC_KT - 1) / ATC_KT;
-  if (ntiles > p.pages_per_req) {
-    if (threadIdx.x == 0 && split == 0) raise_status(p.status, ST_POS_OVERFLOW);
-    ntiles = p.pages_per_req;
-  }
+  // each query row's key ranges (warps 0-3, one row per thread): clean keys
+  // [0, qlim), noised keys [qlo2, qhi2)
+  int qlim = 0, qlo2 = 0, qhi2 = 0;
+  if (warp < 4 && threadIdx.x < nq) p.keys.ranges(p.row_pos, row0 + threadIdx.x / G, qlim, qlo2, qhi2);
+  // the tile's key list: pages of the clean range, then of the noised range
+  const KeyTiles kt = p.keys.tiles(p.row_pos, p.row_slot, row0, ntok, ATC_KT, p.pages_per_req);
+  if (kt.overflow && threadIdx.x == 0 && split == 0) raise_status(p.status, ST_POS_OVERFLOW);
+  const int ntiles = kt.n1 + kt.n2;
   const int t_begin = (int)((long long)ntiles * split / p.n_splits);
   const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
   const int n = t_end - t_begin;
+  auto page_of_tile = [&](int t) {   // pool page of tile t of the list
+    return t < kt.n1 ? p.page_table[(size_t)kt.slot1 * p.pages_per_req + t]
+                     : p.page_table[(size_t)kt.slot2 * p.pages_per_req + kt.p2 + (t - kt.n1)];
+  };
 
   // the split's page numbers, fetched in one round while the q rows load
   __shared__ int s_pages[ATC_PAGE_PF];
   if (warp == 4) {
-    for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32)
-      s_pages[i] = p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+    for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32) s_pages[i] = page_of_tile(t_begin + i);
   }
   tc_fence_before();
   __syncthreads();
@@ -215,8 +219,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         const uint32_t phase = (uint32_t)(i / C::STAGES) & 1;
         if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
         mbar_expect_tx(&kv_full[stage], 3 * C::KV_BYTES);
-        const int page = i < ATC_PAGE_PF ? s_pages[i]
-                                         : p.page_table[(size_t)slot * p.pages_per_req + t_begin + i];
+        const int page = i < ATC_PAGE_PF ? s_pages[i] : page_of_tile(t_begin + i);
         // pool rows of the page's K hi, K lo and V planes for this kv head
         const int rk = (((p.layer * p.n_pages + page) * 3 + 0) * p.Hkv + kvh) * KV_PAGE;
         const int rkl = rk + p.Hkv * KV_PAGE;
@@ -315,16 +318,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // raw scores; keys past the row's position (only in its last tile) -> -inf
-      const int kp0 = (t_begin + i) * ATC_KT;
+      // raw scores; keys outside the row's range of this tile's segment -> -inf
+      // (only the edge tiles of a range need the test)
+      const int ti = t_begin + i;
+      const bool seg2 = ti >= kt.n1;
+      const int kp0 = (seg2 ? kt.p2 + (ti - kt.n1) : ti) * ATC_KT;
+      const int klo = seg2 ? qlo2 : 0, khi = seg2 ? qhi2 : qlim;
       float mx = -INFINITY;
-      if (kp0 + ATC_KT - 1 <= qpos) {
+      if (kp0 >= klo && kp0 + ATC_KT <= khi) {
 #pragma unroll
         for (int j = 0; j < ATC_KT; ++j) mx = fmaxf(mx, s[j]);
       } else {
 #pragma unroll
         for (int j = 0; j < ATC_KT; ++j) {
-          if (kp0 + j > qpos) s[j] = -INFINITY;
+          if (kp0 + j < klo || kp0 + j >= khi) s[j] = -INFINITY;
           mx = fmaxf(mx, s[j]);
         }
       }

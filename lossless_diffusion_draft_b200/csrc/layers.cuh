@@ -48,7 +48,69 @@ struct KvLayout {
 };
 
 // Pass kinds (a pass is one forward over a set of rows).
-enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3 };
+enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3, PASS_TRAIN = 4 };
+
+// The keys each query row sees, by the block-causal rule (blog page "…Uno
+// 的无损加速之路", section Diffusion Distillation：一步蒸馏 + 块级扩散: a clean
+// query sees clean keys up to its own position; a query of a noised block
+// sees the clean keys before its block and the keys of its own block up to
+// its own position).  Keys live in the pool under a slot and a position, so a
+// row's keys are two ranges:
+//   clean range:  slot cslot[r], positions [0, lim) with lim = pos + 1, or the
+//                 block start for a noised row of the training form;
+//   noised range: (training form only, blk[r] >= 0) the row's own slot
+//                 row_slot[r], positions [blk[r], pos + 1).
+// With blk null every row is "causal by position" in its own slot: the
+// decode passes, where the noised block's keys share the request's slot.
+struct KeyTiles {
+  int slot1, n1;      // clean range: slot, pages 0 .. n1-1
+  int slot2, p2, n2;  // noised range: slot, pages p2 .. p2+n2-1 (n2 = 0: none)
+  bool overflow;      // a range reached past the slot's pages (clipped)
+};
+struct RowKeys {
+  const int32_t* cslot;   // [M] clean-range slot (null: row_slot)
+  const int32_t* blk;     // [M] noised block start, -1 for a clean row (null: all clean)
+  __device__ __forceinline__ void ranges(const int32_t* row_pos, int r, int& lim, int& lo2,
+                                         int& hi2) const {
+    const int pos = row_pos[r];
+    const int b = blk ? blk[r] : -1;
+    lim = b < 0 ? pos + 1 : b;
+    lo2 = b < 0 ? 0 : b;
+    hi2 = b < 0 ? 0 : pos + 1;
+  }
+  // The page lists of rows row0 .. row0 + ntok - 1 (one request): the union of
+  // their ranges, in pages of `page` keys.
+  __device__ __forceinline__ KeyTiles tiles(const int32_t* row_pos, const int32_t* row_slot,
+                                            int row0, int ntok, int page, int pages_per_req) const {
+    KeyTiles t{cslot ? cslot[row0] : row_slot[row0], 0, -1, 0, 0, false};
+    int lim1 = 0, lo2 = 0x7fffffff, hi2 = 0;
+    if (!blk) {
+      // causal by position: a request's rows are in position order, so the
+      // last row reaches furthest (one load on the decode passes' path)
+      lim1 = row_pos[row0 + ntok - 1] + 1;
+      ntok = 0;
+    }
+    for (int k = 0; k < ntok; ++k) {
+      int lim, l2, h2;
+      ranges(row_pos, row0 + k, lim, l2, h2);
+      lim1 = max(lim1, lim);
+      if (h2 > l2) {
+        lo2 = min(lo2, l2);
+        hi2 = max(hi2, h2);
+        t.slot2 = row_slot[row0 + k];
+      }
+    }
+    t.n1 = (lim1 + page - 1) / page;
+    if (t.n1 > pages_per_req) { t.n1 = pages_per_req; t.overflow = true; }
+    if (hi2 > 0) {
+      t.p2 = lo2 / page;
+      int e = (hi2 + page - 1) / page;
+      if (e > pages_per_req) { e = pages_per_req; t.overflow = true; }
+      t.n2 = max(0, e - t.p2);
+    }
+    return t;
+  }
+};
 
 struct RowArgs {
   int kind;
@@ -67,6 +129,8 @@ struct RowArgs {
   float* x;                    // [M, d] fp32 residual
   int32_t* status;
   unsigned* zero_ctr; int n_zero;   // the pass's completion counters (zeroed here), or null
+  // training form: per-row key ranges (RowKeys) written here
+  int32_t* row_cslot; int32_t* row_blk;
 };
 
 // a1: build the rows of a pass and gather their embeddings.
@@ -92,6 +156,21 @@ __global__ void build_rows_kernel(const RowArgs a) {
     slot = a.prefill_slot;
     tok = a.prompt[j];
     pos = a.prefill_pos0 + j;
+  } else if (a.kind == PASS_TRAIN) {
+    // training form [x, z] of sequence req: rows j < L are the clean tokens
+    // x_j (gate 0, its clean slot), rows L + i the noised tokens z_i (gate on,
+    // its noised slot) at the same positions; block of position i: B-aligned
+    const int L = a.rows_per_req / 2;
+    const bool noised = j >= L;
+    const int sa = a.req_slot[2 * req], sb = a.req_slot[2 * req + 1];
+    pos = noised ? j - L : j;
+    tok = a.prompt[(size_t)req * a.rows_per_req + j];
+    slot = noised ? sb : sa;
+    gate = noised ? a.lora_scale : 0.f;
+    if (threadIdx.x == 0) {
+      a.row_cslot[row] = sa;
+      a.row_blk[row] = noised ? (pos / a.B) * a.B : -1;
+    }
   } else {
     slot = a.req_slot[req];
     if (slot < 0 || slot >= a.max_batch) { raise_status(a.status, ST_BAD_SLOT); slot = 0; }

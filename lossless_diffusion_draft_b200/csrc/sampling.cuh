@@ -48,6 +48,48 @@ __device__ __forceinline__ float exp_rel(float x, float mL) {
 }
 
 // ---------------------------------------------------------------------------
+// Nucleus (top-p) filter of a row (blog page "…Uno 的无损加速之路", section
+// 我的判断: the lossless claim holds for the sampling distribution of
+// temperature 1 and top-p 0.95).  The nucleus is the smallest set of the most
+// probable tokens whose probability reaches top_p, tokens ordered by
+// probability with ties by token id; it is stored per row as an
+// order-preserving 32-bit key of the crossing logit and the last token id
+// kept among the tokens with exactly that logit.  Every kernel below reads a
+// filtered logit as l if the token is kept and -inf otherwise, so the
+// softmax of the filtered row is the renormalised nucleus distribution.
+// ---------------------------------------------------------------------------
+struct RowFilter { uint32_t key; int32_t id_cut; };
+// key(l) orders floats like their values: higher logit, higher key
+__device__ __forceinline__ uint32_t logit_key(float l) {
+  uint32_t u = __float_as_uint(l);
+  if (u == 0x80000000u) u = 0u;   // -0 and +0 are one value
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+// FILT = false: no filter (compiled out).
+template <bool FILT>
+struct Filt {
+  uint32_t key; int32_t id_cut;
+  __device__ __forceinline__ float operator()(float l, int v) const {
+    if (!FILT) return l;
+    const uint32_t k = logit_key(l);
+    return (k > key || (k == key && v <= id_cut)) ? l : -INFINITY;
+  }
+  __device__ __forceinline__ float4 four(float4 x, int v) const {
+    if (!FILT) return x;
+    return make_float4((*this)(x.x, v), (*this)(x.y, v + 1), (*this)(x.z, v + 2), (*this)(x.w, v + 3));
+  }
+};
+template <bool FILT>
+__device__ __forceinline__ Filt<FILT> filt_of(const RowFilter* f, size_t row) {
+  if (!FILT || !f) return Filt<FILT>{0u, -1};
+  const RowFilter r = f[row];
+  return Filt<FILT>{r.key, r.id_cut};
+}
+
+// ---------------------------------------------------------------------------
 // Phase A: reduce one chunk of one row to (max, sum exp(l - max)).  The
 // CTA's max comes first (warp butterfly, then the warps' maxima in order),
 // then every logit takes one exponential against it and the sums are added
@@ -55,7 +97,9 @@ __device__ __forceinline__ float exp_rel(float x, float mL) {
 // ---------------------------------------------------------------------------
 constexpr int CHUNK_IT = 8;   // float4 per thread: a chunk holds <= 8 * 4 * 256 = 8192 logits
 // red: at least 2 * SAMPLE_THREADS / 32 floats of shared memory.
-__device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red) {
+template <bool FILT = false>
+__device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red,
+                                               Filt<FILT> f = Filt<FILT>{0u, -1}) {
   constexpr int NW = SAMPLE_THREADS / 32;
   // float4 path: rows start on 16-byte boundaries (vocab % 4 == 0 is required)
   const int n4 = (c1 - c0) >> 2;
@@ -66,12 +110,12 @@ __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1,
   for (int i = 0; i < CHUNK_IT; ++i) {
     const int j = threadIdx.x + i * SAMPLE_THREADS;
     if (j < n4) {
-      v[i] = __ldcs(r4 + j);
+      v[i] = f.four(__ldcs(r4 + j), c0 + 4 * j);
       m = fmaxf(m, fmaxf(fmaxf(v[i].x, v[i].y), fmaxf(v[i].z, v[i].w)));
     }
   }
   // scalar tail (chunk length not a multiple of 4: only the row's last chunk)
-  for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) m = fmaxf(m, row[j]);
+  for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) m = fmaxf(m, f(row[j], j));
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -90,7 +134,7 @@ __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1,
       if (j < n4)
         s += (exp_rel(v[i].x, mL) + exp_rel(v[i].y, mL)) + (exp_rel(v[i].z, mL) + exp_rel(v[i].w, mL));
     }
-    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += exp_rel(row[j], mL);
+    for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) s += exp_rel(f(row[j], j), mL);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -171,25 +215,30 @@ __device__ __forceinline__ RowStat combine_row(const float2* part, int nch) {
 
 // Weight functors used by the crossing scan (get4: four weights from v, a
 // multiple of 4).
+template <bool FILT = false>
 struct SoftmaxW {
   const float* row; float ML;          // row max x log2 e
-  __device__ __forceinline__ float operator()(int v) const { return exp_rel(row[v], ML); }
+  Filt<FILT> f;
+  __device__ __forceinline__ float operator()(int v) const { return exp_rel(f(row[v], v), ML); }
   __device__ __forceinline__ void get4(int v, float* w) const {
-    const float4 x = *reinterpret_cast<const float4*>(row + v);
+    const float4 x = f.four(*reinterpret_cast<const float4*>(row + v), v);
     w[0] = exp_rel(x.x, ML); w[1] = exp_rel(x.y, ML); w[2] = exp_rel(x.z, ML); w[3] = exp_rel(x.w, ML);
   }
 };
+template <bool FILT = false>
 struct ResidW {
   const float* p; const float* q; float lpL, lqL;   // lse_p, lse_q x log2 e
-  __device__ __forceinline__ float pair(float pv, float qv) const {
-    const float d = exp_rel(pv, lpL) - exp_rel(qv, lqL);
+  Filt<FILT> fp, fq;
+  __device__ __forceinline__ float pair(float pv, float qv, int v) const {
+    const float d = exp_rel(fp(pv, v), lpL) - exp_rel(fq(qv, v), lqL);
     return d > 0.f ? d : 0.f;
   }
-  __device__ __forceinline__ float operator()(int v) const { return pair(p[v], q[v]); }
+  __device__ __forceinline__ float operator()(int v) const { return pair(p[v], q[v], v); }
   __device__ __forceinline__ void get4(int v, float* w) const {
     const float4 x = *reinterpret_cast<const float4*>(p + v);
     const float4 y = *reinterpret_cast<const float4*>(q + v);
-    w[0] = pair(x.x, y.x); w[1] = pair(x.y, y.y); w[2] = pair(x.z, y.z); w[3] = pair(x.w, y.w);
+    w[0] = pair(x.x, y.x, v); w[1] = pair(x.y, y.y, v + 1); w[2] = pair(x.z, y.z, v + 2);
+    w[3] = pair(x.w, y.w, v + 3);
   }
 };
 
@@ -253,8 +302,10 @@ __device__ int chunk_crossing(const W& w, int c0, int c1, float base, float targ
 }
 
 // Sample a softmax row from its chunk pairs with uniform u (whole CTA).
+template <bool FILT = false>
 __device__ int sample_from_partials(const float* row, const float2* part, int nch, int ch, int V,
-                                    const RowStat& rs, float u, float* red) {
+                                    const RowStat& rs, float u, float* red,
+                                    Filt<FILT> f = Filt<FILT>{0u, -1}) {
   __shared__ int s_k;
   __shared__ float s_base;
   const float target = u * rs.Z;
@@ -269,7 +320,7 @@ __device__ int sample_from_partials(const float* row, const float2* part, int nc
   const float base = s_base;
   __syncthreads();
   if (k < 0) return 0;  // empty row (all -inf): only reachable with invalid logits
-  SoftmaxW w{row, rs.M * SAMPLE_LOG2E};
+  SoftmaxW<FILT> w{row, rs.M * SAMPLE_LOG2E, f};
   int lastpos;
   const int c0 = k * ch, c1 = min(V, c0 + ch);
   int t = chunk_crossing(w, c0, c1, base, target, &lastpos, red);
@@ -297,8 +348,10 @@ struct SampleArgs {
   float2* partial;            // [n_req * rows_per_req, nch]
   unsigned* row_counter;      // [n_req * rows_per_req], zero on entry, left zero
   int32_t* status;
+  const RowFilter* filt;      // nucleus of each logit row [n_req * logit_rows_per_req] (FILT)
 };
 
+template <bool FILT>
 __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const SampleArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last;
@@ -309,8 +362,9 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   const int req = rid / a.rows_per_req, s = rid % a.rows_per_req;
   const int lrow = (a.ar_mode || s == 0) ? 0 : s + 1;
   const float* row = a.logits + ((size_t)req * a.logit_rows_per_req + lrow) * a.V;
+  const Filt<FILT> f = filt_of<FILT>(a.filt, (size_t)req * a.logit_rows_per_req + lrow);
   const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
-  const float2 pr = reduce_chunk(row, c0, c1, red);
+  const float2 pr = reduce_chunk<FILT>(row, c0, c1, red, f);
   if (threadIdx.x == 0) {
     a.partial[(size_t)rid * a.nch + k] = pr;
     __threadfence();
@@ -333,7 +387,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   const int c = a.cached[slot];
   const uint32_t kind = (a.ar_mode || s == 0) ? KIND_FIRST : KIND_DRAFT;
   const float u = philox_uniform(a.seed, a.slot_stream[slot], (uint32_t)(c + 1 + s), kind);
-  const int t = sample_from_partials(row, part, a.nch, a.ch, a.V, rs, u, red);
+  const int t = sample_from_partials<FILT>(row, part, a.nch, a.ch, a.V, rs, u, red, f);
   if (threadIdx.x == 0) {
     if (a.ar_mode) {
       a.out_tok[req] = t;
@@ -380,6 +434,8 @@ struct VerifyArgs {
   // n_tests) tests instead of the accept tests' outcome; the residual
   // redraw or the bonus draw then runs as usual
   int fixed_at;
+  // nucleus of each p row [n_req * p_req_rows] and q row [n_req * q_req_rows] (FILT)
+  const RowFilter* filt_p; const RowFilter* filt_q;
 };
 
 // Slot, position of test 0 and Philox stream of a request.
@@ -430,6 +486,16 @@ __device__ void verify_finish(const VerifyArgs& a, int req, int slot, int pos0, 
 // The decision of request req once every reduced row's lse is in a.lse
 // (whole CTA): the accept tests, the first rejection, and either the bonus
 // draw and the commit here or the hand-over to spec_resid_kernel.
+template <bool FILT>
+__device__ __forceinline__ Filt<FILT> verify_filt_p(const VerifyArgs& a, int req, int prow_idx) {
+  return filt_of<FILT>(a.filt_p, (size_t)req * a.p_req_rows + prow_idx);
+}
+template <bool FILT>
+__device__ __forceinline__ Filt<FILT> verify_filt_q(const VerifyArgs& a, int req, int qrow_idx) {
+  return filt_of<FILT>(a.filt_q, (size_t)req * a.q_req_rows + qrow_idx);
+}
+
+template <bool FILT>
 __device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
   __shared__ int s_a;
   const size_t rbase = (size_t)req * a.rows_red;
@@ -446,7 +512,9 @@ __device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
     const float lse_p = __ldcg(&a.lse[rbase + j]);
     const float lse_q = verify_lse_q(a, req, j);
     const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + j), KIND_ACCEPT);
-    const bool acc = logf(u) < (prow[t] - lse_p) - (qrow[t] - lse_q);
+    const float lp = verify_filt_p<FILT>(a, req, a.p_row0 + j)(prow[t], t);
+    const float lq = verify_filt_q<FILT>(a, req, a.q_row0 + j)(qrow[t], t);
+    const bool acc = logf(u) < (lp - lse_p) - (lq - lse_q);
     if (!acc) atomicMin(&s_a, j);
   }
   __syncthreads();
@@ -466,8 +534,8 @@ __device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
       if (threadIdx.x == 0) s_rs2 = rs;
     }
     __syncthreads();
-    y = sample_from_partials(prow, a.partial + (rbase + a.n_tests) * a.nch, a.nch, a.ch, a.V,
-                             s_rs2, u, red);
+    y = sample_from_partials<FILT>(prow, a.partial + (rbase + a.n_tests) * a.nch, a.nch, a.ch, a.V,
+                                   s_rs2, u, red, verify_filt_p<FILT>(a, req, a.bonus_row));
   }
   if (threadIdx.x == 0) a.at_ws[req] = -1;
   verify_finish(a, req, slot, pos0, at, y);
@@ -482,8 +550,16 @@ __device__ __forceinline__ const float* verify_row(const VerifyArgs& a, int req,
   return a.q + ((size_t)req * a.q_req_rows + a.q_row0 + (r - a.n_p)) * a.V;
 }
 
+// The nucleus of the row a (request, reduced row) CTA reads.
+template <bool FILT>
+__device__ __forceinline__ Filt<FILT> verify_row_filt(const VerifyArgs& a, int req, int r) {
+  if (r < a.n_p) return verify_filt_p<FILT>(a, req, (r < a.n_tests) ? a.p_row0 + r : a.bonus_row);
+  return verify_filt_q<FILT>(a, req, a.q_row0 + (r - a.n_p));
+}
+
 // Fused form (few rows): grid (nch, n_req * rows_red).  The last chunk CTA
 // of a row forms its lse, the last row of a request decides.
+template <bool FILT>
 __global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last, s_req_last;
@@ -494,7 +570,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const Ve
   const int req = rid / a.rows_red, r = rid % a.rows_red;
   const float* row = verify_row(a, req, r);
   const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
-  const float2 pr = reduce_chunk(row, c0, c1, red);
+  const float2 pr = reduce_chunk<FILT>(row, c0, c1, red, verify_row_filt<FILT>(a, req, r));
   if (threadIdx.x == 0) {
     a.partial[(size_t)rid * a.nch + k] = pr;
     __threadfence();
@@ -519,27 +595,30 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const Ve
   __syncthreads();
   if (!s_req_last) return;
   __threadfence();
-  verify_decide(a, req, red);
+  verify_decide<FILT>(a, req, red);
 }
 
 // Split form (many rows), first kernel: grid (nch, n_req * rows_red), every
 // CTA reduces its chunk, writes the pair and exits (no counters, no waiting
 // on a round trip), so the loads of the next CTAs keep HBM busy.
+template <bool FILT>
 __global__ void __launch_bounds__(SAMPLE_THREADS, 4) spec_reduce_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   pdl_trigger();
   pdl_wait();
   const int k = blockIdx.x;
   const int rid = blockIdx.y;
-  const float* row = verify_row(a, rid / a.rows_red, rid % a.rows_red);
+  const int req = rid / a.rows_red, r = rid % a.rows_red;
+  const float* row = verify_row(a, req, r);
   const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
-  const float2 pr = reduce_chunk(row, c0, c1, red);
+  const float2 pr = reduce_chunk<FILT>(row, c0, c1, red, verify_row_filt<FILT>(a, req, r));
   if (threadIdx.x == 0) a.partial[(size_t)rid * a.nch + k] = pr;
 }
 
 // Split form, second kernel: one CTA per request; warp w forms the lse of
 // rows w, w + 8, ... (the same chunk-order combine as the fused form), then
 // the CTA decides.
+template <bool FILT>
 __global__ void __launch_bounds__(SAMPLE_THREADS) spec_decide_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   pdl_trigger();
@@ -552,7 +631,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_decide_kernel(const Verif
     if ((threadIdx.x & 31) == 0) a.lse[rid] = rs.M + logf(rs.Z);
   }
   __syncthreads();
-  verify_decide(a, req, red);
+  verify_decide<FILT>(a, req, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -564,6 +643,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_decide_kernel(const Verif
 // writes the outputs and the commit.  Requests without a rejection (at_ws =
 // -1) were finished by the first stage.
 // ---------------------------------------------------------------------------
+template <bool FILT>
 __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   __shared__ bool s_last;
@@ -577,7 +657,9 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
   const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + at) * a.V;
   const float lse_p = __ldcg(&a.lse[rbase + at]);
   const float lse_q = verify_lse_q(a, req, at);
-  const ResidW w{prow, qrow, lse_p * SAMPLE_LOG2E, lse_q * SAMPLE_LOG2E};
+  const Filt<FILT> fp = verify_filt_p<FILT>(a, req, a.p_row0 + at);
+  const ResidW<FILT> w{prow, qrow, lse_p * SAMPLE_LOG2E, lse_q * SAMPLE_LOG2E, fp,
+                       verify_filt_q<FILT>(a, req, a.q_row0 + at)};
   {
     // chunk sum: 16-byte loads, all of a thread's loads issued first
     const int b0 = k * a.ch, b1 = min(a.V, b0 + a.ch);
@@ -596,8 +678,9 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
 #pragma unroll
       for (int i = 0; i < MAXIT; ++i) {
         const int j = i0 + threadIdx.x + i * SAMPLE_THREADS;
-        if (j < n4) sacc += w.pair(x[i].x, z[i].x) + w.pair(x[i].y, z[i].y) +
-                            w.pair(x[i].z, z[i].z) + w.pair(x[i].w, z[i].w);
+        const int v = b0 + 4 * j;
+        if (j < n4) sacc += w.pair(x[i].x, z[i].x, v) + w.pair(x[i].y, z[i].y, v + 1) +
+                            w.pair(x[i].z, z[i].z, v + 2) + w.pair(x[i].w, z[i].w, v + 3);
       }
     }
     for (int v = b0 + (n4 << 2) + threadIdx.x; v < b1; v += SAMPLE_THREADS) sacc += w(v);
@@ -647,9 +730,183 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
       if (threadIdx.x == 0) s_rs = rs;
     }
     __syncthreads();
-    y = sample_from_partials(prow, a.partial + (rbase + at) * a.nch, a.nch, a.ch, a.V, s_rs, u, red);
+    y = sample_from_partials<FILT>(prow, a.partial + (rbase + at) * a.nch, a.nch, a.ch, a.V, s_rs, u,
+                                   red, fp);
   }
   verify_finish(a, req, slot, pos0, at, y);
+}
+
+
+// ---------------------------------------------------------------------------
+// Nucleus threshold of a row (top-p), one CTA per row.
+//
+// The masses are weights w_v = exp(l_v - max) as fixed-point integers
+// (2^40 units, rounded): integer sums are exact whatever their order, so the
+// result does not depend on scheduling.  A radix select over the 32-bit keys,
+// eight bits per pass from the most significant, finds the key kappa of the
+// token whose cumulative mass (most probable first) first reaches
+// T = top_p * (total mass): each pass builds a mass histogram of the keys
+// that share the prefix found so far (one histogram per warp, then added per
+// bin), and one warp scans the bins from the highest.  Tokens with a key
+// above kappa are kept; of the tokens whose logit is exactly kappa's, the
+// first j by token id are kept, j the least count that reaches T.
+// ---------------------------------------------------------------------------
+constexpr int NUC_THREADS = 1024;
+constexpr int NUC_WARPS = NUC_THREADS / 32;
+constexpr int NUC_SMEM = NUC_WARPS * 256 * 8;          // per-warp histograms
+constexpr float NUC_SCALE = 1099511627776.0f;           // 2^40
+
+struct TopPArgs {
+  const float* logits; int V;            // V % 4 == 0
+  int rows_per_req;                      // rows filtered per request
+  int64_t logit_rows_per_req;
+  int draft_map;                         // 1: filtered row s is logit row (s == 0 ? 0 : s + 1)
+  float top_p;                           // in (0, 1)
+  RowFilter* out;                        // entry of each filtered logit row [n_req * logit_rows_per_req]
+};
+
+__device__ __forceinline__ unsigned long long nuc_weight(float l, float ML) {
+  return __float2ull_rn(exp_rel(l, ML) * NUC_SCALE);
+}
+
+__global__ void __launch_bounds__(NUC_THREADS) top_p_kernel(const TopPArgs a) {
+  extern __shared__ unsigned long long nuc_hist[];       // [NUC_WARPS][256]
+  __shared__ float s_red[NUC_WARPS];
+  __shared__ unsigned long long s_bin[256];
+  __shared__ uint32_t s_prefix;
+  __shared__ unsigned long long s_above, s_mass;
+  __shared__ double s_T;
+  __shared__ int s_need, s_ntied, s_cut;
+  __shared__ int s_cnt[NUC_WARPS];
+  pdl_trigger();
+  pdl_wait();
+  const int rid = blockIdx.x;
+  const int req = rid / a.rows_per_req, srow = rid % a.rows_per_req;
+  const int lrow = (a.draft_map && srow > 0) ? srow + 1 : srow;
+  const size_t orow = (size_t)req * a.logit_rows_per_req + lrow;
+  const float* row = a.logits + orow * a.V;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int n4 = a.V >> 2;
+
+  // the row max
+  float m = -INFINITY;
+  for (int j = tid; j < n4; j += NUC_THREADS) {
+    const float4 x = r4[j];
+    m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+  }
+  m = warp_max(m);
+  if (lane == 0) s_red[wid] = m;
+  __syncthreads();
+  float M = s_red[0];
+  for (int w = 1; w < NUC_WARPS; ++w) M = fmaxf(M, s_red[w]);
+  const float ML = M * SAMPLE_LOG2E;
+
+  unsigned long long* hist = nuc_hist + wid * 256;
+  uint32_t prefix = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = lane; b < 256; b += 32) hist[b] = 0ull;
+    __syncwarp();
+    for (int j = tid; j < n4; j += NUC_THREADS) {
+      const float4 x = r4[j];
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t k = logit_key(xs[e]);
+        if (pass == 0 || (k >> (shift + 8)) == prefix) {
+          const unsigned long long w = nuc_weight(xs[e], ML);
+          if (w) atomicAdd(&hist[(k >> shift) & 255u], w);
+        }
+      }
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += NUC_THREADS) {
+      unsigned long long t = 0;
+      for (int w = 0; w < NUC_WARPS; ++w) t += nuc_hist[w * 256 + b];
+      s_bin[b] = t;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      // lane l holds bins 255 - 8 l - e, e = 0..7: keys in descending order
+      unsigned long long bm[8], lsum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        bm[e] = s_bin[255 - 8 * lane - e];
+        lsum += bm[e];
+      }
+      unsigned long long incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (pass == 0) {
+        // T = top_p * total mass (every key is in range in the first pass)
+        const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) { s_T = (double)a.top_p * (double)tot; s_above = 0ull; }
+        __syncwarp();
+      }
+      const double T = s_T;
+      const unsigned long long above = s_above;
+      __syncwarp();
+      const unsigned hit = __ballot_sync(0xffffffffu, (double)(above + incl) >= T);
+      const int hl = hit ? __ffs(hit) - 1 : 31;
+      if (lane == hl) {
+        unsigned long long run = above + (incl - lsum);
+        int bsel = 255 - 8 * lane - 7;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if ((double)(run + bm[e]) >= T) { bsel = 255 - 8 * lane - e; break; }
+          run += bm[e];
+        }
+        s_prefix = (prefix << 8) | (uint32_t)bsel;
+        s_above = run;
+        s_mass = s_bin[bsel];
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+  }
+  // the tokens whose logit is kappa's: how many, and how many are needed
+  if (tid == 0) {
+    const unsigned long long wk = nuc_weight(key_logit(prefix), ML);
+    long long ntied = wk ? (long long)(s_mass / wk) : 1;
+    if (ntied < 1) ntied = 1;
+    long long need = wk ? (long long)ceil((s_T - (double)s_above) / (double)wk) : 1;
+    need = need < 1 ? 1 : (need > ntied ? ntied : need);
+    s_need = (int)need;
+    s_ntied = (int)ntied;
+    s_cut = a.V - 1;
+  }
+  __syncthreads();
+  if (s_need < s_ntied) {
+    // the need-th token (by id) with key kappa: thread-contiguous segments,
+    // a block scan of the per-thread counts
+    const int per = (a.V + NUC_THREADS - 1) / NUC_THREADS;
+    const int b0 = tid * per, b1 = min(a.V, b0 + per);
+    int cnt = 0;
+    for (int v = b0; v < b1; ++v) cnt += logit_key(row[v]) == prefix;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_cnt[wid] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < wid; ++w) base += s_cnt[w];
+    const int excl = base + incl - cnt;
+    const int need = s_need;
+    if (excl < need && excl + cnt >= need) {
+      int c = excl;
+      for (int v = b0; v < b1; ++v)
+        if (logit_key(row[v]) == prefix && ++c == need) { s_cut = v; break; }
+    }
+    __syncthreads();
+  }
+  if (tid == 0) a.out[orow] = RowFilter{prefix, s_cut};
 }
 
 }  // namespace uno

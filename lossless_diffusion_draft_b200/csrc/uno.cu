@@ -116,16 +116,38 @@ void klaunch(bool pdl, cudaStream_t st, dim3 grid, dim3 block, size_t smem,
 // request combines and decides (one launch more, HBM kept busy).
 constexpr long long VERIFY_SPLIT_CTAS = 4096;
 // Returns the number of kernels launched.
-int launch_verify(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req,
-                  long long split_ctas = VERIFY_SPLIT_CTAS) {
+template <bool FILT>
+int launch_verify_t(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req, long long split_ctas) {
   const dim3 grid(a.nch, n_req * a.rows_red);
   if ((long long)a.nch * n_req * a.rows_red <= split_ctas) {
-    klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_verify_kernel, a);
+    klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_verify_kernel<FILT>, a);
     return 1;
   }
-  klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_reduce_kernel, a);
-  klaunch(pdl, st, dim3(n_req), dim3(SAMPLE_THREADS), 0, spec_decide_kernel, a);
+  klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_reduce_kernel<FILT>, a);
+  klaunch(pdl, st, dim3(n_req), dim3(SAMPLE_THREADS), 0, spec_decide_kernel<FILT>, a);
   return 2;
+}
+// FILT: the p and q rows carry nucleus filters (a.filt_p, a.filt_q).
+int launch_verify(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req,
+                  long long split_ctas = VERIFY_SPLIT_CTAS, bool filt = false) {
+  return filt ? launch_verify_t<true>(pdl, st, a, n_req, split_ctas)
+              : launch_verify_t<false>(pdl, st, a, n_req, split_ctas);
+}
+void launch_resid(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req, bool filt) {
+  if (filt) klaunch(pdl, st, dim3(a.nch, n_req), dim3(SAMPLE_THREADS), 0, spec_resid_kernel<true>, a);
+  else klaunch(pdl, st, dim3(a.nch, n_req), dim3(SAMPLE_THREADS), 0, spec_resid_kernel<false>, a);
+}
+void launch_sample(bool pdl, cudaStream_t st, dim3 grid, const SampleArgs& a) {
+  if (a.filt) klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, sample_rows_kernel<true>, a);
+  else klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, sample_rows_kernel<false>, a);
+}
+// The nucleus threshold of n_req * a.rows_per_req rows (false: the kernel's
+// shared-memory size could not be set).
+bool launch_top_p(bool pdl, cudaStream_t st, const TopPArgs& a, int n_req) {
+  static bool attr[ATTR_DEVS] = {};
+  if (smem_attr_once(top_p_kernel, NUC_SMEM, attr) != cudaSuccess) return false;
+  klaunch(pdl, st, dim3(n_req * a.rows_per_req), dim3(NUC_THREADS), NUC_SMEM, top_p_kernel, a);
+  return true;
 }
 
 struct GemmEnv {
@@ -369,6 +391,9 @@ struct uno_ctx {
   int verify_split_ctas = 4096;   // spec_verify: split form above this many CTAs
   int32_t *row_pos = nullptr, *row_slot = nullptr;
   float* row_gate = nullptr;
+  int32_t *row_cslot = nullptr, *row_blk = nullptr;   // training form: per-row key ranges
+  int32_t* train_slots = nullptr;                     // [2 max_batch] slots of a training pass
+  RowKeys keys{};                                     // key ranges of the current pass
   // completion counters of the fused pass (GEMMs wait on the kernel before
   // them through these instead of pdl_wait), zeroed by each pass's first kernel
   unsigned* dep_ctr = nullptr;
@@ -390,6 +415,9 @@ struct uno_ctx {
   unsigned* row_counter = nullptr;                  // [max_batch * 2B]
   unsigned* req_counter = nullptr;                  // [max_batch]
   int32_t* at_ws = nullptr;                         // [max_batch]
+  float top_p = 1.f;                                // nucleus filter (1: off)
+  RowFilter* filt_d = nullptr;                      // [max_batch, B+1] nucleus of draft rows
+  RowFilter* filt_v = nullptr;                      // [max_batch, B]   nucleus of verify rows
   float* resid_part = nullptr;                      // [max_batch, nch]
   unsigned* resid_counter = nullptr;                // [max_batch]
 
@@ -573,6 +601,7 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   p.rows_per_req = rows_per_req;
   p.row_pos = c->row_pos;
   p.row_slot = c->row_slot;
+  p.keys = c->keys;
   const int G = s.n_heads / s.n_kv_heads;
   p.n_qtiles = ceil_div(rows_per_req, ATC_QROWS / G);
   const int groups = n_req * s.n_kv_heads * p.n_qtiles;
@@ -636,6 +665,7 @@ int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
   p.rows_per_req = rows_per_req;
   p.row_pos = c->row_pos;
   p.row_slot = c->row_slot;
+  p.keys = c->keys;
   const int G = s.n_heads / s.n_kv_heads;
   const int TQ = ATT_MAXQ / G;
   p.n_qtiles = ceil_div(rows_per_req, TQ);
@@ -671,7 +701,8 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   const int d = s.d_model, H = s.n_heads, Hkv = s.n_kv_heads, hd = s.head_dim, F = s.ffn_dim;
   const int r = c->r;
   const int qkv_ld = (H + 2 * Hkv) * hd;
-  const bool lora = (kind == PASS_DRAFT);
+  // the adapter is read by the passes with gated rows (draft, training form)
+  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN);
   cudaStream_t st = c->stream;
 
   RowArgs ra{};
@@ -696,6 +727,9 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   ra.x = c->x;
   ra.status = c->d_status;
   ra.prefill_pos0 = prefill_pos0;
+  ra.row_cslot = c->row_cslot;
+  ra.row_blk = c->row_blk;
+  c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
     klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<T>, ra);
@@ -846,7 +880,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   const int d = s.d_model, H = s.n_heads, Hkv = s.n_kv_heads, hd = s.head_dim, F = s.ffn_dim;
   const int r = c->r;
   const int qkv_n = (H + 2 * Hkv) * hd;
-  const bool lora = (kind == PASS_DRAFT) && r > 0;
+  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN) && r > 0;
   cudaStream_t st = c->stream;
   const bool pdl = c->genv.pdl;
 
@@ -884,6 +918,9 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   };
   ra.zero_ctr = csync ? c->dep_ctr : nullptr;
   ra.n_zero = c->n_dep_ctr;
+  ra.row_cslot = c->row_cslot;
+  ra.row_blk = c->row_blk;
+  c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
     klaunch(pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<bf16>, ra);
@@ -1169,6 +1206,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->row_pos, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_slot, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_gate, (size_t)M * 4) != cudaSuccess) return oom("rows");
+  if (dalloc(&c->row_cslot, (size_t)M * 4) != cudaSuccess) return oom("rows");
+  if (dalloc(&c->row_blk, (size_t)M * 4) != cudaSuccess) return oom("rows");
+  if (dalloc(&c->train_slots, (size_t)2 * max_batch * 4) != cudaSuccess) return oom("rows");
   c->n_dep_ctr = 4 * s.n_layers + 8;
   if (dalloc(&c->dep_ctr, (size_t)c->n_dep_ctr * 4) != cudaSuccess) return oom("counters");
   cudaMemset(c->dep_ctr, 0, (size_t)c->n_dep_ctr * 4);
@@ -1203,6 +1243,10 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->row_counter, rows_ws * 4) != cudaSuccess) return oom("counters");
   if (dalloc(&c->req_counter, (size_t)max_batch * 4) != cudaSuccess) return oom("counters");
   if (dalloc(&c->at_ws, (size_t)max_batch * 4) != cudaSuccess) return oom("verify ws");
+  if (dalloc(&c->filt_d, (size_t)max_batch * (B + 1) * sizeof(RowFilter)) != cudaSuccess) return oom("filters");
+  if (dalloc(&c->filt_v, (size_t)max_batch * B * sizeof(RowFilter)) != cudaSuccess) return oom("filters");
+  cudaMemset(c->filt_d, 0, (size_t)max_batch * (B + 1) * sizeof(RowFilter));
+  cudaMemset(c->filt_v, 0, (size_t)max_batch * B * sizeof(RowFilter));
   if (dalloc(&c->resid_part, (size_t)max_batch * c->nch * 4) != cudaSuccess) return oom("verify ws");
   if (dalloc(&c->resid_counter, (size_t)max_batch * 4) != cudaSuccess) return oom("counters");
   cudaMemset(c->row_counter, 0, rows_ws * 4);
@@ -1291,9 +1335,10 @@ int uno_destroy(uno_ctx* c) {
   cudaDeviceSynchronize();
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
                   c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
+                  c->row_cslot, c->row_blk, c->train_slots,
                   c->dep_ctr, c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
                   c->lse_ws, c->row_counter, c->req_counter, c->at_ws, c->resid_part,
-                  c->resid_counter, c->att_ws, c->att_counters,
+                  c->resid_counter, c->att_ws, c->att_counters, c->filt_d, c->filt_v,
                   c->d_status, c->genv.ws, c->genv.counters, c->genv.part, c->ss};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -1345,6 +1390,53 @@ int uno_prefill(uno_ctx* c, int n_req, const int32_t* prompts_dev, int prompt_st
     CK(cudaGetLastError());
   }
   return UNO_OK;
+}
+
+int uno_train_forward(uno_ctx* c, int n_seq, const int32_t* tokens_dev, int L, float* logits_dev) {
+  if (!c) return UNO_ERR_ARG;
+  c->err.clear();
+  if (n_seq < 1 || L < 1 || !tokens_dev || !logits_dev)
+    return fail(c, UNO_ERR_ARG, "bad train_forward arguments");
+  if ((long long)n_seq * 2 * L > c->M_max)
+    return fail(c, UNO_ERR_CAPACITY, "n_seq * 2L rows exceed the pass capacity");
+  if (L > c->max_ctx) return fail(c, UNO_ERR_ARG, "L exceeds max_ctx");
+  int free_slots = 0;
+  for (int u : c->slot_used) free_slots += !u;
+  const int ppr = c->kv.pages_per_req;
+  if (free_slots < 2 * n_seq || (int)c->free_pages.size() < 2 * n_seq * ppr)
+    return fail(c, UNO_ERR_CAPACITY, "no free request slots or KV pages for the training form");
+  // two slots per sequence: clean keys, noised keys (positions 0 .. L-1 each)
+  std::vector<int32_t> slots;
+  for (int i = 0; i < 2 * n_seq; ++i) {
+    int slot = 0;
+    while (c->slot_used[slot]) ++slot;
+    c->slot_used[slot] = 1;
+    for (int pi = 0; pi < ppr; ++pi) {
+      c->h_page_table[(size_t)slot * ppr + pi] = c->free_pages.back();
+      c->free_pages.pop_back();
+    }
+    slots.push_back(slot);
+  }
+  auto release = [&]() {
+    for (int slot : slots) {
+      for (int pi = 0; pi < ppr; ++pi) c->free_pages.push_back(c->h_page_table[(size_t)slot * ppr + pi]);
+      c->slot_used[slot] = 0;
+    }
+  };
+  for (int slot : slots) {
+    const cudaError_t e = cudaMemcpyAsync(c->d_page_table + (size_t)slot * ppr,
+                                          c->h_page_table.data() + (size_t)slot * ppr, ppr * 4,
+                                          cudaMemcpyHostToDevice, c->stream);
+    if (e != cudaSuccess) { release(); return fail(c, UNO_ERR_CUDA, cudaGetErrorString(e)); }
+  }
+  cudaError_t e = cudaMemcpyAsync(c->train_slots, slots.data(), slots.size() * 4,
+                                  cudaMemcpyHostToDevice, c->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);   // host staging above is local
+  if (e != cudaSuccess) { release(); return fail(c, UNO_ERR_CUDA, cudaGetErrorString(e)); }
+  const int rc = forward_any(c, PASS_TRAIN, n_seq, 2 * L, c->train_slots, tokens_dev, 0, 0, logits_dev);
+  // later work on the stream runs after this pass, so the slots can be reused
+  release();
+  return rc;
 }
 
 }  // extern "C"
@@ -1417,8 +1509,20 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
   const int B = c->B, V = c->s.vocab;
   int rc = forward_any(c, PASS_DRAFT, n_req, B + 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
+  const bool filt = c->top_p < 1.f;
+  auto nucleus = [&](const float* logits, int64_t logit_rows, int draft_map, RowFilter* out) -> int {
+    TopPArgs t{};
+    t.logits = logits; t.V = V; t.rows_per_req = B; t.logit_rows_per_req = logit_rows;
+    t.draft_map = draft_map; t.top_p = c->top_p; t.out = out;
+    Prof prof(c, UNO_K_SAMPLE, (double)n_req * B * V * 4);
+    return launch_top_p(c->genv.pdl, c->stream, t, n_req)
+               ? UNO_OK : fail(c, UNO_ERR_CUDA, "top-p kernel attributes");
+  };
+  // draft rows p_1 (row 0) and q_2..q_B (rows 2..B)
+  if (filt && (rc = nucleus(c->logits_d, B + 1, 1, c->filt_d))) return rc;
   {
     SampleArgs a{};
+    a.filt = filt ? c->filt_d : nullptr;
     a.logits = c->logits_d;
     a.V = V; a.nch = c->nch; a.ch = c->ch;
     a.rows_per_req = B;
@@ -1436,13 +1540,16 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.row_counter = c->row_counter;
     a.status = c->d_status;
     Prof prof(c, UNO_K_SAMPLE, (double)n_req * B * V * 4);
-    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), dim3(SAMPLE_THREADS), 0,
-            sample_rows_kernel, a);
+    launch_sample(c->genv.pdl, c->stream, dim3(c->nch, n_req * B), a);
   }
   rc = forward_any(c, PASS_VERIFY, n_req, B, req_ids_dev, nullptr, 0, 0, c->logits_v);
   if (rc) return rc;
+  // verify rows p_2..p_{B+1}
+  if (filt && (rc = nucleus(c->logits_v, B, 0, c->filt_v))) return rc;
   {
     VerifyArgs a{};
+    a.filt_p = filt ? c->filt_v : nullptr;
+    a.filt_q = filt ? c->filt_d : nullptr;
     a.p = c->logits_v;
     a.q = c->logits_d;
     a.V = V; a.nch = c->nch; a.ch = c->ch;
@@ -1476,12 +1583,12 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
     a.fixed_at = c->fixed_accept > 0 ? c->fixed_accept - 1 : -1;
     {
       Prof prof(c, UNO_K_VERIFY, (double)n_req * B * V * 4);
-      c->prof_launches[UNO_K_VERIFY] += launch_verify(c->genv.pdl, c->stream, a, n_req, c->verify_split_ctas) - 1;
+      c->prof_launches[UNO_K_VERIFY] +=
+          launch_verify(c->genv.pdl, c->stream, a, n_req, c->verify_split_ctas, filt) - 1;
     }
     {
       Prof prof(c, UNO_K_VERIFY, (double)n_req * 2 * V * 4);
-      klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req), dim3(SAMPLE_THREADS), 0,
-              spec_resid_kernel, a);
+      launch_resid(c->genv.pdl, c->stream, a, n_req, filt);
     }
   }
   CK(cudaGetLastError());
@@ -1491,7 +1598,17 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
 int ar_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
   int rc = forward_any(c, PASS_AR, n_req, 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
+  const bool filt = c->top_p < 1.f;
+  if (filt) {
+    TopPArgs t{};
+    t.logits = c->logits_d; t.V = c->s.vocab; t.rows_per_req = 1; t.logit_rows_per_req = 1;
+    t.draft_map = 0; t.top_p = c->top_p; t.out = c->filt_d;
+    Prof prof(c, UNO_K_SAMPLE, (double)n_req * c->s.vocab * 4);
+    if (!launch_top_p(c->genv.pdl, c->stream, t, n_req))
+      return fail(c, UNO_ERR_CUDA, "top-p kernel attributes");
+  }
   SampleArgs a{};
+  a.filt = filt ? c->filt_d : nullptr;
   a.logits = c->logits_d;
   a.V = c->s.vocab; a.nch = c->nch; a.ch = c->ch;
   a.rows_per_req = 1;
@@ -1509,8 +1626,7 @@ int ar_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out
   a.status = c->d_status;
   {
     Prof prof(c, UNO_K_SAMPLE, (double)n_req * a.V * 4);
-    klaunch(c->genv.pdl, c->stream, dim3(c->nch, n_req), dim3(SAMPLE_THREADS), 0,
-            sample_rows_kernel, a);
+    launch_sample(c->genv.pdl, c->stream, dim3(c->nch, n_req), a);
   }
   CK(cudaGetLastError());
   return UNO_OK;
@@ -1570,6 +1686,14 @@ int uno_debug_set_dep_wait(uno_ctx* c, uint64_t limit_ns, uint32_t extra) {
   if (!c || limit_ns == 0) return UNO_ERR_ARG;
   c->dep_limit_ns = limit_ns;
   c->dep_extra = extra;
+  drop_graphs(c);
+  return UNO_OK;
+}
+
+int uno_set_top_p(uno_ctx* c, float top_p) {
+  if (!c) return UNO_ERR_ARG;
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(c, UNO_ERR_ARG, "top_p must be in (0, 1]");
+  c->top_p = top_p;
   drop_graphs(c);
   return UNO_OK;
 }
@@ -1692,6 +1816,8 @@ int uno_debug_read(uno_ctx* c, int which, void* dst, size_t bytes) {
     case UNO_DBG_LOGITS_VERIFY: src = c->logits_v; cap = mb * B * V * 4; break;
     case UNO_DBG_DRAFTS: src = c->drafts; cap = mb * B * 4; break;
     case UNO_DBG_LOGITS_AR: src = c->logits_d; cap = mb * V * 4; break;
+    case UNO_DBG_TOPP_DRAFT: src = c->filt_d; cap = mb * (B + 1) * sizeof(RowFilter); break;
+    case UNO_DBG_TOPP_VERIFY: src = c->filt_v; cap = mb * B * sizeof(RowFilter); break;
     default: return fail(c, UNO_ERR_ARG, "unknown debug buffer");
   }
   if (bytes > cap) return fail(c, UNO_ERR_ARG, "debug read larger than the buffer");
@@ -1799,6 +1925,21 @@ int uno_gated_lora_linear(int dtype, const void* X, const void* W, const void* A
 }
 
 // ---------------------------------------------------------------------------
+// Stand-alone nucleus threshold.
+// ---------------------------------------------------------------------------
+int uno_top_p_filter(const float* logits, int rows, int vocab, float top_p, int32_t* out,
+                     uno_stream_t stream) {
+  if (!logits || !out || rows < 1 || rows > (1 << 30) || vocab < 4 || vocab % 4 ||
+      ((uintptr_t)logits & 15) || !(top_p > 0.f && top_p < 1.f))
+    return UNO_ERR_ARG;
+  TopPArgs t{};
+  t.logits = logits; t.V = vocab; t.rows_per_req = 1; t.logit_rows_per_req = 1;
+  t.draft_map = 0; t.top_p = top_p; t.out = reinterpret_cast<RowFilter*>(out);
+  if (!launch_top_p(false, (cudaStream_t)stream, t, rows)) return UNO_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // Stand-alone spec_verify.
 // ---------------------------------------------------------------------------
 
@@ -1877,7 +2018,7 @@ int uno_spec_verify(const float* p, const float* q, const int32_t* drafts, int n
   a.status = nullptr;
   a.fixed_at = -1;
   launch_verify(false, (cudaStream_t)stream, a, n_req);
-  spec_resid_kernel<<<dim3(nch, n_req), SAMPLE_THREADS, 0, (cudaStream_t)stream>>>(a);
+  launch_resid(false, (cudaStream_t)stream, a, n_req, false);
   return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 

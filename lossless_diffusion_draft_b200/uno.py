@@ -19,7 +19,8 @@ HEADER = os.path.join(ROOT, "include", "uno.h")
 UNO_F32, UNO_BF16 = 0, 1
 UNO_OK, UNO_ERR_ARG, UNO_ERR_OOM, UNO_ERR_CAPACITY, UNO_ERR_CUDA, UNO_ERR_DEVICE_CHECK, \
     UNO_ERR_UNSUPPORTED = range(7)
-UNO_DBG_LOGITS_DRAFT, UNO_DBG_LOGITS_VERIFY, UNO_DBG_DRAFTS, UNO_DBG_LOGITS_AR = range(4)
+UNO_DBG_LOGITS_DRAFT, UNO_DBG_LOGITS_VERIFY, UNO_DBG_DRAFTS, UNO_DBG_LOGITS_AR, \
+    UNO_DBG_TOPP_DRAFT, UNO_DBG_TOPP_VERIFY = range(6)
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 N_PROJ = len(PROJ)
 
@@ -69,6 +70,7 @@ def load_library(path=LIB_PATH):
                            i32, u64, vp, ctypes.POINTER(vp)]),
         "uno_prefill": (i32, [vp, i32, vp, i32, vp, vp, vp]),
         "uno_spec_step": (i32, [vp, i32, vp, vp, vp]),
+        "uno_train_forward": (i32, [vp, i32, vp, i32, vp]),
         "uno_ar_step": (i32, [vp, i32, vp, vp]),
         "uno_release": (i32, [vp, i32]),
         "uno_destroy": (i32, [vp]),
@@ -87,6 +89,8 @@ def load_library(path=LIB_PATH):
         "uno_set_verify_split": (i32, [vp, i32]),
         "uno_set_counter_sync": (i32, [vp, i32]),
         "uno_debug_set_fixed_accept": (i32, [vp, i32]),
+        "uno_set_top_p": (i32, [vp, f32]),
+        "uno_top_p_filter": (i32, [vp, i32, i32, f32, vp, vp]),
         "uno_debug_set_dep_wait": (i32, [vp, u64, ctypes.c_uint32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
         "uno_profile_begin": (i32, [vp, ctypes.c_uint]),
@@ -206,6 +210,14 @@ def uno_prefill(ctx, prompts_dev, prompt_lens, streams=None):
     return list(ids)
 
 
+def uno_train_forward(ctx, tokens_dev, logits_dev):
+    """tokens_dev int32 CUDA [n_seq, 2L] (x then z) -> logits_dev f32 CUDA [n_seq, 2L, vocab]."""
+    n_seq, two_l = tokens_dev.shape
+    code = load_library().uno_train_forward(ctx.handle, n_seq, _ptr(tokens_dev), two_l // 2,
+                                            _ptr(logits_dev))
+    _check(code, ctx.handle)
+
+
 def uno_spec_step(ctx, req_ids_dev, out_tokens_dev, n_new_dev):
     code = load_library().uno_spec_step(ctx.handle, req_ids_dev.numel(), _ptr(req_ids_dev),
                                         _ptr(out_tokens_dev), _ptr(n_new_dev))
@@ -243,6 +255,18 @@ def uno_set_verify_split(ctx, max_ctas):
 def uno_set_counter_sync(ctx, enable):
     """Fused pipeline: GEMMs wait on completion counters (True) or grid dependencies."""
     _check(load_library().uno_set_counter_sync(ctx.handle, int(bool(enable))), ctx.handle)
+
+
+def uno_set_top_p(ctx, top_p):
+    """Nucleus filter of every sampled or verified row (1.0: off)."""
+    _check(load_library().uno_set_top_p(ctx.handle, float(top_p)), ctx.handle)
+
+
+def uno_top_p_filter(logits_dev, top_p, out_dev, stream=None):
+    """logits_dev f32 CUDA [rows, vocab] -> out_dev int32 CUDA [rows, 2] (key, id_cut)."""
+    rows, vocab = logits_dev.shape
+    _check(load_library().uno_top_p_filter(_ptr(logits_dev), rows, vocab, float(top_p),
+                                           _ptr(out_dev), _stream_ptr(stream)))
 
 
 def uno_debug_set_fixed_accept(ctx, a):
