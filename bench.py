@@ -487,9 +487,50 @@ def run_uno(args, rank, world, device):
     if extras:
         del wl
         torch.cuda.empty_cache()
+        res["cohorts"] = run_cohorts(args, cfg, params, rank, world, device)
         res["max_batch"] = run_max_batch(args, cfg, params, rank, world, device, pk)
         res["spec_verify_micro"] = spec_verify_micro(args, device, pk)
     return res
+
+
+def run_cohorts(args, cfg, params, rank, world, device, batch=16):
+    """Cohort-interleaved steps against plain steps on the same requests: 16
+    requests at the 1K-token context, as two cohorts of 8 (each call one
+    forward over 8 drafting and 8 verifying requests) and as plain steps of
+    16 (two forwards).  Device time by CUDA events over the same number of
+    forwards; tokens counted from the emitted counts."""
+    from lossless_diffusion_draft_b200 import uno
+    cfg = dict(cfg, batch=batch)
+    B, K = cfg["B"], max(4, args.steps // 2)
+    wl = Workload(cfg, params, batch, cfg["prompt_len"], rank, device, args)
+    plain = wl.time_steps(K, 3, world, clocks=False)
+    wl.prefill(cfg["prompt_len"])
+    half = batch // 2
+    a, b = wl.req[:half].clone(), wl.req[half:].clone()
+    out = torch.zeros((half, B + 1), dtype=torch.int32, device=device)
+    n_new = torch.zeros((2 * K + 8, half), dtype=torch.int32, device=device)
+    uno.uno_spec_step_cohorts(wl.ctx, a, None, out, n_new[0])
+    for k in range(4):                                   # warm-up (and graph capture)
+        d, v = (b, a) if k % 2 == 0 else (a, b)
+        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new[0])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(2 * K):                               # 2K forwards, as K plain steps
+        d, v = (b, a) if k % 2 == 0 else (a, b)
+        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new[1 + k])
+    e1.record()
+    torch.cuda.synchronize()
+    uno.uno_status(wl.ctx)
+    ms = e0.elapsed_time(e1)
+    tokens = int(n_new[1:1 + 2 * K].sum().item())
+    wl.close()
+    return {"batch": batch, "context": cfg["prompt_len"], "forwards": 2 * K,
+            "plain": {"tokens_per_s": rate(plain), "ms_per_forward": plain["ms"] / plain["K"] / 2},
+            "cohorts": {"tokens_per_s": tokens / (ms / 1e3), "ms_per_forward": ms / (2 * K)},
+            "note": "two cohorts of 8 out of phase (one forward per call) against plain steps of 16 "
+                    "(two forwards per step); per request both do one draft and one verify "
+                    "forward per iteration"}
 
 
 def run_max_batch(args, cfg, params, rank, world, device, pk):
@@ -859,6 +900,8 @@ def main():
             "tokens_per_step": fa["tokens"] / fa["K"], "tpf": fa["tokens"] / fa["K"] / batch / 2,
             "note": "measured with the uno_debug_set_fixed_accept tap forcing a = 4 accepted "
                     "tokens (TPF 2.5, the pages' trained-adapter range); not a parity run"}
+    if "cohorts" in res:
+        line["cohorts"] = res["cohorts"]
     if "max_batch" in res:
         line["max_batch"] = res["max_batch"]
     if "spec_verify_micro" in res:

@@ -158,6 +158,33 @@ int uno_train_forward(uno_ctx *ctx, int n_seq, const int32_t *tokens_dev, int L,
 int uno_spec_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *out_tokens_dev,
                   int32_t *n_new_dev);
 
+/*
+ * Cohort-interleaved Psi-Spec steps (the gated LoRA lets one forward compute
+ * both paths - blog page "…Uno 的无损加速之路", section Diffusion Distillation：
+ * 一步蒸馏 + 块级扩散 - so two request cohorts can run out of phase and share
+ * each weight tile of a forward).  One call runs ONE forward over
+ *   the drafting cohort  (draft_ids_dev, int32 [n_draft] slots): its draft
+ *                        rows [pending, MASK x B], then draft_sample; the
+ *                        block and the draft logits stay with the request;
+ *   the verifying cohort (verify_ids_dev, int32 [n_verify] slots, drafted by
+ *                        an earlier call): its verify rows x_1..x_B (plus x_B
+ *                        once more, so every request has B + 1 rows), then
+ *                        spec_verify and the commit, which emit into
+ *                        out_tokens_dev int32 [n_verify, B+1] and
+ *                        n_new_dev int32 [n_verify].
+ * A request alternates: drafted by one call, verified by a later one (any
+ * number of calls in between, no uno_spec_step on it meanwhile).  Each
+ * request's tokens are exactly those of uno_spec_step (same uniforms, keyed
+ * by request and position).  Either cohort may be empty (not both); slots
+ * must be distinct; a request in the wrong phase raises the device flag.
+ * The first call allocates the per-slot buffers (once, before any stream
+ * capture; 2 * max_batch * (B+1) * vocab fp32 logits).  top_p < 1:
+ * UNO_ERR_UNSUPPORTED.  Graph capture as for uno_spec_step (keyed by all
+ * four pointers and both counts).
+ */
+int uno_spec_step_cohorts(uno_ctx *ctx, int n_draft, const int32_t *draft_ids_dev, int n_verify,
+                          const int32_t *verify_ids_dev, int32_t *out_tokens_dev, int32_t *n_new_dev);
+
 /* AR-only decode (baseline): one forward, the LoRA off, one token per request
  * into out_tokens_dev int32 [n_req]. */
 int uno_ar_step(uno_ctx *ctx, int n_req, const int32_t *req_ids_dev, int32_t *out_tokens_dev);
@@ -292,13 +319,18 @@ int uno_request_state(uno_ctx *ctx, int req_id, int32_t *cached_out, int32_t *pe
  *   UNO_DBG_TOPP_DRAFT    int32 [n_req, B+1, 2]     nucleus of each draft row (top_p < 1;
  *                                                   row 1 unused; AR step: [n_req, 1, 2])
  *   UNO_DBG_TOPP_VERIFY   int32 [n_req, B, 2]       nucleus of each verify row
+ *   UNO_DBG_COHORT_LOGITS f32   [2 max_batch, B+1, vocab]  cohort step: the draft logits
+ *                               of each slot (rows [slot]), then the last call's
+ *                               verify logits (rows [max_batch + i], i-th verified)
+ *   UNO_DBG_COHORT_DRAFTS int32 [max_batch, B]      cohort step: drafted block per slot
  * A nucleus entry is (key, id_cut) as uno_top_p_filter writes it.  The
  * logits are those of the model (before any nucleus filter).
  * bytes must not exceed the buffer's size for max_batch requests.
  */
 enum uno_debug_buf {
   UNO_DBG_LOGITS_DRAFT = 0, UNO_DBG_LOGITS_VERIFY = 1, UNO_DBG_DRAFTS = 2, UNO_DBG_LOGITS_AR = 3,
-  UNO_DBG_TOPP_DRAFT = 4, UNO_DBG_TOPP_VERIFY = 5
+  UNO_DBG_TOPP_DRAFT = 4, UNO_DBG_TOPP_VERIFY = 5, UNO_DBG_COHORT_LOGITS = 6,
+  UNO_DBG_COHORT_DRAFTS = 7
 };
 int uno_debug_read(uno_ctx *ctx, int which, void *dst_host, size_t bytes);
 

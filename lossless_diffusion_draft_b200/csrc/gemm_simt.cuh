@@ -45,6 +45,8 @@ struct GemmParams {
   // and its CTA count (null: the launch waits with pdl_wait)
   const unsigned* dep; unsigned dep_count;
   unsigned long long dep_limit_ns;   // the counter wait gives up after this long
+  // EPI_STORE_F32: element offset of each output row (null: row * ldo)
+  const int64_t* out_row;
 };
 
 template <typename T, int MT, int NC>
@@ -143,7 +145,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmParams p) {
           reinterpret_cast<T*>(p.out)[(size_t)row * p.ldo + n] = from_f<T>(v * p.alpha);
           break;
         case EPI_STORE_F32:
-          reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + n] = v * p.alpha;
+          reinterpret_cast<float*>(p.out)[(p.out_row ? (size_t)p.out_row[row] : (size_t)row * p.ldo) + n] =
+              v * p.alpha;
           break;
         case EPI_ADD_F32:
           reinterpret_cast<float*>(p.out)[(size_t)row * p.ldo + n] += v;

@@ -72,6 +72,7 @@ struct TcParams {
   // DUMP mode only, where X is the one input an earlier kernel wrote
   const unsigned* dep; unsigned dep_count;
   unsigned long long dep_limit_ns;   // give up the counter wait after this long
+  const int64_t* out_row;            // EPI_STORE_F32: element offset of each output row (null: m * ldo)
 };
 
 // ---------------------------------------------------------------------------
@@ -119,7 +120,9 @@ __device__ __forceinline__ void tc_store(const TcParams& p, int m, int n, float 
   const size_t o = (size_t)m * p.ldo + n;
   switch (p.epi) {
     case EPI_STORE: reinterpret_cast<bf16*>(p.out)[o] = from_f<bf16>(v * p.alpha); break;
-    case EPI_STORE_F32: reinterpret_cast<float*>(p.out)[o] = v * p.alpha; break;
+    case EPI_STORE_F32:
+      reinterpret_cast<float*>(p.out)[p.out_row ? (size_t)p.out_row[m] + n : o] = v * p.alpha;
+      break;
     case EPI_ADD_F32: reinterpret_cast<float*>(p.out)[o] += v; break;
     default: {
       const float y = v * p.alpha * p.row_gate[m];

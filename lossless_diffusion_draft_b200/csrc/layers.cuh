@@ -48,7 +48,8 @@ struct KvLayout {
 };
 
 // Pass kinds (a pass is one forward over a set of rows).
-enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3, PASS_TRAIN = 4 };
+enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3, PASS_TRAIN = 4,
+                      PASS_COHORT = 5 };
 
 // The keys each query row sees, by the block-causal rule (blog page "…Uno
 // 的无损加速之路", section Diffusion Distillation：一步蒸馏 + 块级扩散: a clean
@@ -131,6 +132,14 @@ struct RowArgs {
   unsigned* zero_ctr; int n_zero;   // the pass's completion counters (zeroed here), or null
   // training form: per-row key ranges (RowKeys) written here
   int32_t* row_cslot; int32_t* row_blk;
+  // cohort pass: the first n_draft requests run their draft rows, the others
+  // their verify rows (the B drafted tokens and the last one again, so that
+  // every request has B + 1 rows); drafts are kept per slot between calls
+  int n_draft;
+  const int32_t* phase;        // [max_batch] 0: to be drafted, 1: drafted (checked)
+  const int32_t* coh_drafts;   // [max_batch, B]
+  int64_t* row_off;            // [M] element offset of each row's logits
+  int64_t coh_v_row0;          // logits row of the verify cohort's first row
 };
 
 // a1: build the rows of a pass and gather their embeddings.
@@ -175,13 +184,28 @@ __global__ void build_rows_kernel(const RowArgs a) {
     slot = a.req_slot[req];
     if (slot < 0 || slot >= a.max_batch) { raise_status(a.status, ST_BAD_SLOT); slot = 0; }
     const int c = a.cached[slot];
-    if (a.kind == PASS_DRAFT) {            // [pending, MASK x B] at c..c+B
+    int kind = a.kind;
+    if (kind == PASS_COHORT) {
+      const bool draft = req < a.n_draft;
+      if (a.phase[slot] != (draft ? 0 : 1)) raise_status(a.status, ST_BAD_SLOT);
+      if (threadIdx.x == 0)
+        a.row_off[row] = (draft ? (int64_t)slot * (a.B + 1) + j
+                                : a.coh_v_row0 + (int64_t)(req - a.n_draft) * (a.B + 1) + j) * a.vocab;
+      kind = draft ? PASS_DRAFT : PASS_VERIFY;
+    }
+    if (kind == PASS_DRAFT) {              // [pending, MASK x B] at c..c+B
       tok = (j == 0) ? a.pending[slot] : a.mask_id;
       pos = c + j;
       gate = (j == 0) ? 0.f : a.lora_scale;
-    } else if (a.kind == PASS_VERIFY) {    // x_1..x_B at c+1..c+B
-      tok = a.drafts[(size_t)req * a.B + j];
-      pos = c + 1 + j;
+    } else if (kind == PASS_VERIFY) {      // x_1..x_B at c+1..c+B
+      if (a.kind == PASS_COHORT) {         // per-slot drafts; row B repeats row B-1
+        const int jj = j < a.B ? j : a.B - 1;
+        tok = a.coh_drafts[(size_t)slot * a.B + jj];
+        pos = c + 1 + jj;
+      } else {
+        tok = a.drafts[(size_t)req * a.B + j];
+        pos = c + 1 + j;
+      }
     } else {                               // AR: pending at c
       tok = a.pending[slot];
       pos = c;

@@ -349,6 +349,10 @@ struct SampleArgs {
   unsigned* row_counter;      // [n_req * rows_per_req], zero on entry, left zero
   int32_t* status;
   const RowFilter* filt;      // nucleus of each logit row [n_req * logit_rows_per_req] (FILT)
+  // per_slot: logits, drafts, lse and filters are indexed by the request's
+  // slot instead of its position in the batch (the cohort step keeps them
+  // between calls), and phase[slot] is set to 1 (drafted)
+  int per_slot; int32_t* phase;
 };
 
 template <bool FILT>
@@ -361,8 +365,10 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   const int rid = blockIdx.y;
   const int req = rid / a.rows_per_req, s = rid % a.rows_per_req;
   const int lrow = (a.ar_mode || s == 0) ? 0 : s + 1;
-  const float* row = a.logits + ((size_t)req * a.logit_rows_per_req + lrow) * a.V;
-  const Filt<FILT> f = filt_of<FILT>(a.filt, (size_t)req * a.logit_rows_per_req + lrow);
+  const int slot = a.req_slot[req];
+  const int base = a.per_slot ? slot : req;
+  const float* row = a.logits + ((size_t)base * a.logit_rows_per_req + lrow) * a.V;
+  const Filt<FILT> f = filt_of<FILT>(a.filt, (size_t)base * a.logit_rows_per_req + lrow);
   const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
   const float2 pr = reduce_chunk<FILT>(row, c0, c1, red, f);
   if (threadIdx.x == 0) {
@@ -383,7 +389,6 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   }
   __syncthreads();
   const RowStat rs = s_rs;
-  const int slot = a.req_slot[req];
   const int c = a.cached[slot];
   const uint32_t kind = (a.ar_mode || s == 0) ? KIND_FIRST : KIND_DRAFT;
   const float u = philox_uniform(a.seed, a.slot_stream[slot], (uint32_t)(c + 1 + s), kind);
@@ -394,8 +399,9 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
       a.cached[slot] = c + 1;
       a.pending[slot] = t;
     } else {
-      a.out_tok[(size_t)req * a.out_stride + s] = t;
-      if (a.lse_out) a.lse_out[(size_t)req * a.rows_per_req + s] = rs.M + logf(rs.Z);
+      a.out_tok[(size_t)base * a.out_stride + s] = t;
+      if (a.lse_out) a.lse_out[(size_t)base * a.rows_per_req + s] = rs.M + logf(rs.Z);
+      if (a.phase && s == 0) a.phase[slot] = 1;
     }
   }
 }
@@ -436,7 +442,15 @@ struct VerifyArgs {
   int fixed_at;
   // nucleus of each p row [n_req * p_req_rows] and q row [n_req * q_req_rows] (FILT)
   const RowFilter* filt_p; const RowFilter* filt_q;
+  // per_slot (decode mode): q rows, drafts, their lse and filters are indexed
+  // by the request's slot (kept there by the cohort step's draft_sample), and
+  // phase[slot] is reset to 0 at the commit
+  int per_slot; int32_t* phase;
 };
+// Index of a request's draft-side data (q rows, drafts, lse of q).
+__device__ __forceinline__ int verify_qb(const VerifyArgs& a, int req) {
+  return a.per_slot ? a.req_slot[req] : req;
+}
 
 // Slot, position of test 0 and Philox stream of a request.
 __device__ __forceinline__ void verify_request_ctx(const VerifyArgs& a, int req, int* slot,
@@ -454,7 +468,7 @@ __device__ __forceinline__ void verify_request_ctx(const VerifyArgs& a, int req,
 
 // log-normaliser of the draft row of test j.
 __device__ __forceinline__ float verify_lse_q(const VerifyArgs& a, int req, int j) {
-  return a.lse_q_in ? a.lse_q_in[(size_t)req * a.lse_q_stride + a.lse_q_off + j]
+  return a.lse_q_in ? a.lse_q_in[(size_t)verify_qb(a, req) * a.lse_q_stride + a.lse_q_off + j]
                     : __ldcg(&a.lse[(size_t)req * a.rows_red + a.n_p + j]);
 }
 
@@ -464,18 +478,20 @@ __device__ void verify_finish(const VerifyArgs& a, int req, int slot, int pos0, 
   const bool decode = a.req_slot != nullptr;
   const int lead = decode ? 1 : 0;    // decode mode emits x_1 first
   int32_t* out = a.out_tok + (size_t)req * a.out_stride;
+  const int qb = verify_qb(a, req);
   for (int j = threadIdx.x; j < at; j += SAMPLE_THREADS)
-    out[lead + j] = a.drafts[(size_t)req * a.drafts_stride + a.drafts_off + j];
+    out[lead + j] = a.drafts[(size_t)qb * a.drafts_stride + a.drafts_off + j];
   if (threadIdx.x == 0) {
     if (decode) {
       // emitted: x_1, the accepted x_2..x_{1+at}, then y; the cache grows by
       // n tokens (positions c..c+n-1 hold keys/values) and y becomes pending
-      out[0] = a.first_tok[(size_t)req * a.drafts_stride];
+      out[0] = a.first_tok[(size_t)qb * a.drafts_stride];
       const int n = lead + at + 1;
       out[n - 1] = y;
       a.n_out[req] = n;
       a.cached[slot] = pos0 - 2 + n;
       a.pending[slot] = y;
+      if (a.phase) a.phase[slot] = 0;
     } else {
       out[at] = y;          // -1 when every test passed and no bonus row exists
       a.n_out[req] = at;
@@ -492,7 +508,7 @@ __device__ __forceinline__ Filt<FILT> verify_filt_p(const VerifyArgs& a, int req
 }
 template <bool FILT>
 __device__ __forceinline__ Filt<FILT> verify_filt_q(const VerifyArgs& a, int req, int qrow_idx) {
-  return filt_of<FILT>(a.filt_q, (size_t)req * a.q_req_rows + qrow_idx);
+  return filt_of<FILT>(a.filt_q, (size_t)verify_qb(a, req) * a.q_req_rows + qrow_idx);
 }
 
 template <bool FILT>
@@ -504,11 +520,12 @@ __device__ void verify_decide(const VerifyArgs& a, int req, float* red) {
   verify_request_ctx(a, req, &slot, &pos0, &stream);
   if (threadIdx.x == 0) s_a = a.n_tests;
   __syncthreads();
+  const int qb = verify_qb(a, req);
   for (int j = threadIdx.x; j < a.n_tests; j += SAMPLE_THREADS) {
-    int t = a.drafts[(size_t)req * a.drafts_stride + a.drafts_off + j];
+    int t = a.drafts[(size_t)qb * a.drafts_stride + a.drafts_off + j];
     if (t < 0 || t >= a.V) { raise_status(a.status, ST_BAD_TOKEN); t = 0; }
     const float* prow = a.p + ((size_t)req * a.p_req_rows + a.p_row0 + j) * a.V;
-    const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + j) * a.V;
+    const float* qrow = a.q + ((size_t)qb * a.q_req_rows + a.q_row0 + j) * a.V;
     const float lse_p = __ldcg(&a.lse[rbase + j]);
     const float lse_q = verify_lse_q(a, req, j);
     const float u = philox_uniform(a.seed, stream, (uint32_t)(pos0 + j), KIND_ACCEPT);
@@ -547,7 +564,7 @@ __device__ __forceinline__ const float* verify_row(const VerifyArgs& a, int req,
     const int br = (r < a.n_tests) ? a.p_row0 + r : a.bonus_row;
     return a.p + ((size_t)req * a.p_req_rows + br) * a.V;
   }
-  return a.q + ((size_t)req * a.q_req_rows + a.q_row0 + (r - a.n_p)) * a.V;
+  return a.q + ((size_t)verify_qb(a, req) * a.q_req_rows + a.q_row0 + (r - a.n_p)) * a.V;
 }
 
 // The nucleus of the row a (request, reduced row) CTA reads.
@@ -654,7 +671,7 @@ __global__ void __launch_bounds__(SAMPLE_THREADS) spec_resid_kernel(const Verify
   if (at < 0) return;
   const size_t rbase = (size_t)req * a.rows_red;
   const float* prow = a.p + ((size_t)req * a.p_req_rows + a.p_row0 + at) * a.V;
-  const float* qrow = a.q + ((size_t)req * a.q_req_rows + a.q_row0 + at) * a.V;
+  const float* qrow = a.q + ((size_t)verify_qb(a, req) * a.q_req_rows + a.q_row0 + at) * a.V;
   const float lse_p = __ldcg(&a.lse[rbase + at]);
   const float lse_q = verify_lse_q(a, req, at);
   const Filt<FILT> fp = verify_filt_p<FILT>(a, req, a.p_row0 + at);

@@ -275,6 +275,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.dep = DUMP ? p.dep : nullptr;
   tp.dep_count = p.dep_count;
   tp.dep_limit_ns = p.dep_limit_ns ? p.dep_limit_ns : DEP_WAIT_NS;
+  tp.out_row = p.out_row;
 
   using Cfg = TcCfg<NT, SPLIT, KPS>;
   static bool attr[ATTR_DEVS] = {};
@@ -393,6 +394,14 @@ struct uno_ctx {
   float* row_gate = nullptr;
   int32_t *row_cslot = nullptr, *row_blk = nullptr;   // training form: per-row key ranges
   int32_t* train_slots = nullptr;                     // [2 max_batch] slots of a training pass
+  // cohort step (allocated by its first call)
+  float* coh_logits = nullptr;     // [2 max_batch (B+1), V]: per-slot draft rows, then verify rows
+  int32_t* coh_drafts = nullptr;   // [max_batch, B] drafted block per slot
+  float* coh_lse_q = nullptr;      // [max_batch, B]
+  int32_t* coh_phase = nullptr;    // [max_batch] 0: to be drafted, 1: drafted
+  int32_t* coh_rows = nullptr;     // [max_batch] slots of the pass: drafting cohort, then verifying
+  int64_t* coh_rowoff = nullptr;   // [M_max] logits offset of each row
+  int coh_n_draft = 0;
   RowKeys keys{};                                     // key ranges of the current pass
   // completion counters of the fused pass (GEMMs wait on the kernel before
   // them through these instead of pdl_wait), zeroed by each pass's first kernel
@@ -438,7 +447,7 @@ struct uno_ctx {
   // CUDA graphs of whole steps, keyed by their arguments
   struct GraphEntry {
     int kind, n_req;
-    const void *a, *b, *c;
+    const void *a, *b, *c, *d;
     int seen = 0;
     cudaGraphExec_t exec = nullptr;
     int64_t launches[UNO_K_N] = {};
@@ -702,7 +711,7 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   const int r = c->r;
   const int qkv_ld = (H + 2 * Hkv) * hd;
   // the adapter is read by the passes with gated rows (draft, training form)
-  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN);
+  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN || kind == PASS_COHORT);
   cudaStream_t st = c->stream;
 
   RowArgs ra{};
@@ -729,6 +738,11 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   ra.prefill_pos0 = prefill_pos0;
   ra.row_cslot = c->row_cslot;
   ra.row_blk = c->row_blk;
+  ra.n_draft = c->coh_n_draft;
+  ra.phase = c->coh_phase;
+  ra.coh_drafts = c->coh_drafts;
+  ra.row_off = c->coh_rowoff;
+  ra.coh_v_row0 = (int64_t)c->max_batch * (c->B + 1);
   c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
@@ -853,6 +867,7 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
     Gemm g(c->xn, xn_ld, M, d);
     g.seg(c->lm_head, s.vocab).epi(EPI_STORE_F32, logits, s.vocab, 1.0f / s.temperature);
     g.p.lo_off = lo;
+    g.p.out_row = kind == PASS_COHORT ? c->coh_rowoff : nullptr;
     launch_gemm<T>(c, g, st);
   }
   CK(cudaGetLastError());
@@ -880,7 +895,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   const int d = s.d_model, H = s.n_heads, Hkv = s.n_kv_heads, hd = s.head_dim, F = s.ffn_dim;
   const int r = c->r;
   const int qkv_n = (H + 2 * Hkv) * hd;
-  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN) && r > 0;
+  const bool lora = (kind == PASS_DRAFT || kind == PASS_TRAIN || kind == PASS_COHORT) && r > 0;
   cudaStream_t st = c->stream;
   const bool pdl = c->genv.pdl;
 
@@ -920,6 +935,11 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ra.n_zero = c->n_dep_ctr;
   ra.row_cslot = c->row_cslot;
   ra.row_blk = c->row_blk;
+  ra.n_draft = c->coh_n_draft;
+  ra.phase = c->coh_phase;
+  ra.coh_drafts = c->coh_drafts;
+  ra.row_off = c->coh_rowoff;
+  ra.coh_v_row0 = (int64_t)c->max_batch * (c->B + 1);
   c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
@@ -1066,6 +1086,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     Gemm g(c->xn, xn_ld, M, d);
     g.seg(c->lm_head, s.vocab).epi(EPI_STORE_F32, logits, s.vocab, 1.0f / s.temperature);
     g.p.lo_off = lo;
+    g.p.out_row = kind == PASS_COHORT ? c->coh_rowoff : nullptr;
     launch_gemm<bf16>(c, g, st);
   }
   CK(cudaGetLastError());
@@ -1335,7 +1356,8 @@ int uno_destroy(uno_ctx* c) {
   cudaDeviceSynchronize();
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
                   c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
-                  c->row_cslot, c->row_blk, c->train_slots,
+                  c->row_cslot, c->row_blk, c->train_slots, c->coh_logits, c->coh_drafts,
+                  c->coh_lse_q, c->coh_phase, c->coh_rows, c->coh_rowoff,
                   c->dep_ctr, c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
                   c->lse_ws, c->row_counter, c->req_counter, c->at_ws, c->resid_part,
                   c->resid_counter, c->att_ws, c->att_counters, c->filt_d, c->filt_v,
@@ -1388,6 +1410,8 @@ int uno_prefill(uno_ctx* c, int n_req, const int32_t* prompts_dev, int prompt_st
     }
     init_slot_kernel<<<1, 1, 0, c->stream>>>(prompt, P, slot, c->d_cached, c->d_pending);
     CK(cudaGetLastError());
+    // a new request starts undrafted for the cohort step
+    if (c->coh_phase) CK(cudaMemsetAsync(c->coh_phase + slot, 0, 4, c->stream));
   }
   return UNO_OK;
 }
@@ -1449,15 +1473,15 @@ namespace {
 // runs eagerly (its event pairs are host-side bookkeeping).
 template <typename F>
 int run_graphed(uno_ctx* c, int kind, int n_req, const void* a, const void* b, const void* d,
-                F&& body) {
+                F&& body, const void* d2 = nullptr) {
   if (!c->graphs_enabled || c->prof_mask) return body();
   uno_ctx::GraphEntry* e = nullptr;
   for (auto& g : c->graphs)
-    if (g.kind == kind && g.n_req == n_req && g.a == a && g.b == b && g.c == d) e = &g;
+    if (g.kind == kind && g.n_req == n_req && g.a == a && g.b == b && g.c == d && g.d == d2) e = &g;
   if (!e) {
     c->graphs.emplace_back();
     e = &c->graphs.back();
-    e->kind = kind; e->n_req = n_req; e->a = a; e->b = b; e->c = d;
+    e->kind = kind; e->n_req = n_req; e->a = a; e->b = b; e->c = d; e->d = d2;
   }
   if (e->exec) {
     CK(cudaGraphLaunch(e->exec, c->stream));
@@ -1595,6 +1619,93 @@ int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* o
   return UNO_OK;
 }
 
+// One forward over the drafting cohort's draft rows and the verifying
+// cohort's verify rows, then draft_sample of the first and spec_verify +
+// commit of the second (per-slot state in between).
+int cohort_step_body(uno_ctx* c, int n_draft, const int32_t* draft_ids, int n_verify,
+                     const int32_t* verify_ids, int32_t* out_tokens, int32_t* n_new) {
+  const int B = c->B, V = c->s.vocab;
+  const int n = n_draft + n_verify;
+  if (n_draft)
+    CK(cudaMemcpyAsync(c->coh_rows, draft_ids, (size_t)n_draft * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if (n_verify)
+    CK(cudaMemcpyAsync(c->coh_rows + n_draft, verify_ids, (size_t)n_verify * 4, cudaMemcpyDeviceToDevice,
+                       c->stream));
+  c->coh_n_draft = n_draft;
+  int rc = forward_any(c, PASS_COHORT, n, B + 1, c->coh_rows, nullptr, 0, 0, c->coh_logits);
+  if (rc) return rc;
+  if (n_draft) {
+    SampleArgs a{};
+    a.logits = c->coh_logits;
+    a.V = V; a.nch = c->nch; a.ch = c->ch;
+    a.rows_per_req = B;
+    a.logit_rows_per_req = B + 1;
+    a.ar_mode = 0;
+    a.req_slot = c->coh_rows;
+    a.cached = c->d_cached;
+    a.pending = c->d_pending;
+    a.slot_stream = c->d_stream;
+    a.seed = c->seed;
+    a.out_tok = c->coh_drafts;
+    a.out_stride = B;
+    a.lse_out = c->coh_lse_q;
+    a.partial = c->partial;
+    a.row_counter = c->row_counter;
+    a.status = c->d_status;
+    a.per_slot = 1;
+    a.phase = c->coh_phase;
+    Prof prof(c, UNO_K_SAMPLE, (double)n_draft * B * V * 4);
+    launch_sample(c->genv.pdl, c->stream, dim3(c->nch, n_draft * B), a);
+  }
+  if (n_verify) {
+    VerifyArgs a{};
+    a.p = c->coh_logits + (size_t)c->max_batch * (B + 1) * V;
+    a.q = c->coh_logits;
+    a.V = V; a.nch = c->nch; a.ch = c->ch;
+    a.n_tests = B - 1;
+    a.p_req_rows = B + 1;
+    a.q_req_rows = B + 1;
+    a.p_row0 = 0;
+    a.q_row0 = 2;
+    a.bonus_row = B - 1;
+    a.drafts = c->coh_drafts; a.drafts_stride = B; a.drafts_off = 1;
+    a.lse_q_in = c->coh_lse_q; a.lse_q_stride = B; a.lse_q_off = 1;
+    a.seed = c->seed;
+    a.req_slot = c->coh_rows + n_draft;
+    a.cached = c->d_cached;
+    a.pending = c->d_pending;
+    a.slot_stream = c->d_stream;
+    a.first_tok = c->coh_drafts;
+    a.out_tok = out_tokens;
+    a.out_stride = B + 1;
+    a.n_out = n_new;
+    a.partial = c->partial;
+    a.lse = c->lse_ws;
+    a.row_counter = c->row_counter;
+    a.req_counter = c->req_counter;
+    a.at_ws = c->at_ws;
+    a.resid_part = c->resid_part;
+    a.resid_counter = c->resid_counter;
+    a.rows_red = B;
+    a.n_p = B;
+    a.status = c->d_status;
+    a.fixed_at = c->fixed_accept > 0 ? c->fixed_accept - 1 : -1;
+    a.per_slot = 1;
+    a.phase = c->coh_phase;
+    {
+      Prof prof(c, UNO_K_VERIFY, (double)n_verify * B * V * 4);
+      c->prof_launches[UNO_K_VERIFY] +=
+          launch_verify(c->genv.pdl, c->stream, a, n_verify, c->verify_split_ctas, false) - 1;
+    }
+    {
+      Prof prof(c, UNO_K_VERIFY, (double)n_verify * 2 * V * 4);
+      launch_resid(c->genv.pdl, c->stream, a, n_verify, false);
+    }
+  }
+  CK(cudaGetLastError());
+  return UNO_OK;
+}
+
 int ar_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
   int rc = forward_any(c, PASS_AR, n_req, 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
@@ -1646,6 +1757,32 @@ int uno_spec_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* ou
   return run_graphed(c, 0, n_req, req_ids_dev, out_tokens_dev, n_new_dev, [&] {
     return spec_step_body(c, n_req, req_ids_dev, out_tokens_dev, n_new_dev);
   });
+}
+
+int uno_spec_step_cohorts(uno_ctx* c, int n_draft, const int32_t* draft_ids_dev, int n_verify,
+                          const int32_t* verify_ids_dev, int32_t* out_tokens_dev, int32_t* n_new_dev) {
+  if (!c) return UNO_ERR_ARG;
+  c->err.clear();
+  if (n_draft < 0 || n_verify < 0 || n_draft + n_verify < 1 || n_draft + n_verify > c->max_batch ||
+      (n_draft && !draft_ids_dev) || (n_verify && (!verify_ids_dev || !out_tokens_dev || !n_new_dev)))
+    return fail(c, UNO_ERR_ARG, "bad cohort step arguments");
+  if (c->top_p < 1.f) return fail(c, UNO_ERR_UNSUPPORTED, "the cohort step samples without top-p");
+  if (!c->coh_logits) {
+    // first call: the per-slot buffers (one-time allocation)
+    const size_t B = c->B, V = c->s.vocab, mb = c->max_batch;
+    if (dalloc(&c->coh_logits, 2 * mb * (B + 1) * V * 4) != cudaSuccess ||
+        dalloc(&c->coh_drafts, mb * B * 4) != cudaSuccess || dalloc(&c->coh_lse_q, mb * B * 4) != cudaSuccess ||
+        dalloc(&c->coh_phase, mb * 4) != cudaSuccess || dalloc(&c->coh_rows, mb * 4) != cudaSuccess ||
+        dalloc(&c->coh_rowoff, (size_t)c->M_max * 8) != cudaSuccess)
+      return fail(c, UNO_ERR_OOM, "cohort buffers");
+    CK(cudaMemsetAsync(c->coh_phase, 0, mb * 4, c->stream));
+    CK(cudaMemsetAsync(c->coh_drafts, 0, mb * B * 4, c->stream));
+  }
+  return run_graphed(
+      c, 2, n_draft * 65536 + n_verify, draft_ids_dev, verify_ids_dev, out_tokens_dev,
+      [&] { return cohort_step_body(c, n_draft, draft_ids_dev, n_verify, verify_ids_dev,
+                                    out_tokens_dev, n_new_dev); },
+      n_new_dev);
 }
 
 int uno_ar_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev) {
@@ -1818,6 +1955,8 @@ int uno_debug_read(uno_ctx* c, int which, void* dst, size_t bytes) {
     case UNO_DBG_LOGITS_AR: src = c->logits_d; cap = mb * V * 4; break;
     case UNO_DBG_TOPP_DRAFT: src = c->filt_d; cap = mb * (B + 1) * sizeof(RowFilter); break;
     case UNO_DBG_TOPP_VERIFY: src = c->filt_v; cap = mb * B * sizeof(RowFilter); break;
+    case UNO_DBG_COHORT_LOGITS: src = c->coh_logits; cap = c->coh_logits ? 2 * mb * (B + 1) * V * 4 : 0; break;
+    case UNO_DBG_COHORT_DRAFTS: src = c->coh_drafts; cap = c->coh_drafts ? mb * B * 4 : 0; break;
     default: return fail(c, UNO_ERR_ARG, "unknown debug buffer");
   }
   if (bytes > cap) return fail(c, UNO_ERR_ARG, "debug read larger than the buffer");

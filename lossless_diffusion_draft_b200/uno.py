@@ -20,7 +20,7 @@ UNO_F32, UNO_BF16 = 0, 1
 UNO_OK, UNO_ERR_ARG, UNO_ERR_OOM, UNO_ERR_CAPACITY, UNO_ERR_CUDA, UNO_ERR_DEVICE_CHECK, \
     UNO_ERR_UNSUPPORTED = range(7)
 UNO_DBG_LOGITS_DRAFT, UNO_DBG_LOGITS_VERIFY, UNO_DBG_DRAFTS, UNO_DBG_LOGITS_AR, \
-    UNO_DBG_TOPP_DRAFT, UNO_DBG_TOPP_VERIFY = range(6)
+    UNO_DBG_TOPP_DRAFT, UNO_DBG_TOPP_VERIFY, UNO_DBG_COHORT_LOGITS, UNO_DBG_COHORT_DRAFTS = range(8)
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 N_PROJ = len(PROJ)
 
@@ -71,6 +71,7 @@ def load_library(path=LIB_PATH):
         "uno_prefill": (i32, [vp, i32, vp, i32, vp, vp, vp]),
         "uno_spec_step": (i32, [vp, i32, vp, vp, vp]),
         "uno_train_forward": (i32, [vp, i32, vp, i32, vp]),
+        "uno_spec_step_cohorts": (i32, [vp, i32, vp, i32, vp, vp, vp]),
         "uno_ar_step": (i32, [vp, i32, vp, vp]),
         "uno_release": (i32, [vp, i32]),
         "uno_destroy": (i32, [vp]),
@@ -215,6 +216,17 @@ def uno_train_forward(ctx, tokens_dev, logits_dev):
     n_seq, two_l = tokens_dev.shape
     code = load_library().uno_train_forward(ctx.handle, n_seq, _ptr(tokens_dev), two_l // 2,
                                             _ptr(logits_dev))
+    _check(code, ctx.handle)
+
+
+def uno_spec_step_cohorts(ctx, draft_ids_dev, verify_ids_dev, out_tokens_dev, n_new_dev):
+    """One forward: draft rows of draft_ids_dev, verify rows of verify_ids_dev (either may be None)."""
+    nd = 0 if draft_ids_dev is None else draft_ids_dev.numel()
+    nv = 0 if verify_ids_dev is None else verify_ids_dev.numel()
+    code = load_library().uno_spec_step_cohorts(ctx.handle, nd, _ptr(draft_ids_dev) if nd else None, nv,
+                                                _ptr(verify_ids_dev) if nv else None,
+                                                _ptr(out_tokens_dev) if nv else None,
+                                                _ptr(n_new_dev) if nv else None)
     _check(code, ctx.handle)
 
 
