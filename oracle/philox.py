@@ -11,9 +11,10 @@ ten-round variant is the one the authors recommend.
 The uniforms of the Psi-Spec sampler are one Philox block per draw:
 
 * key     = (seed & 0xffffffff, seed >> 32)
-* counter = (stream, position, kind, 0), where ``stream`` is the request's
-  random stream id, ``position`` the absolute 0-based position of the token
-  that the draw decides, and ``kind`` one of the ``KIND_*`` values below;
+* counter = (stream, position, kind, lane), where ``stream`` is the
+  request's random stream id, ``position`` the absolute 0-based position of
+  the token that the draw decides, ``kind`` one of the ``KIND_*`` values
+  below and ``lane`` 0 (the tree sampler's chain index);
 * u = ((x0 >> 9) * 2 + 1) * 2**-24 from output word 0, which lies strictly
   inside (0, 1) and is exact in float32.
 
@@ -69,12 +70,15 @@ def bits_to_uniform(x):
     return ((x >> np.uint64(9)) * np.uint64(2) + np.uint64(1)).astype(np.float64) / float(1 << 24)
 
 
-def uniform(seed, stream, position, kind):
+def uniform(seed, stream, position, kind, lane=0):
     """The uniform of draw ``kind`` for the token at ``position`` of ``stream``.
 
-    Any argument may be an array; the result broadcasts.
+    ``lane`` is counter word 3: 0 for every draw of the linear sampler; the
+    tree sampler numbers its drafted chains with it (chain 0 draws exactly
+    the linear sampler's uniforms).  Any argument may be an array; the
+    result broadcasts.
     """
     seed = int(seed)
     key = (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
-    x0, _, _, _ = philox4x32_10((stream, position, kind, 0), key)
+    x0, _, _, _ = philox4x32_10((stream, position, kind, lane), key)
     return bits_to_uniform(x0)

@@ -120,6 +120,40 @@ def residual_token(p_logits, q_logits, u):
     return _inverse_cdf(r, u)
 
 
+def rrs_token(p_logits, q_logits, cands, u_accept, u_resid):
+    """Recursive rejection over several candidates drawn i.i.d. from q (the
+    tree sampler's step at one position; with one candidate it is the linear
+    sampler's accept test and residual draw).
+
+    The target starts as p.  Candidate j is accepted iff
+    u_accept[j] < r(y_j) / q(y_j) (log domain, strict) for the current
+    target r; on a rejection r becomes max(0, r - q) renormalised (kept as it
+    is if that has no mass after rounding).  If every candidate is rejected
+    the token is drawn from the last r with u_resid.  Returns (j, token):
+    j = index of the accepted candidate, or None with the drawn token.
+    Lossless: the returned token follows p (pinned by exact enumeration).
+    Uniforms are read only when used: u_accept[j] when candidate j is
+    tested, u_resid (a number, or a function of no argument giving it) only
+    for the residual draw.
+    """
+    cands = [int(y) for y in cands]
+    resid_u = u_resid if callable(u_resid) else (lambda: u_resid)
+    if accept_draft(p_logits, q_logits, cands[0], u_accept[0]):
+        return 0, cands[0]
+    if len(cands) == 1:
+        return None, residual_token(p_logits, q_logits, resid_u())
+    q = np.exp(log_softmax(np.asarray(q_logits, np.float64)))
+    r = np.exp(log_softmax(np.asarray(p_logits, np.float64)))
+    for j, y in enumerate(cands):
+        if j > 0 and r[y] > 0 and math.log(u_accept[j]) < math.log(r[y]) - math.log(q[y]):
+            return j, y
+        res = np.maximum(r - q, 0.0)
+        z = float(np.sum(res))
+        if z > 0.0:
+            r = res / z
+    return None, _inverse_cdf(r, resid_u())
+
+
 def verify_block(p_rows, q_rows, drafts, u_accept, u_resid, bonus_row):
     """Rejection step over a drafted block.
 
@@ -264,3 +298,105 @@ def ar_step(model, state, seed, uniform_fn=None, top_p=None):
     cache = state.cache.copy()
     cache.append(k, v, [0])
     return DecodeState(state.tokens + [y], cache, state.stream), logits[0], y
+
+
+# ---------------------------------------------------------------------------
+# Tree sampler (Summary §方法关键点: the linear sampler serves system
+# throughput, the tree sampler per-request throughput at batch 1; the
+# Walkthrough's description of the two candidate-set modes is missing from
+# the page).  Reading: the block's first token x_1 is drawn from the AR row
+# as in the linear sampler; k chains then draft positions 2..B independently
+# from the drafter's rows (chain j draws its token at position c+d with the
+# DRAFT uniform of lane j, so chain 0 is the linear sampler's block).  The
+# AR path verifies every chain [x_1, y_j2, ..., y_jB] in one verify pass (k B
+# rows, each chain seeing the cache and its own earlier tokens).  The walk
+# goes down the tree: at position 2 every chain's token is a candidate
+# (chain order); at a later position the candidates are the continuing
+# chain's token, then the other chains' tokens there (chain order), which,
+# if accepted, end the block because no AR row conditions on them.  Each
+# position is one recursive rejection (rrs_token) with the ACCEPT uniform of
+# the candidate's lane and the RESID uniform of lane 0.  With k = 1 the tree
+# sampler is the linear sampler, uniform for uniform.
+# ---------------------------------------------------------------------------
+
+class _Lazy:
+    """Sequence whose item i is f(i), evaluated when read."""
+
+    def __init__(self, f):
+        self.f = f
+
+    def __getitem__(self, i):
+        return self.f(i)
+
+
+def tree_walk(p_rows, q_rows, chains, c, uniform_fn):
+    """The tree's verification walk.
+
+    p_rows[j][i]: AR logits of position c+2+i given chain j's tokens up to
+    depth i+1 (i = 0..B-1; row 0 is the same for every chain); q_rows[d]:
+    drafter logits of position c+d (d = 2..B); chains[j] = [x_1, y_j2, ...,
+    y_jB].  uniform_fn(kind, position, lane).
+    Returns (path, last, jstar): the accepted tokens along the continuing
+    chain (x_1 first), the final emitted token, and that chain (None when
+    nothing past x_1 was accepted).
+    """
+    k, B = len(chains), len(chains[0])
+    path, jstar = [chains[0][0]], None
+    for d in range(2, B + 1):
+        prow = p_rows[0][0] if d == 2 else p_rows[jstar][d - 2]
+        order = list(range(k)) if d == 2 else [jstar] + [j for j in range(k) if j != jstar]
+        cands = [chains[j][d - 1] for j in order]
+        ua = _Lazy(lambda i, d=d, order=order: uniform_fn(KIND_ACCEPT, c + d, order[i]))
+        idx, tok = rrs_token(prow, q_rows[d], cands, ua, lambda d=d: uniform_fn(KIND_RESID, c + d, 0))
+        if idx is None:
+            return path, tok, jstar
+        j = order[idx]
+        if d == 2 or j == jstar:
+            jstar = j
+            path.append(tok)
+            continue
+        return path, tok, jstar
+    return path, sample_token(p_rows[jstar][B - 1], uniform_fn(KIND_RESID, c + B + 1, 0)), jstar
+
+
+@dataclass
+class TreeResult:
+    c: int
+    logits_draft: np.ndarray            # [B+1, V]
+    logits_verify: list                 # per chain [B, V]
+    chains: list                        # per chain [x_1, y_2, ..., y_B]
+    path: list                          # accepted tokens along the continuing chain
+    jstar: object                       # that chain, or None
+    emitted: list = field(default_factory=list)
+
+
+def tree_spec_step(model, state, B, k, seed, chains=None, uniform_fn=None):
+    """One tree-sampler iteration; returns (new_state, TreeResult).
+
+    ``chains`` (optional) replaces the drafted chains (each [x_1, y_2..y_B])
+    so a test can verify exactly what another implementation drafted.
+    """
+    if uniform_fn is None:
+        def uniform_fn(kind, position, lane=0):
+            return float(uniform(seed, state.stream, position, kind, lane))
+    c = state.c
+    logits_d, kd, vd = draft_pass(model, state, B)
+    if chains is None:
+        x1 = sample_token(logits_d[0], uniform_fn(KIND_FIRST, c + 1, 0))
+        chains = [[x1] + [sample_token(logits_d[d], uniform_fn(KIND_DRAFT, c + d, j))
+                          for d in range(2, B + 1)] for j in range(k)]
+    chains = [[int(t) for t in ch] for ch in chains]
+    cache = state.cache.copy()
+    cache.append(kd, vd, [0])                      # pending token's K/V at position c
+    p_rows, kvs = [], []
+    for ch in chains:
+        lv, kk, vv = verify_pass(model, cache, c, ch)
+        p_rows.append(lv)
+        kvs.append((kk, vv))
+    q_rows = {d: logits_d[d] for d in range(2, B + 1)}
+    path, last, jstar = tree_walk(p_rows, q_rows, chains, c, uniform_fn)
+    kk, vv = kvs[0 if jstar is None else jstar]
+    cache.append(kk, vv, range(len(path)))         # positions c+1..c+len(path)
+    emitted = path + [last]
+    new_state = DecodeState(state.tokens + emitted, cache, state.stream)
+    return new_state, TreeResult(c, logits_d, p_rows, chains, path, jstar, emitted)
