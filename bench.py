@@ -488,6 +488,7 @@ def run_uno(args, rank, world, device):
         del wl
         torch.cuda.empty_cache()
         res["cohorts"] = run_cohorts(args, cfg, params, rank, world, device)
+        res["tree"] = run_tree(args, cfg, params, rank, world, device)
         res["max_batch"] = run_max_batch(args, cfg, params, rank, world, device, pk)
         res["spec_verify_micro"] = spec_verify_micro(args, device, pk)
     return res
@@ -531,6 +532,50 @@ def run_cohorts(args, cfg, params, rank, world, device, batch=16):
             "note": "two cohorts of 8 out of phase (one forward per call) against plain steps of 16 "
                     "(two forwards per step); per request both do one draft and one verify "
                     "forward per iteration"}
+
+
+def run_tree(args, cfg, params, rank, world, device):
+    """The tree sampler at batch 1 and the mean context: one request, k = 1
+    (the linear sampler), 2 and 4 drafted chains, each timed over the same
+    number of steps from the same state.  The context is made with two
+    request slots so that the second slot's pages hold the chains' scratch
+    pages."""
+    from lossless_diffusion_draft_b200 import synth, uno
+    B = cfg["B"]
+    K = max(4, args.steps // 2)
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = cfg["dtype"]
+    max_ctx = cfg["prompt_len"] + cfg["gen_tokens"] + B + 1
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, 2, max_ctx,
+                       cfg["seed"], torch.cuda.current_stream())
+    P = cfg["prompt_len"] + cfg["gen_tokens"] // 2 + 1
+    prompt = torch.from_numpy(synth.make_prompts(cfg, 1, P, seed=cfg["seed"] + 1000 * rank)).to(device)
+    out = torch.zeros((1, B + 1), dtype=torch.int32, device=device)
+    n_new = torch.zeros((K, 1), dtype=torch.int32, device=device)
+    res = {}
+    for k in (1, 2, 4):
+        uno.uno_set_tree(ctx, k)
+        ids = uno.uno_prefill(ctx, prompt, [P], streams=replica_streams(rank, 1))
+        req = torch.tensor(ids, dtype=torch.int32, device=device)
+        for _ in range(3):
+            uno.uno_spec_step(ctx, req, out, n_new[0])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            uno.uno_spec_step(ctx, req, out, n_new[i])
+        e1.record()
+        torch.cuda.synchronize()
+        uno.uno_status(ctx)
+        ms = e0.elapsed_time(e1)
+        tok = int(n_new.sum().item())
+        res[str(k)] = {"tokens_per_s": tok / (ms / 1e3), "ms_per_step": ms / K,
+                       "tokens_per_step": tok / K}
+        uno.uno_release(ctx, ids[0])
+    ctx.close()
+    return {"batch": 1, "context": P - 1, "steps": K, "chains": res,
+            "note": "tree sampler with k drafted chains (k = 1: the linear sampler); random-init "
+                    "weights, so the drafter's acceptance is low"}
 
 
 def run_max_batch(args, cfg, params, rank, world, device, pk):
@@ -902,6 +947,8 @@ def main():
                     "tokens (TPF 2.5, the pages' trained-adapter range); not a parity run"}
     if "cohorts" in res:
         line["cohorts"] = res["cohorts"]
+    if "tree" in res:
+        line["tree"] = res["tree"]
     if "max_batch" in res:
         line["max_batch"] = res["max_batch"]
     if "spec_verify_micro" in res:

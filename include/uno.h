@@ -261,6 +261,32 @@ int uno_debug_set_fixed_accept(uno_ctx *ctx, int a);
 int uno_debug_set_dep_wait(uno_ctx *ctx, uint64_t limit_ns, uint32_t extra);
 
 /*
+ * Tree sampler (summary page "通过离散扩散实现 LLM 无损加速：扩散增强自回归模型",
+ * section 方法关键点: the linear sampler serves system throughput, the tree
+ * sampler per-request throughput at batch 1; the blog page's description of
+ * the two candidate-set modes is lost).  With k >= 2, every later
+ * uno_spec_step drafts k chains that share the AR first token x_1 - chain j
+ * draws positions 2..B from the drafter's rows with its own uniforms - and
+ * verifies all of them in one verify pass (k B rows per request); the walk
+ * then accepts, at each position, one of the candidates by recursive
+ * rejection: at position 2 every chain's token (chain order), later the
+ * continuing chain's token first and then the other chains' tokens, which end
+ * the block when accepted (no AR row conditions on them).  A rejection
+ * replaces the target by max(0, r - q) renormalised; when every candidate is
+ * rejected the token is drawn from the last target.  Emits 2 .. B+1 tokens
+ * per request like the linear sampler and follows the AR distribution
+ * exactly.  k = 1 is the linear sampler (the default).
+ * Each request slot keeps 2 k scratch KV pages for its chains, taken from the
+ * free pages when the setting is made (UNO_ERR_CAPACITY if there are too
+ * few: leave spare request slots); k = 1 gives them back.  A step needs
+ * n_req * k * B <= max(512, max_batch * (B + 1)) rows (else
+ * UNO_ERR_CAPACITY); top_p < 1 with the tree: UNO_ERR_UNSUPPORTED.
+ * Synchronises the stream; drops captured graphs.  k outside [1, 4]:
+ * UNO_ERR_ARG.
+ */
+int uno_set_tree(uno_ctx *ctx, int k);
+
+/*
  * Nucleus (top-p) sampling (blog page "…Uno 的无损加速之路", section 我的判断:
  * the evaluation setting is temperature 1 with top-p 0.95, and losslessness
  * holds with respect to that sampling distribution).  With top_p < 1 every
@@ -323,6 +349,11 @@ int uno_request_state(uno_ctx *ctx, int req_id, int32_t *cached_out, int32_t *pe
  *                               of each slot (rows [slot]), then the last call's
  *                               verify logits (rows [max_batch + i], i-th verified)
  *   UNO_DBG_COHORT_DRAFTS int32 [max_batch, B]      cohort step: drafted block per slot
+ *   UNO_DBG_TREE_CHAINS   int32 [n_req, k, B]       tree sampler: the drafted chains
+ *                               (x_1, y_j2 .. y_jB) of the last step
+ *   UNO_DBG_TREE_LOGITS   f32   [n_req, k, B, vocab] tree sampler: each chain's verify logits
+ *   UNO_DBG_TREE_WALK     int32 [n_req, 3]          tree sampler: c, accepted path length m,
+ *                               the path's chain
  * A nucleus entry is (key, id_cut) as uno_top_p_filter writes it.  The
  * logits are those of the model (before any nucleus filter).
  * bytes must not exceed the buffer's size for max_batch requests.
@@ -330,7 +361,7 @@ int uno_request_state(uno_ctx *ctx, int req_id, int32_t *cached_out, int32_t *pe
 enum uno_debug_buf {
   UNO_DBG_LOGITS_DRAFT = 0, UNO_DBG_LOGITS_VERIFY = 1, UNO_DBG_DRAFTS = 2, UNO_DBG_LOGITS_AR = 3,
   UNO_DBG_TOPP_DRAFT = 4, UNO_DBG_TOPP_VERIFY = 5, UNO_DBG_COHORT_LOGITS = 6,
-  UNO_DBG_COHORT_DRAFTS = 7
+  UNO_DBG_COHORT_DRAFTS = 7, UNO_DBG_TREE_CHAINS = 8, UNO_DBG_TREE_LOGITS = 9, UNO_DBG_TREE_WALK = 10
 };
 int uno_debug_read(uno_ctx *ctx, int which, void *dst_host, size_t bytes);
 

@@ -74,11 +74,13 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
 enum DrawKind : uint32_t { KIND_FIRST = 0, KIND_DRAFT = 1, KIND_ACCEPT = 2, KIND_RESID = 3 };
 
 // Uniform of draw `kind` for the token at absolute `pos` of random stream
-// `stream`: counter (stream, pos, kind, 0), key (seed lo, seed hi), output
+// `stream`: counter (stream, pos, kind, lane), key (seed lo, seed hi), output
 // word 0 mapped to ((x >> 9) * 2 + 1) * 2^-24, exact in fp32 and in (0, 1).
+// lane is 0 for every draw of the linear sampler; the tree sampler numbers
+// its drafted chains with it (chain 0 draws the linear sampler's uniforms).
 __device__ __forceinline__ float philox_uniform(uint64_t seed, uint32_t stream, uint32_t pos,
-                                                uint32_t kind) {
-  const uint4 r = philox4x32_10(make_uint4(stream, pos, kind, 0u),
+                                                uint32_t kind, uint32_t lane = 0u) {
+  const uint4 r = philox4x32_10(make_uint4(stream, pos, kind, lane),
                                 make_uint2((uint32_t)seed, (uint32_t)(seed >> 32)));
   return (float)((r.x >> 9) * 2u + 1u) * (1.0f / 16777216.0f);
 }

@@ -49,7 +49,11 @@ struct KvLayout {
 
 // Pass kinds (a pass is one forward over a set of rows).
 enum PassKind : int { PASS_PREFILL = 0, PASS_DRAFT = 1, PASS_VERIFY = 2, PASS_AR = 3, PASS_TRAIN = 4,
-                      PASS_COHORT = 5 };
+                      PASS_COHORT = 5, PASS_TREE = 6 };
+
+// Tree sampler: at most this many drafted chains; the scratch slot of chain
+// j of request slot r is max_batch + r TREE_MAX_K + j.
+constexpr int TREE_MAX_K = 4;
 
 // The keys each query row sees, by the block-causal rule (blog page "…Uno
 // 的无损加速之路", section Diffusion Distillation：一步蒸馏 + 块级扩散: a clean
@@ -140,6 +144,15 @@ struct RowArgs {
   const int32_t* coh_drafts;   // [max_batch, B]
   int64_t* row_off;            // [M] element offset of each row's logits
   int64_t coh_v_row0;          // logits row of the verify cohort's first row
+  // tree verify pass: rows of chain j of request r form "request" r k + j
+  // (B rows each); each chain keeps its keys in its scratch slot, whose page
+  // table points its pages of positions c+1 .. c+B at the chain's two
+  // scratch pages (written here, by the chain's first row)
+  int tree_k;
+  const int32_t* tree_chains;  // [n_req, k, B]
+  const int32_t* tree_pages;   // [max_batch, TREE_MAX_K, 2] scratch pages
+  int32_t* pt_rw;              // the page table (writable)
+  int pages_per_req;
 };
 
 // a1: build the rows of a pass and gather their embeddings.
@@ -165,6 +178,24 @@ __global__ void build_rows_kernel(const RowArgs a) {
     slot = a.prefill_slot;
     tok = a.prompt[j];
     pos = a.prefill_pos0 + j;
+  } else if (a.kind == PASS_TREE) {
+    const int r = req / a.tree_k, ci = req % a.tree_k;
+    int rslot = a.req_slot[r];
+    if (rslot < 0 || rslot >= a.max_batch) { raise_status(a.status, ST_BAD_SLOT); rslot = 0; }
+    const int c = a.cached[rslot];
+    tok = a.tree_chains[((size_t)r * a.tree_k + ci) * a.B + j];
+    pos = c + 1 + j;
+    slot = a.max_batch + rslot * TREE_MAX_K + ci;
+    if (threadIdx.x == 0) {
+      a.row_cslot[row] = rslot;
+      a.row_blk[row] = c + 1;
+      if (j == 0) {
+        const int p0 = (c + 1) / KV_PAGE;
+        const int32_t* tp = a.tree_pages + ((size_t)rslot * TREE_MAX_K + ci) * 2;
+        if (p0 < a.pages_per_req) a.pt_rw[(size_t)slot * a.pages_per_req + p0] = tp[0];
+        if (p0 + 1 < a.pages_per_req) a.pt_rw[(size_t)slot * a.pages_per_req + p0 + 1] = tp[1];
+      }
+    }
   } else if (a.kind == PASS_TRAIN) {
     // training form [x, z] of sequence req: rows j < L are the clean tokens
     // x_j (gate 0, its clean slot), rows L + i the noised tokens z_i (gate on,

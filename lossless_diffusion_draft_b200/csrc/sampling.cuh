@@ -353,6 +353,11 @@ struct SampleArgs {
   // slot instead of its position in the batch (the cohort step keeps them
   // between calls), and phase[slot] is set to 1 (drafted)
   int per_slot; int32_t* phase;
+  // tree sampler (tree_k >= 1): sampled row 0 is x_1, row 1 + j (B-1) + d - 2
+  // draws chain j's token at position c + d from logit row d with Philox lane
+  // j; out_tok is [n_req, tree_k, B] (x_1 at index 0 of every chain), and
+  // lse_out [n_req, B] keeps lse(q_d) at index d - 1 (from chain 0's rows)
+  int tree_k, tree_B;
 };
 
 template <bool FILT>
@@ -364,7 +369,12 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   const int k = blockIdx.x;
   const int rid = blockIdx.y;
   const int req = rid / a.rows_per_req, s = rid % a.rows_per_req;
-  const int lrow = (a.ar_mode || s == 0) ? 0 : s + 1;
+  int lrow = (a.ar_mode || s == 0) ? 0 : s + 1;
+  int lane = 0;
+  if (a.tree_k > 0 && s > 0) {
+    lane = (s - 1) / (a.tree_B - 1);
+    lrow = 2 + (s - 1) % (a.tree_B - 1);
+  }
   const int slot = a.req_slot[req];
   const int base = a.per_slot ? slot : req;
   const float* row = a.logits + ((size_t)base * a.logit_rows_per_req + lrow) * a.V;
@@ -391,13 +401,23 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) sample_rows_kernel(const Sa
   const RowStat rs = s_rs;
   const int c = a.cached[slot];
   const uint32_t kind = (a.ar_mode || s == 0) ? KIND_FIRST : KIND_DRAFT;
-  const float u = philox_uniform(a.seed, a.slot_stream[slot], (uint32_t)(c + 1 + s), kind);
+  // the token at position c + 1 (x_1) or c + d (logit row d)
+  const int pos = (a.ar_mode || s == 0) ? c + 1 : c + lrow;
+  const float u = philox_uniform(a.seed, a.slot_stream[slot], (uint32_t)pos, kind, (uint32_t)lane);
   const int t = sample_from_partials<FILT>(row, part, a.nch, a.ch, a.V, rs, u, red, f);
   if (threadIdx.x == 0) {
     if (a.ar_mode) {
       a.out_tok[req] = t;
       a.cached[slot] = c + 1;
       a.pending[slot] = t;
+    } else if (a.tree_k > 0) {
+      const int B = a.tree_B;
+      if (s == 0) {
+        for (int j = 0; j < a.tree_k; ++j) a.out_tok[((size_t)req * a.tree_k + j) * B] = t;
+      } else {
+        a.out_tok[((size_t)req * a.tree_k + lane) * B + lrow - 1] = t;
+        if (lane == 0 && a.lse_out) a.lse_out[(size_t)req * B + lrow - 1] = rs.M + logf(rs.Z);
+      }
     } else {
       a.out_tok[(size_t)base * a.out_stride + s] = t;
       if (a.lse_out) a.lse_out[(size_t)base * a.rows_per_req + s] = rs.M + logf(rs.Z);

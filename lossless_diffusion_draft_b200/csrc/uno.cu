@@ -32,6 +32,7 @@
 #include "gemm_tc.cuh"
 #include "layers.cuh"
 #include "sampling.cuh"
+#include "tree.cuh"
 
 using namespace uno;
 
@@ -402,6 +403,16 @@ struct uno_ctx {
   int32_t* coh_rows = nullptr;     // [max_batch] slots of the pass: drafting cohort, then verifying
   int64_t* coh_rowoff = nullptr;   // [M_max] logits offset of each row
   int coh_n_draft = 0;
+  // tree sampler (tree_k >= 2; set by uno_set_tree)
+  int tree_k = 1;
+  float* logits_t = nullptr;       // [max_batch, k, B, V] chain verify logits
+  float* lse_t = nullptr;          // [max_batch, k, B]
+  int32_t* tree_chains = nullptr;  // [max_batch, k, B]
+  float* tree_resid = nullptr;     // [max_batch, 2, V]
+  int32_t* tree_walk = nullptr;    // [max_batch, 3]
+  int32_t* tree_pages = nullptr;   // [max_batch, TREE_MAX_K, 2]
+  std::vector<int32_t> h_tree_pages;   // reserved scratch pages (host copy)
+  size_t tree_cap_k = 0;           // chains the buffers are sized for
   RowKeys keys{};                                     // key ranges of the current pass
   // completion counters of the fused pass (GEMMs wait on the kernel before
   // them through these instead of pdl_wait), zeroed by each pass's first kernel
@@ -743,7 +754,13 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
   ra.coh_drafts = c->coh_drafts;
   ra.row_off = c->coh_rowoff;
   ra.coh_v_row0 = (int64_t)c->max_batch * (c->B + 1);
-  c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
+  ra.tree_k = c->tree_k;
+  ra.tree_chains = c->tree_chains;
+  ra.tree_pages = c->tree_pages;
+  ra.pt_rw = c->d_page_table;
+  ra.pages_per_req = c->kv.pages_per_req;
+  c->keys = (kind == PASS_TRAIN || kind == PASS_TREE) ? RowKeys{c->row_cslot, c->row_blk}
+                                                     : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
     klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<T>, ra);
@@ -940,7 +957,13 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ra.coh_drafts = c->coh_drafts;
   ra.row_off = c->coh_rowoff;
   ra.coh_v_row0 = (int64_t)c->max_batch * (c->B + 1);
-  c->keys = kind == PASS_TRAIN ? RowKeys{c->row_cslot, c->row_blk} : RowKeys{nullptr, nullptr};
+  ra.tree_k = c->tree_k;
+  ra.tree_chains = c->tree_chains;
+  ra.tree_pages = c->tree_pages;
+  ra.pt_rw = c->d_page_table;
+  ra.pages_per_req = c->kv.pages_per_req;
+  c->keys = (kind == PASS_TRAIN || kind == PASS_TREE) ? RowKeys{c->row_cslot, c->row_blk}
+                                                     : RowKeys{nullptr, nullptr};
   {
     Prof prof(c, UNO_K_OTHER, 0.0);
     klaunch(pdl, st, dim3(M), dim3(256), 0, build_rows_kernel<bf16>, ra);
@@ -1197,7 +1220,9 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   // zeroed: keys past a request's length are masked out of the scores, and
   // the values there must be finite so that P V (with P = 0) stays finite
   cudaMemset(c->kv_pool, 0, kv_bytes);
-  if (dalloc(&c->d_page_table, (size_t)max_batch * ppr * 4) != cudaSuccess) return oom("pages");
+  // page-table rows: the request slots, then the tree sampler's chain slots
+  const size_t pt_rows = (size_t)max_batch * (1 + TREE_MAX_K);
+  if (dalloc(&c->d_page_table, pt_rows * ppr * 4) != cudaSuccess) return oom("pages");
   if (dalloc(&c->d_cached, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
   if (dalloc(&c->d_pending, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
   if (dalloc(&c->d_stream, (size_t)max_batch * 4) != cudaSuccess) return oom("state");
@@ -1206,7 +1231,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   for (int i = 0; i < n_pages; ++i) c->free_pages[i] = n_pages - 1 - i;
   c->slot_used.assign(max_batch, 0);
   c->h_page_table.assign((size_t)max_batch * ppr, 0);
-  cudaMemset(c->d_page_table, 0, (size_t)max_batch * ppr * 4);
+  cudaMemset(c->d_page_table, 0, pt_rows * ppr * 4);
   cudaMemset(c->d_cached, 0, (size_t)max_batch * 4);
   cudaMemset(c->d_pending, 0, (size_t)max_batch * 4);
   cudaMemset(c->d_stream, 0, (size_t)max_batch * 4);
@@ -1258,7 +1283,8 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->logits_v, (size_t)max_batch * B * V * 4) != cudaSuccess) return oom("logits");
   if (dalloc(&c->drafts, (size_t)max_batch * B * 4) != cudaSuccess) return oom("drafts");
   if (dalloc(&c->lse_q, (size_t)max_batch * B * 4) != cudaSuccess) return oom("lse");
-  const size_t rows_ws = (size_t)max_batch * 2 * B;
+  // sampled / reduced rows per request: 2B (verify), 1 + k (B - 1) (tree drafts)
+  const size_t rows_ws = (size_t)max_batch * std::max(2 * B, 1 + TREE_MAX_K * (B - 1));
   if (dalloc(&c->partial, rows_ws * c->nch * sizeof(float2)) != cudaSuccess) return oom("partial");
   if (dalloc(&c->lse_ws, rows_ws * 4) != cudaSuccess) return oom("lse");
   if (dalloc(&c->row_counter, rows_ws * 4) != cudaSuccess) return oom("counters");
@@ -1357,7 +1383,8 @@ int uno_destroy(uno_ctx* c) {
   void* bufs[] = {c->kv_pool, c->d_page_table, c->d_cached, c->d_pending, c->d_stream, c->x,
                   c->xn, c->qkv, c->qbuf, c->attn, c->gu, c->U, c->row_pos, c->row_slot, c->row_gate,
                   c->row_cslot, c->row_blk, c->train_slots, c->coh_logits, c->coh_drafts,
-                  c->coh_lse_q, c->coh_phase, c->coh_rows, c->coh_rowoff,
+                  c->coh_lse_q, c->coh_phase, c->coh_rows, c->coh_rowoff, c->logits_t,
+                  c->lse_t, c->tree_chains, c->tree_resid, c->tree_walk, c->tree_pages,
                   c->dep_ctr, c->cos_t, c->sin_t, c->logits_d, c->logits_v, c->drafts, c->lse_q, c->partial,
                   c->lse_ws, c->row_counter, c->req_counter, c->at_ws, c->resid_part,
                   c->resid_counter, c->att_ws, c->att_counters, c->filt_d, c->filt_v,
@@ -1528,8 +1555,78 @@ int run_graphed(uno_ctx* c, int kind, int n_req, const void* a, const void* b, c
   return UNO_OK;
 }
 
+// The tree sampler's iteration (tree_k >= 2): the draft pass, k drafted
+// chains, one verify pass over every chain, the walk and the commit.
+int tree_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev,
+                   int32_t* n_new_dev) {
+  const int B = c->B, V = c->s.vocab, k = c->tree_k;
+  int rc = forward_any(c, PASS_DRAFT, n_req, B + 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
+  if (rc) return rc;
+  const int rows = 1 + k * (B - 1);
+  {
+    SampleArgs a{};
+    a.logits = c->logits_d;
+    a.V = V; a.nch = c->nch; a.ch = c->ch;
+    a.rows_per_req = rows;
+    a.logit_rows_per_req = B + 1;
+    a.ar_mode = 0;
+    a.req_slot = req_ids_dev;
+    a.cached = c->d_cached;
+    a.pending = c->d_pending;
+    a.slot_stream = c->d_stream;
+    a.seed = c->seed;
+    a.out_tok = c->tree_chains;
+    a.out_stride = B;
+    a.lse_out = c->lse_q;
+    a.partial = c->partial;
+    a.row_counter = c->row_counter;
+    a.status = c->d_status;
+    a.tree_k = k;
+    a.tree_B = B;
+    Prof prof(c, UNO_K_SAMPLE, (double)n_req * rows * V * 4);
+    launch_sample(c->genv.pdl, c->stream, dim3(c->nch, n_req * rows), a);
+  }
+  rc = forward_any(c, PASS_TREE, n_req * k, B, req_ids_dev, nullptr, 0, 0, c->logits_t);
+  if (rc) return rc;
+  {
+    Prof prof(c, UNO_K_VERIFY, (double)n_req * k * B * V * 4);
+    klaunch(c->genv.pdl, c->stream, dim3(n_req * k * B), dim3(TREE_THREADS), 0, row_lse_kernel,
+            (const float*)c->logits_t, V, c->lse_t);
+  }
+  {
+    TreeArgs a{};
+    a.q = c->logits_d; a.lse_q = c->lse_q;
+    a.p = c->logits_t; a.lse_p = c->lse_t;
+    a.chains = c->tree_chains;
+    a.V = V; a.B = B; a.k = k;
+    a.seed = c->seed;
+    a.req_slot = req_ids_dev;
+    a.cached = c->d_cached; a.pending = c->d_pending; a.slot_stream = c->d_stream;
+    a.resid = c->tree_resid;
+    a.out_tok = out_tokens_dev; a.out_stride = B + 1; a.n_out = n_new_dev;
+    a.walk = c->tree_walk;
+    a.status = c->d_status;
+    Prof prof(c, UNO_K_VERIFY, (double)n_req * 4 * V * 4);
+    klaunch(c->genv.pdl, c->stream, dim3(n_req), dim3(TREE_THREADS), 0, tree_walk_kernel, a);
+  }
+  {
+    TreeCommitArgs a{};
+    a.kv = c->kv;
+    a.max_batch = c->max_batch;
+    a.esz = c->s.dtype == UNO_BF16 ? 2 : 4;
+    a.req_slot = req_ids_dev;
+    a.walk = c->tree_walk;
+    a.status = c->d_status;
+    Prof prof(c, UNO_K_OTHER, 0.0);
+    klaunch(c->genv.pdl, c->stream, dim3(B, c->s.n_layers, n_req), dim3(256), 0, tree_commit_kernel, a);
+  }
+  CK(cudaGetLastError());
+  return UNO_OK;
+}
+
 int spec_step_body(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* out_tokens_dev,
                    int32_t* n_new_dev) {
+  if (c->tree_k >= 2) return tree_step_body(c, n_req, req_ids_dev, out_tokens_dev, n_new_dev);
   const int B = c->B, V = c->s.vocab;
   int rc = forward_any(c, PASS_DRAFT, n_req, B + 1, req_ids_dev, nullptr, 0, 0, c->logits_d);
   if (rc) return rc;
@@ -1753,6 +1850,10 @@ int uno_spec_step(uno_ctx* c, int n_req, const int32_t* req_ids_dev, int32_t* ou
   c->err.clear();
   if (n_req < 1 || n_req > c->max_batch || !req_ids_dev || !out_tokens_dev || !n_new_dev)
     return fail(c, UNO_ERR_ARG, "bad spec_step arguments");
+  if (c->tree_k >= 2 && (long long)n_req * c->tree_k * c->B > c->M_max)
+    return fail(c, UNO_ERR_CAPACITY, "tree verify rows exceed the pass capacity");
+  if (c->tree_k >= 2 && c->top_p < 1.f)
+    return fail(c, UNO_ERR_UNSUPPORTED, "the tree sampler samples without top-p");
   c->last_n_req = n_req;
   return run_graphed(c, 0, n_req, req_ids_dev, out_tokens_dev, n_new_dev, [&] {
     return spec_step_body(c, n_req, req_ids_dev, out_tokens_dev, n_new_dev);
@@ -1824,6 +1925,52 @@ int uno_debug_set_dep_wait(uno_ctx* c, uint64_t limit_ns, uint32_t extra) {
   c->dep_limit_ns = limit_ns;
   c->dep_extra = extra;
   drop_graphs(c);
+  return UNO_OK;
+}
+
+int uno_set_tree(uno_ctx* c, int k) {
+  if (!c) return UNO_ERR_ARG;
+  if (k < 1 || k > TREE_MAX_K) return fail(c, UNO_ERR_ARG, "tree chains must be in [1, 4]");
+  if (k == c->tree_k) return UNO_OK;
+  CK(cudaStreamSynchronize(c->stream));
+  // give back the scratch pages of the previous setting
+  for (int32_t pg : c->h_tree_pages) c->free_pages.push_back(pg);
+  c->h_tree_pages.clear();
+  c->tree_k = 1;
+  drop_graphs(c);
+  if (k == 1) return UNO_OK;
+  const size_t mb = c->max_batch, B = c->B, V = c->s.vocab;
+  if (c->free_pages.size() < 2 * (size_t)k * mb)
+    return fail(c, UNO_ERR_CAPACITY, "the tree sampler needs 2 k free KV pages per request slot");
+  if ((size_t)k > c->tree_cap_k) {
+    void* bufs[] = {c->logits_t, c->lse_t, c->tree_chains};
+    for (void* b : bufs)
+      if (b) cudaFree(b);
+    c->logits_t = nullptr; c->lse_t = nullptr; c->tree_chains = nullptr;
+    c->tree_cap_k = 0;
+    if (dalloc(&c->logits_t, mb * k * B * V * 4) != cudaSuccess ||
+        dalloc(&c->lse_t, mb * k * B * 4) != cudaSuccess ||
+        dalloc(&c->tree_chains, mb * k * B * 4) != cudaSuccess)
+      return fail(c, UNO_ERR_OOM, "tree buffers");
+    c->tree_cap_k = k;
+  }
+  if (!c->tree_resid) {
+    if (dalloc(&c->tree_resid, mb * 2 * V * 4) != cudaSuccess ||
+        dalloc(&c->tree_walk, mb * 3 * 4) != cudaSuccess ||
+        dalloc(&c->tree_pages, mb * TREE_MAX_K * 2 * 4) != cudaSuccess)
+      return fail(c, UNO_ERR_OOM, "tree buffers");
+  }
+  std::vector<int32_t> pages(mb * TREE_MAX_K * 2, 0);
+  for (size_t r = 0; r < mb; ++r)
+    for (int j = 0; j < k; ++j)
+      for (int e = 0; e < 2; ++e) {
+        const int32_t pg = c->free_pages.back();
+        c->free_pages.pop_back();
+        c->h_tree_pages.push_back(pg);
+        pages[(r * TREE_MAX_K + j) * 2 + e] = pg;
+      }
+  CK(cudaMemcpy(c->tree_pages, pages.data(), pages.size() * 4, cudaMemcpyHostToDevice));
+  c->tree_k = k;
   return UNO_OK;
 }
 
@@ -1957,6 +2104,9 @@ int uno_debug_read(uno_ctx* c, int which, void* dst, size_t bytes) {
     case UNO_DBG_TOPP_VERIFY: src = c->filt_v; cap = mb * B * sizeof(RowFilter); break;
     case UNO_DBG_COHORT_LOGITS: src = c->coh_logits; cap = c->coh_logits ? 2 * mb * (B + 1) * V * 4 : 0; break;
     case UNO_DBG_COHORT_DRAFTS: src = c->coh_drafts; cap = c->coh_drafts ? mb * B * 4 : 0; break;
+    case UNO_DBG_TREE_CHAINS: src = c->tree_chains; cap = c->tree_chains ? mb * c->tree_cap_k * B * 4 : 0; break;
+    case UNO_DBG_TREE_LOGITS: src = c->logits_t; cap = c->logits_t ? mb * c->tree_cap_k * B * V * 4 : 0; break;
+    case UNO_DBG_TREE_WALK: src = c->tree_walk; cap = c->tree_walk ? mb * 3 * 4 : 0; break;
     default: return fail(c, UNO_ERR_ARG, "unknown debug buffer");
   }
   if (bytes > cap) return fail(c, UNO_ERR_ARG, "debug read larger than the buffer");

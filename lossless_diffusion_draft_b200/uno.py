@@ -20,7 +20,8 @@ UNO_F32, UNO_BF16 = 0, 1
 UNO_OK, UNO_ERR_ARG, UNO_ERR_OOM, UNO_ERR_CAPACITY, UNO_ERR_CUDA, UNO_ERR_DEVICE_CHECK, \
     UNO_ERR_UNSUPPORTED = range(7)
 UNO_DBG_LOGITS_DRAFT, UNO_DBG_LOGITS_VERIFY, UNO_DBG_DRAFTS, UNO_DBG_LOGITS_AR, \
-    UNO_DBG_TOPP_DRAFT, UNO_DBG_TOPP_VERIFY, UNO_DBG_COHORT_LOGITS, UNO_DBG_COHORT_DRAFTS = range(8)
+    UNO_DBG_TOPP_DRAFT, UNO_DBG_TOPP_VERIFY, UNO_DBG_COHORT_LOGITS, UNO_DBG_COHORT_DRAFTS, \
+    UNO_DBG_TREE_CHAINS, UNO_DBG_TREE_LOGITS, UNO_DBG_TREE_WALK = range(11)
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 N_PROJ = len(PROJ)
 
@@ -91,6 +92,7 @@ def load_library(path=LIB_PATH):
         "uno_set_counter_sync": (i32, [vp, i32]),
         "uno_debug_set_fixed_accept": (i32, [vp, i32]),
         "uno_set_top_p": (i32, [vp, f32]),
+        "uno_set_tree": (i32, [vp, i32]),
         "uno_top_p_filter": (i32, [vp, i32, i32, f32, vp, vp]),
         "uno_debug_set_dep_wait": (i32, [vp, u64, ctypes.c_uint32]),
         "uno_profile_records": (i32, [vp, vp, i32]),
@@ -267,6 +269,11 @@ def uno_set_verify_split(ctx, max_ctas):
 def uno_set_counter_sync(ctx, enable):
     """Fused pipeline: GEMMs wait on completion counters (True) or grid dependencies."""
     _check(load_library().uno_set_counter_sync(ctx.handle, int(bool(enable))), ctx.handle)
+
+
+def uno_set_tree(ctx, k):
+    """Tree sampler with k drafted chains (1: the linear sampler)."""
+    _check(load_library().uno_set_tree(ctx.handle, int(k)), ctx.handle)
 
 
 def uno_set_top_p(ctx, top_p):
