@@ -342,10 +342,18 @@ class Workload:
         clocks, ctx_window, launches)."""
         uno, stream = self.uno, torch.cuda.current_stream()
         B = self.B
-        n_new = torch.zeros((max(K, 1), self.batch), dtype=torch.int32, device=self.device)
+        # one output buffer for every step, so that each step replays the same
+        # captured graph; each step's counts are copied into n_hist after it
+        n_new = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+        n_hist = torch.zeros((max(K, 1), self.batch), dtype=torch.int32, device=self.device)
         ar_out = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
-        step = (lambda k: uno.uno_ar_step(self.ctx, self.req, ar_out)) if ar else \
-               (lambda k: uno.uno_spec_step(self.ctx, self.req, self.out, n_new[k]))
+
+        def step(k):
+            if ar:
+                uno.uno_ar_step(self.ctx, self.req, ar_out)
+            else:
+                uno.uno_spec_step(self.ctx, self.req, self.out, n_new)
+                n_hist[k].copy_(n_new, non_blocking=True)
         for _ in range(W):
             step(0)
         torch.cuda.synchronize()
@@ -367,7 +375,7 @@ class Workload:
         barrier(world)
         uno.uno_status(self.ctx)
         step_ms = [ev0.elapsed_time(ev[0])] + [ev[k - 1].elapsed_time(ev[k]) for k in range(1, K)]
-        tokens = K * self.batch if ar else int(n_new.sum().item())
+        tokens = K * self.batch if ar else int(n_hist.sum().item())
         return dict(ms=ev0.elapsed_time(ev1), tokens=tokens, step_ms=step_ms,
                     clocks=clk.summary() if clocks else None, ctx_window=[c0, self.cached()],
                     launches=sum(v[0] for v in prof.values()), K=K)
@@ -509,22 +517,24 @@ def run_cohorts(args, cfg, params, rank, world, device, batch=16):
     half = batch // 2
     a, b = wl.req[:half].clone(), wl.req[half:].clone()
     out = torch.zeros((half, B + 1), dtype=torch.int32, device=device)
-    n_new = torch.zeros((2 * K + 8, half), dtype=torch.int32, device=device)
-    uno.uno_spec_step_cohorts(wl.ctx, a, None, out, n_new[0])
+    n_new = torch.zeros(half, dtype=torch.int32, device=device)
+    n_hist = torch.zeros((2 * K, half), dtype=torch.int32, device=device)
+    uno.uno_spec_step_cohorts(wl.ctx, a, None, out, n_new)
     for k in range(4):                                   # warm-up (and graph capture)
         d, v = (b, a) if k % 2 == 0 else (a, b)
-        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new[0])
+        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for k in range(2 * K):                               # 2K forwards, as K plain steps
         d, v = (b, a) if k % 2 == 0 else (a, b)
-        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new[1 + k])
+        uno.uno_spec_step_cohorts(wl.ctx, d, v, out, n_new)
+        n_hist[k].copy_(n_new, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
     uno.uno_status(wl.ctx)
     ms = e0.elapsed_time(e1)
-    tokens = int(n_new[1:1 + 2 * K].sum().item())
+    tokens = int(n_hist.sum().item())
     wl.close()
     return {"batch": batch, "context": cfg["prompt_len"], "forwards": 2 * K,
             "plain": {"tokens_per_s": rate(plain), "ms_per_forward": plain["ms"] / plain["K"] / 2},
@@ -551,24 +561,26 @@ def run_tree(args, cfg, params, rank, world, device):
     P = cfg["prompt_len"] + cfg["gen_tokens"] // 2 + 1
     prompt = torch.from_numpy(synth.make_prompts(cfg, 1, P, seed=cfg["seed"] + 1000 * rank)).to(device)
     out = torch.zeros((1, B + 1), dtype=torch.int32, device=device)
-    n_new = torch.zeros((K, 1), dtype=torch.int32, device=device)
+    n_new = torch.zeros(1, dtype=torch.int32, device=device)
+    n_hist = torch.zeros((K, 1), dtype=torch.int32, device=device)
     res = {}
     for k in (1, 2, 4):
         uno.uno_set_tree(ctx, k)
         ids = uno.uno_prefill(ctx, prompt, [P], streams=replica_streams(rank, 1))
         req = torch.tensor(ids, dtype=torch.int32, device=device)
         for _ in range(3):
-            uno.uno_spec_step(ctx, req, out, n_new[0])
+            uno.uno_spec_step(ctx, req, out, n_new)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for i in range(K):
-            uno.uno_spec_step(ctx, req, out, n_new[i])
+            uno.uno_spec_step(ctx, req, out, n_new)
+            n_hist[i].copy_(n_new, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
         uno.uno_status(ctx)
         ms = e0.elapsed_time(e1)
-        tok = int(n_new.sum().item())
+        tok = int(n_hist.sum().item())
         res[str(k)] = {"tokens_per_s": tok / (ms / 1e3), "ms_per_step": ms / K,
                        "tokens_per_step": tok / K}
         uno.uno_release(ctx, ids[0])

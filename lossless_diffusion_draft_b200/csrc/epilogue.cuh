@@ -97,7 +97,6 @@ struct Geo {
 };
 typedef Geo<9, 2> GeoQkv;     // 17-row draft pass: two row groups
 typedef Geo<9, 2> GeoResid;   // its row groups only: the residual kernel has a 16-byte unit layout
-typedef Geo<9, 2> GeoSwiglu;
 
 // Row groups never straddle an m-tile of the GEMM (the part slots are per
 // m-tile): blockIdx.y = m-tile * groups_per_tile + group.  Returns false for
@@ -598,76 +597,97 @@ __global__ void __launch_bounds__(RESID_THREADS) epi_resid_kernel(const EpiArgs 
 }
 
 // ---------------------------------------------------------------------------
-// gate|up -> silu(gate) * up: grid (F / 128, row groups), GeoSwiglu::THREADS
-// threads; each thread takes the gate and the up column of one feature.
-// Two CTAs per SM (one wave for the decode passes' 2 x F / 128 CTAs): up's
-// adapter half is read after gate's dot.  Gate|up tiles have at most two
-// contributors at these sizes (more take further rounds).
+// gate|up -> silu(gate) * up: grid (F / 128, row groups of GeoResid::RG),
+// RESID_THREADS threads in the residual kernel's unit layout: thread t owns
+// row t / 32 of the group and features 4 (t % 32) .. + 3 of the tile, so every
+// part, U and output access is one 16-byte access per contributor and the
+// row's RMSNorm scale is a warp reduction of its per-tile sums.  Gate's
+// adapter runs first (its rows in registers since before the dependency
+// wait), up's after it (prefetched into L2 meanwhile); both through the
+// same shared U tile.  Two CTAs per SM: the decode passes' 2 x F / 128 CTAs
+// are one wave.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(GeoSwiglu::THREADS, 2) epi_swiglu_kernel(const EpiArgs a) {
-  typedef GeoSwiglu G;
+__global__ void __launch_bounds__(RESID_THREADS, 2) epi_swiglu_kernel(const EpiArgs a) {
+  typedef GeoResid G;
   constexpr int C = 2;
-  __shared__ float s_inv[G::RG];
-  __shared__ float s_ss[G::RG * EPI_MAX_SS];
-  __shared__ __align__(16) bf16 sUh[16 * EPI_UP];     // one adapter at a time
+  __shared__ __align__(16) bf16 sUh[16 * EPI_UP];
   __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
-  __shared__ float sDot[G::RG * TC_BM];
+  __shared__ __align__(16) float sDot[G::RG * TC_BM];
   pdl_trigger();
   const int ft = blockIdx.x;
   int m0, nrows;
   if (!row_group<G>(a, &m0, &nrows)) { dep_signal(a.done); return; }
-  const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
-  const int f = ft * TC_BM + col;
-  const int ut = a.F / TC_BM + ft;         // the up tile of the same features
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = warp;                        // the unit's row in the group
+  const int c0 = 4 * lane;                   // its first feature in the tile
+  const int f = ft * TC_BM + c0;
+  const bool live = j < nrows;
+  const int ut = a.F / TC_BM + ft;           // the up tile of the same features
+  const bool lora = a.lora != 0;
   // adapter rows are weights: gate's into registers and up's into L2 while
   // the GEMM before is still running
   BFrag B;
-  const int fw = ft * TC_BM + 16 * (threadIdx.x >> 5);   // the warp's first feature
-  if (a.lora) {
+  const int fw = ft * TC_BM + 16 * warp;     // the warp's first feature (warps 0-7)
+  if (lora && warp < 8) {
     bfrag_issue(a, 0, fw, B);
     bfrag_prefetch(a, 1, fw);
   }
   pdl_wait();
 
   // ---- every global load first
-  SsLoad<G> ssv;
-  ss_issue(a, m0, nrows, ssv);
-  PartLoad<G, C> LG, LUp, L0, L1;
-  float gate[G::RPT];
-  part_issue(a.pv, ft, m0, nrows, col, q, LG);
-  part_issue(a.pv, ut, m0, nrows, col, q, LUp);
-  if (a.lora) {
-    u_issue(a, 0, m0, nrows, col, q, L0);
-    u_issue(a, 1, m0, nrows, col, q, L1);
-    gate_issue<G>(a, m0, nrows, q, gate);
+  float ss0 = 0.f, ss1 = 0.f;
+  if (a.ss && live) {
+    const float* sr = a.ss + (size_t)(m0 + j) * a.n_ss;
+    if (lane < a.n_ss) ss0 = __ldcg(sr + lane);
+    if (lane + 32 < a.n_ss) ss1 = __ldcg(sr + lane + 32);
+  }
+  Part4<C> LG, LUp, L0, L1;
+  float gt = 0.f;
+  part4_issue(a.pv, ft, m0, j, c0, live, LG);
+  part4_issue(a.pv, ut, m0, j, c0, live, LUp);
+  if (lora) {
+    part4_issue(a.pv, a.lr.u_tile0, m0, j, c0, live, L0);
+    part4_issue(a.pv, a.lr.u_tile0 + 1, m0, j, c0, live, L1);
+    gt = live ? __ldg(a.lr.row_gate + m0 + j) : 0.f;
   }
   // ---- then the arithmetic
-  if (a.lora) u_store(L0, nrows, col, q, sUh, sUl);
-  ss_finish(a, nrows, ssv, s_ss, s_inv);     // syncs: sUh / sUl complete too
-  float g[G::RPT], u[G::RPT];
-  part_add(LG, nrows, q, g);
-  part_add(LUp, nrows, q, u);
-  if (a.lora) {
-    // gate's dots, then up's through the same tiles (up's adapter rows were
-    // prefetched into L2 before the wait)
-    lora_mma(B, sUh, sUl, sDot, nrows);
-    bfrag_issue(a, 1, fw, B);
-    __syncthreads();
-    lora_add<G>(sDot, col, q, nrows, gate, g);
-    u_store(L1, nrows, col, q, sUh, sUl);
-    __syncthreads();
-    lora_mma(B, sUh, sUl, sDot, nrows);
-    __syncthreads();
-    lora_add<G>(sDot, col, q, nrows, gate, u);
-  }
-  bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
+  float inv = 1.f;
+  if (a.ss) {
+    float t = ss0 + ss1;
 #pragma unroll
-  for (int s = 0; s < G::RPT; ++s) {
-    const int j = q + G::NQ * s;
-    if (j < nrows) {
-      const float gv = g[s] * s_inv[j], uv = u[s] * s_inv[j];
-      store_split<bf16>(a.h, lo, (size_t)(m0 + j) * a.F + f, gv / (1.0f + expf(-gv)) * uv);
-    }
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    inv = 1.0f / sqrtf(t / a.d_model + a.eps);
+  }
+  if (lora) {
+    const float4 u = part4_add(L0, live);
+    if (live) store4_split(sUh, sUl, (size_t)j * EPI_UP + c0, u);
+    __syncthreads();
+    if (warp < 8) lora_mma(B, sUh, sUl, sDot, nrows);
+  }
+  float4 g = part4_add(LG, live);
+  float4 u = part4_add(LUp, live);
+  if (lora) {
+    if (warp < 8) bfrag_issue(a, 1, fw, B);
+    const float4 u1 = part4_add(L1, live);
+    __syncthreads();                         // gate's dots complete, U tile free
+    const float4 dg = *reinterpret_cast<const float4*>(sDot + j * TC_BM + c0);
+    g.x += gt * dg.x; g.y += gt * dg.y; g.z += gt * dg.z; g.w += gt * dg.w;
+    if (live) store4_split(sUh, sUl, (size_t)j * EPI_UP + c0, u1);
+    __syncthreads();                         // every thread read its gate dots
+    if (warp < 8) lora_mma(B, sUh, sUl, sDot, nrows);
+    __syncthreads();
+    const float4 du = *reinterpret_cast<const float4*>(sDot + j * TC_BM + c0);
+    u.x += gt * du.x; u.y += gt * du.y; u.z += gt * du.z; u.w += gt * du.w;
+  }
+  if (live) {
+    float4 h;
+    const float gx = g.x * inv, gy = g.y * inv, gz = g.z * inv, gw = g.w * inv;
+    h.x = gx / (1.0f + expf(-gx)) * (u.x * inv);
+    h.y = gy / (1.0f + expf(-gy)) * (u.y * inv);
+    h.z = gz / (1.0f + expf(-gz)) * (u.z * inv);
+    h.w = gw / (1.0f + expf(-gw)) * (u.w * inv);
+    bf16* lo = a.lo_off ? a.h + (size_t)a.lo_off * a.F : nullptr;
+    store4_split(a.h, lo, (size_t)(m0 + j) * a.F + f, h);
   }
   dep_signal(a.done);
 }

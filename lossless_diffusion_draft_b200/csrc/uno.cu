@@ -1090,7 +1090,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     if (rc) return rc;
     set_lora({{c->lB[UNO_PROJ_GATE][l], F}, {c->lB[UNO_PROJ_UP][l], F}});
     ea.ss = c->ss;
-    epi(epi_swiglu_kernel, F / TC_BM, GeoSwiglu::RG, GeoSwiglu::THREADS, true);
+    epi(epi_swiglu_kernel, F / TC_BM, GeoResid::RG, RESID_THREADS, true);
 
     rc = gemm(c->xn, F, F, {{c->w[UNO_PROJ_DOWN][l], d}}, {c->lA[UNO_PROJ_DOWN][l]}, &ea.pv);
     if (rc) return rc;
