@@ -336,7 +336,7 @@ class Workload:
     def cached(self):
         return self.uno.uno_request_state(self.ctx, self.ids[0])[0]
 
-    def time_steps(self, K, W, world, ar=False, clocks=True):
+    def time_steps(self, K, W, world, ar=False, clocks=True, profile_range=False):
         """K timed steps after W untimed ones (device time by CUDA events,
         barrier and synchronize on both sides): dict(ms, tokens, step_ms,
         clocks, ctx_window, launches)."""
@@ -365,12 +365,16 @@ class Workload:
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         with ClockSampler(torch.cuda.current_device(), enabled=clocks) as clk:
             torch.cuda.synchronize()
+            if profile_range:
+                torch.cuda.profiler.start()
             ev0.record(stream)
             for k in range(K):
                 step(k)
                 ev[k].record(stream)
             ev1.record(stream)
             torch.cuda.synchronize()
+            if profile_range:
+                torch.cuda.profiler.stop()
         prof = uno.uno_profile_end(self.ctx)
         barrier(world)
         uno.uno_status(self.ctx)
@@ -465,7 +469,7 @@ def run_uno(args, rank, world, device):
     mean_ctx = prompt_len + gen // 2
     start = max(prompt_len, int(mean_ctx - (W + K) * args.est_tokens_per_step / 2))
     wl = Workload(cfg, params, batch, start, rank, device, args)
-    head = wl.time_steps(K, W, world)
+    head = wl.time_steps(K, W, world, profile_range=args.profile_range)
     kprof, detail = step_profile(wl.ctx, wl.req, wl.out, torch.zeros(batch, dtype=torch.int32,
                                                                      device=device), K, cfg)
     e2e = wl.e2e(K, world)
@@ -850,6 +854,9 @@ def main():
                     help="the batch-1 headline alone (no context sweep, fixed-accept run, "
                          "max-batch line or spec_verify microbenchmark)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket the headline's timed steps with cudaProfilerStart/Stop, for "
+                         "ncu --profile-from-start off")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -17,12 +17,14 @@
 //   warp 4  TMA: one KV page (64 keys) per tile, K and V as 64x64 boxes of the
 //           pool viewed as a 2-D [rows, head_dim] tensor;
 //   warp 5  MMA: S = Q K^T (M=128, N=64) into a double-buffered TMEM score
-//           tile; O += P V (M=128, N=head_dim, B operand MN-major) into one
-//           TMEM accumulator for the whole key range;
+//           tile; O += P V (M=128, N=head_dim, A operand P from TMEM, B
+//           operand MN-major) into one TMEM accumulator for the whole key
+//           range; the score tile is free again when PV has read its P;
 //   warps 0-3 (thread = query row): read the score row, softmax in the log2
 //           domain against a reference max that moves (rescaling O in TMEM)
 //           only when a tile's max exceeds it by more than 2^8, and write P
-//           (fp16) to shared memory in the MMA's swizzled layout.
+//           (fp16) into TMEM over the scores just read, so the softmax of one
+//           tile runs while the PV of the one before it does.
 // With several key splits each CTA writes (m, l, O) partials and
 // attn_merge_kernel (ATC_MERGE_ROWS query rows per CTA) adds them in split
 // order.  Every wait is bounded.  While it runs, idle lanes of the producer
@@ -62,18 +64,39 @@ struct AttnTcParams {
   // producer warp's idle lanes while the KV stream leaves HBM bandwidth
   // unused (null: none); 16-byte aligned, a multiple of 16 bytes
   const char* l2_pf; unsigned long long l2_pf_bytes;
+  // completion counter of the kernel that wrote q and the new K/V rows (null:
+  // pdl_wait instead) and its CTA count; for the merge kernel, the
+  // attention's counter
+  const unsigned* dep; unsigned dep_count;
+  unsigned long long dep_limit_ns;
+  unsigned* done;                   // counter every CTA adds to at its end (or null)
 };
+
+// The inputs' dependency: one thread polls the counter (the TMA producer
+// lane, which then orders its later bulk copies after the generic stores it
+// observed) and the CTA meets it at a barrier; or the grid dependency.
+__device__ __forceinline__ void attn_dep_wait(const AttnTcParams& p, bool poller) {
+  if (p.dep) {
+    if (poller) {
+      if (!dep_wait(p.dep, p.dep_count, p.dep_limit_ns)) raise_status(p.status, ST_DEP_TIMEOUT);
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    __syncthreads();
+  } else {
+    pdl_wait();
+  }
+}
 
 template <int HD>
 struct AtcCfg {
   static constexpr int NB = HD / 64;
   static constexpr int Q_BYTES = ATC_QROWS * HD * 2;
   static constexpr int KV_BYTES = ATC_KT * HD * 2;      // K or V of one stage
-  static constexpr int P_BYTES = ATC_QROWS * ATC_KT * 2;
-  // stages of K hi, K lo and V beside q hi/lo and one P tile: three for
-  // head_dim 128 (224 KB), six for 64
+  // stages of K hi, K lo and V beside q hi/lo (P lives in tensor memory):
+  // three for head_dim 128 (209 KB), six for 64 (177 KB), so that a CTA fits
+  // on an SM beside a q|k|v epilogue CTA and starts while that epilogue runs
   static constexpr int STAGES = HD <= 64 ? 6 : 3;
-  static constexpr int SMEM = 2 * Q_BYTES + STAGES * 3 * KV_BYTES + P_BYTES + 1024 + 256;
+  static constexpr int SMEM = 2 * Q_BYTES + STAGES * 3 * KV_BYTES + 1024 + 256;
   static constexpr int TMEM_COLS = 256;       // 2 score tiles + the output accumulator
   static constexpr int S_COL = 0;             // score tiles at columns 0, 64
   static constexpr int O_COL = 2 * ATC_KT;    // output accumulator at 128 .. 128 + HD
@@ -93,8 +116,11 @@ __device__ __forceinline__ void attn_store_row(bf16* dst, bf16* lo, const float*
   }
 }
 
+// At most 128 registers a thread: two of its warps and two q|k|v epilogue
+// warps (128 each) then fill one SM sub-partition's 16,384 registers, so
+// the CTA starts beside an epilogue CTA.
 template <int HD>
-__global__ void __launch_bounds__(ATC_THREADS, 1)
+__global__ void __maxnreg__(128)
     attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
                    const AttnTcParams p) {
   using C = AtcCfg<HD>;
@@ -106,17 +132,14 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   uint8_t* sK = sQl + C::Q_BYTES;                       // [STAGES] K hi: NB boxes [64 keys x 64]
   uint8_t* sKl = sK + C::STAGES * C::KV_BYTES;          // [STAGES] K lo
   uint8_t* sV = sKl + C::STAGES * C::KV_BYTES;          // [STAGES] V
-  // one P tile [128 rows x 64 keys]: P(i) is written only after PV(i-1), its
-  // previous reader, has completed (the softmax waits for that anyway)
-  uint8_t* sP = sV + C::STAGES * C::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::STAGES * C::KV_BYTES);
   uint64_t* kv_full = bars;                             // [STAGES]
   uint64_t* kv_empty = bars + C::STAGES;                // [STAGES]
   uint64_t* s_full = bars + 2 * C::STAGES;              // [2]
-  uint64_t* s_empty = s_full + 2;                       // [2] (4 warps)
+  uint64_t* s_empty = s_full + 2;                       // [2] (PV of the tile held there)
   uint64_t* p_full = s_empty + 2;                       // [2] (4 warps)
-  uint64_t* o_full = p_full + 2;                        // one phase per PV(i)
-  uint64_t* drain = o_full + 1;
+  uint64_t* o_full = p_full + 2;                        // [2] one phase per PV of a tile there
+  uint64_t* drain = o_full + 2;
   uint64_t* q_full = drain + 1;                         // q hi and lo landed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
@@ -133,10 +156,11 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4);
+      mbar_init(&s_empty[b], 1);
       mbar_init(&p_full[b], 4);
     }
-    mbar_init(o_full, 1);
+    mbar_init(&o_full[0], 1);
+    mbar_init(&o_full[1], 1);
     mbar_init(drain, 1);
     mbar_init(q_full, 1);
     *s_abort = 0;
@@ -164,7 +188,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                    "r"((unsigned)((u1 - u0) << 4))
                    : "memory");
   }
-  pdl_wait();
+  // With a completion counter (the fused pass) the row tables and the page
+  // table are complete when this kernel starts: the pass's first kernel after
+  // build_rows lets the next one launch only once build_rows has completed.
+  // The key list and its pages are then set up, and the cached pages that no
+  // row of this pass writes start loading, while the q|k|v epilogue still
+  // runs (the table loads go through L2: before the dependency wait L1 may
+  // still hold an earlier pass's lines).  Without a counter everything
+  // follows the grid dependency.
+  const bool early = p.dep != nullptr;
+  if (!early) pdl_wait();
   const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
   const int req = z / p.Hkv, kvh = z % p.Hkv;
   const int G = p.H / p.Hkv;
@@ -185,19 +218,61 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   const int t_end = (int)((long long)ntiles * (split + 1) / p.n_splits);
   const int n = t_end - t_begin;
   auto page_of_tile = [&](int t) {   // pool page of tile t of the list
-    return t < kt.n1 ? p.page_table[(size_t)kt.slot1 * p.pages_per_req + t]
-                     : p.page_table[(size_t)kt.slot2 * p.pages_per_req + kt.p2 + (t - kt.n1)];
+    return t < kt.n1 ? __ldcg(p.page_table + (size_t)kt.slot1 * p.pages_per_req + t)
+                     : __ldcg(p.page_table + (size_t)kt.slot2 * p.pages_per_req + kt.p2 + (t - kt.n1));
   };
 
   // the split's page numbers, fetched in one round while the q rows load
   __shared__ int s_pages[ATC_PAGE_PF];
+  int n_safe = 0;   // leading tiles of the split loadable before the wait (warp 4)
   if (warp == 4) {
     for (int i = lane; i < min(n, ATC_PAGE_PF); i += 32) s_pages[i] = page_of_tile(t_begin + i);
+    if (early && !p.keys.cslot && !p.keys.blk) {
+      // every key is in the request's slot and this pass writes K/V only at
+      // its rows' positions there: whole pages below the lowest of those
+      // positions hold cached keys alone
+      int lowest = 0x7fffffff;
+      for (int k = lane; k < p.rows_per_req; k += 32) {
+        const int ps = __ldcg(p.row_pos + req * p.rows_per_req + k);
+        if (ps >= 0) lowest = min(lowest, ps);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lowest = min(lowest, __shfl_xor_sync(0xffffffffu, lowest, o));
+      n_safe = max(0, min(min(n, C::STAGES), lowest / ATC_KT - t_begin));
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+
+  // K hi, K lo and V of list entry i into its ring stage (producer lane)
+  auto issue_tile = [&](int i, uint64_t pol) -> bool {
+    const int stage = i % C::STAGES;
+    const uint32_t phase = (uint32_t)(i / C::STAGES) & 1;
+    if (!mbar_wait(&kv_empty[stage], phase ^ 1)) return false;
+    mbar_expect_tx(&kv_full[stage], 3 * C::KV_BYTES);
+    const int page = i < ATC_PAGE_PF ? s_pages[i] : page_of_tile(t_begin + i);
+    // pool rows of the page's K hi, K lo and V planes for this kv head
+    const int rk = (((p.layer * p.n_pages + page) * 3 + 0) * p.Hkv + kvh) * KV_PAGE;
+    const int rkl = rk + p.Hkv * KV_PAGE;
+    const int rv = rkl + p.Hkv * KV_PAGE;
+#pragma unroll
+    for (int b = 0; b < C::NB; ++b) {
+      const int o = stage * C::KV_BYTES + b * (ATC_KT * 128);
+      tma_load_2d_stream(sK + o, &kvmap, &kv_full[stage], b * 64, rk, pol);
+      tma_load_2d_stream(sKl + o, &kvmap, &kv_full[stage], b * 64, rkl, pol);
+      tma_load_2d_stream(sV + o, &kvmap, &kv_full[stage], b * 64, rv, pol);
+    }
+    return true;
+  };
+  int issued = 0;                 // tiles issued (producer lane)
+  uint64_t pol = 0;               // K/V are read once per pass: evict first
+  if (warp == 4 && lane == 0) {
+    pol = l2_evict_first_policy();
+    while (issued < n_safe && issue_tile(issued, pol)) ++issued;
+  }
+  if (early) attn_dep_wait(p, warp == 4 && lane == 0);
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
@@ -212,25 +287,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           tma_load_3d(sQl + b * (ATC_QROWS * 128), &qmap, q_full, b * 64, kvh * G, p.q_lo_row + row0);
         }
       }
-      const uint64_t pol = l2_evict_first_policy();   // K/V are read once per pass
-      int issued = 0;
-      for (int i = 0; i < n && !*s_abort; ++i) {
-        const int stage = i % C::STAGES;
-        const uint32_t phase = (uint32_t)(i / C::STAGES) & 1;
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1)) { *s_abort = 1; break; }
-        mbar_expect_tx(&kv_full[stage], 3 * C::KV_BYTES);
-        const int page = i < ATC_PAGE_PF ? s_pages[i] : page_of_tile(t_begin + i);
-        // pool rows of the page's K hi, K lo and V planes for this kv head
-        const int rk = (((p.layer * p.n_pages + page) * 3 + 0) * p.Hkv + kvh) * KV_PAGE;
-        const int rkl = rk + p.Hkv * KV_PAGE;
-        const int rv = rkl + p.Hkv * KV_PAGE;
-#pragma unroll
-        for (int b = 0; b < C::NB; ++b) {
-          const int o = stage * C::KV_BYTES + b * (ATC_KT * 128);
-          tma_load_2d_stream(sK + o, &kvmap, &kv_full[stage], b * 64, rk, pol);
-          tma_load_2d_stream(sKl + o, &kvmap, &kv_full[stage], b * 64, rkl, pol);
-          tma_load_2d_stream(sV + o, &kvmap, &kv_full[stage], b * 64, rv, pol);
-        }
+      if (issued < n_safe) *s_abort = 1;   // an early stage wait gave up
+      for (int i = issued; i < n && !*s_abort; ++i) {
+        if (!issue_tile(i, pol)) { *s_abort = 1; break; }
         ++issued;
       }
       if (*s_abort) {
@@ -277,14 +336,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         // P(i) written (and O rescaled, if the softmax warps moved the max)
         if (!mbar_wait(&p_full[b2], (uint32_t)(i >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        // O accumulates in TMEM across tiles
+        // O accumulates in TMEM across tiles; P(i) (fp16, 16 keys per 8
+        // columns) sits over the first half of its score tile
 #pragma unroll
         for (int ks = 0; ks < ATC_KT / 16; ++ks)
-          mma_f16(tmem + C::O_COL, sdesc_k128(smem_u32(sP) + ks * 32),
-                   sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
-                   idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(o_full);            // phase i completes when PV(i) has
+          mma_f16_ts(tmem + C::O_COL, tmem + C::S_COL + b2 * ATC_KT + ks * 8,
+                     sdesc_mn128(smem_u32(sV + stage * C::KV_BYTES) + ks * 2048, ATC_KT * 128),
+                     idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&o_full[b2]);       // completes when PV(i) (and every MMA before it) has
         mma_commit(&kv_empty[stage]);
+        mma_commit(&s_empty[b2]);      // P(i) read: the score tile is free
       }
       if (!ok) {
         *s_abort = 1;
@@ -301,9 +362,11 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     // Lazy rescaling: P is formed against a reference max m that moves only
     // when a tile's max exceeds it by more than RESCALE_LOG2 (so P <= 2^8);
     // O then stays in TMEM and is rewritten only on those (rare) moves.
-    // PV(i) can start only after the softmax signals P(i), so when tile i is
-    // in hand at most PV(0..i-1) have completed: waiting for the o_full phase
-    // of PV(i-1) by parity is unambiguous.
+    // PV(i) can start only after the softmax signals P(i), and the softmax may
+    // run ahead of the PVs, so their completions are counted per score
+    // buffer: tile j's PV is completion j / 2 of o_full[j % 2], and a PV of
+    // the same buffer two tiles on cannot complete before the softmax has
+    // moved past tile j + 1, so a wait by parity is unambiguous.
     constexpr float RESCALE_LOG2 = 8.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -315,9 +378,6 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
       float s[ATC_KT];
       tmem_ld32(lane_base + C::S_COL + sb * ATC_KT, s);
       tmem_ld32(lane_base + C::S_COL + sb * ATC_KT + 32, s + 32);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
       // raw scores; keys outside the row's range of this tile's segment -> -inf
       // (only the edge tiles of a range need the test)
       const int ti = t_begin + i;
@@ -336,14 +396,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         }
       }
       mx *= p.scale_log2;             // log2 units (the scale is positive)
-      bool pv_done = false;           // PV(i-1) known complete
       const bool need = mx > m + RESCALE_LOG2;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mx : m;
         if (i > 0) {
-          bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(i - 1) & 1);
+          bool w2 = !*s_abort && mbar_wait(&o_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1);
           if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-          pv_done = true;
           tc_fence_after();
           const float corr = (m_new == m) ? 1.f : exp2f(m - m_new);   // m = -inf: O row is 0
 #pragma unroll 1
@@ -373,35 +431,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       l += psum;
-      // the P tile was last read by PV(i-1): wait for it before overwriting
-      if (i > 0 && !pv_done) {
-        bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(i - 1) & 1);
-        if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-      }
-      // P row -> shared memory (K-major over keys, 128-byte swizzle)
-      uint8_t* prow = sP + r * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_async_smem();
+      // P row -> tensor memory over the scores just read (this thread's lane;
+      // the tile is not rewritten before PV(i) has read it)
+      tmem_st32u(lane_base + C::S_COL + sb * ATC_KT, pk);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    float o[HD];
-#pragma unroll
-    for (int d = 0; d < HD; ++d) o[d] = 0.f;
     if (ok && n > 0) {
-      bool w2 = !*s_abort && mbar_wait(o_full, (uint32_t)(n - 1) & 1);
-      if (__all_sync(0xffffffffu, w2)) {
-        tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 32) tmem_ld32(lane_base + C::O_COL + c0, o + c0);
-        tc_fence_before();
-      } else {
-        ok = false;
-      }
+      bool w2 = !*s_abort && mbar_wait(&o_full[(n - 1) & 1], (uint32_t)((n - 1) >> 1) & 1);
+      if (!__all_sync(0xffffffffu, w2)) ok = false;
     }
     // epilogue-uniform decision
     if (lane == 0) s_ok[warp] = ok ? 1 : 0;
@@ -409,27 +448,46 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     const bool all_ok = s_ok[0] && s_ok[1] && s_ok[2] && s_ok[3];
     if (!all_ok) {
       *s_abort = 1;
-    } else if (p.n_splits == 1) {
-      if (r < nq) {
-        const int tk = r / G, g = r % G;
-        const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD;
-        attn_store_row<HD>(p.out + oo, p.out_lo ? p.out_lo + oo : nullptr, o, 1.f / l);
-      }
-    } else if (r < nq) {
-      // split partial (o unnormalised, m in log2 units, l); merged by
-      // attn_merge_kernel
+    } else {
+      // O (rows past the tile's queries read too: the TMEM load is warp-wide)
+      // 32 columns at a time, so that few registers hold it
+      tc_fence_after();
+      const int tk = r / G, g = r % G;
+      const size_t oo = (size_t)(row0 + tk) * p.ld_out + (size_t)(kvh * G + g) * HD;
       const size_t group = (size_t)z * p.n_qtiles + qt;
       float* w = p.ws + ((group * p.n_splits + split) * ATC_QROWS + r) * atc_ws_row(HD);
+      const float inv = 1.f / l;
+#pragma unroll 1
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        float o[32];
+        if (n > 0) {
+          tmem_ld32(lane_base + C::O_COL + c0, o);
+        } else {
 #pragma unroll
-      for (int d = 0; d < HD; d += 4)
-        *reinterpret_cast<float4*>(w + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
-      w[HD] = m;
-      w[HD + 1] = l;
+          for (int d = 0; d < 32; ++d) o[d] = 0.f;
+        }
+        if (r >= nq) continue;
+        if (p.n_splits == 1) {
+          attn_store_row<32>(p.out + oo + c0, p.out_lo ? p.out_lo + oo + c0 : nullptr, o, inv);
+        } else {
+          // split partial (o unnormalised, m in log2 units, l); merged by
+          // attn_merge_kernel
+#pragma unroll
+          for (int d = 0; d < 32; d += 4)
+            *reinterpret_cast<float4*>(w + c0 + d) = make_float4(o[d], o[d + 1], o[d + 2], o[d + 3]);
+        }
+      }
+      tc_fence_before();
+      if (p.n_splits > 1 && r < nq) {
+        w[HD] = m;
+        w[HD + 1] = l;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (*s_abort && threadIdx.x == 0) raise_status(p.status, ST_ATTN_TIMEOUT);
+  dep_signal_synced(p.done);        // the split partials are stored
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -449,7 +507,7 @@ constexpr int ATC_MERGE_ROWS = 2;
 template <int HD>
 __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const AttnTcParams p) {
   pdl_trigger();
-  pdl_wait();
+  attn_dep_wait(p, threadIdx.x == 0 && threadIdx.y == 0);
   const int r = blockIdx.x * ATC_MERGE_ROWS + threadIdx.y, group = blockIdx.y;
   const int z = group / p.n_qtiles, qt = group % p.n_qtiles;
   const int req = z / p.Hkv, kvh = z % p.Hkv;
@@ -465,10 +523,12 @@ __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const A
 #pragma unroll
     for (int s = 0; s < ATC_MAX_SPLITS; ++s) {
       if (s < p.n_splits) {
-        const float2 ml = *reinterpret_cast<const float2*>(wg + s * sstride + HD);
+        // through L2: with a completion counter there is no grid wait to
+        // drop L1 lines of an earlier pass
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(wg + s * sstride + HD));
         ms[s] = ml.x;
         ls[s] = ml.y;
-        os[s] = wg[s * sstride + d];
+        os[s] = __ldcg(wg + s * sstride + d);
       } else {
         ms[s] = -INFINITY;
         ls[s] = 0.f;

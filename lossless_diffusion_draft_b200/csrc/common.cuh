@@ -151,6 +151,11 @@ __device__ __forceinline__ void dep_signal(unsigned* ctr) {   // whole CTA, at i
   if (threadIdx.x == 0 && threadIdx.y == 0)
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
+// The same for a CTA that has just passed a barrier after its last write.
+__device__ __forceinline__ void dep_signal_synced(unsigned* ctr) {
+  if (ctr && threadIdx.x == 0 && threadIdx.y == 0)
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
 // limit_ns: how long to poll (global timer) before giving up.
 __device__ __forceinline__ bool dep_wait(const unsigned* ctr, unsigned target,
                                          unsigned long long limit_ns) {   // one thread

@@ -76,8 +76,25 @@ struct EpiArgs {
   // epi_swiglu
   int F; bf16* h;                    // [M][F] (lo rows lo_off below)
   int32_t* status;
-  unsigned* done;                    // completion counter the next GEMM waits on (or null)
+  unsigned* done;                    // completion counter the next kernel waits on (or null)
+  // completion counter of the GEMM whose parts this kernel reads (null:
+  // pdl_wait instead), its CTA count and how long to poll it
+  const unsigned* dep; unsigned dep_count;
+  unsigned long long dep_limit_ns;
 };
+
+// Wait for the GEMM's parts: one thread polls its completion counter and the
+// CTA meets it at a barrier (CTA-uniform call), or, without a counter, the
+// grid dependency.
+__device__ __forceinline__ void epi_wait(const EpiArgs& a) {
+  if (a.dep) {
+    if (threadIdx.x == 0 && !dep_wait(a.dep, a.dep_count, a.dep_limit_ns))
+      raise_status(a.status, ST_DEP_TIMEOUT);
+    __syncthreads();
+  } else {
+    pdl_wait();
+  }
+}
 
 // Thread layout of an epilogue CTA: NQ row slots x 128 columns, the NQ
 // slot threads of a column in adjacent lanes (thread t: slot q = t % NQ,
@@ -341,13 +358,16 @@ __device__ __forceinline__ void gate_issue(const EpiArgs& a, int m0, int nrows, 
                                            float (&g)[G::RPT]) {
 #pragma unroll
   for (int s = 0; s < G::RPT; ++s)
-    g[s] = q + G::NQ * s < nrows ? __ldg(a.lr.row_gate + m0 + q + G::NQ * s) : 0.f;
+    g[s] = q + G::NQ * s < nrows ? __ldcg(a.lr.row_gate + m0 + q + G::NQ * s) : 0.f;
 }
 
 // ---------------------------------------------------------------------------
 // q|k|v: grid ((H + 2 Hkv) hd / 128, row groups), GeoQkv::THREADS threads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs a) {
+// At most 128 registers a thread: two of its warps and two attention warps
+// (128 each) fill one SM sub-partition's 16,384 registers, so the attention
+// starts beside this kernel.
+__global__ void __maxnreg__(128) epi_qkv_kernel(const EpiArgs a) {
   typedef GeoQkv G;
   constexpr int C = 4;
   __shared__ float s_inv[G::RG];
@@ -358,7 +378,7 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
-  if (!row_group<G>(a, &m0, &nrows)) return;
+  if (!row_group<G>(a, &m0, &nrows)) { dep_signal(a.done); return; }
   const int q = threadIdx.x % G::NQ, col = threadIdx.x / G::NQ;
   const int n = nt * TC_BM + col;
   const int qcols = a.H * a.hd, kcols = a.Hkv * a.hd;
@@ -371,27 +391,21 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
   const int seg = a.lora ? lora_seg(a.lr, nt * TC_BM) : 0;
   BFrag B;
   if (a.lora) bfrag_issue(a, seg, nt * TC_BM + 16 * (threadIdx.x >> 5) - a.lr.seg_n0[seg], B);
-  pdl_wait();
-
-  // ---- every global load first
+  // The row tables, the row gates and the page table are complete before
+  // this kernel starts (the pass's first kernel after build_rows waits for
+  // it before letting the next one launch): positions, slots, RoPE entries
+  // and KV pages are fetched while the GEMM before still runs.  Loads before
+  // the wait bypass L1 (ld.global.cg), which may still hold lines of an
+  // earlier pass until the dependency wait.
   int pos[G::RPT], slot[G::RPT];
 #pragma unroll
   for (int s = 0; s < G::RPT; ++s) {
     const int j = q + G::NQ * s;
-    pos[s] = j < nrows ? a.row_pos[m0 + j] : 0;
-    slot[s] = (j < nrows && kv_tile) ? a.row_slot[m0 + j] : 0;
+    pos[s] = j < nrows ? __ldcg(a.row_pos + m0 + j) : 0;
+    slot[s] = (j < nrows && kv_tile) ? __ldcg(a.row_slot + m0 + j) : 0;
   }
-  SsLoad<G> ssv;
-  ss_issue(a, m0, nrows, ssv);
-  PartLoad<G, C> LU, LP;
   float gate[G::RPT];
-  if (a.lora) {
-    u_issue(a, seg, m0, nrows, col, q, LU);
-    gate_issue<G>(a, m0, nrows, q, gate);
-  }
-  part_issue(a.pv, nt, m0, nrows, col, q, LP);
-  // second round, addressed by the rows' positions and slots: RoPE table
-  // entries and the KV pages
+  if (a.lora) gate_issue<G>(a, m0, nrows, q, gate);
   float cs[G::RPT], sn[G::RPT];
   int page[G::RPT], pok[G::RPT];
 #pragma unroll
@@ -404,6 +418,14 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
     page[s] = (j < nrows && kv_tile) ? a.kv.page_of(slot[s], pos[s], ok) : 0;
     pok[s] = ok;
   }
+  epi_wait(a);
+
+  // ---- every load of what the GEMM (and the residual kernel before it) wrote
+  SsLoad<G> ssv;
+  ss_issue(a, m0, nrows, ssv);
+  PartLoad<G, C> LU, LP;
+  if (a.lora) u_issue(a, seg, m0, nrows, col, q, LU);
+  part_issue(a.pv, nt, m0, nrows, col, q, LP);
 
   // ---- then the arithmetic
   if (a.lora) u_store(LU, nrows, col, q, sUh, sUl);
@@ -455,6 +477,7 @@ __global__ void __launch_bounds__(GeoQkv::THREADS) epi_qkv_kernel(const EpiArgs 
       }
     }
   }
+  dep_signal(a.done);   // q rows and K/V rows stored (the attention waits on it)
 }
 
 // ---------------------------------------------------------------------------
@@ -533,6 +556,11 @@ __global__ void __launch_bounds__(RESID_THREADS) epi_resid_kernel(const EpiArgs 
   __shared__ __align__(16) bf16 sUh[16 * EPI_UP];
   __shared__ __align__(16) bf16 sUl[16 * EPI_UP];
   __shared__ __align__(16) float sDot[G::RG * TC_BM];
+  // The layer-0 input preparation is the pass's first kernel after
+  // build_rows: it lets the next kernel launch only after build_rows has
+  // completed, so every later kernel of the pass may read the row tables
+  // before its own wait.
+  if (a.prep) pdl_wait();
   pdl_trigger();
   const int nt = blockIdx.x;
   int m0, nrows;
@@ -553,18 +581,19 @@ __global__ void __launch_bounds__(RESID_THREADS) epi_resid_kernel(const EpiArgs 
   }
   BFrag B;
   if (lora && warp < 8) bfrag_issue(a, 0, nt * TC_BM + 16 * warp, B);
-  pdl_wait();
+  // the row gate (build_rows' table, complete before this kernel starts;
+  // read through L2: L1 may hold an earlier pass's line before the wait)
+  const float gt = (lora && live) ? __ldcg(a.lr.row_gate + m0 + j) : 0.f;
+  epi_wait(a);
 
   // ---- every global load first
   const size_t xi = (size_t)(m0 + j) * a.d + n;
-  float4 xv = live ? *reinterpret_cast<const float4*>(a.x + xi) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // through L2, like every load of another kernel's output here: with a
+  // completion counter there is no grid wait to drop stale L1 lines
+  float4 xv = live ? __ldcg(reinterpret_cast<const float4*>(a.x + xi)) : make_float4(0.f, 0.f, 0.f, 0.f);
   if (!a.prep) {
     Part4<C> LU, LP;
-    float gt = 0.f;
-    if (lora) {
-      part4_issue(a.pv, a.lr.u_tile0, m0, j, c0, live, LU);
-      gt = live ? __ldg(a.lr.row_gate + m0 + j) : 0.f;
-    }
+    if (lora) part4_issue(a.pv, a.lr.u_tile0, m0, j, c0, live, LU);
     part4_issue(a.pv, nt, m0, j, c0, live, LP);
     // ---- then the arithmetic
     if (lora) {
@@ -632,7 +661,10 @@ __global__ void __launch_bounds__(RESID_THREADS, 2) epi_swiglu_kernel(const EpiA
     bfrag_issue(a, 0, fw, B);
     bfrag_prefetch(a, 1, fw);
   }
-  pdl_wait();
+  // the row gate (build_rows' table, complete before this kernel starts;
+  // read through L2: L1 may hold an earlier pass's line before the wait)
+  const float gt = (lora && live) ? __ldcg(a.lr.row_gate + m0 + j) : 0.f;
+  epi_wait(a);
 
   // ---- every global load first
   float ss0 = 0.f, ss1 = 0.f;
@@ -642,13 +674,11 @@ __global__ void __launch_bounds__(RESID_THREADS, 2) epi_swiglu_kernel(const EpiA
     if (lane + 32 < a.n_ss) ss1 = __ldcg(sr + lane + 32);
   }
   Part4<C> LG, LUp, L0, L1;
-  float gt = 0.f;
   part4_issue(a.pv, ft, m0, j, c0, live, LG);
   part4_issue(a.pv, ut, m0, j, c0, live, LUp);
   if (lora) {
     part4_issue(a.pv, a.lr.u_tile0, m0, j, c0, live, L0);
     part4_issue(a.pv, a.lr.u_tile0 + 1, m0, j, c0, live, L1);
-    gt = live ? __ldg(a.lr.row_gate + m0 + j) : 0.f;
   }
   // ---- then the arithmetic
   float inv = 1.f;

@@ -47,6 +47,7 @@ struct GemmParams {
   unsigned long long dep_limit_ns;   // the counter wait gives up after this long
   // EPI_STORE_F32: element offset of each output row (null: row * ldo)
   const int64_t* out_row;
+  unsigned* done;                    // tensor-core DUMP mode: completion counter (see TcParams)
 };
 
 template <typename T, int MT, int NC>

@@ -73,6 +73,9 @@ struct TcParams {
   const unsigned* dep; unsigned dep_count;
   unsigned long long dep_limit_ns;   // give up the counter wait after this long
   const int64_t* out_row;            // EPI_STORE_F32: element offset of each output row (null: m * ldo)
+  // DUMP mode: completion counter every CTA adds to once its parts are
+  // stored (the epilogue kernel after it waits on it), or null
+  unsigned* done;
 };
 
 // ---------------------------------------------------------------------------
@@ -420,6 +423,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (*s_abort && threadIdx.x == 0) raise_status(p.status, ST_GEMM_TIMEOUT);
+  if (DUMP) dep_signal_synced(p.done);   // every part of this CTA is stored
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),

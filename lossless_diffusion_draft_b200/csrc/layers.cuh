@@ -33,7 +33,7 @@ struct KvLayout {
   __device__ __forceinline__ int page_of(int slot, int pos, int& ok) const {
     const int pi = pos / KV_PAGE;
     ok = (pos >= 0 && pi < pages_per_req);
-    return ok ? page_table[(size_t)slot * pages_per_req + pi] : 0;
+    return ok ? __ldcg(page_table + (size_t)slot * pages_per_req + pi) : 0;
   }
   __device__ __forceinline__ size_t offset_in_page(int layer, int page, int pos, int plane,
                                                    int head) const {
@@ -77,8 +77,8 @@ struct RowKeys {
   const int32_t* blk;     // [M] noised block start, -1 for a clean row (null: all clean)
   __device__ __forceinline__ void ranges(const int32_t* row_pos, int r, int& lim, int& lo2,
                                          int& hi2) const {
-    const int pos = row_pos[r];
-    const int b = blk ? blk[r] : -1;
+    const int pos = __ldcg(row_pos + r);
+    const int b = blk ? __ldcg(blk + r) : -1;
     lim = b < 0 ? pos + 1 : b;
     lo2 = b < 0 ? 0 : b;
     hi2 = b < 0 ? 0 : pos + 1;
@@ -87,12 +87,12 @@ struct RowKeys {
   // their ranges, in pages of `page` keys.
   __device__ __forceinline__ KeyTiles tiles(const int32_t* row_pos, const int32_t* row_slot,
                                             int row0, int ntok, int page, int pages_per_req) const {
-    KeyTiles t{cslot ? cslot[row0] : row_slot[row0], 0, -1, 0, 0, false};
+    KeyTiles t{__ldcg((cslot ? cslot : row_slot) + row0), 0, -1, 0, 0, false};
     int lim1 = 0, lo2 = 0x7fffffff, hi2 = 0;
     if (!blk) {
       // causal by position: a request's rows are in position order, so the
       // last row reaches furthest (one load on the decode passes' path)
-      lim1 = row_pos[row0 + ntok - 1] + 1;
+      lim1 = __ldcg(row_pos + row0 + ntok - 1) + 1;
       ntok = 0;
     }
     for (int k = 0; k < ntok; ++k) {
@@ -102,7 +102,7 @@ struct RowKeys {
       if (h2 > l2) {
         lo2 = min(lo2, l2);
         hi2 = max(hi2, h2);
-        t.slot2 = row_slot[row0 + k];
+        t.slot2 = __ldcg(row_slot + row0 + k);
       }
     }
     t.n1 = (lim1 + page - 1) / page;

@@ -92,6 +92,20 @@ cudaError_t smem_attr_once(K kernel, int bytes, bool* done) {
   return e;
 }
 
+// The fused pass's small kernels prefer the largest shared-memory carveout:
+// an SM running one of them then takes a GEMM or attention CTA (200+ KB)
+// beside it without reconfiguring.
+template <typename K>
+void carveout_once(K kernel, bool* done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  if (dev >= 0 && dev < ATTR_DEVS && done[dev]) return;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && dev >= 0 && dev < ATTR_DEVS) done[dev] = true;
+  else cudaGetLastError();   // a preference only: leave no error behind
+}
+
 // Launch with programmatic stream serialisation when `pdl`: the kernel may
 // start while the previous kernel of the stream is still running; inside,
 // pdl_wait() orders every access to data an earlier kernel wrote.
@@ -277,6 +291,7 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   tp.dep_count = p.dep_count;
   tp.dep_limit_ns = p.dep_limit_ns ? p.dep_limit_ns : DEP_WAIT_NS;
   tp.out_row = p.out_row;
+  tp.done = DUMP ? p.done : nullptr;
 
   using Cfg = TcCfg<NT, SPLIT, KPS>;
   static bool attr[ATTR_DEVS] = {};
@@ -600,9 +615,18 @@ int launch_attn_hd(uno_ctx* c, AttnParams& p, int n_req, cudaStream_t st) {
   return UNO_OK;
 }
 
+// Completion counters around the tensor-core attention of the fused pass:
+// the q|k|v epilogue's (dep, its CTA count) and one the attention CTAs add
+// to, which the split merge waits on.
+struct AttnSync {
+  const unsigned* dep = nullptr;
+  unsigned dep_n = 0;
+  unsigned* done = nullptr;
+};
+
 template <int HD>
 int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                   void* out_lo, const void* l2_pf, size_t l2_pf_bytes) {
+                   void* out_lo, const void* l2_pf, size_t l2_pf_bytes, const AttnSync& sync) {
   const uno_shape& s = c->s;
   AttnTcParams p{};
   p.q = (const f16*)c->qbuf;
@@ -639,6 +663,10 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
   const bool pf_ok = l2_pf && l2_pf_bytes >= 16 && ((uintptr_t)l2_pf & 15) == 0;
   p.l2_pf = pf_ok ? (const char*)l2_pf : nullptr;
   p.l2_pf_bytes = pf_ok ? (unsigned long long)(l2_pf_bytes & ~(size_t)15) : 0ull;
+  p.dep = sync.dep;
+  p.dep_count = sync.dep ? sync.dep_n + c->dep_extra : 0u;
+  p.dep_limit_ns = c->dep_limit_ns;
+  p.done = S > 1 ? sync.done : nullptr;
   static bool attr[ATTR_DEVS] = {};
   CK(smem_attr_once(attn_tc_kernel<HD>, AtcCfg<HD>::SMEM, attr));
   {
@@ -651,6 +679,11 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
     Prof prof(c, UNO_K_ATTN, 0.0);
     // only the rows a query tile can hold: tokens per request x heads per kv head
     const int rows = std::min(ATC_QROWS, rows_per_req * G);
+    if (p.done) {
+      p.dep = p.done;
+      p.dep_count = (unsigned)(S * groups) + c->dep_extra;
+      p.done = nullptr;
+    }
     klaunch(c->genv.pdl, c->stream, dim3(ceil_div(rows, ATC_MERGE_ROWS), groups),
             dim3(HD, ATC_MERGE_ROWS), 0, attn_merge_kernel<HD>, p);
   }
@@ -661,14 +694,18 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
 // tensor-core attention while it runs.
 template <typename T>
 int launch_attn(uno_ctx* c, int layer, int n_req, int rows_per_req, bool decode,
-                void* out_lo, const void* l2_pf = nullptr, size_t l2_pf_bytes = 0) {
+                void* out_lo, const void* l2_pf = nullptr, size_t l2_pf_bytes = 0,
+                const AttnSync& sync = AttnSync{}) {
   const uno_shape& s = c->s;
   if (c->kv_map_ok) {
     if (s.head_dim == 128)
-      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes);
+      return launch_attn_tc<128>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes,
+                                 sync);
     if (s.head_dim == 64)
-      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes);
+      return launch_attn_tc<64>(c, layer, n_req, rows_per_req, decode, out_lo, l2_pf, l2_pf_bytes,
+                                sync);
   }
+  // the SIMT attention waits on the grid dependency (sync unused)
   AttnParams p{};
   p.qkv = c->qbuf;
   p.q_lo = sizeof(T) == 2 ? (const char*)c->qbuf + (size_t)c->M_max * s.n_heads * s.head_dim * 2
@@ -938,9 +975,11 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   ra.x = c->x;
   ra.status = c->d_status;
   ra.prefill_pos0 = prefill_pos0;
-  // completion counters: each GEMM waits for the kernel right before it
-  // (its X rows) through a counter that kernel's CTAs add to; the counters
-  // are zeroed by build_rows
+  // completion counters: each GEMM waits for the epilogue before it (its X
+  // rows), each epilogue for its GEMM (the parts), the attention for the
+  // q|k|v epilogue and the split merge for the attention, each through a
+  // counter the producer's CTAs add to at their end; the o GEMM alone waits
+  // on the grid dependency.  The counters are zeroed by build_rows.
   const bool csync = c->counter_sync && c->dep_ctr;
   int n_ctr = 0;
   const unsigned* dep = nullptr;   // counter of the last signalling kernel
@@ -1015,7 +1054,7 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     g.p.dep = dep;
     g.p.dep_count = dep ? dep_n + c->dep_extra : dep_n;
     g.p.dep_limit_ns = c->dep_limit_ns;
-    dep = nullptr;
+    g.p.done = next_ctr();
     DumpShape sh;
     {
       Prof prof(c, UNO_K_GEMM, gemm_bytes(g.p, 2) - (double)M * g.p.N * 2, M, g.p.N, K, 0);
@@ -1024,6 +1063,8 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     }
     *pv = PartView{c->genv.part, sh.NT, sh.units, sh.grid, sh.KBt, sh.m_tiles};
     ea.lr.u_tile0 = n_base / TC_BM;
+    dep = g.p.done;
+    dep_n = (unsigned)sh.grid;
     return UNO_OK;
   };
   auto set_lora = [&](std::initializer_list<std::pair<const void*, int>> b) {
@@ -1039,16 +1080,25 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
   };
   // one epilogue launch: rg rows per CTA (row groups inside the GEMM's
   // m-tiles), `threads` threads
-  // `signal`: the next kernel is a GEMM that waits on this one's counter
+  // `signal`: the next kernel waits on this one's counter
   auto epi = [&](void (*kernel)(const EpiArgs), int tiles, int rg, int threads, bool signal) {
     Prof prof(c, UNO_K_OTHER, 0.0);
     const int groups = ea.pv.m_tiles * epi_groups_per_tile(ea.pv.NT, M, rg);
+    ea.dep = dep;
+    ea.dep_count = dep ? dep_n + c->dep_extra : 0u;
+    ea.dep_limit_ns = c->dep_limit_ns;
     ea.done = signal ? next_ctr() : nullptr;
     dep = ea.done;
     dep_n = (unsigned)(tiles * groups);
     klaunch(pdl, st, dim3(tiles, groups), dim3(threads), 0, kernel, ea);
   };
 
+  {
+    static bool co_qkv[ATTR_DEVS] = {}, co_resid[ATTR_DEVS] = {}, co_swiglu[ATTR_DEVS] = {};
+    carveout_once(epi_qkv_kernel, co_qkv);
+    carveout_once(epi_resid_kernel, co_resid);
+    carveout_once(epi_swiglu_kernel, co_swiglu);
+  }
   // layer-0 input: g * x and the sums of squares of the embedding rows
   ea.prep = 1;
   ea.lora = 0;
@@ -1067,14 +1117,18 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     set_lora({{c->lB[UNO_PROJ_Q][l], H * hd}, {c->lB[UNO_PROJ_K][l], Hkv * hd},
               {c->lB[UNO_PROJ_V][l], Hkv * hd}});
     ea.ss = c->ss;
-    epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS, false);
+    epi(epi_qkv_kernel, qkv_n / TC_BM, GeoQkv::RG, GeoQkv::THREADS, true);
 
     // the o GEMM waits for the attention merge with the grid wait (its CTAs
     // start only as the attention CTAs leave the SMs; measured, a counter
     // poll completed later); while the attention streams K/V, its idle lanes
     // pull W_o into L2
+    AttnSync as;
+    as.dep = dep;
+    as.dep_n = dep_n;
+    as.done = next_ctr();
     rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo,
-                           c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2);
+                           c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2, as);
     if (rc) return rc;
     dep = nullptr;
 
@@ -1255,7 +1309,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
   if (dalloc(&c->row_cslot, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->row_blk, (size_t)M * 4) != cudaSuccess) return oom("rows");
   if (dalloc(&c->train_slots, (size_t)2 * max_batch * 4) != cudaSuccess) return oom("rows");
-  c->n_dep_ctr = 4 * s.n_layers + 8;
+  c->n_dep_ctr = 10 * s.n_layers + 8;
   if (dalloc(&c->dep_ctr, (size_t)c->n_dep_ctr * 4) != cudaSuccess) return oom("counters");
   cudaMemset(c->dep_ctr, 0, (size_t)c->n_dep_ctr * 4);
 
