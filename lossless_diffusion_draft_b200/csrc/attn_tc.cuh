@@ -28,7 +28,7 @@
 // With several key splits each CTA writes (m, l, O) partials and
 // attn_merge_kernel (ATC_MERGE_ROWS query rows per CTA) adds them in split
 // order.  Every wait is bounded.  While it runs, idle lanes of the producer
-// warp prefetch the next projection's weights into L2.
+// warp prefetch part of the next projection's weights into L2.
 #pragma once
 
 #include "layers.cuh"
@@ -191,8 +191,8 @@ __global__ void __maxnreg__(128)
   // With a completion counter (the fused pass) the row tables and the page
   // table are complete when this kernel starts: the pass's first kernel after
   // build_rows lets the next one launch only once build_rows has completed.
-  // The key list and its pages are then set up, and the cached pages that no
-  // row of this pass writes start loading, while the q|k|v epilogue still
+  // The key list and its pages are then set up, and the split's first page,
+  // if no row of this pass writes it, starts loading while the q|k|v epilogue still
   // runs (the table loads go through L2: before the dependency wait L1 may
   // still hold an earlier pass's lines).  Without a counter everything
   // follows the grid dependency.
@@ -238,7 +238,8 @@ __global__ void __maxnreg__(128)
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) lowest = min(lowest, __shfl_xor_sync(0xffffffffu, lowest, o));
-      n_safe = max(0, min(min(n, C::STAGES), lowest / ATC_KT - t_begin));
+      // one page: loading more of them early slowed the epilogue beside it
+      n_safe = max(0, min(min(n, 1), lowest / ATC_KT - t_begin));
     }
   }
   tc_fence_before();

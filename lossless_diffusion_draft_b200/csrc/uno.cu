@@ -1122,13 +1122,15 @@ int forward_fused(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32
     // the o GEMM waits for the attention merge with the grid wait (its CTAs
     // start only as the attention CTAs leave the SMs; measured, a counter
     // poll completed later); while the attention streams K/V, its idle lanes
-    // pull W_o into L2
+    // pull the first half of W_o into L2 (measured per step at 5120: all of
+    // it 8.47 ms, half 8.39, a quarter 8.40, none 8.42: more prefetch traffic
+    // slows the epilogue and attention beside it more than it saves)
     AttnSync as;
     as.dep = dep;
     as.dep_n = dep_n;
     as.done = next_ctr();
     rc = launch_attn<bf16>(c, l, n_req, rows_per_req, kind != PASS_PREFILL, attn_lo,
-                           c->w[UNO_PROJ_O][l], (size_t)d * hhd * 2, as);
+                           c->w[UNO_PROJ_O][l], (size_t)d * hhd, as);
     if (rc) return rc;
     dep = nullptr;
 
