@@ -28,6 +28,20 @@ SAMPLE_TOL = 1e-5
 ACCEPT_TOL = 1e-5
 
 
+def near_tie_budget(positions):
+    """How many traced near-tie disagreements a run may have.
+
+    Each one is already held to a margin below SAMPLE_TOL / ACCEPT_TOL; the
+    count only guards against a systematic bias.  The GPU's fp32 prefix sums
+    put a CDF boundary within about 1e-7 of Z of the exact one, so a draw
+    flips at a rate of about (number of boundaries) x 1e-7: ~3e-3 per draw
+    on the near-flat 32000-token rows of the random-init small model.  A
+    bias of the size of one fp32 rounding per boundary would flip tens of
+    times more often than that.
+    """
+    return 2 + positions // 100
+
+
 @dataclass
 class Tally:
     positions: int = 0
