@@ -62,6 +62,13 @@ struct TcParams {
   int n_tiles, m_tiles;
   int nseg; TcSeg seg[TC_MAX_SEG];
   int units, grid;           // stream-K: units = tiles * (KB + RB), split over grid CTAs
+  // m-tile groups (0: none).  With several token m-tiles, grid = mgroups *
+  // m_tiles: CTA b takes m-tile b % m_tiles, and the mgroups groups split the
+  // units of one m-tile's row of tiles (n_tiles * (KB + RB)) stream-K style,
+  // so the CTAs of a group read the same weight k-blocks at about the same
+  // time (one from HBM, the rest from L2) instead of every CTA re-reading its
+  // own weight tile once per m-tile.  Not in DUMP mode.
+  int mgroups;
   int max_parts;             // partial slots per tile
   int epi; void* out; int ldo; float alpha; const float* row_gate;
   float* ws; unsigned* counters;   // DUMP: ws holds the part slots [tiles + grid][NT][128]
@@ -159,8 +166,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KBt = p.KB + p.RB;
-  const int u0 = sk_start(blockIdx.x, p.units, p.grid);
-  const int u1 = sk_start(blockIdx.x + 1, p.units, p.grid);
+  // the split this CTA belongs to (units are virtual with m-tile groups: the
+  // k-blocks of one row of tiles, this CTA's m-tile fixed)
+  const bool grp = !DUMP && p.mgroups > 0;
+  const int mt_fix = grp ? (int)blockIdx.x % p.m_tiles : 0;
+  const int me = grp ? (int)blockIdx.x / p.m_tiles : (int)blockIdx.x;
+  const int nsplit = grp ? p.mgroups : p.grid;
+  const int vunits = grp ? p.n_tiles * KBt : p.units;
+  const int u0 = sk_start(me, vunits, nsplit);
+  const int u1 = sk_start(me + 1, vunits, nsplit);
+  auto tile_of = [&](int u) { return grp ? (u / KBt) * p.m_tiles + mt_fix : u / KBt; };
 
   // unit u is k-block u % KBt of tile u / KBt; issue i = u - u0 uses
   // ring stage i % STAGES
@@ -172,7 +187,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   };
   // weight tile of unit u: W, then LoRA-B
   auto coords_a = [&](int u, const CUtensorMap*& map, int& x, int& y) {
-    const int t = u / KBt, kb = u % KBt;
+    const int t = tile_of(u), kb = u % KBt;
     const int n_row = (t / p.m_tiles) * TC_BM;
     const int sg = seg_of(n_row);
     map = kb < p.KB ? &maps.w[sg] : &maps.b[sg];
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
 
   auto load_b = [&](int u, int stage) {     // activations: X, then U (hi, lo)
-    const int t = u / KBt, kb = u % KBt;
+    const int t = tile_of(u), kb = u % KBt;
     const int mt = t % p.m_tiles;
 #pragma unroll
     for (int j = 0; j < KPS; ++j) {
@@ -326,7 +341,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int n_local = warp * 32 + lane;
     int part = 0;
     for (int u = u0; u < u1; ++part) {
-      const int t = u / KBt, kb0 = u % KBt;
+      const int t = tile_of(u), kb0 = u % KBt;
       const int kb1 = min(KBt, kb0 + (u1 - u));
       u += kb1 - kb0;
       const int buf = part & 1;
@@ -373,8 +388,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (!DUMP && !whole) {
         __threadfence();
         epi_bar();
-        const int first = sk_owner(t * KBt, p.units, p.grid);
-        const int last = sk_owner(t * KBt + KBt - 1, p.units, p.grid);
+        // the tile's contributors: split positions first..last (CTA
+        // first * m_tiles + mt_fix .. with m-tile groups)
+        const int vt0 = grp ? (t / p.m_tiles) * KBt : t * KBt;   // its first virtual unit
+        const int first = sk_owner(vt0, vunits, nsplit);
+        const int last = sk_owner(vt0 + KBt - 1, vunits, nsplit);
         if (threadIdx.x == 0) {
           const unsigned done = atomicAdd(&p.counters[t], 1u);
           const bool is_last = (done == (unsigned)(last - first));
@@ -399,8 +417,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int i = i0 + c;
                 const float* src = nullptr;
                 if (i <= last) {
-                  const int slot = (sk_start(i, p.units, p.grid) >= t * KBt) ? 0 : 1;
-                  src = tc_slot(p.ws, i, slot, NT) + (size_t)m * TC_BM + n_local;
+                  const int slot = (sk_start(i, vunits, nsplit) >= vt0) ? 0 : 1;
+                  const int cta = grp ? i * p.m_tiles + mt_fix : i;
+                  src = tc_slot(p.ws, cta, slot, NT) + (size_t)m * TC_BM + n_local;
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j)

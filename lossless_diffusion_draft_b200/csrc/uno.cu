@@ -271,6 +271,18 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   // at least TC_MIN_UNITS k-blocks per CTA: a tile is then cut into few
   // parts and its last contributor has few partials to add
   tp.grid = std::max(1, std::min(env.sm_count, tp.units / TC_MIN_UNITS));
+  // several token m-tiles (max batch, prefill chunks): groups of m_tiles CTAs
+  // that read each weight k-block together (measured at M = 1360 without
+  // them: every CTA re-read its weight tile from HBM once per m-tile, 11x
+  // the weight bytes)
+  tp.mgroups = 0;
+  if (!DUMP && tp.m_tiles >= 2) {
+    const int g = std::min(env.sm_count / tp.m_tiles, tp.n_tiles * (tp.KB + tp.RB) / TC_MIN_UNITS);
+    if (g >= 1) {
+      tp.mgroups = g;
+      tp.grid = g * tp.m_tiles;
+    }
+  }
   tp.max_parts = 2;
   tp.epi = p.epi;
   tp.out = p.out;

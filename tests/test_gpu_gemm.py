@@ -56,6 +56,8 @@ def _run(M, N, K, r, dtype, seed=0, cols=None, repeat=1):
     (300, 640, 512, 128),      # two token tiles
     (17, 12288, 4096, 128),    # gate/up width
     (5, 4096, 12288, 128),     # down-projection depth (many k-blocks per tile)
+    (1360, 4224, 4096, 128),   # max-batch rows: six token tiles in m-tile groups, tiles cut
+    (600, 24832, 512, 128),    # three token tiles across a wide row of weight tiles
 ])
 def test_bf16_tensor_core(M, N, K, r):
     before = uno.uno_debug_launch_counts()
@@ -88,8 +90,9 @@ def test_bf16_fallback_shape():
     assert err <= 2e-3 * ref.abs().max().item() + 1e-4, err
 
 
-def test_deterministic_and_workspace_left_zero():
-    _, _, outs, ws = _run(17, 4096, 4096, 128, torch.bfloat16, repeat=3)
+@pytest.mark.parametrize("M", [17, 1360])
+def test_deterministic_and_workspace_left_zero(M):
+    _, _, outs, ws = _run(M, 4096, 4096, 128, torch.bfloat16, repeat=3)
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
     assert int(ws[: (1 << 16) * 4].count_nonzero()) == 0   # counters left zeroed
