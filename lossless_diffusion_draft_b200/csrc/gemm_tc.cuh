@@ -144,6 +144,30 @@ __device__ __forceinline__ void tc_store(const TcParams& p, int m, int n, float 
   }
 }
 
+// Rows m0 .. m0 + R - 1 of column n (rows past mrows or a column past N are
+// skipped).  The residual-add epilogue reads all R old values before it
+// writes any: the compiler cannot tell the rows' addresses apart, and would
+// otherwise serialise R load / store round trips.
+template <int R>
+__device__ __forceinline__ void tc_store_rows(const TcParams& p, int m0, int mrows, int n,
+                                              const float (&v)[R]) {
+  if (n >= p.N) return;
+  if (p.epi == EPI_ADD_F32) {
+    float* out = reinterpret_cast<float*>(p.out);
+    float old[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      old[i] = i < mrows ? __ldcg(out + (size_t)(m0 + i) * p.ldo + n) : 0.f;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      if (i < mrows) out[(size_t)(m0 + i) * p.ldo + n] = old[i] + v[i];
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+    if (i < mrows) tc_store(p, m0 + i, n, v[i]);
+}
+
 template <int NT, bool SPLIT, bool DUMP, int KPS>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
@@ -373,9 +397,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int i = 0; i < 16; ++i) v[i] += vl[i];
         }
         if (whole) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < mrows && n < p.N) tc_store(p, m0 + c0 + i, n, v[i]);
+          tc_store_rows<16>(p, m0 + c0, mrows - c0, n, v);
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -430,9 +452,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] += v[c][j];
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (m + j < mrows && n < p.N) tc_store(p, m0 + m + j, n, acc[j]);
+            tc_store_rows<8>(p, m0 + m, mrows - m, n, acc);
           }
         }
         epi_bar();   // s_last is reused by the next cut part
