@@ -504,8 +504,6 @@ __global__ void __maxnreg__(128)
 // Registers stay small enough (rows x head_dim threads) that a GEMM CTA of
 // the next projection fits on the same SM and starts its weight stream.
 constexpr int ATC_MAX_SPLITS = 24;
-constexpr int ATC_WAVE_SPLITS = 4;   // most key splits when the groups alone fill the SMs
-constexpr int ATC_CTA_PAGES = 3;     // a CTA's fixed cost (set-up, pipeline fill) in pages
 constexpr int ATC_MERGE_ROWS = 2;
 template <int HD>
 __global__ void __launch_bounds__(HD * ATC_MERGE_ROWS) attn_merge_kernel(const AttnTcParams p) {

@@ -325,58 +325,68 @@ __global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* ga
 // cos/sin come from a table [max_pos][head_dim / 2] computed on the host in
 // double precision.
 template <typename T>
-__global__ void rope_kv_kernel(const float* qkv, int ld_qkv, typename KvOf<T>::type* q_out,
-                               typename KvOf<T>::type* q_lo, int ld_q,
-                               const int32_t* row_pos, const int32_t* row_slot, const float* cos_t,
-                               const float* sin_t, int max_pos, int H, int Hkv, int hd, KvLayout kv,
-                               int layer, int32_t* status) {
-  // grid (rows, H + 2 Hkv heads of the fused q|k|v row), hd / 2 threads: one
-  // rotate-half pair (i, i + hd/2) per thread
+__global__ void __launch_bounds__(256) rope_kv_kernel(const float* qkv, int ld_qkv,
+                                                      typename KvOf<T>::type* q_out,
+                                                      typename KvOf<T>::type* q_lo, int ld_q,
+                                                      const int32_t* row_pos, const int32_t* row_slot,
+                                                      const float* cos_t, const float* sin_t,
+                                                      int max_pos, int H, int Hkv, int hd,
+                                                      KvLayout kv, int layer, int32_t* status) {
+  // one CTA per row: thread t takes the rotate-half pairs (i, i + hd/2) of
+  // pair index t, t + blockDim.x, ... over the row's H + 2 Hkv heads
+  // (consecutive threads, consecutive i: coalesced loads and stores).  One
+  // CTA per (row, head) of hd / 2 threads had made a max-batch pass (1360
+  // rows x 48 heads) bound by the launch of its 65k CTAs.
   typedef typename KvOf<T>::type KV;
   pdl_trigger();
   pdl_wait();
-  const int row = blockIdx.x, h = blockIdx.y, i = threadIdx.x;
+  const int row = blockIdx.x;
   const int half = hd / 2;
   const int pos = row_pos[row], slot = row_slot[row];
   const int ok_pos = pos < max_pos;
   const int pc = ok_pos ? pos : 0;
-  const float* src = qkv + (size_t)row * ld_qkv + (size_t)h * hd;
-  const float x1 = src[i], x2 = src[i + half];
-  if (h < H + Hkv) {
-    const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
-    const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
-    if (h < H) {
-      const size_t qi = (size_t)row * ld_q + (size_t)h * hd;
-      const KV a1 = from_f<KV>(y1), a2 = from_f<KV>(y2);
-      q_out[qi + i] = a1;
-      q_out[qi + i + half] = a2;
-      if (q_lo) {   // rounding residual (the attention adds q_hi K + q_lo K)
-        q_lo[qi + i] = from_f<KV>(y1 - to_f(a1));
-        q_lo[qi + i + half] = from_f<KV>(y2 - to_f(a2));
+  const float* rsrc = qkv + (size_t)row * ld_qkv;
+  const int pairs = (H + 2 * Hkv) * half;
+  for (int pi = threadIdx.x; pi < pairs; pi += blockDim.x) {
+    const int h = pi / half, i = pi - h * half;
+    const float* src = rsrc + (size_t)h * hd;
+    const float x1 = src[i], x2 = src[i + half];
+    if (h < H + Hkv) {
+      const float c = cos_t[(size_t)pc * half + i], s = sin_t[(size_t)pc * half + i];
+      const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
+      if (h < H) {
+        const size_t qi = (size_t)row * ld_q + (size_t)h * hd;
+        const KV a1 = from_f<KV>(y1), a2 = from_f<KV>(y2);
+        q_out[qi + i] = a1;
+        q_out[qi + i + half] = a2;
+        if (q_lo) {   // rounding residual (the attention adds q_hi K + q_lo K)
+          q_lo[qi + i] = from_f<KV>(y1 - to_f(a1));
+          q_lo[qi + i + half] = from_f<KV>(y2 - to_f(a2));
+        }
+      } else {
+        int ok;
+        const size_t off = kv.offset(layer, slot, pos, 0, h - H, ok);
+        if (ok && ok_pos) {
+          KV* dst = reinterpret_cast<KV*>(kv.pool) + off;
+          const KV b1 = from_f<KV>(y1), b2 = from_f<KV>(y2);
+          dst[i] = b1;
+          dst[i + half] = b2;
+          if (kv.n_planes == 3) {   // K lo plane
+            dst[kv.plane_stride() + i] = from_f<KV>(y1 - to_f(b1));
+            dst[kv.plane_stride() + i + half] = from_f<KV>(y2 - to_f(b2));
+          }
+        } else if (i == 0) {
+          raise_status(status, ST_POS_OVERFLOW);
+        }
       }
     } else {
       int ok;
-      const size_t off = kv.offset(layer, slot, pos, 0, h - H, ok);
+      const size_t off = kv.offset(layer, slot, pos, kv.v_plane(), h - H - Hkv, ok);
       if (ok && ok_pos) {
         KV* dst = reinterpret_cast<KV*>(kv.pool) + off;
-        const KV b1 = from_f<KV>(y1), b2 = from_f<KV>(y2);
-        dst[i] = b1;
-        dst[i + half] = b2;
-        if (kv.n_planes == 3) {   // K lo plane
-          dst[kv.plane_stride() + i] = from_f<KV>(y1 - to_f(b1));
-          dst[kv.plane_stride() + i + half] = from_f<KV>(y2 - to_f(b2));
-        }
-      } else if (i == 0) {
-        raise_status(status, ST_POS_OVERFLOW);
+        dst[i] = from_f<KV>(x1);
+        dst[i + half] = from_f<KV>(x2);
       }
-    }
-  } else {
-    int ok;
-    const size_t off = kv.offset(layer, slot, pos, kv.v_plane(), h - H - Hkv, ok);
-    if (ok && ok_pos) {
-      KV* dst = reinterpret_cast<KV*>(kv.pool) + off;
-      dst[i] = from_f<KV>(x1);
-      dst[i + half] = from_f<KV>(x2);
     }
   }
 }

@@ -667,20 +667,11 @@ int launch_attn_tc(uno_ctx* c, int layer, int n_req, int rows_per_req, bool deco
     // one CTA per SM (shared memory): at most sm_count CTAs, else a second wave
     S = sm / groups;
     S = std::max(1, std::min(std::min(S, c->kv.pages_per_req / 2), ATC_MAX_SPLITS));
-  } else if (decode) {
-    // several waves of one CTA per SM: the split count (<= ATC_WAVE_SPLITS)
-    // whose waves carry the request's pages best, counting a CTA's fixed
-    // cost as ATC_CTA_PAGES pages (the page count is the slot's capacity: the
-    // context is only known on the device).  At 80 requests x 8 kv heads:
-    // 5 waves unsplit, 13 waves of a third of the pages with three splits.
-    const double ppr = c->kv.pages_per_req;
-    double best = 0.0;
-    for (int s2 = 1; s2 <= ATC_WAVE_SPLITS; ++s2) {
-      const double waves = (double)ceil_div(groups * s2, sm);
-      const double t = waves * (ppr / s2 + ATC_CTA_PAGES);
-      if (s2 == 1 || t < best) { best = t; S = s2; }
-    }
   }
+  // With more groups than SMs the attention runs unsplit, in several waves:
+  // splitting to fill the last wave was measured slower at 80 requests (three
+  // splits: 611 us of attention plus 137 us of merge per layer-pass against
+  // 640 us unsplit)
   while (S > 1 && (size_t)groups * S * ATC_QROWS * atc_ws_row(HD) > c->att_ws_floats) --S;
   if (groups > c->att_groups_max) S = 1;
   p.n_splits = S;
@@ -871,7 +862,7 @@ int forward(uno_ctx* c, int kind, int n_req, int rows_per_req, const int32_t* re
       launch_gemm<T>(c, g, st);
     }
     other([&] {
-      klaunch(c->genv.pdl, st, dim3(M, H + 2 * Hkv), dim3(hd / 2), 0, rope_kv_kernel<T>,
+      klaunch(c->genv.pdl, st, dim3(M), dim3(256), 0, rope_kv_kernel<T>,
               (const float*)c->qkv,
               qkv_ld, (typename KvOf<T>::type*)c->qbuf,
               split ? (typename KvOf<T>::type*)c->qbuf + (size_t)c->M_max * hhd : nullptr, hhd,
@@ -1385,7 +1376,7 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
 
   // attention split workspace: groups x splits <= about two waves of CTAs
   c->att_groups_max = max_batch * Hkv * ceil_div(B + 1, ATT_MAXQ / (H / Hkv));
-  c->att_ws_floats = (size_t)(2 * 148 + ATC_WAVE_SPLITS * c->att_groups_max) * ATC_QROWS * atc_ws_row(hd);
+  c->att_ws_floats = (size_t)(2 * 148 + c->att_groups_max) * ATC_QROWS * atc_ws_row(hd);
   if (dalloc(&c->att_ws, c->att_ws_floats * 4) != cudaSuccess) return oom("attention ws");
   if (dalloc(&c->att_counters, (size_t)c->att_groups_max * 4) != cudaSuccess) return oom("attention ws");
   cudaMemset(c->att_counters, 0, (size_t)c->att_groups_max * 4);

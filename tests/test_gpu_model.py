@@ -393,15 +393,6 @@ def test_small_bf16_many_rows_unfused_and_unsplit_attention():
     assert after["tc_gemm"] > before["tc_gemm"] and after["tc_attn"] > before["tc_attn"]
 
 
-def test_small_bf16_many_rows_split_attention_waves():
-    """Attention groups that fill the SMs several times over (40 requests x 4
-    kv heads = 160 groups) with room for 10 pages per slot: the key splits
-    are chosen by waves (two here), so the unfused max-batch path runs split
-    attention and the merge.  Logits, decisions and KV against the oracle."""
-    tally, _, worst = _run("small", 40, 150, 2, 2e-2, 2e-2, False, max_ctx=600)
-    assert tally.mismatches <= parity.near_tie_budget(tally.positions), tally.notes
-
-
 def test_counter_wait_runs_out_and_raises_the_flag():
     """Bounded waits: with every completion-counter target made unreachable
     and a 2 ms limit, each waiting GEMM gives up, raises the device flag and
