@@ -458,6 +458,8 @@ def run_uno(args, rank, world, device):
     cfg = dict(synth.CONFIGS[args.workload])
     if args.layers:
         cfg["n_layers"] = args.layers
+    if args.batch:
+        cfg["batch"] = args.batch
     B, prompt_len, gen = cfg["B"], cfg["prompt_len"], cfg["gen_tokens"]
     pk = peaks()
     params = synth.make_params(cfg, device)
@@ -846,6 +848,9 @@ def main():
     ap.add_argument("--no-graphs", action="store_true", help="no CUDA-graph capture of steps")
     ap.add_argument("--no-counter-sync", action="store_true",
                     help="fused pipeline: GEMMs wait on grid dependencies, not completion counters")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (profiler captures of a max-batch step on "
+                         "fewer layers; the line's config records it)")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small cases for profiler captures; the "
                          "line's config records it)")
