@@ -192,10 +192,10 @@ __global__ void __maxnreg__(128)
   // table are complete when this kernel starts: the pass's first kernel after
   // build_rows lets the next one launch only once build_rows has completed.
   // The key list and its pages are then set up, and the split's first page,
-  // if no row of this pass writes it, starts loading while the q|k|v epilogue still
-  // runs (the table loads go through L2: before the dependency wait L1 may
-  // still hold an earlier pass's lines).  Without a counter everything
-  // follows the grid dependency.
+  // if no row of this pass writes it, starts loading while the q|k|v
+  // epilogue still runs (the table loads go through L2: before the
+  // dependency wait L1 may still hold an earlier pass's lines).  Without a
+  // counter everything follows the grid dependency.
   const bool early = p.dep != nullptr;
   if (!early) pdl_wait();
   const int split = blockIdx.x, qt = blockIdx.y, z = blockIdx.z;
