@@ -205,11 +205,13 @@ int uno_set_graphs(uno_ctx *ctx, int enable);
 int uno_set_pdl(uno_ctx *ctx, int enable);
 
 /* Completion counters in the fused layer pipeline (implementation choice,
- * on by default).  Each projection GEMM then waits for the kernel right
- * before it (the epilogue or attention merge that wrote its input rows)
- * through a counter that kernel's CTAs increment as they finish, instead of
- * waiting for that whole grid to be retired; its weight stream has started
- * before either wait.  The counters are zeroed by each pass's first kernel.
+ * on by default).  A kernel then waits for the one right before it through a
+ * counter that kernel's CTAs increment as they finish, instead of waiting for
+ * that whole grid to be retired: each projection GEMM for the epilogue that
+ * wrote its input rows (its weight stream has started before either wait),
+ * each epilogue for its GEMM's parts, the attention for the q|k|v epilogue
+ * and the split merge for the attention (the o projection keeps the grid
+ * wait on the merge).  The counters are zeroed by each pass's first kernel.
  * A wait that outlasts about a second gives up and raises the device flag
  * (uno_status returns UNO_ERR_DEVICE_CHECK).  enable = 0 uses grid
  * dependencies only.  Changing it drops captured graphs. */
