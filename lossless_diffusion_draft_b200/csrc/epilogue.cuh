@@ -534,21 +534,6 @@ __device__ __forceinline__ float4 part4_add(Part4<C>& L, bool live) {
   }
   return acc;
 }
-__device__ __forceinline__ void store4_split(bf16* hi, bf16* lo, size_t i, float4 y) {
-  const __nv_bfloat162 h01 = __floats2bfloat162_rn(y.x, y.y), h23 = __floats2bfloat162_rn(y.z, y.w);
-  uint2 hv;
-  hv.x = *reinterpret_cast<const uint32_t*>(&h01);
-  hv.y = *reinterpret_cast<const uint32_t*>(&h23);
-  *reinterpret_cast<uint2*>(hi + i) = hv;
-  if (lo) {
-    const __nv_bfloat162 l01 = __floats2bfloat162_rn(y.x - __low2float(h01), y.y - __high2float(h01));
-    const __nv_bfloat162 l23 = __floats2bfloat162_rn(y.z - __low2float(h23), y.w - __high2float(h23));
-    uint2 lv;
-    lv.x = *reinterpret_cast<const uint32_t*>(&l01);
-    lv.y = *reinterpret_cast<const uint32_t*>(&l23);
-    *reinterpret_cast<uint2*>(lo + i) = lv;
-  }
-}
 
 __global__ void __launch_bounds__(RESID_THREADS) epi_resid_kernel(const EpiArgs a) {
   typedef GeoResid G;

@@ -278,6 +278,27 @@ __device__ __forceinline__ void store_split(T* hi, T* lo, size_t i, float y) {
   hi[i] = h;
   if (lo) lo[i] = from_f<T>(y - to_f(h));
 }
+// Four consecutive values (i a multiple of 4): one 8-byte store per row in
+// bf16, one 16-byte store in fp32 (whose rounding residual is zero).
+__device__ __forceinline__ void store4_split(bf16* hi, bf16* lo, size_t i, float4 y) {
+  const __nv_bfloat162 h01 = __floats2bfloat162_rn(y.x, y.y), h23 = __floats2bfloat162_rn(y.z, y.w);
+  uint2 hv;
+  hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+  hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+  *reinterpret_cast<uint2*>(hi + i) = hv;
+  if (lo) {
+    const __nv_bfloat162 l01 = __floats2bfloat162_rn(y.x - __low2float(h01), y.y - __high2float(h01));
+    const __nv_bfloat162 l23 = __floats2bfloat162_rn(y.z - __low2float(h23), y.w - __high2float(h23));
+    uint2 lv;
+    lv.x = *reinterpret_cast<const uint32_t*>(&l01);
+    lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+    *reinterpret_cast<uint2*>(lo + i) = lv;
+  }
+}
+__device__ __forceinline__ void store4_split(float* hi, float* lo, size_t i, float4 y) {
+  *reinterpret_cast<float4*>(hi + i) = y;
+  if (lo) *reinterpret_cast<float4*>(lo + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
 
 // RMSNorm: out = x / sqrt(mean(x^2) + eps) * gain, one CTA per row.  Each
 // thread holds up to RMS_V float4 of the row in registers (all loads issued
@@ -310,10 +331,9 @@ __global__ void __launch_bounds__(NT) rmsnorm_kernel(const float* x, const T* ga
     const int i = threadIdx.x + k * NT;
     if (i < n4) {
       const int e = 4 * i;
-      store_split<T>(out + o, lrow, e + 0, v[k].x * inv * to_f(gain[e + 0]));
-      store_split<T>(out + o, lrow, e + 1, v[k].y * inv * to_f(gain[e + 1]));
-      store_split<T>(out + o, lrow, e + 2, v[k].z * inv * to_f(gain[e + 2]));
-      store_split<T>(out + o, lrow, e + 3, v[k].w * inv * to_f(gain[e + 3]));
+      store4_split(out + o, lrow, e,
+                   make_float4(v[k].x * inv * to_f(gain[e + 0]), v[k].y * inv * to_f(gain[e + 1]),
+                               v[k].z * inv * to_f(gain[e + 2]), v[k].w * inv * to_f(gain[e + 3])));
     }
   }
 }
@@ -406,10 +426,9 @@ __global__ void swiglu_kernel(const float* gu, int F, T* out, T* lo) {
   const float4 b = *reinterpret_cast<const float4*>(g + F + f);
   const size_t o = (size_t)row * F + f;
   T* lrow = lo ? lo + o : nullptr;
-  store_split<T>(out + o, lrow, 0, a.x / (1.0f + expf(-a.x)) * b.x);
-  store_split<T>(out + o, lrow, 1, a.y / (1.0f + expf(-a.y)) * b.y);
-  store_split<T>(out + o, lrow, 2, a.z / (1.0f + expf(-a.z)) * b.z);
-  store_split<T>(out + o, lrow, 3, a.w / (1.0f + expf(-a.w)) * b.w);
+  store4_split(out + o, lrow, 0,
+               make_float4(a.x / (1.0f + expf(-a.x)) * b.x, a.y / (1.0f + expf(-a.y)) * b.y,
+                           a.z / (1.0f + expf(-a.z)) * b.z, a.w / (1.0f + expf(-a.w)) * b.w));
 }
 
 // Prefill bookkeeping: cached = P - 1, pending = prompt[P - 1].
