@@ -30,6 +30,7 @@
 #include "epilogue.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tokm.cuh"
 #include "layers.cuh"
 #include "sampling.cuh"
 #include "tree.cuh"
@@ -315,6 +316,83 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
   return true;
 }
 
+// The tokens-in-M form (gemm_tokm.cuh) for split inputs of more than one
+// token tile, not DUMP: every segment but the last a whole number of 256-row
+// weight tiles, 16-byte aligned output rows, no row map.  False: not taken,
+// nothing launched.
+bool launch_tokm(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
+  if (p.lo_off <= 0 || p.M <= TK_BM || p.out_row) return false;
+  for (int s = 0; s + 1 < p.nseg; ++s)
+    if (p.seg[s].n % TK_BN) return false;
+  const bool f32 = p.epi == EPI_STORE_F32 || p.epi == EPI_ADD_F32;
+  if (p.ldo % (f32 ? 4 : 8) || ((uintptr_t)p.out & 15) || ((uintptr_t)p.out_lo & 15)) return false;
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const uint64_t xrows = (uint64_t)p.lo_off + std::max<uint64_t>(p.M, TK_BM);
+  if ((uint64_t)env.x_rows_alloc < xrows) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (p.seg[s].n < TC_BM) return false;
+  if (p.U && p.nseg > 3) return false;   // LoRA-B maps: three segments
+  const CUtensorMap* mx = env.map(p.X, xrows, p.K, p.ldx, TK_BM);
+  if (!mx) return false;
+  maps.x = *mx;
+  maps.u = *mx;
+  if (p.U) {
+    const CUtensorMap* mu = env.map(p.U, xrows, p.ldu, p.ldu, TK_BM);
+    if (!mu) return false;
+    maps.u = *mu;
+  }
+  TcParams tp{};
+  tp.M = p.M;
+  tp.N = p.N;
+  tp.KB = p.K / TC_BK;
+  tp.RB = p.U ? p.r / TC_BK : 0;
+  tp.nseg = p.nseg;
+  for (int s = 0; s < p.nseg; ++s) {
+    const GemmSeg& g = p.seg[s];
+    const CUtensorMap* mw = env.map(g.W, g.n, p.K, p.K, TC_BM);
+    if (!mw) return false;
+    maps.w[s] = *mw;
+    if (s < 3) maps.b[s] = *mw;
+    if (p.U) {
+      if (!g.lB) return false;
+      const CUtensorMap* mb = env.map(g.lB, g.n, p.r, p.r, TC_BM);
+      if (!mb) return false;
+      maps.b[s] = *mb;
+    }
+    tp.seg[s] = TcSeg{g.n0, g.n, g.u_off};
+  }
+  tp.n_tiles = (p.N + TK_BN - 1) / TK_BN;
+  tp.m_tiles = (p.M + TK_BM - 1) / TK_BM;
+  if ((long long)tp.n_tiles * tp.m_tiles > TC_COUNTERS) return false;
+  if ((long long)tp.n_tiles * tp.m_tiles * (tp.KB + tp.RB) * env.sm_count >= (1LL << 32)) return false;
+  tp.units = tp.n_tiles * tp.m_tiles * (tp.KB + tp.RB);
+  tp.grid = std::max(1, std::min(env.sm_count, tp.units / TC_MIN_UNITS));
+  tp.mgroups = 0;
+  const int g = std::min(env.sm_count / tp.m_tiles, tp.n_tiles * (tp.KB + tp.RB) / TC_MIN_UNITS);
+  if (g >= 1) {
+    tp.mgroups = g;
+    tp.grid = g * tp.m_tiles;
+  }
+  tp.max_parts = 2;
+  tp.epi = p.epi;
+  tp.out = p.out;
+  tp.ldo = p.ldo;
+  tp.alpha = p.alpha;
+  tp.row_gate = p.row_gate;
+  tp.ws = env.ws;
+  tp.counters = env.counters;
+  tp.status = env.status;
+  tp.lo_off = p.lo_off;
+  tp.out_lo = p.out_lo;
+  tp.dep_limit_ns = DEP_WAIT_NS;
+  static bool attr[ATTR_DEVS] = {};
+  if (smem_attr_once(gemm_tokm_kernel, TkCfg::SMEM, attr) != cudaSuccess) return false;
+  klaunch(env.pdl, st, dim3(tp.grid), dim3(TC_THREADS), TkCfg::SMEM, gemm_tokm_kernel, maps, tp);
+  g_launches[0]++;
+  return true;
+}
+
 // Whether the tensor-core kernel takes this bf16 GEMM: K and r in 64-element
 // blocks, every segment but the last a whole number of 128-row tiles, 16-byte
 // aligned rows.
@@ -368,7 +446,7 @@ template <typename T>
 void gemm_run(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
   if (p.M <= 0 || p.N <= 0) return;
   if (sizeof(T) == 2 && !env.tc_disabled && tc_shape_ok(p) &&
-      launch_tc_any<false>(env, p, st, nullptr))
+      (launch_tokm(env, p, st) || launch_tc_any<false>(env, p, st, nullptr)))
     return;
   gemm_simt_dispatch<T>(p, st, env.pdl);
 }
