@@ -29,61 +29,27 @@ struct TkCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
-// 16 consecutive output columns n .. n + 15 of token row m (row and columns
-// in range; the host checks 16-byte alignment of every row).
+// 16 consecutive fp32 output columns n .. n + 15 of token row m (row and
+// columns in range; the host checks 16-byte alignment of every row): stored
+// scaled by alpha, or added to what is there (the residual stream).
 __device__ __forceinline__ void tk_store16(const TcParams& p, int m, int n, const float (&v)[16]) {
-  const size_t o = (size_t)m * p.ldo + n;
-  if (p.epi == EPI_STORE_F32 || p.epi == EPI_ADD_F32) {
-    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o);
-    float4 w[4];
-    if (p.epi == EPI_ADD_F32) {
+  float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (size_t)m * p.ldo + n);
+  float4 w[4];
+  if (p.epi == EPI_ADD_F32) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = __ldcg(dst + q);
+    for (int q = 0; q < 4; ++q) w[q] = __ldcg(dst + q);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        w[q].x += v[4 * q]; w[q].y += v[4 * q + 1]; w[q].z += v[4 * q + 2]; w[q].w += v[4 * q + 3];
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        w[q] = make_float4(v[4 * q] * p.alpha, v[4 * q + 1] * p.alpha, v[4 * q + 2] * p.alpha,
-                           v[4 * q + 3] * p.alpha);
+    for (int q = 0; q < 4; ++q) {
+      w[q].x += v[4 * q]; w[q].y += v[4 * q + 1]; w[q].z += v[4 * q + 2]; w[q].w += v[4 * q + 3];
     }
+  } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = w[q];
-    return;
+    for (int q = 0; q < 4; ++q)
+      w[q] = make_float4(v[4 * q] * p.alpha, v[4 * q + 1] * p.alpha, v[4 * q + 2] * p.alpha,
+                         v[4 * q + 3] * p.alpha);
   }
-  if (p.epi == EPI_STORE) {
-    uint32_t h[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * q] * p.alpha, v[2 * q + 1] * p.alpha);
-      h[q] = *reinterpret_cast<const uint32_t*>(&b);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + o);
-    dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-    dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-    return;
-  }
-  // gated: bf16 hi (and lo) of v * alpha * gate[m]
-  const float gm = p.alpha * p.row_gate[m];
-  uint32_t h[8], l[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float a = v[2 * q] * gm, b = v[2 * q + 1] * gm;
-    const __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
-    const __nv_bfloat162 lb = __floats2bfloat162_rn(a - __low2float(hb), b - __high2float(hb));
-    h[q] = *reinterpret_cast<const uint32_t*>(&hb);
-    l[q] = *reinterpret_cast<const uint32_t*>(&lb);
-  }
-  uint4* dh = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + o);
-  dh[0] = make_uint4(h[0], h[1], h[2], h[3]);
-  dh[1] = make_uint4(h[4], h[5], h[6], h[7]);
-  if (p.out_lo) {
-    uint4* dl = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out_lo) + o);
-    dl[0] = make_uint4(l[0], l[1], l[2], l[3]);
-    dl[1] = make_uint4(l[4], l[5], l[6], l[7]);
-  }
+  for (int q = 0; q < 4; ++q) dst[q] = w[q];
 }
 // The same for columns that may run past N (scalar, per element).
 __device__ __forceinline__ void tk_store16_edge(const TcParams& p, int m, int n, const float (&v)[16]) {

@@ -317,15 +317,16 @@ bool launch_tc(GemmEnv& env, const GemmParams& p, cudaStream_t st, DumpShape* sh
 }
 
 // The tokens-in-M form (gemm_tokm.cuh) for split inputs of more than one
-// token tile, not DUMP: every segment but the last a whole number of 256-row
-// weight tiles, 16-byte aligned output rows, no row map.  False: not taken,
-// nothing launched.
+// token tile, not DUMP, fp32 outputs (stored or added: every projection of
+// the unfused pass; the LoRA-A products keep the other form): every segment
+// but the last a whole number of 256-row weight tiles, 16-byte aligned output
+// rows, no row map.  False: not taken, nothing launched.
 bool launch_tokm(GemmEnv& env, const GemmParams& p, cudaStream_t st) {
   if (p.lo_off <= 0 || p.M <= TK_BM || p.out_row) return false;
+  if (p.epi != EPI_STORE_F32 && p.epi != EPI_ADD_F32) return false;
   for (int s = 0; s + 1 < p.nseg; ++s)
     if (p.seg[s].n % TK_BN) return false;
-  const bool f32 = p.epi == EPI_STORE_F32 || p.epi == EPI_ADD_F32;
-  if (p.ldo % (f32 ? 4 : 8) || ((uintptr_t)p.out & 15) || ((uintptr_t)p.out_lo & 15)) return false;
+  if (p.ldo % 4 || ((uintptr_t)p.out & 15)) return false;
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
   const uint64_t xrows = (uint64_t)p.lo_off + std::max<uint64_t>(p.M, TK_BM);
