@@ -110,3 +110,45 @@ def test_qwen8b_shape_two_layers(fused):
 def test_qwen8b_first_four_steps():
     """The full 36-layer model, 1024-token prompt, first four iterations."""
     _run()
+
+
+def test_qwen8b_two_layers_eight_requests_lm_head_edge():
+    """Eight requests at once on the Qwen3-8B widths (two layers): 136 draft
+    rows take the tokens-in-M GEMM form, whose last LM-head weight tile is
+    cut by the 151936-token vocabulary (593.5 tiles of 256).  Every request's
+    draft and verify logits within 2e-2 of the oracle's on the GPU's drafts,
+    and the GPU's request states after the step (three of the requests)."""
+    cfg = dict(synth.CONFIGS["qwen8b"], n_layers=2)
+    shape = synth.model_shape(cfg)
+    shape["dtype"] = cfg["dtype"]
+    params = synth.make_params(cfg, "cuda")
+    B, V, seed = cfg["B"], cfg["vocab"], cfg["seed"]
+    n_req, P = 8, 80
+    ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, n_req, P + 2 * (B + 1),
+                       seed, torch.cuda.current_stream())
+    prompts = synth.make_prompts(cfg, n_req, P)
+    ids = uno.uno_prefill(ctx, torch.from_numpy(prompts).cuda(), [P] * n_req,
+                          streams=list(range(n_req)))
+    # two layers: the weights fit the host as fp32 (exact for bf16); the
+    # oracle's products upcast them to fp64
+    model = om.Model(synth.model_shape(cfg), {k: v.float().cpu().numpy() for k, v in params.items()})
+    req = torch.tensor(ids, dtype=torch.int32, device="cuda")
+    out = torch.zeros((n_req, B + 1), dtype=torch.int32, device="cuda")
+    n_new = torch.zeros(n_req, dtype=torch.int32, device="cuda")
+    uno.uno_spec_step(ctx, req, out, n_new)
+    uno.uno_status(ctx)
+    ld = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_DRAFT, torch.empty((n_req, B + 1, V)))
+    lv = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_VERIFY, torch.empty((n_req, B, V)))
+    dr = uno.uno_debug_read(ctx, uno.UNO_DBG_DRAFTS, torch.empty((n_req, B), dtype=torch.int32))
+    nn = n_new.cpu().numpy()
+    # the first request, one in the first token tile's middle, and the last,
+    # whose rows end the second token tile
+    for i in (0, 3, n_req - 1):
+        st = ops.prefill(model, [int(t) for t in prompts[i]], stream=i)
+        _, res = ops.spec_step(model, st, B, seed, drafts=[int(t) for t in dr[i]])
+        err_d = float(np.max(np.abs(ld[i].double().numpy() - res.logits_draft)))
+        err_v = float(np.max(np.abs(lv[i].double().numpy() - res.logits_verify)))
+        assert err_d <= 2e-2 and err_v <= 2e-2, (i, err_d, err_v)
+        c_gpu, _ = uno.uno_request_state(ctx, ids[i])
+        assert c_gpu == st.c + int(nn[i])
+    ctx.close()
