@@ -112,18 +112,23 @@ def test_qwen8b_first_four_steps():
     _run()
 
 
-def test_qwen8b_two_layers_eight_requests_lm_head_edge():
-    """Eight requests at once on the Qwen3-8B widths (two layers): 136 draft
-    rows take the tokens-in-M GEMM form, whose last LM-head weight tile is
-    cut by the 151936-token vocabulary (593.5 tiles of 256).  Every request's
+@pytest.mark.parametrize("n_req,checked", [(8, (0, 3, 7)), (80, (0, 41, 79))],
+                         ids=["8_requests", "80_requests"])
+def test_qwen8b_two_layers_many_requests(n_req, checked):
+    """Several requests at once on the Qwen3-8B widths (two layers, 80-token
+    prompts).  Eight requests: 136 draft rows take the tokens-in-M GEMM form,
+    whose last LM-head weight tile is cut by the 151936-token vocabulary
+    (593.5 tiles of 256).  Eighty requests: the largest batch's launch
+    configuration (1360 draft / 1280 verify rows, m-tile groups, 640
+    unsplit attention groups, more than the SMs).  The checked requests'
     draft and verify logits within 2e-2 of the oracle's on the GPU's drafts,
-    and the GPU's request states after the step (three of the requests)."""
+    and their request states after the step."""
     cfg = dict(synth.CONFIGS["qwen8b"], n_layers=2)
     shape = synth.model_shape(cfg)
     shape["dtype"] = cfg["dtype"]
     params = synth.make_params(cfg, "cuda")
     B, V, seed = cfg["B"], cfg["vocab"], cfg["seed"]
-    n_req, P = 8, 80
+    P = 80
     ctx = uno.uno_init(shape, params, cfg["lora_rank"], cfg["lora_alpha"], B, n_req, P + 2 * (B + 1),
                        seed, torch.cuda.current_stream())
     prompts = synth.make_prompts(cfg, n_req, P)
@@ -141,9 +146,9 @@ def test_qwen8b_two_layers_eight_requests_lm_head_edge():
     lv = uno.uno_debug_read(ctx, uno.UNO_DBG_LOGITS_VERIFY, torch.empty((n_req, B, V)))
     dr = uno.uno_debug_read(ctx, uno.UNO_DBG_DRAFTS, torch.empty((n_req, B), dtype=torch.int32))
     nn = n_new.cpu().numpy()
-    # the first request, one in the first token tile's middle, and the last,
-    # whose rows end the second token tile
-    for i in (0, 3, n_req - 1):
+    # the first request, one in the middle and the last, whose rows end the
+    # last token tile
+    for i in checked:
         st = ops.prefill(model, [int(t) for t in prompts[i]], stream=i)
         _, res = ops.spec_step(model, st, B, seed, drafts=[int(t) for t in dr[i]])
         err_d = float(np.max(np.abs(ld[i].double().numpy() - res.logits_draft)))
