@@ -55,67 +55,141 @@ def peaks():
 # Clock sampling during the timed region.
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clocks and clock-event reasons of one GPU while the timed region
+    runs: NVML read every 10 ms from a thread (the timed regions are a few
+    hundred ms long), else `nvidia-smi -lms 50`.  Read-only: no setting of
+    the GPU is touched."""
+
+    PERIOD_S = 0.01
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    NVML_BITS = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+                 "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index, enabled=True):
+    def __init__(self, gpu_index, enabled=True, nvml=None):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
         self.enabled = enabled
+        self.samples = []          # (time, sm MHz, max sm MHz, set of reason names)
+        self._t0 = float("inf")
+        self.source = None
+        self._nvml = nvml          # a pynvml-like module (tests pass a fake)
+        self._proc = None
+        self._thread = None
+        self._stop = threading.Event()
+
+    def _uuid(self):
+        import re
+        try:
+            u = str(torch.cuda.get_device_properties(self.gpu).uuid)
+        except Exception:
+            return None
+        m = re.search(r"[0-9a-fA-F]{8}(-[0-9a-fA-F]{4}){3}-[0-9a-fA-F]{12}", u)
+        return "GPU-" + m.group(0) if m else None
+
+    def _nvml_start(self):
+        nv = self._nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        uuid, h = self._uuid(), None
+        if uuid:
+            try:
+                h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                h = None
+        if h is None:
+            h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = {}
+        for name, suffix in self.NVML_BITS.items():
+            b = getattr(nv, "nvmlClocksEventReason" + suffix, None)
+            bits[name] = b if b is not None else getattr(nv, "nvmlClocksThrottleReason" + suffix)
+
+        def read():
+            mask = get_reasons(h)
+            return (float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                    float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)),
+                    {n for n, b in bits.items() if mask & b})
+
+        read()   # fails here, before the timed region, if NVML cannot read
+
+        def loop():
+            while not self._stop.is_set():
+                t = time.time()
+                try:
+                    self.samples.append((t,) + read())
+                except Exception:
+                    break
+                self._stop.wait(self.PERIOD_S)
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        self.source = "nvml"
+
+    def _smi_start(self):
+        self._proc = subprocess.Popen(
+            ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+             "--format=csv,noheader,nounits", "-lms", "50"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        lines = []
+
+        def reader():
+            for line in self._proc.stdout:
+                lines.append(line.strip())
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm, mx = float(f[1]), float(f[2])
+                except ValueError:
+                    continue
+                self.samples.append((time.time(), sm, mx, {n for n, v in zip(self.REASONS, f[5:9])
+                                                           if v.lower() == "active"}))
+        self._thread = threading.Thread(target=reader, daemon=True)
+        self._thread.start()
+        # the timed region starts once the sampler is producing lines
+        t0 = time.time()
+        while not lines and time.time() - t0 < 3.0 and self._proc.poll() is None:
+            time.sleep(0.01)
+        self.source = "nvidia-smi"
 
     def __enter__(self):
         if not self.enabled:
             return self
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-            # the timed region starts once the sampler is producing lines;
-            # samples taken before it are dropped
-            t0 = time.time()
-            while not self.lines and time.time() - t0 < 3.0 and self.proc.poll() is None:
-                time.sleep(0.01)
-            self.lines.clear()
-        except OSError:
-            self.proc = None
+            self._nvml_start()
+        except Exception:
+            try:
+                self._smi_start()
+            except OSError:
+                self._proc = None
+        self._t0 = time.time()   # samples taken before the timed region are dropped
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in self.lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        smp = [x for x in self.samples if x[0] >= self._t0]
+        if not smp:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(x[1] for x in smp), "sm_max_mhz": smp[-1][2],
+                "reasons": sorted(set().union(*(x[3] for x in smp))),
+                "samples": len(smp), "source": self.source}
 
 
 # ---------------------------------------------------------------------------

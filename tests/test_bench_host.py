@@ -78,3 +78,59 @@ def test_aggregation_over_two_gloo_ranks():
 def test_single_rank_aggregation_is_identity():
     assert bench.reduce_max(3.5, 1, None) == 3.5
     assert bench.reduce_sum(7, 1, None) == 7
+
+
+class _FakeNvml:
+    """pynvml stand-in: an SM clock that drops under a power cap after the
+    third read."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+
+    def __init__(self):
+        self.reads = 0
+        self.shut = False
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        self.shut = True
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        return ("uuid", uuid)
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("index", i)
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        assert which == self.NVML_CLOCK_SM
+        self.reads += 1
+        return 1965 if self.reads <= 3 else 1800
+
+    def nvmlDeviceGetMaxClockInfo(self, h, which):
+        return 1965
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x1 | (0x4 if self.reads >= 3 else 0)   # idle bit ignored
+
+
+def test_clock_sampler_reads_nvml_without_touching_settings():
+    import time
+    nv = _FakeNvml()
+    with bench.ClockSampler(0, nvml=nv) as clk:
+        time.sleep(0.2)
+    s = clk.summary()
+    assert s["source"] == "nvml" and s["samples"] >= 5
+    assert s["sm_max_mhz"] == 1965 and s["sm_mhz"] == 1800
+    assert s["reasons"] == ["sw_power_cap"]
+    assert nv.shut
+    # the fake has no setter: any call beyond reads would raise AttributeError
+
+
+def test_clock_sampler_disabled_records_nothing():
+    with bench.ClockSampler(0, enabled=False, nvml=_FakeNvml()) as clk:
+        pass
+    assert clk.summary() is None
