@@ -458,27 +458,34 @@ class Workload:
                     clocks=clk.summary() if clocks else None, ctx_window=[c0, self.cached()],
                     launches=sum(v[0] for v in prof.values()), K=K)
 
-    def e2e(self, K, world):
+    def e2e(self, K, W, world):
         """The same steps end to end through the C ABI: request ids copied from
-        pinned host memory, emitted tokens and counts copied back, every step."""
+        pinned host memory, emitted tokens and counts copied back, every step.
+        W untimed steps first, with the same buffers: the library captures a
+        step's graph on the second call with new buffer addresses, which is
+        set-up, not a step."""
         uno, stream = self.uno, torch.cuda.current_stream()
         req_h = torch.tensor(self.ids, dtype=torch.int32).pin_memory()
         out_h = torch.zeros((self.batch, self.B + 1), dtype=torch.int32).pin_memory()
         nn_h = torch.zeros(self.batch, dtype=torch.int32).pin_memory()
         req_d = torch.empty_like(self.req)
         nn_d = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+        def step():
+            req_d.copy_(req_h, non_blocking=True)
+            uno.uno_spec_step(self.ctx, req_d, self.out, nn_d)
+            out_h.copy_(self.out, non_blocking=True)
+            nn_h.copy_(nn_d, non_blocking=True)
+            stream.synchronize()
+            return int(nn_h.sum())
+        for _ in range(W):
+            step()
         tokens = 0
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(K):
-            req_d.copy_(req_h, non_blocking=True)
-            uno.uno_spec_step(self.ctx, req_d, self.out, nn_d)
-            out_h.copy_(self.out, non_blocking=True)
-            nn_h.copy_(nn_d, non_blocking=True)
-            stream.synchronize()
-            tokens += int(nn_h.sum())
+            tokens += step()
         e1.record(stream)
         torch.cuda.synchronize()
         uno.uno_status(self.ctx)
@@ -548,7 +555,7 @@ def run_uno(args, rank, world, device):
     head = wl.time_steps(K, W, world, profile_range=args.profile_range)
     kprof, detail = step_profile(wl.ctx, wl.req, wl.out, torch.zeros(batch, dtype=torch.int32,
                                                                      device=device), K, cfg)
-    e2e = wl.e2e(K, world)
+    e2e = wl.e2e(K, W, world)
     ar = wl.time_steps(K, W, world, ar=True, clocks=False)
     res = dict(cfg=cfg, batch=batch, head=head, kprof=kprof, detail=detail, e2e=e2e, ar=ar,
                fused=wl.fused, prefill_s=wl.prefill_s, weight_bytes=weight_bytes, pk=pk)
@@ -684,7 +691,7 @@ def run_max_batch(args, cfg, params, rank, world, device, pk):
     head = wl.time_steps(K, W, world)
     _, detail = step_profile(wl.ctx, wl.req, wl.out, torch.zeros(batch, dtype=torch.int32,
                                                                  device=device), 2, cfg)
-    e2e = wl.e2e(K, world)
+    e2e = wl.e2e(K, W, world)
     ar = wl.time_steps(K, W, world, ar=True, clocks=False)
     wl.close()
     ms = head["ms"] / head["K"]
@@ -695,7 +702,8 @@ def run_max_batch(args, cfg, params, rank, world, device, pk):
             "tpf": head["tokens"] / K / batch / 2, "context_window": head["ctx_window"],
             "prefill_s": wl.prefill_s,
             "e2e": {"value": e2e["tokens"] / (e2e["ms"] / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": e2e["ms"] / K, "tokens_per_step": e2e["tokens"] / K},
             "ar_only": {"value": ar_value, "unit": "tokens/s", "ms_per_step": ar["ms"] / ar["K"]},
             "psi_spec_over_ar": value / ar_value,
             "roofline": gemm_roofline(detail, cfg, pk), "clocks": head["clocks"],
@@ -1007,7 +1015,8 @@ def main():
         "roofline": roofline, "step_roofline": step_roof,
         "kernel_breakdown": {k: {"launches": v[0], "ms_per_step": v[1] / K} for k, v in kp.items()},
         "e2e": {"value": e2e_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"]},
+                "h2d_bytes_per_step": res["e2e"]["h2d"], "d2h_bytes_per_step": res["e2e"]["d2h"],
+                "ms_per_step": e2e_ms / K, "tokens_per_step": e2e_tokens / K},
         "gpu_launches": head["launches"], "clocks": head["clocks"],
         "kernel_detail": res["detail"][:24],
         "prefill_s": res["prefill_s"],
