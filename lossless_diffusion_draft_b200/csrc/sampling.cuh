@@ -96,23 +96,31 @@ __device__ __forceinline__ Filt<FILT> filt_of(const RowFilter* f, size_t row) {
 // by a butterfly and the warps in order: a fixed tree, and no rescaling.
 // ---------------------------------------------------------------------------
 constexpr int CHUNK_IT = 8;   // float4 per thread: a chunk holds <= 8 * 4 * 256 = 8192 logits
-// red: at least 2 * SAMPLE_THREADS / 32 floats of shared memory.
-template <bool FILT = false>
-__device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red,
-                                               Filt<FILT> f = Filt<FILT>{0u, -1}) {
-  constexpr int NW = SAMPLE_THREADS / 32;
-  // float4 path: rows start on 16-byte boundaries (vocab % 4 == 0 is required)
+// A thread's loads of a chunk (16 bytes each, streaming; rows start on
+// 16-byte boundaries: vocab % 4 == 0 is required), the filter applied.
+template <bool FILT>
+__device__ __forceinline__ void chunk_load(const float* row, int c0, int c1, float4 (&v)[CHUNK_IT],
+                                           Filt<FILT> f) {
   const int n4 = (c1 - c0) >> 2;
   const float4* r4 = reinterpret_cast<const float4*>(row + c0);
-  float4 v[CHUNK_IT];
+#pragma unroll
+  for (int i = 0; i < CHUNK_IT; ++i) {
+    const int j = threadIdx.x + i * SAMPLE_THREADS;
+    if (j < n4) v[i] = f.four(__ldcs(r4 + j), c0 + 4 * j);
+  }
+}
+// The reduction of a chunk whose float4 part chunk_load has brought into v.
+// red: at least 2 * SAMPLE_THREADS / 32 floats of shared memory.
+template <bool FILT>
+__device__ __forceinline__ float2 chunk_reduce(const float* row, int c0, int c1,
+                                               const float4 (&v)[CHUNK_IT], float* red, Filt<FILT> f) {
+  constexpr int NW = SAMPLE_THREADS / 32;
+  const int n4 = (c1 - c0) >> 2;
   float m = -INFINITY;
 #pragma unroll
   for (int i = 0; i < CHUNK_IT; ++i) {
     const int j = threadIdx.x + i * SAMPLE_THREADS;
-    if (j < n4) {
-      v[i] = f.four(__ldcs(r4 + j), c0 + 4 * j);
-      m = fmaxf(m, fmaxf(fmaxf(v[i].x, v[i].y), fmaxf(v[i].z, v[i].w)));
-    }
+    if (j < n4) m = fmaxf(m, fmaxf(fmaxf(v[i].x, v[i].y), fmaxf(v[i].z, v[i].w)));
   }
   // scalar tail (chunk length not a multiple of 4: only the row's last chunk)
   for (int j = c0 + (n4 << 2) + threadIdx.x; j < c1; j += SAMPLE_THREADS) m = fmaxf(m, f(row[j], j));
@@ -144,6 +152,13 @@ __device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1,
 #pragma unroll
   for (int w = 0; w < NW; ++w) S += red[NW + w];
   return make_float2(M, S);
+}
+template <bool FILT = false>
+__device__ __forceinline__ float2 reduce_chunk(const float* row, int c0, int c1, float* red,
+                                               Filt<FILT> f = Filt<FILT>{0u, -1}) {
+  float4 v[CHUNK_IT];
+  chunk_load<FILT>(row, c0, c1, v, f);
+  return chunk_reduce<FILT>(row, c0, c1, v, red, f);
 }
 
 // Chunk-level prefix in chunk order, run by one whole warp: lane l holds
@@ -635,21 +650,35 @@ __global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_verify_kernel(const Ve
   verify_decide<FILT>(a, req, red);
 }
 
-// Split form (many rows), first kernel: grid (nch, n_req * rows_red), every
-// CTA reduces its chunk, writes the pair and exits (no counters, no waiting
-// on a round trip), so the loads of the next CTAs keep HBM busy.
+// Split form (many rows), first kernel: grid (ceil(nch / 2), n_req *
+// rows_red), every CTA reduces two consecutive chunks of a row, writes their
+// pairs and exits (no counters, no waiting on a round trip).  Both chunks'
+// loads are issued before either is reduced, so an SM keeps its three CTAs'
+// 64 KB each in flight through the reductions (measured on 4096 x 151936
+// fp32 p and q: 0.752 ms against 0.957 with one chunk a CTA at four CTAs an
+// SM, and 1.29 / 1.18 ms at five / six).
 template <bool FILT>
-__global__ void __launch_bounds__(SAMPLE_THREADS, 4) spec_reduce_kernel(const VerifyArgs a) {
+__global__ void __launch_bounds__(SAMPLE_THREADS, 3) spec_reduce_kernel(const VerifyArgs a) {
   __shared__ float red[32];
   pdl_trigger();
   pdl_wait();
-  const int k = blockIdx.x;
+  const int k0 = 2 * blockIdx.x;
   const int rid = blockIdx.y;
   const int req = rid / a.rows_red, r = rid % a.rows_red;
   const float* row = verify_row(a, req, r);
-  const int c0 = k * a.ch, c1 = min(a.V, c0 + a.ch);
-  const float2 pr = reduce_chunk<FILT>(row, c0, c1, red, verify_row_filt<FILT>(a, req, r));
-  if (threadIdx.x == 0) a.partial[(size_t)rid * a.nch + k] = pr;
+  const Filt<FILT> f = verify_row_filt<FILT>(a, req, r);
+  const int c0 = k0 * a.ch, c1 = min(a.V, c0 + a.ch);
+  const bool two = k0 + 1 < a.nch;
+  const int d1 = min(a.V, c1 + a.ch);
+  float4 v0[CHUNK_IT], v1[CHUNK_IT];
+  chunk_load<FILT>(row, c0, c1, v0, f);
+  if (two) chunk_load<FILT>(row, c1, d1, v1, f);
+  const float2 p0 = chunk_reduce<FILT>(row, c0, c1, v0, red, f);
+  if (threadIdx.x == 0) a.partial[(size_t)rid * a.nch + k0] = p0;
+  if (two) {
+    const float2 p1 = chunk_reduce<FILT>(row, c1, d1, v1, red, f);
+    if (threadIdx.x == 0) a.partial[(size_t)rid * a.nch + k0 + 1] = p1;
+  }
 }
 
 // Split form, second kernel: one CTA per request; warp w forms the lse of

@@ -139,7 +139,8 @@ int launch_verify_t(bool pdl, cudaStream_t st, const VerifyArgs& a, int n_req, l
     klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_verify_kernel<FILT>, a);
     return 1;
   }
-  klaunch(pdl, st, grid, dim3(SAMPLE_THREADS), 0, spec_reduce_kernel<FILT>, a);
+  klaunch(pdl, st, dim3((a.nch + 1) / 2, n_req * a.rows_red), dim3(SAMPLE_THREADS), 0,
+          spec_reduce_kernel<FILT>, a);
   klaunch(pdl, st, dim3(n_req), dim3(SAMPLE_THREADS), 0, spec_decide_kernel<FILT>, a);
   return 2;
 }
