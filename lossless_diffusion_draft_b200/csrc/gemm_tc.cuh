@@ -89,11 +89,12 @@ struct TcParams {
 // Stream-K partition.
 // ---------------------------------------------------------------------------
 // 32-bit arithmetic: units * grid stays below 2^32 for every launch (the
-// host checks), and a 64-bit division is a long software sequence.
-__device__ __forceinline__ int sk_start(int i, int units, int grid) {
+// host checks), and a 64-bit division is a long software sequence.  Host-
+// callable too, so that the partition is checked on the CPU.
+__host__ __device__ __forceinline__ int sk_start(int i, int units, int grid) {
   return (int)(((unsigned)i * (unsigned)units) / (unsigned)grid);
 }
-__device__ __forceinline__ int sk_owner(int u, int units, int grid) {
+__host__ __device__ __forceinline__ int sk_owner(int u, int units, int grid) {
   int i = (int)(((unsigned)u * (unsigned)grid) / (unsigned)units);
   while (i + 1 < grid && sk_start(i + 1, units, grid) <= u) ++i;
   while (i > 0 && sk_start(i, units, grid) > u) --i;
