@@ -231,11 +231,11 @@ int uno_set_fused(uno_ctx *ctx, int enable);
 
 /* spec_verify's form (implementation choice): when a step's verification
  * has more than max_ctas (row, vocabulary chunk) CTAs (default 4096), it
- * runs as a reduction kernel whose CTAs carry no counters plus one CTA per
- * request that combines the rows and decides; otherwise as one fused kernel
- * whose last CTAs combine and decide.  Both give the same tokens.  0 forces
- * the split form.  Changing it drops captured graphs.  max_ctas < 0:
- * UNO_ERR_ARG. */
+ * runs as a reduction kernel (two chunks of a row per CTA) whose CTAs carry
+ * no counters plus one CTA per request that combines the rows and decides;
+ * otherwise as one fused kernel whose last CTAs combine and decide.  Both
+ * give the same tokens.  0 forces the split form.  Changing it drops
+ * captured graphs.  max_ctas < 0: UNO_ERR_ARG. */
 int uno_set_verify_split(uno_ctx *ctx, int max_ctas);
 
 /*
