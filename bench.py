@@ -325,9 +325,18 @@ def cpu_cores():
 # Workload set-up.
 # ---------------------------------------------------------------------------
 def kv_bytes_per_token(cfg):
-    # bf16 models: K as an fp16 hi/lo pair and V in fp16 (three planes)
+    """KV-cache bytes a token holds in the library's layout (capacity): bf16
+    models keep K as an fp16 hi/lo pair and V in fp16 (three planes)."""
     esz, planes = (2, 3) if cfg["dtype"] == "bf16" else (4, 2)
     return cfg["n_layers"] * planes * cfg["n_kv_heads"] * cfg["head_dim"] * esz
+
+
+def kv_bytes_algorithmic(cfg):
+    """KV bytes of a token in the model's own precision (K and V, each
+    n_layers x n_kv_heads x head_dim elements): the roofline's figure
+    (147,456 bytes for the Qwen3-8B shape in bf16)."""
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    return cfg["n_layers"] * 2 * cfg["n_kv_heads"] * cfg["head_dim"] * esz
 
 
 def max_batch_that_fits(cfg, weight_bytes, max_ctx):
@@ -855,10 +864,11 @@ def reduce_sum(x, world, device):
     return int(t.item())
 
 
-def step_bytes(cfg, batch, ctx_window):
+def step_bytes(cfg, batch, ctx_window, kv_per_token=None):
     """Algorithmic HBM bytes of one iteration: base weights once per pass (the
     embedding table is only gathered), the adapters once (draft pass), each
-    request's KV at the window's mean context once per pass, and the fp32
+    request's KV at the window's mean context once per pass in the model's
+    precision (kv_per_token overrides: the layout's bytes), and the fp32
     logits written and read once."""
     esz = 2 if cfg["dtype"] == "bf16" else 4
     from lossless_diffusion_draft_b200 import synth
@@ -870,7 +880,7 @@ def step_bytes(cfg, batch, ctx_window):
         elif name != "embed":
             base += n
     ctx = sum(ctx_window) / 2
-    kv = ctx * kv_bytes_per_token(cfg) * 2 * batch
+    kv = ctx * (kv_per_token or kv_bytes_algorithmic(cfg)) * 2 * batch
     logits = (2 * cfg["B"] + 1) * cfg["vocab"] * 4 * 2 * batch
     return 2 * base + lora + kv + logits
 
@@ -984,7 +994,11 @@ def main():
     sb = step_bytes(cfg, batch, head["ctx_window"])
     step_roof = {"algorithmic_bytes_per_step": sb, "achieved_GBps": sb / (per_step_ms / 1e3) / 1e9,
                  "frac_of_hbm_peak": sb / (per_step_ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                 "peak_source": pk["source"]}
+                 "peak_source": pk["source"],
+                 "layout_bytes_per_step": step_bytes(cfg, batch, head["ctx_window"],
+                                                     kv_bytes_per_token(cfg)),
+                 "note": "algorithmic bytes count the KV cache in the model's precision (bf16 K and V); "
+                         "layout_bytes_per_step counts the three fp16 planes the kernels read"}
     kp = res["kprof"]
     g_launch, g_ms, g_bytes = kp["gemm"]
     roofline = gemm_roofline(res["detail"], cfg, pk) or {}

@@ -134,3 +134,22 @@ def test_clock_sampler_disabled_records_nothing():
     with bench.ClockSampler(0, enabled=False, nvml=_FakeNvml()) as clk:
         pass
     assert clk.summary() is None
+
+
+def test_step_bytes_match_the_qwen8b_budget():
+    """The per-step roofline's algorithmic bytes for the Qwen3-8B shape at
+    batch 1 and context 5120, from the shape's own counts: 6,945,767,424
+    body + 622,329,856 LM-head parameters (bf16) per pass, 349,175,808 LoRA
+    parameters once, the RMSNorm gains ((2 x 36 + 1) x 4096) per pass,
+    147,456 KV bytes per token per pass (36 layers x K and V x 8 heads x 128
+    x 2 bytes), fp32 logits of 33 rows written and read."""
+    from lossless_diffusion_draft_b200 import synth
+    cfg = dict(synth.CONFIGS["qwen8b"])
+    assert bench.kv_bytes_algorithmic(cfg) == 147_456
+    norms = (2 * 36 + 1) * 4096
+    expect = (2 * (6_945_767_424 + 622_329_856 + norms) * 2 + 349_175_808 * 2 + 5120 * 147_456 * 2
+              + 33 * 151_936 * 4 * 2)
+    assert bench.step_bytes(cfg, 1, [5120, 5120]) == expect
+    # the library's three-plane layout reads half as many KV bytes again
+    extra = bench.step_bytes(cfg, 1, [5120, 5120], bench.kv_bytes_per_token(cfg)) - expect
+    assert extra == 5120 * 147_456 * 2 // 2
