@@ -14,6 +14,9 @@
 //    with the producer's (slot 0 for its first part, 1 for any later one);
 //  - the DUMP-mode part slots (tile + contributor) are distinct and below
 //    n_tiles + grid, the count the host allocates;
+//  - with m-tile groups, the CTA indices (which pick the fix-up slots) are
+//    distinct, below the grid and the SM count, and each CTA's units map to
+//    tiles of its own m-tile;
 //  - the epilogue's row groups (epi_groups_per_tile) cover every row of an
 //    m-tile once and never straddle two.
 // Prints "ok" and exits 0, or prints the first failures and exits 1.
@@ -90,6 +93,33 @@ static void check_partition(int n_tiles, int KBt, int grid) {
   }
 }
 
+// m-tile groups (several token m-tiles, not DUMP): g = min(SMs / m_tiles,
+// units / 8) splits of the n-tiles' units, repeated for every m-tile; CTA
+// i * m_tiles + mt works on m-tile mt.  The CTA indices, which select the
+// fix-up slots of the workspace (two per SM), stay below the grid and the SM
+// count, and every (n-tile, m-tile) tile is reduced from its own m-tile's
+// CTAs only.
+static void check_grouped(int n_tiles, int m_tiles, int KBt, int sm) {
+  ++g_cases;
+  const int vunits = n_tiles * KBt;
+  int g = sm / m_tiles < vunits / 8 ? sm / m_tiles : vunits / 8;
+  if (g < 1) return;   // the host then takes the ungrouped form
+  const int grid = g * m_tiles;
+  CHECK(grid <= sm, "grid %d over %d SMs", grid, sm);
+  std::set<int> ctas;
+  for (int mt = 0; mt < m_tiles; ++mt)
+    for (int i = 0; i < g; ++i) {
+      const int cta = i * m_tiles + mt;
+      CHECK(cta >= 0 && cta < grid && ctas.insert(cta).second, "CTA %d (split %d, m-tile %d)", cta, i, mt);
+      const int u0 = sk_start(i, vunits, g), u1 = sk_start(i + 1, vunits, g);
+      for (int u = u0; u < u1; ++u) {
+        const int t = (u / KBt) * m_tiles + mt;   // the kernel's tile_of
+        CHECK(t % m_tiles == mt && t / m_tiles < n_tiles, "unit %d of CTA %d maps to tile %d", u, cta, t);
+      }
+    }
+  CHECK((int)ctas.size() == grid, "%d CTAs for a grid of %d", (int)ctas.size(), grid);
+}
+
 static void check_row_groups(int M, int NT, int RG) {
   ++g_cases;
   const int m_tiles = (M + NT - 1) / NT;
@@ -129,6 +159,16 @@ int main() {
       for (int grid = 1; grid <= n_tiles * KBt && grid <= 300; ++grid) check_partition(n_tiles, KBt, grid);
   // the LM head of the Qwen3-8B shape (151936 / 128 tiles, K 4096 / 128)
   check_partition(1187, 32, 148);
+  // m-tile groups: max batch (1360 / 1280 rows in 128-row token tiles),
+  // prefill chunks, the tokens-in-M form's 256-wide weight tiles
+  for (int sm : {148, 132})
+    for (int m_tiles : {2, 3, 8, 11, 16, 64})
+      for (int KBt : {32, 96})
+        for (int n_tiles : {2, 16, 17, 33, 48, 96, 194, 594, 1187}) {
+          check_grouped(n_tiles, m_tiles, KBt, sm);
+          const int g = sm / m_tiles < n_tiles * KBt / 8 ? sm / m_tiles : n_tiles * KBt / 8;
+          if (g >= 1) check_partition(n_tiles, KBt, g);
+        }
   // row groups: the draft and verify passes, max batch, prefill chunks
   for (int M : {1, 9, 16, 17, 18, 33, 100, 128, 129, 136, 1280, 1360, 1361})
     for (int NT : {16, 32, 64, 128})
