@@ -1502,9 +1502,13 @@ int uno_init(const uno_shape* shape, const uno_weights* wts, int lora_rank, floa
     }
   }
   // tensor-core attention: the pool (fp16 for bf16 models) as a [rows, head_dim]
-  // tensor, 64x64 boxes
-  if (s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && ATC_QROWS % G == 0) {
-    const uint64_t rows = (uint64_t)L * n_pages * planes * Hkv * KV_PAGE;
+  // tensor, 64x64 boxes.  Its kernel forms pool rows and TMA coordinates as
+  // 32-bit ints: a pool of 2^31 rows or more (about 270 requests of 9232
+  // tokens on the Qwen3-8B shape) takes the SIMT attention instead.
+  const uint64_t kv_rows = (uint64_t)L * n_pages * planes * Hkv * KV_PAGE;
+  if (s.dtype == UNO_BF16 && (hd == 64 || hd == 128) && ATC_QROWS % G == 0 &&
+      kv_rows < ((uint64_t)1 << 31)) {
+    const uint64_t rows = kv_rows;
     const CUtensorMap* m = c->genv.map(c->kv_pool, rows, hd, hd, KV_PAGE, /*fp16=*/true);
     // q: box (64 of head_dim, the G heads of a kv head, the query tile's tokens)
     EncodeTiledFn f = encode_fn();
