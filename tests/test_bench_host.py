@@ -153,3 +153,26 @@ def test_step_bytes_match_the_qwen8b_budget():
     # the library's three-plane layout reads half as many KV bytes again
     extra = bench.step_bytes(cfg, 1, [5120, 5120], bench.kv_bytes_per_token(cfg)) - expect
     assert extra == 5120 * 147_456 * 2 // 2
+
+
+def test_gemm_roofline_arithmetic():
+    """The dominant GEMM's roofline from per-launch times: the gate|up
+    projection of a batch-1 draft pass is HBM-bound (its 203.6 MB over the
+    measured copy rate), the max-batch one tensor-bound (2 M N K flops over
+    the sustained bf16 rate; the hi/lo inputs double the executed flops)."""
+    pk = {"hbm_gbs": 6545.9, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1345.1, "source": "measured"}
+    cfg = {"dtype": "bf16"}
+    small = [{"cls": "gemm", "m": 17, "n": 24832, "k": 4096, "r": 0, "us_per_call": 40.0,
+              "calls_per_step": 36.0, "ms_per_step": 1.44},
+             {"cls": "attn", "us_per_call": 15.0, "calls_per_step": 144.0, "ms_per_step": 2.2}]
+    r = bench.gemm_roofline(small, cfg, pk)
+    b = (24832 * 4096 + 17 * 4096) * 2
+    assert r["bound"] == "hbm" and r["algorithmic_bytes"] == b == 203_563_008
+    assert abs(r["achieved"] - b / 40e-6 / 1e9) < 1e-6 and abs(r["frac"] - r["achieved"] / 6545.9) < 1e-12
+    big = [{"cls": "gemm", "m": 1360, "n": 24576, "k": 4096, "r": 128, "us_per_call": 500.0,
+            "calls_per_step": 36.0, "ms_per_step": 18.0}]
+    r = bench.gemm_roofline(big, cfg, pk)
+    f = 2.0 * 1360 * 24576 * (4096 + 128)
+    assert r["bound"] == "tensor" and r["algorithmic_flops"] == f
+    assert abs(r["achieved"] - f / 500e-6 / 1e12) < 1e-9 and r["peak"] == 1345.1
+    assert abs(r["executed_TFLOPs"] - 2 * r["achieved"]) < 1e-9
