@@ -101,8 +101,10 @@ typedef struct uno_weights {
  *   block_B:   drafted block size B (2 <= B <= 64).
  *   max_batch: request slots; max_ctx: tokens one request may hold (prompt
  *              plus generated).  The KV pool (element type: see
- *              uno_debug_kv) holds max_batch * ceil((max_ctx + B + 1) / 64)
- *              pages of 64 tokens.
+ *              uno_debug_kv) holds max_batch * ceil((max_ctx + B + 2) / 64)
+ *              pages of 64 tokens.  bf16 models whose pool reaches 2^31
+ *              rows of head_dim (n_layers x pages x 3 planes x n_kv_heads x
+ *              64) run the SIMT attention instead of the tensor-core one.
  *   seed:      Philox key of every uniform the sampler draws.
  *   stream:    every later call enqueues on this stream.
  * On success *out receives the context (free it with uno_destroy).
